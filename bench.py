@@ -1,0 +1,563 @@
+#!/usr/bin/env python
+"""MSA (MiniMax Sparse Attention) benchmark on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  msa_index_select      index scores + block max-pool + fused top-k
+  msa_sparse_attn_prefill  reverse index, gathered-query tcgen05 attention,
+                        partial merge
+  msa_sparse_attn_decode   decode step (index scan, top-k, split attention)
+on the 1M-token workload: prefill B=1, L=1,048,576 plus a decode step of 4
+sequences at 1,048,576 cached tokens; 32 query heads, 8 groups, d=128,
+d_idx=128, block=128, top_k=16; i.i.d. N(0,1) bf16 inputs (seed 4).  The
+decode-128K workload (32 sequences, lengths uniform in [65536, 131072]) is
+timed alongside and reported under "decode_128k".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+--impl reference times the fp64 CPU oracle (the only reference this method
+has) on a bounded sample of the same workload per step.
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "MSA prefill tokens/s & decode µs/step at 128K/1M; % of B200 roofline"
+BLOCK = 128
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# --------------------------------------------------------------------- work
+def n_sel(t: np.ndarray, top_k: int) -> np.ndarray:
+    """Tokens a query at position t attends to (selected blocks, s <= t)."""
+    bt = t // BLOCK
+    return BLOCK * (np.minimum(top_k, bt + 1) - 1) + (t % BLOCK) + 1
+
+
+def prefill_index_flops(B, L, G, d_idx, top_k):
+    nb = L // BLOCK
+    tiles = sum(range(top_k, nb)) if nb > top_k else 0
+    return B * G * 2.0 * d_idx * BLOCK * BLOCK * tiles
+
+
+def prefill_main_flops(B, L, H, d, top_k):
+    t = np.arange(L, dtype=np.int64)
+    return B * float(H) * 4.0 * d * float(n_sel(t, top_k).sum())
+
+
+def decode_bytes(seq_lens, H, G, d, d_idx, top_k):
+    n = np.asarray(seq_lens, dtype=np.int64)
+    t = n - 1
+    kv = G * 2 * d * 2 * n_sel(t, top_k)
+    scan = n * d_idx * 2
+    small = len(n) * (H * d * 2 * 2 + G * d_idx * 2)
+    return float((kv + scan).sum() + small)
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        # nvidia-smi numbers GPUs differently from a masked CUDA device list:
+        # address the device by its UUID.
+        try:
+            self.gpu = "GPU-" + str(torch.cuda.get_device_properties(gpu_index).uuid)
+        except Exception:
+            self.gpu = str(gpu_index)
+        self.lines = []
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------- dist
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def dist_max(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(ws: int):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# --------------------------------------------------------------------- oracle leg
+class OracleLeg:
+    """Times the fp64 oracle, as it stands, on a bounded sample of the step:
+    prefill query positions drawn uniformly from [0, L) (every group and head
+    of each) plus whole decode sequences.  A prefill row's cost grows with t,
+    so uniform positions keep the per-row mean unbiased; the sample time is
+    scaled to a whole step.  Host copies are made before the clock starts."""
+
+    def __init__(self, x, dx, shape, dshape):
+        self.x, self.dx, self.shape, self.dshape = x, dx, shape, dshape
+        self.k = x["k"][0].to("cpu")
+        self.v = x["v"][0].to("cpu")
+        self.k_idx64 = x["k_idx"][0].to("cpu").double().numpy()
+        self.dec = {}
+
+    def _dec_host(self, b):
+        if b not in self.dec:
+            dx = self.dx
+            self.dec[b] = (dx["q"][b].to("cpu"), dx["q_idx"][b].to("cpu"), dx["k_cache"][b].to("cpu"),
+                           dx["v_cache"][b].to("cpu"), dx["k_idx_cache"][b].to("cpu").double().numpy(),
+                           int(dx["seq_lens"][b]))
+        return self.dec[b]
+
+    def sample(self, rng, n_tok, n_dec):
+        import oracle.msa_oracle as O
+        f64 = O.as_f64
+        shape, dshape = self.shape, self.dshape
+        L, H, G, d, top_k = shape.L, shape.H, shape.G, shape.d, shape.top_k
+        r = H // G
+        sc = 1.0 / math.sqrt(d)
+        ts = sorted(rng.integers(0, L, size=n_tok).tolist())
+        q_rows = self.x["q"][0, ts].to("cpu")
+        qi_rows = self.x["q_idx"][0, ts].to("cpu")
+        bsel = sorted(rng.choice(dshape.B, size=n_dec, replace=False).tolist())
+        decs = [self._dec_host(b) for b in bsel]
+        t0 = time.perf_counter()
+        for n, t in enumerate(ts):
+            for g in range(G):
+                bs = O.block_scores_row(f64(qi_rows[n, g]), self.k_idx64, t, BLOCK)
+                blocks = O.select_blocks_row(bs, t, BLOCK, top_k)
+                tok = torch.from_numpy(O.selected_tokens(blocks, t, BLOCK))
+                O.attend_rows(f64(q_rows[n, g * r:(g + 1) * r]), f64(self.k[tok, g]), f64(self.v[tok, g]), sc)
+        t_pre = time.perf_counter() - t0
+        t1 = time.perf_counter()
+        for (q, qi, kc, vc, ki64, n) in decs:
+            t = n - 1
+            for g in range(dshape.G):
+                bs = O.block_scores_row(f64(qi[g]), ki64, t, BLOCK)
+                blocks = O.select_blocks_row(bs, t, BLOCK, dshape.top_k)
+                tok = torch.from_numpy(O.selected_tokens(blocks, t, BLOCK))
+                O.attend_rows(f64(q[g * r:(g + 1) * r]), f64(kc[tok, g]), f64(vc[tok, g]), sc)
+        t_dec = time.perf_counter() - t1
+        est = t_pre * (L / n_tok) * shape.B + t_dec * (dshape.B / n_dec)
+        return t_pre + t_dec, est
+
+
+# --------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="1m", choices=["1m", "128k", "32k"],
+                    help="prefill length of the step (1m is the headline workload)")
+    ap.add_argument("--op", default="step", choices=["step", "index", "attn", "decode"],
+                    help="time one operation of the step alone (profiling runs); "
+                         "prints its own short JSON line")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="override the decode batch (profiling runs on a smaller footprint)")
+    args = ap.parse_args()
+    ws_n, rank, local = dist_setup()
+
+    from block_sparse_long_08_b200 import inputs as I
+
+    if args.workload == "1m":
+        shape, dshape, seed = I.PREFILL_1M, I.DECODE_1M, I.SEEDS["1m"]
+    elif args.workload == "128k":
+        shape, dshape, seed = I.PREFILL_128K_PLANTED, I.DECODE_128K, I.SEEDS["128k_planted"]
+    else:
+        shape, dshape, seed = I.PREFILL_32K, I.DECODE_128K, I.SEEDS["32k"]
+    cfg = {"workload": f"MSA prefill B={shape.B} L={shape.L} + decode batch {dshape.B} at "
+                       f"{'%d' % dshape.len_hi if dshape.len_lo == dshape.len_hi else 'U[%d,%d]' % (dshape.len_lo, dshape.len_hi)}",
+           "B": shape.B, "L": shape.L, "H": shape.H, "G": shape.G, "d": shape.d,
+           "d_idx": shape.d_idx, "block": shape.block, "top_k": shape.top_k,
+           "decode_batch": dshape.B, "seed": seed,
+           "l2": "inputs larger than L2 (126 MB) every step; no flush needed"}
+
+    if args.decode_batch > 0:
+        import dataclasses
+        dshape = dataclasses.replace(dshape, B=args.decode_batch)
+        cfg["decode_batch"] = dshape.B
+    if args.impl == "reference":
+        return run_reference(args, shape, dshape, seed, cfg, ws_n, rank)
+    return run_ours(args, shape, dshape, seed, cfg, ws_n, rank, local)
+
+
+def run_reference(args, shape, dshape, seed, cfg, ws_n, rank):
+    if rank != 0:
+        return
+    from block_sparse_long_08_b200 import inputs as I
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = I.prefill_inputs(shape, seed, device=dev)
+    dx = I.decode_inputs(dshape, seed, device=dev)
+    leg = OracleLeg(x, dx, shape, dshape)
+    rng = np.random.default_rng(seed)
+    n_tok, n_dec = 4, 1
+    ests = []
+    for i in range(args.warmup + args.steps):
+        _, est = leg.sample(rng, n_tok, n_dec)
+        if i >= args.warmup:
+            ests.append(est)
+    step_s = statistics.mean(ests)
+    tokens = shape.B * shape.L + dshape.B
+    value = tokens / step_s
+    cores = os.cpu_count()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"per step {n_tok} prefill query positions (all {shape.G} groups) "
+                                       f"+ {n_dec} decode sequence, scaled to the full step"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, shape, dshape, seed, cfg, ws_n, rank, local):
+    from block_sparse_long_08_b200 import inputs as I
+    from block_sparse_long_08_b200 import msa as M
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the product path has no CPU fallback)")
+    dev = torch.device("cuda", local)
+    M.lib()
+    peaks = load_peaks()
+
+    # ---- inputs (device-resident for the kernel-timed leg)
+    need_pre = args.op in ("step", "index", "attn")
+    need_dec = args.op in ("step", "decode")
+    if not need_pre:   # a decode-only profiling run keeps the footprint small
+        import dataclasses
+        shape = dataclasses.replace(shape, L=128)
+    x = I.prefill_inputs(shape, seed, device=dev)
+    if not need_dec:
+        import dataclasses
+        dshape = dataclasses.replace(dshape, B=1, Lmax=128, len_lo=128, len_hi=128)
+    dx = I.decode_inputs(dshape, seed, device=dev)
+    dx["seq_lens"] = dx["seq_lens"].to(dev)
+    B, L, H, G, d, di, K = shape.B, shape.L, shape.H, shape.G, shape.d, shape.d_idx, shape.top_k
+    p = M.make_params(B, L, H, G, d, di, BLOCK, K)
+    pd = M.make_params(dshape.B, dshape.Lmax, dshape.H, dshape.G, dshape.d, dshape.d_idx, BLOCK, dshape.top_k)
+    ws_idx = M.new_workspace(p, M.MSA_OP_INDEX_SELECT, dev)
+    ws_att = M.new_workspace(p, M.MSA_OP_PREFILL_ATTN, dev)
+    ws_dec = M.new_workspace(pd, M.MSA_OP_DECODE, dev)
+    sel = torch.empty((B, G, L, K), dtype=torch.int32, device=dev)
+    out = torch.empty_like(x["q"])
+    dout = torch.empty_like(dx["q"])
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx)
+        if ev:
+            ev[1].record(stream)
+        M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att)
+        if ev:
+            ev[2].record(stream)
+        M.msa_sparse_attn_decode(dx["q"], dx["q_idx"], dx["k_cache"], dx["v_cache"], dx["k_idx_cache"],
+                                 dx["seq_lens"], dshape.top_k, out=dout, ws=ws_dec)
+        if ev:
+            ev[3].record(stream)
+
+    if args.op != "step":
+        return run_single_op(args, M, x, dx, dshape, K, sel, out, dout, ws_idx, ws_att, ws_dec, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    for w in (ws_idx, ws_att, ws_dec):
+        rc = M.msa_read_status(w)
+        if rc != 0:
+            raise SystemExit(f"device status {rc} after warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    dist_barrier(ws_n)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    dist_barrier(ws_n)
+    total_ms = t_start.elapsed_time(t_end)
+    total_ms = dist_max(total_ms, ws_n)
+    idx_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    att_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    dec_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    ms_per_step = total_ms / args.steps
+    tokens_per_step = B * L + dshape.B
+    value = ws_n * tokens_per_step / (ms_per_step / 1e3)
+
+    # ---- rooflines
+    f_idx = prefill_index_flops(B, L, G, di, K)
+    f_main = prefill_main_flops(B, L, H, d, K)
+    seq_lens_host = dx["seq_lens"].cpu().numpy()
+    dbytes = decode_bytes(seq_lens_host, dshape.H, dshape.G, dshape.d, dshape.d_idx, dshape.top_k)
+    peak_t = peaks["bf16_tflops_sustained"]
+    roof_idx = {"bound": "tensor", "achieved": f_idx / (idx_ms / 1e3) / 1e12, "peak": peak_t,
+                "unit": "TFLOP/s", "frac": None, "traffic": None,
+                "kernel": "msa_index_kernel", "peak_kind": f"bf16 sustained ({peaks['source']})"}
+    roof_idx["frac"] = roof_idx["achieved"] / peak_t
+    roof_att = {"bound": "tensor", "achieved": f_main / (att_ms / 1e3) / 1e12, "peak": peak_t,
+                "unit": "TFLOP/s"}
+    roof_att["frac"] = roof_att["achieved"] / peak_t
+    roof_dec = {"bound": "hbm", "achieved": dbytes / (dec_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    roof_dec["frac"] = roof_dec["achieved"] / peaks["hbm_gbs"]
+
+    nchunks = math.ceil(L / M.msa_prefill_chunk_len(p))
+    launches_per_step = 1 + 5 * nchunks + 4
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": cfg, "roofline": roof_idx,
+            "breakdown": {"index_ms": idx_ms, "prefill_attn_ms": att_ms, "decode_us": dec_ms * 1e3,
+                          "prefill_tokens_per_s": B * L / ((idx_ms + att_ms) / 1e3),
+                          "index_flops": f_idx, "main_flops": f_main, "decode_bytes": dbytes,
+                          "prefill_attn_roofline": roof_att, "decode_roofline": roof_dec},
+            "gpu_launches": launches_per_step * args.steps, "clocks": clk}
+
+    # ---- decode at 128K (the decode workload of the pages' 128K setting)
+    if args.workload == "1m" and rank == 0 or args.workload != "1m":
+        line["decode_128k"] = bench_decode_128k(M, I, dev, args, peaks)
+
+    # ---- end to end through the public API with host buffers
+    if not args.no_e2e:
+        line["e2e"] = bench_e2e(M, x, dx, shape, dshape, K, args, ws_n, stream)
+
+    # ---- oracle on the host cores
+    if not args.no_cpu_baseline and rank == 0 and ws_n == 1:
+        leg = OracleLeg(x, dx, shape, dshape)
+        rng = np.random.default_rng(seed)
+        n_tok, n_dec = 24, 1
+        t_s, est = leg.sample(rng, n_tok, n_dec)
+        line["cpu_baseline"] = {
+            "value": tokens_per_step / est, "unit": "tokens/s", "cores": os.cpu_count(),
+            "kind": "oracle",
+            "sample": f"{n_tok} prefill query positions uniform in [0,L) (all {G} groups, {H} heads) "
+                      f"+ {n_dec} of {dshape.B} decode sequences; {t_s:.1f} s of CPU, scaled to one step"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws_n > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_single_op(args, M, x, dx, dshape, K, sel, out, dout, ws_idx, ws_att, ws_dec, stream):
+    """One operation alone, W untimed + K timed launches (profiling aid)."""
+    M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx)  # the attention op needs sel
+
+    def op():
+        if args.op == "index":
+            M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx)
+        elif args.op == "attn":
+            M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att)
+        else:
+            M.msa_sparse_attn_decode(dx["q"], dx["q_idx"], dx["k_cache"], dx["v_cache"],
+                                     dx["k_idx_cache"], dx["seq_lens"], dshape.top_k, out=dout, ws=ws_dec)
+
+    for _ in range(args.warmup):
+        op()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        op()
+    b.record(stream)
+    torch.cuda.synchronize()
+    for w in (ws_idx, ws_att, ws_dec):
+        if M.msa_read_status(w) != 0:
+            raise SystemExit("device status error")
+    print(json.dumps({"op": args.op, "workload": args.workload,
+                      "ms_per_launch": a.elapsed_time(b) / args.steps}), flush=True)
+
+
+def bench_decode_128k(M, I, dev, args, peaks):
+    ds = I.DECODE_128K
+    y = I.decode_inputs(ds, I.SEEDS["decode_128k"], device=dev)
+    seq = y["seq_lens"].to(dev)
+    pd = M.make_params(ds.B, ds.Lmax, ds.H, ds.G, ds.d, ds.d_idx, BLOCK, ds.top_k)
+    ws = M.new_workspace(pd, M.MSA_OP_DECODE, dev)
+    out = torch.empty_like(y["q"])
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def run():
+        M.msa_sparse_attn_decode(y["q"], y["q_idx"], y["k_cache"], y["v_cache"], y["k_idx_cache"], seq,
+                                 ds.top_k, out=out, ws=ws)
+
+    for _ in range(max(3, args.warmup)):
+        run()
+    torch.cuda.synchronize()
+    if M.msa_read_status(ws) != 0:
+        raise SystemExit("decode-128k device status error")
+    iters = 20
+    times = []
+    for _ in range(iters):
+        flush.zero_()   # L2 flush (256 MB > 126 MB L2) outside the timed span
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        run()
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    us = statistics.median(times) * 1e3
+    byts = decode_bytes(y["seq_lens"].numpy(), ds.H, ds.G, ds.d, ds.d_idx, ds.top_k)
+    del y
+    return {"us_per_step": us, "iters": iters, "batch": ds.B,
+            "seq_lens": f"U[{ds.len_lo},{ds.len_hi}] seed {I.SEEDS['decode_128k']}",
+            "l2": "256 MB buffer written between iterations",
+            "roofline": {"bound": "hbm", "achieved": byts / (us / 1e6) / 1e9, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": byts / (us / 1e6) / 1e9 / peaks["hbm_gbs"],
+                         "bytes": byts},
+            "gpu_launches": 4 * iters}
+
+
+def bench_e2e(M, x, dx, shape, dshape, K, args, ws_n, stream):
+    """Same step through the public API (msa_forward + msa_sparse_attn_decode),
+    inputs copied from pinned host memory and outputs read back every step."""
+    dev = x["q"].device
+    names = ("q", "k", "v", "q_idx", "k_idx")
+    host = {n: x[n].to("cpu").pin_memory() for n in names}
+    dnames = ("q", "q_idx")
+    dhost = {n: dx[n].to("cpu").pin_memory() for n in dnames}
+    dbuf = {n: torch.empty_like(x[n]) for n in names}
+    ddbuf = {n: torch.empty_like(dx[n]) for n in dnames}
+    out_h = torch.empty(x["q"].shape, dtype=torch.bfloat16).pin_memory()
+    dout_h = torch.empty(dx["q"].shape, dtype=torch.bfloat16).pin_memory()
+    p = M.make_params(shape.B, shape.L, shape.H, shape.G, shape.d, shape.d_idx, BLOCK, K)
+    pd = M.make_params(dshape.B, dshape.Lmax, dshape.H, dshape.G, dshape.d, dshape.d_idx, BLOCK,
+                       dshape.top_k)
+    ws = M.new_workspace(p, M.MSA_OP_FORWARD, dev)
+    wsd = M.new_workspace(pd, M.MSA_OP_DECODE, dev)
+    out = torch.empty_like(x["q"])
+    dout = torch.empty_like(dx["q"])
+    h2d = sum(host[n].numel() * 2 for n in names) + sum(dhost[n].numel() * 2 for n in dnames)
+    d2h = out_h.numel() * 2 + dout_h.numel() * 2
+
+    def step():
+        for n in names:
+            dbuf[n].copy_(host[n], non_blocking=True)
+        for n in dnames:
+            ddbuf[n].copy_(dhost[n], non_blocking=True)
+        M.msa_forward(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["q_idx"], dbuf["k_idx"], K, out=out, ws=ws)
+        M.msa_sparse_attn_decode(ddbuf["q"], ddbuf["q_idx"], dx["k_cache"], dx["v_cache"],
+                                 dx["k_idx_cache"], dx["seq_lens"], dshape.top_k, out=dout, ws=wsd)
+        out_h.copy_(out, non_blocking=True)
+        dout_h.copy_(dout, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        step()
+    torch.cuda.synchronize()
+    n = max(1, min(args.steps, 3))
+    dist_barrier(ws_n)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = dist_max(a.elapsed_time(b) / n, ws_n)
+    tokens = shape.B * shape.L + dshape.B
+    del host, dhost, dbuf, ddbuf, out_h, dout_h
+    return {"value": ws_n * tokens / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": n,
+            "path": "msa_forward + msa_sparse_attn_decode (C ABI via the Python binding)"}
+
+
+if __name__ == "__main__":
+    main()

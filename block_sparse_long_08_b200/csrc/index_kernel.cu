@@ -1,0 +1,409 @@
+// Index Branch on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// Computes, for every query t and GQA group g, the block scores
+//   S[b,g,t,j] = max_{s in block j} q_idx[b,t,g] . k_idx[b,s]      (j < t/128)
+// ("MiniMax M3 sparse attention" explainer, mlqm.cn/news/533796, §2.1: one
+// index query per group, one shared index key, Block Max Pooling), and either
+// stores them (SCORES mode) or keeps, per row, a running top-(top_k-1) list
+// and writes the selection with the forced local block (FUSED mode;
+// researchpapers.dev "MiniMax Sparse Attention", section "机制").
+//
+// Causality needs no element mask: the local block b_t is always selected,
+// so only blocks j < b_t are scored, and every such block is entirely
+// visible.  For a 128-query tile i the work is the tile row j = 0..i-1.
+//
+// Kernel structure (persistent, one CTA per SM, 6 warps):
+//   warp 0   TMA producer: the tile's q_idx rows for GP groups (resident),
+//            then k_idx blocks two at a time into an NS-deep ring.
+//   warp 1   TMEM owner + MMA issuer: per (stage, group) one
+//            M=128 x N=256 x K=d_idx UMMA into one of two TMEM accumulators.
+//   warps 2-5 epilogue: thread r owns accumulator row r (one query); it
+//            reads 2 x 128 fp32 columns (two key blocks) from TMEM, max-pools
+//            each block and either stores the score or inserts it into its
+//            register-resident sorted list.
+// The two TMEM accumulators let the MMA of one (stage, group) overlap the
+// epilogue of the previous one.  One k_idx stage feeds GP groups, which
+// halves L2->SM traffic for GP = 2.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cfloat>
+#include <climits>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace msa {
+
+namespace {
+
+template <int DI, int GP>
+struct IndexCfg {
+  static constexpr int NCH = DI / 64;                 // 128-B K chunks per row
+  static constexpr int Q_BYTES = GP * NCH * 16384;    // resident q_idx tiles
+  static constexpr int STAGE_BYTES = NCH * 2 * 16384; // two k_idx blocks
+  static constexpr int NS_RAW = (200 * 1024 - Q_BYTES) / STAGE_BYTES;
+  static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;
+  static constexpr int BAR_OFF = Q_BYTES + NS * STAGE_BYTES;
+  static constexpr int SMEM = BAR_OFF + 256 + 1024;   // + barriers + align slack
+  static constexpr int THREADS = 192;
+};
+
+struct IndexWork {
+  int i, b, gp, stages;
+};
+
+__device__ __forceinline__ IndexWork index_work(const IndexArgs &a, int u, int GPn) {
+  const int ngp = a.G / GPn;
+  IndexWork w;
+  w.i = a.nb - 1 - u / (a.B * ngp);
+  const int rem = u % (a.B * ngp);
+  w.b = rem / ngp;
+  w.gp = rem % ngp;
+  const bool need = a.write_scores ? (w.i >= 1) : (w.i >= a.top_k && a.top_k >= 2);
+  w.stages = need ? (w.i + 1) / 2 : 0;
+  return w;
+}
+
+// Work item of this CTA in round r (snake order over CTAs; items are sorted
+// by decreasing tile row length, so consecutive rounds balance out).
+__device__ __forceinline__ int index_item(int r, int n_items) {
+  const int u = r * gridDim.x + ((r & 1) ? (gridDim.x - 1 - blockIdx.x) : blockIdx.x);
+  return u < n_items ? u : -1;
+}
+
+template <int KCAP>
+__device__ __forceinline__ void list_insert(float (&ls)[KCAP], int (&lj)[KCAP], float s, int j) {
+  // Insert (s, j) into the list kept in (score desc, id asc) order.  The
+  // carried entry is compared lexicographically, so an entry pushed down by
+  // the insertion keeps its place ahead of an equal-score entry with a
+  // higher id.
+  float cs = s;
+  int cj = j;
+#pragma unroll
+  for (int k = 0; k < KCAP; ++k) {
+    const bool sw = (cs > ls[k]) || (cs == ls[k] && cj < lj[k]);
+    const float ts = ls[k];
+    const int tj = lj[k];
+    ls[k] = sw ? cs : ts;
+    lj[k] = sw ? cj : tj;
+    cs = sw ? ts : cs;
+    cj = sw ? tj : cj;
+  }
+}
+
+template <int KCAP>
+__device__ __forceinline__ float list_threshold(const float (&ls)[KCAP], int k1) {
+  float thr = -FLT_MAX;
+#pragma unroll
+  for (int k = 0; k < KCAP; ++k)
+    if (k == k1 - 1) thr = ls[k];
+  return thr;
+}
+
+template <int KCAP>
+__device__ __forceinline__ void sort_ids_asc(int (&v)[KCAP]) {
+  // Bitonic network over KCAP (power of two) register values.
+#pragma unroll
+  for (int k = 2; k <= KCAP; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+#pragma unroll
+      for (int x = 0; x < KCAP; ++x) {
+        const int y = x ^ j;
+        if (y > x) {
+          const bool up = (x & k) == 0;
+          const int lo = min(v[x], v[y]), hi = max(v[x], v[y]);
+          v[x] = up ? lo : hi;
+          v[y] = up ? hi : lo;
+        }
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ float max128_from_tmem(uint32_t taddr) {
+  float m = -FLT_MAX;
+  float a[32], c[32];
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    tmem_ld32(taddr + half * 64, a);
+    tmem_ld32(taddr + half * 64 + 32, c);
+    tmem_wait_ld();
+#pragma unroll
+    for (int x = 0; x < 32; x += 2) m = fmaxf(m, fmaxf(fmaxf(a[x], a[x + 1]), fmaxf(c[x], c[x + 1])));
+  }
+  return m;
+}
+
+template <int DI, int GP, int KCAP>
+__global__ void __launch_bounds__(192, 1)
+    msa_index_kernel(const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_k, const IndexArgs a) {
+  using C = IndexCfg<DI, GP>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const uint32_t s_q = smem_u32(smem);
+  const uint32_t s_k = s_q + C::Q_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+  // barrier slots
+  const uint32_t b_qfull = smem_u32(&bars[0]);
+  const uint32_t b_qempty = smem_u32(&bars[1]);
+  const uint32_t b_kfull = smem_u32(&bars[2]);            // + 8*s
+  const uint32_t b_kempty = smem_u32(&bars[2 + C::NS]);   // + 8*s
+  const uint32_t b_accfull = smem_u32(&bars[2 + 2 * C::NS]);   // + 8*slot
+  const uint32_t b_accempty = smem_u32(&bars[4 + 2 * C::NS]);  // + 8*slot
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(&bars[8 + 2 * C::NS]);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_qfull, 1);
+    mbar_init(b_qempty, 1);
+    for (int s = 0; s < C::NS; ++s) {
+      mbar_init(b_kfull + 8 * s, 1);
+      mbar_init(b_kempty + 8 * s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(b_accfull + 8 * s, 1);
+      mbar_init(b_accempty + 8 * s, 4);
+    }
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      int kst = 0;
+      uint32_t kph = 0, qph = 0;
+      for (int r = 0;; ++r) {
+        const int u = index_item(r, a.n_items);
+        if (u < 0) break;
+        const IndexWork w = index_work(a, u, GP);
+        if (w.stages == 0) continue;
+        if (!mbar_wait(b_qempty, qph ^ 1, abort_flag, a.status)) break;
+        qph ^= 1;
+        mbar_arrive_expect_tx(b_qfull, C::Q_BYTES);
+        for (int gi = 0; gi < GP; ++gi)
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_3d(s_q + (gi * C::NCH + c) * 16384, &tm_q, b_qfull, c * 64, w.gp * GP + gi,
+                        w.b * a.L + w.i * kBlock);
+        bool ok = true;
+        for (int s = 0; s < w.stages; ++s) {
+          if (!mbar_wait(b_kempty + 8 * kst, kph ^ 1, abort_flag, a.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(b_kfull + 8 * kst, C::STAGE_BYTES);
+          const uint32_t dst = s_k + kst * C::STAGE_BYTES;
+          const int row0 = w.b * a.L + (2 * s) * kBlock;
+          for (int c = 0; c < C::NCH; ++c) {
+            tma_load_2d(dst + c * 32768, &tm_k, b_kfull + 8 * kst, c * 64, row0);
+            tma_load_2d(dst + c * 32768 + 16384, &tm_k, b_kfull + 8 * kst, c * 64, row0 + kBlock);
+          }
+          if (++kst == C::NS) { kst = 0; kph ^= 1; }
+        }
+        if (!ok) break;
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 256, 0, 0);
+      int kst = 0;
+      uint32_t kph = 0, qph = 0;
+      uint32_t jc = 0;
+      for (int r = 0;; ++r) {
+        const int u = index_item(r, a.n_items);
+        if (u < 0) break;
+        const IndexWork w = index_work(a, u, GP);
+        if (w.stages == 0) continue;
+        if (!mbar_wait(b_qfull, qph, abort_flag, a.status)) break;
+        qph ^= 1;
+        tc_fence_after();
+        bool ok = true;
+        for (int s = 0; s < w.stages && ok; ++s) {
+          if (!mbar_wait(b_kfull + 8 * kst, kph, abort_flag, a.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t kbase = s_k + kst * C::STAGE_BYTES;
+          for (int gi = 0; gi < GP; ++gi) {
+            const uint32_t slot = jc & 1;
+            if (!mbar_wait(b_accempty + 8 * slot, ((jc >> 1) & 1) ^ 1, abort_flag, a.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + slot * 256;
+#pragma unroll
+            for (int kk = 0; kk < DI / 16; ++kk) {
+              const int c = kk >> 2;
+              const uint32_t off = (kk & 3) * 32;
+              const uint64_t ad = sdesc_sw128(s_q + (gi * C::NCH + c) * 16384 + off, 16, 1024);
+              const uint64_t bd = sdesc_sw128(kbase + c * 32768 + off, 16, 1024);
+              umma_f16_ss(d_tmem, ad, bd, idesc, kk > 0 ? 1u : 0u);
+            }
+            umma_commit(b_accfull + 8 * slot);
+            ++jc;
+          }
+          umma_commit(b_kempty + 8 * kst);
+          if (++kst == C::NS) { kst = 0; kph ^= 1; }
+        }
+        umma_commit(b_qempty);
+        if (!ok) break;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_base = tmem_base + (uint32_t(quad * 32) << 16);
+    const int k1 = a.top_k - 1;
+    uint32_t jc = 0;
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int u = index_item(r, a.n_items);
+      if (u < 0) break;
+      const IndexWork w = index_work(a, u, GP);
+      const int t = w.i * kBlock + row;
+      float ls[GP][KCAP];
+      int lj[GP][KCAP];
+      float thr[GP];
+#pragma unroll
+      for (int gi = 0; gi < GP; ++gi) {
+#pragma unroll
+        for (int k = 0; k < KCAP; ++k) { ls[gi][k] = -FLT_MAX; lj[gi][k] = INT_MAX; }
+        thr[gi] = -FLT_MAX;
+      }
+      for (int s = 0; s < w.stages && ok; ++s) {
+#pragma unroll
+        for (int gi = 0; gi < GP; ++gi) {
+          const uint32_t slot = jc & 1;
+          if (!mbar_wait(b_accfull + 8 * slot, (jc >> 1) & 1, abort_flag, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int g = w.gp * GP + gi;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int j = 2 * s + h;
+            if (j < w.i) {
+              const float sc = max128_from_tmem(lane_base + slot * 256 + h * 128);
+              if (a.write_scores) {
+                a.scores[((size_t(w.b) * a.G + g) * a.L + t) * a.nb + j] = sc;
+              } else if (sc > thr[gi]) {
+                list_insert<KCAP>(ls[gi], lj[gi], sc, j);
+                thr[gi] = list_threshold<KCAP>(ls[gi], k1);
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_accempty + 8 * slot);
+          ++jc;
+        }
+      }
+      if (!ok) break;
+#pragma unroll
+      for (int gi = 0; gi < GP; ++gi) {
+        const int g = w.gp * GP + gi;
+        const size_t rowid = (size_t(w.b) * a.G + g) * a.L + t;
+        if (a.write_scores) {
+          float *dst = a.scores + rowid * a.nb;
+          for (int j = w.i; j < a.nb; ++j) dst[j] = -INFINITY;
+          continue;
+        }
+        int32_t *dst = a.sel + rowid * a.top_k;
+        if (w.i + 1 <= a.top_k) {
+          for (int k = 0; k < a.top_k; ++k) dst[k] = (k <= w.i) ? k : -1;
+        } else {
+          int ids[KCAP];
+#pragma unroll
+          for (int k = 0; k < KCAP; ++k) ids[k] = (k < k1) ? lj[gi][k] : INT_MAX;
+          sort_ids_asc<KCAP>(ids);
+          if ((a.top_k & 3) == 0) {
+#pragma unroll
+            for (int k = 0; k < KCAP; k += 4) {
+              if (k < a.top_k) {
+                int4 v;
+                v.x = (k + 0 < k1) ? ids[k + 0] : (k + 0 == k1 ? w.i : -1);
+                v.y = (k + 1 < k1) ? ids[k + 1] : (k + 1 == k1 ? w.i : -1);
+                v.z = (k + 2 < k1) ? ids[k + 2] : (k + 2 == k1 ? w.i : -1);
+                v.w = (k + 3 < k1) ? ids[k + 3] : (k + 3 == k1 ? w.i : -1);
+                *reinterpret_cast<int4 *>(dst + k) = v;
+              }
+            }
+          } else {
+            // top_k can be KCAP + 1 (k1 == KCAP): the local block takes slot KCAP
+#pragma unroll
+            for (int k = 0; k <= KCAP; ++k)
+              if (k < a.top_k)
+                dst[k] = (k < k1) ? ids[k < KCAP ? k : KCAP - 1] : (k == k1 ? w.i : -1);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int DI, int GP, int KCAP>
+cudaError_t launch_index_t(const CUtensorMap &tq, const CUtensorMap &tk, const IndexArgs &a,
+                           int num_sms, cudaStream_t st) {
+  using C = IndexCfg<DI, GP>;
+  auto kern = msa_index_kernel<DI, GP, KCAP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int grid = a.n_items < num_sms ? a.n_items : num_sms;
+  kern<<<grid, C::THREADS, C::SMEM, st>>>(tq, tk, a);
+  return cudaGetLastError();
+}
+
+template <int DI, int GP>
+cudaError_t launch_index_k(const CUtensorMap &tq, const CUtensorMap &tk, const IndexArgs &a,
+                           int num_sms, cudaStream_t st) {
+  const int k1 = a.top_k - 1;
+  if (k1 <= 4) return launch_index_t<DI, GP, 4>(tq, tk, a, num_sms, st);
+  if (k1 <= 8) return launch_index_t<DI, GP, 8>(tq, tk, a, num_sms, st);
+  return launch_index_t<DI, GP, 16>(tq, tk, a, num_sms, st);
+}
+
+}  // namespace
+
+int index_groups_per_cta(int G, int top_k) { return (G % 2 == 0 && top_k - 1 <= 16) ? 2 : 1; }
+
+cudaError_t launch_index_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const IndexArgs &a,
+                                int num_sms, cudaStream_t st) {
+  if (a.n_items <= 0) return cudaSuccess;
+  const int gp = index_groups_per_cta(a.G, a.top_k);
+  if (a.top_k - 1 > 16) {
+    // wide lists: one group per CTA, 32-entry list
+    if (a.d_idx == 64) return launch_index_t<64, 1, 32>(tq, tk, a, num_sms, st);
+    return launch_index_t<128, 1, 32>(tq, tk, a, num_sms, st);
+  }
+  if (a.d_idx == 64)
+    return gp == 2 ? launch_index_k<64, 2>(tq, tk, a, num_sms, st)
+                   : launch_index_k<64, 1>(tq, tk, a, num_sms, st);
+  return gp == 2 ? launch_index_k<128, 2>(tq, tk, a, num_sms, st)
+                 : launch_index_k<128, 1>(tq, tk, a, num_sms, st);
+}
+
+}  // namespace msa

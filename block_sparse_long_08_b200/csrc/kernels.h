@@ -1,0 +1,84 @@
+// Internal launch interface between the C-ABI layer (msa_api.cu) and the
+// kernels.  Not part of the public ABI.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace msa {
+
+struct IndexArgs {
+  int B, L, G, nb, top_k, d_idx;
+  int write_scores;  // 1: store block scores, 0: fused top-k -> sel
+  int n_items;       // B * nb * (G / groups_per_cta)
+  int32_t *sel;      // [B,G,L,top_k]
+  float *scores;     // [B,G,L,nb]
+  int *status;
+};
+int index_groups_per_cta(int G, int top_k);
+cudaError_t launch_index_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const IndexArgs &a,
+                                int num_sms, cudaStream_t st);
+
+struct TopkArgs {
+  int B, G, L, nb, top_k;
+  const float *scores;  // [B,G,L,nb]
+  int32_t *sel;         // [B,G,L,top_k]
+};
+cudaError_t launch_topk_kernel(const TopkArgs &a, cudaStream_t st);
+
+struct RevIdxArgs {
+  int B, G, L, nb, top_k, qpi;  // qpi: queries per 128-row tile (128 / (H/G))
+  int t0, Lc;                   // query chunk [t0, t0 + Lc)
+  const int32_t *sel;           // [B,G,L,top_k]
+  int32_t *cnt;                 // [B*G*nb]      (zeroed by the caller)
+  int32_t *cursor;              // [B*G*nb]
+  int32_t *list_off;            // [B*G*nb + 1]
+  int32_t *item_off;            // [B*G*nb + 1]
+  int32_t *list;                // [B*G*Lc*top_k]
+  int *status;
+};
+cudaError_t launch_revidx(const RevIdxArgs &a, cudaStream_t st);
+
+struct AttnArgs {
+  int B, L, H, G, nb, top_k;
+  float scale, scale_log2;
+  int t0, Lc;
+  int max_items;               // upper bound on the chunk's work items
+  const uint16_t *q;           // [B,L,H,d]
+  const int32_t *list;
+  const int32_t *list_off;
+  const int32_t *item_off;
+  uint16_t *part_o;            // [B,Lc,H,top_k,d] bf16
+  float *part_lse;             // [B,Lc,H,top_k]
+  int *status;
+};
+cudaError_t launch_prefill_attn(const CUtensorMap &tk, const CUtensorMap &tv, const AttnArgs &a,
+                                int num_sms, cudaStream_t st);
+
+struct CombineArgs {
+  int B, L, H, G, top_k;
+  int t0, Lc;
+  const int32_t *sel;          // [B,G,L,top_k]
+  const uint16_t *part_o;      // [B,Lc,H,top_k,d]
+  const float *part_lse;       // [B,Lc,H,top_k]
+  uint16_t *out;               // [B,L,H,d]
+  float *lse;                  // [B,L,H] or null
+};
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
+
+struct DecodeArgs {
+  int B, Lmax, H, G, d_idx, nb_max, top_k;
+  float scale, scale_log2;
+  const uint16_t *q, *q_idx, *k_cache, *v_cache, *k_idx_cache;
+  const int32_t *seq_lens;
+  float *scores;               // [B,G,nb_max]
+  int32_t *sel;                // [B,G,top_k]
+  float *part_o;               // [B,H,top_k,d]
+  float *part_lse;             // [B,H,top_k]
+  uint16_t *out;               // [B,H,d]
+  int *status;
+};
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
+
+}  // namespace msa

@@ -1,0 +1,402 @@
+// C ABI of the MSA library (see include/msa.h): argument checks, workspace
+// planning, TMA descriptor encoding and kernel dispatch.  No allocation, no
+// synchronisation except in msa_read_status.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/msa.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char *where) {
+  return fail(MSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- shape checks ---------------------------------------------------------
+int check_params(const msa_params *p, bool decode) {
+  if (!p) return fail(MSA_ERR_INVALID_ARG, "params is NULL");
+  if (p->B < 0 || p->L < 0 || p->H <= 0 || p->G <= 0 || p->d <= 0 || p->d_idx <= 0 ||
+      p->block <= 0 || p->top_k <= 0)
+    return fail(MSA_ERR_INVALID_ARG, "negative or zero size in params");
+  if (!std::isfinite(p->scale) || p->scale < 0.f)
+    return fail(MSA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  if (p->d != 128) return fail(MSA_ERR_UNSUPPORTED, "d=%d (supported: 128)", p->d);
+  if (p->d_idx != 64 && p->d_idx != 128)
+    return fail(MSA_ERR_UNSUPPORTED, "d_idx=%d (supported: 64, 128)", p->d_idx);
+  if (p->block != 128) return fail(MSA_ERR_UNSUPPORTED, "block=%d (supported: 128)", p->block);
+  if (p->top_k > msa::kMaxTopK)
+    return fail(MSA_ERR_UNSUPPORTED, "top_k=%d (supported: 1..32)", p->top_k);
+  if (p->H % p->G != 0) return fail(MSA_ERR_INVALID_ARG, "H=%d not a multiple of G=%d", p->H, p->G);
+  const int r = p->H / p->G;
+  if (r != 1 && r != 2 && r != 4 && r != 8 && r != 16)
+    return fail(MSA_ERR_UNSUPPORTED, "H/G=%d (supported: 1,2,4,8,16)", r);
+  if (p->L % 128 != 0) return fail(MSA_ERR_UNSUPPORTED, "L=%d not a multiple of 128", p->L);
+  if (decode && p->G > 8) return fail(MSA_ERR_UNSUPPORTED, "decode supports G <= 8 (G=%d)", p->G);
+  if ((long long)p->B * p->L > (1LL << 26))
+    return fail(MSA_ERR_UNSUPPORTED, "B*L=%lld above 2^26", (long long)p->B * p->L);
+  return MSA_OK;
+}
+
+float eff_scale(const msa_params *p) {
+  return p->scale > 0.f ? p->scale : 1.0f / std::sqrt(float(p->d));
+}
+
+// ---- workspace plans --------------------------------------------------------
+// Prefill attention processes queries in chunks of Lc so that the partial
+// results (bf16 [B,Lc,H,top_k,d]) stay within a fixed budget.
+constexpr size_t kPartialBudget = size_t(4608) << 20;  // 4.5 GiB
+
+int prefill_chunk(const msa_params *p) {
+  const size_t per_q = size_t(p->B) * p->H * p->top_k * (p->d * 2 + 4);
+  long long lc = per_q ? (long long)(kPartialBudget / per_q) : p->L;
+  lc = (lc / 128) * 128;
+  if (lc < 128) lc = 128;
+  if (lc > p->L) lc = p->L;
+  return (int)lc;
+}
+
+struct AttnWs {
+  size_t cnt, cursor, list_off, item_off, list, part_o, part_lse, end;
+  int Lc;
+};
+AttnWs attn_ws(const msa_params *p, size_t base) {
+  AttnWs w;
+  w.Lc = prefill_chunk(p);
+  const size_t nb = size_t(p->L) / 128;
+  const size_t nbgj = size_t(p->B) * p->G * nb;
+  size_t o = base;
+  w.cnt = o; o = align_up(o + 4 * nbgj);
+  w.cursor = o; o = align_up(o + 4 * nbgj);
+  w.list_off = o; o = align_up(o + 4 * (nbgj + 1));
+  w.item_off = o; o = align_up(o + 4 * (nbgj + 1));
+  w.list = o; o = align_up(o + 4 * size_t(p->B) * p->G * w.Lc * p->top_k);
+  w.part_o = o; o = align_up(o + 2 * size_t(p->B) * w.Lc * p->H * p->top_k * p->d);
+  w.part_lse = o; o = align_up(o + 4 * size_t(p->B) * w.Lc * p->H * p->top_k);
+  w.end = o;
+  return w;
+}
+
+struct DecWs {
+  size_t scores, sel, part_o, part_lse, end;
+};
+DecWs dec_ws(const msa_params *p) {
+  DecWs w;
+  const size_t nb = size_t(p->L) / 128;
+  size_t o = msa::kWsHeader;
+  w.scores = o; o = align_up(o + 4 * size_t(p->B) * p->G * nb);
+  w.sel = o; o = align_up(o + 4 * size_t(p->B) * p->G * p->top_k);
+  w.part_o = o; o = align_up(o + 4 * size_t(p->B) * p->H * p->top_k * p->d);
+  w.part_lse = o; o = align_up(o + 4 * size_t(p->B) * p->H * p->top_k);
+  w.end = o;
+  return w;
+}
+
+size_t forward_sel_bytes(const msa_params *p) {
+  return align_up(4 * size_t(p->B) * p->G * p->L * p->top_k);
+}
+
+int check_ws(void *ws, size_t ws_bytes, size_t need) {
+  if (!ws) return fail(MSA_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) % kAlign)
+    return fail(MSA_ERR_WORKSPACE, "workspace not %zu-byte aligned", kAlign);
+  if (ws_bytes < need)
+    return fail(MSA_ERR_WORKSPACE, "workspace %zu bytes, need %zu", ws_bytes, need);
+  return MSA_OK;
+}
+
+// ---- TMA descriptors --------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// bf16 tensor of `rank` dims (innermost first), 128B swizzle, box as given.
+int make_tmap(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
+              const uint64_t *strides_bytes, const uint32_t *box) {
+  auto fn = encode_fn();
+  if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  uint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims,
+                  strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return MSA_OK;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+int *status_ptr(void *ws) { return reinterpret_cast<int *>(ws); }
+
+// ---- the operations --------------------------------------------------------
+int run_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 *k_idx,
+                     int32_t *sel, float *block_scores, void *ws, cudaStream_t st) {
+  const int nb = p->L / 128;
+  CUtensorMap tq, tk;
+  {
+    const uint64_t dims[3] = {uint64_t(p->d_idx), uint64_t(p->G), uint64_t(p->B) * p->L};
+    const uint64_t str[2] = {uint64_t(p->d_idx) * 2, uint64_t(p->d_idx) * 2 * p->G};
+    const uint32_t box[3] = {64, 1, 128};
+    int rc = make_tmap(&tq, q_idx, 3, dims, str, box);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[2] = {uint64_t(p->d_idx), uint64_t(p->B) * p->L};
+    const uint64_t str[1] = {uint64_t(p->d_idx) * 2};
+    const uint32_t box[2] = {64, 128};
+    int rc = make_tmap(&tk, k_idx, 2, dims, str, box);
+    if (rc) return rc;
+  }
+  msa::IndexArgs a;
+  a.B = p->B; a.L = p->L; a.G = p->G; a.nb = nb; a.top_k = p->top_k; a.d_idx = p->d_idx;
+  a.write_scores = block_scores ? 1 : 0;
+  a.n_items = p->B * nb * (p->G / msa::index_groups_per_cta(p->G, p->top_k));
+  a.sel = sel;
+  a.scores = block_scores;
+  a.status = status_ptr(ws);
+  cudaError_t e = msa::launch_index_kernel(tq, tk, a, num_sms(), st);
+  if (e != cudaSuccess) return cuda_fail(e, "index kernel launch");
+  if (block_scores) {
+    msa::TopkArgs t;
+    t.B = p->B; t.G = p->G; t.L = p->L; t.nb = nb; t.top_k = p->top_k;
+    t.scores = block_scores;
+    t.sel = sel;
+    e = msa::launch_topk_kernel(t, st);
+    if (e != cudaSuccess) return cuda_fail(e, "top-k kernel launch");
+  }
+  return MSA_OK;
+}
+
+int run_prefill_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
+                     const msa_bf16 *v, const int32_t *sel, msa_bf16 *out, float *lse, void *ws,
+                     size_t ws_base, cudaStream_t st) {
+  const int nb = p->L / 128;
+  const AttnWs w = attn_ws(p, ws_base);
+  uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
+  CUtensorMap tk, tv;
+  const uint64_t dims[3] = {uint64_t(p->d), uint64_t(p->G), uint64_t(p->B) * p->L};
+  const uint64_t str[2] = {uint64_t(p->d) * 2, uint64_t(p->d) * 2 * p->G};
+  const uint32_t box[3] = {64, 1, 128};
+  int rc = make_tmap(&tk, k, 3, dims, str, box);
+  if (rc) return rc;
+  rc = make_tmap(&tv, v, 3, dims, str, box);
+  if (rc) return rc;
+  const int r = p->H / p->G;
+  const int qpi = 128 / r;
+  const float scale = eff_scale(p);
+  const int sms = num_sms();
+  for (int t0 = 0; t0 < p->L; t0 += w.Lc) {
+    const int Lc = (p->L - t0) < w.Lc ? (p->L - t0) : w.Lc;
+    msa::RevIdxArgs ra;
+    ra.B = p->B; ra.G = p->G; ra.L = p->L; ra.nb = nb; ra.top_k = p->top_k; ra.qpi = qpi;
+    ra.t0 = t0; ra.Lc = Lc;
+    ra.sel = sel;
+    ra.cnt = reinterpret_cast<int32_t *>(wsb + w.cnt);
+    ra.cursor = reinterpret_cast<int32_t *>(wsb + w.cursor);
+    ra.list_off = reinterpret_cast<int32_t *>(wsb + w.list_off);
+    ra.item_off = reinterpret_cast<int32_t *>(wsb + w.item_off);
+    ra.list = reinterpret_cast<int32_t *>(wsb + w.list);
+    ra.status = status_ptr(ws);
+    cudaError_t e = msa::launch_revidx(ra, st);
+    if (e != cudaSuccess) return cuda_fail(e, "reverse index launch");
+    msa::AttnArgs aa;
+    aa.B = p->B; aa.L = p->L; aa.H = p->H; aa.G = p->G; aa.nb = nb; aa.top_k = p->top_k;
+    aa.scale = scale;
+    aa.scale_log2 = scale * 1.4426950408889634f;
+    aa.t0 = t0; aa.Lc = Lc;
+    const long long max_items =
+        (long long)p->B * p->G * Lc * p->top_k / qpi + (long long)p->B * p->G * nb;
+    aa.max_items = (int)max_items;
+    aa.q = q;
+    aa.list = ra.list; aa.list_off = ra.list_off; aa.item_off = ra.item_off;
+    aa.part_o = reinterpret_cast<uint16_t *>(wsb + w.part_o);
+    aa.part_lse = reinterpret_cast<float *>(wsb + w.part_lse);
+    aa.status = status_ptr(ws);
+    e = msa::launch_prefill_attn(tk, tv, aa, sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
+    msa::CombineArgs ca;
+    ca.B = p->B; ca.L = p->L; ca.H = p->H; ca.G = p->G; ca.top_k = p->top_k;
+    ca.t0 = t0; ca.Lc = Lc;
+    ca.sel = sel;
+    ca.part_o = aa.part_o; ca.part_lse = aa.part_lse;
+    ca.out = out; ca.lse = lse;
+    e = msa::launch_combine(ca, st);
+    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  }
+  return MSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *msa_last_error(void) { return g_err; }
+
+const char *msa_version(void) { return "msa-b200 0.1 (sm_100a)"; }
+
+size_t msa_workspace_bytes(const msa_params *p, int op) {
+  g_err[0] = 0;
+  if (check_params(p, op == MSA_OP_DECODE) != MSA_OK) return 0;
+  switch (op) {
+    case MSA_OP_INDEX_SELECT: return msa::kWsHeader;
+    case MSA_OP_PREFILL_ATTN: return attn_ws(p, msa::kWsHeader).end;
+    case MSA_OP_DECODE: return dec_ws(p).end;
+    case MSA_OP_FORWARD: return attn_ws(p, msa::kWsHeader + forward_sel_bytes(p)).end;
+    default: fail(MSA_ERR_INVALID_ARG, "unknown op %d", op); return 0;
+  }
+}
+
+int msa_prefill_chunk_len(const msa_params *p) {
+  g_err[0] = 0;
+  if (check_params(p, false) != MSA_OK) return 0;
+  return p->L > 0 ? prefill_chunk(p) : 0;
+}
+
+int msa_read_status(void *ws, msa_stream stream) {
+  g_err[0] = 0;
+  if (!ws) return fail(MSA_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, ws, sizeof(int), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "reading device status");
+  if (v != 0) {
+    e = cudaMemsetAsync(ws, 0, sizeof(int), st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing device status");
+    return fail(v, "device reported status %d (%s)", v,
+                v == MSA_ERR_DEVICE_TIMEOUT ? "a bounded wait ran out" : "invalid device input");
+  }
+  return MSA_OK;
+}
+
+int msa_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 *k_idx,
+                     int32_t *sel, float *block_scores, void *ws, size_t ws_bytes,
+                     msa_stream stream) {
+  g_err[0] = 0;
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (p->B == 0 || p->L == 0) return MSA_OK;
+  if (!q_idx || !k_idx || !sel) return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(sel) ||
+      (block_scores && !aligned16(block_scores)))
+    return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  rc = check_ws(ws, ws_bytes, msa::kWsHeader);
+  if (rc) return rc;
+  return run_index_select(p, q_idx, k_idx, sel, block_scores, ws,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+int msa_sparse_attn_prefill(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
+                            const msa_bf16 *v, const int32_t *sel, msa_bf16 *out, float *lse,
+                            void *ws, size_t ws_bytes, msa_stream stream) {
+  g_err[0] = 0;
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (p->B == 0 || p->L == 0) return MSA_OK;
+  if (!q || !k || !v || !sel || !out) return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(sel) || !aligned16(out) ||
+      (lse && !aligned16(lse)))
+    return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const size_t need = attn_ws(p, msa::kWsHeader).end;
+  rc = check_ws(ws, ws_bytes, need);
+  if (rc) return rc;
+  return run_prefill_attn(p, q, k, v, sel, out, lse, ws, msa::kWsHeader,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+int msa_forward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k, const msa_bf16 *v,
+                const msa_bf16 *q_idx, const msa_bf16 *k_idx, msa_bf16 *out, int32_t *sel,
+                float *lse, void *ws, size_t ws_bytes, msa_stream stream) {
+  g_err[0] = 0;
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (p->B == 0 || p->L == 0) return MSA_OK;
+  if (!q || !k || !v || !q_idx || !k_idx || !out)
+    return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(q_idx) ||
+      !aligned16(k_idx) || !aligned16(out) || (sel && !aligned16(sel)) || (lse && !aligned16(lse)))
+    return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const size_t base = msa::kWsHeader + forward_sel_bytes(p);
+  rc = check_ws(ws, ws_bytes, attn_ws(p, base).end);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t *s = sel ? sel : reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ws) + msa::kWsHeader);
+  rc = run_index_select(p, q_idx, k_idx, s, nullptr, ws, st);
+  if (rc) return rc;
+  return run_prefill_attn(p, q, k, v, s, out, lse, ws, base, st);
+}
+
+int msa_sparse_attn_decode(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
+                           const msa_bf16 *k_cache, const msa_bf16 *v_cache,
+                           const msa_bf16 *k_idx_cache, const int32_t *seq_lens, msa_bf16 *out,
+                           int32_t *sel, void *ws, size_t ws_bytes, msa_stream stream) {
+  g_err[0] = 0;
+  int rc = check_params(p, true);
+  if (rc) return rc;
+  if (p->B == 0) return MSA_OK;
+  if (p->L == 0) return fail(MSA_ERR_INVALID_ARG, "decode needs a cache (L = Lmax > 0)");
+  if (!q || !q_idx || !k_cache || !v_cache || !k_idx_cache || !seq_lens || !out)
+    return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(q_idx) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(k_idx_cache) || !aligned16(out) || (sel && !aligned16(sel)))
+    return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const DecWs w = dec_ws(p);
+  rc = check_ws(ws, ws_bytes, w.end);
+  if (rc) return rc;
+  uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
+  msa::DecodeArgs a;
+  a.B = p->B; a.Lmax = p->L; a.H = p->H; a.G = p->G; a.d_idx = p->d_idx;
+  a.nb_max = p->L / 128; a.top_k = p->top_k;
+  a.scale = eff_scale(p);
+  a.scale_log2 = a.scale * 1.4426950408889634f;
+  a.q = q; a.q_idx = q_idx; a.k_cache = k_cache; a.v_cache = v_cache; a.k_idx_cache = k_idx_cache;
+  a.seq_lens = seq_lens;
+  a.scores = reinterpret_cast<float *>(wsb + w.scores);
+  a.sel = sel ? sel : reinterpret_cast<int32_t *>(wsb + w.sel);
+  a.part_o = reinterpret_cast<float *>(wsb + w.part_o);
+  a.part_lse = reinterpret_cast<float *>(wsb + w.part_lse);
+  a.out = out;
+  a.status = status_ptr(ws);
+  cudaError_t e = msa::launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return MSA_OK;
+}
+
+}  // extern "C"

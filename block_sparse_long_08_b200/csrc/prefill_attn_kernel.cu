@@ -1,0 +1,366 @@
+// Main Branch, prefill: exact softmax attention over the selected blocks,
+// organised key-block-outer ("MiniMax M3 sparse attention" explainer,
+// mlqm.cn/news/533796, §2.2: gather the selected K/V blocks and run ordinary
+// attention, all heads of a group sharing one selection; researchpapers.dev
+// "MiniMax Sparse Attention", sections "机制" and "对工程团队的意义": query
+// gathering and a reverse index; baguaai.com 稀疏注意力 MSA entry: "KV
+// external aggregation Q").
+//
+// One work item = one (b, g, key block j) and up to 128/R queries that
+// selected j, each with its R heads: a 128-row tile.  Per item:
+//   TMA      K_j, V_j (128 x 128 bf16 each, 128B-swizzled) into smem
+//   gather   the tile's q rows (R heads of a query are 256*R contiguous
+//            bytes) into a swizzled smem tile with cp.async
+//   UMMA     S = Q K_j^T   (M=128, N=128, K=128) into TMEM
+//   softmax  thread r owns row r: mask s <= t, row max, exp2, row sum,
+//            P = exp(...) as bf16 into smem (over the dead Q tile)
+//   UMMA     O = P V_j     (V consumed MN-major straight from its TMA tile)
+//   store    O / l as a bf16 partial and lse = ln(sum exp(scale q.k)) per
+//            (t, head, slot); a second kernel merges a row's <= top_k
+//            partials.
+// Two CTAs share an SM (96 KB smem and 256 TMEM columns each), so one CTA's
+// softmax overlaps the other's MMAs and loads.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cfloat>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace msa {
+
+namespace {
+
+constexpr int kAttnThreads = 128;
+constexpr int kSmemK = 0;
+constexpr int kSmemV = 32768;
+constexpr int kSmemQ = 65536;  // Q tile, then P tile
+constexpr int kSmemBar = 98304;
+constexpr int kAttnSmem = kSmemBar + 1024 + 1024;
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+template <int R>
+__global__ void __launch_bounds__(kAttnThreads, 2)
+    msa_prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_k,
+                            const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
+  constexpr int QPI = 128 / R;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  const uint32_t s_k = smem_u32(smem + kSmemK);
+  const uint32_t s_v = smem_u32(smem + kSmemV);
+  const uint32_t s_q = smem_u32(smem + kSmemQ);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSmemBar);
+  const uint32_t b_kv = smem_u32(&bars[0]);
+  const uint32_t b_mma = smem_u32(&bars[1]);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(&bars[2]);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+  int *s_item = reinterpret_cast<int *>(tmem_holder + 2);   // bgj, start, n
+  int *s_list = reinterpret_cast<int *>(smem + kSmemBar + 64);  // <= 128 entries
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  if (tid == 0) {
+    mbar_init(b_kv, 1);
+    mbar_init(b_mma, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_holder), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_s = *tmem_holder;
+  const uint32_t tmem_o = tmem_s + 128;
+  const uint32_t lane_off = uint32_t(warp * 32) << 16;
+
+  const int n_bgj = a.B * a.G * a.nb;
+  const int n_items = a.item_off[n_bgj];
+  if (n_items > a.max_items && tid == 0) atomicCAS(a.status, 0, kStatusBadInput);
+  constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+  constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, 0, 1);
+  uint32_t kv_ph = 0, mma_ph = 0;
+
+  for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
+    // ---- locate the item: bgj with item_off[bgj] <= w < item_off[bgj+1]
+    if (tid == 0) {
+      int lo = 0, hi = n_bgj - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.item_off[mid] <= w) lo = mid; else hi = mid - 1;
+      }
+      const int c = w - a.item_off[lo];
+      const int start = a.list_off[lo] + c * QPI;
+      const int n = min(QPI, a.list_off[lo + 1] - start);
+      s_item[0] = lo;
+      s_item[1] = start;
+      s_item[2] = n;
+      const int j = lo % a.nb;
+      const int bg = lo / a.nb;
+      const int g = bg % a.G;
+      const int b = bg / a.G;
+      mbar_arrive_expect_tx(b_kv, 65536);
+      const int z = b * a.L + j * kBlock;
+      tma_load_3d(s_k, &tm_k, b_kv, 0, g, z);
+      tma_load_3d(s_k + 16384, &tm_k, b_kv, 64, g, z);
+      tma_load_3d(s_v, &tm_v, b_kv, 0, g, z);
+      tma_load_3d(s_v + 16384, &tm_v, b_kv, 64, g, z);
+    }
+    __syncthreads();
+    const int bgj = s_item[0];
+    const int start = s_item[1];
+    const int n = s_item[2];
+    const int j = bgj % a.nb;
+    const int g = (bgj / a.nb) % a.G;
+    const int b = bgj / (a.nb * a.G);
+    if (tid < n) s_list[tid] = a.list[start + tid];
+    __syncthreads();
+
+    // ---- gather the Q tile: row = qi*R + hh, 16 granules of 16 B per row
+#pragma unroll 4
+    for (int it = 0; it < 16; ++it) {
+      const int idx = it * kAttnThreads + tid;
+      const int row = idx >> 4;
+      const int gran = idx & 15;
+      const int qi = row / R;
+      const int hh = row % R;
+      const uint32_t dst = s_q + (gran >> 3) * 16384 + sw128_offset(row, gran & 7);
+      if (qi < n) {
+        const int t = s_list[qi] >> 5;
+        const uint16_t *src =
+            a.q + ((size_t(b) * a.L + t) * a.H + size_t(g) * R + hh) * kHeadDim + gran * 8;
+        cp_async16(dst, src);
+      } else {
+        asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(dst), "r"(0) : "memory");
+      }
+    }
+    cp_async_wait_all();
+    fence_proxy_async_smem();
+    __syncthreads();
+
+    // ---- S = Q K^T
+    int ok_kv = 1;
+    if (tid == 0) {
+      ok_kv = mbar_wait(b_kv, kv_ph, abort_flag, a.status) ? 1 : 0;
+      if (ok_kv) {
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int c = kk >> 2;
+          const uint32_t off = (kk & 3) * 32;
+          umma_f16_ss(tmem_s, sdesc_sw128(s_q + c * 16384 + off, 16, 1024),
+                      sdesc_sw128(s_k + c * 16384 + off, 16, 1024), idesc_s, kk > 0);
+        }
+        umma_commit(b_mma);
+      }
+    }
+    kv_ph ^= 1;
+    // every exit decision below is taken by the whole CTA at one barrier
+    if (__syncthreads_or(!ok_kv)) break;
+    const bool ok1 = mbar_wait(b_mma, mma_ph, abort_flag, a.status);
+    mma_ph ^= 1;
+    if (__syncthreads_or(!ok1)) break;
+    tc_fence_after();
+
+    // ---- softmax on row `tid`
+    const int qi = tid / R;
+    const bool valid = qi < n;
+    const int ent = valid ? s_list[qi] : 0;
+    const int t = ent >> 5;
+    const int lim = valid ? (t - j * kBlock) : -1;  // last visible column
+    float sv[128];
+#pragma unroll
+    for (int c4 = 0; c4 < 4; ++c4) {
+      float tmp[32];
+      tmem_ld32(tmem_s + lane_off + c4 * 32, tmp);
+#pragma unroll
+      for (int x = 0; x < 32; ++x) sv[c4 * 32 + x] = tmp[x];
+    }
+    tmem_wait_ld();
+    float m = -FLT_MAX;
+#pragma unroll
+    for (int c = 0; c < 128; ++c)
+      if (c <= lim) m = fmaxf(m, sv[c]);
+    const float mb = m * a.scale_log2;
+    float l = 0.f;
+    uint8_t *p_row = smem + kSmemQ;
+#pragma unroll
+    for (int gblk = 0; gblk < 16; ++gblk) {
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c0 = gblk * 8 + e * 2;
+        const float p0 = (c0 <= lim) ? fast_exp2(fmaf(sv[c0], a.scale_log2, -mb)) : 0.f;
+        const float p1 = (c0 + 1 <= lim) ? fast_exp2(fmaf(sv[c0 + 1], a.scale_log2, -mb)) : 0.f;
+        l += p0 + p1;
+        w4[e] = pack_bf16x2(p0, p1);
+      }
+      const uint32_t off = (gblk >> 3) * 16384 + sw128_offset(tid, gblk & 7);
+      *reinterpret_cast<uint4 *>(p_row + off) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- O = P V
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const int c = kk >> 2;
+        const uint32_t off = (kk & 3) * 32;
+        umma_f16_ss(tmem_o, sdesc_sw128(s_q + c * 16384 + off, 16, 1024),
+                    sdesc_sw128(s_v + kk * 2048, 16384, 1024), idesc_o, kk > 0);
+      }
+      umma_commit(b_mma);
+    }
+    const bool ok2 = mbar_wait(b_mma, mma_ph, abort_flag, a.status);
+    mma_ph ^= 1;
+    if (__syncthreads_or(!ok2)) break;
+    tc_fence_after();
+
+    // ---- store the normalised partial and its lse
+    {
+      float o[128];
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        float tmp[32];
+        tmem_ld32(tmem_o + lane_off + c4 * 32, tmp);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) o[c4 * 32 + x] = tmp[x];
+      }
+      tmem_wait_ld();
+      if (valid) {
+        const int slot = ent & 31;
+        const int hh = tid % R;
+        const size_t prow =
+            ((size_t(b) * a.Lc + (t - a.t0)) * a.H + size_t(g) * R + hh) * a.top_k + slot;
+        if (lim >= 0) {
+          const float inv = 1.f / l;
+          uint4 *dst = reinterpret_cast<uint4 *>(a.part_o + prow * kHeadDim);
+#pragma unroll
+          for (int x = 0; x < 16; ++x)
+            dst[x] = make_uint4(pack_bf16x2(o[8 * x] * inv, o[8 * x + 1] * inv),
+                                pack_bf16x2(o[8 * x + 2] * inv, o[8 * x + 3] * inv),
+                                pack_bf16x2(o[8 * x + 4] * inv, o[8 * x + 5] * inv),
+                                pack_bf16x2(o[8 * x + 6] * inv, o[8 * x + 7] * inv));
+          a.part_lse[prow] = m * a.scale + __logf(l);
+        } else {
+          a.part_lse[prow] = -INFINITY;
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_s, 256);
+  }
+}
+
+template <int R>
+cudaError_t launch_attn_r(const CUtensorMap &tk, const CUtensorMap &tv, const AttnArgs &a,
+                          int num_sms, cudaStream_t st) {
+  auto kern = msa_prefill_attn_kernel<R>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+  if (e != cudaSuccess) return e;
+  int grid = 2 * num_sms;
+  if (a.max_items < grid) grid = a.max_items > 0 ? a.max_items : 1;
+  kern<<<grid, kAttnThreads, kAttnSmem, st>>>(tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_attn(const CUtensorMap &tk, const CUtensorMap &tv, const AttnArgs &a,
+                                int num_sms, cudaStream_t st) {
+  const int R = a.H / a.G;
+  switch (R) {
+    case 1: return launch_attn_r<1>(tk, tv, a, num_sms, st);
+    case 2: return launch_attn_r<2>(tk, tv, a, num_sms, st);
+    case 4: return launch_attn_r<4>(tk, tv, a, num_sms, st);
+    case 8: return launch_attn_r<8>(tk, tv, a, num_sms, st);
+    case 16: return launch_attn_r<16>(tk, tv, a, num_sms, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// ---------------------------------------------------------------- combine
+namespace {
+
+// One warp per (b, t, h): merge the row's partials (normalised o_s, lse_s)
+// into o = sum_s exp(lse_s - M) o_s / sum_s exp(lse_s - M), M = max lse_s.
+__global__ void __launch_bounds__(256) msa_combine_kernel(const CombineArgs a) {
+  const long long wrow = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const long long n_rows = (long long)a.B * a.Lc * a.H;
+  if (wrow >= n_rows) return;
+  const int h = (int)(wrow % a.H);
+  const long long bt = wrow / a.H;
+  const int tl = (int)(bt % a.Lc);
+  const int b = (int)(bt / a.Lc);
+  const int t = a.t0 + tl;
+  const int g = h / (a.H / a.G);
+  const int32_t *sel = a.sel + ((size_t(b) * a.G + g) * a.L + t) * a.top_k;
+  const size_t prow0 = (((size_t)b * a.Lc + tl) * a.H + h) * a.top_k;
+  const bool mine = lane < a.top_k && sel[lane] >= 0;
+  const float my_lse = mine ? a.part_lse[prow0 + lane] : -INFINITY;
+  float M = my_lse;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float wsum = 0.f;
+  if (M > -INFINITY) {
+    const float wmine = mine ? __expf(my_lse - M) : 0.f;
+    wsum = wmine;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    for (int s = 0; s < a.top_k; ++s) {
+      const float ws = __shfl_sync(0xffffffffu, wmine, s);
+      if (ws == 0.f) continue;
+      const uint2 v = *reinterpret_cast<const uint2 *>(a.part_o + (prow0 + s) * kHeadDim + lane * 4);
+      acc[0] = fmaf(ws, bf16_lo(v.x), acc[0]);
+      acc[1] = fmaf(ws, bf16_hi(v.x), acc[1]);
+      acc[2] = fmaf(ws, bf16_lo(v.y), acc[2]);
+      acc[3] = fmaf(ws, bf16_hi(v.y), acc[3]);
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  uint2 r;
+  r.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  r.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  *reinterpret_cast<uint2 *>(a.out + (((size_t)b * a.L + t) * a.H + h) * kHeadDim + lane * 4) = r;
+  if (a.lse && lane == 0) a.lse[((size_t)b * a.L + t) * a.H + h] = (wsum > 0.f) ? M + __logf(wsum) : -INFINITY;
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st) {
+  const long long n_rows = (long long)a.B * a.Lc * a.H;
+  if (n_rows == 0) return cudaSuccess;
+  msa_combine_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace msa

@@ -1,0 +1,238 @@
+"""Python binding of libmsa.so (ctypes).  Argument marshalling only: every
+step of the computation runs in the library's CUDA kernels; PyTorch supplies
+device memory and the current stream.
+
+The functions carry the C names (msa_index_select, msa_sparse_attn_prefill,
+msa_sparse_attn_decode, msa_forward, msa_workspace_bytes, msa_read_status,
+msa_last_error).  Tensors must be CUDA, contiguous, bf16 (int32 for
+selections and lengths).  Outputs are allocated here unless passed in.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmsa.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "msa.h")
+
+MSA_OK = 0
+MSA_ERR_INVALID_ARG = -1
+MSA_ERR_UNSUPPORTED = -2
+MSA_ERR_WORKSPACE = -3
+MSA_ERR_CUDA = -4
+MSA_ERR_DEVICE_TIMEOUT = -5
+MSA_ERR_DEVICE_INPUT = -6
+
+MSA_OP_INDEX_SELECT = 0
+MSA_OP_PREFILL_ATTN = 1
+MSA_OP_DECODE = 2
+MSA_OP_FORWARD = 3
+
+
+class MSAError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"msa error {code}: {msg}")
+        self.code = code
+
+
+class msa_params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("L", ctypes.c_int32), ("H", ctypes.c_int32),
+                ("G", ctypes.c_int32), ("d", ctypes.c_int32), ("d_idx", ctypes.c_int32),
+                ("block", ctypes.c_int32), ("top_k", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_SZ = ctypes.c_size_t
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmsa.so (built in-tree by block_sparse_long_08_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m block_sparse_long_08_b200.build`")
+        torch.cuda.is_available()  # make sure torch's CUDA runtime is loaded first
+        L = ctypes.CDLL(LIB_PATH)
+        pp = ctypes.POINTER(msa_params)
+        L.msa_index_select.argtypes = [pp, _P, _P, _P, _P, _P, _SZ, _P]
+        L.msa_sparse_attn_prefill.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.msa_sparse_attn_decode.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.msa_forward.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.msa_workspace_bytes.argtypes = [pp, ctypes.c_int]
+        L.msa_workspace_bytes.restype = _SZ
+        L.msa_read_status.argtypes = [_P, _P]
+        L.msa_prefill_chunk_len.argtypes = [pp]
+        L.msa_prefill_chunk_len.restype = ctypes.c_int
+        L.msa_last_error.restype = ctypes.c_char_p
+        L.msa_version.restype = ctypes.c_char_p
+        for f in ("msa_index_select", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
+                  "msa_forward", "msa_read_status"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Entry points declared in include/msa.h."""
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(msa_\w+)\s*\(", txt, re.M)))
+
+
+def msa_last_error() -> str:
+    return lib().msa_last_error().decode()
+
+
+def _check(rc: int):
+    if rc != MSA_OK:
+        raise MSAError(rc, msa_last_error())
+
+
+def make_params(B, L, H, G, d=128, d_idx=128, block=128, top_k=16, scale=0.0) -> msa_params:
+    return msa_params(int(B), int(L), int(H), int(G), int(d), int(d_idx), int(block), int(top_k),
+                      float(scale))
+
+
+def msa_workspace_bytes(p: msa_params, op: int) -> int:
+    n = lib().msa_workspace_bytes(ctypes.byref(p), op)
+    if n == 0:
+        raise MSAError(MSA_ERR_INVALID_ARG, msa_last_error())
+    return int(n)
+
+
+def msa_prefill_chunk_len(p: msa_params) -> int:
+    return int(lib().msa_prefill_chunk_len(ctypes.byref(p)))
+
+
+def new_workspace(p: msa_params, op: int, device) -> torch.Tensor:
+    """Zeroed workspace (the status word must start at zero)."""
+    return torch.zeros(msa_workspace_bytes(p, op), dtype=torch.uint8, device=device)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _req(t: torch.Tensor, name: str, dtype) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ensure_ws(ws, p, op, device):
+    need = msa_workspace_bytes(p, op)
+    if ws is None:
+        return torch.zeros(need, dtype=torch.uint8, device=device)
+    if ws.numel() < need:
+        raise MSAError(MSA_ERR_WORKSPACE, f"workspace has {ws.numel()} bytes, need {need}")
+    return ws
+
+
+def msa_index_select(q_idx: torch.Tensor, k_idx: torch.Tensor, top_k: int, *,
+                     block_scores: bool = False, sel: Optional[torch.Tensor] = None,
+                     ws: Optional[torch.Tensor] = None, stream=None):
+    """q_idx [B,L,G,d_idx], k_idx [B,L,d_idx] -> sel [B,G,L,top_k] int32
+    (and block scores [B,G,L,nb] fp32 when block_scores=True)."""
+    _req(q_idx, "q_idx", torch.bfloat16)
+    _req(k_idx, "k_idx", torch.bfloat16)
+    B, L, G, di = q_idx.shape
+    p = make_params(B, L, G, G, 128, di, 128, top_k)
+    dev = q_idx.device
+    if sel is None:
+        sel = torch.empty((B, G, L, top_k), dtype=torch.int32, device=dev)
+    scores = torch.empty((B, G, L, L // 128), dtype=torch.float32, device=dev) if block_scores else None
+    ws = _ensure_ws(ws, p, MSA_OP_INDEX_SELECT, dev)
+    _check(lib().msa_index_select(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(sel), _ptr(scores),
+                                  _ptr(ws), ws.numel(), _stream(stream)))
+    return (sel, scores) if block_scores else sel
+
+
+def msa_sparse_attn_prefill(q, k, v, sel, *, scale: float = 0.0, want_lse: bool = False,
+                            out=None, ws=None, stream=None):
+    """q [B,L,H,d], k/v [B,L,G,d] bf16, sel [B,G,L,top_k] int32 -> out [B,L,H,d]
+    (and lse [B,L,H] fp32 when want_lse)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _req(t, n, torch.bfloat16)
+    _req(sel, "sel", torch.int32)
+    B, L, H, d = q.shape
+    G = k.shape[2]
+    top_k = sel.shape[3]
+    p = make_params(B, L, H, G, d, 128, 128, top_k, scale)
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((B, L, H), dtype=torch.float32, device=dev) if want_lse else None
+    ws = _ensure_ws(ws, p, MSA_OP_PREFILL_ATTN, dev)
+    _check(lib().msa_sparse_attn_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(sel),
+                                         _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return (out, lse) if want_lse else out
+
+
+def msa_forward(q, k, v, q_idx, k_idx, top_k: int, *, scale: float = 0.0, want_sel: bool = False,
+                want_lse: bool = False, out=None, sel=None, ws=None, stream=None):
+    """Whole prefill: index branch with fused top-k, then the sparse main branch."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("q_idx", q_idx), ("k_idx", k_idx)):
+        _req(t, n, torch.bfloat16)
+    B, L, H, d = q.shape
+    G = k.shape[2]
+    di = q_idx.shape[3]
+    p = make_params(B, L, H, G, d, di, 128, top_k, scale)
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if sel is None and want_sel:
+        sel = torch.empty((B, G, L, top_k), dtype=torch.int32, device=dev)
+    lse = torch.empty((B, L, H), dtype=torch.float32, device=dev) if want_lse else None
+    ws = _ensure_ws(ws, p, MSA_OP_FORWARD, dev)
+    _check(lib().msa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_idx), _ptr(k_idx),
+                             _ptr(out), _ptr(sel), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    res = [out]
+    if want_sel:
+        res.append(sel)
+    if want_lse:
+        res.append(lse)
+    return res[0] if len(res) == 1 else tuple(res)
+
+
+def msa_sparse_attn_decode(q, q_idx, k_cache, v_cache, k_idx_cache, seq_lens, top_k: int, *,
+                           scale: float = 0.0, want_sel: bool = False, out=None, sel=None,
+                           ws=None, stream=None):
+    """q [B,H,d], q_idx [B,G,d_idx], caches [B,Lmax,G,d] / [B,Lmax,d_idx],
+    seq_lens [B] int32 (device) -> out [B,H,d] (and sel [B,G,top_k])."""
+    for n, t in (("q", q), ("q_idx", q_idx), ("k_cache", k_cache), ("v_cache", v_cache),
+                 ("k_idx_cache", k_idx_cache)):
+        _req(t, n, torch.bfloat16)
+    _req(seq_lens, "seq_lens", torch.int32)
+    B, H, d = q.shape
+    Lmax, G = k_cache.shape[1], k_cache.shape[2]
+    di = q_idx.shape[2]
+    p = make_params(B, Lmax, H, G, d, di, 128, top_k, scale)
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if sel is None and want_sel:
+        sel = torch.empty((B, G, top_k), dtype=torch.int32, device=dev)
+    ws = _ensure_ws(ws, p, MSA_OP_DECODE, dev)
+    _check(lib().msa_sparse_attn_decode(ctypes.byref(p), _ptr(q), _ptr(q_idx), _ptr(k_cache),
+                                        _ptr(v_cache), _ptr(k_idx_cache), _ptr(seq_lens), _ptr(out),
+                                        _ptr(sel), _ptr(ws), ws.numel(), _stream(stream)))
+    return (out, sel) if want_sel else out
+
+
+def msa_read_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronise and return (then clear) the device status word in ws."""
+    return lib().msa_read_status(_ptr(ws), _stream(stream))

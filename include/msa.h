@@ -1,0 +1,169 @@
+/*
+ * msa.h -- C ABI of the B200 (sm_100a) MiniMax Sparse Attention library.
+ *
+ * The operation (cited by page title and section):
+ *   Index Branch  -- "MiniMax M3 sparse attention" explainer
+ *     (mlqm.cn/news/533796) §2.1: each GQA group has one index query
+ *     q_idx[t,g]; all groups share one single-head index key k_idx[s]; the
+ *     token score is q_idx . k_idx; "Block Max Pooling" turns token scores
+ *     into block scores; top-k blocks are kept.
+ *     "MiniMax Sparse Attention:百万上下文稀疏注意力" (researchpapers.dev),
+ *     section "机制": only visible tokens (s <= t) are scored, the choice is
+ *     per (query, group), the most recent local block is always kept.
+ *   Main Branch   -- explainer §2.2: gather the selected K/V blocks and run
+ *     ordinary softmax attention; every query head of a GQA group uses the
+ *     group's selection.  researchpapers.dev section "2048 个 KV token":
+ *     16 blocks x 128 tokens per query group.
+ *   Decode        -- explainer §4.1: each new token scores the cache and
+ *     attends only to its selected blocks.
+ *
+ * Definition implemented (readings where the pages are silent are marked R):
+ *   S[b,g,t,j] = max_{s in block j, s <= t} sum_i q_idx[b,t,g,i]*k_idx[b,s,i]
+ *                                          (R: raw dot product, no scale)
+ *   sel[b,g,t] = {b_t} U top_(top_k-1){ S[b,g,t,j] : j < b_t },  b_t = t/block
+ *                (R: top_k counts the local block; equal scores -> lower j;
+ *                 if b_t+1 <= top_k every block 0..b_t is kept)
+ *                stored sorted ascending, padded with -1.
+ *   out[b,t,h] = softmax_s(scale * q[b,t,h].k[b,s,g]) . v[b,s,g]  over the
+ *                tokens s <= t of the blocks in sel[b,g,t], g = h/(H/G).
+ *                (R: scale = 1/sqrt(d) when params.scale == 0)
+ *
+ * Conventions for every entry point:
+ *   - Tensors are DEVICE pointers, row-major, contiguous, 16-byte aligned.
+ *     bf16 tensors are passed as raw 16-bit patterns (msa_bf16).
+ *   - The caller owns every buffer, including the workspace `ws`
+ *     (>= msa_workspace_bytes(p, op) bytes, 256-byte aligned).  The library
+ *     allocates and frees nothing.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and return once the work is queued.
+ *   - The first 4 bytes of `ws` are a device status word.  Zero them once
+ *     before the first call (e.g. allocate ws zeroed); the library only
+ *     ever sets them to an error code, and msa_read_status() clears them.
+ *   - Return value: MSA_OK or a negative MSA_ERR_* code; nothing is launched
+ *     when a call returns an error.  msa_last_error() gives a message
+ *     (thread-local).  Errors found on the device (a bounded wait that ran
+ *     out, an out-of-range decode length) are recorded in a status word at
+ *     the start of `ws`; msa_read_status() synchronises the stream and
+ *     returns/clears it.
+ *   - Supported: d == 128, d_idx in {64, 128}, block == 128,
+ *     1 <= top_k <= 32, H % G == 0 with H/G in {1,2,4,8,16}, L % 128 == 0.
+ *     Other shapes give MSA_ERR_UNSUPPORTED.  B == 0 or L == 0 is a no-op.
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t msa_bf16;   /* raw bfloat16 bits */
+typedef void *msa_stream;    /* cudaStream_t */
+
+typedef struct msa_params {
+  int32_t B;       /* batch (prefill) / number of sequences (decode) */
+  int32_t L;       /* sequence length (prefill) / cache capacity Lmax (decode) */
+  int32_t H;       /* query heads */
+  int32_t G;       /* GQA groups = KV heads = index queries per token */
+  int32_t d;       /* head dim of q/k/v (128) */
+  int32_t d_idx;   /* index dim of q_idx/k_idx (64 or 128) */
+  int32_t block;   /* KV block length (128) */
+  int32_t top_k;   /* blocks kept per (query, group), local block included */
+  float scale;     /* softmax scale of the main branch; 0 -> 1/sqrt(d) */
+} msa_params;
+
+enum {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = -1,    /* null/misaligned pointer, bad size */
+  MSA_ERR_UNSUPPORTED = -2,    /* shape outside the supported set */
+  MSA_ERR_WORKSPACE = -3,      /* ws too small or misaligned */
+  MSA_ERR_CUDA = -4,           /* a CUDA runtime/driver call failed */
+  MSA_ERR_DEVICE_TIMEOUT = -5, /* a bounded device-side wait ran out */
+  MSA_ERR_DEVICE_INPUT = -6    /* device-side check failed (decode length) */
+};
+
+enum {
+  MSA_OP_INDEX_SELECT = 0,
+  MSA_OP_PREFILL_ATTN = 1,
+  MSA_OP_DECODE = 2,
+  MSA_OP_FORWARD = 3
+};
+
+/* Index Branch (explainer §2.1; researchpapers.dev "机制").
+ *   q_idx  [B,L,G,d_idx] bf16, k_idx [B,L,d_idx] bf16            (in)
+ *   sel    [B,G,L,top_k] int32                                    (out)
+ *   block_scores [B,G,L,nb] fp32, nb = L/block, or NULL            (out)
+ *     When given, entry (t, j) holds S[b,g,t,j] for j < t/block and -inf
+ *     for j >= t/block (the local block is forced, never scored), and sel
+ *     is computed from these stored scores by the top-k kernel.  When NULL
+ *     the top-k runs inside the index kernel's epilogue and the L x nb
+ *     score matrix never reaches memory; both routes give the same sel.
+ */
+int msa_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 *k_idx,
+                     int32_t *sel, float *block_scores, void *ws, size_t ws_bytes,
+                     msa_stream stream);
+
+/* Main Branch, prefill (explainer §2.2; researchpapers.dev "机制").
+ *   q [B,L,H,d], k [B,L,G,d], v [B,L,G,d] bf16                      (in)
+ *   sel [B,G,L,top_k] int32: any selection in the layout above: valid
+ *     ids first (any order, each < L/block, each block at most once, the
+ *     query's own block included for a causal result), -1 padding.   (in)
+ *   out [B,L,H,d] bf16                                              (out)
+ *   lse [B,L,H] fp32 natural-log softmax normaliser, or NULL         (out)
+ * Blocks are processed key-block-outer: queries that chose the same block
+ * are gathered into 128-row tiles (reverse index), per-block partial
+ * results are merged at the end.
+ */
+int msa_sparse_attn_prefill(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
+                            const msa_bf16 *v, const int32_t *sel, msa_bf16 *out,
+                            float *lse, void *ws, size_t ws_bytes, msa_stream stream);
+
+/* Decode step (explainer §4.1).  p->B = sequences, p->L = cache capacity.
+ *   q [B,H,d], q_idx [B,G,d_idx] bf16: the new token's queries       (in)
+ *   k_cache, v_cache [B,Lmax,G,d], k_idx_cache [B,Lmax,d_idx] bf16   (in)
+ *   seq_lens [B] int32 DEVICE array: cached tokens per sequence, the new
+ *     token's k/v/k_idx already appended, so the query sits at position
+ *     seq_lens[b]-1.  Values outside [1, Lmax] set MSA_ERR_DEVICE_INPUT in
+ *     the status word and that sequence's output is zero.              (in)
+ *   out [B,H,d] bf16                                                (out)
+ *   sel [B,G,top_k] int32 or NULL: the blocks used                  (out)
+ */
+int msa_sparse_attn_decode(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
+                           const msa_bf16 *k_cache, const msa_bf16 *v_cache,
+                           const msa_bf16 *k_idx_cache, const int32_t *seq_lens,
+                           msa_bf16 *out, int32_t *sel, void *ws, size_t ws_bytes,
+                           msa_stream stream);
+
+/* Whole prefill: msa_index_select (fused top-k) then msa_sparse_attn_prefill.
+ *   sel may be NULL (kept in ws); lse may be NULL.                      */
+int msa_forward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k, const msa_bf16 *v,
+                const msa_bf16 *q_idx, const msa_bf16 *k_idx, msa_bf16 *out, int32_t *sel,
+                float *lse, void *ws, size_t ws_bytes, msa_stream stream);
+
+/* Workspace bytes op (MSA_OP_*) needs for these params; 0 when p is invalid
+ * (see msa_last_error). */
+size_t msa_workspace_bytes(const msa_params *p, int op);
+
+/* Query-chunk length the prefill attention uses for these params: queries
+ * are processed in chunks of this many tokens so that per-block partial
+ * results stay within a fixed workspace budget (about 4.5 GiB).  Each chunk
+ * costs 5 kernel launches.  0 when p is invalid. */
+int msa_prefill_chunk_len(const msa_params *p);
+
+/* Synchronise `stream`, return the device status recorded in ws (MSA_OK or
+ * MSA_ERR_DEVICE_*), and reset it to MSA_OK. */
+int msa_read_status(void *ws, msa_stream stream);
+
+/* Message of the last error on this host thread ("" if none). */
+const char *msa_last_error(void);
+
+/* Library version string. */
+const char *msa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

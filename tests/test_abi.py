@@ -1,0 +1,82 @@
+"""CPU tests of the C-ABI boundary: the library loads, exports every entry
+point its header declares, sizes workspaces and rejects bad arguments
+before touching the device."""
+import ctypes
+
+import pytest
+
+import block_sparse_long_08_b200.msa as M
+
+
+def test_library_exports_header_symbols():
+    lib = M.lib()
+    names = M.header_functions()
+    assert {"msa_index_select", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
+            "msa_forward", "msa_workspace_bytes", "msa_last_error"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version():
+    assert b"sm_100a" in M.lib().msa_version()
+
+
+@pytest.mark.parametrize("L,top_k,G,H,di", [(2048, 4, 2, 8, 64), (32768, 16, 8, 32, 128),
+                                             (1048576, 16, 8, 32, 128)])
+def test_workspace_sizes(L, top_k, G, H, di):
+    p = M.make_params(1, L, H, G, 128, di, 128, top_k)
+    ws_sel = M.msa_workspace_bytes(p, M.MSA_OP_INDEX_SELECT)
+    ws_att = M.msa_workspace_bytes(p, M.MSA_OP_PREFILL_ATTN)
+    ws_fwd = M.msa_workspace_bytes(p, M.MSA_OP_FORWARD)
+    ws_dec = M.msa_workspace_bytes(p, M.MSA_OP_DECODE)
+    assert ws_sel >= 4
+    # forward = selection buffer + attention workspace
+    assert ws_fwd >= ws_att + 4 * L * G * top_k
+    # the partial-result budget bounds the prefill workspace
+    assert ws_att < 6 * 2**30
+    assert ws_dec < 64 * 2**20
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("d", 64, M.MSA_ERR_UNSUPPORTED), ("d_idx", 96, M.MSA_ERR_UNSUPPORTED),
+    ("block", 64, M.MSA_ERR_UNSUPPORTED), ("top_k", 33, M.MSA_ERR_UNSUPPORTED),
+    ("top_k", 0, M.MSA_ERR_INVALID_ARG), ("L", 1000, M.MSA_ERR_UNSUPPORTED),
+    ("H", 12, M.MSA_ERR_UNSUPPORTED), ("G", 3, M.MSA_ERR_INVALID_ARG),
+    ("B", -1, M.MSA_ERR_INVALID_ARG)])
+def test_bad_params_rejected_before_launch(field, value, code):
+    p = M.make_params(1, 2048, 8, 2, 128, 64, 128, 4)
+    setattr(p, field, value)
+    lib = M.lib()
+    dummy = ctypes.c_void_p(256)  # never dereferenced: the check fails first
+    rc = lib.msa_index_select(ctypes.byref(p), dummy, dummy, dummy, None, dummy, 1 << 20, None)
+    assert rc == code, (rc, M.msa_last_error())
+    assert M.msa_last_error()
+    assert lib.msa_workspace_bytes(ctypes.byref(p), 0) == 0
+
+
+def test_null_and_misaligned_pointers_rejected():
+    p = M.make_params(1, 2048, 8, 2, 128, 64, 128, 4)
+    lib = M.lib()
+    ok = ctypes.c_void_p(4096)
+    rc = lib.msa_index_select(ctypes.byref(p), None, ok, ok, None, ok, 1 << 20, None)
+    assert rc == M.MSA_ERR_INVALID_ARG
+    rc = lib.msa_index_select(ctypes.byref(p), ctypes.c_void_p(4098), ok, ok, None, ok, 1 << 20, None)
+    assert rc == M.MSA_ERR_INVALID_ARG
+    rc = lib.msa_index_select(ctypes.byref(p), ok, ok, ok, None, ctypes.c_void_p(4096 + 16), 1 << 20, None)
+    assert rc == M.MSA_ERR_WORKSPACE
+    rc = lib.msa_index_select(ctypes.byref(p), ok, ok, ok, None, ok, 8, None)
+    assert rc == M.MSA_ERR_WORKSPACE
+
+
+def test_empty_problem_is_noop():
+    p = M.make_params(0, 2048, 8, 2, 128, 64, 128, 4)
+    lib = M.lib()
+    assert lib.msa_index_select(ctypes.byref(p), None, None, None, None, None, 0, None) == M.MSA_OK
+    p = M.make_params(1, 0, 8, 2, 128, 64, 128, 4)
+    assert lib.msa_forward(ctypes.byref(p), None, None, None, None, None, None, None, None, None, 0,
+                           None) == M.MSA_OK
+
+
+def test_decode_rejects_more_than_eight_groups():
+    p = M.make_params(2, 4096, 32, 16, 128, 128, 128, 16)
+    assert M.lib().msa_workspace_bytes(ctypes.byref(p), M.MSA_OP_DECODE) == 0
