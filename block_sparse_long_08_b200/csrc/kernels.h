@@ -81,4 +81,7 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 
+// Sets the message msa_last_error() returns; returns `code`.
+int report_error(int code, const char *msg);
+
 }  // namespace msa

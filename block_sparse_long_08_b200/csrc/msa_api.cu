@@ -264,6 +264,11 @@ int run_prefill_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
 
 }  // namespace
 
+namespace msa {
+// Records an error message for msa_last_error() from other translation units.
+int report_error(int code, const char *msg) { return fail(code, "%s", msg); }
+}  // namespace msa
+
 extern "C" {
 
 const char *msa_last_error(void) { return g_err; }

@@ -64,6 +64,8 @@ def lib() -> ctypes.CDLL:
         L.msa_sparse_attn_prefill.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.msa_sparse_attn_decode.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.msa_forward.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.msa_sparse_attn_decode_noalloc.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+        L.msa_sparse_attn_decode_noalloc.restype = ctypes.c_int
         L.msa_workspace_bytes.argtypes = [pp, ctypes.c_int]
         L.msa_workspace_bytes.restype = _SZ
         L.msa_read_status.argtypes = [_P, _P]
@@ -230,6 +232,30 @@ def msa_sparse_attn_decode(q, q_idx, k_cache, v_cache, k_idx_cache, seq_lens, to
     _check(lib().msa_sparse_attn_decode(ctypes.byref(p), _ptr(q), _ptr(q_idx), _ptr(k_cache),
                                         _ptr(v_cache), _ptr(k_idx_cache), _ptr(seq_lens), _ptr(out),
                                         _ptr(sel), _ptr(ws), ws.numel(), _stream(stream)))
+    return (out, sel) if want_sel else out
+
+
+def msa_sparse_attn_decode_noalloc(q, q_idx, k_cache, v_cache, k_idx_cache, seq_lens, top_k: int, *,
+                                   scale: float = 0.0, want_sel: bool = False, out=None, sel=None,
+                                   stream=None):
+    """Decode step that passes no workspace: the library uses its own 16 MiB
+    device scratch (for callers that cannot allocate device memory at the
+    call site).  Same arguments and results as msa_sparse_attn_decode.  Only
+    the outputs are allocated here, and only when not passed in."""
+    for n, t in (("q", q), ("q_idx", q_idx), ("k_cache", k_cache), ("v_cache", v_cache),
+                 ("k_idx_cache", k_idx_cache)):
+        _req(t, n, torch.bfloat16)
+    _req(seq_lens, "seq_lens", torch.int32)
+    B, H, d = q.shape
+    Lmax, G = k_cache.shape[1], k_cache.shape[2]
+    p = make_params(B, Lmax, H, G, d, q_idx.shape[2], 128, top_k, scale)
+    if out is None:
+        out = torch.empty_like(q)
+    if sel is None and want_sel:
+        sel = torch.empty((B, G, top_k), dtype=torch.int32, device=q.device)
+    _check(lib().msa_sparse_attn_decode_noalloc(ctypes.byref(p), _ptr(q), _ptr(q_idx), _ptr(k_cache),
+                                                _ptr(v_cache), _ptr(k_idx_cache), _ptr(seq_lens),
+                                                _ptr(out), _ptr(sel), _stream(stream)))
     return (out, sel) if want_sel else out
 
 

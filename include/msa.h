@@ -136,6 +136,30 @@ int msa_sparse_attn_decode(const msa_params *p, const msa_bf16 *q, const msa_bf1
                            msa_bf16 *out, int32_t *sel, void *ws, size_t ws_bytes,
                            msa_stream stream);
 
+/* Decode step without a workspace argument, for callers that cannot
+ * allocate device memory where they run a decode step (engines that plan all
+ * device buffers at start-up and forbid allocation afterwards, plugin hosts
+ * that pass a library only the call's tensors).  The pages have no
+ * counterpart; this is a deployment convenience.
+ *   Arguments and results are those of msa_sparse_attn_decode, minus ws.
+ *   Scratch: a 16 MiB array in device memory owned by the library (every GPU
+ *     that loads the library keeps it reserved until the process exits).
+ *     Problems needing more scratch than that (msa_workspace_bytes(p,
+ *     MSA_OP_DECODE) > 16 MiB, e.g. 32 sequences at 1M tokens) return
+ *     MSA_ERR_WORKSPACE without launching anything.
+ *   The first call on each device looks the array's device address up with
+ *     cudaGetSymbolAddress; make that first call before any stream capture.
+ *   All calls on a device share the array and it keeps the last call's
+ *     contents: calls whose GPU work overlaps (other streams) race, so order
+ *     them.  Device-side input errors are not reported by this variant (its
+ *     status word is cleared on every call); an out-of-range length still
+ *     yields a zero output for that sequence.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+int msa_sparse_attn_decode_noalloc(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
+                                   const msa_bf16 *k_cache, const msa_bf16 *v_cache,
+                                   const msa_bf16 *k_idx_cache, const int32_t *seq_lens,
+                                   msa_bf16 *out, int32_t *sel, msa_stream stream);
+
 /* Whole prefill: msa_index_select (fused top-k) then msa_sparse_attn_prefill.
  *   sel may be NULL (kept in ws); lse may be NULL.                      */
 int msa_forward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k, const msa_bf16 *v,
