@@ -12,18 +12,25 @@
 // so only blocks j < b_t are scored, and every such block is entirely
 // visible.  For a 128-query tile i the work is the tile row j = 0..i-1.
 //
-// Kernel structure (persistent, one CTA per SM, 6 warps):
-//   warp 0   TMA producer: the tile's q_idx rows for GP groups (resident),
-//            then k_idx blocks two at a time into an NS-deep ring.
-//   warp 1   TMEM owner + MMA issuer: per (stage, group) one
-//            M=128 x N=256 x K=d_idx UMMA into one of two TMEM accumulators.
-//   warps 2-5 epilogue: thread r owns accumulator row r (one query); it
-//            reads 2 x 128 fp32 columns (two key blocks) from TMEM, max-pools
-//            each block and either stores the score or inserts it into its
-//            register-resident sorted list.
-// The two TMEM accumulators let the MMA of one (stage, group) overlap the
-// epilogue of the previous one.  One k_idx stage feeds GP groups, which
-// halves L2->SM traffic for GP = 2.
+// Kernel structure (persistent, one CTA per SM, 12 warps = 3 warpgroups):
+//   warp 0    TMA producer: the tile's q_idx rows for GP groups (resident),
+//             then k_idx blocks two at a time into an NS-deep ring.
+//   warp 1    TMEM owner + MMA issuer: per (stage, group) one
+//             M=128 x N=256 x K=d_idx UMMA into one of two TMEM accumulators.
+//   warps 2-3 idle (they complete the first warpgroup).
+//   warps 4-11 epilogue, two sets of four warps (one warp per TMEM lane
+//             quadrant).  Set h reads key block h (columns 128h..128h+127)
+//             of every accumulator: thread r owns row r (one query), loads
+//             its 128 columns in one TMEM round trip, frees the accumulator,
+//             max-pools the block and stores the score or inserts it into
+//             a register-resident sorted list.  At the end of a tile the two
+//             sets' lists (even / odd blocks) are merged through shared
+//             memory.
+// The TMEM accumulator is freed as soon as its columns sit in registers, so
+// the next UMMA into that slot waits one TMEM round trip, not the max-pool
+// and list work.  The first warpgroup gives registers to the epilogue
+// warpgroups (setmaxnreg: 3 x 128 x 168 = 128 x 56 + 256 x 224).
+// One k_idx stage feeds GP groups, which halves L2->SM traffic for GP = 2.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -38,17 +45,39 @@ namespace msa {
 
 namespace {
 
-template <int DI, int GP>
+template <int DI, int GP, int KCAP>
 struct IndexCfg {
   static constexpr int NCH = DI / 64;                 // 128-B K chunks per row
   static constexpr int Q_BYTES = GP * NCH * 16384;    // resident q_idx tiles
   static constexpr int STAGE_BYTES = NCH * 2 * 16384; // two k_idx blocks
-  static constexpr int NS_RAW = (200 * 1024 - Q_BYTES) / STAGE_BYTES;
+  static constexpr int MERGE_BYTES = GP * KCAP * 128 * 8;  // list exchange
+  static constexpr int NS_RAW = (232448 - 1280 - MERGE_BYTES - Q_BYTES) / STAGE_BYTES;
   static constexpr int NS = NS_RAW > 4 ? 4 : NS_RAW;
   static constexpr int BAR_OFF = Q_BYTES + NS * STAGE_BYTES;
-  static constexpr int SMEM = BAR_OFF + 256 + 1024;   // + barriers + align slack
-  static constexpr int THREADS = 192;
+  static constexpr int MERGE_OFF = BAR_OFF + 256;
+  static constexpr int SMEM = MERGE_OFF + MERGE_BYTES + 1024;  // + align slack
+  static constexpr int THREADS = 384;
+  static_assert(NS >= 2, "k_idx ring needs two stages");
+  static_assert(SMEM <= 232448, "shared memory budget");
 };
+
+// Register split between the warpgroups: the launch gives every thread 168
+// registers (384 threads); the producer/MMA warpgroup keeps 56 and the two
+// epilogue warpgroups take 224 (128*56 + 256*224 = 384*168).
+__device__ __forceinline__ void regs_dec_56() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+}
+__device__ __forceinline__ void regs_inc_224() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
+}
+__device__ __forceinline__ void epi_bar_sync() {  // the 8 epilogue warps
+  asm volatile("bar.sync 1, 256;" ::: "memory");
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 struct IndexWork {
   int i, b, gp, stages;
@@ -123,25 +152,30 @@ __device__ __forceinline__ void sort_ids_asc(int (&v)[KCAP]) {
   }
 }
 
-__device__ __forceinline__ float max128_from_tmem(uint32_t taddr) {
-  float m = -FLT_MAX;
-  float a[32], c[32];
+// Max over 4 x 32 fp32 values with three-input max (4 independent chains).
+__device__ __forceinline__ float max4x32(const float (&a)[32], const float (&b)[32],
+                                         const float (&c)[32], const float (&d)[32]) {
+  float m0 = max3f(a[0], a[1], a[2]), m1 = max3f(b[0], b[1], b[2]);
+  float m2 = max3f(c[0], c[1], c[2]), m3 = max3f(d[0], d[1], d[2]);
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    tmem_ld32(taddr + half * 64, a);
-    tmem_ld32(taddr + half * 64 + 32, c);
-    tmem_wait_ld();
-#pragma unroll
-    for (int x = 0; x < 32; x += 2) m = fmaxf(m, fmaxf(fmaxf(a[x], a[x + 1]), fmaxf(c[x], c[x + 1])));
+  for (int x = 3; x + 2 <= 31; x += 2) {
+    m0 = max3f(m0, a[x], a[x + 1]);
+    m1 = max3f(m1, b[x], b[x + 1]);
+    m2 = max3f(m2, c[x], c[x + 1]);
+    m3 = max3f(m3, d[x], d[x + 1]);
   }
-  return m;
+  m0 = fmaxf(m0, a[31]);
+  m1 = fmaxf(m1, b[31]);
+  m2 = fmaxf(m2, c[31]);
+  m3 = fmaxf(m3, d[31]);
+  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
 template <int DI, int GP, int KCAP>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(384, 1)
     msa_index_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k, const IndexArgs a) {
-  using C = IndexCfg<DI, GP>;
+  using C = IndexCfg<DI, GP, KCAP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -170,7 +204,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(b_accfull + 8 * s, 1);
-      mbar_init(b_accempty + 8 * s, 4);
+      mbar_init(b_accempty + 8 * s, 8);
     }
     *abort_flag = 0;
     mbar_init_fence();
@@ -184,7 +218,11 @@ __global__ void __launch_bounds__(192, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  if (warp == 0) {
+  if (warp < 4) {
+   // setmaxnreg is warpgroup-wide: all four warps of warpgroup 0 execute
+   // this one instruction, then split into their roles.
+   regs_dec_56();
+   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -218,7 +256,7 @@ __global__ void __launch_bounds__(192, 1)
         if (!ok) break;
       }
     }
-  } else if (warp == 1) {
+   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 256, 0, 0);
@@ -264,12 +302,17 @@ __global__ void __launch_bounds__(192, 1)
         if (!ok) break;
       }
     }
+   }  // warps 2-3: idle
   } else {
     // ------------------------------------------------------------ epilogue
+    regs_inc_224();  // the same instruction for both epilogue warpgroups
+    const int eset = (warp - 4) >> 2;          // key block h = eset of each job
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem_base + (uint32_t(quad * 32) << 16);
     const int k1 = a.top_k - 1;
+    float *m_score = reinterpret_cast<float *>(smem + C::MERGE_OFF);
+    int *m_id = reinterpret_cast<int *>(smem + C::MERGE_OFF + C::MERGE_BYTES / 2);
     uint32_t jc = 0;
     bool ok = true;
     for (int r = 0; ok; ++r) {
@@ -295,40 +338,83 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           tc_fence_after();
-          const int g = w.gp * GP + gi;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int j = 2 * s + h;
-            if (j < w.i) {
-              const float sc = max128_from_tmem(lane_base + slot * 256 + h * 128);
-              if (a.write_scores) {
-                a.scores[((size_t(w.b) * a.G + g) * a.L + t) * a.nb + j] = sc;
-              } else if (sc > thr[gi]) {
-                list_insert<KCAP>(ls[gi], lj[gi], sc, j);
-                thr[gi] = list_threshold<KCAP>(ls[gi], k1);
-              }
-            }
+          const int j = 2 * s + eset;
+          float v0[32], v1[32], v2[32], v3[32];
+          if (j < w.i) {
+            const uint32_t ta = lane_base + slot * 256 + eset * 128;
+            tmem_ld32(ta, v0);
+            tmem_ld32(ta + 32, v1);
+            tmem_ld32(ta + 64, v2);
+            tmem_ld32(ta + 96, v3);
+            tmem_wait_ld();
           }
+          // the accumulator is in registers: hand the slot back to the MMA
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(b_accempty + 8 * slot);
           ++jc;
+          if (j < w.i) {
+            const float sc = max4x32(v0, v1, v2, v3);
+            if (a.write_scores) {
+              const int g = w.gp * GP + gi;
+              a.scores[((size_t(w.b) * a.G + g) * a.L + t) * a.nb + j] = sc;
+            } else if (sc > thr[gi]) {
+              list_insert<KCAP>(ls[gi], lj[gi], sc, j);
+              thr[gi] = list_threshold<KCAP>(ls[gi], k1);
+            }
+          }
         }
       }
-      if (!ok) break;
+      // After a failed wait, items without a merge end here; an item with a
+      // merge still meets the other set at both barriers below, then every
+      // epilogue warp leaves together.
+      if (a.write_scores) {
+        if (!ok) break;
+        if (eset == 0) {
 #pragma unroll
-      for (int gi = 0; gi < GP; ++gi) {
-        const int g = w.gp * GP + gi;
-        const size_t rowid = (size_t(w.b) * a.G + g) * a.L + t;
-        if (a.write_scores) {
-          float *dst = a.scores + rowid * a.nb;
-          for (int j = w.i; j < a.nb; ++j) dst[j] = -INFINITY;
-          continue;
+          for (int gi = 0; gi < GP; ++gi) {
+            const int g = w.gp * GP + gi;
+            float *dst = a.scores + ((size_t(w.b) * a.G + g) * a.L + t) * a.nb;
+            for (int j = w.i; j < a.nb; ++j) dst[j] = -INFINITY;
+          }
         }
-        int32_t *dst = a.sel + rowid * a.top_k;
-        if (w.i + 1 <= a.top_k) {
-          for (int k = 0; k < a.top_k; ++k) dst[k] = (k <= w.i) ? k : -1;
-        } else {
+        continue;
+      }
+      if (w.i + 1 <= a.top_k) {
+        if (!ok) break;
+        if (eset == 0) {
+#pragma unroll
+          for (int gi = 0; gi < GP; ++gi) {
+            const int g = w.gp * GP + gi;
+            int32_t *dst = a.sel + ((size_t(w.b) * a.G + g) * a.L + t) * a.top_k;
+            for (int k = 0; k < a.top_k; ++k) dst[k] = (k <= w.i) ? k : -1;
+          }
+        }
+        continue;
+      }
+      // merge the odd-block lists (set 1) into the even-block lists (set 0)
+      if (eset == 1) {
+#pragma unroll
+        for (int gi = 0; gi < GP; ++gi)
+#pragma unroll
+          for (int k = 0; k < KCAP; ++k) {
+            m_score[(gi * KCAP + k) * 128 + row] = ls[gi][k];
+            m_id[(gi * KCAP + k) * 128 + row] = lj[gi][k];
+          }
+      }
+      epi_bar_sync();
+      const bool abort_now = (*abort_flag != 0);   // the same value for all 8 warps
+      if (eset == 0 && !abort_now) {
+#pragma unroll
+        for (int gi = 0; gi < GP; ++gi) {
+#pragma unroll
+          for (int k = 0; k < KCAP; ++k) {
+            const float sc = m_score[(gi * KCAP + k) * 128 + row];
+            const int id = m_id[(gi * KCAP + k) * 128 + row];
+            if (id != INT_MAX) list_insert<KCAP>(ls[gi], lj[gi], sc, id);
+          }
+          const int g = w.gp * GP + gi;
+          int32_t *dst = a.sel + ((size_t(w.b) * a.G + g) * a.L + t) * a.top_k;
           int ids[KCAP];
 #pragma unroll
           for (int k = 0; k < KCAP; ++k) ids[k] = (k < k1) ? lj[gi][k] : INT_MAX;
@@ -337,12 +423,12 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int k = 0; k < KCAP; k += 4) {
               if (k < a.top_k) {
-                int4 v;
-                v.x = (k + 0 < k1) ? ids[k + 0] : (k + 0 == k1 ? w.i : -1);
-                v.y = (k + 1 < k1) ? ids[k + 1] : (k + 1 == k1 ? w.i : -1);
-                v.z = (k + 2 < k1) ? ids[k + 2] : (k + 2 == k1 ? w.i : -1);
-                v.w = (k + 3 < k1) ? ids[k + 3] : (k + 3 == k1 ? w.i : -1);
-                *reinterpret_cast<int4 *>(dst + k) = v;
+                int4 o;
+                o.x = (k + 0 < k1) ? ids[k + 0] : (k + 0 == k1 ? w.i : -1);
+                o.y = (k + 1 < k1) ? ids[k + 1] : (k + 1 == k1 ? w.i : -1);
+                o.z = (k + 2 < k1) ? ids[k + 2] : (k + 2 == k1 ? w.i : -1);
+                o.w = (k + 3 < k1) ? ids[k + 3] : (k + 3 == k1 ? w.i : -1);
+                *reinterpret_cast<int4 *>(dst + k) = o;
               }
             }
           } else {
@@ -354,6 +440,8 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
+      epi_bar_sync();   // set 1 may overwrite the exchange area next tile
+      if (abort_now) break;
     }
   }
 
@@ -368,7 +456,7 @@ __global__ void __launch_bounds__(192, 1)
 template <int DI, int GP, int KCAP>
 cudaError_t launch_index_t(const CUtensorMap &tq, const CUtensorMap &tk, const IndexArgs &a,
                            int num_sms, cudaStream_t st) {
-  using C = IndexCfg<DI, GP>;
+  using C = IndexCfg<DI, GP, KCAP>;
   auto kern = msa_index_kernel<DI, GP, KCAP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
