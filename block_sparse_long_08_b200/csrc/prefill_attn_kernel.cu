@@ -38,7 +38,7 @@ constexpr int kSmemK = 0;
 constexpr int kSmemV = 32768;
 constexpr int kSmemQ = 65536;  // Q tile, then P tile
 constexpr int kSmemBar = 98304;
-constexpr int kAttnSmem = kSmemBar + 1024 + 1024;
+constexpr int kAttnSmem = kSmemBar + 64 + 1024 + 1024;  // bars, items, 2 lists, align slack
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -51,6 +51,36 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
 }
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+template <int R>
+struct AttnItemWalk {  // thread 0's position in the CTA's item range
+  int cur = -1;        // bgj whose K/V sit in shared memory
+  int wb = 0, it_lo = 0, it_hi = 0, l_lo = 0, l_hi = 0;
+};
+
+// Gather the q rows of a work item into the swizzled Q tile: row = qi*R + hh,
+// 16 granules of 16 B per row; rows past the item's queries are zeroed.
+template <int R>
+__device__ __forceinline__ void gather_q(const AttnArgs &a, uint32_t s_q, const int *list, int n,
+                                         int b, int g, int tid) {
+#pragma unroll 4
+  for (int it = 0; it < 16; ++it) {
+    const int idx = it * kAttnThreads + tid;
+    const int row = idx >> 4;
+    const int gran = idx & 15;
+    const int qi = row / R;
+    const int hh = row % R;
+    const uint32_t dst = s_q + (gran >> 3) * 16384 + sw128_offset(row, gran & 7);
+    if (qi < n) {
+      const int t = list[qi] >> 5;
+      const uint16_t *src =
+          a.q + ((size_t(b) * a.L + t) * a.H + size_t(g) * R + hh) * kHeadDim + gran * 8;
+      cp_async16(dst, src);
+    } else {
+      asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(dst), "r"(0) : "memory");
+    }
+  }
 }
 
 template <int R>
@@ -69,8 +99,8 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   const uint32_t b_mma = smem_u32(&bars[1]);
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(&bars[2]);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
-  int *s_item = reinterpret_cast<int *>(tmem_holder + 2);   // bgj, start, n
-  int *s_list = reinterpret_cast<int *>(smem + kSmemBar + 64);  // <= 128 entries
+  int *s_item = reinterpret_cast<int *>(smem + kSmemBar + 32);    // [2][4]: bgj, start, n, new K/V
+  int *s_list = reinterpret_cast<int *>(smem + kSmemBar + 64);    // [2][128]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -98,59 +128,80 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, 0, 1);
   uint32_t kv_ph = 0, mma_ph = 0;
 
-  for (int w = blockIdx.x; w < n_items; w += gridDim.x) {
-    // ---- locate the item: bgj with item_off[bgj] <= w < item_off[bgj+1]
+  // Each CTA takes a contiguous range of work items.  Items are ordered by
+  // (b, g, key block), so consecutive items mostly share their K/V block: it
+  // stays in shared memory and is only fetched again when the block changes.
+  // The next item's descriptor and query list are fetched at the start of an
+  // item, and its q rows and K/V are requested as soon as this item's second
+  // UMMA has consumed the shared tiles, so those loads overlap the stores of
+  // this item's partial results.
+  const int per = (n_items + gridDim.x - 1) / gridDim.x;
+  const int w_begin = blockIdx.x * per;
+  const int w_end = min(n_items, w_begin + per);
+  AttnItemWalk<R> wk;
+  auto describe = [&](int w, int *dst) {  // thread 0: item w -> dst[0..3]
+    while (w >= wk.it_hi) {
+      ++wk.wb;
+      wk.it_lo = wk.it_hi; wk.it_hi = a.item_off[wk.wb + 1];
+      wk.l_lo = wk.l_hi; wk.l_hi = a.list_off[wk.wb + 1];
+    }
+    const int start = wk.l_lo + (w - wk.it_lo) * QPI;
+    dst[0] = wk.wb;
+    dst[1] = start;
+    dst[2] = min(QPI, wk.l_hi - start);
+    dst[3] = (wk.wb != wk.cur);
+    wk.cur = wk.wb;
+  };
+  auto issue_kv = [&](int bgj) {  // thread 0
+    const int j = bgj % a.nb;
+    const int bg = bgj / a.nb;
+    const int g = bg % a.G;
+    const int b = bg / a.G;
+    mbar_arrive_expect_tx(b_kv, 65536);
+    const int z = b * a.L + j * kBlock;
+    tma_load_3d(s_k, &tm_k, b_kv, 0, g, z);
+    tma_load_3d(s_k + 16384, &tm_k, b_kv, 64, g, z);
+    tma_load_3d(s_v, &tm_v, b_kv, 0, g, z);
+    tma_load_3d(s_v + 16384, &tm_v, b_kv, 64, g, z);
+  };
+
+  if (w_begin < w_end) {
     if (tid == 0) {
-      int lo = 0, hi = n_bgj - 1;
+      int lo = 0, hi = n_bgj - 1;  // first bgj with item_off[bgj+1] > w_begin
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (a.item_off[mid] <= w) lo = mid; else hi = mid - 1;
+        if (a.item_off[mid] <= w_begin) lo = mid; else hi = mid - 1;
       }
-      const int c = w - a.item_off[lo];
-      const int start = a.list_off[lo] + c * QPI;
-      const int n = min(QPI, a.list_off[lo + 1] - start);
-      s_item[0] = lo;
-      s_item[1] = start;
-      s_item[2] = n;
-      const int j = lo % a.nb;
-      const int bg = lo / a.nb;
-      const int g = bg % a.G;
-      const int b = bg / a.G;
-      mbar_arrive_expect_tx(b_kv, 65536);
-      const int z = b * a.L + j * kBlock;
-      tma_load_3d(s_k, &tm_k, b_kv, 0, g, z);
-      tma_load_3d(s_k + 16384, &tm_k, b_kv, 64, g, z);
-      tma_load_3d(s_v, &tm_v, b_kv, 0, g, z);
-      tma_load_3d(s_v + 16384, &tm_v, b_kv, 64, g, z);
+      wk.wb = lo;
+      wk.it_lo = a.item_off[lo]; wk.it_hi = a.item_off[lo + 1];
+      wk.l_lo = a.list_off[lo]; wk.l_hi = a.list_off[lo + 1];
+      describe(w_begin, s_item);
+      issue_kv(s_item[0]);
     }
     __syncthreads();
-    const int bgj = s_item[0];
-    const int start = s_item[1];
-    const int n = s_item[2];
+    if (tid < s_item[2]) s_list[tid] = a.list[s_item[1] + tid];
+    __syncthreads();
+    gather_q<R>(a, s_q, s_list, s_item[2], s_item[0] / (a.nb * a.G), (s_item[0] / a.nb) % a.G, tid);
+  }
+
+  int buf = 0;
+  for (int w = w_begin; w < w_end; ++w) {
+    const int *it = s_item + 4 * buf;
+    const int *lst = s_list + 128 * buf;
+    const int bgj = it[0];
+    const int n = it[2];
+    const bool kv_new = it[3] != 0;
     const int j = bgj % a.nb;
     const int g = (bgj / a.nb) % a.G;
     const int b = bgj / (a.nb * a.G);
-    if (tid < n) s_list[tid] = a.list[start + tid];
+    const bool has_next = w + 1 < w_end;
+    int *nit = s_item + 4 * (buf ^ 1);
+    int *nlst = s_list + 128 * (buf ^ 1);
+    if (has_next && tid == 0) describe(w + 1, nit);
     __syncthreads();
+    if (has_next && tid < nit[2]) nlst[tid] = a.list[nit[1] + tid];
 
-    // ---- gather the Q tile: row = qi*R + hh, 16 granules of 16 B per row
-#pragma unroll 4
-    for (int it = 0; it < 16; ++it) {
-      const int idx = it * kAttnThreads + tid;
-      const int row = idx >> 4;
-      const int gran = idx & 15;
-      const int qi = row / R;
-      const int hh = row % R;
-      const uint32_t dst = s_q + (gran >> 3) * 16384 + sw128_offset(row, gran & 7);
-      if (qi < n) {
-        const int t = s_list[qi] >> 5;
-        const uint16_t *src =
-            a.q + ((size_t(b) * a.L + t) * a.H + size_t(g) * R + hh) * kHeadDim + gran * 8;
-        cp_async16(dst, src);
-      } else {
-        asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(dst), "r"(0) : "memory");
-      }
-    }
+    // ---- this item's q rows have landed
     cp_async_wait_all();
     fence_proxy_async_smem();
     __syncthreads();
@@ -158,7 +209,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     // ---- S = Q K^T
     int ok_kv = 1;
     if (tid == 0) {
-      ok_kv = mbar_wait(b_kv, kv_ph, abort_flag, a.status) ? 1 : 0;
+      if (kv_new) ok_kv = mbar_wait(b_kv, kv_ph, abort_flag, a.status) ? 1 : 0;
       if (ok_kv) {
         tc_fence_after();
 #pragma unroll
@@ -171,7 +222,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
         umma_commit(b_mma);
       }
     }
-    kv_ph ^= 1;
+    if (kv_new) kv_ph ^= 1;
     // every exit decision below is taken by the whole CTA at one barrier
     if (__syncthreads_or(!ok_kv)) break;
     const bool ok1 = mbar_wait(b_mma, mma_ph, abort_flag, a.status);
@@ -182,7 +233,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     // ---- softmax on row `tid`
     const int qi = tid / R;
     const bool valid = qi < n;
-    const int ent = valid ? s_list[qi] : 0;
+    const int ent = valid ? lst[qi] : 0;
     const int t = ent >> 5;
     const int lim = valid ? (t - j * kBlock) : -1;  // last visible column
     float sv[128];
@@ -236,6 +287,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     if (__syncthreads_or(!ok2)) break;
     tc_fence_after();
 
+    // ---- the shared tiles are free: request the next item's K/V and q rows
+    if (has_next) {
+      if (tid == 0 && nit[3]) issue_kv(nit[0]);
+      gather_q<R>(a, s_q, nlst, nit[2], nit[0] / (a.nb * a.G), (nit[0] / a.nb) % a.G, tid);
+    }
+
     // ---- store the normalised partial and its lse
     {
       float o[128];
@@ -269,8 +326,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     }
     tc_fence_before();
     __syncthreads();
+    buf ^= 1;
   }
 
+  cp_async_wait_all();   // nothing may still be landing in shared memory
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -336,14 +395,28 @@ __global__ void __launch_bounds__(256) msa_combine_kernel(const CombineArgs a) {
     wsum = wmine;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-    for (int s = 0; s < a.top_k; ++s) {
-      const float ws = __shfl_sync(0xffffffffu, wmine, s);
-      if (ws == 0.f) continue;
-      const uint2 v = *reinterpret_cast<const uint2 *>(a.part_o + (prow0 + s) * kHeadDim + lane * 4);
-      acc[0] = fmaf(ws, bf16_lo(v.x), acc[0]);
-      acc[1] = fmaf(ws, bf16_hi(v.x), acc[1]);
-      acc[2] = fmaf(ws, bf16_lo(v.y), acc[2]);
-      acc[3] = fmaf(ws, bf16_hi(v.y), acc[3]);
+    const unsigned vmask = __ballot_sync(0xffffffffu, mine);
+    // up to 8 partial rows in flight per lane before they are consumed
+    for (int s0 = 0; s0 < a.top_k; s0 += 8) {
+      uint2 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int s = s0 + u;
+        v[u] = make_uint2(0u, 0u);
+        if (s < a.top_k && ((vmask >> s) & 1u))
+          v[u] = __ldcs(reinterpret_cast<const uint2 *>(a.part_o + (prow0 + s) * kHeadDim + lane * 4));
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int s = s0 + u;
+        const float ws = __shfl_sync(0xffffffffu, wmine, s & 31);
+        if (s < a.top_k && ((vmask >> s) & 1u)) {
+          acc[0] = fmaf(ws, bf16_lo(v[u].x), acc[0]);
+          acc[1] = fmaf(ws, bf16_hi(v[u].x), acc[1]);
+          acc[2] = fmaf(ws, bf16_lo(v[u].y), acc[2]);
+          acc[3] = fmaf(ws, bf16_hi(v[u].y), acc[3]);
+        }
+      }
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;

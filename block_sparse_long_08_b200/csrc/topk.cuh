@@ -6,21 +6,75 @@
 // top_k - 1 come from the earlier blocks.  Equal scores go to the lower
 // block id.
 //
-// One warp handles one row of block scores.  The warp keeps the best
-// top_k-1 (score, id) pairs sorted in descending order, one pair per lane,
-// and a threshold (the worst kept score).  Scores are read 32 at a time,
-// coalesced; only lanes beating the threshold enter a ballot, and those
-// candidates are inserted one at a time in lane order (ascending id) with
-// shuffles.  For unstructured scores the expected number of insertions over
-// n blocks is about k*ln(n/k), so the pass costs about one coalesced read of
-// the row.  The kept ids plus the local block are then sorted ascending by
-// a 32-lane bitonic network.
+// A warp keeps the best k1 = top_k-1 (score, id) pairs in (score desc, id
+// asc) order, one pair per lane, and a threshold (the worst kept score).
+// Candidates are offered 32 at a time, in increasing id order; only lanes
+// beating the threshold enter a ballot, and those are inserted one at a time
+// in lane order with shuffles.  Because candidates arrive in id order, an
+// equal score never displaces a kept entry, which is the lower-id rule.  For
+// unstructured scores the expected number of insertions over n blocks is
+// about k*ln(n/k), so a pass costs about one coalesced read of the row.  The
+// kept ids plus the local block are finally sorted ascending by a 32-lane
+// bitonic network.
 #pragma once
 #include <cfloat>
 #include <climits>
 #include <cstdint>
 
 namespace msa {
+
+struct WarpTopk {
+  float ls;   // this lane's kept score (lane < k1)
+  int lj;     // this lane's kept id
+  float thr;  // worst kept score (warp-uniform)
+};
+
+__device__ __forceinline__ void warp_topk_init(WarpTopk &st) {
+  st.ls = -FLT_MAX;
+  st.lj = INT_MAX;
+  st.thr = -FLT_MAX;
+}
+
+// Offer one candidate per lane (s, j, valid); lanes' candidates must be in
+// increasing id order across lanes and after every earlier offer.
+__device__ __forceinline__ void warp_topk_offer(WarpTopk &st, float s, int j, bool valid, int k1) {
+  const int lane = threadIdx.x & 31;
+  unsigned m = __ballot_sync(0xffffffffu, valid && (s > st.thr));
+  while (m) {
+    const int src = __ffs(m) - 1;
+    m &= m - 1;
+    const float cs = __shfl_sync(0xffffffffu, s, src);
+    const int cj = __shfl_sync(0xffffffffu, j, src);
+    if (cs > st.thr) {
+      const int p = __popc(__ballot_sync(0xffffffffu, lane < k1 && st.ls >= cs));
+      const float us = __shfl_up_sync(0xffffffffu, st.ls, 1);
+      const int uj = __shfl_up_sync(0xffffffffu, st.lj, 1);
+      if (lane < k1 && lane > p) { st.ls = us; st.lj = uj; }
+      if (lane == p) { st.ls = cs; st.lj = cj; }
+      st.thr = __shfl_sync(0xffffffffu, st.ls, k1 - 1);
+    }
+  }
+}
+
+// Offer the scores of blocks [lo, hi) of `row`, four coalesced loads ahead.
+__device__ __forceinline__ void warp_topk_scan(WarpTopk &st, const float *__restrict__ row, int lo,
+                                               int hi, int k1) {
+  const int lane = threadIdx.x & 31;
+  for (int base = lo; base < hi; base += 128) {
+    float s4[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = base + u * 32 + lane;
+      s4[u] = (j < hi) ? __ldg(row + j) : -FLT_MAX;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int jb = base + u * 32;
+      if (jb >= hi) break;
+      warp_topk_offer(st, s4[u], jb + lane, jb + lane < hi, k1);
+    }
+  }
+}
 
 __device__ __forceinline__ int warp_bitonic_sort_asc(int v, int lane) {
 #pragma unroll
@@ -36,7 +90,18 @@ __device__ __forceinline__ int warp_bitonic_sort_asc(int v, int lane) {
   return v;
 }
 
-// row: scores of blocks 0..bt-1 (the local block bt is not read).
+// Kept ids + local block bt, ascending, into out[0..top_k).
+__device__ __forceinline__ void warp_topk_write(const WarpTopk &st, int bt, int top_k,
+                                                int32_t *__restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int k1 = top_k - 1;
+  int id = (lane < k1) ? st.lj : (lane == k1 ? bt : INT_MAX);
+  id = warp_bitonic_sort_asc(id, lane);
+  if (lane < top_k) out[lane] = id;
+}
+
+// The selection rule for the block-score row of a query whose local block
+// is bt: blocks 0..bt-1 are candidates (the local block is not read).
 // Writes top_k ints to out: selected ids ascending, -1 padding.
 __device__ __forceinline__ void warp_topk_select(const float *__restrict__ row, int bt, int top_k,
                                                  int32_t *__restrict__ out) {
@@ -45,41 +110,14 @@ __device__ __forceinline__ void warp_topk_select(const float *__restrict__ row, 
     for (int k = lane; k < top_k; k += 32) out[k] = (k <= bt) ? k : -1;
     return;
   }
-  const int k1 = top_k - 1;
-  float ls = -FLT_MAX;
-  int lj = INT_MAX;
-  float thr = -FLT_MAX;
-  for (int base = 0; base < bt; base += 128) {
-    float s4[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int j = base + u * 32 + lane;
-      s4[u] = (j < bt) ? __ldg(row + j) : -FLT_MAX;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int jb = base + u * 32;
-      if (jb >= bt) break;
-      const float s = s4[u];
-      unsigned m = __ballot_sync(0xffffffffu, (jb + lane < bt) && (s > thr));
-      while (m) {
-        const int src = __ffs(m) - 1;
-        m &= m - 1;
-        const float cs = __shfl_sync(0xffffffffu, s, src);
-        if (cs > thr) {
-          const int p = __popc(__ballot_sync(0xffffffffu, lane < k1 && ls >= cs));
-          const float us = __shfl_up_sync(0xffffffffu, ls, 1);
-          const int uj = __shfl_up_sync(0xffffffffu, lj, 1);
-          if (lane < k1 && lane > p) { ls = us; lj = uj; }
-          if (lane == p) { ls = cs; lj = jb + src; }
-          thr = __shfl_sync(0xffffffffu, ls, k1 - 1);
-        }
-      }
-    }
+  if (top_k == 1) {            // only the local block
+    if (lane == 0) out[0] = bt;
+    return;
   }
-  int id = (lane < k1) ? lj : (lane == k1 ? bt : INT_MAX);
-  id = warp_bitonic_sort_asc(id, lane);
-  if (lane < top_k) out[lane] = id;
+  WarpTopk st;
+  warp_topk_init(st);
+  warp_topk_scan(st, row, 0, bt, top_k - 1);
+  warp_topk_write(st, bt, top_k, out);
 }
 
 }  // namespace msa

@@ -232,6 +232,50 @@ def test_decode_matches_oracle(B, Lmax, G, H, di, top_k, lens):
     assert mx <= P.OUT_MAX_ABS and mean <= P.OUT_MEAN_ABS, (mx, mean)
 
 
+@pytest.mark.parametrize("zero_keys", [False, True])
+def test_decode_integer_inputs_select_bit_exact(zero_keys):
+    """Exact scores (small integers) make ties real: the multi-warp top-k
+    merge must keep the lower block id exactly as the oracle does."""
+    shape = I.DecodeShape(B=3, Lmax=8192, H=8, G=2, d=128, d_idx=64, top_k=6)
+    x = I.decode_inputs(shape, 12)
+    qi = I.small_integer_like(x["q_idx"], 13, -1, 1)
+    ki = torch.zeros_like(x["k_idx_cache"]) if zero_keys else I.small_integer_like(x["k_idx_cache"], 14, -1, 1)
+    lens = [8192, 5000, 700]
+    d = {n: x[n].to(DEV) for n in ("q", "k_cache", "v_cache")}
+    _, sel = M.msa_sparse_attn_decode(d["q"], qi.to(DEV), d["k_cache"], d["v_cache"], ki.to(DEV),
+                                      torch.tensor(lens, dtype=torch.int32, device=DEV), 6,
+                                      want_sel=True)
+    sel = sel.cpu().numpy()
+    q64, k64 = O.as_f64(qi), O.as_f64(ki)
+    for b in range(3):
+        t = lens[b] - 1
+        for g in range(2):
+            bs = O.block_scores_row(q64[b, g], k64[b], t, 128)
+            want = O.select_blocks_row(bs, t, 128, 6)
+            assert list(sel[b, g]) == want + [-1] * (6 - len(want)), (b, g, sel[b, g], want)
+
+
+def test_decode_long_row_integer_ties():
+    """One sequence at 1M tokens (8192 blocks): every one of the 16 scanning
+    warps holds candidates, and integer scores force exact ties."""
+    Lmax = 1048576
+    shape = I.DecodeShape(B=1, Lmax=Lmax, H=8, G=2, d=128, d_idx=64, top_k=16)
+    gen = torch.Generator().manual_seed(15)
+    qi = torch.randint(-1, 2, (1, 2, 64), generator=gen).to(torch.bfloat16)
+    ki = torch.randint(-1, 2, (1, Lmax, 64), generator=gen).to(torch.bfloat16)
+    q = torch.randn((1, 8, 128), generator=gen).to(torch.bfloat16)
+    kc = torch.zeros((1, Lmax, 2, 128), dtype=torch.bfloat16)
+    _, sel = M.msa_sparse_attn_decode(q.to(DEV), qi.to(DEV), kc.to(DEV), kc.to(DEV), ki.to(DEV),
+                                      torch.tensor([Lmax], dtype=torch.int32, device=DEV), 16,
+                                      want_sel=True)
+    sel = sel.cpu().numpy()
+    q64, k64 = O.as_f64(qi), O.as_f64(ki)
+    for g in range(2):
+        bs = O.block_scores_row(q64[0, g], k64[0], Lmax - 1, 128)
+        want = O.select_blocks_row(bs, Lmax - 1, 128, 16)
+        assert list(sel[0, g]) == want, (g, sel[0, g], want)
+
+
 def test_decode_bad_length_sets_status():
     shape = I.DecodeShape(B=2, Lmax=1024, H=8, G=2, d=128, d_idx=128, top_k=4)
     x = {n: t.to(DEV) for n, t in I.decode_inputs(shape, 10).items() if t.dtype == torch.bfloat16}
