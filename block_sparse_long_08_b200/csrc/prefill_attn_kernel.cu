@@ -8,18 +8,24 @@
 //
 // One work item = one (b, g, key block j) and up to 128/R queries that
 // selected j, each with its R heads: a 128-row tile.  Per item:
-//   TMA      K_j, V_j (128 x 128 bf16 each, 128B-swizzled) into smem
+//   TMA      K_j (128 x 128 bf16, 128B-swizzled) into the K/V buffer
 //   gather   the tile's q rows (R heads of a query are 256*R contiguous
 //            bytes) into a swizzled smem tile with cp.async
 //   UMMA     S = Q K_j^T   (M=128, N=128, K=128) into TMEM
+//   TMA      V_j into the K/V buffer, now that S has consumed K_j; the load
+//            overlaps the softmax
 //   softmax  thread r owns row r: mask s <= t, row max, exp2, row sum,
 //            P = exp(...) as bf16 into smem (over the dead Q tile)
-//   UMMA     O = P V_j     (V consumed MN-major straight from its TMA tile)
+//   UMMA     O = P V_j into the same TMEM columns as S (V consumed MN-major
+//            straight from its TMA tile)
 //   store    O / l as a bf16 partial and lse = ln(sum exp(scale q.k)) per
 //            (t, head, slot); a second kernel merges a row's <= top_k
 //            partials.
-// Two CTAs share an SM (96 KB smem and 256 TMEM columns each), so one CTA's
-// softmax overlaps the other's MMAs and loads.
+// A CTA holds one 32 KB K/V buffer, one 32 KB Q/P tile and 128 TMEM columns,
+// so three CTAs share an SM and their sequential phases overlap.  The next
+// item's query list is fetched while this item computes, and its K and q
+// rows are requested as soon as this item's second UMMA has consumed the
+// shared tiles, so those loads overlap the partial-result stores.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -34,10 +40,10 @@ namespace msa {
 namespace {
 
 constexpr int kAttnThreads = 128;
-constexpr int kSmemK = 0;
-constexpr int kSmemV = 32768;
-constexpr int kSmemQ = 65536;  // Q tile, then P tile
-constexpr int kSmemBar = 98304;
+constexpr int kAttnCtasPerSm = 3;
+constexpr int kSmemKV = 0;      // K tile, then V tile
+constexpr int kSmemQ = 32768;   // Q tile, then P tile
+constexpr int kSmemBar = 65536;
 constexpr int kAttnSmem = kSmemBar + 64 + 1024 + 1024;  // bars, items, 2 lists, align slack
 
 __device__ __forceinline__ float fast_exp2(float x) {
@@ -53,9 +59,7 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-template <int R>
 struct AttnItemWalk {  // thread 0's position in the CTA's item range
-  int cur = -1;        // bgj whose K/V sit in shared memory
   int wb = 0, it_lo = 0, it_hi = 0, l_lo = 0, l_hi = 0;
 };
 
@@ -84,41 +88,41 @@ __device__ __forceinline__ void gather_q(const AttnArgs &a, uint32_t s_q, const 
 }
 
 template <int R>
-__global__ void __launch_bounds__(kAttnThreads, 2)
+__global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
     msa_prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
   constexpr int QPI = 128 / R;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-  const uint32_t s_k = smem_u32(smem + kSmemK);
-  const uint32_t s_v = smem_u32(smem + kSmemV);
+  const uint32_t s_kv = smem_u32(smem + kSmemKV);
   const uint32_t s_q = smem_u32(smem + kSmemQ);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSmemBar);
-  const uint32_t b_kv = smem_u32(&bars[0]);
-  const uint32_t b_mma = smem_u32(&bars[1]);
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(&bars[2]);
+  const uint32_t b_k = smem_u32(&bars[0]);
+  const uint32_t b_v = smem_u32(&bars[1]);
+  const uint32_t b_mma = smem_u32(&bars[2]);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(&bars[3]);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
-  int *s_item = reinterpret_cast<int *>(smem + kSmemBar + 32);    // [2][4]: bgj, start, n, new K/V
+  int *s_item = reinterpret_cast<int *>(smem + kSmemBar + 32);    // [2][4]: bgj, start, n, -
   int *s_list = reinterpret_cast<int *>(smem + kSmemBar + 64);    // [2][128]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   if (tid == 0) {
-    mbar_init(b_kv, 1);
+    mbar_init(b_k, 1);
+    mbar_init(b_v, 1);
     mbar_init(b_mma, 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_holder), 256);
+    tmem_alloc(smem_u32(tmem_holder), 128);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_s = *tmem_holder;
-  const uint32_t tmem_o = tmem_s + 128;
+  const uint32_t tmem_acc = *tmem_holder;   // S, then O
   const uint32_t lane_off = uint32_t(warp * 32) << 16;
 
   const int n_bgj = a.B * a.G * a.nb;
@@ -126,20 +130,15 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   if (n_items > a.max_items && tid == 0) atomicCAS(a.status, 0, kStatusBadInput);
   constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
   constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, 0, 1);
-  uint32_t kv_ph = 0, mma_ph = 0;
+  uint32_t k_ph = 0, v_ph = 0, mma_ph = 0;
 
-  // Each CTA takes a contiguous range of work items.  Items are ordered by
-  // (b, g, key block), so consecutive items mostly share their K/V block: it
-  // stays in shared memory and is only fetched again when the block changes.
-  // The next item's descriptor and query list are fetched at the start of an
-  // item, and its q rows and K/V are requested as soon as this item's second
-  // UMMA has consumed the shared tiles, so those loads overlap the stores of
-  // this item's partial results.
+  // Each CTA takes a contiguous range of work items (ordered by (b, g, key
+  // block), so consecutive items mostly read the same K/V block from L2).
   const int per = (n_items + gridDim.x - 1) / gridDim.x;
   const int w_begin = blockIdx.x * per;
   const int w_end = min(n_items, w_begin + per);
-  AttnItemWalk<R> wk;
-  auto describe = [&](int w, int *dst) {  // thread 0: item w -> dst[0..3]
+  AttnItemWalk wk;
+  auto describe = [&](int w, int *dst) {  // thread 0: item w -> dst[0..2]
     while (w >= wk.it_hi) {
       ++wk.wb;
       wk.it_lo = wk.it_hi; wk.it_hi = a.item_off[wk.wb + 1];
@@ -149,20 +148,17 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     dst[0] = wk.wb;
     dst[1] = start;
     dst[2] = min(QPI, wk.l_hi - start);
-    dst[3] = (wk.wb != wk.cur);
-    wk.cur = wk.wb;
   };
-  auto issue_kv = [&](int bgj) {  // thread 0
+  // thread 0: one 128-key tile of K or V of block bgj into the K/V buffer
+  auto issue_tile = [&](const CUtensorMap *tm, uint32_t bar, int bgj) {
     const int j = bgj % a.nb;
     const int bg = bgj / a.nb;
     const int g = bg % a.G;
     const int b = bg / a.G;
-    mbar_arrive_expect_tx(b_kv, 65536);
+    mbar_arrive_expect_tx(bar, 32768);
     const int z = b * a.L + j * kBlock;
-    tma_load_3d(s_k, &tm_k, b_kv, 0, g, z);
-    tma_load_3d(s_k + 16384, &tm_k, b_kv, 64, g, z);
-    tma_load_3d(s_v, &tm_v, b_kv, 0, g, z);
-    tma_load_3d(s_v + 16384, &tm_v, b_kv, 64, g, z);
+    tma_load_3d(s_kv, tm, bar, 0, g, z);
+    tma_load_3d(s_kv + 16384, tm, bar, 64, g, z);
   };
 
   if (w_begin < w_end) {
@@ -176,7 +172,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
       wk.it_lo = a.item_off[lo]; wk.it_hi = a.item_off[lo + 1];
       wk.l_lo = a.list_off[lo]; wk.l_hi = a.list_off[lo + 1];
       describe(w_begin, s_item);
-      issue_kv(s_item[0]);
+      issue_tile(&tm_k, b_k, s_item[0]);
     }
     __syncthreads();
     if (tid < s_item[2]) s_list[tid] = a.list[s_item[1] + tid];
@@ -190,7 +186,6 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     const int *lst = s_list + 128 * buf;
     const int bgj = it[0];
     const int n = it[2];
-    const bool kv_new = it[3] != 0;
     const int j = bgj % a.nb;
     const int g = (bgj / a.nb) % a.G;
     const int b = bgj / (a.nb * a.G);
@@ -199,7 +194,10 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     int *nlst = s_list + 128 * (buf ^ 1);
     if (has_next && tid == 0) describe(w + 1, nit);
     __syncthreads();
-    if (has_next && tid < nit[2]) nlst[tid] = a.list[nit[1] + tid];
+    // the next item's query list: loaded now, stored to shared memory after
+    // this item's UMMAs, so its latency hides behind them
+    const int n_next = has_next ? nit[2] : 0;
+    const int next_entry = (tid < n_next) ? a.list[nit[1] + tid] : 0;
 
     // ---- this item's q rows have landed
     cp_async_wait_all();
@@ -207,122 +205,148 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
     __syncthreads();
 
     // ---- S = Q K^T
-    int ok_kv = 1;
+    int ok_k = 1;
     if (tid == 0) {
-      if (kv_new) ok_kv = mbar_wait(b_kv, kv_ph, abort_flag, a.status) ? 1 : 0;
-      if (ok_kv) {
+      ok_k = mbar_wait(b_k, k_ph, abort_flag, a.status) ? 1 : 0;
+      if (ok_k) {
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const int c = kk >> 2;
           const uint32_t off = (kk & 3) * 32;
-          umma_f16_ss(tmem_s, sdesc_sw128(s_q + c * 16384 + off, 16, 1024),
-                      sdesc_sw128(s_k + c * 16384 + off, 16, 1024), idesc_s, kk > 0);
+          umma_f16_ss(tmem_acc, sdesc_sw128(s_q + c * 16384 + off, 16, 1024),
+                      sdesc_sw128(s_kv + c * 16384 + off, 16, 1024), idesc_s, kk > 0);
         }
         umma_commit(b_mma);
       }
     }
-    if (kv_new) kv_ph ^= 1;
+    k_ph ^= 1;
     // every exit decision below is taken by the whole CTA at one barrier
-    if (__syncthreads_or(!ok_kv)) break;
+    if (__syncthreads_or(!ok_k)) break;
     const bool ok1 = mbar_wait(b_mma, mma_ph, abort_flag, a.status);
     mma_ph ^= 1;
     if (__syncthreads_or(!ok1)) break;
     tc_fence_after();
+    // K has been consumed: bring V into the same buffer during the softmax
+    if (tid == 0) issue_tile(&tm_v, b_v, bgj);
 
-    // ---- softmax on row `tid`
+    // ---- softmax on row `tid`, two 64-column halves per pass
     const int qi = tid / R;
     const bool valid = qi < n;
     const int ent = valid ? lst[qi] : 0;
     const int t = ent >> 5;
     const int lim = valid ? (t - j * kBlock) : -1;  // last visible column
-    float sv[128];
-#pragma unroll
-    for (int c4 = 0; c4 < 4; ++c4) {
-      float tmp[32];
-      tmem_ld32(tmem_s + lane_off + c4 * 32, tmp);
-#pragma unroll
-      for (int x = 0; x < 32; ++x) sv[c4 * 32 + x] = tmp[x];
-    }
-    tmem_wait_ld();
     float m = -FLT_MAX;
 #pragma unroll
-    for (int c = 0; c < 128; ++c)
-      if (c <= lim) m = fmaxf(m, sv[c]);
+    for (int h = 0; h < 2; ++h) {
+      float t0[32], t1[32];
+      tmem_ld32(tmem_acc + lane_off + h * 64, t0);
+      tmem_ld32(tmem_acc + lane_off + h * 64 + 32, t1);
+      tmem_wait_ld();
+#pragma unroll
+      for (int x = 0; x < 32; ++x) {
+        if (h * 64 + x <= lim) m = fmaxf(m, t0[x]);
+        if (h * 64 + 32 + x <= lim) m = fmaxf(m, t1[x]);
+      }
+    }
     const float mb = m * a.scale_log2;
     float l = 0.f;
-    uint8_t *p_row = smem + kSmemQ;
+    uint8_t *p_tile = smem + kSmemQ;
+#pragma unroll 1
+    for (int h = 0; h < 2; ++h) {
+      float sv[64];
+      {
+        float t0[32], t1[32];
+        tmem_ld32(tmem_acc + lane_off + h * 64, t0);
+        tmem_ld32(tmem_acc + lane_off + h * 64 + 32, t1);
+        tmem_wait_ld();
 #pragma unroll
-    for (int gblk = 0; gblk < 16; ++gblk) {
-      uint32_t w4[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int c0 = gblk * 8 + e * 2;
-        const float p0 = (c0 <= lim) ? fast_exp2(fmaf(sv[c0], a.scale_log2, -mb)) : 0.f;
-        const float p1 = (c0 + 1 <= lim) ? fast_exp2(fmaf(sv[c0 + 1], a.scale_log2, -mb)) : 0.f;
-        l += p0 + p1;
-        w4[e] = pack_bf16x2(p0, p1);
+        for (int x = 0; x < 32; ++x) { sv[x] = t0[x]; sv[32 + x] = t1[x]; }
       }
-      const uint32_t off = (gblk >> 3) * 16384 + sw128_offset(tid, gblk & 7);
-      *reinterpret_cast<uint4 *>(p_row + off) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+#pragma unroll
+      for (int gblk = 0; gblk < 8; ++gblk) {
+        uint32_t w4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c0 = gblk * 8 + e * 2;
+          const int cg = h * 64 + c0;
+          const float p0 = (cg <= lim) ? fast_exp2(fmaf(sv[c0], a.scale_log2, -mb)) : 0.f;
+          const float p1 = (cg + 1 <= lim) ? fast_exp2(fmaf(sv[c0 + 1], a.scale_log2, -mb)) : 0.f;
+          l += p0 + p1;
+          w4[e] = pack_bf16x2(p0, p1);
+        }
+        *reinterpret_cast<uint4 *>(p_tile + h * 16384 + sw128_offset(tid, gblk)) =
+            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
 
-    // ---- O = P V
+    // ---- O = P V (into the S columns: every thread has read S already)
+    int ok_v = 1;
     if (tid == 0) {
-      tc_fence_after();
+      ok_v = mbar_wait(b_v, v_ph, abort_flag, a.status) ? 1 : 0;
+      if (ok_v) {
+        tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const int c = kk >> 2;
-        const uint32_t off = (kk & 3) * 32;
-        umma_f16_ss(tmem_o, sdesc_sw128(s_q + c * 16384 + off, 16, 1024),
-                    sdesc_sw128(s_v + kk * 2048, 16384, 1024), idesc_o, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) {
+          const int c = kk >> 2;
+          const uint32_t off = (kk & 3) * 32;
+          umma_f16_ss(tmem_acc, sdesc_sw128(s_q + c * 16384 + off, 16, 1024),
+                      sdesc_sw128(s_kv + kk * 2048, 16384, 1024), idesc_o, kk > 0);
+        }
+        umma_commit(b_mma);
       }
-      umma_commit(b_mma);
     }
+    v_ph ^= 1;
+    if (__syncthreads_or(!ok_v)) break;
     const bool ok2 = mbar_wait(b_mma, mma_ph, abort_flag, a.status);
     mma_ph ^= 1;
     if (__syncthreads_or(!ok2)) break;
     tc_fence_after();
 
-    // ---- the shared tiles are free: request the next item's K/V and q rows
+    // ---- the shared tiles are free: request the next item's K and q rows
+    if (tid < n_next) nlst[tid] = next_entry;
+    __syncthreads();
     if (has_next) {
-      if (tid == 0 && nit[3]) issue_kv(nit[0]);
+      if (tid == 0) issue_tile(&tm_k, b_k, nit[0]);
       gather_q<R>(a, s_q, nlst, nit[2], nit[0] / (a.nb * a.G), (nit[0] / a.nb) % a.G, tid);
     }
 
-    // ---- store the normalised partial and its lse
+    // ---- store the normalised partial and its lse.  tcgen05.ld is a
+    // warp-wide (.sync.aligned) instruction: every thread loads, only rows
+    // holding a query store.
     {
-      float o[128];
+      const int slot = ent & 31;
+      const int hh = tid % R;
+      const bool store = valid && lim >= 0;
+      const float inv = store ? 1.f / l : 0.f;
+      const size_t prow =
+          ((size_t(b) * a.Lc + (t - a.t0)) * a.H + size_t(g) * R + hh) * a.top_k + slot;
+      uint4 *dst = reinterpret_cast<uint4 *>(a.part_o + prow * kHeadDim);
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float o0[32], o1[32];
+        tmem_ld32(tmem_acc + lane_off + h * 64, o0);
+        tmem_ld32(tmem_acc + lane_off + h * 64 + 32, o1);
+        tmem_wait_ld();
+        if (store) {
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        float tmp[32];
-        tmem_ld32(tmem_o + lane_off + c4 * 32, tmp);
+          for (int x = 0; x < 4; ++x)
+            dst[h * 8 + x] = make_uint4(pack_bf16x2(o0[8 * x] * inv, o0[8 * x + 1] * inv),
+                                        pack_bf16x2(o0[8 * x + 2] * inv, o0[8 * x + 3] * inv),
+                                        pack_bf16x2(o0[8 * x + 4] * inv, o0[8 * x + 5] * inv),
+                                        pack_bf16x2(o0[8 * x + 6] * inv, o0[8 * x + 7] * inv));
 #pragma unroll
-        for (int x = 0; x < 32; ++x) o[c4 * 32 + x] = tmp[x];
-      }
-      tmem_wait_ld();
-      if (valid) {
-        const int slot = ent & 31;
-        const int hh = tid % R;
-        const size_t prow =
-            ((size_t(b) * a.Lc + (t - a.t0)) * a.H + size_t(g) * R + hh) * a.top_k + slot;
-        if (lim >= 0) {
-          const float inv = 1.f / l;
-          uint4 *dst = reinterpret_cast<uint4 *>(a.part_o + prow * kHeadDim);
-#pragma unroll
-          for (int x = 0; x < 16; ++x)
-            dst[x] = make_uint4(pack_bf16x2(o[8 * x] * inv, o[8 * x + 1] * inv),
-                                pack_bf16x2(o[8 * x + 2] * inv, o[8 * x + 3] * inv),
-                                pack_bf16x2(o[8 * x + 4] * inv, o[8 * x + 5] * inv),
-                                pack_bf16x2(o[8 * x + 6] * inv, o[8 * x + 7] * inv));
-          a.part_lse[prow] = m * a.scale + __logf(l);
-        } else {
-          a.part_lse[prow] = -INFINITY;
+          for (int x = 0; x < 4; ++x)
+            dst[h * 8 + 4 + x] = make_uint4(pack_bf16x2(o1[8 * x] * inv, o1[8 * x + 1] * inv),
+                                            pack_bf16x2(o1[8 * x + 2] * inv, o1[8 * x + 3] * inv),
+                                            pack_bf16x2(o1[8 * x + 4] * inv, o1[8 * x + 5] * inv),
+                                            pack_bf16x2(o1[8 * x + 6] * inv, o1[8 * x + 7] * inv));
         }
       }
+      if (valid) a.part_lse[prow] = store ? m * a.scale + __logf(l) : -INFINITY;
     }
     tc_fence_before();
     __syncthreads();
@@ -334,7 +358,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2)
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem_s, 256);
+    tmem_dealloc(tmem_acc, 128);
   }
 }
 
@@ -344,7 +368,7 @@ cudaError_t launch_attn_r(const CUtensorMap &tk, const CUtensorMap &tv, const At
   auto kern = msa_prefill_attn_kernel<R>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
   if (e != cudaSuccess) return e;
-  int grid = 2 * num_sms;
+  int grid = kAttnCtasPerSm * num_sms;
   if (a.max_items < grid) grid = a.max_items > 0 ? a.max_items : 1;
   kern<<<grid, kAttnThreads, kAttnSmem, st>>>(tk, tv, a);
   return cudaGetLastError();
