@@ -14,7 +14,8 @@
 //                         segments of the block scores, one warp merges.
 //   decode_attn_kernel    split over selected blocks: one CTA per
 //                         (sequence, group, slot) computes the block's
-//                         partial softmax for the R heads of the group.
+//                         partial softmax for the R heads of the group on
+//                         the tensor cores (mma.sync, heads as M rows).
 //   decode_combine_kernel one warp per (sequence, head): merge <= top_k
 //                         partials.
 #include <cuda_runtime.h>
@@ -162,7 +163,11 @@ __global__ void __launch_bounds__(kTopkWarps * 32) decode_topk_kernel(const Deco
     for (int w = 0; w < kTopkWarps; ++w) {
       const int cj = cand_j[w][lane];
       const float cs = cand_s[w][lane];
-      warp_topk_offer(m, cs, cj, lane < k1 && cj != INT_MAX && cs >= t0, k1);
+      const bool ok = lane < k1 && cj != INT_MAX && cs >= t0;
+      if (w == 0)
+        warp_topk_seed(m, cs, cj, ok, k1);
+      else
+        warp_topk_offer(m, cs, cj, ok, k1);
     }
     warp_topk_write(m, bt, a.top_k, out);
   }
@@ -172,47 +177,40 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 
-// One CTA (128 threads) per (slot, group, sequence).  The block's K and V
-// rows (128 x 256 B each, strided by G*d*2 bytes in the cache) are staged in
-// shared memory with coalesced 16-byte cp.async, K and V as two groups so V
-// streams in while the scores are computed.  Phase 1: thread = key, R dot
-// products against the group's query heads.  Phase 2: thread = (d pair, key
-// parity), sum_k p[h][k] v[k][d].
-constexpr int kKPitch = kHeadDim + 8;  // bf16 elements per staged K row (272 B)
-
+// One CTA (4 warps) per (slot, group, sequence) computes the block's partial
+// softmax for the R <= 16 heads of the group on the tensor cores
+// (mma.sync m16n8k16, heads as the 16 M rows):
+//   S = q K^T: warp w owns keys 32w..32w+31 (four 8-key n-tiles).  K rows are
+//     the B operand, read straight from HBM as 16-byte granules with the same
+//     d permutation as the decode index scan (applied to q as well).
+//   softmax: row max / sum with shuffles over the lanes of a row and shared
+//     memory across the 4 warps; keys past the query are masked.
+//   O = P V: S's accumulator fragments are exactly P's A fragments (two
+//     8-key n-tiles form one 16-key k-step); V is staged in shared memory
+//     (rows padded to 272 B) and read with ldmatrix.trans.  The 4 warps'
+//     partial O are summed through shared memory.
+constexpr int kVPitch = kHeadDim + 8;  // bf16 per staged V row (272 B: conflict-free ldmatrix)
 template <int R>
-constexpr int decode_attn_smem() {
-  return kBlock * kKPitch * 2 + kBlock * kHeadDim * 2 + kHeadDim * R * 4 + kBlock * R * 4 +
-         R * kHeadDim * 4 + R * 4 * 4;
+constexpr int dec_attn_smem() {
+  return kBlock * kVPitch * 2 + 4 * R * kHeadDim * 4 + 2 * 4 * 16 * 4;
 }
 
-// q and p are kept head-minor ([d][R] and [key][R]) so one 16-byte shared
-// load feeds four heads.
-template <int R>
-__device__ __forceinline__ void load_heads(const float *base, float (&v)[R]) {
-  if constexpr (R % 4 == 0) {
-#pragma unroll
-    for (int h = 0; h < R; h += 4) {
-      const float4 f = *reinterpret_cast<const float4 *>(base + h);
-      v[h] = f.x; v[h + 1] = f.y; v[h + 2] = f.z; v[h + 3] = f.w;
-    }
-  } else {
-#pragma unroll
-    for (int h = 0; h < R; ++h) v[h] = base[h];
-  }
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
 }
 
 template <int R>
 __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
   extern __shared__ __align__(16) uint8_t dsm[];
-  uint16_t *sK = reinterpret_cast<uint16_t *>(dsm);
-  uint16_t *sV = sK + kBlock * kKPitch;
-  float *s_q = reinterpret_cast<float *>(sV + kBlock * kHeadDim);   // [d][R]
-  float *s_p = s_q + kHeadDim * R;                                   // [key][R]
-  float(*s_acc)[kHeadDim] = reinterpret_cast<float(*)[kHeadDim]>(s_p + kBlock * R);
-  float(*s_red)[4] = reinterpret_cast<float(*)[4]>(&s_acc[R][0]);
+  uint16_t *sV = reinterpret_cast<uint16_t *>(dsm);
+  float *s_o = reinterpret_cast<float *>(sV + kBlock * kVPitch);   // [4 warps][R rows][128]
+  float *s_m = s_o + 4 * R * kHeadDim;                              // [4][16]
+  float *s_l = s_m + 4 * 16;                                        // [4][16]
   const int slot = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g4 = lane >> 2, c = lane & 3;
   const int n = a.seq_lens[b];
   const int j = (n >= 1 && n <= a.Lmax) ? a.sel[(size_t(b) * a.G + g) * a.top_k + slot] : -1;
   const size_t prow0 = (size_t(b) * a.H + size_t(g) * R) * a.top_k + slot;
@@ -225,107 +223,147 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
   const size_t row_stride = size_t(a.G) * kHeadDim;
   const uint16_t *kb = a.k_cache + ((size_t(b) * a.Lmax + size_t(j) * kBlock) * a.G + g) * kHeadDim;
   const uint16_t *vb = a.v_cache + ((size_t(b) * a.Lmax + size_t(j) * kBlock) * a.G + g) * kHeadDim;
-  const uint32_t sK_u = static_cast<uint32_t>(__cvta_generic_to_shared(sK));
+  // V block -> shared memory (coalesced 16-byte cp.async), overlapping S
   const uint32_t sV_u = static_cast<uint32_t>(__cvta_generic_to_shared(sV));
 #pragma unroll 4
   for (int it = 0; it < 16; ++it) {
     const int idx = it * 128 + tid, row = idx >> 4, gran = idx & 15;
-    if (row < nvis) cp_async16(sK_u + (row * kKPitch + gran * 8) * 2, kb + row * row_stride + gran * 8);
+    const uint32_t dst = sV_u + (row * kVPitch + gran * 8) * 2;
+    if (row < nvis)
+      cp_async16(dst, vb + row * row_stride + gran * 8);
+    else  // rows past the query get p = 0; keep them finite (0 * NaN would poison O)
+      asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(dst), "r"(0) : "memory");
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
-#pragma unroll 4
-  for (int it = 0; it < 16; ++it) {
-    const int idx = it * 128 + tid, row = idx >> 4, gran = idx & 15;
-    if (row < nvis) cp_async16(sV_u + (row * kHeadDim + gran * 8) * 2, vb + row * row_stride + gran * 8);
+  // K granules for this warp's four 8-key n-tiles (key row 8*nt + g4)
+  uint4 kg[4][4];
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const int key = warp * 32 + q4 * 8 + g4;
+    const uint16_t *kr = kb + size_t(min(key, nvis - 1)) * row_stride;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) kg[q4][m] = ldg_nc_v4(kr + 8 * (c + 4 * m));
   }
-  asm volatile("cp.async.commit_group;" ::: "memory");
-  for (int x = tid; x < R * kHeadDim; x += 128) {
-    const int h = x / kHeadDim, dd = x % kHeadDim;
-    s_q[dd * R + h] = __bfloat162float(__ushort_as_bfloat16(a.q[(size_t(b) * a.H + g * R + h) * kHeadDim + dd]));
-  }
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
-  __syncthreads();
-  // phase 1: scores (thread = key)
-  const bool vis = tid < nvis;
-  float sc[R];
+  // q A fragments (rows g4 and g4+8; zero beyond R), same d permutation
+  uint32_t qa[4][2][2], qb[4][2][2];
+  {
+    const uint16_t *q0 = a.q + (size_t(b) * a.H + size_t(g) * R + g4) * kHeadDim;
+    const uint16_t *q1 = q0 + 8 * kHeadDim;
 #pragma unroll
-  for (int h = 0; h < R; ++h) sc[h] = 0.f;
-  if (vis) {
-    const uint16_t *krow = sK + tid * kKPitch;
-#pragma unroll 2
-    for (int x = 0; x < 16; ++x) {
-      const uint4 kv = *reinterpret_cast<const uint4 *>(krow + 8 * x);
-      const float kf[8] = {bf16_lo(kv.x), bf16_hi(kv.x), bf16_lo(kv.y), bf16_hi(kv.y),
-                           bf16_lo(kv.z), bf16_hi(kv.z), bf16_lo(kv.w), bf16_hi(kv.w)};
+    for (int m = 0; m < 4; ++m)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float qv[R];
-        load_heads<R>(s_q + (8 * x + e) * R, qv);
-#pragma unroll
-        for (int h = 0; h < R; ++h) sc[h] = fmaf(qv[h], kf[e], sc[h]);
+      for (int h = 0; h < 2; ++h) {
+        uint2 v0 = make_uint2(0u, 0u), v1 = make_uint2(0u, 0u);
+        if (g4 < R) v0 = *reinterpret_cast<const uint2 *>(q0 + 8 * (c + 4 * m) + 4 * h);
+        if (g4 + 8 < R) v1 = *reinterpret_cast<const uint2 *>(q1 + 8 * (c + 4 * m) + 4 * h);
+        qa[m][h][0] = v0.x; qa[m][h][1] = v0.y;
+        qb[m][h][0] = v1.x; qb[m][h][1] = v1.y;
       }
+  }
+  // S tiles: acc[q4] = rows (g4, g4+8) x keys (8*nt + 2c, +1)
+  float sacc[4][4];
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sacc[q4][e] = 0.f;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      mma_bf16_16816(sacc[q4], qa[m][0][0], qb[m][0][0], qa[m][0][1], qb[m][0][1], kg[q4][m].x,
+                     kg[q4][m].y);
+      mma_bf16_16816(sacc[q4], qa[m][1][0], qb[m][1][0], qa[m][1][1], qb[m][1][1], kg[q4][m].z,
+                     kg[q4][m].w);
     }
   }
-  const int lane = tid & 31, warp = tid >> 5;
+  // mask keys past the query, row max over the block
+  float mx0 = -FLT_MAX, mx1 = -FLT_MAX;
 #pragma unroll
-  for (int h = 0; h < R; ++h) {
-    float m = vis ? sc[h] : -FLT_MAX;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) s_red[h][warp] = m;
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const int k0 = warp * 32 + q4 * 8 + 2 * c;
+    if (k0 >= nvis) { sacc[q4][0] = -FLT_MAX; sacc[q4][2] = -FLT_MAX; }
+    if (k0 + 1 >= nvis) { sacc[q4][1] = -FLT_MAX; sacc[q4][3] = -FLT_MAX; }
+    mx0 = fmaxf(mx0, fmaxf(sacc[q4][0], sacc[q4][1]));
+    mx1 = fmaxf(mx1, fmaxf(sacc[q4][2], sacc[q4][3]));
   }
-  __syncthreads();
-  float mrow[R], lrow[R];
 #pragma unroll
-  for (int h = 0; h < R; ++h)
-    mrow[h] = fmaxf(fmaxf(s_red[h][0], s_red[h][1]), fmaxf(s_red[h][2], s_red[h][3]));
-  __syncthreads();
-#pragma unroll
-  for (int h = 0; h < R; ++h) {
-    const float p = vis ? exp2f((sc[h] - mrow[h]) * a.scale_log2) : 0.f;
-    s_p[tid * R + h] = p;
-    float l = p;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) s_red[h][warp] = l;
+  for (int o = 1; o < 4; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
   }
+  if (c == 0) { s_m[warp * 16 + g4] = mx0; s_m[warp * 16 + g4 + 8] = mx1; }
+  __syncthreads();
+  const float m0 = fmaxf(fmaxf(s_m[g4], s_m[16 + g4]), fmaxf(s_m[32 + g4], s_m[48 + g4]));
+  const float m1 = fmaxf(fmaxf(s_m[8 + g4], s_m[24 + g4]), fmaxf(s_m[40 + g4], s_m[56 + g4]));
+  // P = exp(scale (S - m)), packed straight into A fragments
+  uint32_t pa[2][4];
+  float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const float p0 = exp2f((sacc[q4][0] - m0) * a.scale_log2);
+    const float p1 = exp2f((sacc[q4][1] - m0) * a.scale_log2);
+    const float p2 = exp2f((sacc[q4][2] - m1) * a.scale_log2);
+    const float p3 = exp2f((sacc[q4][3] - m1) * a.scale_log2);
+    l0 += p0 + p1;
+    l1 += p2 + p3;
+    const int kt = q4 >> 1, hi = q4 & 1;   // n-tiles (2kt, 2kt+1) -> k-step kt
+    pa[kt][hi ? 2 : 0] = pack_bf16x2(p0, p1);   // row g4
+    pa[kt][hi ? 3 : 1] = pack_bf16x2(p2, p3);   // row g4 + 8
+  }
+#pragma unroll
+  for (int o = 1; o < 4; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  if (c == 0) { s_l[warp * 16 + g4] = l0; s_l[warp * 16 + g4 + 8] = l1; }
+  // O = P V over this warp's 32 keys (two 16-key k-steps) x 16 d-tiles
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
+  float oacc[16][4];
 #pragma unroll
-  for (int h = 0; h < R; ++h) lrow[h] = s_red[h][0] + s_red[h][1] + s_red[h][2] + s_red[h][3];
-  // phase 2: O = P V over the visible keys
-  const int dp = tid & 63, par = tid >> 6;
-  float acc[R][2];
+  for (int dt = 0; dt < 16; ++dt)
 #pragma unroll
-  for (int h = 0; h < R; ++h) acc[h][0] = acc[h][1] = 0.f;
-#pragma unroll 4
-  for (int k = par; k < nvis; k += 2) {
-    const uint32_t w = *reinterpret_cast<const uint32_t *>(sV + k * kHeadDim + 2 * dp);
-    const float v0 = bf16_lo(w), v1 = bf16_hi(w);
-    float pv[R];
-    load_heads<R>(s_p + k * R, pv);
+    for (int e = 0; e < 4; ++e) oacc[dt][e] = 0.f;
 #pragma unroll
-    for (int h = 0; h < R; ++h) {
-      acc[h][0] = fmaf(pv[h], v0, acc[h][0]);
-      acc[h][1] = fmaf(pv[h], v1, acc[h][1]);
+  for (int kt = 0; kt < 2; ++kt) {
+    const int key0 = warp * 32 + kt * 16;
+#pragma unroll
+    for (int dt = 0; dt < 16; dt += 2) {
+      // matrices: (keys 0-7, dt), (keys 8-15, dt), (keys 0-7, dt+1), (keys 8-15, dt+1)
+      const int mi = lane >> 3, r = lane & 7;
+      const int key = key0 + (mi & 1) * 8 + r;
+      const int d0 = (dt + (mi >> 1)) * 8;
+      uint32_t bv[4];
+      ldmatrix_x4_trans(bv, sV_u + (key * kVPitch + d0) * 2);
+      mma_bf16_16816(oacc[dt], pa[kt][0], pa[kt][1], pa[kt][2], pa[kt][3], bv[0], bv[1]);
+      mma_bf16_16816(oacc[dt + 1], pa[kt][0], pa[kt][1], pa[kt][2], pa[kt][3], bv[2], bv[3]);
     }
   }
-  if (par == 1) {
+  // sum the 4 warps' partial O (rows < R only) and normalise
 #pragma unroll
-    for (int h = 0; h < R; ++h) { s_acc[h][2 * dp] = acc[h][0]; s_acc[h][2 * dp + 1] = acc[h][1]; }
+  for (int dt = 0; dt < 16; ++dt) {
+    const int d = dt * 8 + 2 * c;
+    if (g4 < R) {
+      s_o[(warp * R + g4) * kHeadDim + d] = oacc[dt][0];
+      s_o[(warp * R + g4) * kHeadDim + d + 1] = oacc[dt][1];
+    }
+    if (g4 + 8 < R) {
+      s_o[(warp * R + g4 + 8) * kHeadDim + d] = oacc[dt][2];
+      s_o[(warp * R + g4 + 8) * kHeadDim + d + 1] = oacc[dt][3];
+    }
   }
   __syncthreads();
-  if (par == 0) {
-#pragma unroll
-    for (int h = 0; h < R; ++h) {
-      const float inv = 1.f / lrow[h];
-      float2 o2 = make_float2((acc[h][0] + s_acc[h][2 * dp]) * inv, (acc[h][1] + s_acc[h][2 * dp + 1]) * inv);
-      *reinterpret_cast<float2 *>(a.part_o + (prow0 + size_t(h) * a.top_k) * kHeadDim + 2 * dp) = o2;
-    }
+  for (int x = tid; x < R * kHeadDim; x += 128) {
+    const int h = x / kHeadDim, d = x % kHeadDim;
+    const float l = s_l[h] + s_l[16 + h] + s_l[32 + h] + s_l[48 + h];
+    const float o = s_o[h * kHeadDim + d] + s_o[(R + h) * kHeadDim + d] +
+                    s_o[(2 * R + h) * kHeadDim + d] + s_o[(3 * R + h) * kHeadDim + d];
+    a.part_o[(prow0 + size_t(h) * a.top_k) * kHeadDim + d] = o / l;
   }
-#pragma unroll
-  for (int h = 0; h < R; ++h)
-    if (tid == h) a.part_lse[prow0 + size_t(h) * a.top_k] = mrow[h] * a.scale + __logf(lrow[h]);
+  if (tid < R) {
+    const int h = tid;
+    const float mh = fmaxf(fmaxf(s_m[h], s_m[16 + h]), fmaxf(s_m[32 + h], s_m[48 + h]));
+    const float l = s_l[h] + s_l[16 + h] + s_l[32 + h] + s_l[48 + h];
+    a.part_lse[prow0 + size_t(h) * a.top_k] = mh * a.scale + __logf(l);
+  }
 }
 
 __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a) {
@@ -363,7 +401,7 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a)
 
 template <int R>
 cudaError_t launch_decode_attn(const DecodeArgs &a, cudaStream_t st) {
-  constexpr int smem = decode_attn_smem<R>();
+  constexpr int smem = dec_attn_smem<R>();
   cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<R>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;

@@ -35,6 +35,37 @@ __device__ __forceinline__ void warp_topk_init(WarpTopk &st) {
   st.thr = -FLT_MAX;
 }
 
+// (score desc, id asc) order: true if (sa, ja) ranks ahead of (sb, jb).
+__device__ __forceinline__ bool ranks_ahead(float sa, int ja, float sb, int jb) {
+  return sa > sb || (sa == sb && ja < jb);
+}
+
+// First offer into an empty list: sort the 32 candidates with a bitonic
+// network in (score desc, id asc) order and keep the first k1, instead of
+// inserting them one at a time.
+__device__ __forceinline__ void warp_topk_seed(WarpTopk &st, float s, int j, bool valid, int k1) {
+  const int lane = threadIdx.x & 31;
+  float ks = valid ? s : -FLT_MAX;
+  int kj = valid ? j : INT_MAX;
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int d = k >> 1; d > 0; d >>= 1) {
+      const float os = __shfl_xor_sync(0xffffffffu, ks, d);
+      const int oj = __shfl_xor_sync(0xffffffffu, kj, d);
+      const bool first = (lane & k) == 0;   // this k-block is ordered best-first
+      const bool lower = (lane & d) == 0;
+      const bool mine_ahead = ranks_ahead(ks, kj, os, oj);
+      const bool keep = (lower == first) ? mine_ahead : !mine_ahead;
+      ks = keep ? ks : os;
+      kj = keep ? kj : oj;
+    }
+  }
+  st.ls = (lane < k1) ? ks : -FLT_MAX;
+  st.lj = (lane < k1) ? kj : INT_MAX;
+  st.thr = __shfl_sync(0xffffffffu, st.ls, k1 - 1);
+}
+
 // Offer one candidate per lane (s, j, valid); lanes' candidates must be in
 // increasing id order across lanes and after every earlier offer.
 __device__ __forceinline__ void warp_topk_offer(WarpTopk &st, float s, int j, bool valid, int k1) {
@@ -71,7 +102,11 @@ __device__ __forceinline__ void warp_topk_scan(WarpTopk &st, const float *__rest
     for (int u = 0; u < 4; ++u) {
       const int jb = base + u * 32;
       if (jb >= hi) break;
-      warp_topk_offer(st, s4[u], jb + lane, jb + lane < hi, k1);
+      const bool empty = __all_sync(0xffffffffu, st.lj == INT_MAX);  // warp-uniform
+      if (empty)
+        warp_topk_seed(st, s4[u], jb + lane, jb + lane < hi, k1);
+      else
+        warp_topk_offer(st, s4[u], jb + lane, jb + lane < hi, k1);
     }
   }
 }
