@@ -40,6 +40,24 @@ import torch  # noqa: E402
 METRIC = "MSA prefill tokens/s & decode µs/step at 128K/1M; % of B200 roofline"
 BLOCK = 128
 
+# DRAM bytes (read + write) of one msa_index_kernel launch on the 1M-token
+# workload, from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum,
+# a single-pass metric set; see profiles/msa_index_kernel_1m_traffic.md).
+# Keyed to the kernel source it was measured on: a changed kernel reports null.
+INDEX_TRAFFIC_1M = {"bytes": 1.5423e11, "source_sha256_16": "bdf4320d41b4b801"}
+
+
+def index_traffic(workload: str):
+    import hashlib
+    src = os.path.join(ROOT, "block_sparse_long_08_b200", "csrc", "index_kernel.cu")
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if workload != "1m" or h != INDEX_TRAFFIC_1M["source_sha256_16"]:
+        return None
+    return INDEX_TRAFFIC_1M["bytes"]
+
 
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -386,7 +404,7 @@ def run_ours(args, shape, dshape, seed, cfg, ws_n, rank, local):
     dbytes = decode_bytes(seq_lens_host, dshape.H, dshape.G, dshape.d, dshape.d_idx, dshape.top_k)
     peak_t = peaks["bf16_tflops_sustained"]
     roof_idx = {"bound": "tensor", "achieved": f_idx / (idx_ms / 1e3) / 1e12, "peak": peak_t,
-                "unit": "TFLOP/s", "frac": None, "traffic": None,
+                "unit": "TFLOP/s", "frac": None, "traffic": index_traffic(args.workload),
                 "kernel": "msa_index_kernel", "peak_kind": f"bf16 sustained ({peaks['source']})"}
     roof_idx["frac"] = roof_idx["achieved"] / peak_t
     roof_att = {"bound": "tensor", "achieved": f_main / (att_ms / 1e3) / 1e12, "peak": peak_t,
