@@ -394,6 +394,10 @@ namespace {
 
 // One warp per (b, t, h): merge the row's partials (normalised o_s, lse_s)
 // into o = sum_s exp(lse_s - M) o_s / sum_s exp(lse_s - M), M = max lse_s.
+// All of a lane's partial-row loads (4 of the d values of each slot) and its
+// lse load are issued before any reduction, so a row costs one memory round
+// trip after its selection row is known.
+template <int KCAP>
 __global__ void __launch_bounds__(256) msa_combine_kernel(const CombineArgs a) {
   const long long wrow = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -408,7 +412,15 @@ __global__ void __launch_bounds__(256) msa_combine_kernel(const CombineArgs a) {
   const int32_t *sel = a.sel + ((size_t(b) * a.G + g) * a.L + t) * a.top_k;
   const size_t prow0 = (((size_t)b * a.Lc + tl) * a.H + h) * a.top_k;
   const bool mine = lane < a.top_k && sel[lane] >= 0;
-  const float my_lse = mine ? a.part_lse[prow0 + lane] : -INFINITY;
+  const unsigned vmask = __ballot_sync(0xffffffffu, mine);
+  uint2 v[KCAP];
+#pragma unroll
+  for (int s = 0; s < KCAP; ++s) {
+    v[s] = make_uint2(0u, 0u);
+    if ((vmask >> s) & 1u)
+      v[s] = __ldcs(reinterpret_cast<const uint2 *>(a.part_o + (prow0 + s) * kHeadDim + lane * 4));
+  }
+  const float my_lse = mine ? __ldcs(a.part_lse + prow0 + lane) : -INFINITY;
   float M = my_lse;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
@@ -419,28 +431,13 @@ __global__ void __launch_bounds__(256) msa_combine_kernel(const CombineArgs a) {
     wsum = wmine;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-    const unsigned vmask = __ballot_sync(0xffffffffu, mine);
-    // up to 8 partial rows in flight per lane before they are consumed
-    for (int s0 = 0; s0 < a.top_k; s0 += 8) {
-      uint2 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int s = s0 + u;
-        v[u] = make_uint2(0u, 0u);
-        if (s < a.top_k && ((vmask >> s) & 1u))
-          v[u] = __ldcs(reinterpret_cast<const uint2 *>(a.part_o + (prow0 + s) * kHeadDim + lane * 4));
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int s = s0 + u;
-        const float ws = __shfl_sync(0xffffffffu, wmine, s & 31);
-        if (s < a.top_k && ((vmask >> s) & 1u)) {
-          acc[0] = fmaf(ws, bf16_lo(v[u].x), acc[0]);
-          acc[1] = fmaf(ws, bf16_hi(v[u].x), acc[1]);
-          acc[2] = fmaf(ws, bf16_lo(v[u].y), acc[2]);
-          acc[3] = fmaf(ws, bf16_hi(v[u].y), acc[3]);
-        }
-      }
+    for (int s = 0; s < KCAP; ++s) {
+      const float ws = __shfl_sync(0xffffffffu, wmine, s);
+      acc[0] = fmaf(ws, bf16_lo(v[s].x), acc[0]);
+      acc[1] = fmaf(ws, bf16_hi(v[s].x), acc[1]);
+      acc[2] = fmaf(ws, bf16_lo(v[s].y), acc[2]);
+      acc[3] = fmaf(ws, bf16_hi(v[s].y), acc[3]);
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
@@ -456,7 +453,15 @@ __global__ void __launch_bounds__(256) msa_combine_kernel(const CombineArgs a) {
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st) {
   const long long n_rows = (long long)a.B * a.Lc * a.H;
   if (n_rows == 0) return cudaSuccess;
-  msa_combine_kernel<<<(unsigned)((n_rows + 7) / 8), 256, 0, st>>>(a);
+  const unsigned grid = (unsigned)((n_rows + 7) / 8);
+  if (a.top_k <= 4)
+    msa_combine_kernel<4><<<grid, 256, 0, st>>>(a);
+  else if (a.top_k <= 8)
+    msa_combine_kernel<8><<<grid, 256, 0, st>>>(a);
+  else if (a.top_k <= 16)
+    msa_combine_kernel<16><<<grid, 256, 0, st>>>(a);
+  else
+    msa_combine_kernel<32><<<grid, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -42,54 +42,75 @@ __global__ void __launch_bounds__(256) revidx_count_kernel(const RevIdxArgs a) {
   }
 }
 
-// Single CTA, 1024 threads: exclusive scans of cnt and ceil(cnt/qpi).
-__global__ void __launch_bounds__(1024) revidx_scan_kernel(const RevIdxArgs a) {
-  __shared__ int warp_a[32], warp_b[32];
-  const int n = a.B * a.G * a.nb;
-  const int per = (n + blockDim.x - 1) / blockDim.x;
-  const int lo = threadIdx.x * per;
-  const int hi = min(n, lo + per);
-  int sa = 0, sb = 0;
-  for (int x = lo; x < hi; ++x) {
-    const int c = a.cnt[x];
-    sa += c;
-    sb += (c + a.qpi - 1) / a.qpi;
-  }
+// Block-wide inclusive scan of (x, y) pairs over 1024 threads; returns the
+// pair totals through *tot (shared).
+__device__ __forceinline__ void block_scan2(int &x, int &y, int *warp_x, int *warp_y, int *tot) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int ia = sa, ib = sb;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int ya = __shfl_up_sync(0xffffffffu, ia, o);
-    const int yb = __shfl_up_sync(0xffffffffu, ib, o);
-    if (lane >= o) { ia += ya; ib += yb; }
+    const int yx = __shfl_up_sync(0xffffffffu, x, o);
+    const int yy = __shfl_up_sync(0xffffffffu, y, o);
+    if (lane >= o) { x += yx; y += yy; }
   }
-  if (lane == 31) { warp_a[warp] = ia; warp_b[warp] = ib; }
+  if (lane == 31) { warp_x[warp] = x; warp_y[warp] = y; }
   __syncthreads();
   if (warp == 0) {
-    int va = warp_a[lane], vb = warp_b[lane];
+    int vx = warp_x[lane], vy = warp_y[lane];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int ya = __shfl_up_sync(0xffffffffu, va, o);
-      const int yb = __shfl_up_sync(0xffffffffu, vb, o);
-      if (lane >= o) { va += ya; vb += yb; }
+      const int yx = __shfl_up_sync(0xffffffffu, vx, o);
+      const int yy = __shfl_up_sync(0xffffffffu, vy, o);
+      if (lane >= o) { vx += yx; vy += yy; }
     }
-    warp_a[lane] = va;
-    warp_b[lane] = vb;
+    warp_x[lane] = vx;
+    warp_y[lane] = vy;
+    if (lane == 31) { tot[0] = vx; tot[1] = vy; }
   }
   __syncthreads();
-  int ea = ia - sa + (warp > 0 ? warp_a[warp - 1] : 0);
-  int eb = ib - sb + (warp > 0 ? warp_b[warp - 1] : 0);
-  for (int x = lo; x < hi; ++x) {
-    const int c = a.cnt[x];
-    a.list_off[x] = ea;
-    a.item_off[x] = eb;
-    a.cursor[x] = 0;
-    ea += c;
-    eb += (c + a.qpi - 1) / a.qpi;
+  if (warp > 0) { x += warp_x[warp - 1]; y += warp_y[warp - 1]; }
+}
+
+// Single CTA, 1024 threads: exclusive scans of cnt and ceil(cnt/qpi), in
+// tiles of 4096 entries (4 consecutive entries per thread, 16-byte loads).
+__global__ void __launch_bounds__(1024) revidx_scan_kernel(const RevIdxArgs a) {
+  __shared__ int warp_x[32], warp_y[32], tot[2];
+  const int n = a.B * a.G * a.nb;
+  int carry_x = 0, carry_y = 0;
+  for (int base = 0; base < n; base += 4096) {
+    const int i0 = base + 4 * threadIdx.x;
+    int c[4];
+    if (i0 + 3 < n) {
+      const int4 v = *reinterpret_cast<const int4 *>(a.cnt + i0);
+      c[0] = v.x; c[1] = v.y; c[2] = v.z; c[3] = v.w;
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) c[u] = (i0 + u < n) ? a.cnt[i0 + u] : 0;
+    }
+    int ch[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) ch[u] = (c[u] + a.qpi - 1) / a.qpi;
+    const int sx = c[0] + c[1] + c[2] + c[3];
+    const int sy = ch[0] + ch[1] + ch[2] + ch[3];
+    int x = sx, y = sy;
+    block_scan2(x, y, warp_x, warp_y, tot);
+    int ex = carry_x + x - sx, ey = carry_y + y - sy;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (i0 + u < n) {
+        a.list_off[i0 + u] = ex;
+        a.item_off[i0 + u] = ey;
+        a.cursor[i0 + u] = 0;
+      }
+      ex += c[u];
+      ey += ch[u];
+    }
+    carry_x += tot[0];
+    carry_y += tot[1];
+    __syncthreads();   // tot / warp sums are rewritten by the next tile
   }
-  if (threadIdx.x == blockDim.x - 1) {
-    a.list_off[n] = warp_a[31];
-    a.item_off[n] = warp_b[31];
+  if (threadIdx.x == 0) {
+    a.list_off[n] = carry_x;
+    a.item_off[n] = carry_y;
   }
 }
 
