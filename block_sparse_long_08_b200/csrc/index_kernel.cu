@@ -104,10 +104,10 @@ __device__ __forceinline__ int index_item(int r, int n_items) {
 
 template <int KCAP>
 __device__ __forceinline__ void list_insert(float (&ls)[KCAP], int (&lj)[KCAP], float s, int j) {
-  // Insert (s, j) into the list kept in (score desc, id asc) order.  The
-  // carried entry is compared lexicographically, so an entry pushed down by
-  // the insertion keeps its place ahead of an equal-score entry with a
-  // higher id.
+  // Insert (s, j) into the list kept in (score desc, id asc) order, for ids
+  // in any order (the merge of the two sets' lists).  The carried entry is
+  // compared lexicographically, so an entry pushed down by the insertion
+  // keeps its place ahead of an equal-score entry with a higher id.
   float cs = s;
   int cj = j;
 #pragma unroll
@@ -123,12 +123,22 @@ __device__ __forceinline__ void list_insert(float (&ls)[KCAP], int (&lj)[KCAP], 
 }
 
 template <int KCAP>
-__device__ __forceinline__ float list_threshold(const float (&ls)[KCAP], int k1) {
-  float thr = -FLT_MAX;
+__device__ __forceinline__ void list_insert_tail(float (&ls)[KCAP], int (&lj)[KCAP], float s, int j) {
+  // Insert (s, j) when j is above every kept id (the blocks of one epilogue
+  // set arrive in increasing id order): a kept entry ranks ahead of the new
+  // one exactly when its score is >= s, so the insertion point is the number
+  // of such entries and every slot is updated independently -- no carried
+  // compare chain.  Walking k downwards reads ls[k-1] before it is replaced.
+  bool ge[KCAP];
 #pragma unroll
-  for (int k = 0; k < KCAP; ++k)
-    if (k == k1 - 1) thr = ls[k];
-  return thr;
+  for (int k = 0; k < KCAP; ++k) ge[k] = ls[k] >= s;
+#pragma unroll
+  for (int k = KCAP - 1; k >= 1; --k) {
+    ls[k] = ge[k] ? ls[k] : (ge[k - 1] ? s : ls[k - 1]);
+    lj[k] = ge[k] ? lj[k] : (ge[k - 1] ? j : lj[k - 1]);
+  }
+  ls[0] = ge[0] ? ls[0] : s;
+  lj[0] = ge[0] ? lj[0] : j;
 }
 
 template <int KCAP>
@@ -311,6 +321,10 @@ __global__ void __launch_bounds__(384, 1)
     const int row = quad * 32 + lane;
     const uint32_t lane_base = tmem_base + (uint32_t(quad * 32) << 16);
     const int k1 = a.top_k - 1;
+    // Slots [0, KCAP-k1) hold sentinels (+inf, id -1) that rank ahead of
+    // every block and never move; the kept entries occupy the last k1 slots,
+    // so the worst kept score is always ls[KCAP-1].
+    const int n_sent = KCAP - k1;
     float *m_score = reinterpret_cast<float *>(smem + C::MERGE_OFF);
     int *m_id = reinterpret_cast<int *>(smem + C::MERGE_OFF + C::MERGE_BYTES / 2);
     uint32_t jc = 0;
@@ -322,12 +336,13 @@ __global__ void __launch_bounds__(384, 1)
       const int t = w.i * kBlock + row;
       float ls[GP][KCAP];
       int lj[GP][KCAP];
-      float thr[GP];
 #pragma unroll
       for (int gi = 0; gi < GP; ++gi) {
 #pragma unroll
-        for (int k = 0; k < KCAP; ++k) { ls[gi][k] = -FLT_MAX; lj[gi][k] = INT_MAX; }
-        thr[gi] = -FLT_MAX;
+        for (int k = 0; k < KCAP; ++k) {
+          ls[gi][k] = k < n_sent ? INFINITY : -FLT_MAX;
+          lj[gi][k] = k < n_sent ? -1 : INT_MAX;
+        }
       }
       for (int s = 0; s < w.stages && ok; ++s) {
 #pragma unroll
@@ -358,9 +373,8 @@ __global__ void __launch_bounds__(384, 1)
             if (a.write_scores) {
               const int g = w.gp * GP + gi;
               a.scores[((size_t(w.b) * a.G + g) * a.L + t) * a.nb + j] = sc;
-            } else if (sc > thr[gi]) {
-              list_insert<KCAP>(ls[gi], lj[gi], sc, j);
-              thr[gi] = list_threshold<KCAP>(ls[gi], k1);
+            } else if (sc > ls[gi][KCAP - 1]) {
+              list_insert_tail<KCAP>(ls[gi], lj[gi], sc, j);
             }
           }
         }
@@ -411,13 +425,13 @@ __global__ void __launch_bounds__(384, 1)
           for (int k = 0; k < KCAP; ++k) {
             const float sc = m_score[(gi * KCAP + k) * 128 + row];
             const int id = m_id[(gi * KCAP + k) * 128 + row];
-            if (id != INT_MAX) list_insert<KCAP>(ls[gi], lj[gi], sc, id);
+            if (id >= 0 && id != INT_MAX) list_insert<KCAP>(ls[gi], lj[gi], sc, id);
           }
           const int g = w.gp * GP + gi;
           int32_t *dst = a.sel + ((size_t(w.b) * a.G + g) * a.L + t) * a.top_k;
           int ids[KCAP];
 #pragma unroll
-          for (int k = 0; k < KCAP; ++k) ids[k] = (k < k1) ? lj[gi][k] : INT_MAX;
+          for (int k = 0; k < KCAP; ++k) ids[k] = (k >= n_sent) ? lj[gi][k] : INT_MAX;
           sort_ids_asc<KCAP>(ids);
           if ((a.top_k & 3) == 0) {
 #pragma unroll
