@@ -42,9 +42,9 @@ BLOCK = 128
 
 # DRAM bytes (read + write) of one msa_index_kernel launch on the 1M-token
 # workload, from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum,
-# a single-pass metric set; see profiles/msa_index_kernel_1m_traffic.md).
+# a single-pass metric set; see profiles/dram_traffic_msa_1m_and_decode_128k.md).
 # Keyed to the kernel source it was measured on: a changed kernel reports null.
-INDEX_TRAFFIC_1M = {"bytes": 1.5423e11, "source_sha256_16": "bdf4320d41b4b801"}
+INDEX_TRAFFIC_1M = {"bytes": 1.2994e11, "source_sha256_16": "4d8a0c74c7c30bff"}
 
 
 def index_traffic(workload: str):
