@@ -36,6 +36,7 @@ struct RevIdxArgs {
   int32_t *list_off;            // [B*G*nb + 1]
   int32_t *item_off;            // [B*G*nb + 1]
   int32_t *list;                // [B*G*Lc*top_k]
+  int32_t *pos_of;              // [B,G,Lc,top_k]: list position of each selected entry
   int *status;
 };
 cudaError_t launch_revidx(const RevIdxArgs &a, cudaStream_t st);
@@ -49,8 +50,11 @@ struct AttnArgs {
   const int32_t *list;
   const int32_t *list_off;
   const int32_t *item_off;
-  uint16_t *part_o;            // [B,Lc,H,top_k,d] bf16
-  float *part_lse;             // [B,Lc,H,top_k]
+  // Partials by reverse-index list position: entry pos owns rows pos*R + hh
+  // (hh < R = H/G); a row's 16-byte granule c is stored at granule
+  // c ^ (row & 7).
+  uint16_t *part_o;            // [entries*R, d] bf16
+  float *part_lse;             // [entries*R]
   int *status;
 };
 cudaError_t launch_prefill_attn(const CUtensorMap &tk, const CUtensorMap &tv, const AttnArgs &a,
@@ -60,8 +64,9 @@ struct CombineArgs {
   int B, L, H, G, top_k;
   int t0, Lc;
   const int32_t *sel;          // [B,G,L,top_k]
-  const uint16_t *part_o;      // [B,Lc,H,top_k,d]
-  const float *part_lse;       // [B,Lc,H,top_k]
+  const int32_t *pos_of;       // [B,G,Lc,top_k]
+  const uint16_t *part_o;      // see AttnArgs
+  const float *part_lse;
   uint16_t *out;               // [B,L,H,d]
   float *lse;                  // [B,L,H] or null
 };

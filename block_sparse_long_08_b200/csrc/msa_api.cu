@@ -66,7 +66,8 @@ float eff_scale(const msa_params *p) {
 
 // ---- workspace plans --------------------------------------------------------
 // Prefill attention processes queries in chunks of Lc so that the partial
-// results (bf16 [B,Lc,H,top_k,d]) stay within a fixed budget.
+// results (bf16, one 128-wide row per selected (query, head, slot)) stay
+// within a fixed budget.
 constexpr size_t kPartialBudget = size_t(4608) << 20;  // 4.5 GiB
 
 int prefill_chunk(const msa_params *p) {
@@ -79,7 +80,7 @@ int prefill_chunk(const msa_params *p) {
 }
 
 struct AttnWs {
-  size_t cnt, cursor, list_off, item_off, list, part_o, part_lse, end;
+  size_t cnt, cursor, list_off, item_off, list, pos_of, part_o, part_lse, end;
   int Lc;
 };
 AttnWs attn_ws(const msa_params *p, size_t base) {
@@ -93,6 +94,7 @@ AttnWs attn_ws(const msa_params *p, size_t base) {
   w.list_off = o; o = align_up(o + 4 * (nbgj + 1));
   w.item_off = o; o = align_up(o + 4 * (nbgj + 1));
   w.list = o; o = align_up(o + 4 * size_t(p->B) * p->G * w.Lc * p->top_k);
+  w.pos_of = o; o = align_up(o + 4 * size_t(p->B) * p->G * w.Lc * p->top_k);
   w.part_o = o; o = align_up(o + 2 * size_t(p->B) * w.Lc * p->H * p->top_k * p->d);
   w.part_lse = o; o = align_up(o + 4 * size_t(p->B) * w.Lc * p->H * p->top_k);
   w.end = o;
@@ -232,6 +234,7 @@ int run_prefill_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
     ra.list_off = reinterpret_cast<int32_t *>(wsb + w.list_off);
     ra.item_off = reinterpret_cast<int32_t *>(wsb + w.item_off);
     ra.list = reinterpret_cast<int32_t *>(wsb + w.list);
+    ra.pos_of = reinterpret_cast<int32_t *>(wsb + w.pos_of);
     ra.status = status_ptr(ws);
     cudaError_t e = msa::launch_revidx(ra, st);
     if (e != cudaSuccess) return cuda_fail(e, "reverse index launch");
@@ -254,6 +257,7 @@ int run_prefill_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
     ca.B = p->B; ca.L = p->L; ca.H = p->H; ca.G = p->G; ca.top_k = p->top_k;
     ca.t0 = t0; ca.Lc = Lc;
     ca.sel = sel;
+    ca.pos_of = ra.pos_of;
     ca.part_o = aa.part_o; ca.part_lse = aa.part_lse;
     ca.out = out; ca.lse = lse;
     e = msa::launch_combine(ca, st);

@@ -8,24 +8,40 @@
 //
 // One work item = one (b, g, key block j) and up to 128/R queries that
 // selected j, each with its R heads: a 128-row tile.  Per item:
-//   TMA      K_j (128 x 128 bf16, 128B-swizzled) into the K/V buffer
-//   gather   the tile's q rows (R heads of a query are 256*R contiguous
-//            bytes) into a swizzled smem tile with cp.async
-//   UMMA     S = Q K_j^T   (M=128, N=128, K=128) into TMEM
-//   TMA      V_j into the K/V buffer, now that S has consumed K_j; the load
-//            overlaps the softmax
-//   softmax  thread r owns row r: mask s <= t, row max, exp2, row sum,
-//            P = exp(...) as bf16 into smem (over the dead Q tile)
-//   UMMA     O = P V_j into the same TMEM columns as S (V consumed MN-major
-//            straight from its TMA tile)
-//   store    O / l as a bf16 partial and lse = ln(sum exp(scale q.k)) per
-//            (t, head, slot); a second kernel merges a row's <= top_k
-//            partials.
-// A CTA holds one 32 KB K/V buffer, one 32 KB Q/P tile and 128 TMEM columns,
-// so three CTAs share an SM and their sequential phases overlap.  The next
-// item's query list is fetched while this item computes, and its K and q
-// rows are requested as soon as this item's second UMMA has consumed the
-// shared tiles, so those loads overlap the partial-result stores.
+//   S = Q K_j^T   (UMMA M=128, N=128, K=128, fp32 in TMEM)
+//   softmax       row r: mask s <= t (only on the diagonal block), row max,
+//                 exp2, row sum, P as bf16 into shared memory
+//   O = P V_j     (UMMA, V consumed MN-major straight from its TMA tile)
+//   partial       O / l (bf16) and lse = ln(sum exp(scale q.k)) per row; a
+//                 second kernel merges a query row's <= top_k partials.
+//
+// The work is HBM-bound: per item 32 KB of gathered q rows come in and 32 KB
+// of partials go out, against 0.5 us of tensor work.  The kernel is built to
+// keep those transfers in flight (one persistent CTA per SM, 16 warps with
+// fixed roles):
+//   warp 0     K/V producer: TMA loads of K_j and V_j into a ring of four
+//              32 KB tiles, once per run of consecutive items with the same
+//              key block (items are ordered by (b, g, j)).
+//   warp 1     TMEM owner and MMA issuer: issues S_i and O_i in whatever
+//              order their inputs become ready (non-blocking barrier probes).
+//   warps 2-7  three gather groups of 64 threads; group k owns shared stage
+//              k and the items i = k (mod 3): it publishes the item's query
+//              list, gathers the q rows (R heads of a query are 256*R
+//              contiguous bytes) with cp.async into the stage's 128B-swizzled
+//              tile, and prefetches its next item's descriptor meanwhile.
+//   warps 8-15 two softmax warpgroups, even and odd items, each with its own
+//              128-column TMEM slot (S, then O).  After the softmax a group
+//              loads O, stages the bf16 partial rows in the item's stage and
+//              writes them with one bulk copy.
+// A stage holds Q, then P, then the staged partial of one item; three stages
+// let the q gather of item i+3 start as soon as item i's partial has left.
+//
+// Partial layout.  The partials of a chunk are indexed by reverse-index list
+// position: the entry at position pos (query t, slot k of group g) owns rows
+// pos*R + hh (hh < R), so an item's rows are one contiguous range and leave
+// in one bulk copy.  Inside a row of 16 granules of 16 bytes, granule c is
+// stored at granule c ^ (row & 7): the staging writes are then free of bank
+// conflicts, and the merge undoes the permutation when it reads.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -39,17 +55,43 @@ namespace msa {
 
 namespace {
 
-constexpr int kAttnThreads = 128;
-constexpr int kAttnCtasPerSm = 3;
-constexpr int kSmemKV = 0;      // K tile, then V tile
-constexpr int kSmemQ = 32768;   // Q tile, then P tile
-constexpr int kSmemBar = 65536;
-constexpr int kAttnSmem = kSmemBar + 64 + 1024 + 1024;  // bars, items, 2 lists, align slack
+constexpr int kAttnThreads = 512;
+constexpr int kNQ = 3;                               // Q/P/partial stages
+constexpr int kNKV = 4;                              // K/V tiles: two runs in flight
+constexpr int kTile = 32768;                         // 128 rows x 256 B
+constexpr int kSmemQ = 0;
+constexpr int kSmemKV = kNQ * kTile;
+constexpr int kSmemCtl = kSmemKV + kNKV * kTile;     // 229376
+// mbarrier slots (8 bytes each) at kSmemCtl
+constexpr int kBarQFull = 0;                         // [kNQ]  64 gather threads
+constexpr int kBarStEmpty = kBarQFull + kNQ;         // [kNQ]  the storing thread
+constexpr int kBarKvFull = kBarStEmpty + kNQ;        // [kNKV] TMA transaction bytes
+constexpr int kBarKvEmpty = kBarKvFull + kNKV;       // [kNKV] UMMA commit
+constexpr int kBarSFull = kBarKvEmpty + kNKV;        // [2]    UMMA commit
+constexpr int kBarPFull = kBarSFull + 2;             // [2]    128 softmax threads
+constexpr int kBarOFull = kBarPFull + 2;             // [2]    UMMA commit
+constexpr int kBarTmEmpty = kBarOFull + 2;           // [2]    128 softmax threads
+constexpr int kBarDrain = kBarTmEmpty + 2;           // UMMA commit on the way out
+constexpr int kNumBars = kBarDrain + 1;              // 23
+constexpr int kCtlMisc = kNumBars * 8;               // tmem holder, abort flag
+constexpr int kCtlDesc = 192;                        // [kNQ] int4 {bgj, start, n, -}
+constexpr int kCtlPre = kCtlDesc + 16 * kNQ;         // [3] int4: gather groups' next item
+constexpr int kCtlList = kCtlPre + 48;               // [kNQ][128] list entries
+constexpr int kCtlBytes = kCtlList + kNQ * 128 * 4;
+constexpr int kAttnSmem = kSmemCtl + kCtlBytes + 1024;  // + alignment slack
+static_assert(kCtlMisc + 8 <= kCtlDesc, "control layout");
+static_assert(kCtlPre + 48 <= kCtlList, "control layout");
+static_assert(kAttnSmem <= 232448, "shared memory budget");
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
@@ -59,306 +101,447 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-struct AttnItemWalk {  // thread 0's position in the CTA's item range
-  int wb = 0, it_lo = 0, it_hi = 0, l_lo = 0, l_hi = 0;
-};
-
-// Gather the q rows of a work item into the swizzled Q tile: row = qi*R + hh,
-// 16 granules of 16 B per row; rows past the item's queries are zeroed.
-template <int R>
-__device__ __forceinline__ void gather_q(const AttnArgs &a, uint32_t s_q, const int *list, int n,
-                                         int b, int g, int tid) {
-#pragma unroll 4
-  for (int it = 0; it < 16; ++it) {
-    const int idx = it * kAttnThreads + tid;
-    const int row = idx >> 4;
-    const int gran = idx & 15;
-    const int qi = row / R;
-    const int hh = row % R;
-    const uint32_t dst = s_q + (gran >> 3) * 16384 + sw128_offset(row, gran & 7);
-    if (qi < n) {
-      const int t = list[qi] >> 5;
-      const uint16_t *src =
-          a.q + ((size_t(b) * a.L + t) * a.H + size_t(g) * R + hh) * kHeadDim + gran * 8;
-      cp_async16(dst, src);
-    } else {
-      asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(dst), "r"(0) : "memory");
-    }
-  }
+// Register split: the launch gives 128 registers to each of the 512 threads;
+// warpgroups 0-1 (producer, MMA, gatherers) keep 64 and the two softmax
+// warpgroups take 184 (256*64 + 256*184 = 63488 <= 65536).
+__device__ __forceinline__ void regs_dec_64() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 64;" ::: "memory");
+}
+__device__ __forceinline__ void regs_inc_184() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 184;" ::: "memory");
 }
 
+// Position of one thread in the item list of its CTA: item w belongs to the
+// key block bgj with item_off[bgj] <= w < item_off[bgj+1].
+struct ItemWalk {
+  int wb, it_lo, it_hi, l_lo, l_hi;
+  __device__ void init(const AttnArgs &a, int n_bgj, int w) {
+    int lo = 0, hi = n_bgj - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.item_off[mid] <= w) lo = mid; else hi = mid - 1;
+    }
+    wb = lo;
+    it_lo = a.item_off[lo]; it_hi = a.item_off[lo + 1];
+    l_lo = a.list_off[lo]; l_hi = a.list_off[lo + 1];
+  }
+  // {bgj, first list position, number of queries}
+  __device__ int4 describe(const AttnArgs &a, int qpi, int w) {
+    while (w >= it_hi) {
+      ++wb;
+      it_lo = it_hi; it_hi = a.item_off[wb + 1];
+      l_lo = l_hi; l_hi = a.list_off[wb + 1];
+    }
+    const int start = l_lo + (w - it_lo) * qpi;
+    return make_int4(wb, start, min(qpi, l_hi - start), 0);
+  }
+};
+
 template <int R>
-__global__ void __launch_bounds__(kAttnThreads, kAttnCtasPerSm)
+__global__ void __launch_bounds__(kAttnThreads, 1)
     msa_prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
   constexpr int QPI = 128 / R;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-  const uint32_t s_kv = smem_u32(smem + kSmemKV);
-  const uint32_t s_q = smem_u32(smem + kSmemQ);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSmemBar);
-  const uint32_t b_k = smem_u32(&bars[0]);
-  const uint32_t b_v = smem_u32(&bars[1]);
-  const uint32_t b_mma = smem_u32(&bars[2]);
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(&bars[3]);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
-  int *s_item = reinterpret_cast<int *>(smem + kSmemBar + 32);    // [2][4]: bgj, start, n, -
-  int *s_list = reinterpret_cast<int *>(smem + kSmemBar + 64);    // [2][128]
+  const uint32_t s_base = smem_u32(smem);
+  uint8_t *ctl = smem + kSmemCtl;
+  const uint32_t bar0 = smem_u32(ctl);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(ctl + kCtlMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctl + kCtlMisc + 4);
+  int4 *s_desc = reinterpret_cast<int4 *>(ctl + kCtlDesc);
+  int4 *s_pre = reinterpret_cast<int4 *>(ctl + kCtlPre);
+  int *s_list = reinterpret_cast<int *>(ctl + kCtlList);
+  auto bar = [&](int idx) { return bar0 + 8u * uint32_t(idx); };
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  const int lane = tid & 31;
   if (tid == 0) {
-    mbar_init(b_k, 1);
-    mbar_init(b_v, 1);
-    mbar_init(b_mma, 1);
+    for (int s = 0; s < kNQ; ++s) {
+      mbar_init(bar(kBarQFull + s), 64);
+      mbar_init(bar(kBarStEmpty + s), 1);
+    }
+    for (int x = 0; x < kNKV; ++x) {
+      mbar_init(bar(kBarKvFull + x), 1);
+      mbar_init(bar(kBarKvEmpty + x), 1);
+    }
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(bar(kBarSFull + u), 1);
+      mbar_init(bar(kBarPFull + u), 128);
+      mbar_init(bar(kBarOFull + u), 1);
+      mbar_init(bar(kBarTmEmpty + u), 128);
+    }
+    mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(tmem_holder), 128);
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 256);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_acc = *tmem_holder;   // S, then O
-  const uint32_t lane_off = uint32_t(warp * 32) << 16;
+  const uint32_t tmem_base = *tmem_holder;
 
   const int n_bgj = a.B * a.G * a.nb;
   const int n_items = a.item_off[n_bgj];
   if (n_items > a.max_items && tid == 0) atomicCAS(a.status, 0, kStatusBadInput);
-  constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
-  constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, 0, 1);
-  uint32_t k_ph = 0, v_ph = 0, mma_ph = 0;
-
-  // Each CTA takes a contiguous range of work items (ordered by (b, g, key
-  // block), so consecutive items mostly read the same K/V block from L2).
+  // Each CTA takes a contiguous range of work items: consecutive items mostly
+  // share their key block, whose K/V tiles are then loaded once.
   const int per = (n_items + gridDim.x - 1) / gridDim.x;
-  const int w_begin = blockIdx.x * per;
-  const int w_end = min(n_items, w_begin + per);
-  AttnItemWalk wk;
-  auto describe = [&](int w, int *dst) {  // thread 0: item w -> dst[0..2]
-    while (w >= wk.it_hi) {
-      ++wk.wb;
-      wk.it_lo = wk.it_hi; wk.it_hi = a.item_off[wk.wb + 1];
-      wk.l_lo = wk.l_hi; wk.l_hi = a.list_off[wk.wb + 1];
-    }
-    const int start = wk.l_lo + (w - wk.it_lo) * QPI;
-    dst[0] = wk.wb;
-    dst[1] = start;
-    dst[2] = min(QPI, wk.l_hi - start);
-  };
-  // thread 0: one 128-key tile of K or V of block bgj into the K/V buffer
-  auto issue_tile = [&](const CUtensorMap *tm, uint32_t bar, int bgj) {
-    const int j = bgj % a.nb;
-    const int bg = bgj / a.nb;
-    const int g = bg % a.G;
-    const int b = bg / a.G;
-    mbar_arrive_expect_tx(bar, 32768);
-    const int z = b * a.L + j * kBlock;
-    tma_load_3d(s_kv, tm, bar, 0, g, z);
-    tma_load_3d(s_kv + 16384, tm, bar, 64, g, z);
-  };
+  const int w_begin = min(n_items, int(blockIdx.x) * per);
+  const int n_loc = min(n_items, w_begin + per) - w_begin;
 
-  if (w_begin < w_end) {
-    if (tid == 0) {
-      int lo = 0, hi = n_bgj - 1;  // first bgj with item_off[bgj+1] > w_begin
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (a.item_off[mid] <= w_begin) lo = mid; else hi = mid - 1;
-      }
-      wk.wb = lo;
-      wk.it_lo = a.item_off[lo]; wk.it_hi = a.item_off[lo + 1];
-      wk.l_lo = a.list_off[lo]; wk.l_hi = a.list_off[lo + 1];
-      describe(w_begin, s_item);
-      issue_tile(&tm_k, b_k, s_item[0]);
-    }
-    __syncthreads();
-    if (tid < s_item[2]) s_list[tid] = a.list[s_item[1] + tid];
-    __syncthreads();
-    gather_q<R>(a, s_q, s_list, s_item[2], s_item[0] / (a.nb * a.G), (s_item[0] / a.nb) % a.G, tid);
-  }
-
-  int buf = 0;
-  for (int w = w_begin; w < w_end; ++w) {
-    const int *it = s_item + 4 * buf;
-    const int *lst = s_list + 128 * buf;
-    const int bgj = it[0];
-    const int n = it[2];
-    const int j = bgj % a.nb;
-    const int g = (bgj / a.nb) % a.G;
-    const int b = bgj / (a.nb * a.G);
-    const bool has_next = w + 1 < w_end;
-    int *nit = s_item + 4 * (buf ^ 1);
-    int *nlst = s_list + 128 * (buf ^ 1);
-    if (has_next && tid == 0) describe(w + 1, nit);
-    __syncthreads();
-    // the next item's query list: loaded now, stored to shared memory after
-    // this item's UMMAs, so its latency hides behind them
-    const int n_next = has_next ? nit[2] : 0;
-    const int next_entry = (tid < n_next) ? a.list[nit[1] + tid] : 0;
-
-    // ---- this item's q rows have landed
-    cp_async_wait_all();
-    fence_proxy_async_smem();
-    __syncthreads();
-
-    // ---- S = Q K^T
-    int ok_k = 1;
-    if (tid == 0) {
-      ok_k = mbar_wait(b_k, k_ph, abort_flag, a.status) ? 1 : 0;
-      if (ok_k) {
-        tc_fence_after();
+  if (warp < 8) {
+    regs_dec_64();   // warpgroups 0 and 1, one instruction each
+    if (warp == 0) {
+      // ------------------------------------------------------ K/V producer
+      if (lane == 0 && n_loc > 0) {
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        ItemWalk wk;
+        wk.init(a, n_bgj, w_begin);
+        int issued[kNKV] = {-1, -1, -1, -1};
+        int prev = -1, m = -1;
+        bool ok = true;
+        for (int i = 0; i < n_loc && ok; ++i) {
+          const int bgj = wk.describe(a, QPI, w_begin + i).x;
+          if (bgj == prev) continue;
+          prev = bgj;
+          ++m;
+          const int j = bgj % a.nb;
+          const int g = (bgj / a.nb) % a.G;
+          const int b = bgj / (a.nb * a.G);
+          const int z = b * a.L + j * kBlock;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const int c = kk >> 2;
-          const uint32_t off = (kk & 3) * 32;
-          umma_f16_ss(tmem_acc, sdesc_sw128(s_q + c * 16384 + off, 16, 1024),
-                      sdesc_sw128(s_kv + c * 16384 + off, 16, 1024), idesc_s, kk > 0);
+          for (int h = 0; h < 2; ++h) {   // K of run m is tile sequence 2m, V is 2m+1
+            const int tau = 2 * m + h;
+            const int x = tau & (kNKV - 1);
+            if (!mbar_wait(bar(kBarKvEmpty + x), ((tau >> 2) & 1) ^ 1, abort_flag, a.status)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(kBarKvFull + x), kTile);
+            const uint32_t dst = s_base + kSmemKV + x * kTile;
+            const CUtensorMap *tm = h ? &tm_v : &tm_k;
+            tma_load_3d(dst, tm, bar(kBarKvFull + x), 0, g, z);
+            tma_load_3d(dst + 16384, tm, bar(kBarKvFull + x), 64, g, z);
+            issued[x] = tau;
+          }
         }
-        umma_commit(b_mma);
+        // let every load still in flight land before the CTA can exit
+        for (int x = 0; x < kNKV; ++x)
+          if (issued[x] >= 0) mbar_wait_drain(bar(kBarKvFull + x), (issued[x] >> 2) & 1);
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------ MMA issuer
+      if (lane == 0 && n_loc > 0) {
+        constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, 0, 1);
+        int ns = 0, no = 0;          // next S and next O to issue (item indices)
+        int m_s = -1, prev_bgj = -1; // run of item ns-1 and its key block
+        // per in-flight item (ring of 4 by item index): 3 bits = run index mod 4
+        // (enough for the tile index, its parity and run changes between
+        // neighbours) and whether the item opens its run
+        uint32_t ring = 0;
+        bool q_seen = false, cur_new = false;
+        int cur_bgj = -1;
+        bool v_pending = false;      // O of run v_run's last-known item issued, successor unknown
+        int v_run = 0;
+        uint32_t idle = 0;
+        uint64_t t_idle = 0;
+        while (no < n_loc) {
+          bool progressed = false;
+          // ---- S_ns = Q K^T: needs the item's q rows, its K tile, a free TMEM slot
+          if (ns < n_loc && ns < no + 2) {
+            const int s = ns % kNQ;
+            if (!q_seen && mbar_test_wait(bar(kBarQFull + s), (ns / kNQ) & 1)) {
+              q_seen = true;
+              cur_bgj = s_desc[s].x;
+              cur_new = cur_bgj != prev_bgj;
+            }
+            if (q_seen) {
+              const int m = cur_new ? m_s + 1 : m_s;
+              const int xk = (2 * m) & (kNKV - 1);
+              const bool k_ok =
+                  !cur_new || mbar_test_wait(bar(kBarKvFull + xk), ((2 * m) >> 2) & 1);
+              if (k_ok && mbar_test_wait(bar(kBarTmEmpty + (ns & 1)), ((ns >> 1) & 1) ^ 1)) {
+                tc_fence_after();
+                if (cur_new && ns > 0) {
+                  // the previous run's last S is issued: its K tile frees when that completes
+                  umma_commit(bar(kBarKvEmpty + ((2 * m_s) & (kNKV - 1))));
+                  if (v_pending) umma_commit(bar(kBarKvEmpty + ((2 * v_run + 1) & (kNKV - 1))));
+                }
+                v_pending = false;
+                const uint32_t sq = s_base + kSmemQ + s * kTile;
+                const uint32_t sk = s_base + kSmemKV + xk * kTile;
+                const uint32_t d_tmem = tmem_base + (ns & 1) * 128;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                  const int c = kk >> 2;
+                  const uint32_t off = (kk & 3) * 32;
+                  umma_f16_ss(d_tmem, sdesc_sw128(sq + c * 16384 + off, 16, 1024),
+                              sdesc_sw128(sk + c * 16384 + off, 16, 1024), idesc_s, kk > 0);
+                }
+                umma_commit(bar(kBarSFull + (ns & 1)));
+                const uint32_t sh = 3u * uint32_t(ns & 3);
+                ring = (ring & ~(7u << sh)) | ((uint32_t(m & 3) | (cur_new ? 4u : 0u)) << sh);
+                m_s = m;
+                prev_bgj = cur_bgj;
+                q_seen = false;
+                ++ns;
+                progressed = true;
+              }
+            }
+          }
+          // ---- O_no = P V: needs the softmax's P and the item's V tile
+          if (no < ns) {
+            const uint32_t e = (ring >> (3u * uint32_t(no & 3))) & 7u;
+            const int m = int(e & 3u);   // run index mod 4
+            const int xv = (2 * m + 1) & (kNKV - 1);
+            const bool v_ok =
+                !(e & 4u) || mbar_test_wait(bar(kBarKvFull + xv), ((2 * m + 1) >> 2) & 1);
+            if (v_ok && mbar_test_wait(bar(kBarPFull + (no & 1)), (no >> 1) & 1)) {
+              tc_fence_after();
+              const uint32_t sp = s_base + kSmemQ + (no % kNQ) * kTile;
+              const uint32_t sv = s_base + kSmemKV + xv * kTile;
+              const uint32_t d_tmem = tmem_base + (no & 1) * 128;
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const int c = kk >> 2;
+                const uint32_t off = (kk & 3) * 32;
+                umma_f16_ss(d_tmem, sdesc_sw128(sp + c * 16384 + off, 16, 1024),
+                            sdesc_sw128(sv + kk * 2048, 16384, 1024), idesc_o, kk > 0);
+              }
+              umma_commit(bar(kBarOFull + (no & 1)));
+              // free run m's V tile once item no is known to be its last
+              if (no + 1 < ns) {
+                if (int((ring >> (3u * uint32_t((no + 1) & 3))) & 3u) != m)
+                  umma_commit(bar(kBarKvEmpty + xv));
+              } else if (no + 1 < n_loc) {
+                v_pending = true;
+                v_run = m;
+              }
+              ++no;
+              progressed = true;
+            }
+          }
+          if (progressed) {
+            idle = 0;
+            t_idle = 0;
+          } else if ((++idle & 1023u) == 0) {
+            if (*abort_flag) break;
+            const uint64_t now = globaltimer_ns();
+            if (t_idle == 0) {
+              t_idle = now;
+            } else if (now - t_idle > kWaitLimitNs) {
+              *abort_flag = 1;
+              atomicCAS(a.status, 0, kStatusTimeout);
+              break;
+            }
+          }
+        }
+        // every UMMA issued has completed before TMEM can be released
+        umma_commit(bar(kBarDrain));
+        mbar_wait_drain(bar(kBarDrain), 0);
+      }
+    } else {
+      // ------------------------------------------------------ q gatherers
+      const int k = (warp - 2) >> 1;       // group k owns stage k and items i = k (mod 3)
+      const int gtid = tid - 64 * (k + 1);
+      const int bar_id = 1 + k;
+      const int s = k;
+      ItemWalk wk;
+      // descriptor and list entries of the group's next item are fetched one
+      // item ahead, while the previous item's copies land
+      // Every warp of the group keeps the item's list entries in registers
+      // (entry 32c + lane in ent[c]) and looks a query up with a shuffle: the
+      // copy addresses then wait on no shared-memory load.
+      constexpr int NE = (QPI + 31) / 32;
+      int4 d = make_int4(0, 0, 0, 0);
+      int ent[NE];
+      auto load_entries = [&]() {
+#pragma unroll
+        for (int c = 0; c < NE; ++c)
+          ent[c] = (32 * c + lane < d.z) ? a.list[d.y + 32 * c + lane] : 0;
+      };
+      if (gtid == 0 && k < n_loc) {
+        wk.init(a, n_bgj, w_begin + k);
+        s_pre[k] = wk.describe(a, QPI, w_begin + k);
+      }
+      bar_sync_n(bar_id, 64);
+      if (k < n_loc) {
+        d = s_pre[k];
+        load_entries();
+      }
+      const int gran = gtid & 15;
+      for (int i = k; i < n_loc; i += kNQ) {
+        bool ok = mbar_wait(bar(kBarStEmpty + s), ((i / kNQ) & 1) ^ 1, abort_flag, a.status);
+        if (!bar_and_n(bar_id, 64, ok)) break;
+        if (gtid == 0) s_desc[s] = d;
+        if (gtid < 32) {   // the softmax reads t of its rows from shared memory
+#pragma unroll
+          for (int c = 0; c < NE; ++c)
+            if (32 * c + lane < d.z) s_list[s * 128 + 32 * c + lane] = ent[c];
+        }
+        const int bgj = d.x;
+        const int g = (bgj / a.nb) % a.G;
+        const int b = bgj / (a.nb * a.G);
+        const uint16_t *qb = a.q + (size_t(b) * a.L * a.H + size_t(g) * R) * kHeadDim + gran * 8;
+        const uint32_t stq = s_base + kSmemQ + s * kTile + (gran >> 3) * 16384;
+        // rows it*4 + (gtid >> 4), it < 32: the rows of iterations
+        // [c*32/NE, (c+1)*32/NE) hold queries 32c..32c+31, i.e. entries of ent[c]
+#pragma unroll
+        for (int c = 0; c < NE; ++c) {
+#pragma unroll 4
+          for (int it = c * (32 / NE); it < (c + 1) * (32 / NE); ++it) {
+            const int row = it * 4 + (gtid >> 4);
+            const int qi = row / R;
+            const int hh = row % R;
+            const int t = __shfl_sync(0xffffffffu, ent[c], qi & 31) >> 5;
+            if (qi < d.z)
+              cp_async16(stq + sw128_offset(row, gran & 7),
+                         qb + (size_t(t) * a.H + hh) * kHeadDim);
+          }
+        }
+        if (gtid == 0 && i + kNQ < n_loc) s_pre[k] = wk.describe(a, QPI, w_begin + i + kNQ);
+        bar_sync_n(bar_id, 64);   // s_pre published; s_list written (read by the softmax only)
+        if (i + kNQ < n_loc) {
+          d = s_pre[k];
+          load_entries();
+        }
+        cp_async_wait_all();
+        fence_proxy_async_smem();
+        mbar_arrive(bar(kBarQFull + s));
       }
     }
-    k_ph ^= 1;
-    // every exit decision below is taken by the whole CTA at one barrier
-    if (__syncthreads_or(!ok_k)) break;
-    const bool ok1 = mbar_wait(b_mma, mma_ph, abort_flag, a.status);
-    mma_ph ^= 1;
-    if (__syncthreads_or(!ok1)) break;
-    tc_fence_after();
-    // K has been consumed: bring V into the same buffer during the softmax
-    if (tid == 0) issue_tile(&tm_v, b_v, bgj);
+  } else {
+    // -------------------------------------------------------- softmax + partials
+    regs_inc_184();  // warpgroups 2 and 3, one instruction each
+    const int u = (warp - 8) >> 2;         // even / odd items, TMEM slot u
+    const int row = tid - 256 - 128 * u;   // TMEM lane = tile row
+    const int bar_id = 4 + u;
+    const uint32_t tm = tmem_base + u * 128 + (uint32_t((warp & 3) * 32) << 16);
+    for (int i = u; i < n_loc; i += 2) {
+      const int s = i % kNQ;
+      bool ok = mbar_wait(bar(kBarQFull + s), (i / kNQ) & 1, abort_flag, a.status);
+      if (!bar_and_n(bar_id, 128, ok)) break;
+      const int4 d = s_desc[s];
+      const int j = d.x % a.nb;
+      const int qi = row / R;
+      const bool valid = qi < d.z;
+      const int t = valid ? (s_list[s * 128 + qi] >> 5) : 0;
+      const int lim = valid ? (t - j * kBlock) : (kBlock - 1);   // last visible column
+      ok = mbar_wait(bar(kBarSFull + u), (i >> 1) & 1, abort_flag, a.status);
+      if (!bar_and_n(bar_id, 128, ok)) break;
+      tc_fence_after();
 
-    // ---- softmax on row `tid`, two 64-column halves per pass
-    const int qi = tid / R;
-    const bool valid = qi < n;
-    const int ent = valid ? lst[qi] : 0;
-    const int t = ent >> 5;
-    const int lim = valid ? (t - j * kBlock) : -1;  // last visible column
-    float m = -FLT_MAX;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float t0[32], t1[32];
-      tmem_ld32(tmem_acc + lane_off + h * 64, t0);
-      tmem_ld32(tmem_acc + lane_off + h * 64 + 32, t1);
-      tmem_wait_ld();
-#pragma unroll
-      for (int x = 0; x < 32; ++x) {
-        if (h * 64 + x <= lim) m = fmaxf(m, t0[x]);
-        if (h * 64 + 32 + x <= lim) m = fmaxf(m, t1[x]);
-      }
-    }
-    const float mb = m * a.scale_log2;
-    float l = 0.f;
-    uint8_t *p_tile = smem + kSmemQ;
-#pragma unroll 1
-    for (int h = 0; h < 2; ++h) {
-      float sv[64];
+      float v[128];
       {
-        float t0[32], t1[32];
-        tmem_ld32(tmem_acc + lane_off + h * 64, t0);
-        tmem_ld32(tmem_acc + lane_off + h * 64 + 32, t1);
+        float t0[32], t1[32], t2[32], t3[32];
+        tmem_ld32(tm, t0);
+        tmem_ld32(tm + 32, t1);
+        tmem_ld32(tm + 64, t2);
+        tmem_ld32(tm + 96, t3);
         tmem_wait_ld();
 #pragma unroll
-        for (int x = 0; x < 32; ++x) { sv[x] = t0[x]; sv[32 + x] = t1[x]; }
-      }
-#pragma unroll
-      for (int gblk = 0; gblk < 8; ++gblk) {
-        uint32_t w4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c0 = gblk * 8 + e * 2;
-          const int cg = h * 64 + c0;
-          const float p0 = (cg <= lim) ? fast_exp2(fmaf(sv[c0], a.scale_log2, -mb)) : 0.f;
-          const float p1 = (cg + 1 <= lim) ? fast_exp2(fmaf(sv[c0 + 1], a.scale_log2, -mb)) : 0.f;
-          l += p0 + p1;
-          w4[e] = pack_bf16x2(p0, p1);
+        for (int x = 0; x < 32; ++x) {
+          v[x] = t0[x]; v[32 + x] = t1[x]; v[64 + x] = t2[x]; v[96 + x] = t3[x];
         }
-        *reinterpret_cast<uint4 *>(p_tile + h * 16384 + sw128_offset(tid, gblk)) =
-            make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- O = P V (into the S columns: every thread has read S already)
-    int ok_v = 1;
-    if (tid == 0) {
-      ok_v = mbar_wait(b_v, v_ph, abort_flag, a.status) ? 1 : 0;
-      if (ok_v) {
-        tc_fence_after();
+      // causal mask: only rows whose own block is j see fewer than 128 keys
+      if (__any_sync(0xffffffffu, lim < kBlock - 1)) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const int c = kk >> 2;
-          const uint32_t off = (kk & 3) * 32;
-          umma_f16_ss(tmem_acc, sdesc_sw128(s_q + c * 16384 + off, 16, 1024),
-                      sdesc_sw128(s_kv + kk * 2048, 16384, 1024), idesc_o, kk > 0);
-        }
-        umma_commit(b_mma);
+        for (int x = 0; x < 128; ++x) v[x] = (x <= lim) ? v[x] : -INFINITY;
       }
-    }
-    v_ph ^= 1;
-    if (__syncthreads_or(!ok_v)) break;
-    const bool ok2 = mbar_wait(b_mma, mma_ph, abort_flag, a.status);
-    mma_ph ^= 1;
-    if (__syncthreads_or(!ok2)) break;
-    tc_fence_after();
-
-    // ---- the shared tiles are free: request the next item's K and q rows
-    if (tid < n_next) nlst[tid] = next_entry;
-    __syncthreads();
-    if (has_next) {
-      if (tid == 0) issue_tile(&tm_k, b_k, nit[0]);
-      gather_q<R>(a, s_q, nlst, nit[2], nit[0] / (a.nb * a.G), (nit[0] / a.nb) % a.G, tid);
-    }
-
-    // ---- store the normalised partial and its lse.  tcgen05.ld is a
-    // warp-wide (.sync.aligned) instruction: every thread loads, only rows
-    // holding a query store.
-    {
-      const int slot = ent & 31;
-      const int hh = tid % R;
-      const bool store = valid && lim >= 0;
-      const float inv = store ? 1.f / l : 0.f;
-      const size_t prow =
-          ((size_t(b) * a.Lc + (t - a.t0)) * a.H + size_t(g) * R + hh) * a.top_k + slot;
-      uint4 *dst = reinterpret_cast<uint4 *>(a.part_o + prow * kHeadDim);
-#pragma unroll 1
+      float m0 = max3f(v[0], v[1], v[2]), m1 = max3f(v[32], v[33], v[34]);
+      float m2 = max3f(v[64], v[65], v[66]), m3 = max3f(v[96], v[97], v[98]);
+#pragma unroll
+      for (int x = 3; x + 2 <= 31; x += 2) {
+        m0 = max3f(m0, v[x], v[x + 1]);
+        m1 = max3f(m1, v[32 + x], v[33 + x]);
+        m2 = max3f(m2, v[64 + x], v[65 + x]);
+        m3 = max3f(m3, v[96 + x], v[97 + x]);
+      }
+      m0 = fmaxf(m0, v[31]); m1 = fmaxf(m1, v[63]); m2 = fmaxf(m2, v[95]); m3 = fmaxf(m3, v[127]);
+      const float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+      const float mb = m * a.scale_log2;
+      float l = 0.f;
+      uint8_t *stage = smem + kSmemQ + s * kTile;
+#pragma unroll
       for (int h = 0; h < 2; ++h) {
-        float o0[32], o1[32];
-        tmem_ld32(tmem_acc + lane_off + h * 64, o0);
-        tmem_ld32(tmem_acc + lane_off + h * 64 + 32, o1);
-        tmem_wait_ld();
-        if (store) {
 #pragma unroll
-          for (int x = 0; x < 4; ++x)
-            dst[h * 8 + x] = make_uint4(pack_bf16x2(o0[8 * x] * inv, o0[8 * x + 1] * inv),
-                                        pack_bf16x2(o0[8 * x + 2] * inv, o0[8 * x + 3] * inv),
-                                        pack_bf16x2(o0[8 * x + 4] * inv, o0[8 * x + 5] * inv),
-                                        pack_bf16x2(o0[8 * x + 6] * inv, o0[8 * x + 7] * inv));
+        for (int gb = 0; gb < 8; ++gb) {
+          uint32_t w4[4];
 #pragma unroll
-          for (int x = 0; x < 4; ++x)
-            dst[h * 8 + 4 + x] = make_uint4(pack_bf16x2(o1[8 * x] * inv, o1[8 * x + 1] * inv),
-                                            pack_bf16x2(o1[8 * x + 2] * inv, o1[8 * x + 3] * inv),
-                                            pack_bf16x2(o1[8 * x + 4] * inv, o1[8 * x + 5] * inv),
-                                            pack_bf16x2(o1[8 * x + 6] * inv, o1[8 * x + 7] * inv));
+          for (int e = 0; e < 4; ++e) {
+            const int c = h * 64 + gb * 8 + e * 2;
+            const float p0 = fast_exp2(fmaf(v[c], a.scale_log2, -mb));
+            const float p1 = fast_exp2(fmaf(v[c + 1], a.scale_log2, -mb));
+            l += p0 + p1;
+            w4[e] = pack_bf16x2(p0, p1);
+          }
+          *reinterpret_cast<uint4 *>(stage + h * 16384 + sw128_offset(row, gb)) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
       }
-      if (valid) a.part_lse[prow] = store ? m * a.scale + __logf(l) : -INFINITY;
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(kBarPFull + u));
+
+      ok = mbar_wait(bar(kBarOFull + u), (i >> 1) & 1, abort_flag, a.status);
+      if (!bar_and_n(bar_id, 128, ok)) break;
+      tc_fence_after();
+      {
+        float t0[32], t1[32], t2[32], t3[32];
+        tmem_ld32(tm, t0);
+        tmem_ld32(tm + 32, t1);
+        tmem_ld32(tm + 64, t2);
+        tmem_ld32(tm + 96, t3);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          v[x] = t0[x]; v[32 + x] = t1[x]; v[64 + x] = t2[x]; v[96 + x] = t3[x];
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(kBarTmEmpty + u));   // slot u may take the next S
+
+      // stage the normalised bf16 partial row (granule c at c ^ (row & 7))
+      const float inv = 1.f / l;
+      const int rho = d.y * R + row;       // partial row of (list position, head)
+      uint8_t *orow = stage + row * 256;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const uint4 w = make_uint4(pack_bf16x2(v[8 * c] * inv, v[8 * c + 1] * inv),
+                                   pack_bf16x2(v[8 * c + 2] * inv, v[8 * c + 3] * inv),
+                                   pack_bf16x2(v[8 * c + 4] * inv, v[8 * c + 5] * inv),
+                                   pack_bf16x2(v[8 * c + 6] * inv, v[8 * c + 7] * inv));
+        *reinterpret_cast<uint4 *>(orow + ((c ^ (rho & 7)) << 4)) = w;
+      }
+      if (valid) a.part_lse[rho] = m * a.scale + __logf(l);
+      fence_proxy_async_smem();
+      bar_sync_n(bar_id, 128);
+      if (row == 0) {
+        bulk_store(a.part_o + size_t(d.y) * R * kHeadDim, s_base + kSmemQ + s * kTile,
+                   uint32_t(d.z) * R * 256u);
+        bulk_commit();
+        bulk_wait_read_all();
+        mbar_arrive(bar(kBarStEmpty + s));   // the stage may take item i+3
+      }
     }
-    tc_fence_before();
-    __syncthreads();
-    buf ^= 1;
+    if (row == 0) bulk_wait_all();
   }
 
   cp_async_wait_all();   // nothing may still be landing in shared memory
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_acc, 128);
+    tmem_dealloc(tmem_base, 256);
   }
 }
 
@@ -368,7 +551,7 @@ cudaError_t launch_attn_r(const CUtensorMap &tk, const CUtensorMap &tv, const At
   auto kern = msa_prefill_attn_kernel<R>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
   if (e != cudaSuccess) return e;
-  int grid = kAttnCtasPerSm * num_sms;
+  int grid = num_sms;
   if (a.max_items < grid) grid = a.max_items > 0 ? a.max_items : 1;
   kern<<<grid, kAttnThreads, kAttnSmem, st>>>(tk, tv, a);
   return cudaGetLastError();
@@ -394,9 +577,10 @@ namespace {
 
 // One warp per (b, t, h): merge the row's partials (normalised o_s, lse_s)
 // into o = sum_s exp(lse_s - M) o_s / sum_s exp(lse_s - M), M = max lse_s.
-// All of a lane's partial-row loads (4 of the d values of each slot) and its
-// lse load are issued before any reduction, so a row costs one memory round
-// trip after its selection row is known.
+// Slot s of the row lives at partial row rho_s = pos_of[b,g,t,s] * R + hh.
+// The selection row and the positions are loaded independently, then all of
+// a lane's partial-row loads (4 of the d values of each slot, granule order
+// undone) and its lse load are issued before any reduction.
 template <int KCAP>
 __global__ void __launch_bounds__(256) msa_combine_kernel(const CombineArgs a) {
   const long long wrow = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -408,19 +592,28 @@ __global__ void __launch_bounds__(256) msa_combine_kernel(const CombineArgs a) {
   const int tl = (int)(bt % a.Lc);
   const int b = (int)(bt / a.Lc);
   const int t = a.t0 + tl;
-  const int g = h / (a.H / a.G);
+  const int r = a.H / a.G;
+  const int g = h / r;
+  const int hh = h % r;
   const int32_t *sel = a.sel + ((size_t(b) * a.G + g) * a.L + t) * a.top_k;
-  const size_t prow0 = (((size_t)b * a.Lc + tl) * a.H + h) * a.top_k;
-  const bool mine = lane < a.top_k && sel[lane] >= 0;
+  const int32_t *pos = a.pos_of + ((size_t(b) * a.G + g) * a.Lc + tl) * a.top_k;
+  const bool in_k = lane < a.top_k;
+  const int my_sel = in_k ? sel[lane] : -1;
+  const int my_pos = in_k ? pos[lane] : 0;
+  const bool mine = my_sel >= 0;
   const unsigned vmask = __ballot_sync(0xffffffffu, mine);
+  const long long my_rho = mine ? (long long)my_pos * r + hh : 0;
   uint2 v[KCAP];
 #pragma unroll
   for (int s = 0; s < KCAP; ++s) {
     v[s] = make_uint2(0u, 0u);
-    if ((vmask >> s) & 1u)
-      v[s] = __ldcs(reinterpret_cast<const uint2 *>(a.part_o + (prow0 + s) * kHeadDim + lane * 4));
+    const long long rho = __shfl_sync(0xffffffffu, my_rho, s);
+    if ((vmask >> s) & 1u) {
+      const int col = ((((lane >> 1) ^ int(rho & 7)) << 3) | ((lane & 1) << 2));
+      v[s] = __ldcs(reinterpret_cast<const uint2 *>(a.part_o + rho * kHeadDim + col));
+    }
   }
-  const float my_lse = mine ? __ldcs(a.part_lse + prow0 + lane) : -INFINITY;
+  const float my_lse = mine ? __ldcs(a.part_lse + my_rho) : -INFINITY;
   float M = my_lse;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
@@ -441,10 +634,10 @@ __global__ void __launch_bounds__(256) msa_combine_kernel(const CombineArgs a) {
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  uint2 r;
-  r.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-  r.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-  *reinterpret_cast<uint2 *>(a.out + (((size_t)b * a.L + t) * a.H + h) * kHeadDim + lane * 4) = r;
+  uint2 res;
+  res.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  res.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  *reinterpret_cast<uint2 *>(a.out + (((size_t)b * a.L + t) * a.H + h) * kHeadDim + lane * 4) = res;
   if (a.lse && lane == 0) a.lse[((size_t)b * a.L + t) * a.H + h] = (wsum > 0.f) ? M + __logf(wsum) : -INFINITY;
 }
 

@@ -11,7 +11,9 @@
 //              at most qpi queries, i.e. 128 query-head rows, per block)
 //   3. fill    list[list_off[bgj] + k] = t * 32 + slot  (order inside a
 //              list is arbitrary: each (t, slot) partial is computed
-//              independently of the others in its tile)
+//              independently of the others in its tile), and the inverse
+//              map pos_of[b,g,t,slot] = that list position, by which the
+//              merge finds a row's partials
 // Every work item then holds <= qpi queries, so items cost the same and a
 // persistent grid balances itself whatever the causal skew between early
 // and late key blocks.
@@ -128,6 +130,7 @@ __global__ void __launch_bounds__(256) revidx_fill_kernel(const RevIdxArgs a) {
     const long long bgj = bg * a.nb + j;
     const int pos = a.list_off[bgj] + atomicAdd(&a.cursor[bgj], 1);
     a.list[pos] = t * 32 + k;
+    a.pos_of[r * a.top_k + k] = pos;
   }
 }
 

@@ -115,7 +115,7 @@ def test_zero_index_keys_all_ties():
 # ------------------------------------------------------------------ prefill attention
 @pytest.mark.parametrize("L,H,G,top_k,seed", [(2048, 8, 2, 4, 0), (1024, 32, 8, 3, 21),
                                               (768, 16, 16, 2, 22), (512, 16, 1, 3, 23),
-                                              (512, 16, 8, 8, 24)])
+                                              (512, 16, 8, 8, 24), (1024, 16, 2, 5, 25)])
 def test_prefill_attention_on_oracle_selection(L, H, G, top_k, seed):
     di = 64 if L == 2048 else 128
     shape = I.PrefillShape(B=2, L=L, H=H, G=G, d=128, d_idx=di, top_k=top_k)
