@@ -63,8 +63,8 @@ constexpr int kSmemQ = 0;
 constexpr int kSmemKV = kNQ * kTile;
 constexpr int kSmemCtl = kSmemKV + kNKV * kTile;     // 229376
 // mbarrier slots (8 bytes each) at kSmemCtl
-constexpr int kBarQFull = 0;                         // [kNQ]  64 gather threads
-constexpr int kBarStEmpty = kBarQFull + kNQ;         // [kNQ]  the storing thread
+constexpr int kBarQFull = 0;                         // [kNQ]  gather team copies + list
+constexpr int kBarStEmpty = kBarQFull + kNQ;         // [kNQ]  four storing warps
 constexpr int kBarKvFull = kBarStEmpty + kNQ;        // [kNKV] TMA transaction bytes
 constexpr int kBarKvEmpty = kBarKvFull + kNKV;       // [kNKV] UMMA commit
 constexpr int kBarSFull = kBarKvEmpty + kNKV;        // [2]    UMMA commit
@@ -75,7 +75,7 @@ constexpr int kBarDrain = kBarTmEmpty + 2;           // UMMA commit on the way o
 constexpr int kNumBars = kBarDrain + 1;              // 23
 constexpr int kCtlMisc = kNumBars * 8;               // tmem holder, abort flag
 constexpr int kCtlDesc = 192;                        // [kNQ] int4 {bgj, start, n, -}
-constexpr int kCtlPre = kCtlDesc + 16 * kNQ;         // [3] int4: gather groups' next item
+constexpr int kCtlPre = kCtlDesc + 16 * kNQ;         // int4: the gather team's next item
 constexpr int kCtlList = kCtlPre + 48;               // [kNQ][128] list entries
 constexpr int kCtlBytes = kCtlList + kNQ * 128 * 4;
 constexpr int kAttnSmem = kSmemCtl + kCtlBytes + 1024;  // + alignment slack
@@ -94,8 +94,42 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
+// Packed fp32 pair arithmetic (one instruction for two lanes of data).
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mul.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// Arrive on `bar` once every cp.async this thread has issued so far has
+// landed; the arrival is one of the barrier's expected count.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
@@ -160,8 +194,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   const int lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < kNQ; ++s) {
-      mbar_init(bar(kBarQFull + s), 64);
-      mbar_init(bar(kBarStEmpty + s), 1);
+      mbar_init(bar(kBarQFull + s), 193);   // 192 copy completions + the list
+      mbar_init(bar(kBarStEmpty + s), 4);   // the four softmax warps' stores
     }
     for (int x = 0; x < kNKV; ++x) {
       mbar_init(bar(kBarKvFull + x), 1);
@@ -270,6 +304,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                   !cur_new || mbar_test_wait(bar(kBarKvFull + xk), ((2 * m) >> 2) & 1);
               if (k_ok && mbar_test_wait(bar(kBarTmEmpty + (ns & 1)), ((ns >> 1) & 1) ^ 1)) {
                 tc_fence_after();
+                fence_proxy_async_smem();   // cp.async-written q rows -> UMMA operand reads
                 if (cur_new && ns > 0) {
                   // the previous run's last S is issued: its K tile frees when that completes
                   umma_commit(bar(kBarKvEmpty + ((2 * m_s) & (kNKV - 1))));
@@ -332,7 +367,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (progressed) {
             idle = 0;
             t_idle = 0;
-          } else if ((++idle & 1023u) == 0) {
+          } else {
+            // back off between probes: a hot probe loop slows the shared
+            // memory-instruction path of the warps sharing this SM sub-partition
+            __nanosleep(32);
+          }
+          if (!progressed && (++idle & 255u) == 0) {
             if (*abort_flag) break;
             const uint64_t now = globaltimer_ns();
             if (t_idle == 0) {
@@ -349,17 +389,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_wait_drain(bar(kBarDrain), 0);
       }
     } else {
-      // ------------------------------------------------------ q gatherers
-      const int k = (warp - 2) >> 1;       // group k owns stage k and items i = k (mod 3)
-      const int gtid = tid - 64 * (k + 1);
-      const int bar_id = 1 + k;
-      const int s = k;
+      // ------------------------------------------------------ q gather team
+      // All six gather warps work on every item in turn: a warp's copy
+      // issue rate is limited, so an item's 2048 16-byte copies are spread
+      // over 192 threads (11 each).  Completion is signalled by the copies
+      // themselves (cp.async.mbarrier.arrive.noinc), so the team moves on to
+      // the next free stage while they land.
+      const int gtid = tid - 64;             // 0..191
+      const int wg = warp - 2;               // 0..5
+      constexpr int kTeam = 192;
+      constexpr int bar_id = 1;
       ItemWalk wk;
-      // descriptor and list entries of the group's next item are fetched one
-      // item ahead, while the previous item's copies land
-      // Every warp of the group keeps the item's list entries in registers
-      // (entry 32c + lane in ent[c]) and looks a query up with a shuffle: the
-      // copy addresses then wait on no shared-memory load.
+      // Every warp keeps the item's list entries in registers (entry 32c +
+      // lane in ent[c]) and looks a query up with a shuffle.  The next
+      // item's descriptor and entries are fetched while the copies land.
       constexpr int NE = (QPI + 31) / 32;
       int4 d = make_int4(0, 0, 0, 0);
       int ent[NE];
@@ -368,54 +411,59 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int c = 0; c < NE; ++c)
           ent[c] = (32 * c + lane < d.z) ? a.list[d.y + 32 * c + lane] : 0;
       };
-      if (gtid == 0 && k < n_loc) {
-        wk.init(a, n_bgj, w_begin + k);
-        s_pre[k] = wk.describe(a, QPI, w_begin + k);
+      if (gtid == 0 && n_loc > 0) {
+        wk.init(a, n_bgj, w_begin);
+        s_pre[0] = wk.describe(a, QPI, w_begin);
       }
-      bar_sync_n(bar_id, 64);
-      if (k < n_loc) {
-        d = s_pre[k];
+      bar_sync_n(bar_id, kTeam);
+      if (n_loc > 0) {
+        d = s_pre[0];
         load_entries();
       }
-      const int gran = gtid & 15;
-      for (int i = k; i < n_loc; i += kNQ) {
+      const int gran = lane & 15;
+      for (int i = 0; i < n_loc; ++i) {
+        const int s = i % kNQ;
         bool ok = mbar_wait(bar(kBarStEmpty + s), ((i / kNQ) & 1) ^ 1, abort_flag, a.status);
-        if (!bar_and_n(bar_id, 64, ok)) break;
-        if (gtid == 0) s_desc[s] = d;
-        if (gtid < 32) {   // the softmax reads t of its rows from shared memory
+        if (!bar_and_n(bar_id, kTeam, ok)) break;
+        if (gtid < 32) {   // publish the item: the MMA and the softmax read these
+          if (gtid == 0) s_desc[s] = d;
 #pragma unroll
           for (int c = 0; c < NE; ++c)
             if (32 * c + lane < d.z) s_list[s * 128 + 32 * c + lane] = ent[c];
+          __syncwarp();
+          if (gtid == 0) mbar_arrive(bar(kBarQFull + s));
         }
         const int bgj = d.x;
         const int g = (bgj / a.nb) % a.G;
         const int b = bgj / (a.nb * a.G);
         const uint16_t *qb = a.q + (size_t(b) * a.L * a.H + size_t(g) * R) * kHeadDim + gran * 8;
         const uint32_t stq = s_base + kSmemQ + s * kTile + (gran >> 3) * 16384;
-        // rows it*4 + (gtid >> 4), it < 32: the rows of iterations
-        // [c*32/NE, (c+1)*32/NE) hold queries 32c..32c+31, i.e. entries of ent[c]
+        // row pair p = wg + 6*it (rows 2p, 2p+1): one coalesced 512-byte
+        // copy per warp instruction
 #pragma unroll
-        for (int c = 0; c < NE; ++c) {
-#pragma unroll 4
-          for (int it = c * (32 / NE); it < (c + 1) * (32 / NE); ++it) {
-            const int row = it * 4 + (gtid >> 4);
+        for (int it = 0; it < 11; ++it) {
+          const int p = wg + 6 * it;
+          if (p < 64) {
+            const int row = 2 * p + (lane >> 4);
             const int qi = row / R;
             const int hh = row % R;
-            const int t = __shfl_sync(0xffffffffu, ent[c], qi & 31) >> 5;
+            int e = ent[0];
+#pragma unroll
+            for (int c = 1; c < NE; ++c)
+              if ((qi >> 5) == c) e = ent[c];   // warp-uniform: 2p, 2p+1 share qi >> 5
+            const int t = __shfl_sync(0xffffffffu, e, qi & 31) >> 5;
             if (qi < d.z)
               cp_async16(stq + sw128_offset(row, gran & 7),
                          qb + (size_t(t) * a.H + hh) * kHeadDim);
           }
         }
-        if (gtid == 0 && i + kNQ < n_loc) s_pre[k] = wk.describe(a, QPI, w_begin + i + kNQ);
-        bar_sync_n(bar_id, 64);   // s_pre published; s_list written (read by the softmax only)
-        if (i + kNQ < n_loc) {
-          d = s_pre[k];
+        cp_async_arrive_noinc(bar(kBarQFull + s));
+        if (gtid == 0 && i + 1 < n_loc) s_pre[0] = wk.describe(a, QPI, w_begin + i + 1);
+        bar_sync_n(bar_id, kTeam);
+        if (i + 1 < n_loc) {
+          d = s_pre[0];
           load_entries();
         }
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        mbar_arrive(bar(kBarQFull + s));
       }
     }
   } else {
@@ -469,7 +517,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       m0 = fmaxf(m0, v[31]); m1 = fmaxf(m1, v[63]); m2 = fmaxf(m2, v[95]); m3 = fmaxf(m3, v[127]);
       const float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
       const float mb = m * a.scale_log2;
-      float l = 0.f;
+      const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+      const float2 nmb2 = make_float2(-mb, -mb);
+      float2 l2 = make_float2(0.f, 0.f);
       uint8_t *stage = smem + kSmemQ + s * kTile;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -479,10 +529,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = h * 64 + gb * 8 + e * 2;
-            const float p0 = fast_exp2(fmaf(v[c], a.scale_log2, -mb));
-            const float p1 = fast_exp2(fmaf(v[c + 1], a.scale_log2, -mb));
-            l += p0 + p1;
-            w4[e] = pack_bf16x2(p0, p1);
+            const float2 x = fma2(make_float2(v[c], v[c + 1]), sc2, nmb2);
+            const float2 pp = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            l2 = add2(l2, pp);
+            w4[e] = pack_bf16x2(pp.x, pp.y);
           }
           *reinterpret_cast<uint4 *>(stage + h * 16384 + sw128_offset(row, gb)) =
               make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -511,29 +561,39 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(bar(kBarTmEmpty + u));   // slot u may take the next S
 
       // stage the normalised bf16 partial row (granule c at c ^ (row & 7))
+      const float l = l2.x + l2.y;
       const float inv = 1.f / l;
+      const float2 inv2 = make_float2(inv, inv);
       const int rho = d.y * R + row;       // partial row of (list position, head)
       uint8_t *orow = stage + row * 256;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const uint4 w = make_uint4(pack_bf16x2(v[8 * c] * inv, v[8 * c + 1] * inv),
-                                   pack_bf16x2(v[8 * c + 2] * inv, v[8 * c + 3] * inv),
-                                   pack_bf16x2(v[8 * c + 4] * inv, v[8 * c + 5] * inv),
-                                   pack_bf16x2(v[8 * c + 6] * inv, v[8 * c + 7] * inv));
+        const float2 o0 = mul2(make_float2(v[8 * c], v[8 * c + 1]), inv2);
+        const float2 o1 = mul2(make_float2(v[8 * c + 2], v[8 * c + 3]), inv2);
+        const float2 o2 = mul2(make_float2(v[8 * c + 4], v[8 * c + 5]), inv2);
+        const float2 o3 = mul2(make_float2(v[8 * c + 6], v[8 * c + 7]), inv2);
+        const uint4 w = make_uint4(pack_bf16x2(o0.x, o0.y), pack_bf16x2(o1.x, o1.y),
+                                   pack_bf16x2(o2.x, o2.y), pack_bf16x2(o3.x, o3.y));
         *reinterpret_cast<uint4 *>(orow + ((c ^ (rho & 7)) << 4)) = w;
       }
       if (valid) a.part_lse[rho] = m * a.scale + __logf(l);
+      // each warp writes its own 32 rows (those holding a query) as soon as
+      // they are staged
       fence_proxy_async_smem();
-      bar_sync_n(bar_id, 128);
-      if (row == 0) {
-        bulk_store(a.part_o + size_t(d.y) * R * kHeadDim, s_base + kSmemQ + s * kTile,
-                   uint32_t(d.z) * R * 256u);
-        bulk_commit();
-        bulk_wait_read_all();
-        mbar_arrive(bar(kBarStEmpty + s));   // the stage may take item i+3
+      __syncwarp();
+      if (lane == 0) {
+        const int wrow0 = (warp & 3) * 32;
+        const int nrows = min(32, d.z * R - wrow0);
+        if (nrows > 0) {
+          bulk_store(a.part_o + (size_t(d.y) * R + wrow0) * kHeadDim,
+                     s_base + kSmemQ + s * kTile + wrow0 * 256, uint32_t(nrows) * 256u);
+          bulk_commit();
+          bulk_wait_read_all();
+        }
+        mbar_arrive(bar(kBarStEmpty + s));   // with all four: the stage may take item i+3
       }
     }
-    if (row == 0) bulk_wait_all();
+    if (lane == 0) bulk_wait_all();
   }
 
   cp_async_wait_all();   // nothing may still be landing in shared memory
