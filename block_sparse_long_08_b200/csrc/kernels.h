@@ -32,11 +32,10 @@ struct RevIdxArgs {
   int t0, Lc;                   // query chunk [t0, t0 + Lc)
   const int32_t *sel;           // [B,G,L,top_k]
   int32_t *cnt;                 // [B*G*nb]      (zeroed by the caller)
-  int32_t *cursor;              // [B*G*nb]
   int32_t *list_off;            // [B*G*nb + 1]
   int32_t *item_off;            // [B*G*nb + 1]
   int32_t *list;                // [B*G*Lc*top_k]
-  int32_t *pos_of;              // [B,G,Lc,top_k]: list position of each selected entry
+  int32_t *pos_of;              // [B,G,Lc,top_k]: rank in its block's list, then list position
   int *status;
 };
 cudaError_t launch_revidx(const RevIdxArgs &a, cudaStream_t st);

@@ -67,8 +67,11 @@ float eff_scale(const msa_params *p) {
 // ---- workspace plans --------------------------------------------------------
 // Prefill attention processes queries in chunks of Lc so that the partial
 // results (bf16, one 128-wide row per selected (query, head, slot)) stay
-// within a fixed budget.
-constexpr size_t kPartialBudget = size_t(4608) << 20;  // 4.5 GiB
+// within a fixed budget.  Every chunk reads the K/V blocks its queries
+// select, which for long inputs is most of K/V, so fewer, larger chunks
+// cut K/V re-reads: 16 GiB of partials is 9 chunks at 1M tokens, H=32,
+// top_k=16 (a small share of HBM on this part).
+constexpr size_t kPartialBudget = size_t(16) << 30;  // 16 GiB
 
 int prefill_chunk(const msa_params *p) {
   const size_t per_q = size_t(p->B) * p->H * p->top_k * (p->d * 2 + 4);
@@ -80,7 +83,7 @@ int prefill_chunk(const msa_params *p) {
 }
 
 struct AttnWs {
-  size_t cnt, cursor, list_off, item_off, list, pos_of, part_o, part_lse, end;
+  size_t cnt, list_off, item_off, list, pos_of, part_o, part_lse, end;
   int Lc;
 };
 AttnWs attn_ws(const msa_params *p, size_t base) {
@@ -90,7 +93,6 @@ AttnWs attn_ws(const msa_params *p, size_t base) {
   const size_t nbgj = size_t(p->B) * p->G * nb;
   size_t o = base;
   w.cnt = o; o = align_up(o + 4 * nbgj);
-  w.cursor = o; o = align_up(o + 4 * nbgj);
   w.list_off = o; o = align_up(o + 4 * (nbgj + 1));
   w.item_off = o; o = align_up(o + 4 * (nbgj + 1));
   w.list = o; o = align_up(o + 4 * size_t(p->B) * p->G * w.Lc * p->top_k);
@@ -230,7 +232,6 @@ int run_prefill_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
     ra.t0 = t0; ra.Lc = Lc;
     ra.sel = sel;
     ra.cnt = reinterpret_cast<int32_t *>(wsb + w.cnt);
-    ra.cursor = reinterpret_cast<int32_t *>(wsb + w.cursor);
     ra.list_off = reinterpret_cast<int32_t *>(wsb + w.list_off);
     ra.item_off = reinterpret_cast<int32_t *>(wsb + w.item_off);
     ra.list = reinterpret_cast<int32_t *>(wsb + w.list);

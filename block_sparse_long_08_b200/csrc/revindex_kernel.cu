@@ -5,15 +5,18 @@
 // For a query chunk [t0, t0+Lc) it lists, for every (b, g, key block j),
 // the (query, slot) pairs whose selection holds j -- a counting sort of the
 // selection by key block:
-//   1. count   cnt[b,g,j] += 1 for every selected entry
+//   1. count   cnt[b,g,j] += 1 for every selected entry; the value before
+//              the increment (the entry's rank among the entries of block
+//              j) is kept in pos_of
 //   2. scan    list_off = exclusive scan of cnt,
 //              item_off = exclusive scan of ceil(cnt / qpi)  (work items of
 //              at most qpi queries, i.e. 128 query-head rows, per block)
-//   3. fill    list[list_off[bgj] + k] = t * 32 + slot  (order inside a
-//              list is arbitrary: each (t, slot) partial is computed
-//              independently of the others in its tile), and the inverse
-//              map pos_of[b,g,t,slot] = that list position, by which the
-//              merge finds a row's partials
+//   3. fill    pos = list_off[bgj] + rank; list[pos] = t * 32 + slot and
+//              pos_of[b,g,t,slot] = pos (the inverse map by which the merge
+//              finds a row's partials).  No atomics: the order inside a list
+//              is whatever order the count's atomics produced, and each
+//              (t, slot) partial is computed independently of the others in
+//              its tile.
 // Every work item then holds <= qpi queries, so items cost the same and a
 // persistent grid balances itself whatever the causal skew between early
 // and late key blocks.
@@ -40,7 +43,7 @@ __global__ void __launch_bounds__(256) revidx_count_kernel(const RevIdxArgs a) {
       atomicCAS(a.status, 0, kStatusBadInput);
       continue;
     }
-    atomicAdd(&a.cnt[bg * a.nb + j], 1);
+    a.pos_of[r * a.top_k + k] = atomicAdd(&a.cnt[bg * a.nb + j], 1);
   }
 }
 
@@ -101,7 +104,6 @@ __global__ void __launch_bounds__(1024) revidx_scan_kernel(const RevIdxArgs a) {
       if (i0 + u < n) {
         a.list_off[i0 + u] = ex;
         a.item_off[i0 + u] = ey;
-        a.cursor[i0 + u] = 0;
       }
       ex += c[u];
       ey += ch[u];
@@ -127,10 +129,10 @@ __global__ void __launch_bounds__(256) revidx_fill_kernel(const RevIdxArgs a) {
     const int t = a.t0 + tl;
     const int j = a.sel[(bg * a.L + t) * a.top_k + k];
     if (j < 0 || j >= a.nb) continue;
-    const long long bgj = bg * a.nb + j;
-    const int pos = a.list_off[bgj] + atomicAdd(&a.cursor[bgj], 1);
+    const long long e_out = r * a.top_k + k;
+    const int pos = a.list_off[bg * a.nb + j] + a.pos_of[e_out];
     a.list[pos] = t * 32 + k;
-    a.pos_of[r * a.top_k + k] = pos;
+    a.pos_of[e_out] = pos;
   }
 }
 

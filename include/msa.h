@@ -172,7 +172,7 @@ size_t msa_workspace_bytes(const msa_params *p, int op);
 
 /* Query-chunk length the prefill attention uses for these params: queries
  * are processed in chunks of this many tokens so that per-block partial
- * results stay within a fixed workspace budget (about 4.5 GiB).  Each chunk
+ * results stay within a fixed workspace budget (about 16 GiB).  Each chunk
  * costs 5 kernel launches.  0 when p is invalid. */
 int msa_prefill_chunk_len(const msa_params *p);
 

@@ -32,8 +32,12 @@ def test_workspace_sizes(L, top_k, G, H, di):
     assert ws_sel >= 4
     # forward = selection buffer + attention workspace
     assert ws_fwd >= ws_att + 4 * L * G * top_k
-    # the partial-result budget bounds the prefill workspace
-    assert ws_att < 6 * 2**30
+    # the partial-result budget (16 GiB) bounds the prefill workspace; the
+    # chunk always holds the partials of whole queries
+    assert ws_att < 17 * 2**30
+    lc = M.msa_prefill_chunk_len(p)
+    assert lc % 128 == 0 and 128 <= lc <= L
+    assert ws_att >= lc * H * top_k * 128 * 2
     assert ws_dec < 64 * 2**20
 
 
