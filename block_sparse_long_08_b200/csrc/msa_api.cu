@@ -9,6 +9,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/msa.h"
 #include "common.cuh"
@@ -57,6 +58,8 @@ int check_params(const msa_params *p, bool decode) {
   if (decode && p->G > 8) return fail(MSA_ERR_UNSUPPORTED, "decode supports G <= 8 (G=%d)", p->G);
   if ((long long)p->B * p->L > (1LL << 26))
     return fail(MSA_ERR_UNSUPPORTED, "B*L=%lld above 2^26", (long long)p->B * p->L);
+  if (p->chunk < 0 || p->chunk % 128 != 0)
+    return fail(MSA_ERR_INVALID_ARG, "chunk=%d must be 0 or a positive multiple of 128", p->chunk);
   return MSA_OK;
 }
 
@@ -78,6 +81,7 @@ int prefill_chunk(const msa_params *p) {
   long long lc = per_q ? (long long)(kPartialBudget / per_q) : p->L;
   lc = (lc / 128) * 128;
   if (lc < 128) lc = 128;
+  if (p->chunk > 0 && p->chunk < lc) lc = p->chunk;
   if (lc > p->L) lc = p->L;
   return (int)lc;
 }
@@ -207,9 +211,18 @@ int run_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 
   return MSA_OK;
 }
 
+// Where a finished query chunk's output rows go next (msa_forward_host):
+// after the chunk's merge, `copy` waits for it and downloads the rows.
+struct ChunkSink {
+  cudaStream_t copy;
+  cudaEvent_t ev;
+  msa_bf16 *out_h;
+  float *lse_h;
+};
+
 int run_prefill_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
                      const msa_bf16 *v, const int32_t *sel, msa_bf16 *out, float *lse, void *ws,
-                     size_t ws_base, cudaStream_t st) {
+                     size_t ws_base, cudaStream_t st, const ChunkSink *sink = nullptr) {
   const int nb = p->L / 128;
   const AttnWs w = attn_ws(p, ws_base);
   uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
@@ -263,7 +276,50 @@ int run_prefill_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
     ca.out = out; ca.lse = lse;
     e = msa::launch_combine(ca, st);
     if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+    if (sink) {
+      e = cudaEventRecord(sink->ev, st);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(sink->copy, sink->ev, 0);
+      if (e != cudaSuccess) return cuda_fail(e, "chunk event");
+      const size_t row = size_t(p->H) * p->d;   // elements of one token's output
+      for (int b = 0; b < p->B && e == cudaSuccess; ++b) {
+        const size_t off = (size_t(b) * p->L + t0) * row;
+        e = cudaMemcpyAsync(sink->out_h + off, out + off, size_t(Lc) * row * 2,
+                            cudaMemcpyDeviceToHost, sink->copy);
+        if (e == cudaSuccess && sink->lse_h) {
+          const size_t lo = (size_t(b) * p->L + t0) * p->H;
+          e = cudaMemcpyAsync(sink->lse_h + lo, lse + lo, size_t(Lc) * p->H * 4,
+                              cudaMemcpyDeviceToHost, sink->copy);
+        }
+      }
+      if (e != cudaSuccess) return cuda_fail(e, "output download");
+    }
   }
+  return MSA_OK;
+}
+
+// Events of msa_forward_host, created once per device.  Each record is
+// followed at once by the wait that consumes it, under the mutex, so reusing
+// one event per role is safe.
+struct HostEvents {
+  cudaEvent_t idx_in = nullptr, all_in = nullptr, chunk = nullptr, done = nullptr;
+};
+constexpr int kMaxDevices = 64;
+std::mutex g_host_mu;
+HostEvents g_host_ev[kMaxDevices];
+
+int host_events(HostEvents **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MSA_ERR_UNSUPPORTED, "device %d", dev);
+  HostEvents &h = g_host_ev[dev];
+  cudaEvent_t *evs[4] = {&h.idx_in, &h.all_in, &h.chunk, &h.done};
+  for (cudaEvent_t *ev : evs) {
+    if (*ev) continue;
+    e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreateWithFlags");
+  }
+  *out = &h;
   return MSA_OK;
 }
 
@@ -371,6 +427,62 @@ int msa_forward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k, const
   rc = run_index_select(p, q_idx, k_idx, s, nullptr, ws, st);
   if (rc) return rc;
   return run_prefill_attn(p, q, k, v, s, out, lse, ws, base, st);
+}
+
+int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k_h,
+                     const msa_bf16 *v_h, const msa_bf16 *q_idx_h, const msa_bf16 *k_idx_h,
+                     msa_bf16 *out_h, float *lse_h, const msa_staging *dev, void *ws,
+                     size_t ws_bytes, msa_stream stream, msa_stream copy_stream) {
+  g_err[0] = 0;
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (p->B == 0 || p->L == 0) return MSA_OK;
+  if (!q_h || !k_h || !v_h || !q_idx_h || !k_idx_h || !out_h || !dev)
+    return fail(MSA_ERR_INVALID_ARG, "NULL host pointer or staging");
+  if (!dev->q || !dev->k || !dev->v || !dev->q_idx || !dev->k_idx || !dev->out ||
+      (lse_h && !dev->lse))
+    return fail(MSA_ERR_INVALID_ARG, "NULL staging pointer");
+  if (!aligned16(dev->q) || !aligned16(dev->k) || !aligned16(dev->v) || !aligned16(dev->q_idx) ||
+      !aligned16(dev->k_idx) || !aligned16(dev->out) || (dev->lse && !aligned16(dev->lse)))
+    return fail(MSA_ERR_INVALID_ARG, "staging pointers must be 16-byte aligned");
+  const size_t base = msa::kWsHeader + forward_sel_bytes(p);
+  rc = check_ws(ws, ws_bytes, attn_ws(p, base).end);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaStream_t cp = reinterpret_cast<cudaStream_t>(copy_stream);
+  const size_t BL = size_t(p->B) * p->L;
+  const size_t n_q = BL * p->H * p->d, n_kv = BL * p->G * p->d;
+  const size_t n_qi = BL * p->G * p->d_idx, n_ki = BL * p->d_idx;
+
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  HostEvents *ev = nullptr;
+  rc = host_events(&ev);
+  if (rc) return rc;
+  // index inputs first; the index branch waits for them only
+  cudaError_t e = cudaMemcpyAsync(dev->q_idx, q_idx_h, n_qi * 2, cudaMemcpyHostToDevice, cp);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dev->k_idx, k_idx_h, n_ki * 2, cudaMemcpyHostToDevice, cp);
+  if (e == cudaSuccess) e = cudaEventRecord(ev->idx_in, cp);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->idx_in, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "index input upload");
+  int32_t *sel = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ws) + msa::kWsHeader);
+  rc = run_index_select(p, dev->q_idx, dev->k_idx, sel, nullptr, ws, st);
+  if (rc) return rc;
+  // the main branch's inputs go up while the index branch runs
+  e = cudaMemcpyAsync(dev->k, k_h, n_kv * 2, cudaMemcpyHostToDevice, cp);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dev->v, v_h, n_kv * 2, cudaMemcpyHostToDevice, cp);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dev->q, q_h, n_q * 2, cudaMemcpyHostToDevice, cp);
+  if (e == cudaSuccess) e = cudaEventRecord(ev->all_in, cp);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->all_in, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "main input upload");
+  const ChunkSink sink{cp, ev->chunk, out_h, lse_h};
+  rc = run_prefill_attn(p, dev->q, dev->k, dev->v, sel, dev->out, lse_h ? dev->lse : nullptr, ws,
+                        base, st, &sink);
+  if (rc) return rc;
+  // later work on `stream` runs after the last download
+  e = cudaEventRecord(ev->done, cp);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->done, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "download completion");
+  return MSA_OK;
 }
 
 int msa_sparse_attn_decode(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,

@@ -43,7 +43,14 @@ class MSAError(RuntimeError):
 class msa_params(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("L", ctypes.c_int32), ("H", ctypes.c_int32),
                 ("G", ctypes.c_int32), ("d", ctypes.c_int32), ("d_idx", ctypes.c_int32),
-                ("block", ctypes.c_int32), ("top_k", ctypes.c_int32), ("scale", ctypes.c_float)]
+                ("block", ctypes.c_int32), ("top_k", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("chunk", ctypes.c_int32)]
+
+
+class msa_staging(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("q_idx", ctypes.c_void_p), ("k_idx", ctypes.c_void_p), ("out", ctypes.c_void_p),
+                ("lse", ctypes.c_void_p)]
 
 
 _lib = None
@@ -64,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.msa_sparse_attn_prefill.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.msa_sparse_attn_decode.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.msa_forward.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.msa_forward_host.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P,
+                                       ctypes.POINTER(msa_staging), _P, _SZ, _P, _P]
         L.msa_sparse_attn_decode_noalloc.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.msa_sparse_attn_decode_noalloc.restype = ctypes.c_int
         L.msa_workspace_bytes.argtypes = [pp, ctypes.c_int]
@@ -74,7 +83,7 @@ def lib() -> ctypes.CDLL:
         L.msa_last_error.restype = ctypes.c_char_p
         L.msa_version.restype = ctypes.c_char_p
         for f in ("msa_index_select", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
-                  "msa_forward", "msa_read_status"):
+                  "msa_forward", "msa_forward_host", "msa_read_status"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -95,9 +104,10 @@ def _check(rc: int):
         raise MSAError(rc, msa_last_error())
 
 
-def make_params(B, L, H, G, d=128, d_idx=128, block=128, top_k=16, scale=0.0) -> msa_params:
+def make_params(B, L, H, G, d=128, d_idx=128, block=128, top_k=16, scale=0.0,
+                chunk=0) -> msa_params:
     return msa_params(int(B), int(L), int(H), int(G), int(d), int(d_idx), int(block), int(top_k),
-                      float(scale))
+                      float(scale), int(chunk))
 
 
 def msa_workspace_bytes(p: msa_params, op: int) -> int:
@@ -164,7 +174,7 @@ def msa_index_select(q_idx: torch.Tensor, k_idx: torch.Tensor, top_k: int, *,
 
 
 def msa_sparse_attn_prefill(q, k, v, sel, *, scale: float = 0.0, want_lse: bool = False,
-                            out=None, ws=None, stream=None):
+                            out=None, ws=None, stream=None, chunk: int = 0):
     """q [B,L,H,d], k/v [B,L,G,d] bf16, sel [B,G,L,top_k] int32 -> out [B,L,H,d]
     (and lse [B,L,H] fp32 when want_lse)."""
     for n, t in (("q", q), ("k", k), ("v", v)):
@@ -173,7 +183,7 @@ def msa_sparse_attn_prefill(q, k, v, sel, *, scale: float = 0.0, want_lse: bool 
     B, L, H, d = q.shape
     G = k.shape[2]
     top_k = sel.shape[3]
-    p = make_params(B, L, H, G, d, 128, 128, top_k, scale)
+    p = make_params(B, L, H, G, d, 128, 128, top_k, scale, chunk)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
@@ -185,14 +195,14 @@ def msa_sparse_attn_prefill(q, k, v, sel, *, scale: float = 0.0, want_lse: bool 
 
 
 def msa_forward(q, k, v, q_idx, k_idx, top_k: int, *, scale: float = 0.0, want_sel: bool = False,
-                want_lse: bool = False, out=None, sel=None, ws=None, stream=None):
+                want_lse: bool = False, out=None, sel=None, ws=None, stream=None, chunk: int = 0):
     """Whole prefill: index branch with fused top-k, then the sparse main branch."""
     for n, t in (("q", q), ("k", k), ("v", v), ("q_idx", q_idx), ("k_idx", k_idx)):
         _req(t, n, torch.bfloat16)
     B, L, H, d = q.shape
     G = k.shape[2]
     di = q_idx.shape[3]
-    p = make_params(B, L, H, G, d, di, 128, top_k, scale)
+    p = make_params(B, L, H, G, d, di, 128, top_k, scale, chunk)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
@@ -208,6 +218,53 @@ def msa_forward(q, k, v, q_idx, k_idx, top_k: int, *, scale: float = 0.0, want_s
     if want_lse:
         res.append(lse)
     return res[0] if len(res) == 1 else tuple(res)
+
+
+def _req_host(t: torch.Tensor, name: str, dtype) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def msa_forward_host(q, k, v, q_idx, k_idx, top_k: int, *, out, lse=None, staging=None,
+                     scale: float = 0.0, ws=None, stream=None, copy_stream=None, chunk: int = 0,
+                     device=None):
+    """msa_forward on HOST tensors (pinned for overlap): q [B,L,H,d], k/v [B,L,G,d],
+    q_idx [B,L,G,d_idx], k_idx [B,L,d_idx] bf16 in; out [B,L,H,d] bf16 (and lse
+    [B,L,H] fp32) host tensors filled.  `staging` holds the device buffers
+    (dict with q, k, v, q_idx, k_idx, out and, with lse, lse); created when
+    None.  Transfers run on copy_stream (default: a new stream) overlapped
+    with the computation on `stream`; synchronise `stream` before reading out."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("q_idx", q_idx), ("k_idx", k_idx), ("out", out)):
+        _req_host(t, n, torch.bfloat16)
+    if lse is not None:
+        _req_host(lse, "lse", torch.float32)
+    B, L, H, d = q.shape
+    G = k.shape[2]
+    di = q_idx.shape[3]
+    p = make_params(B, L, H, G, d, di, 128, top_k, scale, chunk)
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    if staging is None:
+        staging = {n: torch.empty(t.shape, dtype=t.dtype, device=dev)
+                   for n, t in (("q", q), ("k", k), ("v", v), ("q_idx", q_idx), ("k_idx", k_idx),
+                                ("out", out))}
+        if lse is not None:
+            staging["lse"] = torch.empty(lse.shape, dtype=torch.float32, device=dev)
+    for n in ("q", "k", "v", "q_idx", "k_idx", "out"):
+        _req(staging[n], "staging " + n, torch.bfloat16)
+    st = msa_staging(*(staging[n].data_ptr() for n in ("q", "k", "v", "q_idx", "k_idx", "out")),
+                     staging["lse"].data_ptr() if lse is not None else None)
+    ws = _ensure_ws(ws, p, MSA_OP_FORWARD, dev)
+    if copy_stream is None:
+        copy_stream = torch.cuda.Stream(device=dev)
+    _check(lib().msa_forward_host(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_idx),
+                                  _ptr(k_idx), _ptr(out), _ptr(lse), ctypes.byref(st), _ptr(ws),
+                                  ws.numel(), _stream(stream), _stream(copy_stream)))
+    return (out, lse) if lse is not None else out
 
 
 def msa_sparse_attn_decode(q, q_idx, k_cache, v_cache, k_idx_cache, seq_lens, top_k: int, *,

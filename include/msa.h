@@ -72,6 +72,10 @@ typedef struct msa_params {
   int32_t block;   /* KV block length (128) */
   int32_t top_k;   /* blocks kept per (query, group), local block included */
   float scale;     /* softmax scale of the main branch; 0 -> 1/sqrt(d) */
+  int32_t chunk;   /* prefill query-chunk length, a multiple of 128; 0 -> the
+                      longest chunk whose partials fit the 16 GiB budget.
+                      Smaller chunks need a smaller workspace and re-read
+                      K/V more often. */
 } msa_params;
 
 enum {
@@ -165,6 +169,39 @@ int msa_sparse_attn_decode_noalloc(const msa_params *p, const msa_bf16 *q, const
 int msa_forward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k, const msa_bf16 *v,
                 const msa_bf16 *q_idx, const msa_bf16 *k_idx, msa_bf16 *out, int32_t *sel,
                 float *lse, void *ws, size_t ws_bytes, msa_stream stream);
+
+/* Device buffers that msa_forward_host stages its transfers in: the device
+ * counterparts of msa_forward's tensors (caller-owned, 16-byte aligned).
+ * lse may be NULL when no lse is requested. */
+typedef struct msa_staging {
+  msa_bf16 *q, *k, *v, *q_idx, *k_idx;   /* inputs, device copies   */
+  msa_bf16 *out;                          /* [B,L,H,d] device output */
+  float *lse;                             /* [B,L,H] or NULL         */
+} msa_staging;
+
+/* msa_forward with inputs and outputs in HOST memory, transfers overlapped
+ * with the computation.  There is no counterpart in the pages; this is the
+ * end-to-end path of a caller whose tensors live in host memory.
+ *   q_h, k_h, v_h, q_idx_h, k_idx_h  host inputs, layouts of msa_forward (in)
+ *   out_h [B,L,H,d] bf16, lse_h [B,L,H] fp32 or NULL: host outputs      (out)
+ *   dev       device staging buffers (dev->lse needed iff lse_h)
+ *   ws        as msa_forward (msa_workspace_bytes(p, MSA_OP_FORWARD))
+ *   stream    compute stream;  copy_stream  the transfers (may equal stream,
+ *             which serialises them with the computation)
+ * Order of work: q_idx and k_idx go up first; q, k and v go up on
+ * copy_stream while the index branch runs on stream; each query chunk's
+ * output rows (and lse) come down on copy_stream as soon as the chunk is
+ * merged, while the next chunk computes.  When the call returns everything
+ * is enqueued, and work later enqueued on `stream` runs after the last
+ * download, so synchronising `stream` makes out_h valid.  Host buffers must
+ * be pinned (page-locked) for the copies to overlap; pageable buffers still
+ * give correct results.  Uses four CUDA events per device, created on the
+ * first call on that device and reused; calls from several host threads are
+ * serialised while they enqueue. */
+int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k_h,
+                     const msa_bf16 *v_h, const msa_bf16 *q_idx_h, const msa_bf16 *k_idx_h,
+                     msa_bf16 *out_h, float *lse_h, const msa_staging *dev, void *ws,
+                     size_t ws_bytes, msa_stream stream, msa_stream copy_stream);
 
 /* Workspace bytes op (MSA_OP_*) needs for these params; 0 when p is invalid
  * (see msa_last_error). */

@@ -46,7 +46,8 @@ def test_workspace_sizes(L, top_k, G, H, di):
     ("block", 64, M.MSA_ERR_UNSUPPORTED), ("top_k", 33, M.MSA_ERR_UNSUPPORTED),
     ("top_k", 0, M.MSA_ERR_INVALID_ARG), ("L", 1000, M.MSA_ERR_UNSUPPORTED),
     ("H", 12, M.MSA_ERR_UNSUPPORTED), ("G", 3, M.MSA_ERR_INVALID_ARG),
-    ("B", -1, M.MSA_ERR_INVALID_ARG)])
+    ("B", -1, M.MSA_ERR_INVALID_ARG), ("chunk", 100, M.MSA_ERR_INVALID_ARG),
+    ("chunk", -128, M.MSA_ERR_INVALID_ARG)])
 def test_bad_params_rejected_before_launch(field, value, code):
     p = M.make_params(1, 2048, 8, 2, 128, 64, 128, 4)
     setattr(p, field, value)
@@ -79,6 +80,39 @@ def test_empty_problem_is_noop():
     p = M.make_params(1, 0, 8, 2, 128, 64, 128, 4)
     assert lib.msa_forward(ctypes.byref(p), None, None, None, None, None, None, None, None, None, 0,
                            None) == M.MSA_OK
+
+
+def test_chunk_length_follows_params():
+    p = M.make_params(2, 8192, 32, 8, 128, 128, 128, 16)
+    full = M.msa_prefill_chunk_len(p)
+    assert full == 8192                       # small problems run as one chunk
+    for c, want in ((1024, 1024), (128, 128), (16384, 8192)):
+        p.chunk = c
+        assert M.msa_prefill_chunk_len(p) == want
+    # a shorter chunk needs a smaller prefill workspace
+    p.chunk = 1024
+    small = M.msa_workspace_bytes(p, M.MSA_OP_PREFILL_ATTN)
+    p.chunk = 0
+    assert small < M.msa_workspace_bytes(p, M.MSA_OP_PREFILL_ATTN)
+
+
+def test_forward_host_rejects_bad_arguments():
+    p = M.make_params(1, 2048, 8, 2, 128, 64, 128, 4)
+    lib = M.lib()
+    h = ctypes.c_void_p(4096)
+    st = M.msa_staging(4096, 4096, 4096, 4096, 4096, 4096, None)
+    rc = lib.msa_forward_host(ctypes.byref(p), h, h, h, h, h, h, None, None, h, 1 << 30, None, None)
+    assert rc == M.MSA_ERR_INVALID_ARG          # no staging buffers
+    bad = M.msa_staging(4096 + 8, 4096, 4096, 4096, 4096, 4096, None)
+    rc = lib.msa_forward_host(ctypes.byref(p), h, h, h, h, h, h, None, ctypes.byref(bad), h,
+                              1 << 30, None, None)
+    assert rc == M.MSA_ERR_INVALID_ARG          # misaligned staging
+    rc = lib.msa_forward_host(ctypes.byref(p), h, h, h, h, h, h, h, ctypes.byref(st), h, 1 << 30,
+                              None, None)
+    assert rc == M.MSA_ERR_INVALID_ARG          # lse requested without device lse
+    rc = lib.msa_forward_host(ctypes.byref(p), h, h, h, h, h, h, None, ctypes.byref(st), h, 64,
+                              None, None)
+    assert rc == M.MSA_ERR_WORKSPACE
 
 
 def test_decode_rejects_more_than_eight_groups():
