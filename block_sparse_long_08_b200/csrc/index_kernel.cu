@@ -86,7 +86,7 @@ struct IndexWork {
 __device__ __forceinline__ IndexWork index_work(const IndexArgs &a, int u, int GPn) {
   const int ngp = a.G / GPn;
   IndexWork w;
-  w.i = a.nb - 1 - u / (a.B * ngp);
+  w.i = a.i_hi - 1 - u / (a.B * ngp);
   const int rem = u % (a.B * ngp);
   w.b = rem / ngp;
   w.gp = rem % ngp;

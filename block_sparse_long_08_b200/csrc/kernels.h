@@ -11,7 +11,8 @@ namespace msa {
 struct IndexArgs {
   int B, L, G, nb, top_k, d_idx;
   int write_scores;  // 1: store block scores, 0: fused top-k -> sel
-  int n_items;       // B * nb * (G / groups_per_cta)
+  int i_hi;          // query tiles [i_hi - n_items / (B * G/groups_per_cta), i_hi)
+  int n_items;       // B * (query tiles) * (G / groups_per_cta)
   int32_t *sel;      // [B,G,L,top_k]
   float *scores;     // [B,G,L,nb]
   int *status;

@@ -173,9 +173,13 @@ int num_sms() {
 int *status_ptr(void *ws) { return reinterpret_cast<int *>(ws); }
 
 // ---- the operations --------------------------------------------------------
+// Index branch for the query tiles of tokens [t_lo, t_hi) (multiples of 128;
+// the whole sequence by default).
 int run_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 *k_idx,
-                     int32_t *sel, float *block_scores, void *ws, cudaStream_t st) {
+                     int32_t *sel, float *block_scores, void *ws, cudaStream_t st, int t_lo = 0,
+                     int t_hi = -1) {
   const int nb = p->L / 128;
+  if (t_hi < 0) t_hi = p->L;
   CUtensorMap tq, tk;
   {
     const uint64_t dims[3] = {uint64_t(p->d_idx), uint64_t(p->G), uint64_t(p->B) * p->L};
@@ -194,7 +198,8 @@ int run_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 
   msa::IndexArgs a;
   a.B = p->B; a.L = p->L; a.G = p->G; a.nb = nb; a.top_k = p->top_k; a.d_idx = p->d_idx;
   a.write_scores = block_scores ? 1 : 0;
-  a.n_items = p->B * nb * (p->G / msa::index_groups_per_cta(p->G, p->top_k));
+  a.i_hi = t_hi / 128;
+  a.n_items = p->B * (t_hi / 128 - t_lo / 128) * (p->G / msa::index_groups_per_cta(p->G, p->top_k));
   a.sel = sel;
   a.scores = block_scores;
   a.status = status_ptr(ws);
@@ -220,88 +225,114 @@ struct ChunkSink {
   float *lse_h;
 };
 
-int run_prefill_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
-                     const msa_bf16 *v, const int32_t *sel, msa_bf16 *out, float *lse, void *ws,
-                     size_t ws_base, cudaStream_t st, const ChunkSink *sink = nullptr) {
-  const int nb = p->L / 128;
-  const AttnWs w = attn_ws(p, ws_base);
-  uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
+// Tensor maps and workspace layout shared by the query chunks of one call.
+struct AttnPlan {
   CUtensorMap tk, tv;
+  AttnWs w;
+  int nb, qpi, sms;
+  float scale;
+};
+
+int plan_attn(const msa_params *p, const msa_bf16 *k, const msa_bf16 *v, size_t ws_base,
+              AttnPlan *pl) {
+  pl->nb = p->L / 128;
+  pl->w = attn_ws(p, ws_base);
   const uint64_t dims[3] = {uint64_t(p->d), uint64_t(p->G), uint64_t(p->B) * p->L};
   const uint64_t str[2] = {uint64_t(p->d) * 2, uint64_t(p->d) * 2 * p->G};
   const uint32_t box[3] = {64, 1, 128};
-  int rc = make_tmap(&tk, k, 3, dims, str, box);
+  int rc = make_tmap(&pl->tk, k, 3, dims, str, box);
   if (rc) return rc;
-  rc = make_tmap(&tv, v, 3, dims, str, box);
+  rc = make_tmap(&pl->tv, v, 3, dims, str, box);
   if (rc) return rc;
-  const int r = p->H / p->G;
-  const int qpi = 128 / r;
-  const float scale = eff_scale(p);
-  const int sms = num_sms();
-  for (int t0 = 0; t0 < p->L; t0 += w.Lc) {
-    const int Lc = (p->L - t0) < w.Lc ? (p->L - t0) : w.Lc;
-    msa::RevIdxArgs ra;
-    ra.B = p->B; ra.G = p->G; ra.L = p->L; ra.nb = nb; ra.top_k = p->top_k; ra.qpi = qpi;
-    ra.t0 = t0; ra.Lc = Lc;
-    ra.sel = sel;
-    ra.cnt = reinterpret_cast<int32_t *>(wsb + w.cnt);
-    ra.list_off = reinterpret_cast<int32_t *>(wsb + w.list_off);
-    ra.item_off = reinterpret_cast<int32_t *>(wsb + w.item_off);
-    ra.list = reinterpret_cast<int32_t *>(wsb + w.list);
-    ra.pos_of = reinterpret_cast<int32_t *>(wsb + w.pos_of);
-    ra.status = status_ptr(ws);
-    cudaError_t e = msa::launch_revidx(ra, st);
-    if (e != cudaSuccess) return cuda_fail(e, "reverse index launch");
-    msa::AttnArgs aa;
-    aa.B = p->B; aa.L = p->L; aa.H = p->H; aa.G = p->G; aa.nb = nb; aa.top_k = p->top_k;
-    aa.scale = scale;
-    aa.scale_log2 = scale * 1.4426950408889634f;
-    aa.t0 = t0; aa.Lc = Lc;
-    const long long max_items =
-        (long long)p->B * p->G * Lc * p->top_k / qpi + (long long)p->B * p->G * nb;
-    aa.max_items = (int)max_items;
-    aa.q = q;
-    aa.list = ra.list; aa.list_off = ra.list_off; aa.item_off = ra.item_off;
-    aa.part_o = reinterpret_cast<uint16_t *>(wsb + w.part_o);
-    aa.part_lse = reinterpret_cast<float *>(wsb + w.part_lse);
-    aa.status = status_ptr(ws);
-    e = msa::launch_prefill_attn(tk, tv, aa, sms, st);
-    if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
-    msa::CombineArgs ca;
-    ca.B = p->B; ca.L = p->L; ca.H = p->H; ca.G = p->G; ca.top_k = p->top_k;
-    ca.t0 = t0; ca.Lc = Lc;
-    ca.sel = sel;
-    ca.pos_of = ra.pos_of;
-    ca.part_o = aa.part_o; ca.part_lse = aa.part_lse;
-    ca.out = out; ca.lse = lse;
-    e = msa::launch_combine(ca, st);
-    if (e != cudaSuccess) return cuda_fail(e, "combine launch");
-    if (sink) {
-      e = cudaEventRecord(sink->ev, st);
-      if (e == cudaSuccess) e = cudaStreamWaitEvent(sink->copy, sink->ev, 0);
-      if (e != cudaSuccess) return cuda_fail(e, "chunk event");
-      const size_t row = size_t(p->H) * p->d;   // elements of one token's output
-      for (int b = 0; b < p->B && e == cudaSuccess; ++b) {
-        const size_t off = (size_t(b) * p->L + t0) * row;
-        e = cudaMemcpyAsync(sink->out_h + off, out + off, size_t(Lc) * row * 2,
+  pl->qpi = 128 / (p->H / p->G);
+  pl->scale = eff_scale(p);
+  pl->sms = num_sms();
+  return MSA_OK;
+}
+
+// One query chunk [t0, t0 + Lc): reverse index, attention, merge; then,
+// with a sink, the download of the chunk's output rows.
+int run_attn_chunk(const msa_params *p, const AttnPlan &pl, const msa_bf16 *q, const int32_t *sel,
+                   msa_bf16 *out, float *lse, void *ws, int t0, int Lc, cudaStream_t st,
+                   const ChunkSink *sink) {
+  uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
+  const AttnWs &w = pl.w;
+  msa::RevIdxArgs ra;
+  ra.B = p->B; ra.G = p->G; ra.L = p->L; ra.nb = pl.nb; ra.top_k = p->top_k; ra.qpi = pl.qpi;
+  ra.t0 = t0; ra.Lc = Lc;
+  ra.sel = sel;
+  ra.cnt = reinterpret_cast<int32_t *>(wsb + w.cnt);
+  ra.list_off = reinterpret_cast<int32_t *>(wsb + w.list_off);
+  ra.item_off = reinterpret_cast<int32_t *>(wsb + w.item_off);
+  ra.list = reinterpret_cast<int32_t *>(wsb + w.list);
+  ra.pos_of = reinterpret_cast<int32_t *>(wsb + w.pos_of);
+  ra.status = status_ptr(ws);
+  cudaError_t e = msa::launch_revidx(ra, st);
+  if (e != cudaSuccess) return cuda_fail(e, "reverse index launch");
+  msa::AttnArgs aa;
+  aa.B = p->B; aa.L = p->L; aa.H = p->H; aa.G = p->G; aa.nb = pl.nb; aa.top_k = p->top_k;
+  aa.scale = pl.scale;
+  aa.scale_log2 = pl.scale * 1.4426950408889634f;
+  aa.t0 = t0; aa.Lc = Lc;
+  const long long max_items =
+      (long long)p->B * p->G * Lc * p->top_k / pl.qpi + (long long)p->B * p->G * pl.nb;
+  aa.max_items = (int)max_items;
+  aa.q = q;
+  aa.list = ra.list; aa.list_off = ra.list_off; aa.item_off = ra.item_off;
+  aa.part_o = reinterpret_cast<uint16_t *>(wsb + w.part_o);
+  aa.part_lse = reinterpret_cast<float *>(wsb + w.part_lse);
+  aa.status = status_ptr(ws);
+  e = msa::launch_prefill_attn(pl.tk, pl.tv, aa, pl.sms, st);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
+  msa::CombineArgs ca;
+  ca.B = p->B; ca.L = p->L; ca.H = p->H; ca.G = p->G; ca.top_k = p->top_k;
+  ca.t0 = t0; ca.Lc = Lc;
+  ca.sel = sel;
+  ca.pos_of = ra.pos_of;
+  ca.part_o = aa.part_o; ca.part_lse = aa.part_lse;
+  ca.out = out; ca.lse = lse;
+  e = msa::launch_combine(ca, st);
+  if (e != cudaSuccess) return cuda_fail(e, "combine launch");
+  if (sink) {
+    e = cudaEventRecord(sink->ev, st);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(sink->copy, sink->ev, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "chunk event");
+    const size_t row = size_t(p->H) * p->d;   // elements of one token's output
+    for (int b = 0; b < p->B && e == cudaSuccess; ++b) {
+      const size_t off = (size_t(b) * p->L + t0) * row;
+      e = cudaMemcpyAsync(sink->out_h + off, out + off, size_t(Lc) * row * 2,
+                          cudaMemcpyDeviceToHost, sink->copy);
+      if (e == cudaSuccess && sink->lse_h) {
+        const size_t lo = (size_t(b) * p->L + t0) * p->H;
+        e = cudaMemcpyAsync(sink->lse_h + lo, lse + lo, size_t(Lc) * p->H * 4,
                             cudaMemcpyDeviceToHost, sink->copy);
-        if (e == cudaSuccess && sink->lse_h) {
-          const size_t lo = (size_t(b) * p->L + t0) * p->H;
-          e = cudaMemcpyAsync(sink->lse_h + lo, lse + lo, size_t(Lc) * p->H * 4,
-                              cudaMemcpyDeviceToHost, sink->copy);
-        }
       }
-      if (e != cudaSuccess) return cuda_fail(e, "output download");
     }
+    if (e != cudaSuccess) return cuda_fail(e, "output download");
   }
   return MSA_OK;
 }
 
-// Events of msa_forward_host, created once per device.  Each record is
-// followed at once by the wait that consumes it, under the mutex, so reusing
-// one event per role is safe.
+int run_prefill_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
+                     const msa_bf16 *v, const int32_t *sel, msa_bf16 *out, float *lse, void *ws,
+                     size_t ws_base, cudaStream_t st) {
+  AttnPlan pl;
+  int rc = plan_attn(p, k, v, ws_base, &pl);
+  if (rc) return rc;
+  for (int t0 = 0; t0 < p->L; t0 += pl.w.Lc) {
+    const int Lc = (p->L - t0) < pl.w.Lc ? (p->L - t0) : pl.w.Lc;
+    rc = run_attn_chunk(p, pl, q, sel, out, lse, ws, t0, Lc, st, nullptr);
+    if (rc) return rc;
+  }
+  return MSA_OK;
+}
+
+// Events and download stream of msa_forward_host, created once per device.
+// Each record is followed at once by the wait that consumes it, under the
+// mutex, so reusing one event per role is safe.
 struct HostEvents {
   cudaEvent_t idx_in = nullptr, all_in = nullptr, chunk = nullptr, done = nullptr;
+  cudaStream_t down = nullptr;   // output downloads (the other PCIe direction)
 };
 constexpr int kMaxDevices = 64;
 std::mutex g_host_mu;
@@ -318,6 +349,10 @@ int host_events(HostEvents **out) {
     if (*ev) continue;
     e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
     if (e != cudaSuccess) return cuda_fail(e, "cudaEventCreateWithFlags");
+  }
+  if (!h.down) {
+    e = cudaStreamCreateWithFlags(&h.down, cudaStreamNonBlocking);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamCreateWithFlags");
   }
   *out = &h;
   return MSA_OK;
@@ -450,36 +485,51 @@ int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k
   if (rc) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaStream_t cp = reinterpret_cast<cudaStream_t>(copy_stream);
-  const size_t BL = size_t(p->B) * p->L;
-  const size_t n_q = BL * p->H * p->d, n_kv = BL * p->G * p->d;
-  const size_t n_qi = BL * p->G * p->d_idx, n_ki = BL * p->d_idx;
 
   std::lock_guard<std::mutex> lock(g_host_mu);
   HostEvents *ev = nullptr;
   rc = host_events(&ev);
   if (rc) return rc;
-  // index inputs first; the index branch waits for them only
-  cudaError_t e = cudaMemcpyAsync(dev->q_idx, q_idx_h, n_qi * 2, cudaMemcpyHostToDevice, cp);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dev->k_idx, k_idx_h, n_ki * 2, cudaMemcpyHostToDevice, cp);
-  if (e == cudaSuccess) e = cudaEventRecord(ev->idx_in, cp);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->idx_in, 0);
-  if (e != cudaSuccess) return cuda_fail(e, "index input upload");
+  AttnPlan pl;
+  rc = plan_attn(p, dev->k, dev->v, base, &pl);
+  if (rc) return rc;
   int32_t *sel = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ws) + msa::kWsHeader);
-  rc = run_index_select(p, dev->q_idx, dev->k_idx, sel, nullptr, ws, st);
-  if (rc) return rc;
-  // the main branch's inputs go up while the index branch runs
-  e = cudaMemcpyAsync(dev->k, k_h, n_kv * 2, cudaMemcpyHostToDevice, cp);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dev->v, v_h, n_kv * 2, cudaMemcpyHostToDevice, cp);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dev->q, q_h, n_q * 2, cudaMemcpyHostToDevice, cp);
-  if (e == cudaSuccess) e = cudaEventRecord(ev->all_in, cp);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->all_in, 0);
-  if (e != cudaSuccess) return cuda_fail(e, "main input upload");
-  const ChunkSink sink{cp, ev->chunk, out_h, lse_h};
-  rc = run_prefill_attn(p, dev->q, dev->k, dev->v, sel, dev->out, lse_h ? dev->lse : nullptr, ws,
-                        base, st, &sink);
-  if (rc) return rc;
+  const ChunkSink sink{ev->down, ev->chunk, out_h, lse_h};
+  // Per query chunk [t0, t0+Lc): upload the chunk's rows (index inputs
+  // first), run the index branch for the chunk's query tiles and the main
+  // branch for its queries, download its output.  A chunk only needs rows
+  // < t0 + Lc, so uploads, computation and downloads of neighbouring chunks
+  // overlap; uploads run ahead on copy_stream, downloads on the library's
+  // download stream.
+  for (int t0 = 0; t0 < p->L; t0 += pl.w.Lc) {
+    const int Lc = (p->L - t0) < pl.w.Lc ? (p->L - t0) : pl.w.Lc;
+    cudaError_t e = cudaSuccess;
+    auto up = [&](msa_bf16 *d, const msa_bf16 *h, size_t row) {   // rows [t0, t0+Lc) of each b
+      for (int b = 0; b < p->B && e == cudaSuccess; ++b) {
+        const size_t off = (size_t(b) * p->L + t0) * row;
+        e = cudaMemcpyAsync(d + off, h + off, size_t(Lc) * row * 2, cudaMemcpyHostToDevice, cp);
+      }
+    };
+    up(dev->k_idx, k_idx_h, size_t(p->d_idx));
+    up(dev->q_idx, q_idx_h, size_t(p->G) * p->d_idx);
+    if (e == cudaSuccess) e = cudaEventRecord(ev->idx_in, cp);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->idx_in, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "index input upload");
+    rc = run_index_select(p, dev->q_idx, dev->k_idx, sel, nullptr, ws, st, t0, t0 + Lc);
+    if (rc) return rc;
+    up(dev->k, k_h, size_t(p->G) * p->d);
+    up(dev->v, v_h, size_t(p->G) * p->d);
+    up(dev->q, q_h, size_t(p->H) * p->d);
+    if (e == cudaSuccess) e = cudaEventRecord(ev->all_in, cp);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->all_in, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "main input upload");
+    rc = run_attn_chunk(p, pl, dev->q, sel, dev->out, lse_h ? dev->lse : nullptr, ws, t0, Lc, st,
+                        &sink);
+    if (rc) return rc;
+  }
+  cudaError_t e = cudaSuccess;
   // later work on `stream` runs after the last download
-  e = cudaEventRecord(ev->done, cp);
+  e = cudaEventRecord(ev->done, ev->down);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->done, 0);
   if (e != cudaSuccess) return cuda_fail(e, "download completion");
   return MSA_OK;

@@ -188,16 +188,20 @@ typedef struct msa_staging {
  *   ws        as msa_forward (msa_workspace_bytes(p, MSA_OP_FORWARD))
  *   stream    compute stream;  copy_stream  the transfers (may equal stream,
  *             which serialises them with the computation)
- * Order of work: q_idx and k_idx go up first; q, k and v go up on
- * copy_stream while the index branch runs on stream; each query chunk's
- * output rows (and lse) come down on copy_stream as soon as the chunk is
- * merged, while the next chunk computes.  When the call returns everything
- * is enqueued, and work later enqueued on `stream` runs after the last
- * download, so synchronising `stream` makes out_h valid.  Host buffers must
- * be pinned (page-locked) for the copies to overlap; pageable buffers still
- * give correct results.  Uses four CUDA events per device, created on the
- * first call on that device and reused; calls from several host threads are
- * serialised while they enqueue. */
+ * Order of work, per query chunk [t0, t0+Lc) (msa_prefill_chunk_len): the
+ * chunk's rows of k_idx and q_idx go up on copy_stream, then its rows of k,
+ * v and q; on `stream` the index branch runs for the chunk's query tiles as
+ * soon as its index rows are up, then the main branch for its queries; the
+ * chunk's output rows (and lse) come down on a download stream of the
+ * library as soon as the chunk is merged.  A chunk needs only rows < t0+Lc,
+ * so transfers and computation of neighbouring chunks overlap.  When the
+ * call returns everything is enqueued, and work later enqueued on `stream`
+ * runs after the last download, so synchronising `stream` makes out_h
+ * valid.  Host buffers must be pinned (page-locked) for the copies to
+ * overlap; pageable buffers still give correct results.  Uses four CUDA
+ * events and one stream per device, created on the first call on that
+ * device and reused; calls from several host threads are serialised while
+ * they enqueue. */
 int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k_h,
                      const msa_bf16 *v_h, const msa_bf16 *q_idx_h, const msa_bf16 *k_idx_h,
                      msa_bf16 *out_h, float *lse_h, const msa_staging *dev, void *ws,
