@@ -266,8 +266,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="1m", choices=["1m", "128k", "32k"],
                     help="prefill length of the step (1m is the headline workload)")
-    ap.add_argument("--op", default="step", choices=["step", "index", "attn", "decode"],
-                    help="time one operation of the step alone (profiling runs); "
+    ap.add_argument("--op", default="step", choices=["step", "index", "attn", "decode", "cached"],
+                    help="time one operation of the step alone (profiling runs; 'cached' runs "
+                         "the whole prefill as 8 msa_forward_cached chunks against the caches); "
                          "prints its own short JSON line")
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="override the decode batch (profiling runs on a smaller footprint)")
@@ -340,7 +341,7 @@ def run_ours(args, shape, dshape, seed, cfg, ws_n, rank, local):
     peaks = load_peaks()
 
     # ---- inputs (device-resident for the kernel-timed leg)
-    need_pre = args.op in ("step", "index", "attn")
+    need_pre = args.op in ("step", "index", "attn", "cached")
     need_dec = args.op in ("step", "decode")
     if not need_pre:   # a decode-only profiling run keeps the footprint small
         import dataclasses
@@ -473,8 +474,23 @@ def run_single_op(args, M, x, dx, dshape, K, sel, out, dout, ws_idx, ws_att, ws_
     """One operation alone, W untimed + K timed launches (profiling aid)."""
     M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx)  # the attention op needs sel
 
+    L = x["q"].shape[1]
+    n_c = L // 8
+    qc = [(x["q"][:, t0:t0 + n_c].contiguous(), x["q_idx"][:, t0:t0 + n_c].contiguous())
+          for t0 in range(0, L, n_c)] if args.op == "cached" else []
+    outc = torch.empty_like(qc[0][0]) if qc else None
+    ws_c = None
+    if qc:
+        pc = M.make_params(x["q"].shape[0], L, x["q"].shape[2], x["k"].shape[2], 128,
+                           x["q_idx"].shape[3], 128, K)
+        ws_c = M.new_workspace(pc, M.MSA_OP_FORWARD, x["q"].device)
+
     def op():
-        if args.op == "index":
+        if args.op == "cached":   # the prefill as the serving form: 8 chunks against the caches
+            for c, (q, q_idx) in enumerate(qc):
+                M.msa_forward_cached(q, q_idx, x["k"], x["v"], x["k_idx"], c * n_c, K, out=outc,
+                                     ws=ws_c)
+        elif args.op == "index":
             M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx)
         elif args.op == "attn":
             M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att)
@@ -492,11 +508,15 @@ def run_single_op(args, M, x, dx, dshape, K, sel, out, dout, ws_idx, ws_att, ws_
         op()
     b.record(stream)
     torch.cuda.synchronize()
-    for w in (ws_idx, ws_att, ws_dec):
+    for w in (ws_idx, ws_att, ws_dec) + ((ws_c,) if ws_c is not None else ()):
         if M.msa_read_status(w) != 0:
             raise SystemExit("device status error")
-    print(json.dumps({"op": args.op, "workload": args.workload,
-                      "ms_per_launch": a.elapsed_time(b) / args.steps}), flush=True)
+    ms = a.elapsed_time(b) / args.steps
+    line = {"op": args.op, "workload": args.workload, "ms_per_launch": ms}
+    if args.op == "cached":
+        line["tokens_per_s"] = L * x["q"].shape[0] / (ms / 1e3)
+        line["chunks"] = len(qc)
+    print(json.dumps(line), flush=True)
 
 
 def bench_decode_128k(M, I, dev, args, peaks):

@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(384, 1)
         for (int gi = 0; gi < GP; ++gi)
           for (int c = 0; c < C::NCH; ++c)
             tma_load_3d(s_q + (gi * C::NCH + c) * 16384, &tm_q, b_qfull, c * 64, w.gp * GP + gi,
-                        w.b * a.L + w.i * kBlock);
+                        w.b * a.Lq + w.i * kBlock - a.tq0);
         bool ok = true;
         for (int s = 0; s < w.stages; ++s) {
           if (!mbar_wait(b_kempty + 8 * kst, kph ^ 1, abort_flag, a.status)) { ok = false; break; }
@@ -372,7 +372,7 @@ __global__ void __launch_bounds__(384, 1)
             const float sc = max4x32(v0, v1, v2, v3);
             if (a.write_scores) {
               const int g = w.gp * GP + gi;
-              a.scores[((size_t(w.b) * a.G + g) * a.L + t) * a.nb + j] = sc;
+              a.scores[((size_t(w.b) * a.G + g) * a.Lq + (t - a.tq0)) * a.nb + j] = sc;
             } else if (sc > ls[gi][KCAP - 1]) {
               list_insert_tail<KCAP>(ls[gi], lj[gi], sc, j);
             }
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int gi = 0; gi < GP; ++gi) {
             const int g = w.gp * GP + gi;
-            float *dst = a.scores + ((size_t(w.b) * a.G + g) * a.L + t) * a.nb;
+            float *dst = a.scores + ((size_t(w.b) * a.G + g) * a.Lq + (t - a.tq0)) * a.nb;
             for (int j = w.i; j < a.nb; ++j) dst[j] = -INFINITY;
           }
         }
@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int gi = 0; gi < GP; ++gi) {
             const int g = w.gp * GP + gi;
-            int32_t *dst = a.sel + ((size_t(w.b) * a.G + g) * a.L + t) * a.top_k;
+            int32_t *dst = a.sel + ((size_t(w.b) * a.G + g) * a.Lq + (t - a.tq0)) * a.top_k;
             for (int k = 0; k < a.top_k; ++k) dst[k] = (k <= w.i) ? k : -1;
           }
         }
@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(384, 1)
             if (id >= 0 && id != INT_MAX) list_insert<KCAP>(ls[gi], lj[gi], sc, id);
           }
           const int g = w.gp * GP + gi;
-          int32_t *dst = a.sel + ((size_t(w.b) * a.G + g) * a.L + t) * a.top_k;
+          int32_t *dst = a.sel + ((size_t(w.b) * a.G + g) * a.Lq + (t - a.tq0)) * a.top_k;
           int ids[KCAP];
 #pragma unroll
           for (int k = 0; k < KCAP; ++k) ids[k] = (k >= n_sent) ? lj[gi][k] : INT_MAX;

@@ -8,8 +8,13 @@
 
 namespace msa {
 
+// Query-side tensors (q, q_idx, sel, scores, out, lse) hold Lq rows per
+// sequence, row 0 being position tq0; key-side tensors (k, v, k_idx) hold
+// L rows per sequence from position 0.  A whole-sequence call has Lq = L,
+// tq0 = 0.
 struct IndexArgs {
   int B, L, G, nb, top_k, d_idx;
+  int Lq, tq0;
   int write_scores;  // 1: store block scores, 0: fused top-k -> sel
   int i_hi;          // query tiles [i_hi - n_items / (B * G/groups_per_cta), i_hi)
   int n_items;       // B * (query tiles) * (G / groups_per_cta)
@@ -30,6 +35,7 @@ cudaError_t launch_topk_kernel(const TopkArgs &a, cudaStream_t st);
 
 struct RevIdxArgs {
   int B, G, L, nb, top_k, qpi;  // qpi: queries per 128-row tile (128 / (H/G))
+  int Lq, tq0;                  // query-side geometry (see IndexArgs)
   int t0, Lc;                   // query chunk [t0, t0 + Lc)
   const int32_t *sel;           // [B,G,L,top_k]
   int32_t *cnt;                 // [B*G*nb]      (zeroed by the caller)
@@ -43,6 +49,7 @@ cudaError_t launch_revidx(const RevIdxArgs &a, cudaStream_t st);
 
 struct AttnArgs {
   int B, L, H, G, nb, top_k;
+  int Lq, tq0;                 // query-side geometry (see IndexArgs)
   float scale, scale_log2;
   int t0, Lc;
   int max_items;               // upper bound on the chunk's work items
@@ -62,6 +69,7 @@ cudaError_t launch_prefill_attn(const CUtensorMap &tk, const CUtensorMap &tv, co
 
 struct CombineArgs {
   int B, L, H, G, top_k;
+  int Lq, tq0;                 // query-side geometry (see IndexArgs)
   int t0, Lc;
   const int32_t *sel;          // [B,G,L,top_k]
   const int32_t *pos_of;       // [B,G,Lc,top_k]

@@ -173,16 +173,23 @@ int num_sms() {
 int *status_ptr(void *ws) { return reinterpret_cast<int *>(ws); }
 
 // ---- the operations --------------------------------------------------------
-// Index branch for the query tiles of tokens [t_lo, t_hi) (multiples of 128;
-// the whole sequence by default).
+// Query-side geometry: q, q_idx, sel and out hold Lq rows per sequence, row
+// 0 being position tq0 (Lq = L, tq0 = 0 for a whole sequence); k, v and
+// k_idx hold p->L rows per sequence.
+struct QGeom {
+  int Lq, tq0;
+};
+QGeom whole(const msa_params *p) { return QGeom{p->L, 0}; }
+
+// Index branch for the query tiles of tokens [t_lo, t_hi) (multiples of 128
+// within [tq0, tq0 + Lq)).
 int run_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 *k_idx,
-                     int32_t *sel, float *block_scores, void *ws, cudaStream_t st, int t_lo = 0,
-                     int t_hi = -1) {
+                     int32_t *sel, float *block_scores, void *ws, cudaStream_t st, QGeom qg,
+                     int t_lo, int t_hi) {
   const int nb = p->L / 128;
-  if (t_hi < 0) t_hi = p->L;
   CUtensorMap tq, tk;
   {
-    const uint64_t dims[3] = {uint64_t(p->d_idx), uint64_t(p->G), uint64_t(p->B) * p->L};
+    const uint64_t dims[3] = {uint64_t(p->d_idx), uint64_t(p->G), uint64_t(p->B) * qg.Lq};
     const uint64_t str[2] = {uint64_t(p->d_idx) * 2, uint64_t(p->d_idx) * 2 * p->G};
     const uint32_t box[3] = {64, 1, 128};
     int rc = make_tmap(&tq, q_idx, 3, dims, str, box);
@@ -197,6 +204,7 @@ int run_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 
   }
   msa::IndexArgs a;
   a.B = p->B; a.L = p->L; a.G = p->G; a.nb = nb; a.top_k = p->top_k; a.d_idx = p->d_idx;
+  a.Lq = qg.Lq; a.tq0 = qg.tq0;
   a.write_scores = block_scores ? 1 : 0;
   a.i_hi = t_hi / 128;
   a.n_items = p->B * (t_hi / 128 - t_lo / 128) * (p->G / msa::index_groups_per_cta(p->G, p->top_k));
@@ -231,11 +239,13 @@ struct AttnPlan {
   AttnWs w;
   int nb, qpi, sms;
   float scale;
+  QGeom qg;
 };
 
 int plan_attn(const msa_params *p, const msa_bf16 *k, const msa_bf16 *v, size_t ws_base,
-              AttnPlan *pl) {
+              QGeom qg, AttnPlan *pl) {
   pl->nb = p->L / 128;
+  pl->qg = qg;
   pl->w = attn_ws(p, ws_base);
   const uint64_t dims[3] = {uint64_t(p->d), uint64_t(p->G), uint64_t(p->B) * p->L};
   const uint64_t str[2] = {uint64_t(p->d) * 2, uint64_t(p->d) * 2 * p->G};
@@ -259,6 +269,7 @@ int run_attn_chunk(const msa_params *p, const AttnPlan &pl, const msa_bf16 *q, c
   const AttnWs &w = pl.w;
   msa::RevIdxArgs ra;
   ra.B = p->B; ra.G = p->G; ra.L = p->L; ra.nb = pl.nb; ra.top_k = p->top_k; ra.qpi = pl.qpi;
+  ra.Lq = pl.qg.Lq; ra.tq0 = pl.qg.tq0;
   ra.t0 = t0; ra.Lc = Lc;
   ra.sel = sel;
   ra.cnt = reinterpret_cast<int32_t *>(wsb + w.cnt);
@@ -271,6 +282,7 @@ int run_attn_chunk(const msa_params *p, const AttnPlan &pl, const msa_bf16 *q, c
   if (e != cudaSuccess) return cuda_fail(e, "reverse index launch");
   msa::AttnArgs aa;
   aa.B = p->B; aa.L = p->L; aa.H = p->H; aa.G = p->G; aa.nb = pl.nb; aa.top_k = p->top_k;
+  aa.Lq = pl.qg.Lq; aa.tq0 = pl.qg.tq0;
   aa.scale = pl.scale;
   aa.scale_log2 = pl.scale * 1.4426950408889634f;
   aa.t0 = t0; aa.Lc = Lc;
@@ -286,6 +298,7 @@ int run_attn_chunk(const msa_params *p, const AttnPlan &pl, const msa_bf16 *q, c
   if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
   msa::CombineArgs ca;
   ca.B = p->B; ca.L = p->L; ca.H = p->H; ca.G = p->G; ca.top_k = p->top_k;
+  ca.Lq = pl.qg.Lq; ca.tq0 = pl.qg.tq0;
   ca.t0 = t0; ca.Lc = Lc;
   ca.sel = sel;
   ca.pos_of = ra.pos_of;
@@ -299,11 +312,12 @@ int run_attn_chunk(const msa_params *p, const AttnPlan &pl, const msa_bf16 *q, c
     if (e != cudaSuccess) return cuda_fail(e, "chunk event");
     const size_t row = size_t(p->H) * p->d;   // elements of one token's output
     for (int b = 0; b < p->B && e == cudaSuccess; ++b) {
-      const size_t off = (size_t(b) * p->L + t0) * row;
+      const size_t qr = size_t(b) * pl.qg.Lq + (t0 - pl.qg.tq0);   // query-side row of t0
+      const size_t off = qr * row;
       e = cudaMemcpyAsync(sink->out_h + off, out + off, size_t(Lc) * row * 2,
                           cudaMemcpyDeviceToHost, sink->copy);
       if (e == cudaSuccess && sink->lse_h) {
-        const size_t lo = (size_t(b) * p->L + t0) * p->H;
+        const size_t lo = qr * p->H;
         e = cudaMemcpyAsync(sink->lse_h + lo, lse + lo, size_t(Lc) * p->H * 4,
                             cudaMemcpyDeviceToHost, sink->copy);
       }
@@ -313,14 +327,16 @@ int run_attn_chunk(const msa_params *p, const AttnPlan &pl, const msa_bf16 *q, c
   return MSA_OK;
 }
 
+// Main branch for the queries of positions [qg.tq0, qg.tq0 + qg.Lq).
 int run_prefill_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
                      const msa_bf16 *v, const int32_t *sel, msa_bf16 *out, float *lse, void *ws,
-                     size_t ws_base, cudaStream_t st) {
+                     size_t ws_base, cudaStream_t st, QGeom qg) {
   AttnPlan pl;
-  int rc = plan_attn(p, k, v, ws_base, &pl);
+  int rc = plan_attn(p, k, v, ws_base, qg, &pl);
   if (rc) return rc;
-  for (int t0 = 0; t0 < p->L; t0 += pl.w.Lc) {
-    const int Lc = (p->L - t0) < pl.w.Lc ? (p->L - t0) : pl.w.Lc;
+  const int t_end = qg.tq0 + qg.Lq;
+  for (int t0 = qg.tq0; t0 < t_end; t0 += pl.w.Lc) {
+    const int Lc = (t_end - t0) < pl.w.Lc ? (t_end - t0) : pl.w.Lc;
     rc = run_attn_chunk(p, pl, q, sel, out, lse, ws, t0, Lc, st, nullptr);
     if (rc) return rc;
   }
@@ -421,7 +437,7 @@ int msa_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 
   rc = check_ws(ws, ws_bytes, msa::kWsHeader);
   if (rc) return rc;
   return run_index_select(p, q_idx, k_idx, sel, block_scores, ws,
-                          reinterpret_cast<cudaStream_t>(stream));
+                          reinterpret_cast<cudaStream_t>(stream), whole(p), 0, p->L);
 }
 
 int msa_sparse_attn_prefill(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
@@ -439,7 +455,7 @@ int msa_sparse_attn_prefill(const msa_params *p, const msa_bf16 *q, const msa_bf
   rc = check_ws(ws, ws_bytes, need);
   if (rc) return rc;
   return run_prefill_attn(p, q, k, v, sel, out, lse, ws, msa::kWsHeader,
-                          reinterpret_cast<cudaStream_t>(stream));
+                          reinterpret_cast<cudaStream_t>(stream), whole(p));
 }
 
 int msa_forward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k, const msa_bf16 *v,
@@ -459,9 +475,37 @@ int msa_forward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k, const
   if (rc) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int32_t *s = sel ? sel : reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ws) + msa::kWsHeader);
-  rc = run_index_select(p, q_idx, k_idx, s, nullptr, ws, st);
+  rc = run_index_select(p, q_idx, k_idx, s, nullptr, ws, st, whole(p), 0, p->L);
   if (rc) return rc;
-  return run_prefill_attn(p, q, k, v, s, out, lse, ws, base, st);
+  return run_prefill_attn(p, q, k, v, s, out, lse, ws, base, st, whole(p));
+}
+
+int msa_forward_cached(const msa_params *p, int t0, int n, const msa_bf16 *q,
+                       const msa_bf16 *q_idx, const msa_bf16 *k_cache, const msa_bf16 *v_cache,
+                       const msa_bf16 *k_idx_cache, msa_bf16 *out, int32_t *sel, float *lse,
+                       void *ws, size_t ws_bytes, msa_stream stream) {
+  g_err[0] = 0;
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (t0 < 0 || n < 0 || t0 % 128 != 0 || n % 128 != 0 || (long long)t0 + n > p->L)
+    return fail(MSA_ERR_INVALID_ARG, "t0=%d n=%d: need multiples of 128 with t0 + n <= L=%d", t0,
+                n, p->L);
+  if (p->B == 0 || n == 0) return MSA_OK;
+  if (!q || !q_idx || !k_cache || !v_cache || !k_idx_cache || !out)
+    return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(q_idx) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(k_idx_cache) || !aligned16(out) || (sel && !aligned16(sel)) ||
+      (lse && !aligned16(lse)))
+    return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const size_t base = msa::kWsHeader + forward_sel_bytes(p);
+  rc = check_ws(ws, ws_bytes, attn_ws(p, base).end);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const QGeom qg{n, t0};
+  int32_t *s = sel ? sel : reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ws) + msa::kWsHeader);
+  rc = run_index_select(p, q_idx, k_idx_cache, s, nullptr, ws, st, qg, t0, t0 + n);
+  if (rc) return rc;
+  return run_prefill_attn(p, q, k_cache, v_cache, s, out, lse, ws, base, st, qg);
 }
 
 int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k_h,
@@ -491,7 +535,7 @@ int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k
   rc = host_events(&ev);
   if (rc) return rc;
   AttnPlan pl;
-  rc = plan_attn(p, dev->k, dev->v, base, &pl);
+  rc = plan_attn(p, dev->k, dev->v, base, whole(p), &pl);
   if (rc) return rc;
   int32_t *sel = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ws) + msa::kWsHeader);
   const ChunkSink sink{ev->down, ev->chunk, out_h, lse_h};
@@ -515,7 +559,7 @@ int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k
     if (e == cudaSuccess) e = cudaEventRecord(ev->idx_in, cp);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->idx_in, 0);
     if (e != cudaSuccess) return cuda_fail(e, "index input upload");
-    rc = run_index_select(p, dev->q_idx, dev->k_idx, sel, nullptr, ws, st, t0, t0 + Lc);
+    rc = run_index_select(p, dev->q_idx, dev->k_idx, sel, nullptr, ws, st, whole(p), t0, t0 + Lc);
     if (rc) return rc;
     up(dev->k, k_h, size_t(p->G) * p->d);
     up(dev->v, v_h, size_t(p->G) * p->d);

@@ -436,7 +436,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int bgj = d.x;
         const int g = (bgj / a.nb) % a.G;
         const int b = bgj / (a.nb * a.G);
-        const uint16_t *qb = a.q + (size_t(b) * a.L * a.H + size_t(g) * R) * kHeadDim + gran * 8;
+        const uint16_t *qb = a.q + size_t(g) * R * kHeadDim + gran * 8;
+        const int qrow0 = b * a.Lq - a.tq0;   // + t: the query's row in q (t >= tq0)
         const uint32_t stq = s_base + kSmemQ + s * kTile + (gran >> 3) * 16384;
         // row pair p = wg + 6*it (rows 2p, 2p+1): one coalesced 512-byte
         // copy per warp instruction
@@ -454,7 +455,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int t = __shfl_sync(0xffffffffu, e, qi & 31) >> 5;
             if (qi < d.z)
               cp_async16(stq + sw128_offset(row, gran & 7),
-                         qb + (size_t(t) * a.H + hh) * kHeadDim);
+                         qb + (size_t(qrow0 + t) * a.H + hh) * kHeadDim);
           }
         }
         cp_async_arrive_noinc(bar(kBarQFull + s));
@@ -655,7 +656,7 @@ __global__ void __launch_bounds__(256) msa_combine_kernel(const CombineArgs a) {
   const int r = a.H / a.G;
   const int g = h / r;
   const int hh = h % r;
-  const int32_t *sel = a.sel + ((size_t(b) * a.G + g) * a.L + t) * a.top_k;
+  const int32_t *sel = a.sel + ((size_t(b) * a.G + g) * a.Lq + (t - a.tq0)) * a.top_k;
   const int32_t *pos = a.pos_of + ((size_t(b) * a.G + g) * a.Lc + tl) * a.top_k;
   const bool in_k = lane < a.top_k;
   const int my_sel = in_k ? sel[lane] : -1;
@@ -697,8 +698,9 @@ __global__ void __launch_bounds__(256) msa_combine_kernel(const CombineArgs a) {
   uint2 res;
   res.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   res.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-  *reinterpret_cast<uint2 *>(a.out + (((size_t)b * a.L + t) * a.H + h) * kHeadDim + lane * 4) = res;
-  if (a.lse && lane == 0) a.lse[((size_t)b * a.L + t) * a.H + h] = (wsum > 0.f) ? M + __logf(wsum) : -INFINITY;
+  const size_t orow = (size_t)b * a.Lq + (t - a.tq0);
+  *reinterpret_cast<uint2 *>(a.out + (orow * a.H + h) * kHeadDim + lane * 4) = res;
+  if (a.lse && lane == 0) a.lse[orow * a.H + h] = (wsum > 0.f) ? M + __logf(wsum) : -INFINITY;
 }
 
 }  // namespace

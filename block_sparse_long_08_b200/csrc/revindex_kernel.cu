@@ -37,7 +37,7 @@ __global__ void __launch_bounds__(256) revidx_count_kernel(const RevIdxArgs a) {
     const long long r = e / a.top_k;
     const int tl = (int)(r % a.Lc);
     const long long bg = r / a.Lc;
-    const int j = a.sel[(bg * a.L + a.t0 + tl) * a.top_k + k];
+    const int j = a.sel[(bg * a.Lq + (a.t0 - a.tq0) + tl) * a.top_k + k];
     if (j < 0) continue;
     if (j >= a.nb) {
       atomicCAS(a.status, 0, kStatusBadInput);
@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(256) revidx_fill_kernel(const RevIdxArgs a) {
     const int tl = (int)(r % a.Lc);
     const long long bg = r / a.Lc;
     const int t = a.t0 + tl;
-    const int j = a.sel[(bg * a.L + t) * a.top_k + k];
+    const int j = a.sel[(bg * a.Lq + (t - a.tq0)) * a.top_k + k];
     if (j < 0 || j >= a.nb) continue;
     const long long e_out = r * a.top_k + k;
     const int pos = a.list_off[bg * a.nb + j] + a.pos_of[e_out];

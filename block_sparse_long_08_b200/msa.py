@@ -71,6 +71,8 @@ def lib() -> ctypes.CDLL:
         L.msa_sparse_attn_prefill.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.msa_sparse_attn_decode.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.msa_forward.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.msa_forward_cached.argtypes = [pp, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P,
+                                         _P, _P, _SZ, _P]
         L.msa_forward_host.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P,
                                        ctypes.POINTER(msa_staging), _P, _SZ, _P, _P]
         L.msa_sparse_attn_decode_noalloc.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P]
@@ -83,7 +85,7 @@ def lib() -> ctypes.CDLL:
         L.msa_last_error.restype = ctypes.c_char_p
         L.msa_version.restype = ctypes.c_char_p
         for f in ("msa_index_select", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
-                  "msa_forward", "msa_forward_host", "msa_read_status"):
+                  "msa_forward", "msa_forward_host", "msa_forward_cached", "msa_read_status"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -212,6 +214,39 @@ def msa_forward(q, k, v, q_idx, k_idx, top_k: int, *, scale: float = 0.0, want_s
     ws = _ensure_ws(ws, p, MSA_OP_FORWARD, dev)
     _check(lib().msa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_idx), _ptr(k_idx),
                              _ptr(out), _ptr(sel), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    res = [out]
+    if want_sel:
+        res.append(sel)
+    if want_lse:
+        res.append(lse)
+    return res[0] if len(res) == 1 else tuple(res)
+
+
+def msa_forward_cached(q, q_idx, k_cache, v_cache, k_idx_cache, t0: int, top_k: int, *,
+                       scale: float = 0.0, want_sel: bool = False, want_lse: bool = False,
+                       out=None, sel=None, ws=None, stream=None, chunk: int = 0):
+    """Prefill of the n new tokens at positions [t0, t0+n) against caches that
+    already hold every key up to t0+n: q [B,n,H,d], q_idx [B,n,G,d_idx];
+    k_cache/v_cache [B,Lmax,G,d], k_idx_cache [B,Lmax,d_idx] -> out [B,n,H,d]
+    (and sel [B,G,n,top_k], lse [B,n,H]); equal to rows [t0, t0+n) of
+    msa_forward over a sequence of length t0+n."""
+    for n_, t in (("q", q), ("q_idx", q_idx), ("k_cache", k_cache), ("v_cache", v_cache),
+                  ("k_idx_cache", k_idx_cache)):
+        _req(t, n_, torch.bfloat16)
+    B, n, H, d = q.shape
+    Lmax, G = k_cache.shape[1], k_cache.shape[2]
+    di = q_idx.shape[3]
+    p = make_params(B, Lmax, H, G, d, di, 128, top_k, scale, chunk)
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if sel is None and want_sel:
+        sel = torch.empty((B, G, n, top_k), dtype=torch.int32, device=dev)
+    lse = torch.empty((B, n, H), dtype=torch.float32, device=dev) if want_lse else None
+    ws = _ensure_ws(ws, p, MSA_OP_FORWARD, dev)
+    _check(lib().msa_forward_cached(ctypes.byref(p), int(t0), int(n), _ptr(q), _ptr(q_idx),
+                                    _ptr(k_cache), _ptr(v_cache), _ptr(k_idx_cache), _ptr(out),
+                                    _ptr(sel), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
     res = [out]
     if want_sel:
         res.append(sel)

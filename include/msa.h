@@ -170,6 +170,25 @@ int msa_forward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k, const
                 const msa_bf16 *q_idx, const msa_bf16 *k_idx, msa_bf16 *out, int32_t *sel,
                 float *lse, void *ws, size_t ws_bytes, msa_stream stream);
 
+/* Prefill of n new tokens per sequence, at positions [t0, t0 + n), against
+ * a cache that already holds every key up to t0 + n: the serving form of
+ * the prefill (a prompt processed in chunks, or continued after a cached
+ * prefix; the explainer's serving discussion, §4.1).  Each new query attends
+ * exactly as in msa_forward over a sequence of length t0 + n, so the
+ * results equal rows [t0, t0 + n) of that call.
+ *   p->L = cache capacity Lmax; t0 and n multiples of 128, t0 + n <= Lmax
+ *   q [B,n,H,d], q_idx [B,n,G,d_idx] bf16: the new tokens' queries     (in)
+ *   k_cache, v_cache [B,Lmax,G,d], k_idx_cache [B,Lmax,d_idx] bf16, the
+ *     new tokens' rows already written; rows >= t0 + n are not read     (in)
+ *   out [B,n,H,d] bf16; sel [B,G,n,top_k] int32 or NULL; lse [B,n,H]
+ *     fp32 or NULL                                                   (out)
+ *   ws >= msa_workspace_bytes(p, MSA_OP_FORWARD)
+ * Every sequence of the batch has the same t0 and n. */
+int msa_forward_cached(const msa_params *p, int t0, int n, const msa_bf16 *q,
+                       const msa_bf16 *q_idx, const msa_bf16 *k_cache, const msa_bf16 *v_cache,
+                       const msa_bf16 *k_idx_cache, msa_bf16 *out, int32_t *sel, float *lse,
+                       void *ws, size_t ws_bytes, msa_stream stream);
+
 /* Device buffers that msa_forward_host stages its transfers in: the device
  * counterparts of msa_forward's tensors (caller-owned, 16-byte aligned).
  * lse may be NULL when no lse is requested. */

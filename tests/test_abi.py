@@ -115,6 +115,15 @@ def test_forward_host_rejects_bad_arguments():
     assert rc == M.MSA_ERR_WORKSPACE
 
 
+@pytest.mark.parametrize("t0,n", [(100, 128), (128, 100), (-128, 128), (3968, 256), (0, -128)])
+def test_cached_prefill_rejects_bad_ranges(t0, n):
+    p = M.make_params(1, 4096, 8, 2, 128, 64, 128, 4)
+    ok = ctypes.c_void_p(4096)
+    rc = M.lib().msa_forward_cached(ctypes.byref(p), t0, n, ok, ok, ok, ok, ok, ok, None, None, ok,
+                                    1 << 30, None)
+    assert rc == M.MSA_ERR_INVALID_ARG, (rc, M.msa_last_error())
+
+
 def test_decode_rejects_more_than_eight_groups():
     p = M.make_params(2, 4096, 32, 16, 128, 128, 128, 16)
     assert M.lib().msa_workspace_bytes(ctypes.byref(p), M.MSA_OP_DECODE) == 0
