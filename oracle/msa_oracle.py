@@ -21,6 +21,11 @@ Sources (cited by page title / address and section):
   16 blocks x 128 tokens per query group).
 * [P3] "揭秘MiniMax闪电注意力机制", §1: textbook softmax attention, the
   quadratic baseline that sparse attention avoids.
+* [P1] the long-context engineering essay (the FP8-KV paragraphs): low-
+  precision (FP8) cache storage as the direction to pursue, with error
+  control as its concern.  The FP8 cache format itself is the OCP 8-bit
+  floating point E4M3 encoding; its definition, not the pages, fixes
+  e4m3_to_f64.
 
 Readings taken where the pages are silent (each is also listed in the
 design notes):
@@ -49,6 +54,8 @@ import numpy as np
 
 __all__ = [
     "as_f64",
+    "e4m3_to_f64",
+    "dequant_rows",
     "token_index_scores",
     "block_scores_row",
     "select_blocks_row",
@@ -58,6 +65,27 @@ __all__ = [
     "decode",
     "block_scores_all",
 ]
+
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Value of 8-bit E4M3 floating-point codes (OCP FP8 E4M3, the 'fn'
+    variant): bit 7 sign, bits 6..3 exponent e (bias 7), bits 2..0 mantissa m.
+    e = 0: subnormal, (m / 8) * 2^-6; e = 1..15: (1 + m / 8) * 2^(e - 7),
+    except e = 15, m = 7, which is NaN (the format has no infinities).  The
+    largest finite magnitude is 1.75 * 2^8 = 448."""
+    c = np.asarray(codes).astype(np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & (m == 7), np.nan, mag)
+    return sign * mag
+
+
+def dequant_rows(codes, scale) -> np.ndarray:
+    """Rows of E4M3 codes [..., D] with one scale per row [...]: the stored
+    row is scale * e4m3_to_f64(codes)."""
+    return e4m3_to_f64(codes) * np.asarray(scale, dtype=np.float64)[..., None]
 
 
 def as_f64(x) -> np.ndarray:

@@ -254,8 +254,28 @@ def check_decode_is_last_prefill_row():
     np.testing.assert_array_equal(dec["sel"][1], pre["sel"][1, :, 58])
 
 
+def check_e4m3_against_library_and_closed_forms():
+    # every one of the 256 codes against torch's float8_e4m3fn conversion
+    codes = np.arange(256, dtype=np.uint8)
+    lib = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = O.e4m3_to_f64(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(lib))
+    np.testing.assert_array_equal(got[~np.isnan(got)], lib[~np.isnan(lib)])
+    # values fixed by the format's definition
+    want = {0x00: 0.0, 0x38: 1.0, 0x3C: 1.5, 0xB8: -1.0, 0x7E: 448.0, 0xFE: -448.0,
+            0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x40: 2.0, 0x30: 0.5}
+    for c, v in want.items():
+        assert O.e4m3_to_f64(np.uint8(c)) == v, hex(c)
+    assert math.copysign(1.0, float(O.e4m3_to_f64(np.uint8(0x80)))) == -1.0
+    assert np.isnan(O.e4m3_to_f64(np.uint8(0x7F))) and np.isnan(O.e4m3_to_f64(np.uint8(0xFF)))
+    # dequantization: one scale per row
+    rows = np.array([[0x38, 0x40], [0x3C, 0xB8]], dtype=np.uint8)
+    np.testing.assert_array_equal(O.dequant_rows(rows, [0.25, 4.0]), [[0.25, 0.5], [6.0, -4.0]])
+
+
 CHECKS = {
     "golden": check_golden,
+    "e4m3": check_e4m3_against_library_and_closed_forms,
     "dense_limit": check_dense_limit,
     "block_local_limit": check_block_local_limit,
     "brute_force_float": lambda: check_selection_brute_force(False),
@@ -321,6 +341,19 @@ def _attend_swapped_kv(q_rows, k_tok, v_tok, scale):
 
 _orig_attend = O.attend_rows
 
+
+def _e4m3_bias8(codes):
+    return _orig_e4m3(codes) * 0.5      # exponent bias 8 instead of 7
+
+
+def _e4m3_no_subnormals(codes):
+    v = _orig_e4m3(codes)
+    c = np.asarray(codes).astype(np.uint8)
+    return np.where(((c >> 3) & 0xF) == 0, np.sign(v) * 0.0, v)
+
+
+_orig_e4m3 = O.e4m3_to_f64
+
 MUTANTS = {
     "no_forced_local": ("select_blocks_row", _select_no_local),
     "ties_to_higher_id": ("select_blocks_row", _select_high_tie),
@@ -329,6 +362,8 @@ MUTANTS = {
     "strict_causal": ("selected_tokens", _tokens_strict),
     "scale_dropped": ("attend_rows", _attend_no_scale),
     "k_v_swapped": ("attend_rows", _attend_swapped_kv),
+    "e4m3_bias_8": ("e4m3_to_f64", _e4m3_bias8),
+    "e4m3_no_subnormals": ("e4m3_to_f64", _e4m3_no_subnormals),
 }
 
 
