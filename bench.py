@@ -99,11 +99,14 @@ def prefill_attn_bytes(B, L, H, G, d, top_k):
     return entries * r * (d * 2 * 3 + 4 * 2) + B * float(L) * H * d * 2
 
 
-def decode_bytes(seq_lens, H, G, d, d_idx, top_k):
+def decode_bytes(seq_lens, H, G, d, d_idx, top_k, fp8_index=False):
+    """Bytes a decode step must read: the index-key scan over every cached
+    token (bf16, or E4M3 codes + one fp32 scale per token), the selected K/V
+    tokens, and the small per-step tensors."""
     n = np.asarray(seq_lens, dtype=np.int64)
     t = n - 1
     kv = G * 2 * d * 2 * n_sel(t, top_k)
-    scan = n * d_idx * 2
+    scan = n * (d_idx + 4) if fp8_index else n * d_idx * 2
     small = len(n) * (H * d * 2 * 2 + G * d_idx * 2)
     return float((kv + scan).sum() + small)
 
@@ -529,36 +532,52 @@ def bench_decode_128k(M, I, dev, args, peaks):
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
+    codes, kscale = I.fp8_index_cache(y["k_idx_cache"])   # the same cache stored in FP8
+
     def run():
         M.msa_sparse_attn_decode(y["q"], y["q_idx"], y["k_cache"], y["v_cache"], y["k_idx_cache"], seq,
                                  ds.top_k, out=out, ws=ws)
 
-    for _ in range(max(3, args.warmup)):
-        run()
-    torch.cuda.synchronize()
-    if M.msa_read_status(ws) != 0:
-        raise SystemExit("decode-128k device status error")
-    iters = 20
-    times = []
-    for _ in range(iters):
-        flush.zero_()   # L2 flush (256 MB > 126 MB L2) outside the timed span
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        run()
-        b.record(stream)
+    def run_fp8():
+        M.msa_sparse_attn_decode_fp8idx(y["q"], y["q_idx"], y["k_cache"], y["v_cache"], codes,
+                                        kscale, seq, ds.top_k, out=out, ws=ws)
+
+    def timed(fn):
+        for _ in range(max(3, args.warmup)):
+            fn()
         torch.cuda.synchronize()
-        times.append(a.elapsed_time(b))
-    us = statistics.median(times) * 1e3
-    byts = decode_bytes(y["seq_lens"].numpy(), ds.H, ds.G, ds.d, ds.d_idx, ds.top_k)
-    del y
+        if M.msa_read_status(ws) != 0:
+            raise SystemExit("decode-128k device status error")
+        times = []
+        for _ in range(iters):
+            flush.zero_()   # L2 flush (256 MB > 126 MB L2) outside the timed span
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        return statistics.median(times) * 1e3
+
+    def roof(byts, us):
+        return {"bound": "hbm", "achieved": byts / (us / 1e6) / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": byts / (us / 1e6) / 1e9 / peaks["hbm_gbs"], "bytes": byts}
+
+    iters = 20
+    us = timed(run)
+    us8 = timed(run_fp8)
+    lens = y["seq_lens"].numpy()
+    byts = decode_bytes(lens, ds.H, ds.G, ds.d, ds.d_idx, ds.top_k)
+    byts8 = decode_bytes(lens, ds.H, ds.G, ds.d, ds.d_idx, ds.top_k, fp8_index=True)
+    del y, codes, kscale
     return {"us_per_step": us, "iters": iters, "batch": ds.B,
             "seq_lens": f"U[{ds.len_lo},{ds.len_hi}] seed {I.SEEDS['decode_128k']}",
             "l2": "256 MB buffer written between iterations",
-            "roofline": {"bound": "hbm", "achieved": byts / (us / 1e6) / 1e9, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": byts / (us / 1e6) / 1e9 / peaks["hbm_gbs"],
-                         "bytes": byts},
-            "gpu_launches": 4 * iters}
+            "roofline": roof(byts, us),
+            "fp8_index_cache": {"us_per_step": us8, "roofline": roof(byts8, us8),
+                                "cache": "k_idx as E4M3 codes + fp32 scale per token"},
+            "gpu_launches": 8 * iters}
 
 
 def bench_e2e(M, x, dx, shape, dshape, K, args, ws_n, stream):

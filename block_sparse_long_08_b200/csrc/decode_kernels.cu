@@ -18,6 +18,7 @@
 //                         the tensor cores (mma.sync, heads as M rows).
 //   decode_combine_kernel one warp per (sequence, head): merge <= top_k
 //                         partials.
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cfloat>
@@ -102,6 +103,105 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const DecodeArgs a) {
     }
     mx0 = fmaxf(mx0, fmaxf(acc[0], acc[2]));
     mx1 = fmaxf(mx1, fmaxf(acc[1], acc[3]));
+  }
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+  }
+  if (lane < 4) {
+    const int g0 = 2 * c, g1 = 2 * c + 1;
+    if (g0 < a.G) a.scores[(size_t(b) * a.G + g0) * a.nb_max + j] = mx0;
+    if (g1 < a.G) a.scores[(size_t(b) * a.G + g1) * a.nb_max + j] = mx1;
+  }
+}
+
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                              uint32_t a2, uint32_t a3, uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two E4M3 codes (low byte first) -> two f16 (exact: every E4M3 value is an
+// f16 value).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+  uint32_t r;
+  const uint16_t in = static_cast<uint16_t>(two);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(in));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t f16x2_of(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// decode_index_kernel for an FP8 index-key cache: the stored key of token s
+// is k_idx_scale[s] * E4M3(k_idx8[s]) (one scale per token), so its score is
+// k_idx_scale[s] * (q_idx . E4M3 codes).  Half the bytes of the bf16 scan.
+// The MMA runs in f16: the codes convert exactly, and q_idx (bf16) converts
+// exactly while it stays within the f16 range.  Lane (g4, c) loads 16-byte
+// granules of 16 codes; k-step kk takes d = 16(c + 4(kk/4)) + 4(kk%4) +
+// {0,1} at k positions 2c, 2c+1 and + {2,3} at 2c+8, 2c+9, i.e. the bytes
+// of word kk%4 of granule kk/4.
+template <int DI>
+__global__ void __launch_bounds__(256) decode_index_fp8_kernel(const DecodeArgs a) {
+  constexpr int NG = DI / 64;  // granules per lane per key row
+  constexpr int NK = DI / 16;  // MMA k-steps
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  const int j = blockIdx.x * 8 + warp;
+  const int n = a.seq_lens[b];
+  if (n < 1 || n > a.Lmax) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicCAS(a.status, 0, kStatusBadInput);
+    return;
+  }
+  const int bt = (n - 1) / kBlock;
+  if (bt + 1 <= a.top_k || j >= bt) return;
+  const int g4 = lane >> 2, c = lane & 3;
+  uint32_t bq[NK][2];
+  {
+    const bool gv = g4 < a.G;
+    const uint16_t *qrow = a.q_idx + (size_t(b) * a.G + (gv ? g4 : 0)) * DI;
+#pragma unroll
+    for (int kk = 0; kk < NK; ++kk) {
+      const int d0 = 16 * (c + 4 * (kk >> 2)) + 4 * (kk & 3);
+      const uint2 v = *reinterpret_cast<const uint2 *>(qrow + d0);
+      bq[kk][0] = gv ? f16x2_of(bf16_lo(v.x), bf16_hi(v.x)) : 0u;
+      bq[kk][1] = gv ? f16x2_of(bf16_lo(v.y), bf16_hi(v.y)) : 0u;
+    }
+  }
+  const uint8_t *kbase = a.k_idx8 + (size_t(b) * a.Lmax + size_t(j) * kBlock) * DI;
+  const float *sbase = a.k_idx_scale + size_t(b) * a.Lmax + size_t(j) * kBlock;
+  float mx0 = -FLT_MAX, mx1 = -FLT_MAX;
+#pragma unroll 2
+  for (int rt = 0; rt < 8; ++rt) {
+    const uint8_t *r0 = kbase + size_t(rt * 16 + g4) * DI;
+    const uint8_t *r1 = r0 + 8 * DI;
+    uint4 lo[NG], hi[NG];
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) {
+      lo[gi] = ldg_nc_v4(r0 + 16 * (c + 4 * gi));
+      hi[gi] = ldg_nc_v4(r1 + 16 * (c + 4 * gi));
+    }
+    const float s0 = __ldg(sbase + rt * 16 + g4), s1 = __ldg(sbase + rt * 16 + g4 + 8);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) {
+      const uint32_t wl[4] = {lo[gi].x, lo[gi].y, lo[gi].z, lo[gi].w};
+      const uint32_t wh[4] = {hi[gi].x, hi[gi].y, hi[gi].z, hi[gi].w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w)
+        mma_f16_16816(acc, e4m3x2_to_f16x2(wl[w]), e4m3x2_to_f16x2(wh[w]),
+                      e4m3x2_to_f16x2(wl[w] >> 16), e4m3x2_to_f16x2(wh[w] >> 16),
+                      bq[4 * gi + w][0], bq[4 * gi + w][1]);
+    }
+    mx0 = fmaxf(mx0, fmaxf(acc[0] * s0, acc[2] * s1));
+    mx1 = fmaxf(mx1, fmaxf(acc[1] * s0, acc[3] * s1));
   }
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
@@ -414,10 +514,16 @@ cudaError_t launch_decode_attn(const DecodeArgs &a, cudaStream_t st) {
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st) {
   if (a.B == 0) return cudaSuccess;
   const dim3 gi((a.nb_max + 7) / 8, a.B);
-  if (a.d_idx == 64)
+  if (a.k_idx8) {
+    if (a.d_idx == 64)
+      decode_index_fp8_kernel<64><<<gi, 256, 0, st>>>(a);
+    else
+      decode_index_fp8_kernel<128><<<gi, 256, 0, st>>>(a);
+  } else if (a.d_idx == 64) {
     decode_index_kernel<64><<<gi, 256, 0, st>>>(a);
-  else
+  } else {
     decode_index_kernel<128><<<gi, 256, 0, st>>>(a);
+  }
   decode_topk_kernel<<<a.B * a.G, kTopkWarps * 32, 0, st>>>(a);
   cudaError_t e;
   switch (a.H / a.G) {

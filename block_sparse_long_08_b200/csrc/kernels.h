@@ -84,6 +84,10 @@ struct DecodeArgs {
   int B, Lmax, H, G, d_idx, nb_max, top_k;
   float scale, scale_log2;
   const uint16_t *q, *q_idx, *k_cache, *v_cache, *k_idx_cache;
+  // FP8 index-key cache (when non-null, used instead of k_idx_cache):
+  // E4M3 codes [B,Lmax,d_idx] and one fp32 scale per token [B,Lmax]
+  const uint8_t *k_idx8;
+  const float *k_idx_scale;
   const int32_t *seq_lens;
   float *scores;               // [B,G,nb_max]
   int32_t *sel;                // [B,G,top_k]
@@ -93,6 +97,10 @@ struct DecodeArgs {
   int *status;
 };
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
+
+// Row-wise E4M3 quantization (one fp32 scale per row); cols % 8 == 0.
+cudaError_t launch_quantize_e4m3_rows(const uint16_t *x, long long rows, int cols, uint8_t *codes,
+                                      float *scale, cudaStream_t st);
 
 // Sets the message msa_last_error() returns; returns `code`.
 int report_error(int code, const char *msg);

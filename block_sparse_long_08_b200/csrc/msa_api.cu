@@ -374,6 +374,47 @@ int host_events(HostEvents **out) {
   return MSA_OK;
 }
 
+// Decode step with the index-key cache in bf16 (k_idx_cache) or in FP8
+// (k_idx8 + k_idx_scale); exactly one of the two is given.
+int run_decode(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
+               const msa_bf16 *k_cache, const msa_bf16 *v_cache, const msa_bf16 *k_idx_cache,
+               const uint8_t *k_idx8, const float *k_idx_scale, const int32_t *seq_lens,
+               msa_bf16 *out, int32_t *sel, void *ws, size_t ws_bytes, cudaStream_t st) {
+  int rc = check_params(p, true);
+  if (rc) return rc;
+  if (p->B == 0) return MSA_OK;
+  if (p->L == 0) return fail(MSA_ERR_INVALID_ARG, "decode needs a cache (L = Lmax > 0)");
+  if (!q || !q_idx || !k_cache || !v_cache || !seq_lens || !out || (!k_idx_cache && !k_idx8) ||
+      (k_idx8 && !k_idx_scale))
+    return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(q_idx) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      (k_idx_cache && !aligned16(k_idx_cache)) || (k_idx8 && !aligned16(k_idx8)) ||
+      (k_idx_scale && (reinterpret_cast<uintptr_t>(k_idx_scale) & 3u)) || !aligned16(out) ||
+      (sel && !aligned16(sel)))
+    return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned (scales 4-byte)");
+  const DecWs w = dec_ws(p);
+  rc = check_ws(ws, ws_bytes, w.end);
+  if (rc) return rc;
+  uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
+  msa::DecodeArgs a;
+  a.B = p->B; a.Lmax = p->L; a.H = p->H; a.G = p->G; a.d_idx = p->d_idx;
+  a.nb_max = p->L / 128; a.top_k = p->top_k;
+  a.scale = eff_scale(p);
+  a.scale_log2 = a.scale * 1.4426950408889634f;
+  a.q = q; a.q_idx = q_idx; a.k_cache = k_cache; a.v_cache = v_cache; a.k_idx_cache = k_idx_cache;
+  a.k_idx8 = k_idx8; a.k_idx_scale = k_idx_scale;
+  a.seq_lens = seq_lens;
+  a.scores = reinterpret_cast<float *>(wsb + w.scores);
+  a.sel = sel ? sel : reinterpret_cast<int32_t *>(wsb + w.sel);
+  a.part_o = reinterpret_cast<float *>(wsb + w.part_o);
+  a.part_lse = reinterpret_cast<float *>(wsb + w.part_lse);
+  a.out = out;
+  a.status = status_ptr(ws);
+  cudaError_t e = msa::launch_decode(a, st);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return MSA_OK;
+}
+
 }  // namespace
 
 namespace msa {
@@ -584,34 +625,34 @@ int msa_sparse_attn_decode(const msa_params *p, const msa_bf16 *q, const msa_bf1
                            const msa_bf16 *k_idx_cache, const int32_t *seq_lens, msa_bf16 *out,
                            int32_t *sel, void *ws, size_t ws_bytes, msa_stream stream) {
   g_err[0] = 0;
-  int rc = check_params(p, true);
-  if (rc) return rc;
-  if (p->B == 0) return MSA_OK;
-  if (p->L == 0) return fail(MSA_ERR_INVALID_ARG, "decode needs a cache (L = Lmax > 0)");
-  if (!q || !q_idx || !k_cache || !v_cache || !k_idx_cache || !seq_lens || !out)
-    return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
-  if (!aligned16(q) || !aligned16(q_idx) || !aligned16(k_cache) || !aligned16(v_cache) ||
-      !aligned16(k_idx_cache) || !aligned16(out) || (sel && !aligned16(sel)))
+  return run_decode(p, q, q_idx, k_cache, v_cache, k_idx_cache, nullptr, nullptr, seq_lens, out,
+                    sel, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int msa_sparse_attn_decode_fp8idx(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
+                                  const msa_bf16 *k_cache, const msa_bf16 *v_cache,
+                                  const uint8_t *k_idx8, const float *k_idx_scale,
+                                  const int32_t *seq_lens, msa_bf16 *out, int32_t *sel, void *ws,
+                                  size_t ws_bytes, msa_stream stream) {
+  g_err[0] = 0;
+  if (!k_idx8) return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  return run_decode(p, q, q_idx, k_cache, v_cache, nullptr, k_idx8, k_idx_scale, seq_lens, out,
+                    sel, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int msa_quantize_e4m3_rows(const msa_bf16 *x, long long rows, int cols, uint8_t *codes,
+                           float *scale, msa_stream stream) {
+  g_err[0] = 0;
+  if (rows < 0 || cols <= 0 || cols % 16 != 0)
+    return fail(MSA_ERR_INVALID_ARG, "rows=%lld cols=%d: cols must be a positive multiple of 16",
+                rows, cols);
+  if (rows == 0) return MSA_OK;
+  if (!x || !codes || !scale) return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scale))
     return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-  const DecWs w = dec_ws(p);
-  rc = check_ws(ws, ws_bytes, w.end);
-  if (rc) return rc;
-  uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
-  msa::DecodeArgs a;
-  a.B = p->B; a.Lmax = p->L; a.H = p->H; a.G = p->G; a.d_idx = p->d_idx;
-  a.nb_max = p->L / 128; a.top_k = p->top_k;
-  a.scale = eff_scale(p);
-  a.scale_log2 = a.scale * 1.4426950408889634f;
-  a.q = q; a.q_idx = q_idx; a.k_cache = k_cache; a.v_cache = v_cache; a.k_idx_cache = k_idx_cache;
-  a.seq_lens = seq_lens;
-  a.scores = reinterpret_cast<float *>(wsb + w.scores);
-  a.sel = sel ? sel : reinterpret_cast<int32_t *>(wsb + w.sel);
-  a.part_o = reinterpret_cast<float *>(wsb + w.part_o);
-  a.part_lse = reinterpret_cast<float *>(wsb + w.part_lse);
-  a.out = out;
-  a.status = status_ptr(ws);
-  cudaError_t e = msa::launch_decode(a, reinterpret_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  cudaError_t e = msa::launch_quantize_e4m3_rows(x, rows, cols, codes, scale,
+                                                 reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return MSA_OK;
 }
 

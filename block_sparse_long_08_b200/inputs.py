@@ -132,6 +132,19 @@ def decode_inputs(shape: DecodeShape, seed: int, device="cpu") -> dict:
     return out
 
 
+def fp8_index_cache(k_idx_cache: torch.Tensor) -> tuple:
+    """An FP8 index-key cache holding the given bf16 cache [B,Lmax,d_idx]:
+    E4M3 codes (uint8, same shape) and one fp32 scale per token [B,Lmax],
+    scale = max|row| / 448, codes = the row divided by its scale, rounded to
+    E4M3 by torch's float8_e4m3fn conversion.  (Input preparation: the
+    method consumes codes and scales as given.)"""
+    x = k_idx_cache.float()
+    amax = x.abs().amax(dim=-1)
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    codes = (x / scale[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes.contiguous(), scale.contiguous()
+
+
 def small_integer_like(t: torch.Tensor, seed: int, lo: int = -4, hi: int = 4) -> torch.Tensor:
     """Same shape/dtype/device as t, integers drawn uniformly from [lo, hi].
     Dot products of such bf16 values are exact in fp32 and fp64 alike, which

@@ -76,6 +76,9 @@ def lib() -> ctypes.CDLL:
         L.msa_forward_host.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P,
                                        ctypes.POINTER(msa_staging), _P, _SZ, _P, _P]
         L.msa_sparse_attn_decode_noalloc.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+        L.msa_sparse_attn_decode_fp8idx.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ,
+                                                    _P]
+        L.msa_quantize_e4m3_rows.argtypes = [_P, ctypes.c_longlong, ctypes.c_int, _P, _P, _P]
         L.msa_sparse_attn_decode_noalloc.restype = ctypes.c_int
         L.msa_workspace_bytes.argtypes = [pp, ctypes.c_int]
         L.msa_workspace_bytes.restype = _SZ
@@ -85,7 +88,8 @@ def lib() -> ctypes.CDLL:
         L.msa_last_error.restype = ctypes.c_char_p
         L.msa_version.restype = ctypes.c_char_p
         for f in ("msa_index_select", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
-                  "msa_forward", "msa_forward_host", "msa_forward_cached", "msa_read_status"):
+                  "msa_forward", "msa_forward_host", "msa_forward_cached", "msa_read_status",
+                  "msa_sparse_attn_decode_fp8idx", "msa_quantize_e4m3_rows"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -325,6 +329,48 @@ def msa_sparse_attn_decode(q, q_idx, k_cache, v_cache, k_idx_cache, seq_lens, to
                                         _ptr(v_cache), _ptr(k_idx_cache), _ptr(seq_lens), _ptr(out),
                                         _ptr(sel), _ptr(ws), ws.numel(), _stream(stream)))
     return (out, sel) if want_sel else out
+
+
+def msa_sparse_attn_decode_fp8idx(q, q_idx, k_cache, v_cache, k_idx8, k_idx_scale, seq_lens,
+                                  top_k: int, *, scale: float = 0.0, want_sel: bool = False,
+                                  out=None, sel=None, ws=None, stream=None):
+    """msa_sparse_attn_decode with the index-key cache in FP8: k_idx8 [B,Lmax,d_idx]
+    uint8 E4M3 codes and k_idx_scale [B,Lmax] fp32 (stored key = scale * E4M3(code))."""
+    _req(q, "q", torch.bfloat16)
+    _req(q_idx, "q_idx", torch.bfloat16)
+    _req(k_cache, "k_cache", torch.bfloat16)
+    _req(v_cache, "v_cache", torch.bfloat16)
+    _req(k_idx8, "k_idx8", torch.uint8)
+    _req(k_idx_scale, "k_idx_scale", torch.float32)
+    _req(seq_lens, "seq_lens", torch.int32)
+    B, H, d = q.shape
+    Lmax, G = k_cache.shape[1], k_cache.shape[2]
+    p = make_params(B, Lmax, H, G, d, k_idx8.shape[2], 128, top_k, scale)
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if sel is None and want_sel:
+        sel = torch.empty((B, G, top_k), dtype=torch.int32, device=dev)
+    ws = _ensure_ws(ws, p, MSA_OP_DECODE, dev)
+    _check(lib().msa_sparse_attn_decode_fp8idx(ctypes.byref(p), _ptr(q), _ptr(q_idx), _ptr(k_cache),
+                                               _ptr(v_cache), _ptr(k_idx8), _ptr(k_idx_scale),
+                                               _ptr(seq_lens), _ptr(out), _ptr(sel), _ptr(ws),
+                                               ws.numel(), _stream(stream)))
+    return (out, sel) if want_sel else out
+
+
+def msa_quantize_e4m3_rows(x, *, codes=None, scale=None, stream=None):
+    """bf16 [..., cols] -> (E4M3 codes uint8 [..., cols], fp32 scale [...]), one scale per row."""
+    _req(x, "x", torch.bfloat16)
+    cols = x.shape[-1]
+    rows = x.numel() // cols
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _check(lib().msa_quantize_e4m3_rows(_ptr(x), rows, cols, _ptr(codes), _ptr(scale),
+                                        _stream(stream)))
+    return codes, scale
 
 
 def msa_sparse_attn_decode_noalloc(q, q_idx, k_cache, v_cache, k_idx_cache, seq_lens, top_k: int, *,

@@ -140,6 +140,31 @@ int msa_sparse_attn_decode(const msa_params *p, const msa_bf16 *q, const msa_bf1
                            msa_bf16 *out, int32_t *sel, void *ws, size_t ws_bytes,
                            msa_stream stream);
 
+/* Decode step with the index-key cache stored in FP8 (the essay's low-
+ * precision cache direction): the stored index key of token s is
+ * k_idx_scale[s] * E4M3(k_idx8[s]), E4M3 being the OCP 8-bit floating-point
+ * format (4 exponent bits, bias 7, 3 mantissa bits).  The scan, most of a
+ * decode step's bytes, reads half as much.  Everything else is
+ * msa_sparse_attn_decode.
+ *   k_idx8 [B,Lmax,d_idx] uint8 E4M3 codes, 16-byte aligned           (in)
+ *   k_idx_scale [B,Lmax] fp32, one scale per token                      (in)
+ * Scores are accumulated in fp32 from f16 products: q_idx must lie within
+ * the f16 range (|x| < 65504), where its bf16 values convert exactly.
+ * msa_quantize_e4m3_rows produces codes and scales from bf16 rows. */
+int msa_sparse_attn_decode_fp8idx(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
+                                  const msa_bf16 *k_cache, const msa_bf16 *v_cache,
+                                  const uint8_t *k_idx8, const float *k_idx_scale,
+                                  const int32_t *seq_lens, msa_bf16 *out, int32_t *sel, void *ws,
+                                  size_t ws_bytes, msa_stream stream);
+
+/* Quantize `rows` bf16 rows of `cols` values (cols a multiple of 16) to
+ * E4M3 codes with one fp32 scale per row: scale = max|x| / 448 (1 for an
+ * all-zero row), code = E4M3 round-to-nearest-even of x / scale, saturated
+ * to +-448.  x [rows, cols] bf16 (in); codes [rows, cols] uint8, scale
+ * [rows] fp32 (out).  Device pointers, 16-byte aligned. */
+int msa_quantize_e4m3_rows(const msa_bf16 *x, long long rows, int cols, uint8_t *codes,
+                           float *scale, msa_stream stream);
+
 /* Decode step without a workspace argument, for callers that cannot
  * allocate device memory where they run a decode step (engines that plan all
  * device buffers at start-up and forbid allocation afterwards, plugin hosts
