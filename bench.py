@@ -44,7 +44,7 @@ BLOCK = 128
 # workload, from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum,
 # a single-pass metric set; see profiles/dram_traffic_msa_1m_and_decode_128k.md).
 # Keyed to the kernel source it was measured on: a changed kernel reports null.
-INDEX_TRAFFIC_1M = {"bytes": 8.451e10, "source_sha256_16": "ef70e999486e52cd"}
+INDEX_TRAFFIC_1M = {"bytes": 1.6911e11, "source_sha256_16": "269f1bcdede015c9"}
 
 
 def index_traffic(workload: str):
@@ -269,7 +269,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="1m", choices=["1m", "128k", "32k"],
                     help="prefill length of the step (1m is the headline workload)")
-    ap.add_argument("--op", default="step", choices=["step", "index", "attn", "decode", "cached"],
+    ap.add_argument("--op", default="step",
+                    choices=["step", "index", "attn", "decode", "decode8", "cached"],
                     help="time one operation of the step alone (profiling runs; 'cached' runs "
                          "the whole prefill as 8 msa_forward_cached chunks against the caches); "
                          "prints its own short JSON line")
@@ -345,7 +346,7 @@ def run_ours(args, shape, dshape, seed, cfg, ws_n, rank, local):
 
     # ---- inputs (device-resident for the kernel-timed leg)
     need_pre = args.op in ("step", "index", "attn", "cached")
-    need_dec = args.op in ("step", "decode")
+    need_dec = args.op in ("step", "decode", "decode8")
     if not need_pre:   # a decode-only profiling run keeps the footprint small
         import dataclasses
         shape = dataclasses.replace(shape, L=128)
@@ -477,6 +478,9 @@ def run_single_op(args, M, x, dx, dshape, K, sel, out, dout, ws_idx, ws_att, ws_
     """One operation alone, W untimed + K timed launches (profiling aid)."""
     M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx)  # the attention op needs sel
 
+    if args.op == "decode8":
+        from block_sparse_long_08_b200 import inputs as I
+        codes8, scale8 = I.fp8_index_cache(dx["k_idx_cache"])
     L = x["q"].shape[1]
     n_c = L // 8
     qc = [(x["q"][:, t0:t0 + n_c].contiguous(), x["q_idx"][:, t0:t0 + n_c].contiguous())
@@ -497,6 +501,10 @@ def run_single_op(args, M, x, dx, dshape, K, sel, out, dout, ws_idx, ws_att, ws_
             M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx)
         elif args.op == "attn":
             M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att)
+        elif args.op == "decode8":   # FP8 index-key cache
+            M.msa_sparse_attn_decode_fp8idx(dx["q"], dx["q_idx"], dx["k_cache"], dx["v_cache"],
+                                            codes8, scale8, dx["seq_lens"], dshape.top_k,
+                                            out=dout, ws=ws_dec)
         else:
             M.msa_sparse_attn_decode(dx["q"], dx["q_idx"], dx["k_cache"], dx["v_cache"],
                                      dx["k_idx_cache"], dx["seq_lens"], dshape.top_k, out=dout, ws=ws_dec)
