@@ -99,13 +99,14 @@ def prefill_attn_bytes(B, L, H, G, d, top_k):
     return entries * r * (d * 2 * 3 + 4 * 2) + B * float(L) * H * d * 2
 
 
-def decode_bytes(seq_lens, H, G, d, d_idx, top_k, fp8_index=False):
+def decode_bytes(seq_lens, H, G, d, d_idx, top_k, fp8_index=False, fp8_kv=False):
     """Bytes a decode step must read: the index-key scan over every cached
     token (bf16, or E4M3 codes + one fp32 scale per token), the selected K/V
-    tokens, and the small per-step tensors."""
+    tokens (bf16, or codes + one scale per token and head), and the small
+    per-step tensors."""
     n = np.asarray(seq_lens, dtype=np.int64)
     t = n - 1
-    kv = G * 2 * d * 2 * n_sel(t, top_k)
+    kv = G * 2 * ((d + 4) if fp8_kv else d * 2) * n_sel(t, top_k)
     scan = n * (d_idx + 4) if fp8_index else n * d_idx * 2
     small = len(n) * (H * d * 2 * 2 + G * d_idx * 2)
     return float((kv + scan).sum() + small)
@@ -540,7 +541,9 @@ def bench_decode_128k(M, I, dev, args, peaks):
     stream = torch.cuda.current_stream()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
-    codes, kscale = I.fp8_index_cache(y["k_idx_cache"])   # the same cache stored in FP8
+    codes, kscale = I.fp8_index_cache(y["k_idx_cache"])   # the same caches stored in FP8
+    k8, ks8 = I.fp8_rows(y["k_cache"])
+    v8, vs8 = I.fp8_rows(y["v_cache"])
 
     def run():
         M.msa_sparse_attn_decode(y["q"], y["q_idx"], y["k_cache"], y["v_cache"], y["k_idx_cache"], seq,
@@ -549,6 +552,10 @@ def bench_decode_128k(M, I, dev, args, peaks):
     def run_fp8():
         M.msa_sparse_attn_decode_fp8idx(y["q"], y["q_idx"], y["k_cache"], y["v_cache"], codes,
                                         kscale, seq, ds.top_k, out=out, ws=ws)
+
+    def run_all_fp8():
+        M.msa_sparse_attn_decode_fp8(y["q"], y["q_idx"], k8, ks8, v8, vs8, codes, kscale, seq,
+                                     ds.top_k, out=out, ws=ws)
 
     def timed(fn):
         for _ in range(max(3, args.warmup)):
@@ -575,17 +582,21 @@ def bench_decode_128k(M, I, dev, args, peaks):
     iters = 20
     us = timed(run)
     us8 = timed(run_fp8)
+    us88 = timed(run_all_fp8)
     lens = y["seq_lens"].numpy()
     byts = decode_bytes(lens, ds.H, ds.G, ds.d, ds.d_idx, ds.top_k)
     byts8 = decode_bytes(lens, ds.H, ds.G, ds.d, ds.d_idx, ds.top_k, fp8_index=True)
-    del y, codes, kscale
+    byts88 = decode_bytes(lens, ds.H, ds.G, ds.d, ds.d_idx, ds.top_k, fp8_index=True, fp8_kv=True)
+    del y, codes, kscale, k8, ks8, v8, vs8
     return {"us_per_step": us, "iters": iters, "batch": ds.B,
             "seq_lens": f"U[{ds.len_lo},{ds.len_hi}] seed {I.SEEDS['decode_128k']}",
             "l2": "256 MB buffer written between iterations",
             "roofline": roof(byts, us),
             "fp8_index_cache": {"us_per_step": us8, "roofline": roof(byts8, us8),
                                 "cache": "k_idx as E4M3 codes + fp32 scale per token"},
-            "gpu_launches": 8 * iters}
+            "fp8_all_caches": {"us_per_step": us88, "roofline": roof(byts88, us88),
+                               "cache": "k_idx, K and V as E4M3 codes + fp32 scales"},
+            "gpu_launches": 12 * iters}
 
 
 def bench_e2e(M, x, dx, shape, dshape, K, args, ws_n, stream):

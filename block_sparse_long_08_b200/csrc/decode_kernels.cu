@@ -466,6 +466,209 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
   }
 }
 
+// decode_attn_kernel for FP8 K/V caches: the stored key / value of token s
+// (KV head g) is scale[s,g] * E4M3(code).  Same work split as the bf16
+// kernel, with these differences:
+//   S = q K^T runs in f16 (codes convert exactly; q_idx-style d permutation
+//     over 16-code granules, see decode_index_fp8_kernel) and each key's
+//     score column is then multiplied by its K scale;
+//   V codes are converted (exactly) to bf16 on their way into shared memory,
+//     and each key's V scale is folded into P before P is packed to bf16, so
+//     the P V MMA is the bf16 one; the row sum uses the unscaled P.
+template <int R>
+__global__ void __launch_bounds__(128) decode_attn_fp8_kernel(const DecodeArgs a) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  uint16_t *sV = reinterpret_cast<uint16_t *>(dsm);
+  float *s_o = reinterpret_cast<float *>(sV + kBlock * kVPitch);   // [4 warps][R rows][128]
+  float *s_m = s_o + 4 * R * kHeadDim;                              // [4][16]
+  float *s_l = s_m + 4 * 16;                                        // [4][16]
+  const int slot = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g4 = lane >> 2, c = lane & 3;
+  const int n = a.seq_lens[b];
+  const int j = (n >= 1 && n <= a.Lmax) ? a.sel[(size_t(b) * a.G + g) * a.top_k + slot] : -1;
+  const size_t prow0 = (size_t(b) * a.H + size_t(g) * R) * a.top_k + slot;
+  if (j < 0) {
+    if (tid < R) a.part_lse[prow0 + size_t(tid) * a.top_k] = -INFINITY;
+    return;
+  }
+  const int t = n - 1;
+  const int nvis = min(kBlock, t - j * kBlock + 1);
+  const size_t tok0 = size_t(b) * a.Lmax + size_t(j) * kBlock;   // first token of the block
+  const size_t row_stride = size_t(a.G) * kHeadDim;                // codes between tokens
+  const uint8_t *kb = a.k8 + (tok0 * a.G + g) * kHeadDim;
+  const uint8_t *vb = a.v8 + (tok0 * a.G + g) * kHeadDim;
+  const float *ksb = a.k_scale + tok0 * a.G + g;                   // stride G per token
+  const float *vsb = a.v_scale + tok0 * a.G + g;
+  // V codes: 1024 granules of 16, 8 per thread, loaded now and converted
+  // into shared memory after S
+  uint4 vg[8];
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int idx = it * 128 + tid, row = idx >> 3, gran = idx & 7;
+    vg[it] = (row < nvis) ? ldg_nc_v4(vb + row * row_stride + gran * 16) : make_uint4(0, 0, 0, 0);
+  }
+  // K granules for this warp's four 8-key n-tiles (key row 8*nt + g4)
+  uint4 kg[4][2];
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const int key = warp * 32 + q4 * 8 + g4;
+    const uint8_t *kr = kb + size_t(min(key, nvis - 1)) * row_stride;
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) kg[q4][gi] = ldg_nc_v4(kr + 16 * (c + 4 * gi));
+  }
+  // scales of the keys whose S columns this lane holds: 8*nt + 2c, +1
+  float ksc[4][2], vsc[4][2];
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int key = min(warp * 32 + q4 * 8 + 2 * c + e, nvis - 1);
+      ksc[q4][e] = __ldg(ksb + size_t(key) * a.G);
+      vsc[q4][e] = __ldg(vsb + size_t(key) * a.G);
+    }
+  // q A fragments in f16 (rows g4 and g4+8; zero beyond R), permuted d
+  uint32_t qa[8][2], qb[8][2];
+  {
+    const uint16_t *q0 = a.q + (size_t(b) * a.H + size_t(g) * R + g4) * kHeadDim;
+    const uint16_t *q1 = q0 + 8 * kHeadDim;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const int d0 = 16 * (c + 4 * (kk >> 2)) + 4 * (kk & 3);
+      uint2 v0 = make_uint2(0u, 0u), v1 = make_uint2(0u, 0u);
+      if (g4 < R) v0 = *reinterpret_cast<const uint2 *>(q0 + d0);
+      if (g4 + 8 < R) v1 = *reinterpret_cast<const uint2 *>(q1 + d0);
+      qa[kk][0] = f16x2_of(bf16_lo(v0.x), bf16_hi(v0.x));
+      qa[kk][1] = f16x2_of(bf16_lo(v0.y), bf16_hi(v0.y));
+      qb[kk][0] = f16x2_of(bf16_lo(v1.x), bf16_hi(v1.x));
+      qb[kk][1] = f16x2_of(bf16_lo(v1.y), bf16_hi(v1.y));
+    }
+  }
+  float sacc[4][4];
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sacc[q4][e] = 0.f;
+#pragma unroll
+    for (int gi = 0; gi < 2; ++gi) {
+      const uint32_t wk[4] = {kg[q4][gi].x, kg[q4][gi].y, kg[q4][gi].z, kg[q4][gi].w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int kk = 4 * gi + w;
+        mma_f16_16816(sacc[q4], qa[kk][0], qb[kk][0], qa[kk][1], qb[kk][1],
+                      e4m3x2_to_f16x2(wk[w]), e4m3x2_to_f16x2(wk[w] >> 16));
+      }
+    }
+    sacc[q4][0] *= ksc[q4][0]; sacc[q4][2] *= ksc[q4][0];
+    sacc[q4][1] *= ksc[q4][1]; sacc[q4][3] *= ksc[q4][1];
+  }
+  // V codes -> bf16 rows in shared memory (rows past the query are zero)
+#pragma unroll
+  for (int it = 0; it < 8; ++it) {
+    const int idx = it * 128 + tid, row = idx >> 3, gran = idx & 7;
+    const uint32_t wv[4] = {vg[it].x, vg[it].y, vg[it].z, vg[it].w};
+    uint32_t o[8];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const uint32_t h = e4m3x2_to_f16x2(wv[w] >> (16 * hh));
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h));
+        o[2 * w + hh] = pack_bf16x2(f.x, f.y);
+      }
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(sV + row * kVPitch + gran * 16);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+  // mask keys past the query, row max over the block
+  float mx0 = -FLT_MAX, mx1 = -FLT_MAX;
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const int k0 = warp * 32 + q4 * 8 + 2 * c;
+    if (k0 >= nvis) { sacc[q4][0] = -FLT_MAX; sacc[q4][2] = -FLT_MAX; }
+    if (k0 + 1 >= nvis) { sacc[q4][1] = -FLT_MAX; sacc[q4][3] = -FLT_MAX; }
+    mx0 = fmaxf(mx0, fmaxf(sacc[q4][0], sacc[q4][1]));
+    mx1 = fmaxf(mx1, fmaxf(sacc[q4][2], sacc[q4][3]));
+  }
+#pragma unroll
+  for (int o = 1; o < 4; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+  }
+  if (c == 0) { s_m[warp * 16 + g4] = mx0; s_m[warp * 16 + g4 + 8] = mx1; }
+  __syncthreads();   // also: the staged V rows are complete
+  const float m0 = fmaxf(fmaxf(s_m[g4], s_m[16 + g4]), fmaxf(s_m[32 + g4], s_m[48 + g4]));
+  const float m1 = fmaxf(fmaxf(s_m[8 + g4], s_m[24 + g4]), fmaxf(s_m[40 + g4], s_m[56 + g4]));
+  // P = exp(scale (S - m)); the A fragments carry P * (V scale of the key)
+  uint32_t pa[2][4];
+  float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const float p0 = exp2f((sacc[q4][0] - m0) * a.scale_log2);
+    const float p1 = exp2f((sacc[q4][1] - m0) * a.scale_log2);
+    const float p2 = exp2f((sacc[q4][2] - m1) * a.scale_log2);
+    const float p3 = exp2f((sacc[q4][3] - m1) * a.scale_log2);
+    l0 += p0 + p1;
+    l1 += p2 + p3;
+    const int kt = q4 >> 1, hi = q4 & 1;
+    pa[kt][hi ? 2 : 0] = pack_bf16x2(p0 * vsc[q4][0], p1 * vsc[q4][1]);   // row g4
+    pa[kt][hi ? 3 : 1] = pack_bf16x2(p2 * vsc[q4][0], p3 * vsc[q4][1]);   // row g4 + 8
+  }
+#pragma unroll
+  for (int o = 1; o < 4; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  if (c == 0) { s_l[warp * 16 + g4] = l0; s_l[warp * 16 + g4 + 8] = l1; }
+  const uint32_t sV_u = static_cast<uint32_t>(__cvta_generic_to_shared(sV));
+  float oacc[16][4];
+#pragma unroll
+  for (int dt = 0; dt < 16; ++dt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) oacc[dt][e] = 0.f;
+#pragma unroll
+  for (int kt = 0; kt < 2; ++kt) {
+    const int key0 = warp * 32 + kt * 16;
+#pragma unroll
+    for (int dt = 0; dt < 16; dt += 2) {
+      const int mi = lane >> 3, r = lane & 7;
+      const int key = key0 + (mi & 1) * 8 + r;
+      const int d0 = (dt + (mi >> 1)) * 8;
+      uint32_t bv[4];
+      ldmatrix_x4_trans(bv, sV_u + (key * kVPitch + d0) * 2);
+      mma_bf16_16816(oacc[dt], pa[kt][0], pa[kt][1], pa[kt][2], pa[kt][3], bv[0], bv[1]);
+      mma_bf16_16816(oacc[dt + 1], pa[kt][0], pa[kt][1], pa[kt][2], pa[kt][3], bv[2], bv[3]);
+    }
+  }
+#pragma unroll
+  for (int dt = 0; dt < 16; ++dt) {
+    const int d = dt * 8 + 2 * c;
+    if (g4 < R) {
+      s_o[(warp * R + g4) * kHeadDim + d] = oacc[dt][0];
+      s_o[(warp * R + g4) * kHeadDim + d + 1] = oacc[dt][1];
+    }
+    if (g4 + 8 < R) {
+      s_o[(warp * R + g4 + 8) * kHeadDim + d] = oacc[dt][2];
+      s_o[(warp * R + g4 + 8) * kHeadDim + d + 1] = oacc[dt][3];
+    }
+  }
+  __syncthreads();
+  for (int x = tid; x < R * kHeadDim; x += 128) {
+    const int h = x / kHeadDim, d = x % kHeadDim;
+    const float l = s_l[h] + s_l[16 + h] + s_l[32 + h] + s_l[48 + h];
+    const float o = s_o[h * kHeadDim + d] + s_o[(R + h) * kHeadDim + d] +
+                    s_o[(2 * R + h) * kHeadDim + d] + s_o[(3 * R + h) * kHeadDim + d];
+    a.part_o[(prow0 + size_t(h) * a.top_k) * kHeadDim + d] = o / l;
+  }
+  if (tid < R) {
+    const int h = tid;
+    const float mh = fmaxf(fmaxf(s_m[h], s_m[16 + h]), fmaxf(s_m[32 + h], s_m[48 + h]));
+    const float l = s_l[h] + s_l[16 + h] + s_l[32 + h] + s_l[48 + h];
+    a.part_lse[prow0 + size_t(h) * a.top_k] = mh * a.scale + __logf(l);
+  }
+}
+
 __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a) {
   const int row = blockIdx.x * 8 + (threadIdx.x >> 5);  // b*H + h
   const int lane = threadIdx.x & 31;
@@ -502,10 +705,10 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a)
 template <int R>
 cudaError_t launch_decode_attn(const DecodeArgs &a, cudaStream_t st) {
   constexpr int smem = dec_attn_smem<R>();
-  cudaError_t e = cudaFuncSetAttribute(decode_attn_kernel<R>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  auto kern = a.k8 ? decode_attn_fp8_kernel<R> : decode_attn_kernel<R>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  decode_attn_kernel<R><<<dim3(a.top_k, a.G, a.B), 128, smem, st>>>(a);
+  kern<<<dim3(a.top_k, a.G, a.B), 128, smem, st>>>(a);
   return cudaGetLastError();
 }
 

@@ -88,6 +88,10 @@ struct DecodeArgs {
   // E4M3 codes [B,Lmax,d_idx] and one fp32 scale per token [B,Lmax]
   const uint8_t *k_idx8;
   const float *k_idx_scale;
+  // FP8 K/V caches (when non-null, used instead of k_cache / v_cache): E4M3
+  // codes [B,Lmax,G,d] and one fp32 scale per (token, KV head) [B,Lmax,G]
+  const uint8_t *k8, *v8;
+  const float *k_scale, *v_scale;
   const int32_t *seq_lens;
   float *scores;               // [B,G,nb_max]
   int32_t *sel;                // [B,G,top_k]

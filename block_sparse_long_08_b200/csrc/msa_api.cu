@@ -374,20 +374,37 @@ int host_events(HostEvents **out) {
   return MSA_OK;
 }
 
-// Decode step with the index-key cache in bf16 (k_idx_cache) or in FP8
-// (k_idx8 + k_idx_scale); exactly one of the two is given.
+// FP8 caches of a decode step: E4M3 codes with their scales (null: bf16).
+struct Fp8Caches {
+  const uint8_t *k_idx8 = nullptr;
+  const float *k_idx_scale = nullptr;
+  const uint8_t *k8 = nullptr, *v8 = nullptr;
+  const float *k_scale = nullptr, *v_scale = nullptr;
+};
+
+// Decode step.  The index-key cache is bf16 (k_idx_cache) or FP8
+// (f8.k_idx8 + scale); K/V are bf16 (k_cache, v_cache) or FP8 (f8.k8/v8 +
+// scales).
 int run_decode(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
                const msa_bf16 *k_cache, const msa_bf16 *v_cache, const msa_bf16 *k_idx_cache,
-               const uint8_t *k_idx8, const float *k_idx_scale, const int32_t *seq_lens,
-               msa_bf16 *out, int32_t *sel, void *ws, size_t ws_bytes, cudaStream_t st) {
+               const Fp8Caches &f8, const int32_t *seq_lens, msa_bf16 *out, int32_t *sel,
+               void *ws, size_t ws_bytes, cudaStream_t st) {
+  const uint8_t *k_idx8 = f8.k_idx8;
+  const float *k_idx_scale = f8.k_idx_scale;
   int rc = check_params(p, true);
   if (rc) return rc;
   if (p->B == 0) return MSA_OK;
   if (p->L == 0) return fail(MSA_ERR_INVALID_ARG, "decode needs a cache (L = Lmax > 0)");
-  if (!q || !q_idx || !k_cache || !v_cache || !seq_lens || !out || (!k_idx_cache && !k_idx8) ||
-      (k_idx8 && !k_idx_scale))
+  const bool kv8 = f8.k8 != nullptr;
+  if (!q || !q_idx || !seq_lens || !out || (!k_idx_cache && !k_idx8) || (k_idx8 && !k_idx_scale) ||
+      (!kv8 && (!k_cache || !v_cache)) ||
+      (kv8 && (!f8.v8 || !f8.k_scale || !f8.v_scale)))
     return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
-  if (!aligned16(q) || !aligned16(q_idx) || !aligned16(k_cache) || !aligned16(v_cache) ||
+  auto al4 = [](const void *ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; };
+  if (kv8 && (!aligned16(f8.k8) || !aligned16(f8.v8) || !al4(f8.k_scale) || !al4(f8.v_scale)))
+    return fail(MSA_ERR_INVALID_ARG, "FP8 caches must be 16-byte aligned (scales 4-byte)");
+  if (!aligned16(q) || !aligned16(q_idx) || (k_cache && !aligned16(k_cache)) ||
+      (v_cache && !aligned16(v_cache)) ||
       (k_idx_cache && !aligned16(k_idx_cache)) || (k_idx8 && !aligned16(k_idx8)) ||
       (k_idx_scale && (reinterpret_cast<uintptr_t>(k_idx_scale) & 3u)) || !aligned16(out) ||
       (sel && !aligned16(sel)))
@@ -403,6 +420,7 @@ int run_decode(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
   a.scale_log2 = a.scale * 1.4426950408889634f;
   a.q = q; a.q_idx = q_idx; a.k_cache = k_cache; a.v_cache = v_cache; a.k_idx_cache = k_idx_cache;
   a.k_idx8 = k_idx8; a.k_idx_scale = k_idx_scale;
+  a.k8 = f8.k8; a.v8 = f8.v8; a.k_scale = f8.k_scale; a.v_scale = f8.v_scale;
   a.seq_lens = seq_lens;
   a.scores = reinterpret_cast<float *>(wsb + w.scores);
   a.sel = sel ? sel : reinterpret_cast<int32_t *>(wsb + w.sel);
@@ -625,8 +643,8 @@ int msa_sparse_attn_decode(const msa_params *p, const msa_bf16 *q, const msa_bf1
                            const msa_bf16 *k_idx_cache, const int32_t *seq_lens, msa_bf16 *out,
                            int32_t *sel, void *ws, size_t ws_bytes, msa_stream stream) {
   g_err[0] = 0;
-  return run_decode(p, q, q_idx, k_cache, v_cache, k_idx_cache, nullptr, nullptr, seq_lens, out,
-                    sel, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+  return run_decode(p, q, q_idx, k_cache, v_cache, k_idx_cache, Fp8Caches{}, seq_lens, out, sel,
+                    ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int msa_sparse_attn_decode_fp8idx(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
@@ -636,8 +654,29 @@ int msa_sparse_attn_decode_fp8idx(const msa_params *p, const msa_bf16 *q, const 
                                   size_t ws_bytes, msa_stream stream) {
   g_err[0] = 0;
   if (!k_idx8) return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
-  return run_decode(p, q, q_idx, k_cache, v_cache, nullptr, k_idx8, k_idx_scale, seq_lens, out,
-                    sel, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+  Fp8Caches f8;
+  f8.k_idx8 = k_idx8;
+  f8.k_idx_scale = k_idx_scale;
+  return run_decode(p, q, q_idx, k_cache, v_cache, nullptr, f8, seq_lens, out, sel, ws, ws_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+int msa_sparse_attn_decode_fp8(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
+                               const uint8_t *k8, const float *k_scale, const uint8_t *v8,
+                               const float *v_scale, const uint8_t *k_idx8,
+                               const float *k_idx_scale, const int32_t *seq_lens, msa_bf16 *out,
+                               int32_t *sel, void *ws, size_t ws_bytes, msa_stream stream) {
+  g_err[0] = 0;
+  if (!k_idx8 || !k8) return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  Fp8Caches f8;
+  f8.k_idx8 = k_idx8;
+  f8.k_idx_scale = k_idx_scale;
+  f8.k8 = k8;
+  f8.v8 = v8;
+  f8.k_scale = k_scale;
+  f8.v_scale = v_scale;
+  return run_decode(p, q, q_idx, nullptr, nullptr, nullptr, f8, seq_lens, out, sel, ws, ws_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 int msa_quantize_e4m3_rows(const msa_bf16 *x, long long rows, int cols, uint8_t *codes,

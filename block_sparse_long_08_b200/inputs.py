@@ -134,11 +134,17 @@ def decode_inputs(shape: DecodeShape, seed: int, device="cpu") -> dict:
 
 def fp8_index_cache(k_idx_cache: torch.Tensor) -> tuple:
     """An FP8 index-key cache holding the given bf16 cache [B,Lmax,d_idx]:
-    E4M3 codes (uint8, same shape) and one fp32 scale per token [B,Lmax],
-    scale = max|row| / 448, codes = the row divided by its scale, rounded to
-    E4M3 by torch's float8_e4m3fn conversion.  (Input preparation: the
-    method consumes codes and scales as given.)"""
-    x = k_idx_cache.float()
+    E4M3 codes (uint8, same shape) and one fp32 scale per token [B,Lmax]
+    (fp8_rows of it)."""
+    return fp8_rows(k_idx_cache)
+
+
+def fp8_rows(t: torch.Tensor) -> tuple:
+    """E4M3 codes of a bf16 tensor [..., D] with one fp32 scale per row
+    [...]: scale = max|row| / 448, codes = the row divided by its scale,
+    rounded to E4M3 by torch's float8_e4m3fn conversion.  (Input
+    preparation: the method consumes codes and scales as given.)"""
+    x = t.float()
     amax = x.abs().amax(dim=-1)
     scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
     codes = (x / scale[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)

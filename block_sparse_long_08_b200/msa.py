@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.msa_sparse_attn_decode_fp8idx.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ,
                                                     _P]
         L.msa_quantize_e4m3_rows.argtypes = [_P, ctypes.c_longlong, ctypes.c_int, _P, _P, _P]
+        L.msa_sparse_attn_decode_fp8.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                                 _P, _SZ, _P]
         L.msa_sparse_attn_decode_noalloc.restype = ctypes.c_int
         L.msa_workspace_bytes.argtypes = [pp, ctypes.c_int]
         L.msa_workspace_bytes.restype = _SZ
@@ -89,7 +91,8 @@ def lib() -> ctypes.CDLL:
         L.msa_version.restype = ctypes.c_char_p
         for f in ("msa_index_select", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
                   "msa_forward", "msa_forward_host", "msa_forward_cached", "msa_read_status",
-                  "msa_sparse_attn_decode_fp8idx", "msa_quantize_e4m3_rows"):
+                  "msa_sparse_attn_decode_fp8idx", "msa_quantize_e4m3_rows",
+                  "msa_sparse_attn_decode_fp8"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -356,6 +359,34 @@ def msa_sparse_attn_decode_fp8idx(q, q_idx, k_cache, v_cache, k_idx8, k_idx_scal
                                                _ptr(v_cache), _ptr(k_idx8), _ptr(k_idx_scale),
                                                _ptr(seq_lens), _ptr(out), _ptr(sel), _ptr(ws),
                                                ws.numel(), _stream(stream)))
+    return (out, sel) if want_sel else out
+
+
+def msa_sparse_attn_decode_fp8(q, q_idx, k8, k_scale, v8, v_scale, k_idx8, k_idx_scale,
+                               seq_lens, top_k: int, *, scale: float = 0.0, want_sel: bool = False,
+                               out=None, sel=None, ws=None, stream=None):
+    """Decode step with every cache in FP8: k8/v8 [B,Lmax,G,d] uint8 E4M3 with
+    k_scale/v_scale [B,Lmax,G] fp32, k_idx8 [B,Lmax,d_idx] with k_idx_scale [B,Lmax]."""
+    _req(q, "q", torch.bfloat16)
+    _req(q_idx, "q_idx", torch.bfloat16)
+    for n_, t in (("k8", k8), ("v8", v8), ("k_idx8", k_idx8)):
+        _req(t, n_, torch.uint8)
+    for n_, t in (("k_scale", k_scale), ("v_scale", v_scale), ("k_idx_scale", k_idx_scale)):
+        _req(t, n_, torch.float32)
+    _req(seq_lens, "seq_lens", torch.int32)
+    B, H, d = q.shape
+    Lmax, G = k8.shape[1], k8.shape[2]
+    p = make_params(B, Lmax, H, G, d, k_idx8.shape[2], 128, top_k, scale)
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    if sel is None and want_sel:
+        sel = torch.empty((B, G, top_k), dtype=torch.int32, device=dev)
+    ws = _ensure_ws(ws, p, MSA_OP_DECODE, dev)
+    _check(lib().msa_sparse_attn_decode_fp8(ctypes.byref(p), _ptr(q), _ptr(q_idx), _ptr(k8),
+                                            _ptr(k_scale), _ptr(v8), _ptr(v_scale), _ptr(k_idx8),
+                                            _ptr(k_idx_scale), _ptr(seq_lens), _ptr(out),
+                                            _ptr(sel), _ptr(ws), ws.numel(), _stream(stream)))
     return (out, sel) if want_sel else out
 
 

@@ -157,6 +157,22 @@ int msa_sparse_attn_decode_fp8idx(const msa_params *p, const msa_bf16 *q, const 
                                   const int32_t *seq_lens, msa_bf16 *out, int32_t *sel, void *ws,
                                   size_t ws_bytes, msa_stream stream);
 
+/* Decode step with every cache in FP8: the index keys as in
+ * msa_sparse_attn_decode_fp8idx, and the keys and values as E4M3 codes
+ * with one fp32 scale per (token, KV head): the stored key of token s,
+ * head g is k_scale[s,g] * E4M3(k8[s,g,:]), likewise for values.
+ *   k8, v8 [B,Lmax,G,d] uint8 E4M3 codes, 16-byte aligned             (in)
+ *   k_scale, v_scale [B,Lmax,G] fp32                                    (in)
+ *   k_idx8 [B,Lmax,d_idx] uint8, k_idx_scale [B,Lmax] fp32              (in)
+ * The main branch's scores run in f16 (q must lie within the f16 range);
+ * each value's scale is folded into its softmax weight before the weights
+ * are rounded to bf16 for the P V product. */
+int msa_sparse_attn_decode_fp8(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
+                               const uint8_t *k8, const float *k_scale, const uint8_t *v8,
+                               const float *v_scale, const uint8_t *k_idx8,
+                               const float *k_idx_scale, const int32_t *seq_lens, msa_bf16 *out,
+                               int32_t *sel, void *ws, size_t ws_bytes, msa_stream stream);
+
 /* Quantize `rows` bf16 rows of `cols` values (cols a multiple of 16) to
  * E4M3 codes with one fp32 scale per row: scale = max|x| / 448 (1 for an
  * all-zero row), code = E4M3 round-to-nearest-even of x / scale, saturated

@@ -1,4 +1,5 @@
-"""GPU tests of the FP8 index-key cache for decode (msa_sparse_attn_decode_fp8idx)
+"""GPU tests of the FP8 caches for decode (msa_sparse_attn_decode_fp8idx: index
+keys in FP8; msa_sparse_attn_decode_fp8: index keys, keys and values in FP8)
 and of the row quantizer (msa_quantize_e4m3_rows).
 
 The oracle reads the same E4M3 codes and per-token scales, decoded by its own
@@ -95,3 +96,43 @@ def test_fp8idx_integer_codes_select_bit_exact():
             bs = O.block_scores_row(q64[b, g], k64[b], t, 128)
             want = O.select_blocks_row(bs, t, 128, 6)
             assert list(sel[b, g]) == want + [-1] * (6 - len(want)), (b, g, sel[b, g], want)
+
+
+@pytest.mark.parametrize("B,Lmax,G,H,di,top_k,lens", [
+    (4, 4096, 8, 32, 128, 16, [4096, 1, 129, 3000]),
+    (5, 2048, 2, 8, 64, 4, [2048, 128, 127, 777, 1500]),
+    (2, 1024, 1, 16, 128, 3, [1024, 300]),
+])
+def test_all_fp8_decode_matches_oracle(B, Lmax, G, H, di, top_k, lens):
+    shape = I.DecodeShape(B=B, Lmax=Lmax, H=H, G=G, d=128, d_idx=di, top_k=top_k)
+    x = I.decode_inputs(shape, 56)
+    ki8, kis = I.fp8_rows(x["k_idx_cache"])
+    k8, ks = I.fp8_rows(x["k_cache"])
+    v8, vs = I.fp8_rows(x["v_cache"])
+    # garbage past each sequence's length, including NaN codes: never read
+    for b, n in enumerate(lens):
+        for t in (ki8, k8, v8):
+            t[b, n:] = 0x7F
+    dv = lambda t: t.to(DEV)
+    out, sel = M.msa_sparse_attn_decode_fp8(dv(x["q"]), dv(x["q_idx"]), dv(k8), dv(ks), dv(v8),
+                                            dv(vs), dv(ki8), dv(kis),
+                                            torch.tensor(lens, dtype=torch.int32, device=DEV),
+                                            top_k, want_sel=True)
+    torch.cuda.synchronize()
+    kd = O.dequant_rows(k8.numpy(), ks.numpy())
+    vd = O.dequant_rows(v8.numpy(), vs.numpy())
+    kid = O.dequant_rows(ki8.numpy(), kis.numpy())
+    ref = O.decode(x["q"], x["q_idx"], kd, vd, kid, lens, top_k)
+    sel_c = sel.cpu().numpy()
+    qi = P.f64(x["q_idx"])
+    any_swap = False
+    for b in range(B):
+        t = lens[b] - 1
+        for g in range(G):
+            bs = O.block_scores_row(qi[b, g], kid[b], t, 128)
+            if not P.check_selection_row(sel_c[b, g], ref["sel"][b, g], bs, t, top_k):
+                any_swap = True
+    if any_swap:
+        ref = O.decode(x["q"], x["q_idx"], kd, vd, kid, lens, top_k, sel_override=sel_c)
+    mx, mean = P.out_errors(out.float().cpu().numpy(), ref["out"])
+    assert mx <= P.OUT_MAX_ABS and mean <= P.OUT_MEAN_ABS, (mx, mean)
