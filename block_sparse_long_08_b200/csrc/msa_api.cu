@@ -567,6 +567,40 @@ int msa_forward_cached(const msa_params *p, int t0, int n, const msa_bf16 *q,
   return run_prefill_attn(p, q, k_cache, v_cache, s, out, lse, ws, base, st, qg);
 }
 
+int msa_forward_cached_varlen(const msa_params *p, const int32_t *t0, const int32_t *n,
+                              const msa_bf16 *q, const msa_bf16 *q_idx, const msa_bf16 *k_cache,
+                              const msa_bf16 *v_cache, const msa_bf16 *k_idx_cache,
+                              msa_bf16 *out, float *lse, void *ws, size_t ws_bytes,
+                              msa_stream stream) {
+  g_err[0] = 0;
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (p->B == 0) return MSA_OK;
+  if (!t0 || !n) return fail(MSA_ERR_INVALID_ARG, "NULL t0 or n (host arrays)");
+  for (int b = 0; b < p->B; ++b)
+    if (t0[b] < 0 || n[b] < 0 || t0[b] % 128 || n[b] % 128 || (long long)t0[b] + n[b] > p->L)
+      return fail(MSA_ERR_INVALID_ARG, "sequence %d: t0=%d n=%d (multiples of 128, t0+n <= L=%d)",
+                  b, t0[b], n[b], p->L);
+  msa_params p1 = *p;
+  p1.B = 1;
+  const size_t kv_rows = size_t(p->L);   // cache rows per sequence
+  long long row0 = 0;
+  for (int b = 0; b < p->B; ++b) {
+    if (n[b] > 0) {
+      rc = msa_forward_cached(&p1, t0[b], n[b], q + size_t(row0) * p->H * p->d,
+                              q_idx + size_t(row0) * p->G * p->d_idx,
+                              k_cache + size_t(b) * kv_rows * p->G * p->d,
+                              v_cache + size_t(b) * kv_rows * p->G * p->d,
+                              k_idx_cache + size_t(b) * kv_rows * p->d_idx,
+                              out + size_t(row0) * p->H * p->d, nullptr,
+                              lse ? lse + size_t(row0) * p->H : nullptr, ws, ws_bytes, stream);
+      if (rc) return rc;
+    }
+    row0 += n[b];
+  }
+  return MSA_OK;
+}
+
 int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k_h,
                      const msa_bf16 *v_h, const msa_bf16 *q_idx_h, const msa_bf16 *k_idx_h,
                      msa_bf16 *out_h, float *lse_h, const msa_staging *dev, void *ws,

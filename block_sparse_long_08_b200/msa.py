@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.msa_forward.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.msa_forward_cached.argtypes = [pp, ctypes.c_int, ctypes.c_int, _P, _P, _P, _P, _P, _P, _P,
                                          _P, _P, _SZ, _P]
+        L.msa_forward_cached_varlen.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ,
+                                                _P]
         L.msa_forward_host.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P,
                                        ctypes.POINTER(msa_staging), _P, _SZ, _P, _P]
         L.msa_sparse_attn_decode_noalloc.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P]
@@ -92,7 +94,7 @@ def lib() -> ctypes.CDLL:
         for f in ("msa_index_select", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
                   "msa_forward", "msa_forward_host", "msa_forward_cached", "msa_read_status",
                   "msa_sparse_attn_decode_fp8idx", "msa_quantize_e4m3_rows",
-                  "msa_sparse_attn_decode_fp8"):
+                  "msa_sparse_attn_decode_fp8", "msa_forward_cached_varlen"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -260,6 +262,36 @@ def msa_forward_cached(q, q_idx, k_cache, v_cache, k_idx_cache, t0: int, top_k: 
     if want_lse:
         res.append(lse)
     return res[0] if len(res) == 1 else tuple(res)
+
+
+def msa_forward_cached_varlen(q, q_idx, k_cache, v_cache, k_idx_cache, t0, n, top_k: int, *,
+                              scale: float = 0.0, want_lse: bool = False, out=None, ws=None,
+                              stream=None, chunk: int = 0):
+    """Ragged batch of cached prefills: sequence b continues at position t0[b]
+    with n[b] new tokens whose query rows are packed in q [sum n,H,d] and
+    q_idx [sum n,G,d_idx]; caches [B,Lmax,...].  Returns out [sum n,H,d]
+    (and lse [sum n,H])."""
+    for n_, t in (("q", q), ("q_idx", q_idx), ("k_cache", k_cache), ("v_cache", v_cache),
+                  ("k_idx_cache", k_idx_cache)):
+        _req(t, n_, torch.bfloat16)
+    B, Lmax, G = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
+    H, d = q.shape[1], q.shape[2]
+    t0a = (ctypes.c_int32 * B)(*[int(v) for v in t0])
+    na = (ctypes.c_int32 * B)(*[int(v) for v in n])
+    if sum(int(v) for v in n) != q.shape[0]:
+        raise ValueError("q rows must equal sum(n)")
+    p = make_params(B, Lmax, H, G, d, q_idx.shape[2], 128, top_k, scale, chunk)
+    p1 = make_params(1, Lmax, H, G, d, q_idx.shape[2], 128, top_k, scale, chunk)
+    dev = q.device
+    if out is None:
+        out = torch.empty_like(q)
+    lse = torch.empty((q.shape[0], H), dtype=torch.float32, device=dev) if want_lse else None
+    ws = _ensure_ws(ws, p1, MSA_OP_FORWARD, dev)
+    _check(lib().msa_forward_cached_varlen(ctypes.byref(p), t0a, na, _ptr(q), _ptr(q_idx),
+                                           _ptr(k_cache), _ptr(v_cache), _ptr(k_idx_cache),
+                                           _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                           _stream(stream)))
+    return (out, lse) if want_lse else out
 
 
 def _req_host(t: torch.Tensor, name: str, dtype) -> torch.Tensor:

@@ -230,6 +230,25 @@ int msa_forward_cached(const msa_params *p, int t0, int n, const msa_bf16 *q,
                        const msa_bf16 *k_idx_cache, msa_bf16 *out, int32_t *sel, float *lse,
                        void *ws, size_t ws_bytes, msa_stream stream);
 
+/* msa_forward_cached for a batch whose sequences continue at different
+ * positions with different numbers of new tokens (a ragged serving batch).
+ * The new tokens' query rows are packed: sequence b owns rows
+ * [row0_b, row0_b + n[b]) with row0_b = n[0] + ... + n[b-1].
+ *   t0[B], n[B]: HOST int32 arrays; every t0[b] and n[b] a multiple of 128,
+ *     t0[b] + n[b] <= Lmax (n[b] may be 0)
+ *   q [sum n, H, d], q_idx [sum n, G, d_idx] bf16 (packed)              (in)
+ *   k_cache, v_cache [B,Lmax,G,d], k_idx_cache [B,Lmax,d_idx]            (in)
+ *   out [sum n, H, d] bf16 (packed); lse [sum n, H] fp32 or NULL        (out)
+ *   ws >= msa_workspace_bytes(p, MSA_OP_FORWARD) with p->B = 1
+ * Sequences are processed one after another on `stream`, each exactly as
+ * msa_forward_cached with B = 1.  (Kernels that take the whole ragged
+ * batch in one launch are not built.) */
+int msa_forward_cached_varlen(const msa_params *p, const int32_t *t0, const int32_t *n,
+                              const msa_bf16 *q, const msa_bf16 *q_idx, const msa_bf16 *k_cache,
+                              const msa_bf16 *v_cache, const msa_bf16 *k_idx_cache,
+                              msa_bf16 *out, float *lse, void *ws, size_t ws_bytes,
+                              msa_stream stream);
+
 /* Device buffers that msa_forward_host stages its transfers in: the device
  * counterparts of msa_forward's tensors (caller-owned, 16-byte aligned).
  * lse may be NULL when no lse is requested. */

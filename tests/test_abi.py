@@ -124,6 +124,16 @@ def test_cached_prefill_rejects_bad_ranges(t0, n):
     assert rc == M.MSA_ERR_INVALID_ARG, (rc, M.msa_last_error())
 
 
+def test_varlen_rejects_bad_ranges():
+    p = M.make_params(2, 4096, 8, 2, 128, 64, 128, 4)
+    ok = ctypes.c_void_p(4096)
+    for t0, n in (([0, 100], [128, 128]), ([0, 3968], [128, 256]), ([-128, 0], [128, 128])):
+        rc = M.lib().msa_forward_cached_varlen(ctypes.byref(p), (ctypes.c_int32 * 2)(*t0),
+                                               (ctypes.c_int32 * 2)(*n), ok, ok, ok, ok, ok, ok,
+                                               None, ok, 1 << 30, None)
+        assert rc == M.MSA_ERR_INVALID_ARG, (t0, n, M.msa_last_error())
+
+
 def test_decode_rejects_more_than_eight_groups():
     p = M.make_params(2, 4096, 32, 16, 128, 128, 128, 16)
     assert M.lib().msa_workspace_bytes(ctypes.byref(p), M.MSA_OP_DECODE) == 0

@@ -77,3 +77,28 @@ def test_cached_prefill_against_oracle():
             errs.append(np.abs(out_c[b, t - t0, g * r:(g + 1) * r] - o_ref))
     e = np.concatenate([v.ravel() for v in errs])
     assert e.max() <= P.OUT_MAX_ABS and e.mean() <= P.OUT_MEAN_ABS, (e.max(), e.mean())
+
+
+def test_ragged_batch_equals_whole_sequence_rows(full_run):
+    """Sequences continuing at different positions with different numbers of
+    new tokens (one with none), query rows packed."""
+    shape, x, out, sel, lse = full_run
+    t0, n = [1024, 2944], [768, 1152]
+    t0, n = t0 + [0], n + [0]          # a third sequence with no new tokens
+    B = 2
+    q = torch.cat([x["q"][b, t0[b]:t0[b] + n[b]] for b in range(B)])
+    q_idx = torch.cat([x["q_idx"][b, t0[b]:t0[b] + n[b]] for b in range(B)])
+    o_c, l_c = M.msa_forward_cached_varlen(q, q_idx, x["k"], x["v"], x["k_idx"], t0[:B], n[:B],
+                                           shape.top_k, want_lse=True)
+    torch.cuda.synchronize()
+    want_o = torch.cat([out[b, t0[b]:t0[b] + n[b]] for b in range(B)])
+    want_l = torch.cat([lse[b, t0[b]:t0[b] + n[b]] for b in range(B)])
+    assert torch.equal(o_c, want_o)
+    assert torch.equal(l_c, want_l)
+    # an empty sequence in the batch
+    k3 = torch.cat([x["k"], x["k"][:1]])
+    v3 = torch.cat([x["v"], x["v"][:1]])
+    ki3 = torch.cat([x["k_idx"], x["k_idx"][:1]])
+    o3 = M.msa_forward_cached_varlen(q, q_idx, k3, v3, ki3, t0, n, shape.top_k)
+    torch.cuda.synchronize()
+    assert torch.equal(o3, want_o)
