@@ -19,9 +19,9 @@
 // of partials go out, against 0.5 us of tensor work.  The kernel is built to
 // keep those transfers in flight (one persistent CTA per SM, 16 warps with
 // fixed roles):
-//   warp 0     K/V producer: TMA loads of K_j and V_j into a ring of four
-//              32 KB tiles, once per run of consecutive items with the same
-//              key block (items are ordered by (b, g, j)).
+//   warp 0     K/V producer: TMA loads of K_j and V_j into a ring of 32 KB
+//              tiles, once per run of consecutive items with the same key
+//              block (items are ordered by (b, g, j)).
 //   warp 1     TMEM owner and MMA issuer: issues S_i and O_i in whatever
 //              order their inputs become ready (non-blocking barrier probes).
 //   warps 2-7  three gather groups of 64 threads; group k owns shared stage
@@ -33,8 +33,9 @@
 //              128-column TMEM slot (S, then O).  After the softmax a group
 //              loads O, stages the bf16 partial rows in the item's stage and
 //              writes them with one bulk copy.
-// A stage holds Q, then P, then the staged partial of one item; three stages
-// let the q gather of item i+3 start as soon as item i's partial has left.
+// A stage holds Q, then P, then the staged partial of one item; with NQ
+// stages the q gather of item i+NQ starts as soon as item i's partial has
+// left.  Seven 32 KB tiles are split between stages and K/V tiles (AttnCfg).
 //
 // Partial layout.  The partials of a chunk are indexed by reverse-index list
 // position: the entry at position pos (query t, slot k of group g) owns rows
@@ -56,32 +57,39 @@ namespace msa {
 namespace {
 
 constexpr int kAttnThreads = 512;
-constexpr int kNQ = 3;                               // Q/P/partial stages
-constexpr int kNKV = 4;                              // K/V tiles: two runs in flight
 constexpr int kTile = 32768;                         // 128 rows x 256 B
-constexpr int kSmemQ = 0;
-constexpr int kSmemKV = kNQ * kTile;
-constexpr int kSmemCtl = kSmemKV + kNKV * kTile;     // 229376
-// mbarrier slots (8 bytes each) at kSmemCtl
-constexpr int kBarQFull = 0;                         // [kNQ]  gather team copies + list
-constexpr int kBarStEmpty = kBarQFull + kNQ;         // [kNQ]  four storing warps
-constexpr int kBarKvFull = kBarStEmpty + kNQ;        // [kNKV] TMA transaction bytes
-constexpr int kBarKvEmpty = kBarKvFull + kNKV;       // [kNKV] UMMA commit
-constexpr int kBarSFull = kBarKvEmpty + kNKV;        // [2]    UMMA commit
-constexpr int kBarPFull = kBarSFull + 2;             // [2]    128 softmax threads
-constexpr int kBarOFull = kBarPFull + 2;             // [2]    UMMA commit
-constexpr int kBarTmEmpty = kBarOFull + 2;           // [2]    128 softmax threads
-constexpr int kBarDrain = kBarTmEmpty + 2;           // UMMA commit on the way out
-constexpr int kNumBars = kBarDrain + 1;              // 23
-constexpr int kCtlMisc = kNumBars * 8;               // tmem holder, abort flag
-constexpr int kCtlDesc = 192;                        // [kNQ] int4 {bgj, start, n, -}
-constexpr int kCtlPre = kCtlDesc + 16 * kNQ;         // int4: the gather team's next item
-constexpr int kCtlList = kCtlPre + 48;               // [kNQ][128] list entries
-constexpr int kCtlBytes = kCtlList + kNQ * 128 * 4;
-constexpr int kAttnSmem = kSmemCtl + kCtlBytes + 1024;  // + alignment slack
-static_assert(kCtlMisc + 8 <= kCtlDesc, "control layout");
-static_assert(kCtlPre + 48 <= kCtlList, "control layout");
-static_assert(kAttnSmem <= 232448, "shared memory budget");
+
+// Shared-memory plan per head ratio R.  Seven 32 KB tiles: NQ Q/P/partial
+// stages and NKV K/V tiles.  Four stages (with three K/V tiles, enough when
+// items of one key block come in runs) for R >= 2; for R = 1 the 128-entry
+// item lists leave room for three stages only, with four K/V tiles.
+template <int R>
+struct AttnCfg {
+  static constexpr int QPI = 128 / R;                 // queries per item
+  static constexpr int NQ = (R == 1) ? 3 : 4;
+  static constexpr int NKV = 7 - NQ;
+  static constexpr int SMEM_Q = 0;
+  static constexpr int SMEM_KV = NQ * kTile;
+  static constexpr int SMEM_CTL = SMEM_KV + NKV * kTile;   // 229376
+  // mbarrier slots (8 bytes each) at SMEM_CTL
+  static constexpr int BAR_QFULL = 0;                 // [NQ]  gather team copies + list
+  static constexpr int BAR_STEMPTY = NQ;              // [NQ]  four storing warps
+  static constexpr int BAR_KVFULL = 2 * NQ;           // [NKV] TMA transaction bytes
+  static constexpr int BAR_KVEMPTY = 2 * NQ + NKV;    // [NKV] UMMA commit
+  static constexpr int BAR_SFULL = 2 * NQ + 2 * NKV;  // [2]   UMMA commit
+  static constexpr int BAR_PFULL = BAR_SFULL + 2;     // [2]   128 softmax threads
+  static constexpr int BAR_OFULL = BAR_PFULL + 2;     // [2]   UMMA commit
+  static constexpr int BAR_TMEMPTY = BAR_OFULL + 2;   // [2]   128 softmax threads
+  static constexpr int BAR_DRAIN = BAR_TMEMPTY + 2;   // UMMA commit on the way out
+  static constexpr int NUM_BARS = BAR_DRAIN + 1;
+  static constexpr int CTL_MISC = NUM_BARS * 8;       // tmem holder, abort flag
+  static constexpr int CTL_DESC = (CTL_MISC + 8 + 15) & ~15;   // [NQ] int4 {bgj, start, n, -}
+  static constexpr int CTL_PRE = CTL_DESC + 16 * NQ;  // int4: the gather team's next item
+  static constexpr int CTL_LIST = CTL_PRE + 16;       // [NQ][QPI] list entries
+  static constexpr int CTL_BYTES = CTL_LIST + NQ * QPI * 4;
+  static constexpr int SMEM = SMEM_CTL + CTL_BYTES + 1024;   // + alignment slack
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
 
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
@@ -175,39 +183,40 @@ template <int R>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     msa_prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
-  constexpr int QPI = 128 / R;
+  using C = AttnCfg<R>;
+  constexpr int QPI = C::QPI;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
   const uint32_t s_base = smem_u32(smem);
-  uint8_t *ctl = smem + kSmemCtl;
+  uint8_t *ctl = smem + C::SMEM_CTL;
   const uint32_t bar0 = smem_u32(ctl);
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(ctl + kCtlMisc);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctl + kCtlMisc + 4);
-  int4 *s_desc = reinterpret_cast<int4 *>(ctl + kCtlDesc);
-  int4 *s_pre = reinterpret_cast<int4 *>(ctl + kCtlPre);
-  int *s_list = reinterpret_cast<int *>(ctl + kCtlList);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(ctl + C::CTL_MISC);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(ctl + C::CTL_MISC + 4);
+  int4 *s_desc = reinterpret_cast<int4 *>(ctl + C::CTL_DESC);
+  int4 *s_pre = reinterpret_cast<int4 *>(ctl + C::CTL_PRE);
+  int *s_list = reinterpret_cast<int *>(ctl + C::CTL_LIST);
   auto bar = [&](int idx) { return bar0 + 8u * uint32_t(idx); };
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
   if (tid == 0) {
-    for (int s = 0; s < kNQ; ++s) {
-      mbar_init(bar(kBarQFull + s), 193);   // 192 copy completions + the list
-      mbar_init(bar(kBarStEmpty + s), 4);   // the four softmax warps' stores
+    for (int s = 0; s < C::NQ; ++s) {
+      mbar_init(bar(C::BAR_QFULL + s), 193);   // 192 copy completions + the list
+      mbar_init(bar(C::BAR_STEMPTY + s), 4);   // the four softmax warps' stores
     }
-    for (int x = 0; x < kNKV; ++x) {
-      mbar_init(bar(kBarKvFull + x), 1);
-      mbar_init(bar(kBarKvEmpty + x), 1);
+    for (int x = 0; x < C::NKV; ++x) {
+      mbar_init(bar(C::BAR_KVFULL + x), 1);
+      mbar_init(bar(C::BAR_KVEMPTY + x), 1);
     }
     for (int u = 0; u < 2; ++u) {
-      mbar_init(bar(kBarSFull + u), 1);
-      mbar_init(bar(kBarPFull + u), 128);
-      mbar_init(bar(kBarOFull + u), 1);
-      mbar_init(bar(kBarTmEmpty + u), 128);
+      mbar_init(bar(C::BAR_SFULL + u), 1);
+      mbar_init(bar(C::BAR_PFULL + u), 128);
+      mbar_init(bar(C::BAR_OFULL + u), 1);
+      mbar_init(bar(C::BAR_TMEMPTY + u), 128);
     }
-    mbar_init(bar(kBarDrain), 1);
+    mbar_init(bar(C::BAR_DRAIN), 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -238,7 +247,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tma_prefetch_desc(&tm_v);
         ItemWalk wk;
         wk.init(a, n_bgj, w_begin);
-        int issued[kNKV] = {-1, -1, -1, -1};
+        int issued[C::NKV];
+#pragma unroll
+        for (int x = 0; x < C::NKV; ++x) issued[x] = -1;
         int prev = -1, m = -1;
         bool ok = true;
         for (int i = 0; i < n_loc && ok; ++i) {
@@ -253,22 +264,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 #pragma unroll
           for (int h = 0; h < 2; ++h) {   // K of run m is tile sequence 2m, V is 2m+1
             const int tau = 2 * m + h;
-            const int x = tau & (kNKV - 1);
-            if (!mbar_wait(bar(kBarKvEmpty + x), ((tau >> 2) & 1) ^ 1, abort_flag, a.status)) {
+            const int x = tau % C::NKV;
+            if (!mbar_wait(bar(C::BAR_KVEMPTY + x), ((tau / C::NKV) & 1) ^ 1, abort_flag, a.status)) {
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(bar(kBarKvFull + x), kTile);
-            const uint32_t dst = s_base + kSmemKV + x * kTile;
+            mbar_arrive_expect_tx(bar(C::BAR_KVFULL + x), kTile);
+            const uint32_t dst = s_base + C::SMEM_KV + x * kTile;
             const CUtensorMap *tm = h ? &tm_v : &tm_k;
-            tma_load_3d(dst, tm, bar(kBarKvFull + x), 0, g, z);
-            tma_load_3d(dst + 16384, tm, bar(kBarKvFull + x), 64, g, z);
+            tma_load_3d(dst, tm, bar(C::BAR_KVFULL + x), 0, g, z);
+            tma_load_3d(dst + 16384, tm, bar(C::BAR_KVFULL + x), 64, g, z);
             issued[x] = tau;
           }
         }
         // let every load still in flight land before the CTA can exit
-        for (int x = 0; x < kNKV; ++x)
-          if (issued[x] >= 0) mbar_wait_drain(bar(kBarKvFull + x), (issued[x] >> 2) & 1);
+        for (int x = 0; x < C::NKV; ++x)
+          if (issued[x] >= 0) mbar_wait_drain(bar(C::BAR_KVFULL + x), (issued[x] / C::NKV) & 1);
       }
     } else if (warp == 1) {
       // ------------------------------------------------------ MMA issuer
@@ -277,42 +288,41 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, 0, 1);
         int ns = 0, no = 0;          // next S and next O to issue (item indices)
         int m_s = -1, prev_bgj = -1; // run of item ns-1 and its key block
-        // per in-flight item (ring of 4 by item index): 3 bits = run index mod 4
-        // (enough for the tile index, its parity and run changes between
-        // neighbours) and whether the item opens its run
+        // per in-flight item (ring of 4 by item index), 4 bits: the V tile of
+        // its run (2), that tile's phase (1), whether the item opens its run (1)
         uint32_t ring = 0;
         bool q_seen = false, cur_new = false;
         int cur_bgj = -1;
-        bool v_pending = false;      // O of run v_run's last-known item issued, successor unknown
-        int v_run = 0;
+        bool v_pending = false;      // O of a run's last-known item issued, successor unknown
+        int v_tile = 0;              // ... and that run's V tile
         uint32_t idle = 0;
         uint64_t t_idle = 0;
         while (no < n_loc) {
           bool progressed = false;
           // ---- S_ns = Q K^T: needs the item's q rows, its K tile, a free TMEM slot
           if (ns < n_loc && ns < no + 2) {
-            const int s = ns % kNQ;
-            if (!q_seen && mbar_test_wait(bar(kBarQFull + s), (ns / kNQ) & 1)) {
+            const int s = ns % C::NQ;
+            if (!q_seen && mbar_test_wait(bar(C::BAR_QFULL + s), (ns / C::NQ) & 1)) {
               q_seen = true;
               cur_bgj = s_desc[s].x;
               cur_new = cur_bgj != prev_bgj;
             }
             if (q_seen) {
               const int m = cur_new ? m_s + 1 : m_s;
-              const int xk = (2 * m) & (kNKV - 1);
+              const int xk = (2 * m) % C::NKV;
               const bool k_ok =
-                  !cur_new || mbar_test_wait(bar(kBarKvFull + xk), ((2 * m) >> 2) & 1);
-              if (k_ok && mbar_test_wait(bar(kBarTmEmpty + (ns & 1)), ((ns >> 1) & 1) ^ 1)) {
+                  !cur_new || mbar_test_wait(bar(C::BAR_KVFULL + xk), ((2 * m) / C::NKV) & 1);
+              if (k_ok && mbar_test_wait(bar(C::BAR_TMEMPTY + (ns & 1)), ((ns >> 1) & 1) ^ 1)) {
                 tc_fence_after();
                 fence_proxy_async_smem();   // cp.async-written q rows -> UMMA operand reads
                 if (cur_new && ns > 0) {
                   // the previous run's last S is issued: its K tile frees when that completes
-                  umma_commit(bar(kBarKvEmpty + ((2 * m_s) & (kNKV - 1))));
-                  if (v_pending) umma_commit(bar(kBarKvEmpty + ((2 * v_run + 1) & (kNKV - 1))));
+                  umma_commit(bar(C::BAR_KVEMPTY + (2 * m_s) % C::NKV));
+                  if (v_pending) umma_commit(bar(C::BAR_KVEMPTY + v_tile));
                 }
                 v_pending = false;
-                const uint32_t sq = s_base + kSmemQ + s * kTile;
-                const uint32_t sk = s_base + kSmemKV + xk * kTile;
+                const uint32_t sq = s_base + C::SMEM_Q + s * kTile;
+                const uint32_t sk = s_base + C::SMEM_KV + xk * kTile;
                 const uint32_t d_tmem = tmem_base + (ns & 1) * 128;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -321,9 +331,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                   umma_f16_ss(d_tmem, sdesc_sw128(sq + c * 16384 + off, 16, 1024),
                               sdesc_sw128(sk + c * 16384 + off, 16, 1024), idesc_s, kk > 0);
                 }
-                umma_commit(bar(kBarSFull + (ns & 1)));
-                const uint32_t sh = 3u * uint32_t(ns & 3);
-                ring = (ring & ~(7u << sh)) | ((uint32_t(m & 3) | (cur_new ? 4u : 0u)) << sh);
+                umma_commit(bar(C::BAR_SFULL + (ns & 1)));
+                {   // per in-flight item: V tile, its phase, whether the item opens a run
+                  const int tv = 2 * m + 1;
+                  const uint32_t e = uint32_t(tv % C::NKV) | (uint32_t((tv / C::NKV) & 1) << 2) |
+                                     (cur_new ? 8u : 0u);
+                  const uint32_t sh = 4u * uint32_t(ns & 3);
+                  ring = (ring & ~(15u << sh)) | (e << sh);
+                }
                 m_s = m;
                 prev_bgj = cur_bgj;
                 q_seen = false;
@@ -334,15 +349,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
           // ---- O_no = P V: needs the softmax's P and the item's V tile
           if (no < ns) {
-            const uint32_t e = (ring >> (3u * uint32_t(no & 3))) & 7u;
-            const int m = int(e & 3u);   // run index mod 4
-            const int xv = (2 * m + 1) & (kNKV - 1);
-            const bool v_ok =
-                !(e & 4u) || mbar_test_wait(bar(kBarKvFull + xv), ((2 * m + 1) >> 2) & 1);
-            if (v_ok && mbar_test_wait(bar(kBarPFull + (no & 1)), (no >> 1) & 1)) {
+            const uint32_t e = (ring >> (4u * uint32_t(no & 3))) & 15u;
+            const int xv = int(e & 3u);
+            const bool v_ok = !(e & 8u) || mbar_test_wait(bar(C::BAR_KVFULL + xv), (e >> 2) & 1u);
+            if (v_ok && mbar_test_wait(bar(C::BAR_PFULL + (no & 1)), (no >> 1) & 1)) {
               tc_fence_after();
-              const uint32_t sp = s_base + kSmemQ + (no % kNQ) * kTile;
-              const uint32_t sv = s_base + kSmemKV + xv * kTile;
+              const uint32_t sp = s_base + C::SMEM_Q + (no % C::NQ) * kTile;
+              const uint32_t sv = s_base + C::SMEM_KV + xv * kTile;
               const uint32_t d_tmem = tmem_base + (no & 1) * 128;
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk) {
@@ -351,14 +364,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 umma_f16_ss(d_tmem, sdesc_sw128(sp + c * 16384 + off, 16, 1024),
                             sdesc_sw128(sv + kk * 2048, 16384, 1024), idesc_o, kk > 0);
               }
-              umma_commit(bar(kBarOFull + (no & 1)));
+              umma_commit(bar(C::BAR_OFULL + (no & 1)));
               // free run m's V tile once item no is known to be its last
               if (no + 1 < ns) {
-                if (int((ring >> (3u * uint32_t((no + 1) & 3))) & 3u) != m)
-                  umma_commit(bar(kBarKvEmpty + xv));
+                if ((ring >> (4u * uint32_t((no + 1) & 3))) & 8u)   // item no+1 opens a run
+                  umma_commit(bar(C::BAR_KVEMPTY + xv));
               } else if (no + 1 < n_loc) {
                 v_pending = true;
-                v_run = m;
+                v_tile = xv;
               }
               ++no;
               progressed = true;
@@ -385,8 +398,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         // every UMMA issued has completed before TMEM can be released
-        umma_commit(bar(kBarDrain));
-        mbar_wait_drain(bar(kBarDrain), 0);
+        umma_commit(bar(C::BAR_DRAIN));
+        mbar_wait_drain(bar(C::BAR_DRAIN), 0);
       }
     } else {
       // ------------------------------------------------------ q gather team
@@ -422,23 +435,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       const int gran = lane & 15;
       for (int i = 0; i < n_loc; ++i) {
-        const int s = i % kNQ;
-        bool ok = mbar_wait(bar(kBarStEmpty + s), ((i / kNQ) & 1) ^ 1, abort_flag, a.status);
+        const int s = i % C::NQ;
+        bool ok = mbar_wait(bar(C::BAR_STEMPTY + s), ((i / C::NQ) & 1) ^ 1, abort_flag, a.status);
         if (!bar_and_n(bar_id, kTeam, ok)) break;
         if (gtid < 32) {   // publish the item: the MMA and the softmax read these
           if (gtid == 0) s_desc[s] = d;
 #pragma unroll
           for (int c = 0; c < NE; ++c)
-            if (32 * c + lane < d.z) s_list[s * 128 + 32 * c + lane] = ent[c];
+            if (32 * c + lane < d.z) s_list[s * QPI + 32 * c + lane] = ent[c];
           __syncwarp();
-          if (gtid == 0) mbar_arrive(bar(kBarQFull + s));
+          if (gtid == 0) mbar_arrive(bar(C::BAR_QFULL + s));
         }
         const int bgj = d.x;
         const int g = (bgj / a.nb) % a.G;
         const int b = bgj / (a.nb * a.G);
         const uint16_t *qb = a.q + size_t(g) * R * kHeadDim + gran * 8;
         const int qrow0 = b * a.Lq - a.tq0;   // + t: the query's row in q (t >= tq0)
-        const uint32_t stq = s_base + kSmemQ + s * kTile + (gran >> 3) * 16384;
+        const uint32_t stq = s_base + C::SMEM_Q + s * kTile + (gran >> 3) * 16384;
         // row pair p = wg + 6*it (rows 2p, 2p+1): one coalesced 512-byte
         // copy per warp instruction
 #pragma unroll
@@ -458,7 +471,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                          qb + (size_t(qrow0 + t) * a.H + hh) * kHeadDim);
           }
         }
-        cp_async_arrive_noinc(bar(kBarQFull + s));
+        cp_async_arrive_noinc(bar(C::BAR_QFULL + s));
         if (gtid == 0 && i + 1 < n_loc) s_pre[0] = wk.describe(a, QPI, w_begin + i + 1);
         bar_sync_n(bar_id, kTeam);
         if (i + 1 < n_loc) {
@@ -475,16 +488,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int bar_id = 4 + u;
     const uint32_t tm = tmem_base + u * 128 + (uint32_t((warp & 3) * 32) << 16);
     for (int i = u; i < n_loc; i += 2) {
-      const int s = i % kNQ;
-      bool ok = mbar_wait(bar(kBarQFull + s), (i / kNQ) & 1, abort_flag, a.status);
+      const int s = i % C::NQ;
+      bool ok = mbar_wait(bar(C::BAR_QFULL + s), (i / C::NQ) & 1, abort_flag, a.status);
       if (!bar_and_n(bar_id, 128, ok)) break;
       const int4 d = s_desc[s];
       const int j = d.x % a.nb;
       const int qi = row / R;
       const bool valid = qi < d.z;
-      const int t = valid ? (s_list[s * 128 + qi] >> 5) : 0;
+      const int t = valid ? (s_list[s * QPI + qi] >> 5) : 0;
       const int lim = valid ? (t - j * kBlock) : (kBlock - 1);   // last visible column
-      ok = mbar_wait(bar(kBarSFull + u), (i >> 1) & 1, abort_flag, a.status);
+      ok = mbar_wait(bar(C::BAR_SFULL + u), (i >> 1) & 1, abort_flag, a.status);
       if (!bar_and_n(bar_id, 128, ok)) break;
       tc_fence_after();
 
@@ -521,7 +534,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
       const float2 nmb2 = make_float2(-mb, -mb);
       float2 l2 = make_float2(0.f, 0.f);
-      uint8_t *stage = smem + kSmemQ + s * kTile;
+      uint8_t *stage = smem + C::SMEM_Q + s * kTile;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
 #pragma unroll
@@ -541,9 +554,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bar(kBarPFull + u));
+      mbar_arrive(bar(C::BAR_PFULL + u));
 
-      ok = mbar_wait(bar(kBarOFull + u), (i >> 1) & 1, abort_flag, a.status);
+      ok = mbar_wait(bar(C::BAR_OFULL + u), (i >> 1) & 1, abort_flag, a.status);
       if (!bar_and_n(bar_id, 128, ok)) break;
       tc_fence_after();
       {
@@ -559,7 +572,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(bar(kBarTmEmpty + u));   // slot u may take the next S
+      mbar_arrive(bar(C::BAR_TMEMPTY + u));   // slot u may take the next S
 
       // stage the normalised bf16 partial row (granule c at c ^ (row & 7))
       const float l = l2.x + l2.y;
@@ -587,11 +600,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int nrows = min(32, d.z * R - wrow0);
         if (nrows > 0) {
           bulk_store(a.part_o + (size_t(d.y) * R + wrow0) * kHeadDim,
-                     s_base + kSmemQ + s * kTile + wrow0 * 256, uint32_t(nrows) * 256u);
+                     s_base + C::SMEM_Q + s * kTile + wrow0 * 256, uint32_t(nrows) * 256u);
           bulk_commit();
           bulk_wait_read_all();
         }
-        mbar_arrive(bar(kBarStEmpty + s));   // with all four: the stage may take item i+3
+        mbar_arrive(bar(C::BAR_STEMPTY + s));   // with all four: the stage may take item i+3
       }
     }
     if (lane == 0) bulk_wait_all();
@@ -610,11 +623,11 @@ template <int R>
 cudaError_t launch_attn_r(const CUtensorMap &tk, const CUtensorMap &tv, const AttnArgs &a,
                           int num_sms, cudaStream_t st) {
   auto kern = msa_prefill_attn_kernel<R>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kAttnSmem);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnCfg<R>::SMEM);
   if (e != cudaSuccess) return e;
   int grid = num_sms;
   if (a.max_items < grid) grid = a.max_items > 0 ? a.max_items : 1;
-  kern<<<grid, kAttnThreads, kAttnSmem, st>>>(tk, tv, a);
+  kern<<<grid, kAttnThreads, AttnCfg<R>::SMEM, st>>>(tk, tv, a);
   return cudaGetLastError();
 }
 
