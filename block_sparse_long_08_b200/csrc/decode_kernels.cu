@@ -292,7 +292,10 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
 constexpr int kVPitch = kHeadDim + 8;  // bf16 per staged V row (272 B: conflict-free ldmatrix)
 template <int R>
 constexpr int dec_attn_smem() {
-  return kBlock * kVPitch * 2 + 4 * R * kHeadDim * 4 + 2 * 4 * 16 * 4;
+  // staged V, then the row max / sum exchange; the 4 warps' partial O reuse
+  // the V area once every warp has read V (6 CTAs fit on an SM)
+  static_assert(4 * R * kHeadDim * 4 <= kBlock * kVPitch * 2, "partial O must fit the V area");
+  return kBlock * kVPitch * 2 + 2 * 4 * 16 * 4;
 }
 
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
@@ -305,8 +308,8 @@ template <int R>
 __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
   extern __shared__ __align__(16) uint8_t dsm[];
   uint16_t *sV = reinterpret_cast<uint16_t *>(dsm);
-  float *s_o = reinterpret_cast<float *>(sV + kBlock * kVPitch);   // [4 warps][R rows][128]
-  float *s_m = s_o + 4 * R * kHeadDim;                              // [4][16]
+  float *s_o = reinterpret_cast<float *>(dsm);                     // [4 warps][R rows][128], over V
+  float *s_m = reinterpret_cast<float *>(sV + kBlock * kVPitch);   // [4][16]
   float *s_l = s_m + 4 * 16;                                        // [4][16]
   const int slot = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -437,7 +440,9 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
       mma_bf16_16816(oacc[dt + 1], pa[kt][0], pa[kt][1], pa[kt][2], pa[kt][3], bv[2], bv[3]);
     }
   }
-  // sum the 4 warps' partial O (rows < R only) and normalise
+  // sum the 4 warps' partial O (rows < R only) and normalise; the partial O
+  // area overlays the staged V, so every warp must be done reading V
+  __syncthreads();
 #pragma unroll
   for (int dt = 0; dt < 16; ++dt) {
     const int d = dt * 8 + 2 * c;
@@ -479,8 +484,8 @@ template <int R>
 __global__ void __launch_bounds__(128) decode_attn_fp8_kernel(const DecodeArgs a) {
   extern __shared__ __align__(16) uint8_t dsm[];
   uint16_t *sV = reinterpret_cast<uint16_t *>(dsm);
-  float *s_o = reinterpret_cast<float *>(sV + kBlock * kVPitch);   // [4 warps][R rows][128]
-  float *s_m = s_o + 4 * R * kHeadDim;                              // [4][16]
+  float *s_o = reinterpret_cast<float *>(dsm);                     // [4 warps][R rows][128], over V
+  float *s_m = reinterpret_cast<float *>(sV + kBlock * kVPitch);   // [4][16]
   float *s_l = s_m + 4 * 16;                                        // [4][16]
   const int slot = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -641,6 +646,7 @@ __global__ void __launch_bounds__(128) decode_attn_fp8_kernel(const DecodeArgs a
       mma_bf16_16816(oacc[dt + 1], pa[kt][0], pa[kt][1], pa[kt][2], pa[kt][3], bv[2], bv[3]);
     }
   }
+  __syncthreads();   // the partial O area overlays the staged V: all warps done with V
 #pragma unroll
   for (int dt = 0; dt < 16; ++dt) {
     const int d = dt * 8 + 2 * c;
