@@ -271,7 +271,7 @@ def main():
     ap.add_argument("--workload", default="1m", choices=["1m", "128k", "32k"],
                     help="prefill length of the step (1m is the headline workload)")
     ap.add_argument("--op", default="step",
-                    choices=["step", "index", "attn", "decode", "decode8", "cached"],
+                    choices=["step", "index", "scores", "attn", "decode", "decode8", "cached"],
                     help="time one operation of the step alone (profiling runs; 'cached' runs "
                          "the whole prefill as 8 msa_forward_cached chunks against the caches); "
                          "prints its own short JSON line")
@@ -346,7 +346,7 @@ def run_ours(args, shape, dshape, seed, cfg, ws_n, rank, local):
     peaks = load_peaks()
 
     # ---- inputs (device-resident for the kernel-timed leg)
-    need_pre = args.op in ("step", "index", "attn", "cached")
+    need_pre = args.op in ("step", "index", "scores", "attn", "cached")
     need_dec = args.op in ("step", "decode", "decode8")
     if not need_pre:   # a decode-only profiling run keeps the footprint small
         import dataclasses
@@ -500,6 +500,8 @@ def run_single_op(args, M, x, dx, dshape, K, sel, out, dout, ws_idx, ws_att, ws_
                                      ws=ws_c)
         elif args.op == "index":
             M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx)
+        elif args.op == "scores":   # stored block scores + the standalone top-k kernel
+            M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx, block_scores=True)
         elif args.op == "attn":
             M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att)
         elif args.op == "decode8":   # FP8 index-key cache
