@@ -26,6 +26,11 @@ Sources (cited by page title / address and section):
   control as its concern.  The FP8 cache format itself is the OCP 8-bit
   floating point E4M3 encoding; its definition, not the pages, fixes
   e4m3_to_f64.
+* Training paragraph of [P4] "机制": the index branch learns from a KL loss
+  against the main branch on the selected blocks, and the index path's
+  gradient into the main attention is cut.  The main branch's backward pass
+  is therefore the gradient of its exact attention over the selected tokens
+  with the selection held fixed (prefill_backward).
 
 Readings taken where the pages are silent (each is also listed in the
 design notes):
@@ -64,6 +69,8 @@ __all__ = [
     "prefill",
     "decode",
     "block_scores_all",
+    "attend_rows_grad",
+    "prefill_backward",
 ]
 
 
@@ -297,3 +304,59 @@ def decode(q, q_idx, k_cache, v_cache, k_idx_cache, seq_lens, top_k: int,
             out[b, heads] = o
             lse[b, heads] = l_
     return {"sel": sel, "out": out, "lse": lse}
+
+
+# ---------------------------------------------------------------------------
+# Main Branch backward  ([P4] "机制", training paragraph)
+# ---------------------------------------------------------------------------
+
+def attend_rows_grad(q_rows: np.ndarray, k_tok: np.ndarray, v_tok: np.ndarray,
+                     do_rows: np.ndarray, scale: float):
+    """Gradient of sum(do * o) for o = attend_rows(q_rows, k_tok, v_tok).
+
+    With P the softmax probabilities and dP = do v^T, the softmax Jacobian
+    gives dZ = P * (dP - rowsum(P * dP)) for the scaled logits Z, and
+    rowsum(P * dP) = rowsum(do * o).  Then dq = scale dZ k, dk = scale dZ^T q
+    and dv = P^T do.  Returns (dq [r,d], dk [n,d], dv [n,d]).
+    """
+    o, _, p = attend_rows(q_rows, k_tok, v_tok, scale)
+    dp = do_rows @ v_tok.T
+    delta = np.sum(do_rows * o, axis=1, keepdims=True)
+    dz = p * (dp - delta)
+    return scale * (dz @ k_tok), scale * (dz.T @ q_rows), p.T @ do_rows
+
+
+def prefill_backward(q, k, v, sel, dout, block: int = 128, scale: Optional[float] = None):
+    """Main-branch backward of MSA prefill for a given selection.
+
+    The index path is detached from the main attention ([P4] "机制"), so the
+    selection sel [B,G,L,top_k] is a constant here and only q, k and v get
+    gradients: every (query, group) row contributes through the tokens of its
+    selected blocks with s <= t (the same token set as prefill), and a key or
+    value token sums the contributions of every row that attends to it.
+    dout has the shape of the output [B,L,H,d].  Returns dict(dq [B,L,H,d],
+    dk [B,L,G,d], dv [B,L,G,d]) in fp64.
+    """
+    q, k, v, dout = as_f64(q), as_f64(k), as_f64(v), as_f64(dout)
+    sel = np.asarray(sel)
+    B, L, H, d = q.shape
+    G = k.shape[2]
+    r = H // G
+    sc = _scale_of(d, scale)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for t in range(L):
+            for g in range(G):
+                blocks = [int(x) for x in sel[b, g, t] if x >= 0]
+                tok = selected_tokens(blocks, t, block)
+                if tok.size == 0:
+                    continue
+                heads = list(range(g * r, (g + 1) * r))
+                gq, gk, gv = attend_rows_grad(q[b, t, heads], k[b, tok, g], v[b, tok, g],
+                                              dout[b, t, heads], sc)
+                dq[b, t, heads] = gq
+                np.add.at(dk[b, :, g], tok, gk)
+                np.add.at(dv[b, :, g], tok, gv)
+    return {"dq": dq, "dk": dk, "dv": dv}

@@ -273,6 +273,85 @@ def check_e4m3_against_library_and_closed_forms():
     np.testing.assert_array_equal(O.dequant_rows(rows, [0.25, 4.0]), [[0.25, 0.5], [6.0, -4.0]])
 
 
+def _bwd_problem(seed, top_k=2, L=64):
+    """Small fp64 problem with a sparse selection (4 blocks of 16, top_k=2)."""
+    blk = 16
+    p = _small_problem(seed, B=1, L=L, H=4, G=2, d=8, di=8)
+    sel = O.prefill(p["q"], p["k"], p["v"], p["q_idx"], p["k_idx"], top_k=top_k, block=blk)["sel"]
+    dout = np.random.default_rng(seed).standard_normal(p["q"].shape)
+    return p, sel, dout, blk
+
+
+def check_backward_finite_differences():
+    """Directional derivatives of sum(dout * out) by central differences
+    (fp64, h = 1e-5) against the oracle's gradients: random directions over
+    whole tensors, and directions confined to the diagonal (local) block and
+    to one earlier key block."""
+    p, sel, dout, blk = _bwd_problem(101)
+    g = O.prefill_backward(p["q"], p["k"], p["v"], sel, dout, block=blk)
+    grads = {"q": g["dq"], "k": g["dk"], "v": g["dv"]}
+
+    def loss(**kw):
+        x = {n: kw.get(n, p[n]) for n in ("q", "k", "v")}
+        out = O.prefill(x["q"], x["k"], x["v"], p["q_idx"], p["k_idx"], top_k=sel.shape[-1],
+                        block=blk, sel_override=sel)["out"]
+        return float(np.sum(out * dout))
+
+    rng = np.random.default_rng(7)
+    h = 1e-5
+    L = p["q"].shape[1]
+    for name in ("q", "k", "v"):
+        dirs = [rng.standard_normal(p[name].shape) for _ in range(3)]
+        for lo, hi in ((L - blk, L), (blk, 2 * blk)):
+            u = np.zeros(p[name].shape)
+            u[:, lo:hi] = rng.standard_normal(u[:, lo:hi].shape)
+            dirs.append(u)
+        for u in dirs:
+            fd = (loss(**{name: p[name] + h * u}) - loss(**{name: p[name] - h * u})) / (2 * h)
+            an = float(np.sum(grads[name] * u))
+            assert abs(fd - an) <= 1e-6 * (1.0 + abs(an)), (name, fd, an)
+
+
+def check_backward_dense_limit():
+    """top_k >= nb: every earlier block is selected, so the gradients are
+    those of dense causal GQA attention -- torch autograd through
+    scaled_dot_product_attention in fp64."""
+    p, _, dout, blk = _bwd_problem(102)
+    nb = p["q"].shape[1] // blk
+    sel = O.prefill(p["q"], p["k"], p["v"], p["q_idx"], p["k_idx"], top_k=nb, block=blk)["sel"]
+    g = O.prefill_backward(p["q"], p["k"], p["v"], sel, dout, block=blk)
+    qt, kt, vt = (torch.from_numpy(p[n].copy()).requires_grad_() for n in ("q", "k", "v"))
+    r = qt.shape[2] // kt.shape[2]
+    o = F.scaled_dot_product_attention(qt.permute(0, 2, 1, 3),
+                                       kt.permute(0, 2, 1, 3).repeat_interleave(r, dim=1),
+                                       vt.permute(0, 2, 1, 3).repeat_interleave(r, dim=1),
+                                       is_causal=True).permute(0, 2, 1, 3)
+    (o * torch.from_numpy(dout)).sum().backward()
+    np.testing.assert_allclose(g["dq"], qt.grad.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(g["dk"], kt.grad.numpy(), rtol=1e-10, atol=1e-11)
+    np.testing.assert_allclose(g["dv"], vt.grad.numpy(), rtol=1e-10, atol=1e-11)
+
+
+def check_backward_sums():
+    """Closed forms that hold for any selection: each softmax row sums to 1,
+    so the value gradients of a group sum to the group's summed output
+    gradient, and the logit gradients of a row sum to 0, so the key
+    gradients of a group sum to 0."""
+    p, sel, dout, blk = _bwd_problem(103, top_k=2, L=80)
+    g = O.prefill_backward(p["q"], p["k"], p["v"], sel, dout, block=blk)
+    G = p["k"].shape[2]
+    r = p["q"].shape[2] // G
+    for gi in range(G):
+        want_v = dout[0, :, gi * r:(gi + 1) * r].sum(axis=(0, 1))
+        np.testing.assert_allclose(g["dv"][0, :, gi].sum(axis=0), want_v, rtol=0, atol=1e-11)
+        np.testing.assert_allclose(g["dk"][0, :, gi].sum(axis=0), 0.0, rtol=0, atol=1e-11)
+    # keys of blocks that no query selects get no gradient
+    used = set(int(j) for j in sel.ravel() if j >= 0)
+    for j in range(p["k"].shape[1] // blk):
+        if j not in used:
+            assert not g["dk"][0, j * blk:(j + 1) * blk].any()
+
+
 CHECKS = {
     "golden": check_golden,
     "e4m3": check_e4m3_against_library_and_closed_forms,
@@ -287,6 +366,9 @@ CHECKS = {
     "order_invariance": check_sel_order_invariance,
     "zero_query_mean": check_zero_query_mean,
     "decode_last_row": check_decode_is_last_prefill_row,
+    "backward_finite_differences": check_backward_finite_differences,
+    "backward_dense_limit": check_backward_dense_limit,
+    "backward_sums": check_backward_sums,
 }
 
 
@@ -354,6 +436,26 @@ def _e4m3_no_subnormals(codes):
 
 _orig_e4m3 = O.e4m3_to_f64
 
+
+def _grad_no_delta(q_rows, k_tok, v_tok, do_rows, scale):
+    _, _, p = _orig_attend(q_rows, k_tok, v_tok, scale)
+    dz = p * (do_rows @ v_tok.T)                 # the rowsum(do * o) term dropped
+    return scale * (dz @ k_tok), scale * (dz.T @ q_rows), p.T @ do_rows
+
+
+def _grad_dk_unscaled(q_rows, k_tok, v_tok, do_rows, scale):
+    dq, dk, dv = _orig_grad(q_rows, k_tok, v_tok, do_rows, scale)
+    return dq, dk / scale, dv
+
+
+def _grad_dq_through_v(q_rows, k_tok, v_tok, do_rows, scale):
+    o, _, p = _orig_attend(q_rows, k_tok, v_tok, scale)
+    dz = p * (do_rows @ v_tok.T - np.sum(do_rows * o, axis=1, keepdims=True))
+    return scale * (dz @ v_tok), scale * (dz.T @ q_rows), p.T @ do_rows
+
+
+_orig_grad = O.attend_rows_grad
+
 MUTANTS = {
     "no_forced_local": ("select_blocks_row", _select_no_local),
     "ties_to_higher_id": ("select_blocks_row", _select_high_tie),
@@ -364,6 +466,9 @@ MUTANTS = {
     "k_v_swapped": ("attend_rows", _attend_swapped_kv),
     "e4m3_bias_8": ("e4m3_to_f64", _e4m3_bias8),
     "e4m3_no_subnormals": ("e4m3_to_f64", _e4m3_no_subnormals),
+    "bwd_delta_dropped": ("attend_rows_grad", _grad_no_delta),
+    "bwd_dk_unscaled": ("attend_rows_grad", _grad_dk_unscaled),
+    "bwd_dq_through_v": ("attend_rows_grad", _grad_dq_through_v),
 }
 
 
