@@ -99,6 +99,27 @@ def prefill_attn_bytes(B, L, H, G, d, top_k):
     return entries * r * (d * 2 * 3 + 4 * 2) + B * float(L) * H * d * 2
 
 
+def prefill_bwd_bytes(B, L, H, G, d, top_k):
+    """Bytes the key-block-outer backward must move: every selected (query,
+    group, block) entry gathers its R q rows and R do rows, reads R lse and
+    D values, and writes and reads back R fp32 dq partial rows; K/V are read
+    once per key block and dk/dv written once; D = do . o reads o and do,
+    and dq is written once."""
+    t = np.arange(L, dtype=np.int64)
+    entries = B * G * float(np.minimum(top_k, t // BLOCK + 1).sum())
+    r = H // G
+    rows = B * float(L) * H * d * 2
+    kv = B * float(L) * G * d * 2
+    return entries * r * (d * 2 * 2 + d * 4 * 2 + 8) + 3 * rows + 4 * kv
+
+
+def prefill_bwd_flops(B, L, H, d, top_k):
+    """Five products per (query, head, attended token) of 2d flops each:
+    S, dP, dV, dK, dQ."""
+    t = np.arange(L, dtype=np.int64)
+    return B * float(H) * 10.0 * d * float(n_sel(t, top_k).sum())
+
+
 def decode_bytes(seq_lens, H, G, d, d_idx, top_k, fp8_index=False, fp8_kv=False):
     """Bytes a decode step must read: the index-key scan over every cached
     token (bf16, or E4M3 codes + one fp32 scale per token), the selected K/V
@@ -268,10 +289,12 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="1m", choices=["1m", "128k", "32k"],
-                    help="prefill length of the step (1m is the headline workload)")
+    ap.add_argument("--workload", default="1m", choices=["1m", "128k", "32k", "8k"],
+                    help="prefill length of the step (1m is the headline workload; 8k is a "
+                         "small-footprint case for profiler captures)")
     ap.add_argument("--op", default="step",
-                    choices=["step", "index", "scores", "attn", "decode", "decode8", "cached"],
+                    choices=["step", "index", "scores", "attn", "decode", "decode8", "cached",
+                             "bwd"],
                     help="time one operation of the step alone (profiling runs; 'cached' runs "
                          "the whole prefill as 8 msa_forward_cached chunks against the caches); "
                          "prints its own short JSON line")
@@ -286,8 +309,12 @@ def main():
         shape, dshape, seed = I.PREFILL_1M, I.DECODE_1M, I.SEEDS["1m"]
     elif args.workload == "128k":
         shape, dshape, seed = I.PREFILL_128K_PLANTED, I.DECODE_128K, I.SEEDS["128k_planted"]
-    else:
+    elif args.workload == "32k":
         shape, dshape, seed = I.PREFILL_32K, I.DECODE_128K, I.SEEDS["32k"]
+    else:
+        import dataclasses
+        shape, dshape, seed = (dataclasses.replace(I.PREFILL_32K, L=8192), I.DECODE_128K,
+                               I.SEEDS["32k"])
     cfg = {"workload": f"MSA prefill B={shape.B} L={shape.L} + decode batch {dshape.B} at "
                        f"{'%d' % dshape.len_hi if dshape.len_lo == dshape.len_hi else 'U[%d,%d]' % (dshape.len_lo, dshape.len_hi)}",
            "B": shape.B, "L": shape.L, "H": shape.H, "G": shape.G, "d": shape.d,
@@ -346,7 +373,7 @@ def run_ours(args, shape, dshape, seed, cfg, ws_n, rank, local):
     peaks = load_peaks()
 
     # ---- inputs (device-resident for the kernel-timed leg)
-    need_pre = args.op in ("step", "index", "scores", "attn", "cached")
+    need_pre = args.op in ("step", "index", "scores", "attn", "cached", "bwd")
     need_dec = args.op in ("step", "decode", "decode8")
     if not need_pre:   # a decode-only profiling run keeps the footprint small
         import dataclasses
@@ -450,6 +477,10 @@ def run_ours(args, shape, dshape, seed, cfg, ws_n, rank, local):
     if args.workload == "1m" and rank == 0 or args.workload != "1m":
         line["decode_128k"] = bench_decode_128k(M, I, dev, args, peaks)
 
+    # ---- main-branch backward at 32K
+    if args.workload == "1m" and rank == 0 or args.workload != "1m":
+        line["backward_32k"] = bench_backward_32k(M, I, dev, args, peaks)
+
     # ---- end to end through the public API with host buffers (the timed
     # leg's workspace and outputs are released first)
     del ws_att, sel, out
@@ -493,6 +524,16 @@ def run_single_op(args, M, x, dx, dshape, K, sel, out, dout, ws_idx, ws_att, ws_
                            x["q_idx"].shape[3], 128, K)
         ws_c = M.new_workspace(pc, M.MSA_OP_FORWARD, x["q"].device)
 
+    if args.op == "bwd":
+        from block_sparse_long_08_b200 import inputs as I
+        Bq, Lq, Hq, dq_ = x["q"].shape
+        sh_b = I.PrefillShape(B=Bq, L=Lq, H=Hq, G=x["k"].shape[2], d=dq_, d_idx=x["q_idx"].shape[3],
+                              top_k=K)
+        dout_b = I.output_grad(sh_b, 0, device=x["q"].device)
+        out, lse_b = M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, want_lse=True)
+        ws_b = M.new_workspace(M.make_params(Bq, Lq, Hq, sh_b.G, dq_, sh_b.d_idx, 128, K),
+                               M.MSA_OP_BACKWARD, x["q"].device)
+
     def op():
         if args.op == "cached":   # the prefill as the serving form: 8 chunks against the caches
             for c, (q, q_idx) in enumerate(qc):
@@ -504,6 +545,8 @@ def run_single_op(args, M, x, dx, dshape, K, sel, out, dout, ws_idx, ws_att, ws_
             M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx, block_scores=True)
         elif args.op == "attn":
             M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att)
+        elif args.op == "bwd":
+            M.msa_sparse_attn_backward(x["q"], x["k"], x["v"], out, lse_b, dout_b, sel, ws=ws_b)
         elif args.op == "decode8":   # FP8 index-key cache
             M.msa_sparse_attn_decode_fp8idx(dx["q"], dx["q_idx"], dx["k_cache"], dx["v_cache"],
                                             codes8, scale8, dx["seq_lens"], dshape.top_k,
@@ -522,7 +565,8 @@ def run_single_op(args, M, x, dx, dshape, K, sel, out, dout, ws_idx, ws_att, ws_
         op()
     b.record(stream)
     torch.cuda.synchronize()
-    for w in (ws_idx, ws_att, ws_dec) + ((ws_c,) if ws_c is not None else ()):
+    extra = ((ws_c,) if ws_c is not None else ()) + ((ws_b,) if args.op == "bwd" else ())
+    for w in (ws_idx, ws_att, ws_dec) + extra:
         if M.msa_read_status(w) != 0:
             raise SystemExit("device status error")
     ms = a.elapsed_time(b) / args.steps
@@ -599,6 +643,54 @@ def bench_decode_128k(M, I, dev, args, peaks):
             "fp8_all_caches": {"us_per_step": us88, "roofline": roof(byts88, us88),
                                "cache": "k_idx, K and V as E4M3 codes + fp32 scales"},
             "gpu_launches": 12 * iters}
+
+
+def bench_backward_32k(M, I, dev, args, peaks):
+    """Main-branch backward at the 32K prefill workload (seed of the 32K
+    config), on the forward's own selection, output and lse."""
+    sh = I.PREFILL_32K
+    x = I.prefill_inputs(sh, I.SEEDS["32k"], device=dev)
+    dout = I.output_grad(sh, I.SEEDS["32k"], device=dev)
+    out, sel, lse = M.msa_forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], sh.top_k,
+                                  want_sel=True, want_lse=True)
+    p = M.make_params(sh.B, sh.L, sh.H, sh.G, sh.d, sh.d_idx, BLOCK, sh.top_k)
+    ws = M.new_workspace(p, M.MSA_OP_BACKWARD, dev)
+    dq, dk, dv = torch.empty_like(x["q"]), torch.empty_like(x["k"]), torch.empty_like(x["v"])
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def run():
+        M.msa_sparse_attn_backward(x["q"], x["k"], x["v"], out, lse, dout, sel, dq=dq, dk=dk,
+                                   dv=dv, ws=ws)
+
+    for _ in range(max(3, args.warmup)):
+        run()
+    torch.cuda.synchronize()
+    if M.msa_read_status(ws) != 0:
+        raise SystemExit("backward device status error")
+    iters = 10
+    times = []
+    for _ in range(iters):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        run()
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    byts = prefill_bwd_bytes(sh.B, sh.L, sh.H, sh.G, sh.d, sh.top_k)
+    fl = prefill_bwd_flops(sh.B, sh.L, sh.H, sh.d, sh.top_k)
+    del x, dout, out, sel, lse, ws, dq, dk, dv
+    return {"ms": ms, "iters": iters, "tokens_per_s": sh.B * sh.L / (ms / 1e3),
+            "workload": f"B={sh.B} L={sh.L} H={sh.H} G={sh.G} d={sh.d} top_k={sh.top_k}",
+            "roofline": {"bound": "hbm", "achieved": byts / (ms / 1e3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], "bytes": byts},
+            "tensor": {"flops": fl, "tflops": fl / (ms / 1e3) / 1e12,
+                       "frac_of_sustained": fl / (ms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"]},
+            "gpu_launches": 6 * iters}
 
 
 def bench_e2e(M, x, dx, shape, dshape, K, args, ws_n, stream):

@@ -80,6 +80,25 @@ struct CombineArgs {
 };
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
 
+// Main-branch backward over a whole-sequence reverse index (t0 = 0, Lc = L).
+struct BwdArgs {
+  int B, L, H, G, nb, top_k;
+  float scale, scale_log2;
+  const uint16_t *q;           // [B,L,H,d]
+  const uint16_t *out, *dout;  // [B,L,H,d]: forward output and its gradient
+  const float *lse;            // [B,L,H]: forward log-sum-exp (natural log)
+  const int32_t *sel;          // [B,G,L,top_k]
+  const int32_t *list, *list_off, *pos_of;   // reverse index (see RevIdxArgs)
+  float *delta;                // [B,L,H]: do . o
+  float *part_dq;              // [entries*R, d] fp32: dq of (list position, head), scaled
+  uint16_t *dq;                // [B,L,H,d]
+  uint16_t *dk, *dv;           // [B,L,G,d]
+  int *unit_ctr;               // work counter (zeroed by the launcher)
+  int *status;
+};
+cudaError_t launch_backward(const CUtensorMap &tk, const CUtensorMap &tv, const BwdArgs &a,
+                            int num_sms, cudaStream_t st);
+
 struct DecodeArgs {
   int B, Lmax, H, G, d_idx, nb_max, top_k;
   float scale, scale_log2;

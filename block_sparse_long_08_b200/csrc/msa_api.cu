@@ -107,6 +107,28 @@ AttnWs attn_ws(const msa_params *p, size_t base) {
   return w;
 }
 
+// Backward: a whole-sequence reverse index, D = do . o per row, and one
+// fp32 dq partial row per (query, head, slot).
+struct BwdWs {
+  size_t cnt, list_off, item_off, list, pos_of, delta, part_dq, end;
+};
+BwdWs bwd_ws(const msa_params *p) {
+  BwdWs w;
+  const size_t nb = size_t(p->L) / 128;
+  const size_t nbgj = size_t(p->B) * p->G * nb;
+  const size_t entries = size_t(p->B) * p->G * p->L * p->top_k;
+  size_t o = msa::kWsHeader;
+  w.cnt = o; o = align_up(o + 4 * nbgj);
+  w.list_off = o; o = align_up(o + 4 * (nbgj + 1));
+  w.item_off = o; o = align_up(o + 4 * (nbgj + 1));
+  w.list = o; o = align_up(o + 4 * entries);
+  w.pos_of = o; o = align_up(o + 4 * entries);
+  w.delta = o; o = align_up(o + 4 * size_t(p->B) * p->L * p->H);
+  w.part_dq = o; o = align_up(o + 4 * entries * (p->H / p->G) * size_t(p->d));
+  w.end = o;
+  return w;
+}
+
 struct DecWs {
   size_t scores, sel, part_o, part_lse, end;
 };
@@ -454,6 +476,7 @@ size_t msa_workspace_bytes(const msa_params *p, int op) {
     case MSA_OP_PREFILL_ATTN: return attn_ws(p, msa::kWsHeader).end;
     case MSA_OP_DECODE: return dec_ws(p).end;
     case MSA_OP_FORWARD: return attn_ws(p, msa::kWsHeader + forward_sel_bytes(p)).end;
+    case MSA_OP_BACKWARD: return bwd_ws(p).end;
     default: fail(MSA_ERR_INVALID_ARG, "unknown op %d", op); return 0;
   }
 }
@@ -669,6 +692,69 @@ int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k
   e = cudaEventRecord(ev->done, ev->down);
   if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->done, 0);
   if (e != cudaSuccess) return cuda_fail(e, "download completion");
+  return MSA_OK;
+}
+
+int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
+                             const msa_bf16 *v, const msa_bf16 *out, const float *lse,
+                             const msa_bf16 *dout, const int32_t *sel, msa_bf16 *dq,
+                             msa_bf16 *dk, msa_bf16 *dv, void *ws, size_t ws_bytes,
+                             msa_stream stream) {
+  g_err[0] = 0;
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (p->B == 0 || p->L == 0) return MSA_OK;
+  if (!q || !k || !v || !out || !lse || !dout || !sel || !dq || !dk || !dv)
+    return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
+      !aligned16(dout) || !aligned16(sel) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const size_t entries = size_t(p->B) * p->G * p->L * p->top_k;
+  if (entries * (p->H / p->G) >= (size_t(1) << 31))
+    return fail(MSA_ERR_UNSUPPORTED, "B*L*H*top_k = %zu partial rows (limit 2^31)",
+                entries * (p->H / p->G));
+  const BwdWs w = bwd_ws(p);
+  rc = check_ws(ws, ws_bytes, w.end);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
+  const int nb = p->L / 128;
+  msa::RevIdxArgs ra;
+  ra.B = p->B; ra.G = p->G; ra.L = p->L; ra.nb = nb; ra.top_k = p->top_k;
+  ra.qpi = 128 / (p->H / p->G);
+  ra.Lq = p->L; ra.tq0 = 0; ra.t0 = 0; ra.Lc = p->L;
+  ra.sel = sel;
+  ra.cnt = reinterpret_cast<int32_t *>(wsb + w.cnt);
+  ra.list_off = reinterpret_cast<int32_t *>(wsb + w.list_off);
+  ra.item_off = reinterpret_cast<int32_t *>(wsb + w.item_off);
+  ra.list = reinterpret_cast<int32_t *>(wsb + w.list);
+  ra.pos_of = reinterpret_cast<int32_t *>(wsb + w.pos_of);
+  ra.status = status_ptr(ws);
+  cudaError_t e = msa::launch_revidx(ra, st);
+  if (e != cudaSuccess) return cuda_fail(e, "reverse index launch");
+  CUtensorMap tk, tv;
+  {
+    const uint64_t dims[3] = {uint64_t(p->d), uint64_t(p->G), uint64_t(p->B) * p->L};
+    const uint64_t str[2] = {uint64_t(p->d) * 2, uint64_t(p->d) * 2 * p->G};
+    const uint32_t box[3] = {64, 1, 128};
+    rc = make_tmap(&tk, k, 3, dims, str, box);
+    if (rc) return rc;
+    rc = make_tmap(&tv, v, 3, dims, str, box);
+    if (rc) return rc;
+  }
+  msa::BwdArgs a;
+  a.B = p->B; a.L = p->L; a.H = p->H; a.G = p->G; a.nb = nb; a.top_k = p->top_k;
+  a.scale = eff_scale(p);
+  a.scale_log2 = a.scale * 1.4426950408889634f;
+  a.q = q; a.out = out; a.dout = dout; a.lse = lse; a.sel = sel;
+  a.list = ra.list; a.list_off = ra.list_off; a.pos_of = ra.pos_of;
+  a.delta = reinterpret_cast<float *>(wsb + w.delta);
+  a.part_dq = reinterpret_cast<float *>(wsb + w.part_dq);
+  a.dq = dq; a.dk = dk; a.dv = dv;
+  a.unit_ctr = reinterpret_cast<int *>(wsb + 16);
+  a.status = status_ptr(ws);
+  e = msa::launch_backward(tk, tv, a, num_sms(), st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward launch");
   return MSA_OK;
 }
 

@@ -104,6 +104,16 @@ def prefill_inputs(shape: PrefillShape, seed: int, device="cpu",
     return out
 
 
+def output_grad(shape: PrefillShape, seed: int, device="cpu") -> torch.Tensor:
+    """Gradient arriving at the attention output, dout [B,L,H,d]: i.i.d.
+    N(0,1) sampled in fp32 and rounded to bf16, from its own seed stream
+    (seed + 3_000_017) so the forward inputs of the same seed are unchanged."""
+    s = shape
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed + 3_000_017)
+    return _normal_bf16(gen, (s.B, s.L, s.H, s.d), device)
+
+
 def decode_lengths(shape: DecodeShape, seed: int) -> torch.Tensor:
     """Ragged cache lengths, uniform integers in [len_lo, len_hi] (CPU int32)."""
     s = shape

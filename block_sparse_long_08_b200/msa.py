@@ -32,6 +32,7 @@ MSA_OP_INDEX_SELECT = 0
 MSA_OP_PREFILL_ATTN = 1
 MSA_OP_DECODE = 2
 MSA_OP_FORWARD = 3
+MSA_OP_BACKWARD = 4
 
 
 class MSAError(RuntimeError):
@@ -84,6 +85,8 @@ def lib() -> ctypes.CDLL:
         L.msa_sparse_attn_decode_fp8.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                                  _P, _SZ, _P]
         L.msa_sparse_attn_decode_noalloc.restype = ctypes.c_int
+        L.msa_sparse_attn_backward.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                               _SZ, _P]
         L.msa_workspace_bytes.argtypes = [pp, ctypes.c_int]
         L.msa_workspace_bytes.restype = _SZ
         L.msa_read_status.argtypes = [_P, _P]
@@ -94,7 +97,8 @@ def lib() -> ctypes.CDLL:
         for f in ("msa_index_select", "msa_sparse_attn_prefill", "msa_sparse_attn_decode",
                   "msa_forward", "msa_forward_host", "msa_forward_cached", "msa_read_status",
                   "msa_sparse_attn_decode_fp8idx", "msa_quantize_e4m3_rows",
-                  "msa_sparse_attn_decode_fp8", "msa_forward_cached_varlen"):
+                  "msa_sparse_attn_decode_fp8", "msa_forward_cached_varlen",
+                  "msa_sparse_attn_backward"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -203,6 +207,30 @@ def msa_sparse_attn_prefill(q, k, v, sel, *, scale: float = 0.0, want_lse: bool 
     _check(lib().msa_sparse_attn_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(sel),
                                          _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
     return (out, lse) if want_lse else out
+
+
+def msa_sparse_attn_backward(q, k, v, out, lse, dout, sel, *, scale: float = 0.0, dq=None,
+                             dk=None, dv=None, ws=None, stream=None):
+    """Main-branch gradients for a fixed selection: q [B,L,H,d], k/v
+    [B,L,G,d], the forward's out [B,L,H,d] and lse [B,L,H] fp32, dout
+    [B,L,H,d], sel [B,G,L,top_k] -> (dq, dk, dv) bf16, shaped like q, k, v."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        _req(t, n, torch.bfloat16)
+    _req(lse, "lse", torch.float32)
+    _req(sel, "sel", torch.int32)
+    B, L, H, d = q.shape
+    G = k.shape[2]
+    top_k = sel.shape[3]
+    p = make_params(B, L, H, G, d, 128, 128, top_k, scale)
+    dev = q.device
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    ws = _ensure_ws(ws, p, MSA_OP_BACKWARD, dev)
+    _check(lib().msa_sparse_attn_backward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                          _ptr(lse), _ptr(dout), _ptr(sel), _ptr(dq), _ptr(dk),
+                                          _ptr(dv), _ptr(ws), ws.numel(), _stream(stream)))
+    return dq, dk, dv
 
 
 def msa_forward(q, k, v, q_idx, k_idx, top_k: int, *, scale: float = 0.0, want_sel: bool = False,

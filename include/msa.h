@@ -92,7 +92,8 @@ enum {
   MSA_OP_INDEX_SELECT = 0,
   MSA_OP_PREFILL_ATTN = 1,
   MSA_OP_DECODE = 2,
-  MSA_OP_FORWARD = 3
+  MSA_OP_FORWARD = 3,
+  MSA_OP_BACKWARD = 4
 };
 
 /* Index Branch (explainer §2.1; researchpapers.dev "机制").
@@ -285,6 +286,30 @@ int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k
                      const msa_bf16 *v_h, const msa_bf16 *q_idx_h, const msa_bf16 *k_idx_h,
                      msa_bf16 *out_h, float *lse_h, const msa_staging *dev, void *ws,
                      size_t ws_bytes, msa_stream stream, msa_stream copy_stream);
+
+/* Main Branch, backward pass (researchpapers.dev "机制", training
+ * paragraph: the index path is cut from the main attention's gradient, so
+ * the selection is a constant and only q, k and v receive gradients).
+ *   q [B,L,H,d], k [B,L,G,d], v [B,L,G,d] bf16: forward inputs        (in)
+ *   out [B,L,H,d] bf16, lse [B,L,H] fp32: msa_sparse_attn_prefill's
+ *     outputs for the same inputs and selection                       (in)
+ *   dout [B,L,H,d] bf16: gradient of the loss with respect to out     (in)
+ *   sel [B,G,L,top_k] int32: the forward's selection                  (in)
+ *   dq [B,L,H,d], dk [B,L,G,d], dv [B,L,G,d] bf16                    (out)
+ * For each (t, h) with probabilities P over its attended tokens s:
+ * dZ_s = P_s (do . v_s - do . o), dq = scale sum_s dZ_s k_s, and every
+ * attended token gets dk_s += scale dZ_s q, dv_s += P_s do; tokens no query
+ * attends to get zero.  dq is bit-identical from run to run; dk and dv sum
+ * a key block's queries in the reverse index's list order, which follows
+ * atomics, so runs agree up to fp32 summation order.  ws >= msa_workspace_bytes(p, MSA_OP_BACKWARD): the
+ * reverse index plus one fp32 dq partial row per (query, head, slot),
+ * B*L*H*top_k*512 bytes (8.6 GB at L = 32K, H = 32, top_k = 16); there is
+ * no query chunking, so the size is bounded by device memory. */
+int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
+                             const msa_bf16 *v, const msa_bf16 *out, const float *lse,
+                             const msa_bf16 *dout, const int32_t *sel, msa_bf16 *dq,
+                             msa_bf16 *dk, msa_bf16 *dv, void *ws, size_t ws_bytes,
+                             msa_stream stream);
 
 /* Workspace bytes op (MSA_OP_*) needs for these params; 0 when p is invalid
  * (see msa_last_error). */

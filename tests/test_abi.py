@@ -137,3 +137,24 @@ def test_varlen_rejects_bad_ranges():
 def test_decode_rejects_more_than_eight_groups():
     p = M.make_params(2, 4096, 32, 16, 128, 128, 128, 16)
     assert M.lib().msa_workspace_bytes(ctypes.byref(p), M.MSA_OP_DECODE) == 0
+
+
+def test_backward_rejects_bad_arguments():
+    """Argument checks of msa_sparse_attn_backward run before any CUDA call."""
+    p = M.make_params(1, 1024, 8, 2, 128, 128, 128, 4)
+    lib = M.lib()
+    ok = ctypes.c_void_p(4096)
+    need = M.msa_workspace_bytes(p, M.MSA_OP_BACKWARD)
+    args = [ok] * 10
+    rc = lib.msa_sparse_attn_backward(ctypes.byref(p), *args[:4], None, *args[5:], ok, need, None)
+    assert rc == M.MSA_ERR_INVALID_ARG                       # lse is required
+    bad = list(args)
+    bad[6] = ctypes.c_void_p(4096 + 4)                        # misaligned sel
+    rc = lib.msa_sparse_attn_backward(ctypes.byref(p), *bad, ok, need, None)
+    assert rc == M.MSA_ERR_INVALID_ARG
+    rc = lib.msa_sparse_attn_backward(ctypes.byref(p), *args, ok, need - 1, None)
+    assert rc == M.MSA_ERR_WORKSPACE
+    # workspace: reverse index + D + one fp32 dq row per (query, head, slot)
+    assert need >= 1024 * 8 * 4 * 128 * 4 + 1024 * 8 * 4
+    p0 = M.make_params(0, 1024, 8, 2, 128, 128, 128, 4)
+    assert lib.msa_sparse_attn_backward(ctypes.byref(p0), *([None] * 10), None, 0, None) == M.MSA_OK
