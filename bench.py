@@ -102,7 +102,7 @@ def prefill_attn_bytes(B, L, H, G, d, top_k):
 def prefill_bwd_bytes(B, L, H, G, d, top_k):
     """Bytes the key-block-outer backward must move: every selected (query,
     group, block) entry gathers its R q rows and R do rows, reads R lse and
-    D values, and writes and reads back R fp32 dq partial rows; K/V are read
+    D values, and writes and reads back R bf16 dq partial rows; K/V are read
     once per key block and dk/dv written once; D = do . o reads o and do,
     and dq is written once."""
     t = np.arange(L, dtype=np.int64)
@@ -110,7 +110,7 @@ def prefill_bwd_bytes(B, L, H, G, d, top_k):
     r = H // G
     rows = B * float(L) * H * d * 2
     kv = B * float(L) * G * d * 2
-    return entries * r * (d * 2 * 2 + d * 4 * 2 + 8) + 3 * rows + 4 * kv
+    return entries * r * (d * 2 * 2 + d * 2 * 2 + 8) + 3 * rows + 4 * kv
 
 
 def prefill_bwd_flops(B, L, H, d, top_k):

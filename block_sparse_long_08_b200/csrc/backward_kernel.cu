@@ -20,12 +20,13 @@
 //   dV_j += P^T dO, dK_j += dZ^T Q       (UMMA, A operand MN-major: the
 //                                         same tiles read transposed)
 //   dQ_part = dZ K_j                     (UMMA into TMEM cols 0-127)
-//   dQ_part * scale -> fp32 partial row of (list position, head)
+//   dQ_part * scale -> bf16 partial row of (list position, head)
 // and after the unit's last item dK_j (* scale) and dV_j leave as bf16.  A
 // second kernel sums each query row's <= top_k partials into dq.  The next
-// item's gather and the next unit's K/V loads are issued as soon as the
-// MMAs that read those buffers complete, so they overlap the dQ and dK/dV
-// epilogues.  Units are handed out by an atomic counter, low key blocks
+// item's gather starts as soon as the dV/dK products have read the q/do
+// tiles (the dQ product has its own commit), and the next unit's K/V loads
+// as soon as the dQ product has read K; both overlap the epilogues.  The dQ
+// partial rows are staged in the P tile and leave by bulk copy.  Units are handed out by an atomic counter, low key blocks
 // (the longest lists) first.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -43,7 +44,7 @@ constexpr int kTileB = 32768;                 // 128 rows x 256 B
 // shared memory (from a 1024-byte aligned base)
 constexpr int kSK = 0, kSV = kTileB, kSQ = 2 * kTileB, kSDO = 3 * kTileB, kSP = 4 * kTileB,
               kSDZ = 5 * kTileB, kSCtl = 6 * kTileB;
-constexpr int kBarKv = 0, kBarQ = 1, kBarMma = 2, kBarDrain = 3;
+constexpr int kBarKv = 0, kBarQ = 1, kBarMma = 2, kBarDrain = 3, kBarDq = 4;
 constexpr int kCtlHolder = 32, kCtlAbort = 36, kCtlUnit = 40;
 constexpr int kBwdSmem = kSCtl + 64 + 1024;
 static_assert(kBwdSmem <= 232448, "shared memory budget");
@@ -82,6 +83,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(bar(kBarQ), kBwdThreads);   // one cp.async completion per thread
     mbar_init(bar(kBarMma), 1);
     mbar_init(bar(kBarDrain), 1);
+    mbar_init(bar(kBarDq), 1);
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -140,20 +142,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tma_load_3d(s_base + kSV, &tm_v, bar(kBarKv), 0, un.g, z);
     tma_load_3d(s_base + kSV + 16384, &tm_v, bar(kBarKv), 64, un.g, z);
   };
-  // q and do rows of item `it` of a unit (all threads): row pairs
-  // p = warp + 8 i (rows 2p, 2p+1), one 512-byte copy per warp instruction
-  auto gather = [&](const Unit &un, int it) {
+  // Query positions of this thread's eight gather rows of item `it` of a
+  // unit (-1 past the item's end): row pairs p = warp + 8 i (rows 2p, 2p+1).
+  auto gather_rows = [&](const Unit &un, int it, int (&tq)[8]) {
     const int start = un.l_lo + it * QPI;
     const int n = min(QPI, un.n_q - it * QPI);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {   // all loads first: one memory latency
+      const int qi = (2 * (warp + 8 * i) + (lane >> 4)) / R;
+      tq[i] = qi < n ? (a.list[start + qi] >> 5) : -1;
+    }
+  };
+  // q and do rows of a unit's item (all threads), one 512-byte copy per warp
+  // instruction, given the rows' query positions
+  auto gather = [&](const Unit &un, const int (&tq)[8]) {
     const int gran = lane & 15;
     const uint32_t off_g = (gran >> 3) * 16384;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int r = 2 * (warp + 8 * i) + (lane >> 4);
-      const int qi = r / R;
-      if (qi < n) {
-        const int t = a.list[start + qi] >> 5;
-        const size_t src = ((size_t(un.b) * a.L + t) * a.H + un.g * R + r % R) * kHeadDim + gran * 8;
+      if (tq[i] >= 0) {
+        const size_t src =
+            ((size_t(un.b) * a.L + tq[i]) * a.H + un.g * R + r % R) * kHeadDim + gran * 8;
         const uint32_t dst = off_g + sw128_offset(r, gran & 7);
         cp_async16(s_base + kSQ + dst, a.q + src);
         cp_async16(s_base + kSDO + dst, a.dout + src);
@@ -172,7 +182,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       load_kv(cur);
       kv_inflight = true;
     }
-    gather(cur, 0);
+    int tq0[8];
+    gather_rows(cur, 0, tq0);
+    gather(cur, tq0);
   }
   int it = 0;          // item of the current unit
   uint32_t n_items = 0, n_units_done = 0;
@@ -193,6 +205,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       dlt = a.delta[ri];
       lim = min(kBlock - 1, t - cur.j * kBlock);
     }
+    // the next item's gather rows, when it belongs to this unit: loaded now,
+    // their latency hides behind this item's products
+    int tq_next[8];
+    const bool next_in_unit = (it + 1) * QPI < cur.n_q;
+    if (next_in_unit) gather_rows(cur, it + 1, tq_next);
     // ---- S = Q K^T, dP = dO V^T
     ok = mbar_wait(bar(kBarQ), n_items & 1, abort_flag, a.status);
     if (ok && it == 0) ok = mbar_wait(bar(kBarKv), n_units_done & 1, abort_flag, a.status);
@@ -218,6 +235,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       umma_commit(bar(kBarMma));
     }
     ok = mbar_wait(bar(kBarMma), 0, abort_flag, a.status);
+    if (lane == 0 && half == 0) bulk_wait_read_all();   // the last item's staged dq rows
     if (!__syncthreads_and(ok)) break;
     tc_fence_after();
     // ---- P and dZ (bf16, key columns half*64 .. +64 of this row)
@@ -268,48 +286,66 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         umma_f16_ss(tmem_base + kTmDK, sdesc_sw128(s_base + kSDZ + off, 16384, 1024),
                     sdesc_sw128(s_base + kSQ + off, 16384, 1024), idesc_t, (it > 0 || kk > 0));
       }
+      umma_commit(bar(kBarMma));   // the q/do tiles are free once these complete
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {   // K = 16 keys per step
         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
         umma_f16_ss(tmem_base + kTmS, sdesc_sw128(s_base + kSDZ + off, 16, 1024),
                     sdesc_sw128(s_base + kSK + kk * 2048, 16384, 1024), idesc_q, kk > 0);
       }
-      umma_commit(bar(kBarMma));
+      umma_commit(bar(kBarDq));
     }
     ok = mbar_wait(bar(kBarMma), 1, abort_flag, a.status);
     if (!__syncthreads_and(ok)) break;
-    tc_fence_after();
     ++n_items;
-    // ---- the q/do tiles, and at a unit's end the K/V tiles, are free: start
-    // the next item's copies before the epilogues
-    const bool unit_end = (it + 1) * QPI >= cur.n_q;
+    // ---- the q/do tiles are free: start the next item's copies while the
+    // dQ product and the epilogues run
+    const bool unit_end = !next_in_unit;
     Unit nxt = cur;
     bool have_next = true;
-    if (unit_end) {
-      have_next = fetch_unit(nxt);
-      if (have_next && tid == 0) {
-        load_kv(nxt);
-        kv_inflight = true;
-      }
+    if (unit_end) have_next = fetch_unit(nxt);
+    if (have_next) {
+      if (unit_end) gather_rows(nxt, 0, tq_next);
+      gather(nxt, tq_next);
     }
-    if (have_next) gather(nxt, unit_end ? 0 : it + 1);
-    // ---- dQ partial rows: (list position start + qi, head hh) -> row start*R + r
+    ok = mbar_wait(bar(kBarDq), (n_items - 1) & 1, abort_flag, a.status);
+    if (!__syncthreads_and(ok)) break;
+    tc_fence_after();
+    // the K/V tiles (read by the dQ product) are free at a unit's end
+    if (unit_end && have_next && tid == 0) {
+      load_kv(nxt);
+      kv_inflight = true;
+    }
+    // ---- dQ partial rows: (list position start + qi, head hh) -> partial
+    // row rho = start*R + r, bf16, its 16-byte granule c at c ^ (rho & 7);
+    // staged in the P tile (free now) and written with one bulk copy per
+    // 32 rows
     {
       float q0[32], q1[32];
-      tmem_ld32(tm_row + kTmS + half * 64, q0);   // warp-wide: before the row test
+      tmem_ld32(tm_row + kTmS + half * 64, q0);
       tmem_ld32(tm_row + kTmS + half * 64 + 32, q1);
       tmem_wait_ld();
-      if (row < n * R) {
-      float4 *dst = reinterpret_cast<float4 *>(a.part_dq + (size_t(start) * R + row) * kHeadDim +
-                                               half * 64);
+      const int rho7 = (start * R + row) & 7;
+      uint8_t *srow = smem + kSP + row * 256;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        dst[c] = make_float4(q0[4 * c] * a.scale, q0[4 * c + 1] * a.scale, q0[4 * c + 2] * a.scale,
-                             q0[4 * c + 3] * a.scale);
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-        dst[8 + c] = make_float4(q1[4 * c] * a.scale, q1[4 * c + 1] * a.scale,
-                                 q1[4 * c + 2] * a.scale, q1[4 * c + 3] * a.scale);
+      for (int c = 0; c < 8; ++c) {
+        const float *x = c < 4 ? q0 + 8 * c : q1 + 8 * (c - 4);
+        const uint4 w = make_uint4(pack_bf16x2(x[0] * a.scale, x[1] * a.scale),
+                                   pack_bf16x2(x[2] * a.scale, x[3] * a.scale),
+                                   pack_bf16x2(x[4] * a.scale, x[5] * a.scale),
+                                   pack_bf16x2(x[6] * a.scale, x[7] * a.scale));
+        *reinterpret_cast<uint4 *>(srow + ((half * 8 + (c ^ rho7)) << 4)) = w;
+      }
+      fence_proxy_async_smem();
+      __syncthreads();   // both halves of each row staged
+      if (half == 0 && lane == 0) {
+        const int wrow0 = warp * 32;
+        const int nrows = min(32, n * R - wrow0);
+        if (nrows > 0) {
+          bulk_store(a.part_dq + (size_t(start) * R + wrow0) * kHeadDim,
+                     s_base + kSP + wrow0 * 256, uint32_t(nrows) * 256u);
+          bulk_commit();
+        }
       }
     }
     // ---- unit end: dK_j (* scale) and dV_j rows (key = TMEM lane) as bf16
@@ -349,6 +385,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // nothing may still be landing in shared memory or running on the tensor
   // cores when the CTA releases them
   cp_async_wait_all();
+  if (lane == 0 && half == 0) bulk_wait_all();
   if (tid == 0) {
     if (kv_inflight) mbar_wait_drain(bar(kBarKv), n_units_done & 1);
     if (mma_issued) {
@@ -400,17 +437,21 @@ __global__ void __launch_bounds__(256) bwd_dq_reduce_kernel(const BwdArgs a) {
   const bool in_k = lane < a.top_k;
   const int my_sel = in_k ? a.sel[e0 + lane] : -1;
   const long long my_rho = (my_sel >= 0) ? (long long)a.pos_of[e0 + lane] * r + hh : -1;
-  float4 v[KCAP];
+  uint2 v[KCAP];
 #pragma unroll
   for (int s = 0; s < KCAP; ++s) {
     const long long rho = __shfl_sync(0xffffffffu, my_rho, s);
-    v[s] = rho >= 0 ? __ldcs(reinterpret_cast<const float4 *>(a.part_dq + rho * kHeadDim) + lane)
-                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    v[s] = make_uint2(0u, 0u);
+    if (rho >= 0) {
+      const int col = (((lane >> 1) ^ int(rho & 7)) << 3) | ((lane & 1) << 2);
+      v[s] = __ldcs(reinterpret_cast<const uint2 *>(a.part_dq + rho * kHeadDim + col));
+    }
   }
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
   for (int s = 0; s < KCAP; ++s) {
-    acc.x += v[s].x; acc.y += v[s].y; acc.z += v[s].z; acc.w += v[s].w;
+    acc.x += bf16_lo(v[s].x); acc.y += bf16_hi(v[s].x);
+    acc.z += bf16_lo(v[s].y); acc.w += bf16_hi(v[s].y);
   }
   *reinterpret_cast<uint2 *>(a.dq + w * kHeadDim + lane * 4) =
       make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));

@@ -90,7 +90,9 @@ struct BwdArgs {
   const int32_t *sel;          // [B,G,L,top_k]
   const int32_t *list, *list_off, *pos_of;   // reverse index (see RevIdxArgs)
   float *delta;                // [B,L,H]: do . o
-  float *part_dq;              // [entries*R, d] fp32: dq of (list position, head), scaled
+  // dq of (list position, head), scaled, bf16 [entries*R, d]; granule c
+  // of partial row rho is stored at granule c ^ (rho & 7) (as AttnArgs)
+  uint16_t *part_dq;
   uint16_t *dq;                // [B,L,H,d]
   uint16_t *dk, *dv;           // [B,L,G,d]
   int *unit_ctr;               // work counter (zeroed by the launcher)

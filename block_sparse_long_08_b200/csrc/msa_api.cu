@@ -108,7 +108,7 @@ AttnWs attn_ws(const msa_params *p, size_t base) {
 }
 
 // Backward: a whole-sequence reverse index, D = do . o per row, and one
-// fp32 dq partial row per (query, head, slot).
+// bf16 dq partial row per (query, head, slot).
 struct BwdWs {
   size_t cnt, list_off, item_off, list, pos_of, delta, part_dq, end;
 };
@@ -124,7 +124,7 @@ BwdWs bwd_ws(const msa_params *p) {
   w.list = o; o = align_up(o + 4 * entries);
   w.pos_of = o; o = align_up(o + 4 * entries);
   w.delta = o; o = align_up(o + 4 * size_t(p->B) * p->L * p->H);
-  w.part_dq = o; o = align_up(o + 4 * entries * (p->H / p->G) * size_t(p->d));
+  w.part_dq = o; o = align_up(o + 2 * entries * (p->H / p->G) * size_t(p->d));
   w.end = o;
   return w;
 }
@@ -749,7 +749,7 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
   a.q = q; a.out = out; a.dout = dout; a.lse = lse; a.sel = sel;
   a.list = ra.list; a.list_off = ra.list_off; a.pos_of = ra.pos_of;
   a.delta = reinterpret_cast<float *>(wsb + w.delta);
-  a.part_dq = reinterpret_cast<float *>(wsb + w.part_dq);
+  a.part_dq = reinterpret_cast<uint16_t *>(wsb + w.part_dq);
   a.dq = dq; a.dk = dk; a.dv = dv;
   a.unit_ctr = reinterpret_cast<int *>(wsb + 16);
   a.status = status_ptr(ws);

@@ -302,8 +302,8 @@ int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k
  * attends to get zero.  dq is bit-identical from run to run; dk and dv sum
  * a key block's queries in the reverse index's list order, which follows
  * atomics, so runs agree up to fp32 summation order.  ws >= msa_workspace_bytes(p, MSA_OP_BACKWARD): the
- * reverse index plus one fp32 dq partial row per (query, head, slot),
- * B*L*H*top_k*512 bytes (8.6 GB at L = 32K, H = 32, top_k = 16); there is
+ * reverse index plus one bf16 dq partial row per (query, head, slot),
+ * B*L*H*top_k*256 bytes (4.3 GB at L = 32K, H = 32, top_k = 16); there is
  * no query chunking, so the size is bounded by device memory. */
 int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
                              const msa_bf16 *v, const msa_bf16 *out, const float *lse,

@@ -155,6 +155,6 @@ def test_backward_rejects_bad_arguments():
     rc = lib.msa_sparse_attn_backward(ctypes.byref(p), *args, ok, need - 1, None)
     assert rc == M.MSA_ERR_WORKSPACE
     # workspace: reverse index + D + one fp32 dq row per (query, head, slot)
-    assert need >= 1024 * 8 * 4 * 128 * 4 + 1024 * 8 * 4
+    assert need >= 1024 * 8 * 4 * 128 * 2 + 1024 * 8 * 4
     p0 = M.make_params(0, 1024, 8, 2, 128, 128, 128, 4)
     assert lib.msa_sparse_attn_backward(ctypes.byref(p0), *([None] * 10), None, 0, None) == M.MSA_OK
