@@ -52,8 +52,9 @@ static_assert(kBwdSmem <= 232448, "shared memory budget");
 // TMEM columns: S / dQ, dP, dV, dK (128 lanes x 128 fp32 each).
 constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDV = 256, kTmDK = 384;
 
+// One (b, g, key block j) unit: its reverse-index list [l_lo, l_lo + n_q).
 struct Unit {
-  int u, bgj, b, g, j, l_lo, n_q;
+  int bgj, b, g, j, l_lo, n_q;
 };
 
 template <int R>
@@ -115,7 +116,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int u = *s_unit;
       __syncthreads();
       if (u >= n_units) return false;
-      un.u = u;
       un.j = u / n_bg;
       const int bg = u % n_bg;
       un.b = bg / a.G;

@@ -39,6 +39,12 @@ def test_workspace_sizes(L, top_k, G, H, di):
     assert lc % 128 == 0 and 128 <= lc <= L
     assert ws_att >= lc * H * top_k * 128 * 2
     assert ws_dec < 64 * 2**20
+    # backward: whole-sequence reverse index, D, one bf16 dq row per (query,
+    # head, slot); no chunking, so it grows with L
+    ws_bwd = M.msa_workspace_bytes(p, M.MSA_OP_BACKWARD)
+    entries = L * G * top_k
+    assert ws_bwd >= entries * (H // G) * 128 * 2 + 2 * 4 * entries + 4 * L * H
+    assert ws_bwd <= entries * (H // G) * 128 * 2 + 2 * 4 * entries + 4 * L * H + 2 * 2**20
 
 
 @pytest.mark.parametrize("field,value,code", [
