@@ -22,7 +22,11 @@
 //   dQ_part = dZ K_j                     (UMMA into TMEM cols 0-127)
 //   dQ_part * scale -> bf16 partial row of (list position, head)
 // and after the unit's last item dK_j (* scale) and dV_j leave as bf16.  A
-// second kernel sums each query row's <= top_k partials into dq.  The next
+// second kernel sums each query row's <= top_k partials into dq.  Long
+// inputs run in query chunks, each with its own reverse index; dK/dV are
+// then carried across chunks in fp32 accumulators (read, added to and
+// rewritten by the one CTA that owns the block) and the last chunk writes
+// them as bf16.  The next
 // item's gather starts as soon as the dV/dK products have read the q/do
 // tiles (the dQ product has its own commit), and the next unit's K/V loads
 // as soon as the dQ product has read K; both overlap the epilogues.  The dQ
@@ -51,6 +55,39 @@ static_assert(kBwdSmem <= 232448, "shared memory budget");
 
 // TMEM columns: S / dQ, dP, dV, dK (128 lanes x 128 fp32 each).
 constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDV = 256, kTmDK = 384;
+
+// 32 consecutive dk or dv values of one row (element offset e0): x * f for
+// this query chunk (x null: nothing from this chunk).  A single-chunk call
+// writes them as bf16.  With several chunks they are added to the fp32
+// accumulator (zeroed before the first chunk), and the last chunk writes
+// the sum as bf16.
+__device__ __forceinline__ void put_grad32(const float *x, float f, size_t e0, uint16_t *out,
+                                           float *acc, bool last) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = x ? x[i] * f : 0.f;
+  if (acc) {
+    const float4 *src = reinterpret_cast<const float4 *>(acc + e0);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 w = src[c];
+      v[4 * c] += w.x; v[4 * c + 1] += w.y; v[4 * c + 2] += w.z; v[4 * c + 3] += w.w;
+    }
+  }
+  if (!acc || last) {
+    uint4 *dst = reinterpret_cast<uint4 *>(out + e0);
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      dst[c] = make_uint4(pack_bf16x2(v[8 * c], v[8 * c + 1]), pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
+                          pack_bf16x2(v[8 * c + 4], v[8 * c + 5]),
+                          pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+  } else {
+    float4 *dst = reinterpret_cast<float4 *>(acc + e0);
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      dst[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+  }
+}
 
 // One (b, g, key block j) unit: its reverse-index list [l_lo, l_lo + n_q).
 struct Unit {
@@ -124,13 +161,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       un.l_lo = a.list_off[un.bgj];
       un.n_q = a.list_off[un.bgj + 1] - un.l_lo;
       if (un.n_q > 0) return true;
+      if (a.acc_dk && !a.last) continue;   // an earlier or later chunk writes this block
       const size_t r0 = ((size_t(un.b) * a.L + size_t(un.j) * kBlock + row) * a.G + un.g) *
                             kHeadDim + half * 64;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        reinterpret_cast<uint4 *>(a.dk + r0)[c] = make_uint4(0u, 0u, 0u, 0u);
-        reinterpret_cast<uint4 *>(a.dv + r0)[c] = make_uint4(0u, 0u, 0u, 0u);
-      }
+      put_grad32(nullptr, 0.f, r0, a.dk, a.acc_dk, a.last);
+      put_grad32(nullptr, 0.f, r0 + 32, a.dk, a.acc_dk, a.last);
+      put_grad32(nullptr, 0.f, r0, a.dv, a.acc_dv, a.last);
+      put_grad32(nullptr, 0.f, r0 + 32, a.dv, a.acc_dv, a.last);
     }
   };
   // K_j and V_j of a unit into their tiles (thread 0)
@@ -352,26 +389,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (unit_end) {
       const size_t r0 = ((size_t(cur.b) * a.L + size_t(cur.j) * kBlock + row) * a.G + cur.g) *
                             kHeadDim + half * 64;
-#pragma unroll
+#pragma unroll 1
       for (int m = 0; m < 2; ++m) {
         float x0[32], x1[32];
         tmem_ld32(tm_row + (m ? kTmDK : kTmDV) + half * 64, x0);
         tmem_ld32(tm_row + (m ? kTmDK : kTmDV) + half * 64 + 32, x1);
         tmem_wait_ld();
         const float f = m ? a.scale : 1.f;
-        uint4 *dst = reinterpret_cast<uint4 *>((m ? a.dk : a.dv) + r0);
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          dst[c] = make_uint4(pack_bf16x2(x0[8 * c] * f, x0[8 * c + 1] * f),
-                              pack_bf16x2(x0[8 * c + 2] * f, x0[8 * c + 3] * f),
-                              pack_bf16x2(x0[8 * c + 4] * f, x0[8 * c + 5] * f),
-                              pack_bf16x2(x0[8 * c + 6] * f, x0[8 * c + 7] * f));
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          dst[4 + c] = make_uint4(pack_bf16x2(x1[8 * c] * f, x1[8 * c + 1] * f),
-                                  pack_bf16x2(x1[8 * c + 2] * f, x1[8 * c + 3] * f),
-                                  pack_bf16x2(x1[8 * c + 4] * f, x1[8 * c + 5] * f),
-                                  pack_bf16x2(x1[8 * c + 6] * f, x1[8 * c + 7] * f));
+        uint16_t *out = m ? a.dk : a.dv;
+        float *acc = m ? a.acc_dk : a.acc_dv;
+        put_grad32(x0, f, r0, out, acc, a.last);
+        put_grad32(x1, f, r0 + 32, out, acc, a.last);
       }
       ++n_units_done;
     }
@@ -425,18 +453,20 @@ template <int KCAP>
 __global__ void __launch_bounds__(256) bwd_dq_reduce_kernel(const BwdArgs a) {
   const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  const long long n_rows = (long long)a.B * a.L * a.H;
+  const long long n_rows = (long long)a.B * a.Lc * a.H;   // the chunk's rows
   if (w >= n_rows) return;
   const int h = (int)(w % a.H);
   const long long bt = w / a.H;
-  const int t = (int)(bt % a.L);
-  const int b = (int)(bt / a.L);
+  const int tl = (int)(bt % a.Lc);
+  const int b = (int)(bt / a.Lc);
+  const int t = a.t0 + tl;
   const int r = a.H / a.G;
   const int g = h / r, hh = h % r;
-  const size_t e0 = ((size_t(b) * a.G + g) * a.L + t) * a.top_k;
+  const size_t es = ((size_t(b) * a.G + g) * a.L + t) * a.top_k;     // sel row
+  const size_t ep = ((size_t(b) * a.G + g) * a.Lc + tl) * a.top_k;   // pos_of row (chunk)
   const bool in_k = lane < a.top_k;
-  const int my_sel = in_k ? a.sel[e0 + lane] : -1;
-  const long long my_rho = (my_sel >= 0) ? (long long)a.pos_of[e0 + lane] * r + hh : -1;
+  const int my_sel = in_k ? a.sel[es + lane] : -1;
+  const long long my_rho = (my_sel >= 0) ? (long long)a.pos_of[ep + lane] * r + hh : -1;
   uint2 v[KCAP];
 #pragma unroll
   for (int s = 0; s < KCAP; ++s) {
@@ -453,7 +483,7 @@ __global__ void __launch_bounds__(256) bwd_dq_reduce_kernel(const BwdArgs a) {
     acc.x += bf16_lo(v[s].x); acc.y += bf16_hi(v[s].x);
     acc.z += bf16_lo(v[s].y); acc.w += bf16_hi(v[s].y);
   }
-  *reinterpret_cast<uint2 *>(a.dq + w * kHeadDim + lane * 4) =
+  *reinterpret_cast<uint2 *>(a.dq + ((size_t(b) * a.L + t) * a.H + h) * kHeadDim + lane * 4) =
       make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
 }
 
@@ -471,14 +501,18 @@ cudaError_t launch_bwd_r(const CUtensorMap &tk, const CUtensorMap &tv, const Bwd
 
 }  // namespace
 
-cudaError_t launch_backward(const CUtensorMap &tk, const CUtensorMap &tv, const BwdArgs &a,
-                            int num_sms, cudaStream_t st) {
+cudaError_t launch_bwd_delta(const BwdArgs &a, cudaStream_t st) {
   const long long rows = (long long)a.B * a.L * a.H;
   if (rows == 0) return cudaSuccess;
-  cudaError_t e = cudaMemsetAsync(a.unit_ctr, 0, sizeof(int), st);
-  if (e != cudaSuccess) return e;
   bwd_delta_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(a.out, a.dout, a.delta, rows);
-  e = cudaGetLastError();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_backward(const CUtensorMap &tk, const CUtensorMap &tv, const BwdArgs &a,
+                            int num_sms, cudaStream_t st) {
+  const long long rows = (long long)a.B * a.Lc * a.H;
+  if (rows == 0) return cudaSuccess;
+  cudaError_t e = cudaMemsetAsync(a.unit_ctr, 0, sizeof(int), st);
   if (e != cudaSuccess) return e;
   switch (a.H / a.G) {
     case 1: e = launch_bwd_r<1>(tk, tv, a, num_sms, st); break;

@@ -80,9 +80,12 @@ struct CombineArgs {
 };
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
 
-// Main-branch backward over a whole-sequence reverse index (t0 = 0, Lc = L).
+// Main-branch backward for the query chunk [t0, t0 + Lc), over that chunk's
+// reverse index.
 struct BwdArgs {
   int B, L, H, G, nb, top_k;
+  int t0, Lc;
+  int last;                    // the last query chunk (writes dk, dv when chunked)
   float scale, scale_log2;
   const uint16_t *q;           // [B,L,H,d]
   const uint16_t *out, *dout;  // [B,L,H,d]: forward output and its gradient
@@ -95,11 +98,15 @@ struct BwdArgs {
   uint16_t *part_dq;
   uint16_t *dq;                // [B,L,H,d]
   uint16_t *dk, *dv;           // [B,L,G,d]
+  // fp32 [B,L,G,d] dk/dv accumulators across query chunks (zeroed before the
+  // first chunk), or null for a single chunk
+  float *acc_dk, *acc_dv;
   int *unit_ctr;               // work counter (zeroed by the launcher)
   int *status;
 };
+cudaError_t launch_bwd_delta(const BwdArgs &a, cudaStream_t st);   // D for all rows
 cudaError_t launch_backward(const CUtensorMap &tk, const CUtensorMap &tv, const BwdArgs &a,
-                            int num_sms, cudaStream_t st);
+                            int num_sms, cudaStream_t st);      // one chunk: kernel + dq sums
 
 struct DecodeArgs {
   int B, Lmax, H, G, d_idx, nb_max, top_k;

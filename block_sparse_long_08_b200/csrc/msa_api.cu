@@ -107,16 +107,19 @@ AttnWs attn_ws(const msa_params *p, size_t base) {
   return w;
 }
 
-// Backward: a whole-sequence reverse index, D = do . o per row, and one
-// bf16 dq partial row per (query, head, slot).
+// Backward: D = do . o per row; per query chunk (the prefill's chunk length)
+// a reverse index and one bf16 dq partial row per (query, head, slot); with
+// more than one chunk, fp32 dk/dv accumulators over the whole sequence.
 struct BwdWs {
-  size_t cnt, list_off, item_off, list, pos_of, delta, part_dq, end;
+  size_t cnt, list_off, item_off, list, pos_of, delta, part_dq, acc_dk, acc_dv, end;
+  int Lc;
 };
 BwdWs bwd_ws(const msa_params *p) {
   BwdWs w;
+  w.Lc = prefill_chunk(p);
   const size_t nb = size_t(p->L) / 128;
   const size_t nbgj = size_t(p->B) * p->G * nb;
-  const size_t entries = size_t(p->B) * p->G * p->L * p->top_k;
+  const size_t entries = size_t(p->B) * p->G * w.Lc * p->top_k;
   size_t o = msa::kWsHeader;
   w.cnt = o; o = align_up(o + 4 * nbgj);
   w.list_off = o; o = align_up(o + 4 * (nbgj + 1));
@@ -125,6 +128,12 @@ BwdWs bwd_ws(const msa_params *p) {
   w.pos_of = o; o = align_up(o + 4 * entries);
   w.delta = o; o = align_up(o + 4 * size_t(p->B) * p->L * p->H);
   w.part_dq = o; o = align_up(o + 2 * entries * (p->H / p->G) * size_t(p->d));
+  w.acc_dk = w.acc_dv = 0;
+  if (w.Lc < p->L) {
+    const size_t kv = 4 * size_t(p->B) * p->L * p->G * p->d;
+    w.acc_dk = o; o = align_up(o + kv);
+    w.acc_dv = o; o = align_up(o + kv);
+  }
   w.end = o;
   return w;
 }
@@ -709,29 +718,16 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(lse) ||
       !aligned16(dout) || !aligned16(sel) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-  const size_t entries = size_t(p->B) * p->G * p->L * p->top_k;
-  if (entries * (p->H / p->G) >= (size_t(1) << 31))
-    return fail(MSA_ERR_UNSUPPORTED, "B*L*H*top_k = %zu partial rows (limit 2^31)",
-                entries * (p->H / p->G));
   const BwdWs w = bwd_ws(p);
+  const size_t entries = size_t(p->B) * p->G * w.Lc * p->top_k;
+  if (entries * (p->H / p->G) >= (size_t(1) << 31))
+    return fail(MSA_ERR_UNSUPPORTED, "B*chunk*H*top_k = %zu partial rows (limit 2^31)",
+                entries * (p->H / p->G));
   rc = check_ws(ws, ws_bytes, w.end);
   if (rc) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
   const int nb = p->L / 128;
-  msa::RevIdxArgs ra;
-  ra.B = p->B; ra.G = p->G; ra.L = p->L; ra.nb = nb; ra.top_k = p->top_k;
-  ra.qpi = 128 / (p->H / p->G);
-  ra.Lq = p->L; ra.tq0 = 0; ra.t0 = 0; ra.Lc = p->L;
-  ra.sel = sel;
-  ra.cnt = reinterpret_cast<int32_t *>(wsb + w.cnt);
-  ra.list_off = reinterpret_cast<int32_t *>(wsb + w.list_off);
-  ra.item_off = reinterpret_cast<int32_t *>(wsb + w.item_off);
-  ra.list = reinterpret_cast<int32_t *>(wsb + w.list);
-  ra.pos_of = reinterpret_cast<int32_t *>(wsb + w.pos_of);
-  ra.status = status_ptr(ws);
-  cudaError_t e = msa::launch_revidx(ra, st);
-  if (e != cudaSuccess) return cuda_fail(e, "reverse index launch");
   CUtensorMap tk, tv;
   {
     const uint64_t dims[3] = {uint64_t(p->d), uint64_t(p->G), uint64_t(p->B) * p->L};
@@ -742,6 +738,17 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
     rc = make_tmap(&tv, v, 3, dims, str, box);
     if (rc) return rc;
   }
+  msa::RevIdxArgs ra;
+  ra.B = p->B; ra.G = p->G; ra.L = p->L; ra.nb = nb; ra.top_k = p->top_k;
+  ra.qpi = 128 / (p->H / p->G);
+  ra.Lq = p->L; ra.tq0 = 0;
+  ra.sel = sel;
+  ra.cnt = reinterpret_cast<int32_t *>(wsb + w.cnt);
+  ra.list_off = reinterpret_cast<int32_t *>(wsb + w.list_off);
+  ra.item_off = reinterpret_cast<int32_t *>(wsb + w.item_off);
+  ra.list = reinterpret_cast<int32_t *>(wsb + w.list);
+  ra.pos_of = reinterpret_cast<int32_t *>(wsb + w.pos_of);
+  ra.status = status_ptr(ws);
   msa::BwdArgs a;
   a.B = p->B; a.L = p->L; a.H = p->H; a.G = p->G; a.nb = nb; a.top_k = p->top_k;
   a.scale = eff_scale(p);
@@ -751,10 +758,28 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
   a.delta = reinterpret_cast<float *>(wsb + w.delta);
   a.part_dq = reinterpret_cast<uint16_t *>(wsb + w.part_dq);
   a.dq = dq; a.dk = dk; a.dv = dv;
+  a.acc_dk = w.acc_dk ? reinterpret_cast<float *>(wsb + w.acc_dk) : nullptr;
+  a.acc_dv = w.acc_dv ? reinterpret_cast<float *>(wsb + w.acc_dv) : nullptr;
   a.unit_ctr = reinterpret_cast<int *>(wsb + 16);
   a.status = status_ptr(ws);
-  e = msa::launch_backward(tk, tv, a, num_sms(), st);
-  if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+  cudaError_t e = msa::launch_bwd_delta(a, st);
+  if (e != cudaSuccess) return cuda_fail(e, "backward D launch");
+  if (a.acc_dk) {
+    e = cudaMemsetAsync(wsb + w.acc_dk, 0, w.acc_dv - w.acc_dk, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(wsb + w.acc_dv, 0, w.end - w.acc_dv, st);
+    if (e != cudaSuccess) return cuda_fail(e, "backward accumulator reset");
+  }
+  const int sms = num_sms();
+  for (int t0 = 0; t0 < p->L; t0 += w.Lc) {
+    const int Lc = (p->L - t0) < w.Lc ? (p->L - t0) : w.Lc;
+    ra.t0 = t0; ra.Lc = Lc;
+    e = msa::launch_revidx(ra, st);
+    if (e != cudaSuccess) return cuda_fail(e, "reverse index launch");
+    a.t0 = t0; a.Lc = Lc;
+    a.last = (t0 + Lc >= p->L) ? 1 : 0;
+    e = msa::launch_backward(tk, tv, a, sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "backward launch");
+  }
   return MSA_OK;
 }
 

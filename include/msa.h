@@ -301,10 +301,13 @@ int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k
  * attended token gets dk_s += scale dZ_s q, dv_s += P_s do; tokens no query
  * attends to get zero.  dq is bit-identical from run to run; dk and dv sum
  * a key block's queries in the reverse index's list order, which follows
- * atomics, so runs agree up to fp32 summation order.  ws >= msa_workspace_bytes(p, MSA_OP_BACKWARD): the
- * reverse index plus one bf16 dq partial row per (query, head, slot),
- * B*L*H*top_k*256 bytes (4.3 GB at L = 32K, H = 32, top_k = 16); there is
- * no query chunking, so the size is bounded by device memory. */
+ * atomics, so runs agree up to fp32 summation order.
+ * Queries are processed in the prefill's chunks (msa_prefill_chunk_len;
+ * p->chunk overrides it), each with its own reverse index and one bf16 dq
+ * partial row per (query, head, slot) of the chunk (at most about 16 GiB).
+ * With more than one chunk, dk and dv are summed across chunks in fp32
+ * accumulators (2 * B*L*G*d*4 bytes of workspace) and rounded to bf16 once.
+ * ws >= msa_workspace_bytes(p, MSA_OP_BACKWARD). */
 int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
                              const msa_bf16 *v, const msa_bf16 *out, const float *lse,
                              const msa_bf16 *dout, const int32_t *sel, msa_bf16 *dq,

@@ -150,3 +150,33 @@ def test_backward_32k_sampled():
             gv[tok[m] - j * blk] += gvt[m]
         _grad_close(f"dk block {j} g={g} ({rows.size} rows)", P.f64(dk[0, j * blk:(j + 1) * blk, g]), gk)
         _grad_close(f"dv block {j} g={g}", P.f64(dv[0, j * blk:(j + 1) * blk, g]), gv)
+
+
+def test_backward_query_chunks():
+    """Four query chunks of 256 (p->chunk): dq equals the one-chunk run bit
+    for bit (each partial row depends only on its own query row); dk and dv
+    are summed across chunks in fp32 and match the oracle under the same
+    bounds.  A selection leaving blocks unselected keeps them at zero
+    through every chunk."""
+    shape = I.PrefillShape(B=2, L=1024, H=8, G=2, d=128, d_idx=128, top_k=3)
+    x = _inputs(shape, 27)
+    out, sel, lse = M.msa_forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], 3,
+                                  want_sel=True, want_lse=True)
+    one = M.msa_sparse_attn_backward(x["q"], x["k"], x["v"], out, lse, x["dout"], sel)
+    four = M.msa_sparse_attn_backward(x["q"], x["k"], x["v"], out, lse, x["dout"], sel, chunk=256)
+    torch.cuda.synchronize()
+    assert torch.equal(one[0], four[0])
+    ref = O.prefill_backward(x["q"], x["k"], x["v"], sel.cpu().numpy(), x["dout"], block=128)
+    for name, g in zip(("dq", "dk", "dv"), four):
+        _grad_close(f"{name} (4 chunks)", P.f64(g), ref[name])
+    # block 0 only: blocks 1.. are attended by nobody in any chunk
+    sel0 = torch.full_like(sel, -1)
+    sel0[..., 0] = 0
+    out0, lse0 = M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel0, want_lse=True)
+    dq0, dk0, dv0 = M.msa_sparse_attn_backward(x["q"], x["k"], x["v"], out0, lse0, x["dout"], sel0,
+                                               chunk=128)
+    torch.cuda.synchronize()
+    assert not dk0[:, 128:].any() and not dv0[:, 128:].any()
+    ref0 = O.prefill_backward(x["q"], x["k"], x["v"], sel0.cpu().numpy(), x["dout"], block=128)
+    _grad_close("dk block 0 (8 chunks)", P.f64(dk0[:, :128]), ref0["dk"][:, :128])
+    _grad_close("dv block 0 (8 chunks)", P.f64(dv0[:, :128]), ref0["dv"][:, :128])
