@@ -60,6 +60,7 @@ def _forward_backward(x, top_k, sel=None):
     (1, 768, 32, 2, 2, 22),      # R = 16 (8 queries per item)
     (1, 512, 8, 1, 8, 23),       # top_k >= nb: dense causal attention
     (1, 1152, 16, 8, 1, 24),     # top_k = 1: the local block only
+    (1, 2560, 16, 2, 17, 28),    # R = 8, top_k = 17 (32-slot dq reduction)
 ])
 def test_backward_matches_oracle(B, L, H, G, top_k, seed):
     shape = I.PrefillShape(B=B, L=L, H=H, G=G, d=128, d_idx=128, top_k=top_k)
