@@ -16,6 +16,10 @@
  *     16 blocks x 128 tokens per query group.
  *   Decode        -- explainer §4.1: each new token scores the cache and
  *     attends only to its selected blocks.
+ *   Backward      -- researchpapers.dev section "机制", training paragraph:
+ *     the index branch is trained separately (KL loss) and its path into
+ *     the main attention carries no gradient, so the main branch is
+ *     differentiated with the selection held fixed.
  *
  * Definition implemented (readings where the pages are silent are marked R):
  *   S[b,g,t,j] = max_{s in block j, s <= t} sum_i q_idx[b,t,g,i]*k_idx[b,s,i]
@@ -27,6 +31,8 @@
  *   out[b,t,h] = softmax_s(scale * q[b,t,h].k[b,s,g]) . v[b,s,g]  over the
  *                tokens s <= t of the blocks in sel[b,g,t], g = h/(H/G).
  *                (R: scale = 1/sqrt(d) when params.scale == 0)
+ *   dq, dk, dv = gradients of sum(dout * out) with respect to q, k, v, for
+ *                a given sel (a constant).
  *
  * Conventions for every entry point:
  *   - Tensors are DEVICE pointers, row-major, contiguous, 16-byte aligned.
@@ -72,10 +78,10 @@ typedef struct msa_params {
   int32_t block;   /* KV block length (128) */
   int32_t top_k;   /* blocks kept per (query, group), local block included */
   float scale;     /* softmax scale of the main branch; 0 -> 1/sqrt(d) */
-  int32_t chunk;   /* prefill query-chunk length, a multiple of 128; 0 -> the
-                      longest chunk whose partials fit the 16 GiB budget.
-                      Smaller chunks need a smaller workspace and re-read
-                      K/V more often. */
+  int32_t chunk;   /* query-chunk length of the prefill attention and the
+                      backward, a multiple of 128; 0 -> the longest chunk
+                      whose partials fit the 16 GiB budget.  Smaller chunks
+                      need a smaller workspace and re-read K/V more often. */
 } msa_params;
 
 enum {
