@@ -2,6 +2,7 @@
 point its header declares, sizes workspaces and rejects bad arguments
 before touching the device."""
 import ctypes
+import os
 
 import pytest
 
@@ -167,3 +168,50 @@ def test_backward_rejects_bad_arguments():
     assert need >= 1024 * 8 * 4 * 128 * 2 + 1024 * 8 * 4
     p0 = M.make_params(0, 1024, 8, 2, 128, 128, 128, 4)
     assert lib.msa_sparse_attn_backward(ctypes.byref(p0), *([None] * 10), None, 0, None) == M.MSA_OK
+
+
+def test_plain_c_program_uses_the_library(tmp_path):
+    """The boundary is a C ABI: a C99 program, compiled with warnings as
+    errors against include/msa.h alone, links libmsa.so and calls its
+    host-side entry points (workspace sizing, argument checks, version)
+    without Python or torch."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(M.LIB_PATH)
+    src = tmp_path / "use_msa.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "msa.h"
+int main(void) {
+  msa_params p;
+  memset(&p, 0, sizeof p);
+  p.B = 1; p.L = 32768; p.H = 32; p.G = 8; p.d = 128; p.d_idx = 128; p.block = 128;
+  p.top_k = 16;
+  size_t w = msa_workspace_bytes(&p, MSA_OP_BACKWARD);
+  int rc = msa_index_select(&p, NULL, NULL, NULL, NULL, NULL, 0, NULL);
+  printf("%s|%zu|%d|%s\n", msa_version(), w, rc, msa_last_error());
+  return (w > 0 && rc == MSA_ERR_INVALID_ARG) ? 0 : 1;
+}
+''')
+    exe = tmp_path / "use_msa"
+    cuda_lib = "/usr/local/cuda/lib64"
+    cmd = [gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+           "-I" + os.path.join(root, "include"), str(src), "-o", str(exe),
+           "-L" + libdir, "-lmsa", "-Wl,-rpath," + libdir]
+    if os.path.isdir(cuda_lib):
+        cmd += ["-L" + cuda_lib, "-Wl,-rpath," + cuda_lib]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, (r.stdout, r.stderr)
+    version, ws, rc, msg = r.stdout.strip().split("|")
+    assert "sm_100a" in version
+    assert int(ws) == M.msa_workspace_bytes(M.make_params(1, 32768, 32, 8, top_k=16),
+                                            M.MSA_OP_BACKWARD)
+    assert int(rc) == M.MSA_ERR_INVALID_ARG and msg
