@@ -215,3 +215,17 @@ int main(void) {
     assert int(ws) == M.msa_workspace_bytes(M.make_params(1, 32768, 32, 8, top_k=16),
                                             M.MSA_OP_BACKWARD)
     assert int(rc) == M.MSA_ERR_INVALID_ARG and msg
+
+
+def test_backward_workspace_follows_chunking():
+    """One chunk: no dk/dv accumulators.  Several chunks (p.chunk): the
+    reverse index and dq partials shrink to one chunk, and fp32 dk/dv
+    accumulators for the whole sequence are added."""
+    L, H, G, K = 4096, 16, 4, 8
+    whole = M.msa_workspace_bytes(M.make_params(1, L, H, G, top_k=K), M.MSA_OP_BACKWARD)
+    half = M.msa_workspace_bytes(M.make_params(1, L, H, G, top_k=K, chunk=L // 2),
+                                 M.MSA_OP_BACKWARD)
+    per_chunk = lambda lc: lc * G * K * (H // G) * 128 * 2 + 2 * 4 * lc * G * K
+    acc = 2 * L * G * 128 * 4
+    assert abs((whole - per_chunk(L)) - (half - per_chunk(L // 2) - acc)) <= 4096
+    assert M.msa_prefill_chunk_len(M.make_params(1, L, H, G, top_k=K, chunk=L // 2)) == L // 2
