@@ -39,11 +39,13 @@ import torch  # noqa: E402
 
 METRIC = "MSA prefill tokens/s & decode µs/step at 128K/1M; % of B200 roofline"
 BLOCK = 128
+SPEC_BF16_TFLOPS = 2250.0   # dense bf16 tensor peak of the part (spec sheet)
+SPEC_HBM_GBS = 8000.0       # HBM3e bandwidth of the part (spec sheet)
 
 # DRAM bytes (read + write) of one msa_index_kernel launch on the 1M-token
 # workload, from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum,
-# a single-pass metric set; see profiles/dram_traffic_msa_1m_and_decode_128k.md).
-# Keyed to the kernel source it was measured on: a changed kernel reports null.
+# a single-pass metric set).  Keyed to the kernel source it was measured on:
+# a changed kernel reports null.
 INDEX_TRAFFIC_1M = {"bytes": 1.6911e11, "source_sha256_16": "269f1bcdede015c9"}
 
 
@@ -63,10 +65,12 @@ def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
+        clk = d.get("clocks_under_load", {}).get("sm_mhz_median")
         return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "sm_mhz": clk,
+                "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
-            "source": "fallback"}
+            "sm_mhz": None, "source": "fallback"}
 
 
 # --------------------------------------------------------------------- work
@@ -225,59 +229,115 @@ def dist_barrier(ws: int):
 
 
 # --------------------------------------------------------------------- oracle leg
+def _bits(t: torch.Tensor) -> np.ndarray:
+    """Host copy of a bf16 tensor as its raw 16-bit patterns (numpy)."""
+    return t.to("cpu").contiguous().view(torch.int16).numpy()
+
+
+def _f64(bits: np.ndarray) -> np.ndarray:
+    """Exact fp64 values of bf16 bit patterns (a bf16 value is the upper half
+    of the fp32 with the same bits)."""
+    return (bits.astype(np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
 class OracleLeg:
-    """Times the fp64 oracle, as it stands, on a bounded sample of the step:
-    prefill query positions drawn uniformly from [0, L) (every group and head
-    of each) plus whole decode sequences.  A prefill row's cost grows with t,
-    so uniform positions keep the per-row mean unbiased; the sample time is
-    scaled to a whole step.  Host copies are made before the clock starts."""
+    """Times the fp64 oracle, as it stands, on the host cores.
 
-    def __init__(self, x, dx, shape, dshape):
+    Prefill work is timed per query position (every group and head of the
+    position); decode work per whole sequence.  Host copies (bf16 K/V rows,
+    the fp64 index keys) are made before any clock starts.  A prefill
+    position's cost grows with t, so sampled positions are stratified: [0, L)
+    is cut into n equal strata with one uniform position in each, and the
+    whole prefill's oracle time is extrapolated as the sum over strata of the
+    stratum's width times its position's time."""
+
+    def __init__(self, x=None, dx=None, shape=None, dshape=None):
         self.x, self.dx, self.shape, self.dshape = x, dx, shape, dshape
-        self.k = x["k"][0].to("cpu")
-        self.v = x["v"][0].to("cpu")
-        self.k_idx64 = x["k_idx"][0].to("cpu").double().numpy()
-        self.dec = {}
+        self._pre = None
 
-    def _dec_host(self, b):
-        if b not in self.dec:
-            dx = self.dx
-            self.dec[b] = (dx["q"][b].to("cpu"), dx["q_idx"][b].to("cpu"), dx["k_cache"][b].to("cpu"),
-                           dx["v_cache"][b].to("cpu"), dx["k_idx_cache"][b].to("cpu").double().numpy(),
-                           int(dx["seq_lens"][b]))
-        return self.dec[b]
+    def _prefill_host(self):
+        if self._pre is None:
+            x, B = self.x, self.shape.B
+            self._pre = [(_bits(x["k"][b]), _bits(x["v"][b]),
+                          x["k_idx"][b].to("cpu").double().numpy()) for b in range(B)]
+        return self._pre
 
-    def sample(self, rng, n_tok, n_dec):
+    def prefill_positions(self, positions):
+        """Oracle seconds of each (b, t) position (all groups and heads)."""
         import oracle.msa_oracle as O
         f64 = O.as_f64
-        shape, dshape = self.shape, self.dshape
-        L, H, G, d, top_k = shape.L, shape.H, shape.G, shape.d, shape.top_k
-        r = H // G
-        sc = 1.0 / math.sqrt(d)
-        ts = sorted(rng.integers(0, L, size=n_tok).tolist())
-        q_rows = self.x["q"][0, ts].to("cpu")
-        qi_rows = self.x["q_idx"][0, ts].to("cpu")
-        bsel = sorted(rng.choice(dshape.B, size=n_dec, replace=False).tolist())
-        decs = [self._dec_host(b) for b in bsel]
-        t0 = time.perf_counter()
-        for n, t in enumerate(ts):
-            for g in range(G):
-                bs = O.block_scores_row(f64(qi_rows[n, g]), self.k_idx64, t, BLOCK)
-                blocks = O.select_blocks_row(bs, t, BLOCK, top_k)
-                tok = torch.from_numpy(O.selected_tokens(blocks, t, BLOCK))
-                O.attend_rows(f64(q_rows[n, g * r:(g + 1) * r]), f64(self.k[tok, g]), f64(self.v[tok, g]), sc)
-        t_pre = time.perf_counter() - t0
-        t1 = time.perf_counter()
-        for (q, qi, kc, vc, ki64, n) in decs:
+        s = self.shape
+        r = s.H // s.G
+        sc = 1.0 / math.sqrt(s.d)
+        host = self._prefill_host()
+        pos = list(positions)
+        q_rows = [self.x["q"][b, t].to("cpu") for (b, t) in pos]
+        qi_rows = [self.x["q_idx"][b, t].to("cpu") for (b, t) in pos]
+        times = []
+        for n, (b, t) in enumerate(pos):
+            k, v, k_idx64 = host[b]
+            t0 = time.perf_counter()
+            for g in range(s.G):
+                bs = O.block_scores_row(f64(qi_rows[n][g]), k_idx64, t, s.block)
+                blocks = O.select_blocks_row(bs, t, s.block, s.top_k)
+                tok = O.selected_tokens(blocks, t, s.block)
+                O.attend_rows(f64(q_rows[n][g * r:(g + 1) * r]), _f64(k[tok, g]), _f64(v[tok, g]),
+                              sc)
+            times.append(time.perf_counter() - t0)
+        return times
+
+    def prefill_full(self):
+        """(seconds, (query, group) rows) of the oracle over every position."""
+        s = self.shape
+        times = self.prefill_positions([(b, t) for b in range(s.B) for t in range(s.L)])
+        return sum(times), s.B * s.L * s.G
+
+    def prefill_stratified(self, rng, n_strata):
+        """(sampled seconds, extrapolated whole-prefill seconds, sampled rows)."""
+        s = self.shape
+        pos, width = [], []
+        for b in range(s.B):
+            for i in range(n_strata):
+                lo, hi = i * s.L // n_strata, (i + 1) * s.L // n_strata
+                if hi > lo:
+                    pos.append((b, int(rng.integers(lo, hi))))
+                    width.append(hi - lo)
+        times = self.prefill_positions(pos)
+        return sum(times), sum(w * tm for w, tm in zip(width, times)), len(pos) * s.G
+
+    def decode_sequences(self, seqs):
+        """Oracle seconds of whole decode sequences (every group and head).
+        One sequence's caches are on the host at a time."""
+        import oracle.msa_oracle as O
+        f64 = O.as_f64
+        dx, s = self.dx, self.dshape
+        r = s.H // s.G
+        sc = 1.0 / math.sqrt(s.d)
+        total = 0.0
+        for b in seqs:
+            n = int(dx["seq_lens"][b])
+            q, qi = dx["q"][b].to("cpu"), dx["q_idx"][b].to("cpu")
+            kc, vc = _bits(dx["k_cache"][b, :n]), _bits(dx["v_cache"][b, :n])
+            ki64 = dx["k_idx_cache"][b, :n].to("cpu").double().numpy()
             t = n - 1
-            for g in range(dshape.G):
-                bs = O.block_scores_row(f64(qi[g]), ki64, t, BLOCK)
-                blocks = O.select_blocks_row(bs, t, BLOCK, dshape.top_k)
-                tok = torch.from_numpy(O.selected_tokens(blocks, t, BLOCK))
-                O.attend_rows(f64(q[g * r:(g + 1) * r]), f64(kc[tok, g]), f64(vc[tok, g]), sc)
-        t_dec = time.perf_counter() - t1
-        est = t_pre * (L / n_tok) * shape.B + t_dec * (dshape.B / n_dec)
-        return t_pre + t_dec, est
+            t0 = time.perf_counter()
+            for g in range(s.G):
+                bs = O.block_scores_row(f64(qi[g]), ki64, t, s.block)
+                blocks = O.select_blocks_row(bs, t, s.block, s.top_k)
+                tok = O.selected_tokens(blocks, t, s.block)
+                O.attend_rows(f64(q[g * r:(g + 1) * r]), _f64(kc[tok, g]), _f64(vc[tok, g]), sc)
+            total += time.perf_counter() - t0
+            del kc, vc, ki64
+        return total
+
+    def sample(self, rng, n_tok, n_dec):
+        """Bounded sample of one step (the reference arm): n_tok stratified
+        prefill positions and n_dec decode sequences.  Returns (sampled
+        seconds, extrapolated seconds of the whole step)."""
+        t_pre, est_pre, _ = self.prefill_stratified(rng, n_tok)
+        bsel = sorted(rng.choice(self.dshape.B, size=n_dec, replace=False).tolist())
+        t_dec = self.decode_sequences(bsel)
+        return t_pre + t_dec, est_pre + t_dec * (self.dshape.B / n_dec)
 
 
 # --------------------------------------------------------------------- main
@@ -289,6 +349,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the tiny / 32K / 128K-planted prefill legs")
     ap.add_argument("--workload", default="1m", choices=["1m", "128k", "32k", "8k"],
                     help="prefill length of the step (1m is the headline workload; 8k is a "
                          "small-footprint case for profiler captures)")
@@ -452,6 +514,15 @@ def run_ours(args, shape, dshape, seed, cfg, ws_n, rank, local):
                 "unit": "TFLOP/s", "frac": None, "traffic": index_traffic(args.workload),
                 "kernel": "msa_index_kernel", "peak_kind": f"bf16 sustained ({peaks['source']})"}
     roof_idx["frac"] = roof_idx["achieved"] / peak_t
+    # The sustained peak was measured at a power-capped median clock; the
+    # index kernel runs at its own power-capped clock.  Secondary fractions:
+    # against the measured peak scaled to the clock sampled during this run,
+    # and against the 2.25 PFLOP/s dense bf16 spec.
+    if clk.get("sm_mhz") and peaks.get("sm_mhz"):
+        scaled = peak_t * clk["sm_mhz"] / peaks["sm_mhz"]
+        roof_idx["peak_clock_scaled"] = scaled
+        roof_idx["frac_clock_scaled"] = roof_idx["achieved"] / scaled
+    roof_idx["frac_of_spec"] = roof_idx["achieved"] / SPEC_BF16_TFLOPS
     b_att = prefill_attn_bytes(B, L, H, G, d, K)
     roof_att = {"bound": "hbm", "achieved": b_att / (att_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "bytes": b_att,
@@ -488,17 +559,28 @@ def run_ours(args, shape, dshape, seed, cfg, ws_n, rank, local):
     if not args.no_e2e:
         line["e2e"] = bench_e2e(M, x, dx, shape, dshape, K, args, ws_n, stream)
 
+    # ---- every configuration at 1 GPU: the 1M step above, decode-128K, and
+    # the tiny, 32K and 128K-planted prefills, each beside the oracle
+    if rank == 0 and ws_n == 1 and not args.no_configs:
+        line["per_config"] = bench_configs(M, I, dev, args, peaks, line)
+
     # ---- oracle on the host cores
     if not args.no_cpu_baseline and rank == 0 and ws_n == 1:
         leg = OracleLeg(x, dx, shape, dshape)
         rng = np.random.default_rng(seed)
-        n_tok, n_dec = 24, 1
-        t_s, est = leg.sample(rng, n_tok, n_dec)
+        n_strata = 64
+        t_pre, est_pre, rows = leg.prefill_stratified(rng, n_strata)
+        t_dec = leg.decode_sequences(range(dshape.B))
+        est = est_pre + t_dec
         line["cpu_baseline"] = {
-            "value": tokens_per_step / est, "unit": "tokens/s", "cores": os.cpu_count(),
-            "kind": "oracle",
-            "sample": f"{n_tok} prefill query positions uniform in [0,L) (all {G} groups, {H} heads) "
-                      f"+ {n_dec} of {dshape.B} decode sequences; {t_s:.1f} s of CPU, scaled to one step"}
+            "value": tokens_per_step / est, "unit": "tokens/s", "cores": oracle_threads(),
+            "kind": "oracle", "extrapolated": True, "seconds_per_step": est,
+            "sample": f"prefill: {rows} (query, group) rows, one uniform position in each of "
+                      f"{n_strata} equal strata of [0,L) with all {G} groups and {H} heads, "
+                      f"{t_pre:.1f} s, extrapolated to the whole prefill by stratum width; "
+                      f"decode: all {dshape.B} sequences in full, {t_dec:.1f} s"}
+        if "per_config" in line:
+            line["per_config"]["1m"]["oracle"] = line["cpu_baseline"]
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws_n > 1:
@@ -630,6 +712,14 @@ def bench_decode_128k(M, I, dev, args, peaks):
     us8 = timed(run_fp8)
     us88 = timed(run_all_fp8)
     lens = y["seq_lens"].numpy()
+    oracle = None
+    if not args.no_cpu_baseline:   # the full oracle: every sequence, every group and head
+        del codes, kscale, k8, ks8, v8, vs8
+        secs = OracleLeg(None, y, None, ds).decode_sequences(range(ds.B))
+        oracle = {"seconds": secs, "us_per_step": secs * 1e6, "cores": oracle_threads(),
+                  "kind": "oracle", "extrapolated": False,
+                  "sample": f"all {ds.B} sequences, every group and head"}
+        codes = kscale = k8 = ks8 = v8 = vs8 = None
     byts = decode_bytes(lens, ds.H, ds.G, ds.d, ds.d_idx, ds.top_k)
     byts8 = decode_bytes(lens, ds.H, ds.G, ds.d, ds.d_idx, ds.top_k, fp8_index=True)
     byts88 = decode_bytes(lens, ds.H, ds.G, ds.d, ds.d_idx, ds.top_k, fp8_index=True, fp8_kv=True)
@@ -642,7 +732,7 @@ def bench_decode_128k(M, I, dev, args, peaks):
                                 "cache": "k_idx as E4M3 codes + fp32 scale per token"},
             "fp8_all_caches": {"us_per_step": us88, "roofline": roof(byts88, us88),
                                "cache": "k_idx, K and V as E4M3 codes + fp32 scales"},
-            "gpu_launches": 12 * iters}
+            "gpu_launches": 12 * iters, "oracle": oracle}
 
 
 def bench_backward_32k(M, I, dev, args, peaks):
@@ -691,6 +781,148 @@ def bench_backward_32k(M, I, dev, args, peaks):
             "tensor": {"flops": fl, "tflops": fl / (ms / 1e3) / 1e12,
                        "frac_of_sustained": fl / (ms / 1e3) / 1e12 / peaks["bf16_tflops_sustained"]},
             "gpu_launches": 6 * iters}
+
+
+def oracle_threads() -> int:
+    """Threads the oracle runs on: numpy's BLAS pool (matrix products) or
+    torch's intra-op pool (row gathers), whichever is larger."""
+    n = torch.get_num_threads()
+    try:
+        from threadpoolctl import threadpool_info
+        n = max([n] + [int(i.get("num_threads", 1)) for i in threadpool_info()])
+    except Exception:
+        pass
+    return int(n)
+
+
+def needle_hit_rate(sel: torch.Tensor, needle_blocks: torch.Tensor):
+    """Over every query t after group g's first needle block and every needle
+    block j < t/128 of g: how often j is in sel[0, g, t].  sel [1,G,L,K]."""
+    G, L = sel.shape[1], sel.shape[2]
+    bt = torch.arange(L, device=sel.device) // BLOCK
+    hit = tot = 0
+    for g in range(G):
+        js = needle_blocks[g].tolist()
+        start = (min(js) + 1) * BLOCK
+        rows, btg = sel[0, g, start:], bt[start:]
+        for j in js:
+            vis = btg > j
+            tot += int(vis.sum())
+            hit += int(((rows == j).any(-1) & vis).sum())
+    return hit, tot
+
+
+def bench_prefill_config(M, I, dev, args, peaks, name, shape, seed, needles=0,
+                         oracle_full=False, n_strata=64, iters=10):
+    """One prefill configuration at 1 GPU: msa_index_select (fused top-k) then
+    msa_sparse_attn_prefill, as in the step, timed per launch with CUDA events
+    and an L2 flush between iterations; rooflines of both ops; the oracle on
+    the host cores beside it (every position, or stratified positions
+    extrapolated to the whole prefill)."""
+    x = I.prefill_inputs(shape, seed, device=dev, needles=needles, needle_alpha=3.0)
+    B, L, H, G, d, di, K = shape.B, shape.L, shape.H, shape.G, shape.d, shape.d_idx, shape.top_k
+    p = M.make_params(B, L, H, G, d, di, BLOCK, K)
+    ws_idx = M.new_workspace(p, M.MSA_OP_INDEX_SELECT, dev)
+    ws_att = M.new_workspace(p, M.MSA_OP_PREFILL_ATTN, dev)
+    sel = torch.empty((B, G, L, K), dtype=torch.int32, device=dev)
+    out = torch.empty_like(x["q"])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx)
+        M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att)
+    torch.cuda.synchronize()
+    if M.msa_read_status(ws_idx) != 0 or M.msa_read_status(ws_att) != 0:
+        raise SystemExit(f"{name}: device status error")
+    t_idx, t_att, t_pre = [], [], []
+    for _ in range(iters):
+        flush.zero_()   # L2 flush (256 MB > 126 MB L2) outside the timed span
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(stream)
+        M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx)
+        ev[1].record(stream)
+        M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att)
+        ev[2].record(stream)
+        torch.cuda.synchronize()
+        t_idx.append(ev[0].elapsed_time(ev[1]))
+        t_att.append(ev[1].elapsed_time(ev[2]))
+        t_pre.append(ev[0].elapsed_time(ev[2]))
+    idx_ms, att_ms, pre_ms = (statistics.median(v) for v in (t_idx, t_att, t_pre))
+    f_idx = prefill_index_flops(B, L, G, di, K)
+    f_main = prefill_main_flops(B, L, H, d, K)
+    b_att = prefill_attn_bytes(B, L, H, G, d, K)
+    burst = peaks["bf16_tflops"]
+    nchunks = math.ceil(L / M.msa_prefill_chunk_len(p))
+    res = {"workload": f"B={B} L={L} H={H} G={G} d={d} d_idx={di} block={BLOCK} top_k={K}"
+                       + (f", {needles} planted needle blocks per group (alpha 3)" if needles else ""),
+           "seed": seed, "iters": iters, "l2": "256 MB buffer written between iterations",
+           "prefill_ms": pre_ms, "tokens_per_s": B * L / (pre_ms / 1e3),
+           "index_ms": idx_ms, "attn_ms": att_ms,
+           "prefill_tensor": {"flops": f_idx + f_main,
+                              "tflops": (f_idx + f_main) / (pre_ms / 1e3) / 1e12,
+                              "frac_of_burst": (f_idx + f_main) / (pre_ms / 1e3) / 1e12 / burst,
+                              "frac_of_spec": (f_idx + f_main) / (pre_ms / 1e3) / 1e12
+                              / SPEC_BF16_TFLOPS},
+           "index_roofline": {"bound": "tensor", "achieved": f_idx / (idx_ms / 1e3) / 1e12,
+                              "peak": burst, "unit": "TFLOP/s",
+                              "frac": f_idx / (idx_ms / 1e3) / 1e12 / burst, "flops": f_idx,
+                              "peak_kind": f"bf16 burst ({peaks['source']}): kernel timed alone"},
+           "attn_roofline": {"bound": "hbm", "achieved": b_att / (att_ms / 1e3) / 1e9,
+                             "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": b_att / (att_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                             "bytes": b_att, "tflops": f_main / (att_ms / 1e3) / 1e12},
+           "gpu_launches": (1 + 5 * nchunks) * iters}
+    if needles:
+        hit, tot = needle_hit_rate(sel, x["needle_blocks"])
+        res["needle_hit_rate"] = {"alpha": 3.0, "hits": hit, "of": tot,
+                                  "rate": hit / tot if tot else None}
+    del ws_att, out, flush
+    torch.cuda.empty_cache()
+    if not args.no_cpu_baseline:
+        leg = OracleLeg(x, None, shape, None)
+        if oracle_full:
+            secs, rows = leg.prefill_full()
+            sample = f"every position: {rows} (query, group) rows"
+        else:
+            rng = np.random.default_rng(seed)
+            t_s, secs, rows = leg.prefill_stratified(rng, n_strata)
+            sample = (f"{rows} (query, group) rows: one uniform position in each of {n_strata} "
+                      f"equal strata of [0,L), all groups and heads; {t_s:.1f} s, extrapolated to "
+                      f"the whole prefill by stratum width")
+        res["oracle"] = {"seconds": secs, "tokens_per_s": B * L / secs, "cores": oracle_threads(),
+                         "kind": "oracle", "extrapolated": not oracle_full, "sample": sample}
+        res["gpu_over_oracle"] = secs / (pre_ms / 1e3)
+    del x, sel
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_configs(M, I, dev, args, peaks, line):
+    """Every configuration at 1 GPU.  The 1M step and decode-128K were timed
+    above; the tiny, 32K and 128K-planted prefills are timed here."""
+    cfgs = {}
+    cfgs["tiny"] = bench_prefill_config(M, I, dev, args, peaks, "tiny", I.PREFILL_TINY,
+                                        I.SEEDS["tiny"], oracle_full=True, iters=20)
+    cfgs["32k"] = bench_prefill_config(M, I, dev, args, peaks, "32k", I.PREFILL_32K,
+                                       I.SEEDS["32k"], iters=10)
+    cfgs["128k_planted"] = bench_prefill_config(M, I, dev, args, peaks, "128k_planted",
+                                                I.PREFILL_128K_PLANTED, I.SEEDS["128k_planted"],
+                                                needles=12, iters=5)
+    if "decode_128k" in line:
+        d = line["decode_128k"]
+        cfgs["decode_128k"] = {"us_per_step": d["us_per_step"], "roofline": d["roofline"],
+                               "frac_of_8tbs": d["roofline"]["achieved"] / SPEC_HBM_GBS,
+                               "oracle": d.get("oracle")}
+    bd = line["breakdown"]
+    cfgs["1m"] = {"ms_per_step": line["ms_per_step"], "tokens_per_s": line["value"],
+                  "prefill_tokens_per_s": bd["prefill_tokens_per_s"],
+                  "index_roofline": line["roofline"],
+                  "prefill_tensor_frac_of_spec": (bd["index_flops"] + bd["main_flops"])
+                  / ((bd["index_ms"] + bd["prefill_attn_ms"]) / 1e3) / 1e12 / SPEC_BF16_TFLOPS,
+                  "attn_roofline": bd["prefill_attn_roofline"],
+                  "decode_us": bd["decode_us"], "decode_roofline": bd["decode_roofline"],
+                  "decode_frac_of_8tbs": bd["decode_roofline"]["achieved"] / SPEC_HBM_GBS}
+    return cfgs
 
 
 def bench_e2e(M, x, dx, shape, dshape, K, args, ws_n, stream):

@@ -16,6 +16,7 @@
 // streams, or graphs replayed concurrently) race on it; callers must order
 // such calls.  The status word at the start of the array is cleared on every
 // call; nothing else in it needs to start at zero.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -31,12 +32,24 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
+// The array's device address belongs to the module as loaded in one CUDA
+// context.  cudaDeviceReset destroys the device's primary context, and the
+// next runtime call creates a new one with the module loaded again, possibly
+// at another address; a caller running its own driver-API context on the
+// device also sees its own copy.  So the address is cached per device
+// together with the unique id of the context it was looked up in, and
+// looked up again whenever the current context's id differs.
+struct ScratchSlot {
+  void *ptr = nullptr;
+  unsigned long long ctx_id = 0;   // 0: not cached
+};
 std::mutex g_scratch_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
+ScratchSlot g_scratch[kMaxDevices];
 
-// Device address of g_decode_scratch on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address is looked up once
-// per device with cudaGetSymbolAddress (with that device current) and cached.
+// Device address of g_decode_scratch in the current context.  In host code
+// the array's name is only a host-side stand-in, so the address comes from
+// cudaGetSymbolAddress, called with the device current: once per device and
+// context, then cached (see ScratchSlot).
 int scratch_on_current_device(void **out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -48,17 +61,22 @@ int scratch_on_current_device(void **out) {
   if (dev < 0 || dev >= kMaxDevices)
     return msa::report_error(MSA_ERR_UNSUPPORTED, "device ordinal above 63");
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void *ptr = nullptr;
-    e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
-    if (e != cudaSuccess || !ptr) {
-      char m[256];
-      snprintf(m, sizeof(m), "cudaGetSymbolAddress(decode scratch): %s", cudaGetErrorString(e));
-      return msa::report_error(MSA_ERR_CUDA, m);
-    }
-    g_scratch_ptr[dev] = ptr;
+  ScratchSlot &slot = g_scratch[dev];
+  unsigned long long id = 0;
+  if (slot.ptr && msa::current_context_id(&id) && id == slot.ctx_id) {
+    *out = slot.ptr;
+    return MSA_OK;
   }
-  *out = g_scratch_ptr[dev];
+  void *ptr = nullptr;
+  e = cudaGetSymbolAddress(&ptr, g_decode_scratch);   // creates the context if there is none
+  if (e != cudaSuccess || !ptr) {
+    char m[256];
+    snprintf(m, sizeof(m), "cudaGetSymbolAddress(decode scratch): %s", cudaGetErrorString(e));
+    return msa::report_error(MSA_ERR_CUDA, m);
+  }
+  slot.ptr = ptr;
+  slot.ctx_id = msa::current_context_id(&id) ? id : 0;   // 0: look it up again next call
+  *out = ptr;
   return MSA_OK;
 }
 

@@ -137,4 +137,12 @@ cudaError_t launch_quantize_e4m3_rows(const uint16_t *x, long long rows, int col
 // Sets the message msa_last_error() returns; returns `code`.
 int report_error(int code, const char *msg);
 
+// Unique id of the calling thread's current CUDA context (never reused by a
+// later context, unlike a context handle or a device number); false when no
+// context is current or the driver lacks the entry points.  Per-device state
+// the library caches (device addresses of its own arrays, streams, events)
+// is keyed on it, so a context rebuilt by cudaDeviceReset is not handed
+// objects of the one it replaced.
+bool current_context_id(unsigned long long *id);
+
 }  // namespace msa

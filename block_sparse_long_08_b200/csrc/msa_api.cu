@@ -380,6 +380,7 @@ int run_prefill_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
 struct HostEvents {
   cudaEvent_t idx_in = nullptr, all_in = nullptr, chunk = nullptr, done = nullptr;
   cudaStream_t down = nullptr;   // output downloads (the other PCIe direction)
+  unsigned long long ctx_id = 0; // context they were created in
 };
 constexpr int kMaxDevices = 64;
 std::mutex g_host_mu;
@@ -391,6 +392,15 @@ int host_events(HostEvents **out) {
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(MSA_ERR_UNSUPPORTED, "device %d", dev);
   HostEvents &h = g_host_ev[dev];
+  // Events and streams belong to the context they were created in; after the
+  // device's context is rebuilt (cudaDeviceReset) they are created anew.
+  unsigned long long id = 0;
+  e = cudaSetDevice(dev);   // makes the device's primary context current (creating it if needed)
+  if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+  if (msa::current_context_id(&id) && id != h.ctx_id) {
+    h = HostEvents{};
+    h.ctx_id = id;
+  }
   cudaEvent_t *evs[4] = {&h.idx_in, &h.all_in, &h.chunk, &h.done};
   for (cudaEvent_t *ev : evs) {
     if (*ev) continue;
@@ -469,6 +479,30 @@ int run_decode(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
 namespace msa {
 // Records an error message for msa_last_error() from other translation units.
 int report_error(int code, const char *msg) { return fail(code, "%s", msg); }
+
+bool current_context_id(unsigned long long *id) {
+  // Driver entry points resolved through the runtime, so the library needs
+  // no link against libcuda.
+  using CtxGetCurrentFn = CUresult (*)(CUcontext *);
+  using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(fn);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS && *id != 0;
+}
 }  // namespace msa
 
 extern "C" {

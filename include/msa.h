@@ -52,7 +52,9 @@
  *     the start of `ws`; msa_read_status() synchronises the stream and
  *     returns/clears it.
  *   - Supported: d == 128, d_idx in {64, 128}, block == 128,
- *     1 <= top_k <= 32, H % G == 0 with H/G in {1,2,4,8,16}, L % 128 == 0.
+ *     1 <= top_k <= 32, H % G == 0 with H/G in {1,2,4,8,16}, L % 128 == 0;
+ *     the decode entry points also need G <= 8 (the cache scan scores all
+ *     groups of a key in one 8-column tensor-core product).
  *     Other shapes give MSA_ERR_UNSUPPORTED.  B == 0 or L == 0 is a no-op.
  */
 #ifndef MSA_H_
@@ -201,6 +203,9 @@ int msa_quantize_e4m3_rows(const msa_bf16 *x, long long rows, int cols, uint8_t 
  *     MSA_ERR_WORKSPACE without launching anything.
  *   The first call on each device looks the array's device address up with
  *     cudaGetSymbolAddress; make that first call before any stream capture.
+ *     The address is cached with the id of the context it belongs to and is
+ *     looked up again in a new context (after cudaDeviceReset, or under
+ *     another driver-API context on the device).
  *   All calls on a device share the array and it keeps the last call's
  *     contents: calls whose GPU work overlaps (other streams) race, so order
  *     them.  Device-side input errors are not reported by this variant (its

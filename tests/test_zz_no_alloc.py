@@ -11,6 +11,9 @@ call's leftovers in the shared scratch do not leak into the next result.
 The file is named to be collected last.
 """
 import ctypes
+import os
+import subprocess
+import sys
 
 import pytest
 import torch
@@ -63,3 +66,31 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
                                                 fake, None, None)
     assert rc == M.MSA_ERR_WORKSPACE
     assert "no-allocation" in M.msa_last_error()
+
+
+def test_noalloc_without_sel_and_with_a_bad_length():
+    """sel = NULL (the selection then lives in the shared scratch) and a
+    length above Lmax: that sequence's output is zero, the others match the
+    workspace entry point (which also reports the bad length on the device)."""
+    d = _problem(4, 4096, 2, 8, 64, 4, [4096, 5000, 300, 1], seed=103)
+    ws = M.new_workspace(M.make_params(4, 4096, 8, 2, 128, 64, 128, 4), M.MSA_OP_DECODE, DEV)
+    ref = M.msa_sparse_attn_decode(d["q"], d["q_idx"], d["k_cache"], d["v_cache"], d["k_idx_cache"],
+                                   d["seq_lens"], 4, ws=ws)
+    assert M.msa_read_status(ws) == M.MSA_ERR_DEVICE_INPUT
+    for _ in range(2):
+        got = M.msa_sparse_attn_decode_noalloc(d["q"], d["q_idx"], d["k_cache"], d["v_cache"],
+                                               d["k_idx_cache"], d["seq_lens"], 4)
+        torch.cuda.synchronize()
+        assert torch.count_nonzero(got[1]).item() == 0
+        err = (got.float() - ref.float()).abs()
+        assert err.max().item() <= OUT_MAX_ABS and err.mean().item() <= OUT_MEAN_ABS
+
+
+def test_noalloc_across_device_reset():
+    """A reset rebuilds the context and may move the scratch array; the
+    entry point must look its address up again (run in a child process
+    without torch, see _noalloc_reset_child.py)."""
+    child = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_noalloc_reset_child.py")
+    r = subprocess.run([sys.executable, child], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "ok" in r.stdout
