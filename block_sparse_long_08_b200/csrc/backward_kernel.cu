@@ -453,17 +453,16 @@ template <int KCAP>
 __global__ void __launch_bounds__(256) bwd_dq_reduce_kernel(const BwdArgs a) {
   const long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  const long long n_rows = (long long)a.B * a.Lc * a.H;   // the chunk's rows
+  const long long n_rows = (long long)a.Rc * a.H;   // the chunk's rows
   if (w >= n_rows) return;
   const int h = (int)(w % a.H);
-  const long long bt = w / a.H;
-  const int tl = (int)(bt % a.Lc);
-  const int b = (int)(bt / a.Lc);
-  const int t = a.t0 + tl;
+  const int rl = (int)(w / a.H);
+  const int row = a.r0 + rl;              // packed row b*L + t
+  const int b = row / a.L, t = row % a.L;
   const int r = a.H / a.G;
   const int g = h / r, hh = h % r;
   const size_t es = ((size_t(b) * a.G + g) * a.L + t) * a.top_k;     // sel row
-  const size_t ep = ((size_t(b) * a.G + g) * a.Lc + tl) * a.top_k;   // pos_of row (chunk)
+  const size_t ep = (size_t(g) * a.Rc + rl) * a.top_k;               // pos_of row (chunk)
   const bool in_k = lane < a.top_k;
   const int my_sel = in_k ? a.sel[es + lane] : -1;
   const long long my_rho = (my_sel >= 0) ? (long long)a.pos_of[ep + lane] * r + hh : -1;
@@ -483,7 +482,7 @@ __global__ void __launch_bounds__(256) bwd_dq_reduce_kernel(const BwdArgs a) {
     acc.x += bf16_lo(v[s].x); acc.y += bf16_hi(v[s].x);
     acc.z += bf16_lo(v[s].y); acc.w += bf16_hi(v[s].y);
   }
-  *reinterpret_cast<uint2 *>(a.dq + ((size_t(b) * a.L + t) * a.H + h) * kHeadDim + lane * 4) =
+  *reinterpret_cast<uint2 *>(a.dq + (size_t(row) * a.H + h) * kHeadDim + lane * 4) =
       make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
 }
 
@@ -510,7 +509,7 @@ cudaError_t launch_bwd_delta(const BwdArgs &a, cudaStream_t st) {
 
 cudaError_t launch_backward(const CUtensorMap &tk, const CUtensorMap &tv, const BwdArgs &a,
                             int num_sms, cudaStream_t st) {
-  const long long rows = (long long)a.B * a.Lc * a.H;
+  const long long rows = (long long)a.Rc * a.H;
   if (rows == 0) return cudaSuccess;
   cudaError_t e = cudaMemsetAsync(a.unit_ctr, 0, sizeof(int), st);
   if (e != cudaSuccess) return e;

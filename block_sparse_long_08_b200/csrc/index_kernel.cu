@@ -86,13 +86,30 @@ struct IndexWork {
 __device__ __forceinline__ IndexWork index_work(const IndexArgs &a, int u, int GPn) {
   const int ngp = a.G / GPn;
   IndexWork w;
-  w.i = a.i_hi - 1 - u / (a.B * ngp);
-  const int rem = u % (a.B * ngp);
-  w.b = rem / ngp;
-  w.gp = rem % ngp;
+  if (a.items) {   // ragged batch: the host's (b, i) list, every group pair of each
+    const int2 it = a.items[u / ngp];
+    w.b = it.x;
+    w.i = it.y;
+    w.gp = u % ngp;
+  } else {
+    w.i = a.i_hi - 1 - u / (a.B * ngp);
+    const int rem = u % (a.B * ngp);
+    w.b = rem / ngp;
+    w.gp = rem % ngp;
+  }
   const bool need = a.write_scores ? (w.i >= 1) : (w.i >= a.top_k && a.top_k >= 2);
   w.stages = need ? (w.i + 1) / 2 : 0;
   return w;
+}
+
+// Selection / score row of position t of the item's sequence for group g,
+// or -1 when t is not one of the launch's query rows.
+__device__ __forceinline__ long long index_out_row(const IndexArgs &a, const int4 &s, int g,
+                                                   int t) {
+  const int tl = t - s.y;
+  const int r = s.x + tl;
+  if (tl < 0 || tl >= s.z || r < a.r_lo || r >= a.r_hi) return -1;
+  return (long long)s.w + (long long)g * a.q.sel_gs + tl;
 }
 
 // Work item of this CTA in round r (snake order over CTAs; items are sorted
@@ -247,10 +264,13 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait(b_qempty, qph ^ 1, abort_flag, a.status)) break;
         qph ^= 1;
         mbar_arrive_expect_tx(b_qfull, C::Q_BYTES);
+        // the tile's q_idx rows (rows outside the sequence load as zeros or
+        // another sequence's values; their results are never written)
+        const int4 sq = qgeo_seq(a.q, w.b);
         for (int gi = 0; gi < GP; ++gi)
           for (int c = 0; c < C::NCH; ++c)
             tma_load_3d(s_q + (gi * C::NCH + c) * 16384, &tm_q, b_qfull, c * 64, w.gp * GP + gi,
-                        w.b * a.Lq + w.i * kBlock - a.tq0);
+                        sq.x + w.i * kBlock - sq.y);
         bool ok = true;
         for (int s = 0; s < w.stages; ++s) {
           if (!mbar_wait(b_kempty + 8 * kst, kph ^ 1, abort_flag, a.status)) { ok = false; break; }
@@ -334,6 +354,7 @@ __global__ void __launch_bounds__(384, 1)
       if (u < 0) break;
       const IndexWork w = index_work(a, u, GP);
       const int t = w.i * kBlock + row;
+      const int4 sq = qgeo_seq(a.q, w.b);
       float ls[GP][KCAP];
       int lj[GP][KCAP];
 #pragma unroll
@@ -371,8 +392,8 @@ __global__ void __launch_bounds__(384, 1)
           if (j < w.i) {
             const float sc = max4x32(v0, v1, v2, v3);
             if (a.write_scores) {
-              const int g = w.gp * GP + gi;
-              a.scores[((size_t(w.b) * a.G + g) * a.Lq + (t - a.tq0)) * a.nb + j] = sc;
+              const long long orow = index_out_row(a, sq, w.gp * GP + gi, t);
+              if (orow >= 0) a.scores[orow * a.nb + j] = sc;
             } else if (sc > ls[gi][KCAP - 1]) {
               list_insert_tail<KCAP>(ls[gi], lj[gi], sc, j);
             }
@@ -387,8 +408,9 @@ __global__ void __launch_bounds__(384, 1)
         if (eset == 0) {
 #pragma unroll
           for (int gi = 0; gi < GP; ++gi) {
-            const int g = w.gp * GP + gi;
-            float *dst = a.scores + ((size_t(w.b) * a.G + g) * a.Lq + (t - a.tq0)) * a.nb;
+            const long long orow = index_out_row(a, sq, w.gp * GP + gi, t);
+            if (orow < 0) continue;
+            float *dst = a.scores + orow * a.nb;
             for (int j = w.i; j < a.nb; ++j) dst[j] = -INFINITY;
           }
         }
@@ -399,8 +421,9 @@ __global__ void __launch_bounds__(384, 1)
         if (eset == 0) {
 #pragma unroll
           for (int gi = 0; gi < GP; ++gi) {
-            const int g = w.gp * GP + gi;
-            int32_t *dst = a.sel + ((size_t(w.b) * a.G + g) * a.Lq + (t - a.tq0)) * a.top_k;
+            const long long orow = index_out_row(a, sq, w.gp * GP + gi, t);
+            if (orow < 0) continue;
+            int32_t *dst = a.sel + orow * a.top_k;
             for (int k = 0; k < a.top_k; ++k) dst[k] = (k <= w.i) ? k : -1;
           }
         }
@@ -427,8 +450,9 @@ __global__ void __launch_bounds__(384, 1)
             const int id = m_id[(gi * KCAP + k) * 128 + row];
             if (id >= 0 && id != INT_MAX) list_insert<KCAP>(ls[gi], lj[gi], sc, id);
           }
-          const int g = w.gp * GP + gi;
-          int32_t *dst = a.sel + ((size_t(w.b) * a.G + g) * a.Lq + (t - a.tq0)) * a.top_k;
+          const long long orow = index_out_row(a, sq, w.gp * GP + gi, t);
+          if (orow < 0) continue;
+          int32_t *dst = a.sel + orow * a.top_k;
           int ids[KCAP];
 #pragma unroll
           for (int k = 0; k < KCAP; ++k) ids[k] = (k >= n_sent) ? lj[gi][k] : INT_MAX;

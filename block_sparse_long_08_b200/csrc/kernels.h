@@ -8,18 +8,56 @@
 
 namespace msa {
 
-// Query-side tensors (q, q_idx, sel, scores, out, lse) hold Lq rows per
-// sequence, row 0 being position tq0; key-side tensors (k, v, k_idx) hold
-// L rows per sequence from position 0.  A whole-sequence call has Lq = L,
-// tq0 = 0.
+// Query-side geometry.  Query rows are packed: sequence b owns rows
+// [qrow0_b, qrow0_b + nq_b) of q, q_idx, out and lse, holding positions
+// [tq0_b, tq0_b + nq_b); its keys are rows [b*L, b*L + tq0_b + nq_b) of k, v
+// and k_idx (L = rows per sequence on the key side).  Its selection row for
+// group g and position t is sel_base_b + g*sel_gs + (t - tq0_b) (in units of
+// top_k entries; block scores use the same row index, in units of nb).
+//   uniform batch (seqs == nullptr): qrow0_b = b*Lq, tq0_b = tq0, nq_b = Lq,
+//     sel_base_b = b*G*Lq, sel_gs = Lq, N = B*Lq -- the [B,G,Lq,top_k]
+//     selection layout of the C ABI;
+//   ragged batch: seqs[b] = {qrow0, tq0, nq, sel_base} in device memory
+//     (sequences in row order; nq may be 0), sel_gs = N -- a [G,N,top_k]
+//     selection over the packed rows.
+struct QGeo {
+  const int4 *seqs;
+  int B, G, Lq, tq0;
+  int N;        // packed query rows
+  int sel_gs;   // selection rows between groups
+};
+
+__device__ __forceinline__ int4 qgeo_seq(const QGeo &q, int b) {
+  if (q.seqs) return q.seqs[b];
+  return make_int4(b * q.Lq, q.tq0, q.Lq, b * q.G * q.Lq);
+}
+
+// Sequence that owns packed row r: the last b with qrow0_b <= r (empty
+// sequences share their successor's qrow0 and are skipped that way).
+__device__ __forceinline__ int qgeo_seq_of_row(const QGeo &q, int r) {
+  if (!q.seqs) return r / q.Lq;
+  int lo = 0, hi = q.B - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (q.seqs[mid].x <= r) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Index branch.  Work items are (b, 128-query tile i, group pair): either
+// every b with the tiles [i_hi - n_tiles, i_hi), longest first (items ==
+// nullptr), or the (b, i) pairs of items[0 .. n_tab) (ragged batches,
+// ordered longest first by the host), each with every group pair.
 struct IndexArgs {
   int B, L, G, nb, top_k, d_idx;
-  int Lq, tq0;
+  QGeo q;
   int write_scores;  // 1: store block scores, 0: fused top-k -> sel
-  int i_hi;          // query tiles [i_hi - n_items / (B * G/groups_per_cta), i_hi)
-  int n_items;       // B * (query tiles) * (G / groups_per_cta)
-  int32_t *sel;      // [B,G,L,top_k]
-  float *scores;     // [B,G,L,nb]
+  int i_hi, n_tiles; // uniform item range (items == nullptr)
+  const int2 *items; // {b, i} pairs (ragged)
+  int n_items;       // items this launch: (B * n_tiles or n_tab) * (G / groups_per_cta)
+  int r_lo, r_hi;    // packed query rows whose sel / scores this launch writes
+  int32_t *sel;      // selection rows (see QGeo)
+  float *scores;     // block-score rows (see QGeo), nb entries each
   int *status;
 };
 int index_groups_per_cta(int G, int top_k);
@@ -33,27 +71,34 @@ struct TopkArgs {
 };
 cudaError_t launch_topk_kernel(const TopkArgs &a, cudaStream_t st);
 
+// Reverse index and attention over one query chunk: the packed rows
+// [r0, r0 + Rc).  Per-entry arrays of the chunk (pos_of) are laid out
+// [G][Rc][top_k].
 struct RevIdxArgs {
-  int B, G, L, nb, top_k, qpi;  // qpi: queries per 128-row tile (128 / (H/G))
-  int Lq, tq0;                  // query-side geometry (see IndexArgs)
-  int t0, Lc;                   // query chunk [t0, t0 + Lc)
-  const int32_t *sel;           // [B,G,L,top_k]
-  int32_t *cnt;                 // [B*G*nb]      (zeroed by the caller)
+  int G, nb, top_k, qpi;        // qpi: queries per 128-row tile (128 / (H/G))
+  QGeo q;
+  int r0, Rc;                   // query chunk
+  const int32_t *sel;           // selection rows (see QGeo)
+  int32_t *cnt;                 // [B*G*nb]      (zeroed by the launcher)
   int32_t *list_off;            // [B*G*nb + 1]
   int32_t *item_off;            // [B*G*nb + 1]
-  int32_t *list;                // [B*G*Lc*top_k]
-  int32_t *pos_of;              // [B,G,Lc,top_k]: rank in its block's list, then list position
+  int32_t *list;                // [G*Rc*top_k]: t * 32 + slot
+  int32_t *pos_of;              // [G][Rc][top_k]: rank in its block's list, then list position
   int *status;
 };
 cudaError_t launch_revidx(const RevIdxArgs &a, cudaStream_t st);
 
 struct AttnArgs {
-  int B, L, H, G, nb, top_k;
-  int Lq, tq0;                 // query-side geometry (see IndexArgs)
+  int L, H, G, nb, top_k;      // L: key rows per sequence
+  QGeo q;
   float scale, scale_log2;
-  int t0, Lc;
   int max_items;               // upper bound on the chunk's work items
-  const uint16_t *q;           // [B,L,H,d]
+  const uint16_t *q_ptr;       // packed query rows [N,H,d]
+  // Per-sequence K and V tensor maps in device memory ({K, V} of sequence b
+  // at 2b, 2b+1; 4-D, batch extent 1), or null: the launch's own maps (4-D
+  // over the whole batch).  Either way a map's row extent ends at the
+  // sequence's last key, so rows past it load as zeros.
+  const CUtensorMap *kv_maps;
   const int32_t *list;
   const int32_t *list_off;
   const int32_t *item_off;
@@ -68,30 +113,31 @@ cudaError_t launch_prefill_attn(const CUtensorMap &tk, const CUtensorMap &tv, co
                                 int num_sms, cudaStream_t st);
 
 struct CombineArgs {
-  int B, L, H, G, top_k;
-  int Lq, tq0;                 // query-side geometry (see IndexArgs)
-  int t0, Lc;
-  const int32_t *sel;          // [B,G,L,top_k]
-  const int32_t *pos_of;       // [B,G,Lc,top_k]
+  int H, G, top_k;
+  QGeo q;
+  int r0, Rc;                  // query chunk (packed rows)
+  const int32_t *sel;          // selection rows (see QGeo)
+  const int32_t *pos_of;       // [G][Rc][top_k]
   const uint16_t *part_o;      // see AttnArgs
   const float *part_lse;
-  uint16_t *out;               // [B,L,H,d]
-  float *lse;                  // [B,L,H] or null
+  uint16_t *out;               // packed rows [N,H,d]
+  float *lse;                  // packed rows [N,H] or null
 };
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
 
-// Main-branch backward for the query chunk [t0, t0 + Lc), over that chunk's
-// reverse index.
+// Main-branch backward for the query chunk of packed rows [r0, r0 + Rc)
+// (uniform batch, whole sequences: row b*L + t is position t of sequence b),
+// over that chunk's reverse index.
 struct BwdArgs {
   int B, L, H, G, nb, top_k;
-  int t0, Lc;
+  int r0, Rc;
   int last;                    // the last query chunk (writes dk, dv when chunked)
   float scale, scale_log2;
   const uint16_t *q;           // [B,L,H,d]
   const uint16_t *out, *dout;  // [B,L,H,d]: forward output and its gradient
   const float *lse;            // [B,L,H]: forward log-sum-exp (natural log)
   const int32_t *sel;          // [B,G,L,top_k]
-  const int32_t *list, *list_off, *pos_of;   // reverse index (see RevIdxArgs)
+  const int32_t *list, *list_off, *pos_of;   // reverse index of the chunk (see RevIdxArgs)
   float *delta;                // [B,L,H]: do . o
   // dq of (list position, head), scaled, bf16 [entries*R, d]; granule c
   // of partial row rho is stored at granule c ^ (rho & 7) (as AttnArgs)

@@ -9,7 +9,9 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
+#include <vector>
 
 #include "../../include/msa.h"
 #include "common.cuh"
@@ -37,7 +39,9 @@ size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---- shape checks ---------------------------------------------------------
-int check_params(const msa_params *p, bool decode) {
+// whole_blocks: the operation needs L to be a multiple of the block length
+// (the backward); the prefill and decode paths take any length.
+int check_params(const msa_params *p, bool decode, bool whole_blocks = false) {
   if (!p) return fail(MSA_ERR_INVALID_ARG, "params is NULL");
   if (p->B < 0 || p->L < 0 || p->H <= 0 || p->G <= 0 || p->d <= 0 || p->d_idx <= 0 ||
       p->block <= 0 || p->top_k <= 0)
@@ -54,7 +58,8 @@ int check_params(const msa_params *p, bool decode) {
   const int r = p->H / p->G;
   if (r != 1 && r != 2 && r != 4 && r != 8 && r != 16)
     return fail(MSA_ERR_UNSUPPORTED, "H/G=%d (supported: 1,2,4,8,16)", r);
-  if (p->L % 128 != 0) return fail(MSA_ERR_UNSUPPORTED, "L=%d not a multiple of 128", p->L);
+  if (whole_blocks && p->L % 128 != 0)
+    return fail(MSA_ERR_UNSUPPORTED, "L=%d: this operation needs a multiple of 128", p->L);
   if (decode && p->G > 8) return fail(MSA_ERR_UNSUPPORTED, "decode supports G <= 8 (G=%d)", p->G);
   if ((long long)p->B * p->L > (1LL << 26))
     return fail(MSA_ERR_UNSUPPORTED, "B*L=%lld above 2^26", (long long)p->B * p->L);
@@ -67,70 +72,77 @@ float eff_scale(const msa_params *p) {
   return p->scale > 0.f ? p->scale : 1.0f / std::sqrt(float(p->d));
 }
 
+int nblocks(int L) { return (L + 127) / 128; }
+
 // ---- workspace plans --------------------------------------------------------
-// Prefill attention processes queries in chunks of Lc so that the partial
-// results (bf16, one 128-wide row per selected (query, head, slot)) stay
-// within a fixed budget.  Every chunk reads the K/V blocks its queries
-// select, which for long inputs is most of K/V, so fewer, larger chunks
-// cut K/V re-reads: 16 GiB of partials is 9 chunks at 1M tokens, H=32,
-// top_k=16 (a small share of HBM on this part).
+// Prefill attention processes the packed query rows in chunks of Rc so that
+// the partial results (bf16, one 128-wide row per selected (query, head,
+// slot)) stay within a fixed budget.  Every chunk reads the K/V blocks its
+// queries select, which for long inputs is most of K/V, so fewer, larger
+// chunks cut K/V re-reads: 16 GiB of partials is 9 chunks at 1M tokens,
+// H=32, top_k=16 (a small share of HBM on this part).
 constexpr size_t kPartialBudget = size_t(16) << 30;  // 16 GiB
 
-int prefill_chunk(const msa_params *p) {
-  const size_t per_q = size_t(p->B) * p->H * p->top_k * (p->d * 2 + 4);
-  long long lc = per_q ? (long long)(kPartialBudget / per_q) : p->L;
-  lc = (lc / 128) * 128;
-  if (lc < 128) lc = 128;
-  if (p->chunk > 0 && p->chunk < lc) lc = p->chunk;
-  if (lc > p->L) lc = p->L;
-  return (int)lc;
+int prefill_chunk(const msa_params *p, long long n_rows) {
+  const size_t per_row = size_t(p->H) * p->top_k * (p->d * 2 + 4);
+  long long rc = (long long)(kPartialBudget / per_row);
+  rc = (rc / 128) * 128;
+  if (rc < 128) rc = 128;
+  if (p->chunk > 0 && p->chunk < rc) rc = p->chunk;
+  if (rc > n_rows) rc = n_rows;
+  return (int)rc;
 }
 
 struct AttnWs {
   size_t cnt, list_off, item_off, list, pos_of, part_o, part_lse, end;
-  int Lc;
+  int Rc;
 };
-AttnWs attn_ws(const msa_params *p, size_t base) {
+// n_rows packed query rows of n_seq sequences of up to p->L keys each.
+AttnWs attn_ws(const msa_params *p, size_t base, long long n_rows, int n_seq) {
   AttnWs w;
-  w.Lc = prefill_chunk(p);
-  const size_t nb = size_t(p->L) / 128;
-  const size_t nbgj = size_t(p->B) * p->G * nb;
+  w.Rc = prefill_chunk(p, n_rows);
+  const size_t nbgj = size_t(n_seq) * p->G * nblocks(p->L);
+  const size_t entries = size_t(p->G) * w.Rc * p->top_k;
   size_t o = base;
   w.cnt = o; o = align_up(o + 4 * nbgj);
   w.list_off = o; o = align_up(o + 4 * (nbgj + 1));
   w.item_off = o; o = align_up(o + 4 * (nbgj + 1));
-  w.list = o; o = align_up(o + 4 * size_t(p->B) * p->G * w.Lc * p->top_k);
-  w.pos_of = o; o = align_up(o + 4 * size_t(p->B) * p->G * w.Lc * p->top_k);
-  w.part_o = o; o = align_up(o + 2 * size_t(p->B) * w.Lc * p->H * p->top_k * p->d);
-  w.part_lse = o; o = align_up(o + 4 * size_t(p->B) * w.Lc * p->H * p->top_k);
+  w.list = o; o = align_up(o + 4 * entries);
+  w.pos_of = o; o = align_up(o + 4 * entries);
+  w.part_o = o; o = align_up(o + 2 * entries * (p->H / p->G) * size_t(p->d));
+  w.part_lse = o; o = align_up(o + 4 * entries * (p->H / p->G));
   w.end = o;
   return w;
 }
+AttnWs attn_ws(const msa_params *p, size_t base) {
+  return attn_ws(p, base, (long long)p->B * p->L, p->B);
+}
 
-// Backward: D = do . o per row; per query chunk (the prefill's chunk length)
-// a reverse index and one bf16 dq partial row per (query, head, slot); with
-// more than one chunk, fp32 dk/dv accumulators over the whole sequence.
+// Backward: D = do . o per row; per query chunk (the prefill's chunk length,
+// packed rows b*L + t) a reverse index and one bf16 dq partial row per
+// (query, head, slot); with more than one chunk, fp32 dk/dv accumulators
+// over the whole batch.
 struct BwdWs {
   size_t cnt, list_off, item_off, list, pos_of, delta, part_dq, acc_dk, acc_dv, end;
-  int Lc;
+  int Rc;
 };
 BwdWs bwd_ws(const msa_params *p) {
   BwdWs w;
-  w.Lc = prefill_chunk(p);
-  const size_t nb = size_t(p->L) / 128;
-  const size_t nbgj = size_t(p->B) * p->G * nb;
-  const size_t entries = size_t(p->B) * p->G * w.Lc * p->top_k;
+  const long long n_rows = (long long)p->B * p->L;
+  w.Rc = prefill_chunk(p, n_rows);
+  const size_t nbgj = size_t(p->B) * p->G * nblocks(p->L);
+  const size_t entries = size_t(p->G) * w.Rc * p->top_k;
   size_t o = msa::kWsHeader;
   w.cnt = o; o = align_up(o + 4 * nbgj);
   w.list_off = o; o = align_up(o + 4 * (nbgj + 1));
   w.item_off = o; o = align_up(o + 4 * (nbgj + 1));
   w.list = o; o = align_up(o + 4 * entries);
   w.pos_of = o; o = align_up(o + 4 * entries);
-  w.delta = o; o = align_up(o + 4 * size_t(p->B) * p->L * p->H);
+  w.delta = o; o = align_up(o + 4 * size_t(n_rows) * p->H);
   w.part_dq = o; o = align_up(o + 2 * entries * (p->H / p->G) * size_t(p->d));
   w.acc_dk = w.acc_dv = 0;
-  if (w.Lc < p->L) {
-    const size_t kv = 4 * size_t(p->B) * p->L * p->G * p->d;
+  if (w.Rc < n_rows) {
+    const size_t kv = 4 * size_t(n_rows) * p->G * p->d;
     w.acc_dk = o; o = align_up(o + kv);
     w.acc_dv = o; o = align_up(o + kv);
   }
@@ -143,7 +155,7 @@ struct DecWs {
 };
 DecWs dec_ws(const msa_params *p) {
   DecWs w;
-  const size_t nb = size_t(p->L) / 128;
+  const size_t nb = size_t(nblocks(p->L));
   size_t o = msa::kWsHeader;
   w.scores = o; o = align_up(o + 4 * size_t(p->B) * p->G * nb);
   w.sel = o; o = align_up(o + 4 * size_t(p->B) * p->G * p->top_k);
@@ -155,6 +167,24 @@ DecWs dec_ws(const msa_params *p) {
 
 size_t forward_sel_bytes(const msa_params *p) {
   return align_up(4 * size_t(p->B) * p->G * p->L * p->top_k);
+}
+
+// Ragged batch (msa_forward_cached_varlen): device tables at the start of
+// the workspace, after the header -- two 4-D K/V tensor maps per sequence,
+// the per-sequence query geometry, and the index branch's (b, tile) list --
+// then the selection of the packed rows, then the attention workspace.
+struct VarlenWs {
+  size_t maps, seqs, items, sel, attn_base;
+};
+VarlenWs varlen_ws(const msa_params *p) {
+  VarlenWs w;
+  size_t o = msa::kWsHeader;
+  w.maps = o; o = align_up(o + 2 * sizeof(CUtensorMap) * size_t(p->B));
+  w.seqs = o; o = align_up(o + sizeof(int4) * size_t(p->B));
+  w.items = o; o = align_up(o + sizeof(int2) * size_t(p->B) * nblocks(p->L));
+  w.sel = o; o += forward_sel_bytes(p);
+  w.attn_base = o;
+  return w;
 }
 
 int check_ws(void *ws, size_t ws_bytes, size_t need) {
@@ -181,17 +211,28 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // bf16 tensor of `rank` dims (innermost first), 128B swizzle, box as given.
+// Elements outside the dims load as zeros.
 int make_tmap(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
               const uint64_t *strides_bytes, const uint32_t *box) {
   auto fn = encode_fn();
   if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
-  uint32_t estr[3] = {1, 1, 1};
+  uint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(base), dims,
                   strides_bytes, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
   return MSA_OK;
+}
+
+// 4-D map (d, G, key rows, sequences) over K or V [nseq, L, G, d], the row
+// extent cut at kv_rows: rows >= kv_rows of each sequence load as zeros.
+int make_kv_tmap(CUtensorMap *m, const void *base, const msa_params *p, int kv_rows, int nseq) {
+  const uint64_t dims[4] = {uint64_t(p->d), uint64_t(p->G), uint64_t(kv_rows), uint64_t(nseq)};
+  const uint64_t str[3] = {uint64_t(p->d) * 2, uint64_t(p->d) * 2 * p->G,
+                           uint64_t(p->d) * 2 * p->G * p->L};
+  const uint32_t box[4] = {64, 1, 128, 1};
+  return make_tmap(m, base, 4, dims, str, box);
 }
 
 int num_sms() {
@@ -204,23 +245,49 @@ int num_sms() {
 int *status_ptr(void *ws) { return reinterpret_cast<int *>(ws); }
 
 // ---- the operations --------------------------------------------------------
-// Query-side geometry: q, q_idx, sel and out hold Lq rows per sequence, row
-// 0 being position tq0 (Lq = L, tq0 = 0 for a whole sequence); k, v and
-// k_idx hold p->L rows per sequence.
-struct QGeom {
-  int Lq, tq0;
-};
-QGeom whole(const msa_params *p) { return QGeom{p->L, 0}; }
+// Query-side geometry of a uniform batch: every sequence has Lq query rows at
+// positions [tq0, tq0 + Lq) (see msa::QGeo).
+msa::QGeo uniform_geo(const msa_params *p, int Lq, int tq0) {
+  msa::QGeo q;
+  q.seqs = nullptr;
+  q.B = p->B; q.G = p->G; q.Lq = Lq; q.tq0 = tq0;
+  q.N = p->B * Lq;
+  q.sel_gs = Lq;
+  return q;
+}
+msa::QGeo whole(const msa_params *p) { return uniform_geo(p, p->L, 0); }
 
-// Index branch for the query tiles of tokens [t_lo, t_hi) (multiples of 128
-// within [tq0, tq0 + Lq)).
+// Which index work a launch does and which rows it writes.
+struct IndexWork {
+  int i_hi = 0, n_tiles = 0;        // uniform: tiles [i_hi - n_tiles, i_hi) of every sequence
+  const int2 *items = nullptr;      // ragged: (b, tile) pairs in device memory
+  int n_tab = 0;
+  int r_lo = 0, r_hi = 0;           // packed rows written
+};
+
+// Uniform work: the tiles covering positions [t_lo, t_hi) of every sequence,
+// writing the packed rows of those positions.
+IndexWork uniform_index_work(const msa::QGeo &q, int t_lo, int t_hi) {
+  IndexWork w;
+  w.i_hi = (t_hi + 127) / 128;
+  w.n_tiles = w.i_hi - t_lo / 128;
+  if (q.B == 1) {
+    w.r_lo = t_lo - q.tq0;
+    w.r_hi = t_hi - q.tq0;
+  } else {   // whole sequences
+    w.r_lo = 0;
+    w.r_hi = q.N;
+  }
+  return w;
+}
+
 int run_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 *k_idx,
-                     int32_t *sel, float *block_scores, void *ws, cudaStream_t st, QGeom qg,
-                     int t_lo, int t_hi) {
-  const int nb = p->L / 128;
+                     int32_t *sel, float *block_scores, void *ws, cudaStream_t st,
+                     const msa::QGeo &qg, const IndexWork &iw) {
+  const int nb = nblocks(p->L);
   CUtensorMap tq, tk;
   {
-    const uint64_t dims[3] = {uint64_t(p->d_idx), uint64_t(p->G), uint64_t(p->B) * qg.Lq};
+    const uint64_t dims[3] = {uint64_t(p->d_idx), uint64_t(p->G), uint64_t(qg.N)};
     const uint64_t str[2] = {uint64_t(p->d_idx) * 2, uint64_t(p->d_idx) * 2 * p->G};
     const uint32_t box[3] = {64, 1, 128};
     int rc = make_tmap(&tq, q_idx, 3, dims, str, box);
@@ -235,10 +302,15 @@ int run_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 
   }
   msa::IndexArgs a;
   a.B = p->B; a.L = p->L; a.G = p->G; a.nb = nb; a.top_k = p->top_k; a.d_idx = p->d_idx;
-  a.Lq = qg.Lq; a.tq0 = qg.tq0;
+  a.q = qg;
   a.write_scores = block_scores ? 1 : 0;
-  a.i_hi = t_hi / 128;
-  a.n_items = p->B * (t_hi / 128 - t_lo / 128) * (p->G / msa::index_groups_per_cta(p->G, p->top_k));
+  a.i_hi = iw.i_hi;
+  a.n_tiles = iw.n_tiles;
+  a.items = iw.items;
+  const int ngp = p->G / msa::index_groups_per_cta(p->G, p->top_k);
+  a.n_items = (iw.items ? iw.n_tab : p->B * iw.n_tiles) * ngp;
+  a.r_lo = iw.r_lo;
+  a.r_hi = iw.r_hi;
   a.sel = sel;
   a.scores = block_scores;
   a.status = status_ptr(ws);
@@ -266,24 +338,25 @@ struct ChunkSink {
 
 // Tensor maps and workspace layout shared by the query chunks of one call.
 struct AttnPlan {
-  CUtensorMap tk, tv;
+  CUtensorMap tk, tv;               // launch maps (uniform batch)
+  const CUtensorMap *kv_maps;       // per-sequence maps in device memory (ragged), or null
   AttnWs w;
   int nb, qpi, sms;
   float scale;
-  QGeom qg;
+  msa::QGeo qg;
 };
 
+// kv_rows: key rows every sequence may attend (uniform batch; rows past it
+// load as zeros); kv_maps: per-sequence maps instead (ragged batch).
 int plan_attn(const msa_params *p, const msa_bf16 *k, const msa_bf16 *v, size_t ws_base,
-              QGeom qg, AttnPlan *pl) {
-  pl->nb = p->L / 128;
+              const msa::QGeo &qg, int kv_rows, const CUtensorMap *kv_maps, AttnPlan *pl) {
+  pl->nb = nblocks(p->L);
   pl->qg = qg;
-  pl->w = attn_ws(p, ws_base);
-  const uint64_t dims[3] = {uint64_t(p->d), uint64_t(p->G), uint64_t(p->B) * p->L};
-  const uint64_t str[2] = {uint64_t(p->d) * 2, uint64_t(p->d) * 2 * p->G};
-  const uint32_t box[3] = {64, 1, 128};
-  int rc = make_tmap(&pl->tk, k, 3, dims, str, box);
+  pl->kv_maps = kv_maps;
+  pl->w = attn_ws(p, ws_base, qg.N, qg.B);
+  int rc = make_kv_tmap(&pl->tk, k, p, kv_rows, p->B);
   if (rc) return rc;
-  rc = make_tmap(&pl->tv, v, 3, dims, str, box);
+  rc = make_kv_tmap(&pl->tv, v, p, kv_rows, p->B);
   if (rc) return rc;
   pl->qpi = 128 / (p->H / p->G);
   pl->scale = eff_scale(p);
@@ -291,17 +364,17 @@ int plan_attn(const msa_params *p, const msa_bf16 *k, const msa_bf16 *v, size_t 
   return MSA_OK;
 }
 
-// One query chunk [t0, t0 + Lc): reverse index, attention, merge; then,
-// with a sink, the download of the chunk's output rows.
+// One query chunk, packed rows [r0, r0 + Rc): reverse index, attention,
+// merge; then, with a sink, the download of the chunk's output rows.
 int run_attn_chunk(const msa_params *p, const AttnPlan &pl, const msa_bf16 *q, const int32_t *sel,
-                   msa_bf16 *out, float *lse, void *ws, int t0, int Lc, cudaStream_t st,
+                   msa_bf16 *out, float *lse, void *ws, int r0, int Rc, cudaStream_t st,
                    const ChunkSink *sink) {
   uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
   const AttnWs &w = pl.w;
   msa::RevIdxArgs ra;
-  ra.B = p->B; ra.G = p->G; ra.L = p->L; ra.nb = pl.nb; ra.top_k = p->top_k; ra.qpi = pl.qpi;
-  ra.Lq = pl.qg.Lq; ra.tq0 = pl.qg.tq0;
-  ra.t0 = t0; ra.Lc = Lc;
+  ra.G = p->G; ra.nb = pl.nb; ra.top_k = p->top_k; ra.qpi = pl.qpi;
+  ra.q = pl.qg;
+  ra.r0 = r0; ra.Rc = Rc;
   ra.sel = sel;
   ra.cnt = reinterpret_cast<int32_t *>(wsb + w.cnt);
   ra.list_off = reinterpret_cast<int32_t *>(wsb + w.list_off);
@@ -312,15 +385,15 @@ int run_attn_chunk(const msa_params *p, const AttnPlan &pl, const msa_bf16 *q, c
   cudaError_t e = msa::launch_revidx(ra, st);
   if (e != cudaSuccess) return cuda_fail(e, "reverse index launch");
   msa::AttnArgs aa;
-  aa.B = p->B; aa.L = p->L; aa.H = p->H; aa.G = p->G; aa.nb = pl.nb; aa.top_k = p->top_k;
-  aa.Lq = pl.qg.Lq; aa.tq0 = pl.qg.tq0;
+  aa.L = p->L; aa.H = p->H; aa.G = p->G; aa.nb = pl.nb; aa.top_k = p->top_k;
+  aa.q = pl.qg;
   aa.scale = pl.scale;
   aa.scale_log2 = pl.scale * 1.4426950408889634f;
-  aa.t0 = t0; aa.Lc = Lc;
   const long long max_items =
-      (long long)p->B * p->G * Lc * p->top_k / pl.qpi + (long long)p->B * p->G * pl.nb;
+      (long long)p->G * Rc * p->top_k / pl.qpi + (long long)pl.qg.B * p->G * pl.nb;
   aa.max_items = (int)max_items;
-  aa.q = q;
+  aa.q_ptr = q;
+  aa.kv_maps = pl.kv_maps;
   aa.list = ra.list; aa.list_off = ra.list_off; aa.item_off = ra.item_off;
   aa.part_o = reinterpret_cast<uint16_t *>(wsb + w.part_o);
   aa.part_lse = reinterpret_cast<float *>(wsb + w.part_lse);
@@ -328,9 +401,9 @@ int run_attn_chunk(const msa_params *p, const AttnPlan &pl, const msa_bf16 *q, c
   e = msa::launch_prefill_attn(pl.tk, pl.tv, aa, pl.sms, st);
   if (e != cudaSuccess) return cuda_fail(e, "prefill attention launch");
   msa::CombineArgs ca;
-  ca.B = p->B; ca.L = p->L; ca.H = p->H; ca.G = p->G; ca.top_k = p->top_k;
-  ca.Lq = pl.qg.Lq; ca.tq0 = pl.qg.tq0;
-  ca.t0 = t0; ca.Lc = Lc;
+  ca.H = p->H; ca.G = p->G; ca.top_k = p->top_k;
+  ca.q = pl.qg;
+  ca.r0 = r0; ca.Rc = Rc;
   ca.sel = sel;
   ca.pos_of = ra.pos_of;
   ca.part_o = aa.part_o; ca.part_lse = aa.part_lse;
@@ -341,34 +414,23 @@ int run_attn_chunk(const msa_params *p, const AttnPlan &pl, const msa_bf16 *q, c
     e = cudaEventRecord(sink->ev, st);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(sink->copy, sink->ev, 0);
     if (e != cudaSuccess) return cuda_fail(e, "chunk event");
-    const size_t row = size_t(p->H) * p->d;   // elements of one token's output
-    for (int b = 0; b < p->B && e == cudaSuccess; ++b) {
-      const size_t qr = size_t(b) * pl.qg.Lq + (t0 - pl.qg.tq0);   // query-side row of t0
-      const size_t off = qr * row;
-      e = cudaMemcpyAsync(sink->out_h + off, out + off, size_t(Lc) * row * 2,
-                          cudaMemcpyDeviceToHost, sink->copy);
-      if (e == cudaSuccess && sink->lse_h) {
-        const size_t lo = qr * p->H;
-        e = cudaMemcpyAsync(sink->lse_h + lo, lse + lo, size_t(Lc) * p->H * 4,
-                            cudaMemcpyDeviceToHost, sink->copy);
-      }
-    }
+    const size_t row = size_t(p->H) * p->d;   // elements of one query row's output
+    e = cudaMemcpyAsync(sink->out_h + size_t(r0) * row, out + size_t(r0) * row,
+                        size_t(Rc) * row * 2, cudaMemcpyDeviceToHost, sink->copy);
+    if (e == cudaSuccess && sink->lse_h)
+      e = cudaMemcpyAsync(sink->lse_h + size_t(r0) * p->H, lse + size_t(r0) * p->H,
+                          size_t(Rc) * p->H * 4, cudaMemcpyDeviceToHost, sink->copy);
     if (e != cudaSuccess) return cuda_fail(e, "output download");
   }
   return MSA_OK;
 }
 
-// Main branch for the queries of positions [qg.tq0, qg.tq0 + qg.Lq).
-int run_prefill_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
-                     const msa_bf16 *v, const int32_t *sel, msa_bf16 *out, float *lse, void *ws,
-                     size_t ws_base, cudaStream_t st, QGeom qg) {
-  AttnPlan pl;
-  int rc = plan_attn(p, k, v, ws_base, qg, &pl);
-  if (rc) return rc;
-  const int t_end = qg.tq0 + qg.Lq;
-  for (int t0 = qg.tq0; t0 < t_end; t0 += pl.w.Lc) {
-    const int Lc = (t_end - t0) < pl.w.Lc ? (t_end - t0) : pl.w.Lc;
-    rc = run_attn_chunk(p, pl, q, sel, out, lse, ws, t0, Lc, st, nullptr);
+// Main branch for every packed query row of the plan.
+int run_prefill_attn(const msa_params *p, const AttnPlan &pl, const msa_bf16 *q,
+                     const int32_t *sel, msa_bf16 *out, float *lse, void *ws, cudaStream_t st) {
+  for (int r0 = 0; r0 < pl.qg.N; r0 += pl.w.Rc) {
+    const int Rc = (pl.qg.N - r0) < pl.w.Rc ? (pl.qg.N - r0) : pl.w.Rc;
+    const int rc = run_attn_chunk(p, pl, q, sel, out, lse, ws, r0, Rc, st, nullptr);
     if (rc) return rc;
   }
   return MSA_OK;
@@ -456,7 +518,7 @@ int run_decode(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
   uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
   msa::DecodeArgs a;
   a.B = p->B; a.Lmax = p->L; a.H = p->H; a.G = p->G; a.d_idx = p->d_idx;
-  a.nb_max = p->L / 128; a.top_k = p->top_k;
+  a.nb_max = nblocks(p->L); a.top_k = p->top_k;
   a.scale = eff_scale(p);
   a.scale_log2 = a.scale * 1.4426950408889634f;
   a.q = q; a.q_idx = q_idx; a.k_cache = k_cache; a.v_cache = v_cache; a.k_idx_cache = k_idx_cache;
@@ -513,13 +575,14 @@ const char *msa_version(void) { return "msa-b200 0.1 (sm_100a)"; }
 
 size_t msa_workspace_bytes(const msa_params *p, int op) {
   g_err[0] = 0;
-  if (check_params(p, op == MSA_OP_DECODE) != MSA_OK) return 0;
+  if (check_params(p, op == MSA_OP_DECODE, op == MSA_OP_BACKWARD) != MSA_OK) return 0;
   switch (op) {
     case MSA_OP_INDEX_SELECT: return msa::kWsHeader;
     case MSA_OP_PREFILL_ATTN: return attn_ws(p, msa::kWsHeader).end;
     case MSA_OP_DECODE: return dec_ws(p).end;
     case MSA_OP_FORWARD: return attn_ws(p, msa::kWsHeader + forward_sel_bytes(p)).end;
     case MSA_OP_BACKWARD: return bwd_ws(p).end;
+    case MSA_OP_FORWARD_VARLEN: return attn_ws(p, varlen_ws(p).attn_base).end;
     default: fail(MSA_ERR_INVALID_ARG, "unknown op %d", op); return 0;
   }
 }
@@ -527,7 +590,7 @@ size_t msa_workspace_bytes(const msa_params *p, int op) {
 int msa_prefill_chunk_len(const msa_params *p) {
   g_err[0] = 0;
   if (check_params(p, false) != MSA_OK) return 0;
-  return p->L > 0 ? prefill_chunk(p) : 0;
+  return p->L > 0 && p->B > 0 ? prefill_chunk(p, (long long)p->B * p->L) : 0;
 }
 
 int msa_read_status(void *ws, msa_stream stream) {
@@ -561,8 +624,10 @@ int msa_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 
     return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
   rc = check_ws(ws, ws_bytes, msa::kWsHeader);
   if (rc) return rc;
+  const msa::QGeo qg = whole(p);
   return run_index_select(p, q_idx, k_idx, sel, block_scores, ws,
-                          reinterpret_cast<cudaStream_t>(stream), whole(p), 0, p->L);
+                          reinterpret_cast<cudaStream_t>(stream), qg,
+                          uniform_index_work(qg, 0, p->L));
 }
 
 int msa_sparse_attn_prefill(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k,
@@ -576,11 +641,12 @@ int msa_sparse_attn_prefill(const msa_params *p, const msa_bf16 *q, const msa_bf
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(sel) || !aligned16(out) ||
       (lse && !aligned16(lse)))
     return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
-  const size_t need = attn_ws(p, msa::kWsHeader).end;
-  rc = check_ws(ws, ws_bytes, need);
+  rc = check_ws(ws, ws_bytes, attn_ws(p, msa::kWsHeader).end);
   if (rc) return rc;
-  return run_prefill_attn(p, q, k, v, sel, out, lse, ws, msa::kWsHeader,
-                          reinterpret_cast<cudaStream_t>(stream), whole(p));
+  AttnPlan pl;
+  rc = plan_attn(p, k, v, msa::kWsHeader, whole(p), p->L, nullptr, &pl);
+  if (rc) return rc;
+  return run_prefill_attn(p, pl, q, sel, out, lse, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int msa_forward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k, const msa_bf16 *v,
@@ -600,9 +666,13 @@ int msa_forward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k, const
   if (rc) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   int32_t *s = sel ? sel : reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ws) + msa::kWsHeader);
-  rc = run_index_select(p, q_idx, k_idx, s, nullptr, ws, st, whole(p), 0, p->L);
+  const msa::QGeo qg = whole(p);
+  rc = run_index_select(p, q_idx, k_idx, s, nullptr, ws, st, qg, uniform_index_work(qg, 0, p->L));
   if (rc) return rc;
-  return run_prefill_attn(p, q, k, v, s, out, lse, ws, base, st, whole(p));
+  AttnPlan pl;
+  rc = plan_attn(p, k, v, base, qg, p->L, nullptr, &pl);
+  if (rc) return rc;
+  return run_prefill_attn(p, pl, q, s, out, lse, ws, st);
 }
 
 int msa_forward_cached(const msa_params *p, int t0, int n, const msa_bf16 *q,
@@ -612,9 +682,8 @@ int msa_forward_cached(const msa_params *p, int t0, int n, const msa_bf16 *q,
   g_err[0] = 0;
   int rc = check_params(p, false);
   if (rc) return rc;
-  if (t0 < 0 || n < 0 || t0 % 128 != 0 || n % 128 != 0 || (long long)t0 + n > p->L)
-    return fail(MSA_ERR_INVALID_ARG, "t0=%d n=%d: need multiples of 128 with t0 + n <= L=%d", t0,
-                n, p->L);
+  if (t0 < 0 || n < 0 || (long long)t0 + n > p->L)
+    return fail(MSA_ERR_INVALID_ARG, "t0=%d n=%d: need t0, n >= 0 and t0 + n <= L=%d", t0, n, p->L);
   if (p->B == 0 || n == 0) return MSA_OK;
   if (!q || !q_idx || !k_cache || !v_cache || !k_idx_cache || !out)
     return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
@@ -626,11 +695,17 @@ int msa_forward_cached(const msa_params *p, int t0, int n, const msa_bf16 *q,
   rc = check_ws(ws, ws_bytes, attn_ws(p, base).end);
   if (rc) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const QGeom qg{n, t0};
+  const msa::QGeo qg = uniform_geo(p, n, t0);
   int32_t *s = sel ? sel : reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ws) + msa::kWsHeader);
-  rc = run_index_select(p, q_idx, k_idx_cache, s, nullptr, ws, st, qg, t0, t0 + n);
+  IndexWork iw = uniform_index_work(qg, t0, t0 + n);
+  iw.r_lo = 0;
+  iw.r_hi = qg.N;
+  rc = run_index_select(p, q_idx, k_idx_cache, s, nullptr, ws, st, qg, iw);
   if (rc) return rc;
-  return run_prefill_attn(p, q, k_cache, v_cache, s, out, lse, ws, base, st, qg);
+  AttnPlan pl;
+  rc = plan_attn(p, k_cache, v_cache, base, qg, t0 + n, nullptr, &pl);
+  if (rc) return rc;
+  return run_prefill_attn(p, pl, q, s, out, lse, ws, st);
 }
 
 int msa_forward_cached_varlen(const msa_params *p, const int32_t *t0, const int32_t *n,
@@ -643,28 +718,69 @@ int msa_forward_cached_varlen(const msa_params *p, const int32_t *t0, const int3
   if (rc) return rc;
   if (p->B == 0) return MSA_OK;
   if (!t0 || !n) return fail(MSA_ERR_INVALID_ARG, "NULL t0 or n (host arrays)");
-  for (int b = 0; b < p->B; ++b)
-    if (t0[b] < 0 || n[b] < 0 || t0[b] % 128 || n[b] % 128 || (long long)t0[b] + n[b] > p->L)
-      return fail(MSA_ERR_INVALID_ARG, "sequence %d: t0=%d n=%d (multiples of 128, t0+n <= L=%d)",
-                  b, t0[b], n[b], p->L);
-  msa_params p1 = *p;
-  p1.B = 1;
-  const size_t kv_rows = size_t(p->L);   // cache rows per sequence
-  long long row0 = 0;
+  long long N = 0;
   for (int b = 0; b < p->B; ++b) {
-    if (n[b] > 0) {
-      rc = msa_forward_cached(&p1, t0[b], n[b], q + size_t(row0) * p->H * p->d,
-                              q_idx + size_t(row0) * p->G * p->d_idx,
-                              k_cache + size_t(b) * kv_rows * p->G * p->d,
-                              v_cache + size_t(b) * kv_rows * p->G * p->d,
-                              k_idx_cache + size_t(b) * kv_rows * p->d_idx,
-                              out + size_t(row0) * p->H * p->d, nullptr,
-                              lse ? lse + size_t(row0) * p->H : nullptr, ws, ws_bytes, stream);
-      if (rc) return rc;
-    }
+    if (t0[b] < 0 || n[b] < 0 || (long long)t0[b] + n[b] > p->L)
+      return fail(MSA_ERR_INVALID_ARG, "sequence %d: t0=%d n=%d (need t0, n >= 0, t0+n <= L=%d)",
+                  b, t0[b], n[b], p->L);
+    N += n[b];
+  }
+  if (N == 0) return MSA_OK;
+  if (!q || !q_idx || !k_cache || !v_cache || !k_idx_cache || !out)
+    return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(q_idx) || !aligned16(k_cache) || !aligned16(v_cache) ||
+      !aligned16(k_idx_cache) || !aligned16(out) || (lse && !aligned16(lse)))
+    return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const VarlenWs vw = varlen_ws(p);
+  rc = check_ws(ws, ws_bytes, attn_ws(p, vw.attn_base).end);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
+
+  // Host-built tables: per-sequence K/V maps (row extent t0 + n, so keys past
+  // a sequence's end load as zeros), query geometry, and the index branch's
+  // (b, tile) work list, longest tiles first.
+  const int B = p->B;
+  std::vector<uint8_t> tab(vw.sel - vw.maps, 0);
+  CUtensorMap *maps = reinterpret_cast<CUtensorMap *>(tab.data());
+  int4 *seqs = reinterpret_cast<int4 *>(tab.data() + (vw.seqs - vw.maps));
+  int2 *items = reinterpret_cast<int2 *>(tab.data() + (vw.items - vw.maps));
+  const size_t kv_seq = size_t(p->L) * p->G * p->d;   // elements per sequence
+  int row0 = 0, n_tab = 0;
+  for (int b = 0; b < B; ++b) {
+    const int kv_rows = t0[b] + n[b] > 0 ? t0[b] + n[b] : 1;
+    rc = make_kv_tmap(&maps[2 * b], k_cache + b * kv_seq, p, kv_rows, 1);
+    if (rc) return rc;
+    rc = make_kv_tmap(&maps[2 * b + 1], v_cache + b * kv_seq, p, kv_rows, 1);
+    if (rc) return rc;
+    seqs[b] = make_int4(row0, t0[b], n[b], row0);
+    if (n[b] > 0)
+      for (int i = t0[b] / 128; i < (t0[b] + n[b] + 127) / 128; ++i) items[n_tab++] = make_int2(b, i);
     row0 += n[b];
   }
-  return MSA_OK;
+  std::stable_sort(items, items + n_tab, [](const int2 &x, const int2 &y) { return x.y > y.y; });
+  const size_t tab_bytes = (vw.items - vw.maps) + sizeof(int2) * size_t(n_tab);
+  cudaError_t e = cudaMemcpyAsync(wsb + vw.maps, tab.data(), tab_bytes, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e, "ragged batch tables upload");
+
+  msa::QGeo qg;
+  qg.seqs = reinterpret_cast<const int4 *>(wsb + vw.seqs);
+  qg.B = B; qg.G = p->G; qg.Lq = 0; qg.tq0 = 0;
+  qg.N = (int)N;
+  qg.sel_gs = (int)N;
+  int32_t *sel = reinterpret_cast<int32_t *>(wsb + vw.sel);
+  IndexWork iw;
+  iw.items = reinterpret_cast<const int2 *>(wsb + vw.items);
+  iw.n_tab = n_tab;
+  iw.r_lo = 0;
+  iw.r_hi = (int)N;
+  rc = run_index_select(p, q_idx, k_idx_cache, sel, nullptr, ws, st, qg, iw);
+  if (rc) return rc;
+  AttnPlan pl;
+  rc = plan_attn(p, k_cache, v_cache, vw.attn_base, qg, p->L,
+                 reinterpret_cast<const CUtensorMap *>(wsb + vw.maps), &pl);
+  if (rc) return rc;
+  return run_prefill_attn(p, pl, q, sel, out, lse, ws, st);
 }
 
 int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k_h,
@@ -693,42 +809,52 @@ int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k
   HostEvents *ev = nullptr;
   rc = host_events(&ev);
   if (rc) return rc;
-  AttnPlan pl;
-  rc = plan_attn(p, dev->k, dev->v, base, whole(p), &pl);
-  if (rc) return rc;
+  // One sequence at a time (a B = 1 problem at the sequence's offsets), each
+  // pipelined per query chunk [t0, t0+Lc): upload the chunk's rows (index
+  // inputs first), run the index branch for the chunk's query tiles and the
+  // main branch for its queries, download its output.  A chunk only needs
+  // rows < t0 + Lc, so uploads, computation and downloads of neighbouring
+  // chunks overlap; uploads run ahead on copy_stream, downloads on the
+  // library's download stream.
+  msa_params p1 = *p;
+  p1.B = 1;
+  const msa::QGeo qg = whole(&p1);
   int32_t *sel = reinterpret_cast<int32_t *>(reinterpret_cast<uint8_t *>(ws) + msa::kWsHeader);
-  const ChunkSink sink{ev->down, ev->chunk, out_h, lse_h};
-  // Per query chunk [t0, t0+Lc): upload the chunk's rows (index inputs
-  // first), run the index branch for the chunk's query tiles and the main
-  // branch for its queries, download its output.  A chunk only needs rows
-  // < t0 + Lc, so uploads, computation and downloads of neighbouring chunks
-  // overlap; uploads run ahead on copy_stream, downloads on the library's
-  // download stream.
-  for (int t0 = 0; t0 < p->L; t0 += pl.w.Lc) {
-    const int Lc = (p->L - t0) < pl.w.Lc ? (p->L - t0) : pl.w.Lc;
-    cudaError_t e = cudaSuccess;
-    auto up = [&](msa_bf16 *d, const msa_bf16 *h, size_t row) {   // rows [t0, t0+Lc) of each b
-      for (int b = 0; b < p->B && e == cudaSuccess; ++b) {
-        const size_t off = (size_t(b) * p->L + t0) * row;
+  for (int b = 0; b < p->B; ++b) {
+    const size_t rows0 = size_t(b) * p->L;   // first row of sequence b
+    auto at = [&](auto *ptr, size_t row_elems) { return ptr + rows0 * row_elems; };
+    const size_t e_q = size_t(p->H) * p->d, e_kv = size_t(p->G) * p->d;
+    const size_t e_qi = size_t(p->G) * p->d_idx, e_ki = size_t(p->d_idx);
+    AttnPlan pl;
+    rc = plan_attn(&p1, at(dev->k, e_kv), at(dev->v, e_kv), base, qg, p->L, nullptr, &pl);
+    if (rc) return rc;
+    const ChunkSink sink{ev->down, ev->chunk, at(out_h, e_q), lse_h ? at(lse_h, size_t(p->H)) : nullptr};
+    for (int t0 = 0; t0 < p->L; t0 += pl.w.Rc) {
+      const int Lc = (p->L - t0) < pl.w.Rc ? (p->L - t0) : pl.w.Rc;
+      cudaError_t e = cudaSuccess;
+      auto up = [&](msa_bf16 *d, const msa_bf16 *h, size_t row) {   // rows [t0, t0+Lc)
+        if (e != cudaSuccess) return;
+        const size_t off = (rows0 + t0) * row;
         e = cudaMemcpyAsync(d + off, h + off, size_t(Lc) * row * 2, cudaMemcpyHostToDevice, cp);
-      }
-    };
-    up(dev->k_idx, k_idx_h, size_t(p->d_idx));
-    up(dev->q_idx, q_idx_h, size_t(p->G) * p->d_idx);
-    if (e == cudaSuccess) e = cudaEventRecord(ev->idx_in, cp);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->idx_in, 0);
-    if (e != cudaSuccess) return cuda_fail(e, "index input upload");
-    rc = run_index_select(p, dev->q_idx, dev->k_idx, sel, nullptr, ws, st, whole(p), t0, t0 + Lc);
-    if (rc) return rc;
-    up(dev->k, k_h, size_t(p->G) * p->d);
-    up(dev->v, v_h, size_t(p->G) * p->d);
-    up(dev->q, q_h, size_t(p->H) * p->d);
-    if (e == cudaSuccess) e = cudaEventRecord(ev->all_in, cp);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->all_in, 0);
-    if (e != cudaSuccess) return cuda_fail(e, "main input upload");
-    rc = run_attn_chunk(p, pl, dev->q, sel, dev->out, lse_h ? dev->lse : nullptr, ws, t0, Lc, st,
-                        &sink);
-    if (rc) return rc;
+      };
+      up(dev->k_idx, k_idx_h, e_ki);
+      up(dev->q_idx, q_idx_h, e_qi);
+      if (e == cudaSuccess) e = cudaEventRecord(ev->idx_in, cp);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->idx_in, 0);
+      if (e != cudaSuccess) return cuda_fail(e, "index input upload");
+      rc = run_index_select(&p1, at(dev->q_idx, e_qi), at(dev->k_idx, e_ki), sel, nullptr, ws, st,
+                            qg, uniform_index_work(qg, t0, t0 + Lc));
+      if (rc) return rc;
+      up(dev->k, k_h, e_kv);
+      up(dev->v, v_h, e_kv);
+      up(dev->q, q_h, e_q);
+      if (e == cudaSuccess) e = cudaEventRecord(ev->all_in, cp);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(st, ev->all_in, 0);
+      if (e != cudaSuccess) return cuda_fail(e, "main input upload");
+      rc = run_attn_chunk(&p1, pl, at(dev->q, e_q), sel, at(dev->out, e_q),
+                          lse_h ? at(dev->lse, size_t(p->H)) : nullptr, ws, t0, Lc, st, &sink);
+      if (rc) return rc;
+    }
   }
   cudaError_t e = cudaSuccess;
   // later work on `stream` runs after the last download
@@ -744,7 +870,7 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
                              msa_bf16 *dk, msa_bf16 *dv, void *ws, size_t ws_bytes,
                              msa_stream stream) {
   g_err[0] = 0;
-  int rc = check_params(p, false);
+  int rc = check_params(p, false, true);
   if (rc) return rc;
   if (p->B == 0 || p->L == 0) return MSA_OK;
   if (!q || !k || !v || !out || !lse || !dout || !sel || !dq || !dk || !dv)
@@ -753,18 +879,19 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
       !aligned16(dout) || !aligned16(sel) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
   const BwdWs w = bwd_ws(p);
-  const size_t entries = size_t(p->B) * p->G * w.Lc * p->top_k;
+  const size_t entries = size_t(p->G) * w.Rc * p->top_k;
   if (entries * (p->H / p->G) >= (size_t(1) << 31))
-    return fail(MSA_ERR_UNSUPPORTED, "B*chunk*H*top_k = %zu partial rows (limit 2^31)",
+    return fail(MSA_ERR_UNSUPPORTED, "chunk*H*top_k = %zu partial rows (limit 2^31)",
                 entries * (p->H / p->G));
   rc = check_ws(ws, ws_bytes, w.end);
   if (rc) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
   const int nb = p->L / 128;
+  const int N = p->B * p->L;
   CUtensorMap tk, tv;
   {
-    const uint64_t dims[3] = {uint64_t(p->d), uint64_t(p->G), uint64_t(p->B) * p->L};
+    const uint64_t dims[3] = {uint64_t(p->d), uint64_t(p->G), uint64_t(N)};
     const uint64_t str[2] = {uint64_t(p->d) * 2, uint64_t(p->d) * 2 * p->G};
     const uint32_t box[3] = {64, 1, 128};
     rc = make_tmap(&tk, k, 3, dims, str, box);
@@ -773,9 +900,9 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
     if (rc) return rc;
   }
   msa::RevIdxArgs ra;
-  ra.B = p->B; ra.G = p->G; ra.L = p->L; ra.nb = nb; ra.top_k = p->top_k;
+  ra.G = p->G; ra.nb = nb; ra.top_k = p->top_k;
   ra.qpi = 128 / (p->H / p->G);
-  ra.Lq = p->L; ra.tq0 = 0;
+  ra.q = whole(p);
   ra.sel = sel;
   ra.cnt = reinterpret_cast<int32_t *>(wsb + w.cnt);
   ra.list_off = reinterpret_cast<int32_t *>(wsb + w.list_off);
@@ -804,13 +931,13 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
     if (e != cudaSuccess) return cuda_fail(e, "backward accumulator reset");
   }
   const int sms = num_sms();
-  for (int t0 = 0; t0 < p->L; t0 += w.Lc) {
-    const int Lc = (p->L - t0) < w.Lc ? (p->L - t0) : w.Lc;
-    ra.t0 = t0; ra.Lc = Lc;
+  for (int r0 = 0; r0 < N; r0 += w.Rc) {
+    const int Rc = (N - r0) < w.Rc ? (N - r0) : w.Rc;
+    ra.r0 = r0; ra.Rc = Rc;
     e = msa::launch_revidx(ra, st);
     if (e != cudaSuccess) return cuda_fail(e, "reverse index launch");
-    a.t0 = t0; a.Lc = Lc;
-    a.last = (t0 + Lc >= p->L) ? 1 : 0;
+    a.r0 = r0; a.Rc = Rc;
+    a.last = (r0 + Rc >= N) ? 1 : 0;
     e = msa::launch_backward(tk, tv, a, sms, st);
     if (e != cudaSuccess) return cuda_fail(e, "backward launch");
   }

@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  const int n_bgj = a.B * a.G * a.nb;
+  const int n_bgj = a.q.B * a.G * a.nb;
   const int n_items = a.item_off[n_bgj];
   if (n_items > a.max_items && tid == 0) atomicCAS(a.status, 0, kStatusBadInput);
   // Each CTA takes a contiguous range of work items: consecutive items mostly
@@ -244,7 +244,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           const int j = bgj % a.nb;
           const int g = (bgj / a.nb) % a.G;
           const int b = bgj / (a.nb * a.G);
-          const int z = b * a.L + j * kBlock;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {   // K of run m is tile sequence 2m, V is 2m+1
             const int tau = 2 * m + h;
@@ -255,9 +254,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             }
             mbar_arrive_expect_tx(bar(C::BAR_KVFULL + x), kTile);
             const uint32_t dst = s_base + C::SMEM_KV + x * kTile;
-            const CUtensorMap *tm = h ? &tm_v : &tm_k;
-            tma_load_3d(dst, tm, bar(C::BAR_KVFULL + x), 0, g, z);
-            tma_load_3d(dst + 16384, tm, bar(C::BAR_KVFULL + x), 64, g, z);
+            // 4-D maps (d, G, key rows, sequences): the sequence's own map
+            // (batch coordinate 0) or the launch's map over the batch
+            const void *tm = a.kv_maps ? static_cast<const void *>(&a.kv_maps[2 * b + h])
+                                       : (h ? static_cast<const void *>(&tm_v)
+                                            : static_cast<const void *>(&tm_k));
+            const int zb = a.kv_maps ? 0 : b;
+            if (a.kv_maps) tensormap_acquire(tm);
+            tma_load_4d(dst, tm, bar(C::BAR_KVFULL + x), 0, g, j * kBlock, zb);
+            tma_load_4d(dst + 16384, tm, bar(C::BAR_KVFULL + x), 64, g, j * kBlock, zb);
             issued[x] = tau;
           }
         }
@@ -433,8 +438,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int bgj = d.x;
         const int g = (bgj / a.nb) % a.G;
         const int b = bgj / (a.nb * a.G);
-        const uint16_t *qb = a.q + size_t(g) * R * kHeadDim + gran * 8;
-        const int qrow0 = b * a.Lq - a.tq0;   // + t: the query's row in q (t >= tq0)
+        const uint16_t *qb = a.q_ptr + size_t(g) * R * kHeadDim + gran * 8;
+        const int4 sq = qgeo_seq(a.q, b);
+        const int qrow0 = sq.x - sq.y;        // + t: the query's packed row in q
         const uint32_t stq = s_base + C::SMEM_Q + s * kTile + (gran >> 3) * 16384;
         // row pair p = wg + 6*it (rows 2p, 2p+1): one coalesced 512-byte
         // copy per warp instruction
@@ -633,28 +639,28 @@ cudaError_t launch_prefill_attn(const CUtensorMap &tk, const CUtensorMap &tv, co
 // ---------------------------------------------------------------- combine
 namespace {
 
-// One warp per (b, t, h): merge the row's partials (normalised o_s, lse_s)
-// into o = sum_s exp(lse_s - M) o_s / sum_s exp(lse_s - M), M = max lse_s.
-// Slot s of the row lives at partial row rho_s = pos_of[b,g,t,s] * R + hh.
-// The selection row and the positions are loaded independently, then all of
-// a lane's partial-row loads (4 of the d values of each slot, granule order
-// undone) and its lse load are issued before any reduction.
+// One warp per (packed row, h): merge the row's partials (normalised o_s,
+// lse_s) into o = sum_s exp(lse_s - M) o_s / sum_s exp(lse_s - M), M = max
+// lse_s.  Slot s of the row lives at partial row rho_s = pos_of[g,row,s] * R
+// + hh.  The selection row and the positions are loaded independently, then
+// all of a lane's partial-row loads (4 of the d values of each slot, granule
+// order undone) and its lse load are issued before any reduction.
 template <int KCAP>
 __global__ void __launch_bounds__(256) msa_combine_kernel(const CombineArgs a) {
   const long long wrow = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  const long long n_rows = (long long)a.B * a.Lc * a.H;
+  const long long n_rows = (long long)a.Rc * a.H;
   if (wrow >= n_rows) return;
   const int h = (int)(wrow % a.H);
-  const long long bt = wrow / a.H;
-  const int tl = (int)(bt % a.Lc);
-  const int b = (int)(bt / a.Lc);
-  const int t = a.t0 + tl;
+  const int rl = (int)(wrow / a.H);
+  const int row = a.r0 + rl;
+  const int b = qgeo_seq_of_row(a.q, row);
+  const int4 sq = qgeo_seq(a.q, b);
   const int r = a.H / a.G;
   const int g = h / r;
   const int hh = h % r;
-  const int32_t *sel = a.sel + ((size_t(b) * a.G + g) * a.Lq + (t - a.tq0)) * a.top_k;
-  const int32_t *pos = a.pos_of + ((size_t(b) * a.G + g) * a.Lc + tl) * a.top_k;
+  const int32_t *sel = a.sel + ((long long)sq.w + (long long)g * a.q.sel_gs + (row - sq.x)) * a.top_k;
+  const int32_t *pos = a.pos_of + ((long long)g * a.Rc + rl) * a.top_k;
   const bool in_k = lane < a.top_k;
   const int my_sel = in_k ? sel[lane] : -1;
   const int my_pos = in_k ? pos[lane] : 0;
@@ -695,15 +701,14 @@ __global__ void __launch_bounds__(256) msa_combine_kernel(const CombineArgs a) {
   uint2 res;
   res.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   res.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-  const size_t orow = (size_t)b * a.Lq + (t - a.tq0);
-  *reinterpret_cast<uint2 *>(a.out + (orow * a.H + h) * kHeadDim + lane * 4) = res;
-  if (a.lse && lane == 0) a.lse[orow * a.H + h] = (wsum > 0.f) ? M + __logf(wsum) : -INFINITY;
+  *reinterpret_cast<uint2 *>(a.out + ((size_t)row * a.H + h) * kHeadDim + lane * 4) = res;
+  if (a.lse && lane == 0) a.lse[(size_t)row * a.H + h] = (wsum > 0.f) ? M + __logf(wsum) : -INFINITY;
 }
 
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st) {
-  const long long n_rows = (long long)a.B * a.Lc * a.H;
+  const long long n_rows = (long long)a.Rc * a.H;
   if (n_rows == 0) return cudaSuccess;
   const unsigned grid = (unsigned)((n_rows + 7) / 8);
   if (a.top_k <= 4)

@@ -2,9 +2,9 @@
 // of researchpapers.dev "MiniMax Sparse Attention", section "对工程团队的意义";
 // "KV external aggregation Q" of the baguaai.com 稀疏注意力 MSA entry).
 //
-// For a query chunk [t0, t0+Lc) it lists, for every (b, g, key block j),
-// the (query, slot) pairs whose selection holds j -- a counting sort of the
-// selection by key block:
+// For a query chunk (the packed query rows [r0, r0+Rc), see QGeo) it lists,
+// for every (b, g, key block j), the (query, slot) pairs whose selection
+// holds j -- a counting sort of the selection by key block:
 //   1. count   cnt[b,g,j] += 1 for every selected entry; the value before
 //              the increment (the entry's rank among the entries of block
 //              j) is kept in pos_of
@@ -12,11 +12,11 @@
 //              item_off = exclusive scan of ceil(cnt / qpi)  (work items of
 //              at most qpi queries, i.e. 128 query-head rows, per block)
 //   3. fill    pos = list_off[bgj] + rank; list[pos] = t * 32 + slot and
-//              pos_of[b,g,t,slot] = pos (the inverse map by which the merge
-//              finds a row's partials).  No atomics: the order inside a list
-//              is whatever order the count's atomics produced, and each
-//              (t, slot) partial is computed independently of the others in
-//              its tile.
+//              pos_of[g, row, slot] = pos (the inverse map by which the
+//              merge finds a row's partials).  No atomics: the order inside
+//              a list is whatever order the count's atomics produced, and
+//              each (t, slot) partial is computed independently of the
+//              others in its tile.
 // Every work item then holds <= qpi queries, so items cost the same and a
 // persistent grid balances itself whatever the causal skew between early
 // and late key blocks.
@@ -29,21 +29,38 @@ namespace msa {
 
 namespace {
 
+// Entry e of the chunk, in [G][Rc][top_k] order: its group, sequence,
+// position and selection slot address.
+struct RevEntry {
+  int k, g, b, t;
+  long long sel_idx;
+};
+__device__ __forceinline__ RevEntry rev_entry(const RevIdxArgs &a, long long e) {
+  RevEntry x;
+  x.k = (int)(e % a.top_k);
+  const long long gr = e / a.top_k;
+  const int rl = (int)(gr % a.Rc);
+  x.g = (int)(gr / a.Rc);
+  const int r = a.r0 + rl;
+  x.b = qgeo_seq_of_row(a.q, r);
+  const int4 s = qgeo_seq(a.q, x.b);
+  x.t = s.y + (r - s.x);
+  x.sel_idx = ((long long)s.w + (long long)x.g * a.q.sel_gs + (r - s.x)) * a.top_k + x.k;
+  return x;
+}
+
 __global__ void __launch_bounds__(256) revidx_count_kernel(const RevIdxArgs a) {
-  const long long n = (long long)a.B * a.G * a.Lc * a.top_k;
+  const long long n = (long long)a.G * a.Rc * a.top_k;
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
        e += (long long)gridDim.x * blockDim.x) {
-    const int k = (int)(e % a.top_k);
-    const long long r = e / a.top_k;
-    const int tl = (int)(r % a.Lc);
-    const long long bg = r / a.Lc;
-    const int j = a.sel[(bg * a.Lq + (a.t0 - a.tq0) + tl) * a.top_k + k];
+    const RevEntry x = rev_entry(a, e);
+    const int j = a.sel[x.sel_idx];
     if (j < 0) continue;
     if (j >= a.nb) {
       atomicCAS(a.status, 0, kStatusBadInput);
       continue;
     }
-    a.pos_of[r * a.top_k + k] = atomicAdd(&a.cnt[bg * a.nb + j], 1);
+    a.pos_of[e] = atomicAdd(&a.cnt[((long long)x.b * a.G + x.g) * a.nb + j], 1);
   }
 }
 
@@ -79,7 +96,7 @@ __device__ __forceinline__ void block_scan2(int &x, int &y, int *warp_x, int *wa
 // tiles of 4096 entries (4 consecutive entries per thread, 16-byte loads).
 __global__ void __launch_bounds__(1024) revidx_scan_kernel(const RevIdxArgs a) {
   __shared__ int warp_x[32], warp_y[32], tot[2];
-  const int n = a.B * a.G * a.nb;
+  const int n = a.q.B * a.G * a.nb;
   int carry_x = 0, carry_y = 0;
   for (int base = 0; base < n; base += 4096) {
     const int i0 = base + 4 * threadIdx.x;
@@ -119,34 +136,29 @@ __global__ void __launch_bounds__(1024) revidx_scan_kernel(const RevIdxArgs a) {
 }
 
 __global__ void __launch_bounds__(256) revidx_fill_kernel(const RevIdxArgs a) {
-  const long long n = (long long)a.B * a.G * a.Lc * a.top_k;
+  const long long n = (long long)a.G * a.Rc * a.top_k;
   for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n;
        e += (long long)gridDim.x * blockDim.x) {
-    const int k = (int)(e % a.top_k);
-    const long long r = e / a.top_k;
-    const int tl = (int)(r % a.Lc);
-    const long long bg = r / a.Lc;
-    const int t = a.t0 + tl;
-    const int j = a.sel[(bg * a.Lq + (t - a.tq0)) * a.top_k + k];
+    const RevEntry x = rev_entry(a, e);
+    const int j = a.sel[x.sel_idx];
     if (j < 0 || j >= a.nb) continue;
-    const long long e_out = r * a.top_k + k;
-    const int pos = a.list_off[bg * a.nb + j] + a.pos_of[e_out];
-    a.list[pos] = t * 32 + k;
-    a.pos_of[e_out] = pos;
+    const int pos = a.list_off[((long long)x.b * a.G + x.g) * a.nb + j] + a.pos_of[e];
+    a.list[pos] = x.t * 32 + x.k;
+    a.pos_of[e] = pos;
   }
 }
 
 }  // namespace
 
 cudaError_t launch_revidx(const RevIdxArgs &a, cudaStream_t st) {
-  const int n_cnt = a.B * a.G * a.nb;
+  const int n_cnt = a.q.B * a.G * a.nb;
   cudaError_t e = cudaMemsetAsync(a.cnt, 0, sizeof(int32_t) * n_cnt, st);
   if (e != cudaSuccess) return e;
-  const long long n = (long long)a.B * a.G * a.Lc * a.top_k;
+  const long long n = (long long)a.G * a.Rc * a.top_k;
   const int grid = (int)((n + 255) / 256 < 148 * 16 ? (n + 255) / 256 : 148 * 16);
-  revidx_count_kernel<<<grid, 256, 0, st>>>(a);
+  if (n > 0) revidx_count_kernel<<<grid, 256, 0, st>>>(a);
   revidx_scan_kernel<<<1, 1024, 0, st>>>(a);
-  revidx_fill_kernel<<<grid, 256, 0, st>>>(a);
+  if (n > 0) revidx_fill_kernel<<<grid, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 

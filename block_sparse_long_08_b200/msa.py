@@ -33,6 +33,7 @@ MSA_OP_PREFILL_ATTN = 1
 MSA_OP_DECODE = 2
 MSA_OP_FORWARD = 3
 MSA_OP_BACKWARD = 4
+MSA_OP_FORWARD_VARLEN = 5
 
 
 class MSAError(RuntimeError):
@@ -181,7 +182,8 @@ def msa_index_select(q_idx: torch.Tensor, k_idx: torch.Tensor, top_k: int, *,
     dev = q_idx.device
     if sel is None:
         sel = torch.empty((B, G, L, top_k), dtype=torch.int32, device=dev)
-    scores = torch.empty((B, G, L, L // 128), dtype=torch.float32, device=dev) if block_scores else None
+    scores = torch.empty((B, G, L, (L + 127) // 128), dtype=torch.float32,
+                         device=dev) if block_scores else None
     ws = _ensure_ws(ws, p, MSA_OP_INDEX_SELECT, dev)
     _check(lib().msa_index_select(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(sel), _ptr(scores),
                                   _ptr(ws), ws.numel(), _stream(stream)))
@@ -309,12 +311,11 @@ def msa_forward_cached_varlen(q, q_idx, k_cache, v_cache, k_idx_cache, t0, n, to
     if sum(int(v) for v in n) != q.shape[0]:
         raise ValueError("q rows must equal sum(n)")
     p = make_params(B, Lmax, H, G, d, q_idx.shape[2], 128, top_k, scale, chunk)
-    p1 = make_params(1, Lmax, H, G, d, q_idx.shape[2], 128, top_k, scale, chunk)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
     lse = torch.empty((q.shape[0], H), dtype=torch.float32, device=dev) if want_lse else None
-    ws = _ensure_ws(ws, p1, MSA_OP_FORWARD, dev)
+    ws = _ensure_ws(ws, p, MSA_OP_FORWARD_VARLEN, dev)
     _check(lib().msa_forward_cached_varlen(ctypes.byref(p), t0a, na, _ptr(q), _ptr(q_idx),
                                            _ptr(k_cache), _ptr(v_cache), _ptr(k_idx_cache),
                                            _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),

@@ -52,9 +52,11 @@
  *     the start of `ws`; msa_read_status() synchronises the stream and
  *     returns/clears it.
  *   - Supported: d == 128, d_idx in {64, 128}, block == 128,
- *     1 <= top_k <= 32, H % G == 0 with H/G in {1,2,4,8,16}, L % 128 == 0;
- *     the decode entry points also need G <= 8 (the cache scan scores all
- *     groups of a key in one 8-column tensor-core product).
+ *     1 <= top_k <= 32, H % G == 0 with H/G in {1,2,4,8,16}, B*L <= 2^26.
+ *     Any L: the last block of a sequence may be partial (nb = ceil(L/128)
+ *     blocks); only the backward needs L % 128 == 0.  The decode entry
+ *     points also need G <= 8 (the cache scan scores all groups of a key in
+ *     one 8-column tensor-core product).
  *     Other shapes give MSA_ERR_UNSUPPORTED.  B == 0 or L == 0 is a no-op.
  */
 #ifndef MSA_H_
@@ -80,10 +82,11 @@ typedef struct msa_params {
   int32_t block;   /* KV block length (128) */
   int32_t top_k;   /* blocks kept per (query, group), local block included */
   float scale;     /* softmax scale of the main branch; 0 -> 1/sqrt(d) */
-  int32_t chunk;   /* query-chunk length of the prefill attention and the
-                      backward, a multiple of 128; 0 -> the longest chunk
-                      whose partials fit the 16 GiB budget.  Smaller chunks
-                      need a smaller workspace and re-read K/V more often. */
+  int32_t chunk;   /* query rows per chunk of the prefill attention and the
+                      backward (rows of the packed batch, b*L + t), a
+                      multiple of 128; 0 -> the longest chunk whose partials
+                      fit the 16 GiB budget.  Smaller chunks need a smaller
+                      workspace and re-read K/V more often. */
 } msa_params;
 
 enum {
@@ -101,13 +104,14 @@ enum {
   MSA_OP_PREFILL_ATTN = 1,
   MSA_OP_DECODE = 2,
   MSA_OP_FORWARD = 3,
-  MSA_OP_BACKWARD = 4
+  MSA_OP_BACKWARD = 4,
+  MSA_OP_FORWARD_VARLEN = 5
 };
 
 /* Index Branch (explainer §2.1; researchpapers.dev "机制").
  *   q_idx  [B,L,G,d_idx] bf16, k_idx [B,L,d_idx] bf16            (in)
  *   sel    [B,G,L,top_k] int32                                    (out)
- *   block_scores [B,G,L,nb] fp32, nb = L/block, or NULL            (out)
+ *   block_scores [B,G,L,nb] fp32, nb = ceil(L/block), or NULL       (out)
  *     When given, entry (t, j) holds S[b,g,t,j] for j < t/block and -inf
  *     for j >= t/block (the local block is forced, never scored), and sel
  *     is computed from these stored scores by the top-k kernel.  When NULL
@@ -229,7 +233,7 @@ int msa_forward(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k, const
  * prefix; the explainer's serving discussion, §4.1).  Each new query attends
  * exactly as in msa_forward over a sequence of length t0 + n, so the
  * results equal rows [t0, t0 + n) of that call.
- *   p->L = cache capacity Lmax; t0 and n multiples of 128, t0 + n <= Lmax
+ *   p->L = cache capacity Lmax; any t0, n >= 0 with t0 + n <= Lmax
  *   q [B,n,H,d], q_idx [B,n,G,d_idx] bf16: the new tokens' queries     (in)
  *   k_cache, v_cache [B,Lmax,G,d], k_idx_cache [B,Lmax,d_idx] bf16, the
  *     new tokens' rows already written; rows >= t0 + n are not read     (in)
@@ -246,15 +250,20 @@ int msa_forward_cached(const msa_params *p, int t0, int n, const msa_bf16 *q,
  * positions with different numbers of new tokens (a ragged serving batch).
  * The new tokens' query rows are packed: sequence b owns rows
  * [row0_b, row0_b + n[b]) with row0_b = n[0] + ... + n[b-1].
- *   t0[B], n[B]: HOST int32 arrays; every t0[b] and n[b] a multiple of 128,
+ *   t0[B], n[B]: HOST int32 arrays; any t0[b], n[b] >= 0 with
  *     t0[b] + n[b] <= Lmax (n[b] may be 0)
  *   q [sum n, H, d], q_idx [sum n, G, d_idx] bf16 (packed)              (in)
  *   k_cache, v_cache [B,Lmax,G,d], k_idx_cache [B,Lmax,d_idx]            (in)
  *   out [sum n, H, d] bf16 (packed); lse [sum n, H] fp32 or NULL        (out)
- *   ws >= msa_workspace_bytes(p, MSA_OP_FORWARD) with p->B = 1
- * Sequences are processed one after another on `stream`, each exactly as
- * msa_forward_cached with B = 1.  (Kernels that take the whole ragged
- * batch in one launch are not built.) */
+ *   ws >= msa_workspace_bytes(p, MSA_OP_FORWARD_VARLEN)
+ * The whole batch runs in one launch per kernel (per query chunk of
+ * packed rows): the call builds, on the host, each sequence's K/V tensor
+ * maps (row extent t0[b] + n[b], so keys past a sequence's end are never
+ * read), the per-sequence query geometry and the index branch's list of
+ * (sequence, 128-query tile) work items, longest first, and uploads them
+ * into ws with one cudaMemcpyAsync (from pageable memory: the call returns
+ * once they are staged).  Every row equals msa_forward_cached's row for its
+ * sequence. */
 int msa_forward_cached_varlen(const msa_params *p, const int32_t *t0, const int32_t *n,
                               const msa_bf16 *q, const msa_bf16 *q_idx, const msa_bf16 *k_cache,
                               const msa_bf16 *v_cache, const msa_bf16 *k_idx_cache,
@@ -313,9 +322,10 @@ int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k
  * attends to get zero.  dq is bit-identical from run to run; dk and dv sum
  * a key block's queries in the reverse index's list order, which follows
  * atomics, so runs agree up to fp32 summation order.
- * Queries are processed in the prefill's chunks (msa_prefill_chunk_len;
- * p->chunk overrides it), each with its own reverse index and one bf16 dq
- * partial row per (query, head, slot) of the chunk (at most about 16 GiB).
+ * Needs L % 128 == 0.  Queries are processed in the prefill's chunks of
+ * packed rows (msa_prefill_chunk_len; p->chunk overrides it), each with its
+ * own reverse index and one bf16 dq partial row per (query, head, slot) of
+ * the chunk (at most about 16 GiB).
  * With more than one chunk, dk and dv are summed across chunks in fp32
  * accumulators (2 * B*L*G*d*4 bytes of workspace) and rounded to bf16 once.
  * ws >= msa_workspace_bytes(p, MSA_OP_BACKWARD). */
@@ -329,10 +339,11 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
  * (see msa_last_error). */
 size_t msa_workspace_bytes(const msa_params *p, int op);
 
-/* Query-chunk length the prefill attention uses for these params: queries
- * are processed in chunks of this many tokens so that per-block partial
- * results stay within a fixed workspace budget (about 16 GiB).  Each chunk
- * costs 5 kernel launches.  0 when p is invalid. */
+/* Query-chunk length the prefill attention uses for these params: the
+ * packed query rows (b*L + t) are processed in chunks of this many rows so
+ * that per-block partial results stay within a fixed workspace budget
+ * (about 16 GiB).  Each chunk costs 5 kernel launches.  0 when p is
+ * invalid. */
 int msa_prefill_chunk_len(const msa_params *p);
 
 /* Synchronise `stream`, return the device status recorded in ws (MSA_OK or

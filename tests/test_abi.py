@@ -54,7 +54,7 @@ def test_workspace_sizes(L, top_k, G, H, di):
 @pytest.mark.parametrize("field,value,code", [
     ("d", 64, M.MSA_ERR_UNSUPPORTED), ("d_idx", 96, M.MSA_ERR_UNSUPPORTED),
     ("block", 64, M.MSA_ERR_UNSUPPORTED), ("top_k", 33, M.MSA_ERR_UNSUPPORTED),
-    ("top_k", 0, M.MSA_ERR_INVALID_ARG), ("L", 1000, M.MSA_ERR_UNSUPPORTED),
+    ("top_k", 0, M.MSA_ERR_INVALID_ARG), ("L", -5, M.MSA_ERR_INVALID_ARG),
     ("H", 12, M.MSA_ERR_UNSUPPORTED), ("G", 3, M.MSA_ERR_INVALID_ARG),
     ("B", -1, M.MSA_ERR_INVALID_ARG), ("chunk", 100, M.MSA_ERR_INVALID_ARG),
     ("chunk", -128, M.MSA_ERR_INVALID_ARG)])
@@ -95,8 +95,8 @@ def test_empty_problem_is_noop():
 def test_chunk_length_follows_params():
     p = M.make_params(2, 8192, 32, 8, 128, 128, 128, 16)
     full = M.msa_prefill_chunk_len(p)
-    assert full == 8192                       # small problems run as one chunk
-    for c, want in ((1024, 1024), (128, 128), (16384, 8192)):
+    assert full == 16384                      # small problems run as one chunk of packed rows
+    for c, want in ((1024, 1024), (128, 128), (16384, 16384), (32768, 16384)):
         p.chunk = c
         assert M.msa_prefill_chunk_len(p) == want
     # a shorter chunk needs a smaller prefill workspace
@@ -125,7 +125,7 @@ def test_forward_host_rejects_bad_arguments():
     assert rc == M.MSA_ERR_WORKSPACE
 
 
-@pytest.mark.parametrize("t0,n", [(100, 128), (128, 100), (-128, 128), (3968, 256), (0, -128)])
+@pytest.mark.parametrize("t0,n", [(-128, 128), (3968, 256), (0, -128), (4000, 97), (-1, 1)])
 def test_cached_prefill_rejects_bad_ranges(t0, n):
     p = M.make_params(1, 4096, 8, 2, 128, 64, 128, 4)
     ok = ctypes.c_void_p(4096)
@@ -137,7 +137,8 @@ def test_cached_prefill_rejects_bad_ranges(t0, n):
 def test_varlen_rejects_bad_ranges():
     p = M.make_params(2, 4096, 8, 2, 128, 64, 128, 4)
     ok = ctypes.c_void_p(4096)
-    for t0, n in (([0, 100], [128, 128]), ([0, 3968], [128, 256]), ([-128, 0], [128, 128])):
+    for t0, n in (([0, 4000], [128, 100]), ([0, 3968], [128, 256]), ([-128, 0], [128, 128]),
+                  ([5, 0], [-1, 128])):
         rc = M.lib().msa_forward_cached_varlen(ctypes.byref(p), (ctypes.c_int32 * 2)(*t0),
                                                (ctypes.c_int32 * 2)(*n), ok, ok, ok, ok, ok, ok,
                                                None, ok, 1 << 30, None)
@@ -229,3 +230,20 @@ def test_backward_workspace_follows_chunking():
     acc = 2 * L * G * 128 * 4
     assert abs((whole - per_chunk(L)) - (half - per_chunk(L // 2) - acc)) <= 4096
     assert M.msa_prefill_chunk_len(M.make_params(1, L, H, G, top_k=K, chunk=L // 2)) == L // 2
+
+
+def test_any_length_except_backward():
+    """L need not be a multiple of the block length: the last block of a
+    sequence is partial.  Only the backward keeps L % 128 == 0."""
+    lib = M.lib()
+    for L in (1, 127, 1000, 2049):
+        p = M.make_params(2, L, 16, 4, 128, 128, 128, 5)
+        for op in (M.MSA_OP_INDEX_SELECT, M.MSA_OP_PREFILL_ATTN, M.MSA_OP_DECODE, M.MSA_OP_FORWARD,
+                   M.MSA_OP_FORWARD_VARLEN):
+            assert lib.msa_workspace_bytes(ctypes.byref(p), op) > 0, (L, op, M.msa_last_error())
+        assert lib.msa_workspace_bytes(ctypes.byref(p), M.MSA_OP_BACKWARD) == 0
+        assert "multiple of 128" in M.msa_last_error()
+    # the ragged-batch workspace holds the uniform forward's plus its tables
+    p = M.make_params(4, 4096, 16, 4, 128, 128, 128, 8)
+    assert (M.msa_workspace_bytes(p, M.MSA_OP_FORWARD_VARLEN)
+            >= M.msa_workspace_bytes(p, M.MSA_OP_FORWARD) + 4 * (2 * 128 + 16 + 32 * 8))

@@ -29,7 +29,10 @@ def full_run():
 
 
 @pytest.mark.parametrize("t0,n,chunk", [(0, 1024, 0), (1536, 1024, 0), (3072, 1024, 0),
-                                        (1024, 2048, 512)])
+                                        (1024, 2048, 512),
+                                        # positions and counts of any size
+                                        (100, 700, 0), (1000, 1, 0), (4000, 96, 0),
+                                        (1, 4095, 1024), (2047, 2, 0), (0, 77, 0)])
 def test_cached_prefill_equals_whole_sequence_rows(full_run, t0, n, chunk):
     shape, x, out, sel, lse = full_run
     cache = {nm: x[nm].clone() for nm in ("k", "v", "k_idx")}
@@ -79,26 +82,42 @@ def test_cached_prefill_against_oracle():
     assert e.max() <= P.OUT_MAX_ABS and e.mean() <= P.OUT_MEAN_ABS, (e.max(), e.mean())
 
 
-def test_ragged_batch_equals_whole_sequence_rows(full_run):
+@pytest.mark.parametrize("t0,n,chunk", [([1024, 2944], [768, 1152], 0),
+                                        ([100, 2947], [700, 1149], 0),
+                                        ([0, 3000], [77, 1], 0),
+                                        ([5, 129], [3000, 3967], 1024)])
+def test_ragged_batch_equals_whole_sequence_rows(full_run, t0, n, chunk):
     """Sequences continuing at different positions with different numbers of
-    new tokens (one with none), query rows packed."""
+    new tokens (one with none), query rows packed, the whole batch in one
+    launch per kernel.  Cache rows past each sequence's t0 + n hold NaN:
+    they must never be read."""
     shape, x, out, sel, lse = full_run
-    t0, n = [1024, 2944], [768, 1152]
     t0, n = t0 + [0], n + [0]          # a third sequence with no new tokens
     B = 2
     q = torch.cat([x["q"][b, t0[b]:t0[b] + n[b]] for b in range(B)])
     q_idx = torch.cat([x["q_idx"][b, t0[b]:t0[b] + n[b]] for b in range(B)])
-    o_c, l_c = M.msa_forward_cached_varlen(q, q_idx, x["k"], x["v"], x["k_idx"], t0[:B], n[:B],
-                                           shape.top_k, want_lse=True)
+    cache = {nm: x[nm].clone() for nm in ("k", "v", "k_idx")}
+    for c in cache.values():
+        for b in range(B):
+            c[b, t0[b] + n[b]:] = float("nan")
+    o_c, l_c = M.msa_forward_cached_varlen(q, q_idx, cache["k"], cache["v"], cache["k_idx"],
+                                           t0[:B], n[:B], shape.top_k, want_lse=True, chunk=chunk)
     torch.cuda.synchronize()
     want_o = torch.cat([out[b, t0[b]:t0[b] + n[b]] for b in range(B)])
     want_l = torch.cat([lse[b, t0[b]:t0[b] + n[b]] for b in range(B)])
     assert torch.equal(o_c, want_o)
     assert torch.equal(l_c, want_l)
     # an empty sequence in the batch
-    k3 = torch.cat([x["k"], x["k"][:1]])
-    v3 = torch.cat([x["v"], x["v"][:1]])
-    ki3 = torch.cat([x["k_idx"], x["k_idx"][:1]])
+    k3 = torch.cat([cache["k"], cache["k"][:1]])
+    v3 = torch.cat([cache["v"], cache["v"][:1]])
+    ki3 = torch.cat([cache["k_idx"], cache["k_idx"][:1]])
     o3 = M.msa_forward_cached_varlen(q, q_idx, k3, v3, ki3, t0, n, shape.top_k)
     torch.cuda.synchronize()
     assert torch.equal(o3, want_o)
+    # an empty sequence first, then the others
+    o4 = M.msa_forward_cached_varlen(q, q_idx, torch.cat([k3[2:], cache["k"]]),
+                                     torch.cat([v3[2:], cache["v"]]),
+                                     torch.cat([ki3[2:], cache["k_idx"]]), [0] + t0[:B],
+                                     [0] + n[:B], shape.top_k)
+    torch.cuda.synchronize()
+    assert torch.equal(o4, want_o)

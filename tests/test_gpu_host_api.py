@@ -20,8 +20,11 @@ def _inputs(shape, seed):
     return I.prefill_inputs(shape, seed, device=DEV)
 
 
-def test_chunked_prefill_is_bit_identical():
-    shape = I.PrefillShape(B=2, L=4096, H=16, G=4, d=128, d_idx=128, top_k=8)
+@pytest.mark.parametrize("L", [4096, 3000])
+def test_chunked_prefill_is_bit_identical(L):
+    """Chunks are ranges of the packed query rows b*L + t, so with B = 2 some
+    chunks span the end of one sequence and the start of the next."""
+    shape = I.PrefillShape(B=2, L=L, H=16, G=4, d=128, d_idx=128, top_k=8)
     x = _inputs(shape, 31)
     sel = M.msa_index_select(x["q_idx"], x["k_idx"], shape.top_k)
     o_ref, l_ref = M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, want_lse=True)
@@ -32,8 +35,9 @@ def test_chunked_prefill_is_bit_identical():
         assert torch.equal(l, l_ref), chunk
 
 
-def test_forward_host_matches_device_forward():
-    shape = I.PrefillShape(B=2, L=4096, H=32, G=8, d=128, d_idx=128, top_k=16)
+@pytest.mark.parametrize("L", [4096, 2049])
+def test_forward_host_matches_device_forward(L):
+    shape = I.PrefillShape(B=2, L=L, H=32, G=8, d=128, d_idx=128, top_k=16)
     x = _inputs(shape, 32)
     o_ref, l_ref = M.msa_forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], shape.top_k,
                                  want_lse=True)

@@ -52,7 +52,8 @@ def _rows_sample(L, n, seed, block=128):
 @pytest.mark.parametrize("L,G,di,top_k,seed", [(2048, 2, 64, 4, 0), (1024, 8, 128, 3, 5),
                                                (640, 1, 128, 2, 6), (1152, 4, 64, 17, 7),
                                                (2048, 2, 128, 9, 8), (2560, 2, 64, 5, 9),
-                                               (3200, 1, 64, 17, 10), (2048, 4, 128, 12, 11)])
+                                               (3200, 1, 64, 17, 10), (2048, 4, 128, 12, 11),
+                                               (1000, 2, 64, 4, 12), (2049, 4, 128, 5, 13)])
 def test_block_scores_and_selection(L, G, di, top_k, seed):
     shape = I.PrefillShape(B=2, L=L, H=G * 4, G=G, d=128, d_idx=di, top_k=top_k)
     x = _prefill(shape, seed)
@@ -64,7 +65,7 @@ def test_block_scores_and_selection(L, G, di, top_k, seed):
     sc = scores.cpu().numpy()
     sel = sel_f.cpu().numpy()
     qi, ki = P.f64(x["q_idx"]), P.f64(x["k_idx"])
-    nb = L // 128
+    nb = (L + 127) // 128       # the last block may be partial
     n_swaps = 0
     for b in range(2):
         for t in range(0, L, 3 if L > 1024 else 1):
@@ -115,7 +116,8 @@ def test_zero_index_keys_all_ties():
 # ------------------------------------------------------------------ prefill attention
 @pytest.mark.parametrize("L,H,G,top_k,seed", [(2048, 8, 2, 4, 0), (1024, 32, 8, 3, 21),
                                               (768, 16, 16, 2, 22), (512, 16, 1, 3, 23),
-                                              (512, 16, 8, 8, 24), (1024, 16, 2, 5, 25)])
+                                              (512, 16, 8, 8, 24), (1024, 16, 2, 5, 25),
+                                              (1000, 8, 2, 4, 26), (2049, 16, 4, 5, 27)])
 def test_prefill_attention_on_oracle_selection(L, H, G, top_k, seed):
     di = 64 if L == 2048 else 128
     shape = I.PrefillShape(B=2, L=L, H=H, G=G, d=128, d_idx=di, top_k=top_k)
@@ -156,6 +158,9 @@ def test_prefill_dense_limit_and_permuted_selection():
 @pytest.mark.parametrize("shape,seed,nrows", [
     (I.PREFILL_TINY, I.SEEDS["tiny"], None),
     (I.PrefillShape(B=1, L=8192, H=32, G=8, d=128, d_idx=128, top_k=16), 8, 40),
+    # lengths that are not a multiple of the block: a partial last block
+    (I.PrefillShape(B=1, L=1000, H=8, G=2, d=128, d_idx=64, top_k=4), 14, None),
+    (I.PrefillShape(B=1, L=2049, H=16, G=4, d=128, d_idx=128, top_k=5), 15, None),
 ])
 def test_forward_matches_oracle(shape, seed, nrows):
     x = _prefill(shape, seed)
