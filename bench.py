@@ -74,31 +74,33 @@ def load_peaks():
 
 
 # --------------------------------------------------------------------- work
-def n_sel(t: np.ndarray, top_k: int) -> np.ndarray:
+def n_sel(t: np.ndarray, top_k: int, block: int = BLOCK) -> np.ndarray:
     """Tokens a query at position t attends to (selected blocks, s <= t)."""
-    bt = t // BLOCK
-    return BLOCK * (np.minimum(top_k, bt + 1) - 1) + (t % BLOCK) + 1
+    bt = t // block
+    return block * (np.minimum(top_k, bt + 1) - 1) + (t % block) + 1
 
 
-def prefill_index_flops(B, L, G, d_idx, top_k):
-    nb = L // BLOCK
-    tiles = sum(range(top_k, nb)) if nb > top_k else 0
-    return B * G * 2.0 * d_idx * BLOCK * BLOCK * tiles
+def prefill_index_flops(B, L, G, d_idx, top_k, block=BLOCK):
+    """Index scores a prefill must compute: every row whose local block b_t
+    is at least top_k scores the b_t * block keys of its earlier blocks."""
+    bt = np.arange(L, dtype=np.int64) // block
+    keys = float(np.where(bt >= top_k, bt * block, 0).sum())
+    return B * G * 2.0 * d_idx * keys
 
 
-def prefill_main_flops(B, L, H, d, top_k):
+def prefill_main_flops(B, L, H, d, top_k, block=BLOCK):
     t = np.arange(L, dtype=np.int64)
-    return B * float(H) * 4.0 * d * float(n_sel(t, top_k).sum())
+    return B * float(H) * 4.0 * d * float(n_sel(t, top_k, block).sum())
 
 
-def prefill_attn_bytes(B, L, H, G, d, top_k):
+def prefill_attn_bytes(B, L, H, G, d, top_k, block=BLOCK):
     """Bytes the key-block-outer prefill attention must move: every selected
     (query, group, block) entry gathers its R = H/G q rows once and writes and
     reads back one bf16 partial row (+ fp32 lse) per head, and the merged
     output is written once.  K/V block reads (once per query chunk that
     selects the block) are not counted."""
     t = np.arange(L, dtype=np.int64)
-    entries = B * G * float(np.minimum(top_k, t // BLOCK + 1).sum())
+    entries = B * G * float(np.minimum(top_k, t // block + 1).sum())
     r = H // G
     return entries * r * (d * 2 * 3 + 4 * 2) + B * float(L) * H * d * 2
 
@@ -124,14 +126,14 @@ def prefill_bwd_flops(B, L, H, d, top_k):
     return B * float(H) * 10.0 * d * float(n_sel(t, top_k).sum())
 
 
-def decode_bytes(seq_lens, H, G, d, d_idx, top_k, fp8_index=False, fp8_kv=False):
+def decode_bytes(seq_lens, H, G, d, d_idx, top_k, fp8_index=False, fp8_kv=False, block=BLOCK):
     """Bytes a decode step must read: the index-key scan over every cached
     token (bf16, or E4M3 codes + one fp32 scale per token), the selected K/V
     tokens (bf16, or codes + one scale per token and head), and the small
     per-step tensors."""
     n = np.asarray(seq_lens, dtype=np.int64)
     t = n - 1
-    kv = G * 2 * ((d + 4) if fp8_kv else d * 2) * n_sel(t, top_k)
+    kv = G * 2 * ((d + 4) if fp8_kv else d * 2) * n_sel(t, top_k, block)
     scan = n * (d_idx + 4) if fp8_index else n * d_idx * 2
     small = len(n) * (H * d * 2 * 2 + G * d_idx * 2)
     return float((kv + scan).sum() + small)
@@ -533,7 +535,7 @@ def run_ours(args, shape, dshape, seed, cfg, ws_n, rank, local):
     roof_dec["frac"] = roof_dec["achieved"] / peaks["hbm_gbs"]
 
     nchunks = math.ceil(L / M.msa_prefill_chunk_len(p))
-    launches_per_step = 1 + 5 * nchunks + 4
+    launches_per_step = 1 + 5 * nchunks + 3   # index; per chunk 3 reverse-index + attention + merge; decode 3
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws_n,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -732,7 +734,7 @@ def bench_decode_128k(M, I, dev, args, peaks):
                                 "cache": "k_idx as E4M3 codes + fp32 scale per token"},
             "fp8_all_caches": {"us_per_step": us88, "roofline": roof(byts88, us88),
                                "cache": "k_idx, K and V as E4M3 codes + fp32 scales"},
-            "gpu_launches": 12 * iters, "oracle": oracle}
+            "gpu_launches": 9 * iters, "oracle": oracle}
 
 
 def bench_backward_32k(M, I, dev, args, peaks):
@@ -821,7 +823,8 @@ def bench_prefill_config(M, I, dev, args, peaks, name, shape, seed, needles=0,
     extrapolated to the whole prefill)."""
     x = I.prefill_inputs(shape, seed, device=dev, needles=needles, needle_alpha=3.0)
     B, L, H, G, d, di, K = shape.B, shape.L, shape.H, shape.G, shape.d, shape.d_idx, shape.top_k
-    p = M.make_params(B, L, H, G, d, di, BLOCK, K)
+    blk = shape.block
+    p = M.make_params(B, L, H, G, d, di, blk, K)
     ws_idx = M.new_workspace(p, M.MSA_OP_INDEX_SELECT, dev)
     ws_att = M.new_workspace(p, M.MSA_OP_PREFILL_ATTN, dev)
     sel = torch.empty((B, G, L, K), dtype=torch.int32, device=dev)
@@ -829,8 +832,8 @@ def bench_prefill_config(M, I, dev, args, peaks, name, shape, seed, needles=0,
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     for _ in range(max(3, args.warmup)):
-        M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx)
-        M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att)
+        M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx, block=blk)
+        M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att, block=blk)
     torch.cuda.synchronize()
     if M.msa_read_status(ws_idx) != 0 or M.msa_read_status(ws_att) != 0:
         raise SystemExit(f"{name}: device status error")
@@ -839,21 +842,21 @@ def bench_prefill_config(M, I, dev, args, peaks, name, shape, seed, needles=0,
         flush.zero_()   # L2 flush (256 MB > 126 MB L2) outside the timed span
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         ev[0].record(stream)
-        M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx)
+        M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx, block=blk)
         ev[1].record(stream)
-        M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att)
+        M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att, block=blk)
         ev[2].record(stream)
         torch.cuda.synchronize()
         t_idx.append(ev[0].elapsed_time(ev[1]))
         t_att.append(ev[1].elapsed_time(ev[2]))
         t_pre.append(ev[0].elapsed_time(ev[2]))
     idx_ms, att_ms, pre_ms = (statistics.median(v) for v in (t_idx, t_att, t_pre))
-    f_idx = prefill_index_flops(B, L, G, di, K)
-    f_main = prefill_main_flops(B, L, H, d, K)
-    b_att = prefill_attn_bytes(B, L, H, G, d, K)
+    f_idx = prefill_index_flops(B, L, G, di, K, blk)
+    f_main = prefill_main_flops(B, L, H, d, K, blk)
+    b_att = prefill_attn_bytes(B, L, H, G, d, K, blk)
     burst = peaks["bf16_tflops"]
-    nchunks = math.ceil(L / M.msa_prefill_chunk_len(p))
-    res = {"workload": f"B={B} L={L} H={H} G={G} d={d} d_idx={di} block={BLOCK} top_k={K}"
+    nchunks = math.ceil(B * L / M.msa_prefill_chunk_len(p))
+    res = {"workload": f"B={B} L={L} H={H} G={G} d={d} d_idx={di} block={blk} top_k={K}"
                        + (f", {needles} planted needle blocks per group (alpha 3)" if needles else ""),
            "seed": seed, "iters": iters, "l2": "256 MB buffer written between iterations",
            "prefill_ms": pre_ms, "tokens_per_s": B * L / (pre_ms / 1e3),
@@ -897,6 +900,79 @@ def bench_prefill_config(M, I, dev, args, peaks, name, shape, seed, needles=0,
     return res
 
 
+def bench_ragged_batch(M, I, dev, args, peaks):
+    """A serving batch of prompt chunks continuing cached prefixes: 16
+    sequences with caches of 131,072 tokens, each continuing at a seeded
+    position t0 with n new tokens (n uniform in [1, 16384], t0 uniform in
+    [0, Lmax - n]), every length unaligned.  msa_forward_cached_varlen runs
+    the batch with one launch per kernel; the same batch sequence by sequence
+    (msa_forward_cached, B = 1 each) is timed beside it."""
+    s = I.RAGGED_BATCH
+    rng = np.random.default_rng(I.SEEDS["ragged"])
+    n = rng.integers(1, s.n_hi + 1, size=s.B).tolist()
+    t0 = [int(rng.integers(0, s.Lmax - nb + 1)) for nb in n]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(I.SEEDS["ragged"])
+    N = int(sum(n))
+    mk = lambda shp: torch.randn(shp, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+    q, q_idx = mk((N, s.H, s.d)), mk((N, s.G, s.d_idx))
+    k, v, k_idx = mk((s.B, s.Lmax, s.G, s.d)), mk((s.B, s.Lmax, s.G, s.d)), mk((s.B, s.Lmax, s.d_idx))
+    out = torch.empty_like(q)
+    p = M.make_params(s.B, s.Lmax, s.H, s.G, s.d, s.d_idx, BLOCK, s.top_k)
+    ws = M.new_workspace(p, M.MSA_OP_FORWARD_VARLEN, dev)
+    p1 = M.make_params(1, s.Lmax, s.H, s.G, s.d, s.d_idx, BLOCK, s.top_k)
+    ws1 = M.new_workspace(p1, M.MSA_OP_FORWARD, dev)
+    rows0 = np.concatenate([[0], np.cumsum(n)]).tolist()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def one_launch():
+        M.msa_forward_cached_varlen(q, q_idx, k, v, k_idx, t0, n, s.top_k, out=out, ws=ws)
+
+    def per_sequence():
+        for b in range(s.B):
+            r0, r1 = rows0[b], rows0[b + 1]
+            M.msa_forward_cached(q[r0:r1].unsqueeze(0), q_idx[r0:r1].unsqueeze(0), k[b:b + 1],
+                                 v[b:b + 1], k_idx[b:b + 1], t0[b], s.top_k,
+                                 out=out[r0:r1].unsqueeze(0), ws=ws1)
+
+    def timed(fn, iters=5):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        torch.cuda.synchronize()
+        if M.msa_read_status(ws) != 0 or M.msa_read_status(ws1) != 0:
+            raise SystemExit("ragged batch: device status error")
+        ts = []
+        for _ in range(iters):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    ms = timed(one_launch)
+    ms_seq = timed(per_sequence)
+    f = 0.0
+    for b in range(s.B):
+        t = np.arange(t0[b], t0[b] + n[b], dtype=np.int64)
+        bt = t // BLOCK
+        f += s.G * 2.0 * s.d_idx * float(np.where(bt >= s.top_k, bt * BLOCK, 0).sum())
+        f += s.H * 4.0 * s.d * float(n_sel(t, s.top_k).sum())
+    del q, q_idx, k, v, k_idx, out, ws, ws1, flush
+    torch.cuda.empty_cache()
+    return {"workload": f"{s.B} sequences, caches of {s.Lmax}, n uniform in [1, {s.n_hi}], "
+                        f"H={s.H} G={s.G} d={s.d} d_idx={s.d_idx} block={BLOCK} top_k={s.top_k}",
+            "seed": I.SEEDS["ragged"], "new_tokens": N, "ms": ms,
+            "tokens_per_s": N / (ms / 1e3), "ms_sequence_by_sequence": ms_seq,
+            "one_launch_speedup": ms_seq / ms,
+            "tensor": {"flops": f, "tflops": f / (ms / 1e3) / 1e12,
+                       "frac_of_burst": f / (ms / 1e3) / 1e12 / peaks["bf16_tflops"]},
+            "l2": "256 MB buffer written between iterations"}
+
+
 def bench_configs(M, I, dev, args, peaks, line):
     """Every configuration at 1 GPU.  The 1M step and decode-128K were timed
     above; the tiny, 32K and 128K-planted prefills are timed here."""
@@ -908,6 +984,10 @@ def bench_configs(M, I, dev, args, peaks, line):
     cfgs["128k_planted"] = bench_prefill_config(M, I, dev, args, peaks, "128k_planted",
                                                 I.PREFILL_128K_PLANTED, I.SEEDS["128k_planted"],
                                                 needles=12, iters=5)
+    # the 64-token block variant at the same 2048-token budget (32 blocks)
+    cfgs["32k_block64"] = bench_prefill_config(M, I, dev, args, peaks, "32k_block64",
+                                               I.PREFILL_32K_BLOCK64, I.SEEDS["32k"], iters=10)
+    cfgs["ragged_batch"] = bench_ragged_batch(M, I, dev, args, peaks)
     if "decode_128k" in line:
         d = line["decode_128k"]
         cfgs["decode_128k"] = {"us_per_step": d["us_per_step"], "roofline": d["roofline"],

@@ -5,19 +5,24 @@
 // dominant stream is the k_idx cache scan (seq_len * d_idx * 2 bytes per
 // sequence).
 //
-//   decode_index_kernel   one warp per (sequence, key block j < b_t):
-//                         scores of the 128 keys against all G index
-//                         queries with mma.sync m16n8k16 (N = 8 groups),
-//                         then the per-group block max.  k_idx rows stream
-//                         straight from HBM in 16-byte loads.
+//   decode_index_kernel   one warp per (sequence, 128-key chunk before the
+//                         local block): scores of the keys against all G
+//                         index queries with mma.sync m16n8k16 (N = 8
+//                         groups), then the per-group block max (one block
+//                         per chunk, or two with 64-token blocks).  k_idx
+//                         rows stream straight from HBM in 16-byte loads.
 //   decode_topk_kernel    one CTA per (sequence, group): 16 warps scan
 //                         segments of the block scores, one warp merges.
 //   decode_attn_kernel    split over selected blocks: one CTA per
 //                         (sequence, group, slot) computes the block's
 //                         partial softmax for the R heads of the group on
-//                         the tensor cores (mma.sync, heads as M rows).
-//   decode_combine_kernel one warp per (sequence, head): merge <= top_k
-//                         partials.
+//                         the tensor cores (mma.sync, heads as M rows); the
+//                         last CTA of each (sequence, group) to finish, found
+//                         with an atomic ticket, merges the <= top_k
+//                         partials into the output.
+// The top-k and attention kernels are launched as programmatic dependents
+// of the kernel before them (their launch overlaps its tail) and wait for
+// its results with griddepcontrol.wait before reading them.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -49,25 +54,101 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// A warp scores one 128-key block against the (up to 8) index queries of
+// Programmatic dependent launch: wait until the grid this kernel depends on
+// has completed and its memory is visible (a no-op without the launch
+// attribute).
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Called by every CTA of decode_attn_kernel once its partial (or, for an
+// unused slot, its -inf lse) is written.  The last of the top_k CTAs of
+// (sequence b, group g) to get here merges the slot partials of the group's
+// R heads: o = sum_s exp(lse_s - M) o_s / sum_s exp(lse_s - M), M = max lse_s,
+// thread x taking column x of each head.  The ticket counters are zeroed by
+// decode_topk_kernel.
+template <int R>
+__device__ __forceinline__ void dec_merge_if_last(const DecodeArgs &a, int b, int g) {
+  __shared__ int s_last;
+  const int tid = threadIdx.x;
+  __threadfence();   // this CTA's partial, visible before its ticket
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(&a.tickets[b * a.G + g], 1) == a.top_k - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+#pragma unroll 1
+  for (int hh = 0; hh < R; ++hh) {
+    const size_t p0 = (size_t(b) * a.H + size_t(g) * R + hh) * a.top_k;
+    float M = -INFINITY;
+    for (int s = 0; s < a.top_k; ++s) M = fmaxf(M, __ldcg(a.part_lse + p0 + s));
+    float acc = 0.f, wsum = 0.f;
+    if (M > -INFINITY) {
+      for (int s = 0; s < a.top_k; ++s) {
+        const float ls = __ldcg(a.part_lse + p0 + s);
+        if (ls == -INFINITY) continue;
+        const float w = __expf(ls - M);
+        wsum += w;
+        acc = fmaf(w, __ldcg(a.part_o + (p0 + s) * kHeadDim + tid), acc);
+      }
+    }
+    const float o = wsum > 0.f ? acc * (1.f / wsum) : 0.f;
+    a.out[(size_t(b) * a.H + size_t(g) * R + hh) * kHeadDim + tid] =
+        __bfloat16_as_ushort(__float2bfloat16_rn(o));
+  }
+}
+
+// Reduce a warp's per-lane block maxima over the 8 lanes of each group pair
+// and store them: block jb0 of groups 2c, 2c+1 (lanes c < 4), and with
+// 64-token blocks also block jb0 + 1 unless it is the local block bt.
+template <int BLK>
+__device__ __forceinline__ void store_block_max(const DecodeArgs &a, int b, int jb0, int bt,
+                                                int lane, float mx0, float mx1, float my0,
+                                                float my1) {
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    if (BLK == 64) {
+      my0 = fmaxf(my0, __shfl_xor_sync(0xffffffffu, my0, o));
+      my1 = fmaxf(my1, __shfl_xor_sync(0xffffffffu, my1, o));
+    }
+  }
+  if (lane < 4) {
+    const int g0 = 2 * lane, g1 = 2 * lane + 1;
+    float *s0 = a.scores + (size_t(b) * a.G + g0) * a.nb_max;
+    float *s1 = a.scores + (size_t(b) * a.G + g1) * a.nb_max;
+    if (g0 < a.G) s0[jb0] = mx0;
+    if (g1 < a.G) s1[jb0] = mx1;
+    if (BLK == 64 && jb0 + 1 < bt) {
+      if (g0 < a.G) s0[jb0 + 1] = my0;
+      if (g1 < a.G) s1[jb0 + 1] = my1;
+    }
+  }
+}
+
+// A warp scores one 128-key chunk against the (up to 8) index queries of
 // its sequence.  The MMA's k dimension is a fixed permutation of d_idx
 // applied to both operands, chosen so that each lane reads whole 16-byte
 // granules of k_idx: for k-step kk = 2m + h, lane (g4 = lane/4, c = lane%4)
 // feeds d = 8(c + 4m) + 4h + {0,1} at k positions 2c, 2c+1 and
 // d = 8(c + 4m) + 4h + {2,3} at k positions 2c+8, 2c+9.
-template <int DI>
+template <int DI, int BLK>
 __global__ void __launch_bounds__(256) decode_index_kernel(const DecodeArgs a) {
   constexpr int NM = DI / 32;  // 16-byte granules per lane per key row
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
-  const int j = blockIdx.x * 8 + warp;
+  const int j = blockIdx.x * 8 + warp;   // 128-key chunk
   const int n = a.seq_lens[b];
   if (n < 1 || n > a.Lmax) {
     if (blockIdx.x == 0 && threadIdx.x == 0) atomicCAS(a.status, 0, kStatusBadInput);
     return;
   }
-  const int bt = (n - 1) / kBlock;
-  if (bt + 1 <= a.top_k || j >= bt) return;
+  const int bt = (n - 1) / BLK;          // local block
+  const int jb0 = (BLK == 128) ? j : 2 * j;   // first block of the chunk
+  if (bt + 1 <= a.top_k || jb0 >= bt) return;
+  // with 64-token blocks, the chunk's second half may be the local block
+  const int nrt = (BLK == 128 || jb0 + 1 < bt) ? 8 : 4;   // 16-key row tiles to score
   const int g4 = lane >> 2, c = lane & 3;
   // B fragments: q_idx[b, group g4, permuted d]
   uint32_t bf[NM][2][2];
@@ -83,10 +164,11 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const DecodeArgs a) {
         bf[m][h][1] = gv ? v.y : 0u;
       }
   }
-  const uint16_t *kbase = a.k_idx_cache + (size_t(b) * a.Lmax + size_t(j) * kBlock) * DI;
-  float mx0 = -FLT_MAX, mx1 = -FLT_MAX;
+  const uint16_t *kbase = a.k_idx_cache + (size_t(b) * a.Lmax + size_t(j) * 128) * DI;
+  float mx0 = -FLT_MAX, mx1 = -FLT_MAX;   // first block of the chunk, groups 2c, 2c+1
+  float my0 = -FLT_MAX, my1 = -FLT_MAX;   // second block (BLK 64)
 #pragma unroll 2
-  for (int rt = 0; rt < 8; ++rt) {
+  for (int rt = 0; rt < nrt; ++rt) {
     const uint16_t *r0 = kbase + size_t(rt * 16 + g4) * DI;
     const uint16_t *r1 = r0 + 8 * DI;
     uint4 lo[NM], hi[NM];
@@ -101,19 +183,15 @@ __global__ void __launch_bounds__(256) decode_index_kernel(const DecodeArgs a) {
       mma_bf16_16816(acc, lo[m].x, hi[m].x, lo[m].y, hi[m].y, bf[m][0][0], bf[m][0][1]);
       mma_bf16_16816(acc, lo[m].z, hi[m].z, lo[m].w, hi[m].w, bf[m][1][0], bf[m][1][1]);
     }
-    mx0 = fmaxf(mx0, fmaxf(acc[0], acc[2]));
-    mx1 = fmaxf(mx1, fmaxf(acc[1], acc[3]));
+    if (BLK == 128 || rt < 4) {
+      mx0 = fmaxf(mx0, fmaxf(acc[0], acc[2]));
+      mx1 = fmaxf(mx1, fmaxf(acc[1], acc[3]));
+    } else {
+      my0 = fmaxf(my0, fmaxf(acc[0], acc[2]));
+      my1 = fmaxf(my1, fmaxf(acc[1], acc[3]));
+    }
   }
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-  }
-  if (lane < 4) {
-    const int g0 = 2 * c, g1 = 2 * c + 1;
-    if (g0 < a.G) a.scores[(size_t(b) * a.G + g0) * a.nb_max + j] = mx0;
-    if (g1 < a.G) a.scores[(size_t(b) * a.G + g1) * a.nb_max + j] = mx1;
-  }
+  store_block_max<BLK>(a, b, jb0, bt, lane, mx0, mx1, my0, my1);
 }
 
 __device__ __forceinline__ void mma_f16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
@@ -148,20 +226,22 @@ __device__ __forceinline__ uint32_t f16x2_of(float lo, float hi) {
 // granules of 16 codes; k-step kk takes d = 16(c + 4(kk/4)) + 4(kk%4) +
 // {0,1} at k positions 2c, 2c+1 and + {2,3} at 2c+8, 2c+9, i.e. the bytes
 // of word kk%4 of granule kk/4.
-template <int DI>
+template <int DI, int BLK>
 __global__ void __launch_bounds__(256) decode_index_fp8_kernel(const DecodeArgs a) {
   constexpr int NG = DI / 64;  // granules per lane per key row
   constexpr int NK = DI / 16;  // MMA k-steps
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.y;
-  const int j = blockIdx.x * 8 + warp;
+  const int j = blockIdx.x * 8 + warp;   // 128-key chunk
   const int n = a.seq_lens[b];
   if (n < 1 || n > a.Lmax) {
     if (blockIdx.x == 0 && threadIdx.x == 0) atomicCAS(a.status, 0, kStatusBadInput);
     return;
   }
-  const int bt = (n - 1) / kBlock;
-  if (bt + 1 <= a.top_k || j >= bt) return;
+  const int bt = (n - 1) / BLK;
+  const int jb0 = (BLK == 128) ? j : 2 * j;
+  if (bt + 1 <= a.top_k || jb0 >= bt) return;
+  const int nrt = (BLK == 128 || jb0 + 1 < bt) ? 8 : 4;
   const int g4 = lane >> 2, c = lane & 3;
   uint32_t bq[NK][2];
   {
@@ -175,11 +255,11 @@ __global__ void __launch_bounds__(256) decode_index_fp8_kernel(const DecodeArgs 
       bq[kk][1] = gv ? f16x2_of(bf16_lo(v.y), bf16_hi(v.y)) : 0u;
     }
   }
-  const uint8_t *kbase = a.k_idx8 + (size_t(b) * a.Lmax + size_t(j) * kBlock) * DI;
-  const float *sbase = a.k_idx_scale + size_t(b) * a.Lmax + size_t(j) * kBlock;
-  float mx0 = -FLT_MAX, mx1 = -FLT_MAX;
+  const uint8_t *kbase = a.k_idx8 + (size_t(b) * a.Lmax + size_t(j) * 128) * DI;
+  const float *sbase = a.k_idx_scale + size_t(b) * a.Lmax + size_t(j) * 128;
+  float mx0 = -FLT_MAX, mx1 = -FLT_MAX, my0 = -FLT_MAX, my1 = -FLT_MAX;
 #pragma unroll 2
-  for (int rt = 0; rt < 8; ++rt) {
+  for (int rt = 0; rt < nrt; ++rt) {
     const uint8_t *r0 = kbase + size_t(rt * 16 + g4) * DI;
     const uint8_t *r1 = r0 + 8 * DI;
     uint4 lo[NG], hi[NG];
@@ -200,19 +280,15 @@ __global__ void __launch_bounds__(256) decode_index_fp8_kernel(const DecodeArgs 
                       e4m3x2_to_f16x2(wl[w] >> 16), e4m3x2_to_f16x2(wh[w] >> 16),
                       bq[4 * gi + w][0], bq[4 * gi + w][1]);
     }
-    mx0 = fmaxf(mx0, fmaxf(acc[0] * s0, acc[2] * s1));
-    mx1 = fmaxf(mx1, fmaxf(acc[1] * s0, acc[3] * s1));
+    if (BLK == 128 || rt < 4) {
+      mx0 = fmaxf(mx0, fmaxf(acc[0] * s0, acc[2] * s1));
+      mx1 = fmaxf(mx1, fmaxf(acc[1] * s0, acc[3] * s1));
+    } else {
+      my0 = fmaxf(my0, fmaxf(acc[0] * s0, acc[2] * s1));
+      my1 = fmaxf(my1, fmaxf(acc[1] * s0, acc[3] * s1));
+    }
   }
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-  }
-  if (lane < 4) {
-    const int g0 = 2 * c, g1 = 2 * c + 1;
-    if (g0 < a.G) a.scores[(size_t(b) * a.G + g0) * a.nb_max + j] = mx0;
-    if (g1 < a.G) a.scores[(size_t(b) * a.G + g1) * a.nb_max + j] = mx1;
-  }
+  store_block_max<BLK>(a, b, jb0, bt, lane, mx0, mx1, my0, my1);
 }
 
 // One CTA per (sequence, group): 16 warps each keep the top_k-1 of a
@@ -227,13 +303,15 @@ __global__ void __launch_bounds__(kTopkWarps * 32) decode_topk_kernel(const Deco
   const int row = blockIdx.x;  // b * G + g
   const int b = row / a.G;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  griddep_wait();                              // the scan's block scores
+  if (threadIdx.x == 0) a.tickets[row] = 0;    // the attention's merge ticket
   const int n = a.seq_lens[b];
   int32_t *out = a.sel + size_t(row) * a.top_k;
   if (n < 1 || n > a.Lmax) {
     if (warp == 0 && lane < a.top_k) out[lane] = -1;
     return;
   }
-  const int bt = (n - 1) / kBlock;
+  const int bt = (n - 1) / a.blk;
   if (bt + 1 <= a.top_k) {
     if (warp == 0)
       for (int k = lane; k < a.top_k; k += 32) out[k] = (k <= bt) ? k : -1;
@@ -290,12 +368,17 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
 //     (rows padded to 272 B) and read with ldmatrix.trans.  The 4 warps'
 //     partial O are summed through shared memory.
 constexpr int kVPitch = kHeadDim + 8;  // bf16 per staged V row (272 B: conflict-free ldmatrix)
-template <int R>
+template <int R, int BLK>
+constexpr int dec_attn_area() {
+  // staged V; the 4 warps' partial O reuse the area once every warp has
+  // read V (with 128-token blocks the V rows are the larger of the two)
+  return (BLK * kVPitch * 2 > 4 * R * kHeadDim * 4) ? BLK * kVPitch * 2 : 4 * R * kHeadDim * 4;
+}
+template <int R, int BLK>
 constexpr int dec_attn_smem() {
-  // staged V, then the row max / sum exchange; the 4 warps' partial O reuse
-  // the V area once every warp has read V (6 CTAs fit on an SM)
-  static_assert(4 * R * kHeadDim * 4 <= kBlock * kVPitch * 2, "partial O must fit the V area");
-  return kBlock * kVPitch * 2 + 2 * 4 * 16 * 4;
+  // the V / partial-O area, then the row max / sum exchange (6 CTAs fit on
+  // an SM with 128-token blocks)
+  return dec_attn_area<R, BLK>() + 2 * 4 * 16 * 4;
 }
 
 __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
@@ -304,32 +387,36 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t add
                : "r"(addr));
 }
 
-template <int R>
+template <int R, int BLK>
 __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
+  constexpr int KW = BLK / 4;   // keys per warp
+  constexpr int NT = KW / 8;    // 8-key n-tiles per warp
   extern __shared__ __align__(16) uint8_t dsm[];
   uint16_t *sV = reinterpret_cast<uint16_t *>(dsm);
   float *s_o = reinterpret_cast<float *>(dsm);                     // [4 warps][R rows][128], over V
-  float *s_m = reinterpret_cast<float *>(sV + kBlock * kVPitch);   // [4][16]
+  float *s_m = reinterpret_cast<float *>(dsm + dec_attn_area<R, BLK>());   // [4][16]
   float *s_l = s_m + 4 * 16;                                        // [4][16]
   const int slot = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g4 = lane >> 2, c = lane & 3;
+  griddep_wait();   // the top-k's selection
   const int n = a.seq_lens[b];
   const int j = (n >= 1 && n <= a.Lmax) ? a.sel[(size_t(b) * a.G + g) * a.top_k + slot] : -1;
   const size_t prow0 = (size_t(b) * a.H + size_t(g) * R) * a.top_k + slot;
-  if (j < 0) {
+  if (j < 0) {   // an unused slot: an empty partial
     if (tid < R) a.part_lse[prow0 + size_t(tid) * a.top_k] = -INFINITY;
+    dec_merge_if_last<R>(a, b, g);
     return;
   }
   const int t = n - 1;
-  const int nvis = min(kBlock, t - j * kBlock + 1);
+  const int nvis = min(BLK, t - j * BLK + 1);
   const size_t row_stride = size_t(a.G) * kHeadDim;
-  const uint16_t *kb = a.k_cache + ((size_t(b) * a.Lmax + size_t(j) * kBlock) * a.G + g) * kHeadDim;
-  const uint16_t *vb = a.v_cache + ((size_t(b) * a.Lmax + size_t(j) * kBlock) * a.G + g) * kHeadDim;
+  const uint16_t *kb = a.k_cache + ((size_t(b) * a.Lmax + size_t(j) * BLK) * a.G + g) * kHeadDim;
+  const uint16_t *vb = a.v_cache + ((size_t(b) * a.Lmax + size_t(j) * BLK) * a.G + g) * kHeadDim;
   // V block -> shared memory (coalesced 16-byte cp.async), overlapping S
   const uint32_t sV_u = static_cast<uint32_t>(__cvta_generic_to_shared(sV));
 #pragma unroll 4
-  for (int it = 0; it < 16; ++it) {
+  for (int it = 0; it < BLK / 8; ++it) {
     const int idx = it * 128 + tid, row = idx >> 4, gran = idx & 15;
     const uint32_t dst = sV_u + (row * kVPitch + gran * 8) * 2;
     if (row < nvis)
@@ -338,11 +425,11 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
       asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(dst), "r"(0) : "memory");
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
-  // K granules for this warp's four 8-key n-tiles (key row 8*nt + g4)
-  uint4 kg[4][4];
+  // K granules for this warp's NT 8-key n-tiles (key row 8*nt + g4)
+  uint4 kg[NT][4];
 #pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
-    const int key = warp * 32 + q4 * 8 + g4;
+  for (int q4 = 0; q4 < NT; ++q4) {
+    const int key = warp * KW + q4 * 8 + g4;
     const uint16_t *kr = kb + size_t(min(key, nvis - 1)) * row_stride;
 #pragma unroll
     for (int m = 0; m < 4; ++m) kg[q4][m] = ldg_nc_v4(kr + 8 * (c + 4 * m));
@@ -364,9 +451,9 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
       }
   }
   // S tiles: acc[q4] = rows (g4, g4+8) x keys (8*nt + 2c, +1)
-  float sacc[4][4];
+  float sacc[NT][4];
 #pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
+  for (int q4 = 0; q4 < NT; ++q4) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) sacc[q4][e] = 0.f;
 #pragma unroll
@@ -380,8 +467,8 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
   // mask keys past the query, row max over the block
   float mx0 = -FLT_MAX, mx1 = -FLT_MAX;
 #pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
-    const int k0 = warp * 32 + q4 * 8 + 2 * c;
+  for (int q4 = 0; q4 < NT; ++q4) {
+    const int k0 = warp * KW + q4 * 8 + 2 * c;
     if (k0 >= nvis) { sacc[q4][0] = -FLT_MAX; sacc[q4][2] = -FLT_MAX; }
     if (k0 + 1 >= nvis) { sacc[q4][1] = -FLT_MAX; sacc[q4][3] = -FLT_MAX; }
     mx0 = fmaxf(mx0, fmaxf(sacc[q4][0], sacc[q4][1]));
@@ -397,10 +484,10 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
   const float m0 = fmaxf(fmaxf(s_m[g4], s_m[16 + g4]), fmaxf(s_m[32 + g4], s_m[48 + g4]));
   const float m1 = fmaxf(fmaxf(s_m[8 + g4], s_m[24 + g4]), fmaxf(s_m[40 + g4], s_m[56 + g4]));
   // P = exp(scale (S - m)), packed straight into A fragments
-  uint32_t pa[2][4];
+  uint32_t pa[NT / 2][4];
   float l0 = 0.f, l1 = 0.f;
 #pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
+  for (int q4 = 0; q4 < NT; ++q4) {
     const float p0 = exp2f((sacc[q4][0] - m0) * a.scale_log2);
     const float p1 = exp2f((sacc[q4][1] - m0) * a.scale_log2);
     const float p2 = exp2f((sacc[q4][2] - m1) * a.scale_log2);
@@ -426,8 +513,8 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) oacc[dt][e] = 0.f;
 #pragma unroll
-  for (int kt = 0; kt < 2; ++kt) {
-    const int key0 = warp * 32 + kt * 16;
+  for (int kt = 0; kt < NT / 2; ++kt) {
+    const int key0 = warp * KW + kt * 16;
 #pragma unroll
     for (int dt = 0; dt < 16; dt += 2) {
       // matrices: (keys 0-7, dt), (keys 8-15, dt), (keys 0-7, dt+1), (keys 8-15, dt+1)
@@ -469,6 +556,7 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
     const float l = s_l[h] + s_l[16 + h] + s_l[32 + h] + s_l[48 + h];
     a.part_lse[prow0 + size_t(h) * a.top_k] = mh * a.scale + __logf(l);
   }
+  dec_merge_if_last<R>(a, b, g);
 }
 
 // decode_attn_kernel for FP8 K/V caches: the stored key / value of token s
@@ -480,55 +568,60 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const DecodeArgs a) {
 //   V codes are converted (exactly) to bf16 on their way into shared memory,
 //     and each key's V scale is folded into P before P is packed to bf16, so
 //     the P V MMA is the bf16 one; the row sum uses the unscaled P.
-template <int R>
+template <int R, int BLK>
 __global__ void __launch_bounds__(128) decode_attn_fp8_kernel(const DecodeArgs a) {
+  constexpr int KW = BLK / 4;   // keys per warp
+  constexpr int NT = KW / 8;    // 8-key n-tiles per warp
+  constexpr int NV = BLK / 16;  // 16-code V granules per thread
   extern __shared__ __align__(16) uint8_t dsm[];
   uint16_t *sV = reinterpret_cast<uint16_t *>(dsm);
   float *s_o = reinterpret_cast<float *>(dsm);                     // [4 warps][R rows][128], over V
-  float *s_m = reinterpret_cast<float *>(sV + kBlock * kVPitch);   // [4][16]
+  float *s_m = reinterpret_cast<float *>(dsm + dec_attn_area<R, BLK>());   // [4][16]
   float *s_l = s_m + 4 * 16;                                        // [4][16]
   const int slot = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g4 = lane >> 2, c = lane & 3;
+  griddep_wait();   // the top-k's selection
   const int n = a.seq_lens[b];
   const int j = (n >= 1 && n <= a.Lmax) ? a.sel[(size_t(b) * a.G + g) * a.top_k + slot] : -1;
   const size_t prow0 = (size_t(b) * a.H + size_t(g) * R) * a.top_k + slot;
-  if (j < 0) {
+  if (j < 0) {   // an unused slot: an empty partial
     if (tid < R) a.part_lse[prow0 + size_t(tid) * a.top_k] = -INFINITY;
+    dec_merge_if_last<R>(a, b, g);
     return;
   }
   const int t = n - 1;
-  const int nvis = min(kBlock, t - j * kBlock + 1);
-  const size_t tok0 = size_t(b) * a.Lmax + size_t(j) * kBlock;   // first token of the block
+  const int nvis = min(BLK, t - j * BLK + 1);
+  const size_t tok0 = size_t(b) * a.Lmax + size_t(j) * BLK;   // first token of the block
   const size_t row_stride = size_t(a.G) * kHeadDim;                // codes between tokens
   const uint8_t *kb = a.k8 + (tok0 * a.G + g) * kHeadDim;
   const uint8_t *vb = a.v8 + (tok0 * a.G + g) * kHeadDim;
   const float *ksb = a.k_scale + tok0 * a.G + g;                   // stride G per token
   const float *vsb = a.v_scale + tok0 * a.G + g;
-  // V codes: 1024 granules of 16, 8 per thread, loaded now and converted
-  // into shared memory after S
-  uint4 vg[8];
+  // V codes: BLK * 8 granules of 16, NV per thread, loaded now and
+  // converted into shared memory after S
+  uint4 vg[NV];
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
+  for (int it = 0; it < NV; ++it) {
     const int idx = it * 128 + tid, row = idx >> 3, gran = idx & 7;
     vg[it] = (row < nvis) ? ldg_nc_v4(vb + row * row_stride + gran * 16) : make_uint4(0, 0, 0, 0);
   }
-  // K granules for this warp's four 8-key n-tiles (key row 8*nt + g4)
-  uint4 kg[4][2];
+  // K granules for this warp's NT 8-key n-tiles (key row 8*nt + g4)
+  uint4 kg[NT][2];
 #pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
-    const int key = warp * 32 + q4 * 8 + g4;
+  for (int q4 = 0; q4 < NT; ++q4) {
+    const int key = warp * KW + q4 * 8 + g4;
     const uint8_t *kr = kb + size_t(min(key, nvis - 1)) * row_stride;
 #pragma unroll
     for (int gi = 0; gi < 2; ++gi) kg[q4][gi] = ldg_nc_v4(kr + 16 * (c + 4 * gi));
   }
   // scales of the keys whose S columns this lane holds: 8*nt + 2c, +1
-  float ksc[4][2], vsc[4][2];
+  float ksc[NT][2], vsc[NT][2];
 #pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4)
+  for (int q4 = 0; q4 < NT; ++q4)
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const int key = min(warp * 32 + q4 * 8 + 2 * c + e, nvis - 1);
+      const int key = min(warp * KW + q4 * 8 + 2 * c + e, nvis - 1);
       ksc[q4][e] = __ldg(ksb + size_t(key) * a.G);
       vsc[q4][e] = __ldg(vsb + size_t(key) * a.G);
     }
@@ -549,9 +642,9 @@ __global__ void __launch_bounds__(128) decode_attn_fp8_kernel(const DecodeArgs a
       qb[kk][1] = f16x2_of(bf16_lo(v1.y), bf16_hi(v1.y));
     }
   }
-  float sacc[4][4];
+  float sacc[NT][4];
 #pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
+  for (int q4 = 0; q4 < NT; ++q4) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) sacc[q4][e] = 0.f;
 #pragma unroll
@@ -569,7 +662,7 @@ __global__ void __launch_bounds__(128) decode_attn_fp8_kernel(const DecodeArgs a
   }
   // V codes -> bf16 rows in shared memory (rows past the query are zero)
 #pragma unroll
-  for (int it = 0; it < 8; ++it) {
+  for (int it = 0; it < NV; ++it) {
     const int idx = it * 128 + tid, row = idx >> 3, gran = idx & 7;
     const uint32_t wv[4] = {vg[it].x, vg[it].y, vg[it].z, vg[it].w};
     uint32_t o[8];
@@ -589,8 +682,8 @@ __global__ void __launch_bounds__(128) decode_attn_fp8_kernel(const DecodeArgs a
   // mask keys past the query, row max over the block
   float mx0 = -FLT_MAX, mx1 = -FLT_MAX;
 #pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
-    const int k0 = warp * 32 + q4 * 8 + 2 * c;
+  for (int q4 = 0; q4 < NT; ++q4) {
+    const int k0 = warp * KW + q4 * 8 + 2 * c;
     if (k0 >= nvis) { sacc[q4][0] = -FLT_MAX; sacc[q4][2] = -FLT_MAX; }
     if (k0 + 1 >= nvis) { sacc[q4][1] = -FLT_MAX; sacc[q4][3] = -FLT_MAX; }
     mx0 = fmaxf(mx0, fmaxf(sacc[q4][0], sacc[q4][1]));
@@ -606,10 +699,10 @@ __global__ void __launch_bounds__(128) decode_attn_fp8_kernel(const DecodeArgs a
   const float m0 = fmaxf(fmaxf(s_m[g4], s_m[16 + g4]), fmaxf(s_m[32 + g4], s_m[48 + g4]));
   const float m1 = fmaxf(fmaxf(s_m[8 + g4], s_m[24 + g4]), fmaxf(s_m[40 + g4], s_m[56 + g4]));
   // P = exp(scale (S - m)); the A fragments carry P * (V scale of the key)
-  uint32_t pa[2][4];
+  uint32_t pa[NT / 2][4];
   float l0 = 0.f, l1 = 0.f;
 #pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) {
+  for (int q4 = 0; q4 < NT; ++q4) {
     const float p0 = exp2f((sacc[q4][0] - m0) * a.scale_log2);
     const float p1 = exp2f((sacc[q4][1] - m0) * a.scale_log2);
     const float p2 = exp2f((sacc[q4][2] - m1) * a.scale_log2);
@@ -633,8 +726,8 @@ __global__ void __launch_bounds__(128) decode_attn_fp8_kernel(const DecodeArgs a
 #pragma unroll
     for (int e = 0; e < 4; ++e) oacc[dt][e] = 0.f;
 #pragma unroll
-  for (int kt = 0; kt < 2; ++kt) {
-    const int key0 = warp * 32 + kt * 16;
+  for (int kt = 0; kt < NT / 2; ++kt) {
+    const int key0 = warp * KW + kt * 16;
 #pragma unroll
     for (int dt = 0; dt < 16; dt += 2) {
       const int mi = lane >> 3, r = lane & 7;
@@ -673,48 +766,63 @@ __global__ void __launch_bounds__(128) decode_attn_fp8_kernel(const DecodeArgs a
     const float l = s_l[h] + s_l[16 + h] + s_l[32 + h] + s_l[48 + h];
     a.part_lse[prow0 + size_t(h) * a.top_k] = mh * a.scale + __logf(l);
   }
+  dec_merge_if_last<R>(a, b, g);
 }
 
-__global__ void __launch_bounds__(256) decode_combine_kernel(const DecodeArgs a) {
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);  // b*H + h
-  const int lane = threadIdx.x & 31;
-  if (row >= a.B * a.H) return;
-  const size_t p0 = size_t(row) * a.top_k;
-  const float my = lane < a.top_k ? a.part_lse[p0 + lane] : -INFINITY;
-  float M = my;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  float wsum = 0.f;
-  if (M > -INFINITY) {
-    const float wm = (my > -INFINITY) ? __expf(my - M) : 0.f;
-    wsum = wm;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
-    for (int s = 0; s < a.top_k; ++s) {
-      const float ws = __shfl_sync(0xffffffffu, wm, s);
-      if (ws == 0.f) continue;
-      const float4 v = *reinterpret_cast<const float4 *>(a.part_o + (p0 + s) * kHeadDim + lane * 4);
-      acc[0] = fmaf(ws, v.x, acc[0]);
-      acc[1] = fmaf(ws, v.y, acc[1]);
-      acc[2] = fmaf(ws, v.z, acc[2]);
-      acc[3] = fmaf(ws, v.w, acc[3]);
-    }
-  }
-  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  uint2 r;
-  r.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-  r.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-  *reinterpret_cast<uint2 *>(a.out + size_t(row) * kHeadDim + lane * 4) = r;
+// Launch as a programmatic dependent of the previous kernel in the stream.
+template <typename Kern>
+cudaError_t launch_dependent(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             const DecodeArgs &a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int R>
+template <int R, int BLK>
 cudaError_t launch_decode_attn(const DecodeArgs &a, cudaStream_t st) {
-  constexpr int smem = dec_attn_smem<R>();
-  auto kern = a.k8 ? decode_attn_fp8_kernel<R> : decode_attn_kernel<R>;
+  constexpr int smem = dec_attn_smem<R, BLK>();
+  auto kern = a.k8 ? decode_attn_fp8_kernel<R, BLK> : decode_attn_kernel<R, BLK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  kern<<<dim3(a.top_k, a.G, a.B), 128, smem, st>>>(a);
+  return launch_dependent(kern, dim3(a.top_k, a.G, a.B), dim3(128), smem, st, a);
+}
+
+template <int BLK>
+cudaError_t launch_decode_b(const DecodeArgs &a, cudaStream_t st) {
+  // the scan: one warp per 128-key chunk, 8 chunks per CTA
+  const int chunks = (a.Lmax + 127) / 128;
+  const dim3 gi((chunks + 7) / 8, a.B);
+  if (a.k_idx8) {
+    if (a.d_idx == 64)
+      decode_index_fp8_kernel<64, BLK><<<gi, 256, 0, st>>>(a);
+    else
+      decode_index_fp8_kernel<128, BLK><<<gi, 256, 0, st>>>(a);
+  } else if (a.d_idx == 64) {
+    decode_index_kernel<64, BLK><<<gi, 256, 0, st>>>(a);
+  } else {
+    decode_index_kernel<128, BLK><<<gi, 256, 0, st>>>(a);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_dependent(decode_topk_kernel, dim3(a.B * a.G), dim3(kTopkWarps * 32), 0, st, a);
+  if (e != cudaSuccess) return e;
+  switch (a.H / a.G) {
+    case 1: e = launch_decode_attn<1, BLK>(a, st); break;
+    case 2: e = launch_decode_attn<2, BLK>(a, st); break;
+    case 4: e = launch_decode_attn<4, BLK>(a, st); break;
+    case 8: e = launch_decode_attn<8, BLK>(a, st); break;
+    case 16: e = launch_decode_attn<16, BLK>(a, st); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -722,30 +830,7 @@ cudaError_t launch_decode_attn(const DecodeArgs &a, cudaStream_t st) {
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st) {
   if (a.B == 0) return cudaSuccess;
-  const dim3 gi((a.nb_max + 7) / 8, a.B);
-  if (a.k_idx8) {
-    if (a.d_idx == 64)
-      decode_index_fp8_kernel<64><<<gi, 256, 0, st>>>(a);
-    else
-      decode_index_fp8_kernel<128><<<gi, 256, 0, st>>>(a);
-  } else if (a.d_idx == 64) {
-    decode_index_kernel<64><<<gi, 256, 0, st>>>(a);
-  } else {
-    decode_index_kernel<128><<<gi, 256, 0, st>>>(a);
-  }
-  decode_topk_kernel<<<a.B * a.G, kTopkWarps * 32, 0, st>>>(a);
-  cudaError_t e;
-  switch (a.H / a.G) {
-    case 1: e = launch_decode_attn<1>(a, st); break;
-    case 2: e = launch_decode_attn<2>(a, st); break;
-    case 4: e = launch_decode_attn<4>(a, st); break;
-    case 8: e = launch_decode_attn<8>(a, st); break;
-    case 16: e = launch_decode_attn<16>(a, st); break;
-    default: return cudaErrorInvalidValue;
-  }
-  if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<(a.B * a.H + 7) / 8, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  return a.blk == 64 ? launch_decode_b<64>(a, st) : launch_decode_b<128>(a, st);
 }
 
 }  // namespace msa

@@ -10,7 +10,10 @@
 //
 // Causality needs no element mask: the local block b_t is always selected,
 // so only blocks j < b_t are scored, and every such block is entirely
-// visible.  For a 128-query tile i the work is the tile row j = 0..i-1.
+// visible.  For a 128-query tile i the work is the tile row of 128-key
+// chunks j = 0..i-1.  With 64-token blocks (BLK = 64) a chunk holds two
+// blocks, pooled separately, and the tile's second half (rows 64..127, local
+// block 2i+1) also scores block 2i, the first half of chunk i.
 //
 // Kernel structure (persistent, one CTA per SM, 12 warps = 3 warpgroups):
 //   warp 0    TMA producer: the tile's q_idx rows for GP groups (resident),
@@ -83,6 +86,7 @@ struct IndexWork {
   int i, b, gp, stages;
 };
 
+template <int BLK>
 __device__ __forceinline__ IndexWork index_work(const IndexArgs &a, int u, int GPn) {
   const int ngp = a.G / GPn;
   IndexWork w;
@@ -97,8 +101,11 @@ __device__ __forceinline__ IndexWork index_work(const IndexArgs &a, int u, int G
     w.b = rem / ngp;
     w.gp = rem % ngp;
   }
-  const bool need = a.write_scores ? (w.i >= 1) : (w.i >= a.top_k && a.top_k >= 2);
-  w.stages = need ? (w.i + 1) / 2 : 0;
+  // largest local block among the tile's rows; chunks 0..i-1 (BLK 128) or
+  // 0..i (BLK 64) hold every block a row of the tile may score
+  const int max_bt = (BLK == 128) ? w.i : 2 * w.i + 1;
+  const bool need = a.write_scores ? (max_bt >= 1) : (max_bt >= a.top_k && a.top_k >= 2);
+  w.stages = need ? ((BLK == 128) ? (w.i + 1) / 2 : w.i / 2 + 1) : 0;
   return w;
 }
 
@@ -179,6 +186,17 @@ __device__ __forceinline__ void sort_ids_asc(int (&v)[KCAP]) {
   }
 }
 
+// Max over 2 x 32 fp32 values (two independent chains).
+__device__ __forceinline__ float max2x32(const float (&a)[32], const float (&b)[32]) {
+  float m0 = max3f(a[0], a[1], a[2]), m1 = max3f(b[0], b[1], b[2]);
+#pragma unroll
+  for (int x = 3; x + 2 <= 31; x += 2) {
+    m0 = max3f(m0, a[x], a[x + 1]);
+    m1 = max3f(m1, b[x], b[x + 1]);
+  }
+  return fmaxf(fmaxf(m0, a[31]), fmaxf(m1, b[31]));
+}
+
 // Max over 4 x 32 fp32 values with three-input max (4 independent chains).
 __device__ __forceinline__ float max4x32(const float (&a)[32], const float (&b)[32],
                                          const float (&c)[32], const float (&d)[32]) {
@@ -198,7 +216,20 @@ __device__ __forceinline__ float max4x32(const float (&a)[32], const float (&b)[
   return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
 }
 
-template <int DI, int GP, int KCAP>
+// One block score of a row: stored (SCORES mode) or offered to the row's
+// running list (FUSED mode; ids arrive in increasing order within a set).
+template <int KCAP>
+__device__ __forceinline__ void put_score(const IndexArgs &a, const int4 &sq, int g, int t,
+                                          float (&ls)[KCAP], int (&lj)[KCAP], float sc, int jb) {
+  if (a.write_scores) {
+    const long long orow = index_out_row(a, sq, g, t);
+    if (orow >= 0) a.scores[orow * a.nb + jb] = sc;
+  } else if (sc > ls[KCAP - 1]) {
+    list_insert_tail<KCAP>(ls, lj, sc, jb);
+  }
+}
+
+template <int DI, int GP, int KCAP, int BLK>
 __global__ void __launch_bounds__(384, 1)
     msa_index_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k, const IndexArgs a) {
@@ -259,7 +290,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int r = 0;; ++r) {
         const int u = index_item(r, a.n_items);
         if (u < 0) break;
-        const IndexWork w = index_work(a, u, GP);
+        const IndexWork w = index_work<BLK>(a, u, GP);
         if (w.stages == 0) continue;
         if (!mbar_wait(b_qempty, qph ^ 1, abort_flag, a.status)) break;
         qph ^= 1;
@@ -270,16 +301,16 @@ __global__ void __launch_bounds__(384, 1)
         for (int gi = 0; gi < GP; ++gi)
           for (int c = 0; c < C::NCH; ++c)
             tma_load_3d(s_q + (gi * C::NCH + c) * 16384, &tm_q, b_qfull, c * 64, w.gp * GP + gi,
-                        sq.x + w.i * kBlock - sq.y);
+                        sq.x + w.i * 128 - sq.y);
         bool ok = true;
         for (int s = 0; s < w.stages; ++s) {
           if (!mbar_wait(b_kempty + 8 * kst, kph ^ 1, abort_flag, a.status)) { ok = false; break; }
           mbar_arrive_expect_tx(b_kfull + 8 * kst, C::STAGE_BYTES);
           const uint32_t dst = s_k + kst * C::STAGE_BYTES;
-          const int row0 = w.b * a.L + (2 * s) * kBlock;
+          const int row0 = w.b * a.L + (2 * s) * 128;   // 128-key chunks 2s, 2s+1
           for (int c = 0; c < C::NCH; ++c) {
             tma_load_2d(dst + c * 32768, &tm_k, b_kfull + 8 * kst, c * 64, row0);
-            tma_load_2d(dst + c * 32768 + 16384, &tm_k, b_kfull + 8 * kst, c * 64, row0 + kBlock);
+            tma_load_2d(dst + c * 32768 + 16384, &tm_k, b_kfull + 8 * kst, c * 64, row0 + 128);
           }
           if (++kst == C::NS) { kst = 0; kph ^= 1; }
         }
@@ -296,7 +327,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int r = 0;; ++r) {
         const int u = index_item(r, a.n_items);
         if (u < 0) break;
-        const IndexWork w = index_work(a, u, GP);
+        const IndexWork w = index_work<BLK>(a, u, GP);
         if (w.stages == 0) continue;
         if (!mbar_wait(b_qfull, qph, abort_flag, a.status)) break;
         qph ^= 1;
@@ -352,8 +383,9 @@ __global__ void __launch_bounds__(384, 1)
     for (int r = 0; ok; ++r) {
       const int u = index_item(r, a.n_items);
       if (u < 0) break;
-      const IndexWork w = index_work(a, u, GP);
-      const int t = w.i * kBlock + row;
+      const IndexWork w = index_work<BLK>(a, u, GP);
+      const int t = w.i * 128 + row;   // query tiles hold 128 queries whatever the block
+      const int bt = t / BLK;          // this row's local block
       const int4 sq = qgeo_seq(a.q, w.b);
       float ls[GP][KCAP];
       int lj[GP][KCAP];
@@ -374,9 +406,11 @@ __global__ void __launch_bounds__(384, 1)
             break;
           }
           tc_fence_after();
-          const int j = 2 * s + eset;
+          const int j = 2 * s + eset;   // 128-key chunk
+          // warp-uniform: a warp's rows are all below or all above 64
+          const bool use = (BLK == 128) ? (j < w.i) : (j < w.i || (j == w.i && row >= 64));
           float v0[32], v1[32], v2[32], v3[32];
-          if (j < w.i) {
+          if (use) {
             const uint32_t ta = lane_base + slot * 256 + eset * 128;
             tmem_ld32(ta, v0);
             tmem_ld32(ta + 32, v1);
@@ -389,13 +423,16 @@ __global__ void __launch_bounds__(384, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(b_accempty + 8 * slot);
           ++jc;
-          if (j < w.i) {
-            const float sc = max4x32(v0, v1, v2, v3);
-            if (a.write_scores) {
-              const long long orow = index_out_row(a, sq, w.gp * GP + gi, t);
-              if (orow >= 0) a.scores[orow * a.nb + j] = sc;
-            } else if (sc > ls[gi][KCAP - 1]) {
-              list_insert_tail<KCAP>(ls[gi], lj[gi], sc, j);
+          if (use) {
+            if (BLK == 128) {
+              put_score<KCAP>(a, sq, w.gp * GP + gi, t, ls[gi], lj[gi], max4x32(v0, v1, v2, v3), j);
+            } else {
+              // blocks 2j (columns 0..63) and 2j+1 (64..127); block 2i+1 is
+              // a local block, never scored
+              put_score<KCAP>(a, sq, w.gp * GP + gi, t, ls[gi], lj[gi], max2x32(v0, v1), 2 * j);
+              if (j < w.i)
+                put_score<KCAP>(a, sq, w.gp * GP + gi, t, ls[gi], lj[gi], max2x32(v2, v3),
+                                2 * j + 1);
             }
           }
         }
@@ -411,12 +448,12 @@ __global__ void __launch_bounds__(384, 1)
             const long long orow = index_out_row(a, sq, w.gp * GP + gi, t);
             if (orow < 0) continue;
             float *dst = a.scores + orow * a.nb;
-            for (int j = w.i; j < a.nb; ++j) dst[j] = -INFINITY;
+            for (int j = bt; j < a.nb; ++j) dst[j] = -INFINITY;
           }
         }
         continue;
       }
-      if (w.i + 1 <= a.top_k) {
+      if (((BLK == 128) ? w.i : 2 * w.i + 1) + 1 <= a.top_k) {   // every row keeps all its blocks
         if (!ok) break;
         if (eset == 0) {
 #pragma unroll
@@ -424,7 +461,7 @@ __global__ void __launch_bounds__(384, 1)
             const long long orow = index_out_row(a, sq, w.gp * GP + gi, t);
             if (orow < 0) continue;
             int32_t *dst = a.sel + orow * a.top_k;
-            for (int k = 0; k < a.top_k; ++k) dst[k] = (k <= w.i) ? k : -1;
+            for (int k = 0; k < a.top_k; ++k) dst[k] = (k <= bt) ? k : -1;
           }
         }
         continue;
@@ -453,6 +490,10 @@ __global__ void __launch_bounds__(384, 1)
           const long long orow = index_out_row(a, sq, w.gp * GP + gi, t);
           if (orow < 0) continue;
           int32_t *dst = a.sel + orow * a.top_k;
+          if (bt + 1 <= a.top_k) {   // (BLK 64) this half of the tile keeps all its blocks
+            for (int k = 0; k < a.top_k; ++k) dst[k] = (k <= bt) ? k : -1;
+            continue;
+          }
           int ids[KCAP];
 #pragma unroll
           for (int k = 0; k < KCAP; ++k) ids[k] = (k >= n_sent) ? lj[gi][k] : INT_MAX;
@@ -462,10 +503,10 @@ __global__ void __launch_bounds__(384, 1)
             for (int k = 0; k < KCAP; k += 4) {
               if (k < a.top_k) {
                 int4 o;
-                o.x = (k + 0 < k1) ? ids[k + 0] : (k + 0 == k1 ? w.i : -1);
-                o.y = (k + 1 < k1) ? ids[k + 1] : (k + 1 == k1 ? w.i : -1);
-                o.z = (k + 2 < k1) ? ids[k + 2] : (k + 2 == k1 ? w.i : -1);
-                o.w = (k + 3 < k1) ? ids[k + 3] : (k + 3 == k1 ? w.i : -1);
+                o.x = (k + 0 < k1) ? ids[k + 0] : (k + 0 == k1 ? bt : -1);
+                o.y = (k + 1 < k1) ? ids[k + 1] : (k + 1 == k1 ? bt : -1);
+                o.z = (k + 2 < k1) ? ids[k + 2] : (k + 2 == k1 ? bt : -1);
+                o.w = (k + 3 < k1) ? ids[k + 3] : (k + 3 == k1 ? bt : -1);
                 *reinterpret_cast<int4 *>(dst + k) = o;
               }
             }
@@ -474,7 +515,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int k = 0; k <= KCAP; ++k)
               if (k < a.top_k)
-                dst[k] = (k < k1) ? ids[k < KCAP ? k : KCAP - 1] : (k == k1 ? w.i : -1);
+                dst[k] = (k < k1) ? ids[k < KCAP ? k : KCAP - 1] : (k == k1 ? bt : -1);
           }
         }
       }
@@ -491,11 +532,11 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <int DI, int GP, int KCAP>
+template <int DI, int GP, int KCAP, int BLK>
 cudaError_t launch_index_t(const CUtensorMap &tq, const CUtensorMap &tk, const IndexArgs &a,
                            int num_sms, cudaStream_t st) {
   using C = IndexCfg<DI, GP, KCAP>;
-  auto kern = msa_index_kernel<DI, GP, KCAP>;
+  auto kern = msa_index_kernel<DI, GP, KCAP, BLK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = a.n_items < num_sms ? a.n_items : num_sms;
@@ -503,13 +544,29 @@ cudaError_t launch_index_t(const CUtensorMap &tq, const CUtensorMap &tk, const I
   return cudaGetLastError();
 }
 
-template <int DI, int GP>
+template <int DI, int GP, int BLK>
 cudaError_t launch_index_k(const CUtensorMap &tq, const CUtensorMap &tk, const IndexArgs &a,
                            int num_sms, cudaStream_t st) {
   const int k1 = a.top_k - 1;
-  if (k1 <= 4) return launch_index_t<DI, GP, 4>(tq, tk, a, num_sms, st);
-  if (k1 <= 8) return launch_index_t<DI, GP, 8>(tq, tk, a, num_sms, st);
-  return launch_index_t<DI, GP, 16>(tq, tk, a, num_sms, st);
+  if (k1 <= 4) return launch_index_t<DI, GP, 4, BLK>(tq, tk, a, num_sms, st);
+  if (k1 <= 8) return launch_index_t<DI, GP, 8, BLK>(tq, tk, a, num_sms, st);
+  return launch_index_t<DI, GP, 16, BLK>(tq, tk, a, num_sms, st);
+}
+
+template <int BLK>
+cudaError_t launch_index_b(const CUtensorMap &tq, const CUtensorMap &tk, const IndexArgs &a,
+                           int num_sms, cudaStream_t st) {
+  const int gp = index_groups_per_cta(a.G, a.top_k);
+  if (a.top_k - 1 > 16) {
+    // wide lists: one group per CTA, 32-entry list
+    if (a.d_idx == 64) return launch_index_t<64, 1, 32, BLK>(tq, tk, a, num_sms, st);
+    return launch_index_t<128, 1, 32, BLK>(tq, tk, a, num_sms, st);
+  }
+  if (a.d_idx == 64)
+    return gp == 2 ? launch_index_k<64, 2, BLK>(tq, tk, a, num_sms, st)
+                   : launch_index_k<64, 1, BLK>(tq, tk, a, num_sms, st);
+  return gp == 2 ? launch_index_k<128, 2, BLK>(tq, tk, a, num_sms, st)
+                 : launch_index_k<128, 1, BLK>(tq, tk, a, num_sms, st);
 }
 
 }  // namespace
@@ -519,17 +576,8 @@ int index_groups_per_cta(int G, int top_k) { return (G % 2 == 0 && top_k - 1 <= 
 cudaError_t launch_index_kernel(const CUtensorMap &tq, const CUtensorMap &tk, const IndexArgs &a,
                                 int num_sms, cudaStream_t st) {
   if (a.n_items <= 0) return cudaSuccess;
-  const int gp = index_groups_per_cta(a.G, a.top_k);
-  if (a.top_k - 1 > 16) {
-    // wide lists: one group per CTA, 32-entry list
-    if (a.d_idx == 64) return launch_index_t<64, 1, 32>(tq, tk, a, num_sms, st);
-    return launch_index_t<128, 1, 32>(tq, tk, a, num_sms, st);
-  }
-  if (a.d_idx == 64)
-    return gp == 2 ? launch_index_k<64, 2>(tq, tk, a, num_sms, st)
-                   : launch_index_k<64, 1>(tq, tk, a, num_sms, st);
-  return gp == 2 ? launch_index_k<128, 2>(tq, tk, a, num_sms, st)
-                 : launch_index_k<128, 1>(tq, tk, a, num_sms, st);
+  if (a.blk == 64) return launch_index_b<64>(tq, tk, a, num_sms, st);
+  return launch_index_b<128>(tq, tk, a, num_sms, st);
 }
 
 }  // namespace msa

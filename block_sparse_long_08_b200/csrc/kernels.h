@@ -50,6 +50,7 @@ __device__ __forceinline__ int qgeo_seq_of_row(const QGeo &q, int r) {
 // ordered longest first by the host), each with every group pair.
 struct IndexArgs {
   int B, L, G, nb, top_k, d_idx;
+  int blk;           // block length: 128 or 64 (query tiles are 128 rows either way)
   QGeo q;
   int write_scores;  // 1: store block scores, 0: fused top-k -> sel
   int i_hi, n_tiles; // uniform item range (items == nullptr)
@@ -65,7 +66,7 @@ cudaError_t launch_index_kernel(const CUtensorMap &tq, const CUtensorMap &tk, co
                                 int num_sms, cudaStream_t st);
 
 struct TopkArgs {
-  int B, G, L, nb, top_k;
+  int B, G, L, nb, top_k, blk;
   const float *scores;  // [B,G,L,nb]
   int32_t *sel;         // [B,G,L,top_k]
 };
@@ -90,6 +91,7 @@ cudaError_t launch_revidx(const RevIdxArgs &a, cudaStream_t st);
 
 struct AttnArgs {
   int L, H, G, nb, top_k;      // L: key rows per sequence
+  int blk;                     // block length: 128 or 64
   QGeo q;
   float scale, scale_log2;
   int max_items;               // upper bound on the chunk's work items
@@ -156,6 +158,7 @@ cudaError_t launch_backward(const CUtensorMap &tk, const CUtensorMap &tv, const 
 
 struct DecodeArgs {
   int B, Lmax, H, G, d_idx, nb_max, top_k;
+  int blk;                     // block length: 128 or 64 (nb_max = ceil(Lmax / blk))
   float scale, scale_log2;
   const uint16_t *q, *q_idx, *k_cache, *v_cache, *k_idx_cache;
   // FP8 index-key cache (when non-null, used instead of k_idx_cache):
@@ -171,6 +174,7 @@ struct DecodeArgs {
   int32_t *sel;                // [B,G,top_k]
   float *part_o;               // [B,H,top_k,d]
   float *part_lse;             // [B,H,top_k]
+  int *tickets;                // [B,G]: merge tickets of the attention (zeroed by the top-k)
   uint16_t *out;               // [B,H,d]
   int *status;
 };

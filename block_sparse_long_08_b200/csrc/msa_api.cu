@@ -51,7 +51,8 @@ int check_params(const msa_params *p, bool decode, bool whole_blocks = false) {
   if (p->d != 128) return fail(MSA_ERR_UNSUPPORTED, "d=%d (supported: 128)", p->d);
   if (p->d_idx != 64 && p->d_idx != 128)
     return fail(MSA_ERR_UNSUPPORTED, "d_idx=%d (supported: 64, 128)", p->d_idx);
-  if (p->block != 128) return fail(MSA_ERR_UNSUPPORTED, "block=%d (supported: 128)", p->block);
+  if (p->block != 128 && p->block != 64)
+    return fail(MSA_ERR_UNSUPPORTED, "block=%d (supported: 64, 128)", p->block);
   if (p->top_k > msa::kMaxTopK)
     return fail(MSA_ERR_UNSUPPORTED, "top_k=%d (supported: 1..32)", p->top_k);
   if (p->H % p->G != 0) return fail(MSA_ERR_INVALID_ARG, "H=%d not a multiple of G=%d", p->H, p->G);
@@ -60,6 +61,8 @@ int check_params(const msa_params *p, bool decode, bool whole_blocks = false) {
     return fail(MSA_ERR_UNSUPPORTED, "H/G=%d (supported: 1,2,4,8,16)", r);
   if (whole_blocks && p->L % 128 != 0)
     return fail(MSA_ERR_UNSUPPORTED, "L=%d: this operation needs a multiple of 128", p->L);
+  if (whole_blocks && p->block != 128)
+    return fail(MSA_ERR_UNSUPPORTED, "block=%d: this operation needs 128-token blocks", p->block);
   if (decode && p->G > 8) return fail(MSA_ERR_UNSUPPORTED, "decode supports G <= 8 (G=%d)", p->G);
   if ((long long)p->B * p->L > (1LL << 26))
     return fail(MSA_ERR_UNSUPPORTED, "B*L=%lld above 2^26", (long long)p->B * p->L);
@@ -72,7 +75,9 @@ float eff_scale(const msa_params *p) {
   return p->scale > 0.f ? p->scale : 1.0f / std::sqrt(float(p->d));
 }
 
-int nblocks(int L) { return (L + 127) / 128; }
+// Key blocks of a sequence of L tokens (the last one may be partial).
+int nblocks(const msa_params *p, int L) { return (L + p->block - 1) / p->block; }
+int nblocks(const msa_params *p) { return nblocks(p, p->L); }
 
 // ---- workspace plans --------------------------------------------------------
 // Prefill attention processes the packed query rows in chunks of Rc so that
@@ -101,7 +106,7 @@ struct AttnWs {
 AttnWs attn_ws(const msa_params *p, size_t base, long long n_rows, int n_seq) {
   AttnWs w;
   w.Rc = prefill_chunk(p, n_rows);
-  const size_t nbgj = size_t(n_seq) * p->G * nblocks(p->L);
+  const size_t nbgj = size_t(n_seq) * p->G * nblocks(p);
   const size_t entries = size_t(p->G) * w.Rc * p->top_k;
   size_t o = base;
   w.cnt = o; o = align_up(o + 4 * nbgj);
@@ -130,7 +135,7 @@ BwdWs bwd_ws(const msa_params *p) {
   BwdWs w;
   const long long n_rows = (long long)p->B * p->L;
   w.Rc = prefill_chunk(p, n_rows);
-  const size_t nbgj = size_t(p->B) * p->G * nblocks(p->L);
+  const size_t nbgj = size_t(p->B) * p->G * nblocks(p);
   const size_t entries = size_t(p->G) * w.Rc * p->top_k;
   size_t o = msa::kWsHeader;
   w.cnt = o; o = align_up(o + 4 * nbgj);
@@ -151,16 +156,17 @@ BwdWs bwd_ws(const msa_params *p) {
 }
 
 struct DecWs {
-  size_t scores, sel, part_o, part_lse, end;
+  size_t scores, sel, part_o, part_lse, tickets, end;
 };
 DecWs dec_ws(const msa_params *p) {
   DecWs w;
-  const size_t nb = size_t(nblocks(p->L));
+  const size_t nb = size_t(nblocks(p));
   size_t o = msa::kWsHeader;
   w.scores = o; o = align_up(o + 4 * size_t(p->B) * p->G * nb);
   w.sel = o; o = align_up(o + 4 * size_t(p->B) * p->G * p->top_k);
   w.part_o = o; o = align_up(o + 4 * size_t(p->B) * p->H * p->top_k * p->d);
   w.part_lse = o; o = align_up(o + 4 * size_t(p->B) * p->H * p->top_k);
+  w.tickets = o; o = align_up(o + 4 * size_t(p->B) * p->G);
   w.end = o;
   return w;
 }
@@ -181,7 +187,7 @@ VarlenWs varlen_ws(const msa_params *p) {
   size_t o = msa::kWsHeader;
   w.maps = o; o = align_up(o + 2 * sizeof(CUtensorMap) * size_t(p->B));
   w.seqs = o; o = align_up(o + sizeof(int4) * size_t(p->B));
-  w.items = o; o = align_up(o + sizeof(int2) * size_t(p->B) * nblocks(p->L));
+  w.items = o; o = align_up(o + sizeof(int2) * size_t(p->B) * ((p->L + 127) / 128));   // query tiles
   w.sel = o; o += forward_sel_bytes(p);
   w.attn_base = o;
   return w;
@@ -227,11 +233,12 @@ int make_tmap(CUtensorMap *m, const void *base, int rank, const uint64_t *dims,
 
 // 4-D map (d, G, key rows, sequences) over K or V [nseq, L, G, d], the row
 // extent cut at kv_rows: rows >= kv_rows of each sequence load as zeros.
+// A box is one block of keys (p->block rows) of one KV head, half of d.
 int make_kv_tmap(CUtensorMap *m, const void *base, const msa_params *p, int kv_rows, int nseq) {
   const uint64_t dims[4] = {uint64_t(p->d), uint64_t(p->G), uint64_t(kv_rows), uint64_t(nseq)};
   const uint64_t str[3] = {uint64_t(p->d) * 2, uint64_t(p->d) * 2 * p->G,
                            uint64_t(p->d) * 2 * p->G * p->L};
-  const uint32_t box[4] = {64, 1, 128, 1};
+  const uint32_t box[4] = {64, 1, uint32_t(p->block), 1};
   return make_tmap(m, base, 4, dims, str, box);
 }
 
@@ -284,7 +291,7 @@ IndexWork uniform_index_work(const msa::QGeo &q, int t_lo, int t_hi) {
 int run_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 *k_idx,
                      int32_t *sel, float *block_scores, void *ws, cudaStream_t st,
                      const msa::QGeo &qg, const IndexWork &iw) {
-  const int nb = nblocks(p->L);
+  const int nb = nblocks(p);
   CUtensorMap tq, tk;
   {
     const uint64_t dims[3] = {uint64_t(p->d_idx), uint64_t(p->G), uint64_t(qg.N)};
@@ -302,6 +309,7 @@ int run_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 
   }
   msa::IndexArgs a;
   a.B = p->B; a.L = p->L; a.G = p->G; a.nb = nb; a.top_k = p->top_k; a.d_idx = p->d_idx;
+  a.blk = p->block;
   a.q = qg;
   a.write_scores = block_scores ? 1 : 0;
   a.i_hi = iw.i_hi;
@@ -318,7 +326,7 @@ int run_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 
   if (e != cudaSuccess) return cuda_fail(e, "index kernel launch");
   if (block_scores) {
     msa::TopkArgs t;
-    t.B = p->B; t.G = p->G; t.L = p->L; t.nb = nb; t.top_k = p->top_k;
+    t.B = p->B; t.G = p->G; t.L = p->L; t.nb = nb; t.top_k = p->top_k; t.blk = p->block;
     t.scores = block_scores;
     t.sel = sel;
     e = msa::launch_topk_kernel(t, st);
@@ -350,7 +358,7 @@ struct AttnPlan {
 // load as zeros); kv_maps: per-sequence maps instead (ragged batch).
 int plan_attn(const msa_params *p, const msa_bf16 *k, const msa_bf16 *v, size_t ws_base,
               const msa::QGeo &qg, int kv_rows, const CUtensorMap *kv_maps, AttnPlan *pl) {
-  pl->nb = nblocks(p->L);
+  pl->nb = nblocks(p);
   pl->qg = qg;
   pl->kv_maps = kv_maps;
   pl->w = attn_ws(p, ws_base, qg.N, qg.B);
@@ -386,6 +394,7 @@ int run_attn_chunk(const msa_params *p, const AttnPlan &pl, const msa_bf16 *q, c
   if (e != cudaSuccess) return cuda_fail(e, "reverse index launch");
   msa::AttnArgs aa;
   aa.L = p->L; aa.H = p->H; aa.G = p->G; aa.nb = pl.nb; aa.top_k = p->top_k;
+  aa.blk = p->block;
   aa.q = pl.qg;
   aa.scale = pl.scale;
   aa.scale_log2 = pl.scale * 1.4426950408889634f;
@@ -518,7 +527,8 @@ int run_decode(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
   uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
   msa::DecodeArgs a;
   a.B = p->B; a.Lmax = p->L; a.H = p->H; a.G = p->G; a.d_idx = p->d_idx;
-  a.nb_max = nblocks(p->L); a.top_k = p->top_k;
+  a.nb_max = nblocks(p); a.top_k = p->top_k;
+  a.blk = p->block;
   a.scale = eff_scale(p);
   a.scale_log2 = a.scale * 1.4426950408889634f;
   a.q = q; a.q_idx = q_idx; a.k_cache = k_cache; a.v_cache = v_cache; a.k_idx_cache = k_idx_cache;
@@ -529,6 +539,7 @@ int run_decode(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
   a.sel = sel ? sel : reinterpret_cast<int32_t *>(wsb + w.sel);
   a.part_o = reinterpret_cast<float *>(wsb + w.part_o);
   a.part_lse = reinterpret_cast<float *>(wsb + w.part_lse);
+  a.tickets = reinterpret_cast<int *>(wsb + w.tickets);
   a.out = out;
   a.status = status_ptr(ws);
   cudaError_t e = msa::launch_decode(a, st);

@@ -7,8 +7,9 @@
 // external aggregation Q").
 //
 // One work item = one (b, g, key block j) and up to 128/R queries that
-// selected j, each with its R heads: a 128-row tile.  Per item:
-//   S = Q K_j^T   (UMMA M=128, N=128, K=128, fp32 in TMEM)
+// selected j, each with its R heads: a 128-row tile.  Blocks hold BLK = 128
+// or 64 keys (the explainer's §4.2 reasons with 64-token blocks).  Per item:
+//   S = Q K_j^T   (UMMA M=128, N=BLK, K=128, fp32 in TMEM)
 //   softmax       row r: mask s <= t (only on the diagonal block), row max,
 //                 exp2, row sum, P as bf16 into shared memory
 //   O = P V_j     (UMMA, V consumed MN-major straight from its TMA tile)
@@ -163,12 +164,15 @@ struct ItemWalk {
   }
 };
 
-template <int R>
+template <int R, int BLK>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     msa_prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_k,
                             const __grid_constant__ CUtensorMap tm_v, const AttnArgs a) {
   using C = AttnCfg<R>;
   constexpr int QPI = C::QPI;
+  // a K or V tile: BLK rows of 256 B as two 128B-swizzled halves (d 0..63,
+  // 64..127) of BLK * 128 bytes each, in a 32 KB slot
+  constexpr uint32_t kHalf = BLK * 128;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -252,7 +256,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               ok = false;
               break;
             }
-            mbar_arrive_expect_tx(bar(C::BAR_KVFULL + x), kTile);
+            mbar_arrive_expect_tx(bar(C::BAR_KVFULL + x), 2 * kHalf);
             const uint32_t dst = s_base + C::SMEM_KV + x * kTile;
             // 4-D maps (d, G, key rows, sequences): the sequence's own map
             // (batch coordinate 0) or the launch's map over the batch
@@ -261,8 +265,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                             : static_cast<const void *>(&tm_k));
             const int zb = a.kv_maps ? 0 : b;
             if (a.kv_maps) tensormap_acquire(tm);
-            tma_load_4d(dst, tm, bar(C::BAR_KVFULL + x), 0, g, j * kBlock, zb);
-            tma_load_4d(dst + 16384, tm, bar(C::BAR_KVFULL + x), 64, g, j * kBlock, zb);
+            tma_load_4d(dst, tm, bar(C::BAR_KVFULL + x), 0, g, j * BLK, zb);
+            tma_load_4d(dst + kHalf, tm, bar(C::BAR_KVFULL + x), 64, g, j * BLK, zb);
             issued[x] = tau;
           }
         }
@@ -273,7 +277,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     } else if (warp == 1) {
       // ------------------------------------------------------ MMA issuer
       if (lane == 0 && n_loc > 0) {
-        constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint32_t idesc_s = idesc_bf16_f32(128, BLK, 0, 0);
         constexpr uint32_t idesc_o = idesc_bf16_f32(128, 128, 0, 1);
         int ns = 0, no = 0;          // next S and next O to issue (item indices)
         int m_s = -1, prev_bgj = -1; // run of item ns-1 and its key block
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                   const int c = kk >> 2;
                   const uint32_t off = (kk & 3) * 32;
                   umma_f16_ss(d_tmem, sdesc_sw128(sq + c * 16384 + off, 16, 1024),
-                              sdesc_sw128(sk + c * 16384 + off, 16, 1024), idesc_s, kk > 0);
+                              sdesc_sw128(sk + c * kHalf + off, 16, 1024), idesc_s, kk > 0);
                 }
                 umma_commit(bar(C::BAR_SFULL + (ns & 1)));
                 {   // per in-flight item: V tile, its phase, whether the item opens a run
@@ -347,11 +351,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
               const uint32_t sv = s_base + C::SMEM_KV + xv * kTile;
               const uint32_t d_tmem = tmem_base + (no & 1) * 128;
 #pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
+              for (int kk = 0; kk < BLK / 16; ++kk) {   // P's keys: 64 per 16 KB half
                 const int c = kk >> 2;
                 const uint32_t off = (kk & 3) * 32;
                 umma_f16_ss(d_tmem, sdesc_sw128(sp + c * 16384 + off, 16, 1024),
-                            sdesc_sw128(sv + kk * 2048, 16384, 1024), idesc_o, kk > 0);
+                            sdesc_sw128(sv + kk * 2048, kHalf, 1024), idesc_o, kk > 0);
               }
               umma_commit(bar(C::BAR_OFULL + (no & 1)));
               // free run m's V tile once item no is known to be its last
@@ -486,47 +490,56 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int qi = row / R;
       const bool valid = qi < d.z;
       const int t = valid ? (s_list[s * QPI + qi] >> 5) : 0;
-      const int lim = valid ? (t - j * kBlock) : (kBlock - 1);   // last visible column
+      const int lim = valid ? (t - j * BLK) : (BLK - 1);   // last visible column
       ok = mbar_wait(bar(C::BAR_SFULL + u), (i >> 1) & 1, abort_flag, a.status);
       if (!bar_and_n(bar_id, 128, ok)) break;
       tc_fence_after();
 
-      float v[128];
+      float v[BLK];
       {
+        // every load is issued, then waited for, before any value is read
         float t0[32], t1[32], t2[32], t3[32];
         tmem_ld32(tm, t0);
         tmem_ld32(tm + 32, t1);
-        tmem_ld32(tm + 64, t2);
-        tmem_ld32(tm + 96, t3);
+        if (BLK == 128) {
+          tmem_ld32(tm + 64, t2);
+          tmem_ld32(tm + 96, t3);
+        }
         tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-          v[x] = t0[x]; v[32 + x] = t1[x]; v[64 + x] = t2[x]; v[96 + x] = t3[x];
+          v[x] = t0[x];
+          v[32 + x] = t1[x];
+          if (BLK == 128) {
+            v[64 + x] = t2[x];
+            v[96 + x] = t3[x];
+          }
         }
       }
-      // causal mask: only rows whose own block is j see fewer than 128 keys
-      if (__any_sync(0xffffffffu, lim < kBlock - 1)) {
+      // causal mask: only rows whose own block is j see fewer than BLK keys
+      if (__any_sync(0xffffffffu, lim < BLK - 1)) {
 #pragma unroll
-        for (int x = 0; x < 128; ++x) v[x] = (x <= lim) ? v[x] : -INFINITY;
+        for (int x = 0; x < BLK; ++x) v[x] = (x <= lim) ? v[x] : -INFINITY;
       }
-      float m0 = max3f(v[0], v[1], v[2]), m1 = max3f(v[32], v[33], v[34]);
-      float m2 = max3f(v[64], v[65], v[66]), m3 = max3f(v[96], v[97], v[98]);
+      float mc[BLK / 32];   // independent max chains, one per 32 columns
+#pragma unroll
+      for (int c4 = 0; c4 < BLK / 32; ++c4) mc[c4] = max3f(v[32 * c4], v[32 * c4 + 1], v[32 * c4 + 2]);
 #pragma unroll
       for (int x = 3; x + 2 <= 31; x += 2) {
-        m0 = max3f(m0, v[x], v[x + 1]);
-        m1 = max3f(m1, v[32 + x], v[33 + x]);
-        m2 = max3f(m2, v[64 + x], v[65 + x]);
-        m3 = max3f(m3, v[96 + x], v[97 + x]);
+#pragma unroll
+        for (int c4 = 0; c4 < BLK / 32; ++c4)
+          mc[c4] = max3f(mc[c4], v[32 * c4 + x], v[32 * c4 + x + 1]);
       }
-      m0 = fmaxf(m0, v[31]); m1 = fmaxf(m1, v[63]); m2 = fmaxf(m2, v[95]); m3 = fmaxf(m3, v[127]);
-      const float m = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+      float m = fmaxf(mc[0], v[31]);
+#pragma unroll
+      for (int c4 = 1; c4 < BLK / 32; ++c4) m = fmaxf(m, fmaxf(mc[c4], v[32 * c4 + 31]));
       const float mb = m * a.scale_log2;
       const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
       const float2 nmb2 = make_float2(-mb, -mb);
       float2 l2 = make_float2(0.f, 0.f);
       uint8_t *stage = smem + C::SMEM_Q + s * kTile;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < BLK / 64; ++h) {
 #pragma unroll
         for (int gb = 0; gb < 8; ++gb) {
           uint32_t w4[4];
@@ -549,6 +562,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ok = mbar_wait(bar(C::BAR_OFULL + u), (i >> 1) & 1, abort_flag, a.status);
       if (!bar_and_n(bar_id, 128, ok)) break;
       tc_fence_after();
+      float ov[kHeadDim];   // the item's O row (all of d, whatever the block length)
       {
         float t0[32], t1[32], t2[32], t3[32];
         tmem_ld32(tm, t0);
@@ -558,7 +572,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
-          v[x] = t0[x]; v[32 + x] = t1[x]; v[64 + x] = t2[x]; v[96 + x] = t3[x];
+          ov[x] = t0[x]; ov[32 + x] = t1[x]; ov[64 + x] = t2[x]; ov[96 + x] = t3[x];
         }
       }
       tc_fence_before();
@@ -572,10 +586,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       uint8_t *orow = stage + row * 256;
 #pragma unroll
       for (int c = 0; c < 16; ++c) {
-        const float2 o0 = mul2(make_float2(v[8 * c], v[8 * c + 1]), inv2);
-        const float2 o1 = mul2(make_float2(v[8 * c + 2], v[8 * c + 3]), inv2);
-        const float2 o2 = mul2(make_float2(v[8 * c + 4], v[8 * c + 5]), inv2);
-        const float2 o3 = mul2(make_float2(v[8 * c + 6], v[8 * c + 7]), inv2);
+        const float2 o0 = mul2(make_float2(ov[8 * c], ov[8 * c + 1]), inv2);
+        const float2 o1 = mul2(make_float2(ov[8 * c + 2], ov[8 * c + 3]), inv2);
+        const float2 o2 = mul2(make_float2(ov[8 * c + 4], ov[8 * c + 5]), inv2);
+        const float2 o3 = mul2(make_float2(ov[8 * c + 6], ov[8 * c + 7]), inv2);
         const uint4 w = make_uint4(pack_bf16x2(o0.x, o0.y), pack_bf16x2(o1.x, o1.y),
                                    pack_bf16x2(o2.x, o2.y), pack_bf16x2(o3.x, o3.y));
         *reinterpret_cast<uint4 *>(orow + ((c ^ (rho & 7)) << 4)) = w;
@@ -609,10 +623,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   }
 }
 
-template <int R>
+template <int R, int BLK>
 cudaError_t launch_attn_r(const CUtensorMap &tk, const CUtensorMap &tv, const AttnArgs &a,
                           int num_sms, cudaStream_t st) {
-  auto kern = msa_prefill_attn_kernel<R>;
+  auto kern = msa_prefill_attn_kernel<R, BLK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, AttnCfg<R>::SMEM);
   if (e != cudaSuccess) return e;
   int grid = num_sms;
@@ -621,19 +635,25 @@ cudaError_t launch_attn_r(const CUtensorMap &tk, const CUtensorMap &tv, const At
   return cudaGetLastError();
 }
 
+template <int BLK>
+cudaError_t launch_attn_b(const CUtensorMap &tk, const CUtensorMap &tv, const AttnArgs &a,
+                          int num_sms, cudaStream_t st) {
+  switch (a.H / a.G) {
+    case 1: return launch_attn_r<1, BLK>(tk, tv, a, num_sms, st);
+    case 2: return launch_attn_r<2, BLK>(tk, tv, a, num_sms, st);
+    case 4: return launch_attn_r<4, BLK>(tk, tv, a, num_sms, st);
+    case 8: return launch_attn_r<8, BLK>(tk, tv, a, num_sms, st);
+    case 16: return launch_attn_r<16, BLK>(tk, tv, a, num_sms, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_prefill_attn(const CUtensorMap &tk, const CUtensorMap &tv, const AttnArgs &a,
                                 int num_sms, cudaStream_t st) {
-  const int R = a.H / a.G;
-  switch (R) {
-    case 1: return launch_attn_r<1>(tk, tv, a, num_sms, st);
-    case 2: return launch_attn_r<2>(tk, tv, a, num_sms, st);
-    case 4: return launch_attn_r<4>(tk, tv, a, num_sms, st);
-    case 8: return launch_attn_r<8>(tk, tv, a, num_sms, st);
-    case 16: return launch_attn_r<16>(tk, tv, a, num_sms, st);
-    default: return cudaErrorInvalidValue;
-  }
+  return a.blk == 64 ? launch_attn_b<64>(tk, tv, a, num_sms, st)
+                     : launch_attn_b<128>(tk, tv, a, num_sms, st);
 }
 
 // ---------------------------------------------------------------- combine

@@ -135,6 +135,90 @@ __device__ __forceinline__ void warp_topk_write(const WarpTopk &st, int bt, int 
   if (lane < top_k) out[lane] = id;
 }
 
+// Descending bitonic sort of one float per lane (lane 0 ends with the
+// largest).
+__device__ __forceinline__ float warp_sort_desc(float x, int lane) {
+#pragma unroll
+  for (int k = 2; k <= 32; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const float o = __shfl_xor_sync(0xffffffffu, x, j);
+      const bool first = (lane & k) == 0;
+      const bool lower = (lane & j) == 0;
+      x = (lower == first) ? fmaxf(x, o) : fminf(x, o);
+    }
+  }
+  return x;
+}
+
+// Threshold form of the same selection, for rows of at most 32 * VPL
+// scores (held in registers).  Lane l holds scores l, l+32, ...; T, the
+// k1-th largest of the 32 lane maxima, has at least k1 scores at or above
+// it (those lane maxima), so the k1-th score of the row is >= T and every
+// kept block scores >= T.  The few candidates >= T (about 20 for k1 = 15 on
+// unstructured scores) are gathered in id order through shared memory and
+// ranked once with the bitonic (score desc, id asc) network; more than 32
+// candidates (exact ties, adversarial rows) fall back to the insertion
+// scan.  Same result as warp_topk_select, ties included.
+// s_cs / s_cj: 32 floats / ints of shared memory per warp.
+template <int VPL>
+__device__ __forceinline__ void warp_topk_select_thr(const float *__restrict__ row, int bt,
+                                                     int top_k, int32_t *__restrict__ out,
+                                                     float *s_cs, int *s_cj) {
+  const int lane = threadIdx.x & 31;
+  if (bt + 1 <= top_k) {
+    for (int k = lane; k < top_k; k += 32) out[k] = (k <= bt) ? k : -1;
+    return;
+  }
+  if (top_k == 1) {
+    if (lane == 0) out[0] = bt;
+    return;
+  }
+  const int k1 = top_k - 1;
+  float v[VPL];
+  float m = -FLT_MAX;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {   // every load issued before any use
+    const int j = i * 32 + lane;
+    v[i] = (j < bt) ? __ldg(row + j) : -FLT_MAX;
+  }
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) m = fmaxf(m, v[i]);
+  const float T = __shfl_sync(0xffffffffu, warp_sort_desc(m, lane), k1 - 1);
+  int c = 0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) c += (i * 32 + lane < bt && v[i] >= T) ? 1 : 0;
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  WarpTopk st;
+  if (total <= 32) {
+    int pos = incl - c;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      if (i * 32 + lane < bt && v[i] >= T) {
+        s_cs[pos] = v[i];
+        s_cj[pos] = i * 32 + lane;
+        ++pos;
+      }
+    }
+    __syncwarp();
+    const bool have = lane < total;
+    const float cs = have ? s_cs[lane] : -FLT_MAX;
+    const int cj = have ? s_cj[lane] : INT_MAX;
+    __syncwarp();   // the next row of this warp rewrites the exchange area
+    warp_topk_seed(st, cs, cj, have, k1);
+  } else {
+    warp_topk_init(st);
+    warp_topk_scan(st, row, 0, bt, k1);
+  }
+  warp_topk_write(st, bt, top_k, out);
+}
+
 // The selection rule for the block-score row of a query whose local block
 // is bt: blocks 0..bt-1 are candidates (the local block is not read).
 // Writes top_k ints to out: selected ids ascending, -1 padding.

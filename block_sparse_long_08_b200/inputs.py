@@ -57,7 +57,30 @@ DECODE_128K = DecodeShape(B=32, Lmax=131072, H=32, G=8, len_lo=65536, len_hi=131
 PREFILL_1M = PrefillShape(B=1, L=1048576, H=32, G=8)
 DECODE_1M = DecodeShape(B=4, Lmax=1048576, H=32, G=8, len_lo=1048576, len_hi=1048576)
 
-SEEDS = {"tiny": 0, "32k": 1, "128k_planted": 2, "decode_128k": 3, "1m": 4}
+# The 64-token block variant of the 32K prefill at the same 2048-token
+# budget ("MiniMax M3 sparse attention" explainer §4.2 reasons with 64-token
+# blocks): 32 blocks of 64.
+PREFILL_32K_BLOCK64 = PrefillShape(B=1, L=32768, H=32, G=8, block=64, top_k=32)
+
+
+@dataclasses.dataclass(frozen=True)
+class RaggedBatchShape:
+    """Prompt chunks continuing cached prefixes: B sequences, caches of Lmax
+    tokens, n_b new tokens uniform in [1, n_hi], positions t0_b uniform in
+    [0, Lmax - n_b]."""
+    B: int
+    Lmax: int
+    n_hi: int
+    H: int
+    G: int
+    d: int = 128
+    d_idx: int = 128
+    top_k: int = 16
+
+
+RAGGED_BATCH = RaggedBatchShape(B=16, Lmax=131072, n_hi=16384, H=32, G=8)
+
+SEEDS = {"tiny": 0, "32k": 1, "128k_planted": 2, "decode_128k": 3, "1m": 4, "ragged": 5}
 
 
 def _normal_bf16(gen: torch.Generator, shape, device) -> torch.Tensor:

@@ -172,17 +172,17 @@ def _ensure_ws(ws, p, op, device):
 
 def msa_index_select(q_idx: torch.Tensor, k_idx: torch.Tensor, top_k: int, *,
                      block_scores: bool = False, sel: Optional[torch.Tensor] = None,
-                     ws: Optional[torch.Tensor] = None, stream=None):
+                     ws: Optional[torch.Tensor] = None, stream=None, block: int = 128):
     """q_idx [B,L,G,d_idx], k_idx [B,L,d_idx] -> sel [B,G,L,top_k] int32
     (and block scores [B,G,L,nb] fp32 when block_scores=True)."""
     _req(q_idx, "q_idx", torch.bfloat16)
     _req(k_idx, "k_idx", torch.bfloat16)
     B, L, G, di = q_idx.shape
-    p = make_params(B, L, G, G, 128, di, 128, top_k)
+    p = make_params(B, L, G, G, 128, di, block, top_k)
     dev = q_idx.device
     if sel is None:
         sel = torch.empty((B, G, L, top_k), dtype=torch.int32, device=dev)
-    scores = torch.empty((B, G, L, (L + 127) // 128), dtype=torch.float32,
+    scores = torch.empty((B, G, L, (L + block - 1) // block), dtype=torch.float32,
                          device=dev) if block_scores else None
     ws = _ensure_ws(ws, p, MSA_OP_INDEX_SELECT, dev)
     _check(lib().msa_index_select(ctypes.byref(p), _ptr(q_idx), _ptr(k_idx), _ptr(sel), _ptr(scores),
@@ -191,7 +191,7 @@ def msa_index_select(q_idx: torch.Tensor, k_idx: torch.Tensor, top_k: int, *,
 
 
 def msa_sparse_attn_prefill(q, k, v, sel, *, scale: float = 0.0, want_lse: bool = False,
-                            out=None, ws=None, stream=None, chunk: int = 0):
+                            out=None, ws=None, stream=None, chunk: int = 0, block: int = 128):
     """q [B,L,H,d], k/v [B,L,G,d] bf16, sel [B,G,L,top_k] int32 -> out [B,L,H,d]
     (and lse [B,L,H] fp32 when want_lse)."""
     for n, t in (("q", q), ("k", k), ("v", v)):
@@ -200,7 +200,7 @@ def msa_sparse_attn_prefill(q, k, v, sel, *, scale: float = 0.0, want_lse: bool 
     B, L, H, d = q.shape
     G = k.shape[2]
     top_k = sel.shape[3]
-    p = make_params(B, L, H, G, d, 128, 128, top_k, scale, chunk)
+    p = make_params(B, L, H, G, d, 128, block, top_k, scale, chunk)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
@@ -236,14 +236,14 @@ def msa_sparse_attn_backward(q, k, v, out, lse, dout, sel, *, scale: float = 0.0
 
 
 def msa_forward(q, k, v, q_idx, k_idx, top_k: int, *, scale: float = 0.0, want_sel: bool = False,
-                want_lse: bool = False, out=None, sel=None, ws=None, stream=None, chunk: int = 0):
+                want_lse: bool = False, out=None, sel=None, ws=None, stream=None, chunk: int = 0, block: int = 128):
     """Whole prefill: index branch with fused top-k, then the sparse main branch."""
     for n, t in (("q", q), ("k", k), ("v", v), ("q_idx", q_idx), ("k_idx", k_idx)):
         _req(t, n, torch.bfloat16)
     B, L, H, d = q.shape
     G = k.shape[2]
     di = q_idx.shape[3]
-    p = make_params(B, L, H, G, d, di, 128, top_k, scale, chunk)
+    p = make_params(B, L, H, G, d, di, block, top_k, scale, chunk)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
@@ -263,7 +263,7 @@ def msa_forward(q, k, v, q_idx, k_idx, top_k: int, *, scale: float = 0.0, want_s
 
 def msa_forward_cached(q, q_idx, k_cache, v_cache, k_idx_cache, t0: int, top_k: int, *,
                        scale: float = 0.0, want_sel: bool = False, want_lse: bool = False,
-                       out=None, sel=None, ws=None, stream=None, chunk: int = 0):
+                       out=None, sel=None, ws=None, stream=None, chunk: int = 0, block: int = 128):
     """Prefill of the n new tokens at positions [t0, t0+n) against caches that
     already hold every key up to t0+n: q [B,n,H,d], q_idx [B,n,G,d_idx];
     k_cache/v_cache [B,Lmax,G,d], k_idx_cache [B,Lmax,d_idx] -> out [B,n,H,d]
@@ -275,7 +275,7 @@ def msa_forward_cached(q, q_idx, k_cache, v_cache, k_idx_cache, t0: int, top_k: 
     B, n, H, d = q.shape
     Lmax, G = k_cache.shape[1], k_cache.shape[2]
     di = q_idx.shape[3]
-    p = make_params(B, Lmax, H, G, d, di, 128, top_k, scale, chunk)
+    p = make_params(B, Lmax, H, G, d, di, block, top_k, scale, chunk)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
@@ -296,7 +296,7 @@ def msa_forward_cached(q, q_idx, k_cache, v_cache, k_idx_cache, t0: int, top_k: 
 
 def msa_forward_cached_varlen(q, q_idx, k_cache, v_cache, k_idx_cache, t0, n, top_k: int, *,
                               scale: float = 0.0, want_lse: bool = False, out=None, ws=None,
-                              stream=None, chunk: int = 0):
+                              stream=None, chunk: int = 0, block: int = 128):
     """Ragged batch of cached prefills: sequence b continues at position t0[b]
     with n[b] new tokens whose query rows are packed in q [sum n,H,d] and
     q_idx [sum n,G,d_idx]; caches [B,Lmax,...].  Returns out [sum n,H,d]
@@ -310,7 +310,7 @@ def msa_forward_cached_varlen(q, q_idx, k_cache, v_cache, k_idx_cache, t0, n, to
     na = (ctypes.c_int32 * B)(*[int(v) for v in n])
     if sum(int(v) for v in n) != q.shape[0]:
         raise ValueError("q rows must equal sum(n)")
-    p = make_params(B, Lmax, H, G, d, q_idx.shape[2], 128, top_k, scale, chunk)
+    p = make_params(B, Lmax, H, G, d, q_idx.shape[2], block, top_k, scale, chunk)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
@@ -335,7 +335,7 @@ def _req_host(t: torch.Tensor, name: str, dtype) -> torch.Tensor:
 
 def msa_forward_host(q, k, v, q_idx, k_idx, top_k: int, *, out, lse=None, staging=None,
                      scale: float = 0.0, ws=None, stream=None, copy_stream=None, chunk: int = 0,
-                     device=None):
+                     device=None, block: int = 128):
     """msa_forward on HOST tensors (pinned for overlap): q [B,L,H,d], k/v [B,L,G,d],
     q_idx [B,L,G,d_idx], k_idx [B,L,d_idx] bf16 in; out [B,L,H,d] bf16 (and lse
     [B,L,H] fp32) host tensors filled.  `staging` holds the device buffers
@@ -349,7 +349,7 @@ def msa_forward_host(q, k, v, q_idx, k_idx, top_k: int, *, out, lse=None, stagin
     B, L, H, d = q.shape
     G = k.shape[2]
     di = q_idx.shape[3]
-    p = make_params(B, L, H, G, d, di, 128, top_k, scale, chunk)
+    p = make_params(B, L, H, G, d, di, block, top_k, scale, chunk)
     dev = torch.device("cuda") if device is None else torch.device(device)
     if staging is None:
         staging = {n: torch.empty(t.shape, dtype=t.dtype, device=dev)
@@ -372,7 +372,7 @@ def msa_forward_host(q, k, v, q_idx, k_idx, top_k: int, *, out, lse=None, stagin
 
 def msa_sparse_attn_decode(q, q_idx, k_cache, v_cache, k_idx_cache, seq_lens, top_k: int, *,
                            scale: float = 0.0, want_sel: bool = False, out=None, sel=None,
-                           ws=None, stream=None):
+                           ws=None, stream=None, block: int = 128):
     """q [B,H,d], q_idx [B,G,d_idx], caches [B,Lmax,G,d] / [B,Lmax,d_idx],
     seq_lens [B] int32 (device) -> out [B,H,d] (and sel [B,G,top_k])."""
     for n, t in (("q", q), ("q_idx", q_idx), ("k_cache", k_cache), ("v_cache", v_cache),
@@ -382,7 +382,7 @@ def msa_sparse_attn_decode(q, q_idx, k_cache, v_cache, k_idx_cache, seq_lens, to
     B, H, d = q.shape
     Lmax, G = k_cache.shape[1], k_cache.shape[2]
     di = q_idx.shape[2]
-    p = make_params(B, Lmax, H, G, d, di, 128, top_k, scale)
+    p = make_params(B, Lmax, H, G, d, di, block, top_k, scale)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
@@ -397,7 +397,7 @@ def msa_sparse_attn_decode(q, q_idx, k_cache, v_cache, k_idx_cache, seq_lens, to
 
 def msa_sparse_attn_decode_fp8idx(q, q_idx, k_cache, v_cache, k_idx8, k_idx_scale, seq_lens,
                                   top_k: int, *, scale: float = 0.0, want_sel: bool = False,
-                                  out=None, sel=None, ws=None, stream=None):
+                                  out=None, sel=None, ws=None, stream=None, block: int = 128):
     """msa_sparse_attn_decode with the index-key cache in FP8: k_idx8 [B,Lmax,d_idx]
     uint8 E4M3 codes and k_idx_scale [B,Lmax] fp32 (stored key = scale * E4M3(code))."""
     _req(q, "q", torch.bfloat16)
@@ -409,7 +409,7 @@ def msa_sparse_attn_decode_fp8idx(q, q_idx, k_cache, v_cache, k_idx8, k_idx_scal
     _req(seq_lens, "seq_lens", torch.int32)
     B, H, d = q.shape
     Lmax, G = k_cache.shape[1], k_cache.shape[2]
-    p = make_params(B, Lmax, H, G, d, k_idx8.shape[2], 128, top_k, scale)
+    p = make_params(B, Lmax, H, G, d, k_idx8.shape[2], block, top_k, scale)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
@@ -425,7 +425,7 @@ def msa_sparse_attn_decode_fp8idx(q, q_idx, k_cache, v_cache, k_idx8, k_idx_scal
 
 def msa_sparse_attn_decode_fp8(q, q_idx, k8, k_scale, v8, v_scale, k_idx8, k_idx_scale,
                                seq_lens, top_k: int, *, scale: float = 0.0, want_sel: bool = False,
-                               out=None, sel=None, ws=None, stream=None):
+                               out=None, sel=None, ws=None, stream=None, block: int = 128):
     """Decode step with every cache in FP8: k8/v8 [B,Lmax,G,d] uint8 E4M3 with
     k_scale/v_scale [B,Lmax,G] fp32, k_idx8 [B,Lmax,d_idx] with k_idx_scale [B,Lmax]."""
     _req(q, "q", torch.bfloat16)
@@ -437,7 +437,7 @@ def msa_sparse_attn_decode_fp8(q, q_idx, k8, k_scale, v8, v_scale, k_idx8, k_idx
     _req(seq_lens, "seq_lens", torch.int32)
     B, H, d = q.shape
     Lmax, G = k8.shape[1], k8.shape[2]
-    p = make_params(B, Lmax, H, G, d, k_idx8.shape[2], 128, top_k, scale)
+    p = make_params(B, Lmax, H, G, d, k_idx8.shape[2], block, top_k, scale)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
@@ -467,7 +467,7 @@ def msa_quantize_e4m3_rows(x, *, codes=None, scale=None, stream=None):
 
 def msa_sparse_attn_decode_noalloc(q, q_idx, k_cache, v_cache, k_idx_cache, seq_lens, top_k: int, *,
                                    scale: float = 0.0, want_sel: bool = False, out=None, sel=None,
-                                   stream=None):
+                                   stream=None, block: int = 128):
     """Decode step that passes no workspace: the library uses its own 16 MiB
     device scratch (for callers that cannot allocate device memory at the
     call site).  Same arguments and results as msa_sparse_attn_decode.  Only
@@ -478,7 +478,7 @@ def msa_sparse_attn_decode_noalloc(q, q_idx, k_cache, v_cache, k_idx_cache, seq_
     _req(seq_lens, "seq_lens", torch.int32)
     B, H, d = q.shape
     Lmax, G = k_cache.shape[1], k_cache.shape[2]
-    p = make_params(B, Lmax, H, G, d, q_idx.shape[2], 128, top_k, scale)
+    p = make_params(B, Lmax, H, G, d, q_idx.shape[2], block, top_k, scale)
     if out is None:
         out = torch.empty_like(q)
     if sel is None and want_sel:

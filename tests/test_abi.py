@@ -53,7 +53,7 @@ def test_workspace_sizes(L, top_k, G, H, di):
 
 @pytest.mark.parametrize("field,value,code", [
     ("d", 64, M.MSA_ERR_UNSUPPORTED), ("d_idx", 96, M.MSA_ERR_UNSUPPORTED),
-    ("block", 64, M.MSA_ERR_UNSUPPORTED), ("top_k", 33, M.MSA_ERR_UNSUPPORTED),
+    ("block", 32, M.MSA_ERR_UNSUPPORTED), ("top_k", 33, M.MSA_ERR_UNSUPPORTED),
     ("top_k", 0, M.MSA_ERR_INVALID_ARG), ("L", -5, M.MSA_ERR_INVALID_ARG),
     ("H", 12, M.MSA_ERR_UNSUPPORTED), ("G", 3, M.MSA_ERR_INVALID_ARG),
     ("B", -1, M.MSA_ERR_INVALID_ARG), ("chunk", 100, M.MSA_ERR_INVALID_ARG),

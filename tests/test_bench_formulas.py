@@ -16,7 +16,7 @@ from block_sparse_long_08_b200 import inputs as I
 BLK = 128
 
 
-def _sel(L, G, top_k, seed):
+def _sel(L, G, top_k, seed, blk=BLK):
     """Selections of an N(0,1) problem, from the oracle (rows of every
     (query, group))."""
     x = I.prefill_inputs_small(1, L, G, G, 8, 8, seed)
@@ -24,39 +24,56 @@ def _sel(L, G, top_k, seed):
     sel = []
     for t in range(L):
         for g in range(G):
-            bs = O.block_scores_row(qi[0, t, g], ki[0], t, BLK)
-            sel.append((t, g, O.select_blocks_row(bs, t, BLK, top_k)))
+            bs = O.block_scores_row(qi[0, t, g], ki[0], t, blk)
+            sel.append((t, g, O.select_blocks_row(bs, t, blk, top_k)))
     return sel
 
 
-@pytest.mark.parametrize("L,G,H,top_k", [(1024, 2, 8, 4), (2048, 1, 4, 16), (1280, 2, 2, 3)])
-def test_prefill_formulas_match_row_counts(L, G, H, top_k):
+@pytest.mark.parametrize("L,G,H,top_k,blk", [(1024, 2, 8, 4, 128), (2048, 1, 4, 16, 128),
+                                             (1280, 2, 2, 3, 128), (1024, 2, 8, 8, 64),
+                                             (1000, 1, 4, 5, 64), (1100, 2, 4, 3, 128)])
+def test_prefill_formulas_match_row_counts(L, G, H, top_k, blk):
     d, d_idx = 128, 64
     r = H // G
-    sel = _sel(L, G, top_k, seed=L + top_k)
-    n_tok = {(t, g): len(O.selected_tokens(b, t, BLK)) for (t, g, b) in sel}
+    sel = _sel(L, G, top_k, seed=L + top_k, blk=blk)
+    n_tok = {(t, g): len(O.selected_tokens(b, t, blk)) for (t, g, b) in sel}
     entries = sum(len(b) for (_, _, b) in sel)
     # main branch: 2 products of 2d flops per (query, head, attended token)
     main = sum(H // G * 4.0 * d * n for n in n_tok.values())
-    assert bench.prefill_main_flops(1, L, H, d, top_k) == pytest.approx(main, rel=1e-12)
-    # backward: 5 products
-    assert bench.prefill_bwd_flops(1, L, H, d, top_k) == pytest.approx(main * 2.5, rel=1e-12)
+    assert bench.prefill_main_flops(1, L, H, d, top_k, blk) == pytest.approx(main, rel=1e-12)
     # forward attention bytes: per (query, group, block) entry, R q rows
     # gathered and R bf16 partial rows written and read back (+ fp32 lse
     # written and read); the merged output written once
     att = entries * r * (3 * d * 2 + 2 * 4) + L * H * d * 2
-    assert bench.prefill_attn_bytes(1, L, H, G, d, top_k) == pytest.approx(att, rel=1e-12)
-    # backward bytes: q and do gathered, bf16 dq partial written and read
-    # back, lse and D read, per entry row; o, do read and dq written per
-    # token; k, v read and dk, dv written once
-    bwd = entries * r * (2 * d * 2 + 2 * d * 2 + 8) + 3 * L * H * d * 2 + 4 * L * G * d * 2
-    assert bench.prefill_bwd_bytes(1, L, H, G, d, top_k) == pytest.approx(bwd, rel=1e-12)
-    # index: for every 128-query tile whose rows need scores (b_t >= top_k)
-    # and every earlier key tile, one 128 x 128 x d_idx product per group
-    nb = L // BLK
-    tiles = sum(1 for i in range(nb) for j in range(i) if i >= top_k)
-    idx = G * tiles * 2.0 * d_idx * BLK * BLK
-    assert bench.prefill_index_flops(1, L, G, d_idx, top_k) == pytest.approx(idx, rel=1e-12)
+    assert bench.prefill_attn_bytes(1, L, H, G, d, top_k, blk) == pytest.approx(att, rel=1e-12)
+    # index: every (query, group) row that chooses among its earlier blocks
+    # (b_t >= top_k) scores every token of those blocks, one d_idx dot
+    # product each (counted from the oracle's token scores of the row)
+    x = I.prefill_inputs_small(1, L, G, G, 8, 8, L + top_k)
+    scored = 0
+    for t in range(L):
+        bt = t // blk
+        if bt >= top_k:
+            scored += len(O.token_index_scores(O.as_f64(x["q_idx"][0, t, 0]),
+                                               O.as_f64(x["k_idx"][0, :bt * blk])))
+    assert bench.prefill_index_flops(1, L, G, d_idx, top_k, blk) == \
+        pytest.approx(G * 2.0 * d_idx * scored, rel=1e-12)
+    if blk == 128:
+        # the same count as 128 x 128 tiles: every 128-query tile whose rows
+        # need scores times every earlier key tile
+        nb = L // BLK
+        tiles = sum(1 for i in range(nb) for j in range(i) if i >= top_k)
+        full = (L % BLK == 0)
+        if full:
+            idx = G * tiles * 2.0 * d_idx * BLK * BLK
+            assert bench.prefill_index_flops(1, L, G, d_idx, top_k) == pytest.approx(idx, rel=1e-12)
+        # backward: 5 products per (query, head, attended token)
+        assert bench.prefill_bwd_flops(1, L, H, d, top_k) == pytest.approx(main * 2.5, rel=1e-12)
+        # backward bytes: q and do gathered, bf16 dq partial written and
+        # read back, lse and D read, per entry row; o, do read and dq written
+        # per token; k, v read and dk, dv written once
+        bwd = entries * r * (2 * d * 2 + 2 * d * 2 + 8) + 3 * L * H * d * 2 + 4 * L * G * d * 2
+        assert bench.prefill_bwd_bytes(1, L, H, G, d, top_k) == pytest.approx(bwd, rel=1e-12)
 
 
 def test_decode_bytes_match_token_counts():

@@ -30,14 +30,14 @@ def _sample_rows(L, n, seed, top_k, block=128):
 
 
 def _run_prefill(shape, x):
-    B, L, H, G, K = shape.B, shape.L, shape.H, shape.G, shape.top_k
-    p = M.make_params(B, L, H, G, 128, shape.d_idx, 128, K)
+    B, L, H, G, K, blk = shape.B, shape.L, shape.H, shape.G, shape.top_k, shape.block
+    p = M.make_params(B, L, H, G, 128, shape.d_idx, blk, K)
     ws_idx = M.new_workspace(p, M.MSA_OP_INDEX_SELECT, DEV)
     ws_att = M.new_workspace(p, M.MSA_OP_PREFILL_ATTN, DEV)
     sel = torch.empty((B, G, L, K), dtype=torch.int32, device=DEV)
     out = torch.empty_like(x["q"])
-    M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx)
-    M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att)
+    M.msa_index_select(x["q_idx"], x["k_idx"], K, sel=sel, ws=ws_idx, block=blk)
+    M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, out=out, ws=ws_att, block=blk)
     torch.cuda.synchronize()
     assert M.msa_read_status(ws_idx) == M.MSA_OK
     assert M.msa_read_status(ws_att) == M.MSA_OK
@@ -47,7 +47,7 @@ def _run_prefill(shape, x):
 def _check_prefill_rows(shape, x, sel, out, rows):
     cpu = {n: x[n][0].to("cpu") for n in ("k", "v", "k_idx")}
     k_idx64 = cpu["k_idx"].double().numpy()
-    G, r, K = shape.G, shape.H // shape.G, shape.top_k
+    G, r, K, blk = shape.G, shape.H // shape.G, shape.top_k, shape.block
     sc = 1.0 / np.sqrt(shape.d)
     q_rows = x["q"][0, rows].to("cpu")
     qi_rows = x["q_idx"][0, rows].to("cpu")
@@ -56,12 +56,13 @@ def _check_prefill_rows(shape, x, sel, out, rows):
     errs, swaps = [], 0
     for n, t in enumerate(rows):
         for g in range(G):
-            bs = O.block_scores_row(O.as_f64(qi_rows[n, g]), k_idx64, t, 128)
-            want = O.select_blocks_row(bs, t, 128, K)
-            exact = P.check_selection_row(sel_c[g, n], want + [-1] * (K - len(want)), bs, t, K)
+            bs = O.block_scores_row(O.as_f64(qi_rows[n, g]), k_idx64, t, blk)
+            want = O.select_blocks_row(bs, t, blk, K)
+            exact = P.check_selection_row(sel_c[g, n], want + [-1] * (K - len(want)), bs, t, K,
+                                          block=blk)
             swaps += 0 if exact else 1
             blocks = P.sel_set(sel_c[g, n])      # validated GPU selection
-            tok = torch.from_numpy(O.selected_tokens(blocks, t, 128))
+            tok = torch.from_numpy(O.selected_tokens(blocks, t, blk))
             o, _, _ = O.attend_rows(O.as_f64(q_rows[n, g * r:(g + 1) * r]), O.as_f64(cpu["k"][tok, g]),
                                     O.as_f64(cpu["v"][tok, g]), sc)
             errs.append(np.abs(out_c[n, g * r:(g + 1) * r] - o).ravel())
@@ -115,6 +116,16 @@ def test_prefill_32k():
     assert swaps <= 0.05 * len(rows) * shape.G
 
 
+def test_prefill_32k_block64():
+    """The 64-token block variant at the 2048-token budget (top_k = 32)."""
+    shape = I.PREFILL_32K_BLOCK64
+    x = I.prefill_inputs(shape, I.SEEDS["32k"], device=DEV)
+    sel, out = _run_prefill(shape, x)
+    rows = _sample_rows(shape.L, 48, 1, shape.top_k, block=64)
+    swaps = _check_prefill_rows(shape, x, sel, out, rows)
+    assert swaps <= 0.05 * len(rows) * shape.G
+
+
 def test_prefill_128k_planted():
     shape = I.PREFILL_128K_PLANTED
     x = I.prefill_inputs(shape, I.SEEDS["128k_planted"], device=DEV, needles=12, needle_alpha=3.0)
@@ -146,11 +157,27 @@ def test_decode_128k():
     _check_decode(dshape, y, out, sel)
 
 
+def _rows_per_chunk(shape, per_chunk, seed):
+    """Boundary rows plus per_chunk uniform rows inside every query chunk of
+    the prefill attention (msa_prefill_chunk_len), so that a fault confined
+    to one chunk of the 1M path shows."""
+    p = M.make_params(shape.B, shape.L, shape.H, shape.G, 128, shape.d_idx, 128, shape.top_k)
+    lc = M.msa_prefill_chunk_len(p)
+    rng = np.random.default_rng(seed)
+    rows = set(_sample_rows(shape.L, 0, seed, shape.top_k))
+    for c0 in range(0, shape.L, lc):
+        c1 = min(shape.L, c0 + lc)
+        rows |= {c0, c1 - 1}
+        rows |= set(rng.integers(c0, c1, size=per_chunk).tolist())
+    return sorted(rows), (shape.L + lc - 1) // lc
+
+
 def test_1m_prefill_and_decode():
     shape, dshape = I.PREFILL_1M, I.DECODE_1M
     x = I.prefill_inputs(shape, I.SEEDS["1m"], device=DEV)
     sel, out = _run_prefill(shape, x)
-    rows = _sample_rows(shape.L, 16, 4, shape.top_k)
+    rows, n_chunks = _rows_per_chunk(shape, 14, 4)
+    assert n_chunks >= 9 and len(rows) >= 128
     _check_prefill_rows(shape, x, sel, out, rows)
     del x, sel, out
     torch.cuda.empty_cache()
