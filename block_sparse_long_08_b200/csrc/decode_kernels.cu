@@ -64,37 +64,56 @@ __device__ __forceinline__ void griddep_wait() {
 // Called by every CTA of decode_attn_kernel once its partial (or, for an
 // unused slot, its -inf lse) is written.  The last of the top_k CTAs of
 // (sequence b, group g) to get here merges the slot partials of the group's
-// R heads: o = sum_s exp(lse_s - M) o_s / sum_s exp(lse_s - M), M = max lse_s,
-// thread x taking column x of each head.  The ticket counters are zeroed by
-// decode_topk_kernel.
+// R heads: o = sum_s exp(lse_s - M) o_s / sum_s exp(lse_s - M), M = max lse_s.
+// Warp w takes heads w, w+4, ...: lane s holds lse_s, and each lane merges
+// four columns, with the slots' loads issued 16 at a time before any sum
+// (this merge ends the decode step, so its latency is on the critical
+// path).  The ticket counters are zeroed by decode_topk_kernel.
 template <int R>
 __device__ __forceinline__ void dec_merge_if_last(const DecodeArgs &a, int b, int g) {
   __shared__ int s_last;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   __threadfence();   // this CTA's partial, visible before its ticket
   __syncthreads();
   if (tid == 0) s_last = (atomicAdd(&a.tickets[b * a.G + g], 1) == a.top_k - 1);
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-#pragma unroll 1
-  for (int hh = 0; hh < R; ++hh) {
+  for (int hh = warp; hh < R; hh += 4) {
     const size_t p0 = (size_t(b) * a.H + size_t(g) * R + hh) * a.top_k;
-    float M = -INFINITY;
-    for (int s = 0; s < a.top_k; ++s) M = fmaxf(M, __ldcg(a.part_lse + p0 + s));
-    float acc = 0.f, wsum = 0.f;
-    if (M > -INFINITY) {
-      for (int s = 0; s < a.top_k; ++s) {
-        const float ls = __ldcg(a.part_lse + p0 + s);
-        if (ls == -INFINITY) continue;
-        const float w = __expf(ls - M);
-        wsum += w;
-        acc = fmaf(w, __ldcg(a.part_o + (p0 + s) * kHeadDim + tid), acc);
+    const float my = lane < a.top_k ? __ldcg(a.part_lse + p0 + lane) : -INFINITY;
+    float M = my;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float wm = (my > -INFINITY) ? __expf(my - M) : 0.f;
+    float wsum = wm;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < a.top_k; s0 += 16) {
+      float4 v[16];
+#pragma unroll
+      for (int s = 0; s < 16; ++s)
+        v[s] = (s0 + s < a.top_k)
+                   ? __ldcg(reinterpret_cast<const float4 *>(a.part_o + (p0 + s0 + s) * kHeadDim) + lane)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int s = 0; s < 16; ++s) {
+        const float w = __shfl_sync(0xffffffffu, wm, (s0 + s) & 31);
+        if (s0 + s < a.top_k && w > 0.f) {
+          acc.x = fmaf(w, v[s].x, acc.x);
+          acc.y = fmaf(w, v[s].y, acc.y);
+          acc.z = fmaf(w, v[s].z, acc.z);
+          acc.w = fmaf(w, v[s].w, acc.w);
+        }
       }
     }
-    const float o = wsum > 0.f ? acc * (1.f / wsum) : 0.f;
-    a.out[(size_t(b) * a.H + size_t(g) * R + hh) * kHeadDim + tid] =
-        __bfloat16_as_ushort(__float2bfloat16_rn(o));
+    const float inv = (M > -INFINITY && wsum > 0.f) ? 1.f / wsum : 0.f;
+    uint2 r;
+    r.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    r.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2 *>(a.out + (size_t(b) * a.H + size_t(g) * R + hh) * kHeadDim +
+                               lane * 4) = r;
   }
 }
 

@@ -12,7 +12,9 @@ namespace {
 
 // Rows of up to 256 candidate blocks (query positions below 32,896 with
 // 128-token blocks) take the threshold form with the row in registers;
-// longer rows take the insertion scan.
+// longer rows take the insertion scan.  (Four rows per warp with their
+// networks interleaved measured slower: the extra registers cost more
+// occupancy than the independent chains recovered.)
 constexpr int kTopkVpl = 8;
 
 __global__ void __launch_bounds__(256) msa_topk_kernel(const TopkArgs a) {
