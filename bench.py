@@ -353,9 +353,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the tiny / 32K / 128K-planted prefill legs")
-    ap.add_argument("--workload", default="1m", choices=["1m", "128k", "32k", "8k"],
+    ap.add_argument("--workload", default="1m", choices=["1m", "512k", "128k", "32k", "8k"],
                     help="prefill length of the step (1m is the headline workload; 8k is a "
-                         "small-footprint case for profiler captures)")
+                         "small-footprint case for profiler captures, 512k the smallest "
+                         "whose index keys (134 MB) exceed the 126 MB L2)")
     ap.add_argument("--op", default="step",
                     choices=["step", "index", "scores", "attn", "decode", "decode8", "cached",
                              "bwd"],
@@ -371,6 +372,10 @@ def main():
 
     if args.workload == "1m":
         shape, dshape, seed = I.PREFILL_1M, I.DECODE_1M, I.SEEDS["1m"]
+    elif args.workload == "512k":
+        import dataclasses
+        shape, dshape, seed = (dataclasses.replace(I.PREFILL_1M, L=524288), I.DECODE_128K,
+                               I.SEEDS["1m"])
     elif args.workload == "128k":
         shape, dshape, seed = I.PREFILL_128K_PLANTED, I.DECODE_128K, I.SEEDS["128k_planted"]
     elif args.workload == "32k":

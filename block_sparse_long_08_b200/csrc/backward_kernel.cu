@@ -12,7 +12,10 @@
 // Organised key-block-outer, on the forward's reverse index: one unit =
 // one (b, g, key block j) with every (query, slot) that selected j, taken
 // whole by one CTA so that dK_j and dV_j accumulate in TMEM and are written
-// once, without atomics.  A unit's queries are processed as 128-row items
+// once, without atomics.  The key tile is 128 rows: a 128-token block fills
+// it, a 64-token block fills its first half (the other keys are masked out
+// of P and dZ, so their dK/dV rows stay zero and are not written), and the
+// block that holds a sequence's last key loads zeros past it.  A unit's queries are processed as 128-row items
 // (128/R queries x R heads), as in the forward:
 //   gather   q and do rows of the item (cp.async, 128B-swizzled K-major)
 //   S  = Q K_j^T, dP = dO V_j^T          (UMMA, fp32 in TMEM cols 0-255)
@@ -94,7 +97,7 @@ struct Unit {
   int bgj, b, g, j, l_lo, n_q;
 };
 
-template <int R>
+template <int R, int BLK>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     msa_backward_kernel(const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const BwdArgs a) {
@@ -125,10 +128,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     *abort_flag = 0;
     mbar_init_fence();
   }
-  // padding rows of a partial item keep whatever the buffers held; start
-  // from zeros so that they are finite (their P and dZ are 0)
-  for (int x = tid; x < 2 * kTileB / 16; x += kBwdThreads)
-    reinterpret_cast<uint4 *>(smem + kSQ)[x] = make_uint4(0u, 0u, 0u, 0u);
+  // padding rows of a partial item, and with 64-key blocks key rows 64..127
+  // of the K/V tiles, keep whatever the buffers held; start from zeros so
+  // that they are finite (their P and dZ are 0)
+  for (int x = tid; x < 4 * kTileB / 16; x += kBwdThreads)
+    reinterpret_cast<uint4 *>(smem + kSK)[x] = make_uint4(0u, 0u, 0u, 0u);
   if (warp == 0) {
     tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
@@ -162,22 +166,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       un.n_q = a.list_off[un.bgj + 1] - un.l_lo;
       if (un.n_q > 0) return true;
       if (a.acc_dk && !a.last) continue;   // an earlier or later chunk writes this block
-      const size_t r0 = ((size_t(un.b) * a.L + size_t(un.j) * kBlock + row) * a.G + un.g) *
-                            kHeadDim + half * 64;
-      put_grad32(nullptr, 0.f, r0, a.dk, a.acc_dk, a.last);
-      put_grad32(nullptr, 0.f, r0 + 32, a.dk, a.acc_dk, a.last);
-      put_grad32(nullptr, 0.f, r0, a.dv, a.acc_dv, a.last);
-      put_grad32(nullptr, 0.f, r0 + 32, a.dv, a.acc_dv, a.last);
+      const int key = un.j * BLK + row;
+      if (row < BLK && key < a.L) {
+        const size_t r0 = ((size_t(un.b) * a.L + key) * a.G + un.g) * kHeadDim + half * 64;
+        put_grad32(nullptr, 0.f, r0, a.dk, a.acc_dk, a.last);
+        put_grad32(nullptr, 0.f, r0 + 32, a.dk, a.acc_dk, a.last);
+        put_grad32(nullptr, 0.f, r0, a.dv, a.acc_dv, a.last);
+        put_grad32(nullptr, 0.f, r0 + 32, a.dv, a.acc_dv, a.last);
+      }
     }
   };
-  // K_j and V_j of a unit into their tiles (thread 0)
+  // K_j and V_j of a unit into their tiles (thread 0): BLK key rows, the
+  // maps' row extent ending at the sequence's last key (rows past it load
+  // as zeros)
   auto load_kv = [&](const Unit &un) {
-    const int z = un.b * a.L + un.j * kBlock;
-    mbar_arrive_expect_tx(bar(kBarKv), 2 * kTileB);
-    tma_load_3d(s_base + kSK, &tm_k, bar(kBarKv), 0, un.g, z);
-    tma_load_3d(s_base + kSK + 16384, &tm_k, bar(kBarKv), 64, un.g, z);
-    tma_load_3d(s_base + kSV, &tm_v, bar(kBarKv), 0, un.g, z);
-    tma_load_3d(s_base + kSV + 16384, &tm_v, bar(kBarKv), 64, un.g, z);
+    const int z = un.j * BLK;
+    mbar_arrive_expect_tx(bar(kBarKv), 4u * BLK * 128u);
+    tma_load_4d(s_base + kSK, &tm_k, bar(kBarKv), 0, un.g, z, un.b);
+    tma_load_4d(s_base + kSK + 16384, &tm_k, bar(kBarKv), 64, un.g, z, un.b);
+    tma_load_4d(s_base + kSV, &tm_v, bar(kBarKv), 0, un.g, z, un.b);
+    tma_load_4d(s_base + kSV + 16384, &tm_v, bar(kBarKv), 64, un.g, z, un.b);
   };
   // Query positions of this thread's eight gather rows of item `it` of a
   // unit (-1 past the item's end): row pairs p = warp + 8 i (rows 2p, 2p+1).
@@ -240,7 +248,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const size_t ri = (size_t(cur.b) * a.L + t) * a.H + cur.g * R + row % R;
       lse2 = a.lse[ri] * log2e;
       dlt = a.delta[ri];
-      lim = min(kBlock - 1, t - cur.j * kBlock);
+      lim = min(BLK - 1, t - cur.j * BLK);
     }
     // the next item's gather rows, when it belongs to this unit: loaded now,
     // their latency hides behind this item's products
@@ -387,14 +395,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     // ---- unit end: dK_j (* scale) and dV_j rows (key = TMEM lane) as bf16
     if (unit_end) {
-      const size_t r0 = ((size_t(cur.b) * a.L + size_t(cur.j) * kBlock + row) * a.G + cur.g) *
-                            kHeadDim + half * 64;
+      const int key = cur.j * BLK + row;
+      const bool own = row < BLK && key < a.L;   // TMEM lanes of this block's keys
+      const size_t r0 = ((size_t(cur.b) * a.L + key) * a.G + cur.g) * kHeadDim + half * 64;
 #pragma unroll 1
       for (int m = 0; m < 2; ++m) {
-        float x0[32], x1[32];
+        float x0[32], x1[32];   // (the loads are warp-wide: every lane takes part)
         tmem_ld32(tm_row + (m ? kTmDK : kTmDV) + half * 64, x0);
         tmem_ld32(tm_row + (m ? kTmDK : kTmDV) + half * 64 + 32, x1);
         tmem_wait_ld();
+        if (!own) continue;
         const float f = m ? a.scale : 1.f;
         uint16_t *out = m ? a.dk : a.dv;
         float *acc = m ? a.acc_dk : a.acc_dv;
@@ -489,7 +499,7 @@ __global__ void __launch_bounds__(256) bwd_dq_reduce_kernel(const BwdArgs a) {
 template <int R>
 cudaError_t launch_bwd_r(const CUtensorMap &tk, const CUtensorMap &tv, const BwdArgs &a,
                          int num_sms, cudaStream_t st) {
-  auto kern = msa_backward_kernel<R>;
+  auto kern = a.blk == 64 ? msa_backward_kernel<R, 64> : msa_backward_kernel<R, 128>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwdSmem);
   if (e != cudaSuccess) return e;
   const int n_units = a.B * a.G * a.nb;

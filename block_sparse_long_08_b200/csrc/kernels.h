@@ -85,9 +85,13 @@ struct RevIdxArgs {
   int32_t *item_off;            // [B*G*nb + 1]
   int32_t *list;                // [G*Rc*top_k]: t * 32 + slot
   int32_t *pos_of;              // [G][Rc][top_k]: rank in its block's list, then list position
+  // > 0: sort every list by query position (run-to-run stable order);
+  // ceil(rows / 32) for the most rows one sequence has in a chunk
+  int order_words;
   int *status;
 };
 cudaError_t launch_revidx(const RevIdxArgs &a, cudaStream_t st);
+size_t revidx_order_smem(int order_words);   // shared memory of the ordering step
 
 struct AttnArgs {
   int L, H, G, nb, top_k;      // L: key rows per sequence
@@ -132,6 +136,7 @@ cudaError_t launch_combine(const CombineArgs &a, cudaStream_t st);
 // over that chunk's reverse index.
 struct BwdArgs {
   int B, L, H, G, nb, top_k;
+  int blk;                     // block length: 128 or 64
   int r0, Rc;
   int last;                    // the last query chunk (writes dk, dv when chunked)
   float scale, scale_log2;

@@ -39,9 +39,8 @@ size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---- shape checks ---------------------------------------------------------
-// whole_blocks: the operation needs L to be a multiple of the block length
-// (the backward); the prefill and decode paths take any length.
-int check_params(const msa_params *p, bool decode, bool whole_blocks = false) {
+// Every operation takes any sequence length and either block length.
+int check_params(const msa_params *p, bool decode) {
   if (!p) return fail(MSA_ERR_INVALID_ARG, "params is NULL");
   if (p->B < 0 || p->L < 0 || p->H <= 0 || p->G <= 0 || p->d <= 0 || p->d_idx <= 0 ||
       p->block <= 0 || p->top_k <= 0)
@@ -59,10 +58,6 @@ int check_params(const msa_params *p, bool decode, bool whole_blocks = false) {
   const int r = p->H / p->G;
   if (r != 1 && r != 2 && r != 4 && r != 8 && r != 16)
     return fail(MSA_ERR_UNSUPPORTED, "H/G=%d (supported: 1,2,4,8,16)", r);
-  if (whole_blocks && p->L % 128 != 0)
-    return fail(MSA_ERR_UNSUPPORTED, "L=%d: this operation needs a multiple of 128", p->L);
-  if (whole_blocks && p->block != 128)
-    return fail(MSA_ERR_UNSUPPORTED, "block=%d: this operation needs 128-token blocks", p->block);
   if (decode && p->G > 8) return fail(MSA_ERR_UNSUPPORTED, "decode supports G <= 8 (G=%d)", p->G);
   if ((long long)p->B * p->L > (1LL << 26))
     return fail(MSA_ERR_UNSUPPORTED, "B*L=%lld above 2^26", (long long)p->B * p->L);
@@ -131,10 +126,15 @@ struct BwdWs {
   size_t cnt, list_off, item_off, list, pos_of, delta, part_dq, acc_dk, acc_dv, end;
   int Rc;
 };
+// At most 2^19 rows per chunk: the reverse index's ordering step keeps a
+// bitmap of one sequence's rows in a chunk, and its prefix counts, in
+// shared memory (128 KiB at that bound).
+constexpr int kBwdMaxChunkRows = 1 << 19;
 BwdWs bwd_ws(const msa_params *p) {
   BwdWs w;
   const long long n_rows = (long long)p->B * p->L;
   w.Rc = prefill_chunk(p, n_rows);
+  if (w.Rc > kBwdMaxChunkRows) w.Rc = kBwdMaxChunkRows;
   const size_t nbgj = size_t(p->B) * p->G * nblocks(p);
   const size_t entries = size_t(p->G) * w.Rc * p->top_k;
   size_t o = msa::kWsHeader;
@@ -382,6 +382,7 @@ int run_attn_chunk(const msa_params *p, const AttnPlan &pl, const msa_bf16 *q, c
   msa::RevIdxArgs ra;
   ra.G = p->G; ra.nb = pl.nb; ra.top_k = p->top_k; ra.qpi = pl.qpi;
   ra.q = pl.qg;
+  ra.order_words = 0;   // attention partials are merged in slot order: any list order
   ra.r0 = r0; ra.Rc = Rc;
   ra.sel = sel;
   ra.cnt = reinterpret_cast<int32_t *>(wsb + w.cnt);
@@ -586,7 +587,7 @@ const char *msa_version(void) { return "msa-b200 0.1 (sm_100a)"; }
 
 size_t msa_workspace_bytes(const msa_params *p, int op) {
   g_err[0] = 0;
-  if (check_params(p, op == MSA_OP_DECODE, op == MSA_OP_BACKWARD) != MSA_OK) return 0;
+  if (check_params(p, op == MSA_OP_DECODE) != MSA_OK) return 0;
   switch (op) {
     case MSA_OP_INDEX_SELECT: return msa::kWsHeader;
     case MSA_OP_PREFILL_ATTN: return attn_ws(p, msa::kWsHeader).end;
@@ -881,7 +882,7 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
                              msa_bf16 *dk, msa_bf16 *dv, void *ws, size_t ws_bytes,
                              msa_stream stream) {
   g_err[0] = 0;
-  int rc = check_params(p, false, true);
+  int rc = check_params(p, false);
   if (rc) return rc;
   if (p->B == 0 || p->L == 0) return MSA_OK;
   if (!q || !k || !v || !out || !lse || !dout || !sel || !dq || !dk || !dv)
@@ -898,18 +899,13 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
   if (rc) return rc;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
-  const int nb = p->L / 128;
+  const int nb = nblocks(p);
   const int N = p->B * p->L;
   CUtensorMap tk, tv;
-  {
-    const uint64_t dims[3] = {uint64_t(p->d), uint64_t(p->G), uint64_t(N)};
-    const uint64_t str[2] = {uint64_t(p->d) * 2, uint64_t(p->d) * 2 * p->G};
-    const uint32_t box[3] = {64, 1, 128};
-    rc = make_tmap(&tk, k, 3, dims, str, box);
-    if (rc) return rc;
-    rc = make_tmap(&tv, v, 3, dims, str, box);
-    if (rc) return rc;
-  }
+  rc = make_kv_tmap(&tk, k, p, p->L, p->B);
+  if (rc) return rc;
+  rc = make_kv_tmap(&tv, v, p, p->L, p->B);
+  if (rc) return rc;
   msa::RevIdxArgs ra;
   ra.G = p->G; ra.nb = nb; ra.top_k = p->top_k;
   ra.qpi = 128 / (p->H / p->G);
@@ -920,9 +916,12 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
   ra.item_off = reinterpret_cast<int32_t *>(wsb + w.item_off);
   ra.list = reinterpret_cast<int32_t *>(wsb + w.list);
   ra.pos_of = reinterpret_cast<int32_t *>(wsb + w.pos_of);
+  // lists in query order: dk and dv sum a block's items in a fixed order
+  ra.order_words = ((w.Rc < p->L ? w.Rc : p->L) + 31) / 32;
   ra.status = status_ptr(ws);
   msa::BwdArgs a;
   a.B = p->B; a.L = p->L; a.H = p->H; a.G = p->G; a.nb = nb; a.top_k = p->top_k;
+  a.blk = p->block;
   a.scale = eff_scale(p);
   a.scale_log2 = a.scale * 1.4426950408889634f;
   a.q = q; a.out = out; a.dout = dout; a.lse = lse; a.sel = sel;

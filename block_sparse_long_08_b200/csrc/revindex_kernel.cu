@@ -17,6 +17,15 @@
 //              a list is whatever order the count's atomics produced, and
 //              each (t, slot) partial is computed independently of the
 //              others in its tile.
+//   4. order   (when order_words > 0) each list sorted by query position,
+//              so that the order -- and whatever is summed in it -- is the
+//              same from run to run; pos_of follows.  A row selects a block
+//              at most once, so the positions in a list are distinct and an
+//              entry's rank is the number of smaller positions: counted
+//              directly in shared memory for lists of up to kOrderDirect
+//              entries, read from a bitmap over the sequence's rows in the
+//              chunk (and per-word prefix counts) for longer ones, the slot
+//              then found in the row's selection.
 // Every work item then holds <= qpi queries, so items cost the same and a
 // persistent grid balances itself whatever the causal skew between early
 // and late key blocks.
@@ -148,7 +157,118 @@ __global__ void __launch_bounds__(256) revidx_fill_kernel(const RevIdxArgs a) {
   }
 }
 
+constexpr int kOrderDirect = 2048;
+constexpr int kOrderThreads = 256;
+
+// Exclusive prefix of x over the CTA's 256 threads; tot gets the sum (all
+// threads).  warp_sums and total are shared scratch.
+__device__ __forceinline__ int cta_exclusive_scan(int x, int *warp_sums, int *total, int &tot) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int v = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  if (lane == 31) warp_sums[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kOrderThreads / 32 ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < kOrderThreads / 32) warp_sums[lane] = w;
+    if (lane == kOrderThreads / 32 - 1) *total = w;
+  }
+  __syncthreads();
+  const int ex = v - x + (warp > 0 ? warp_sums[warp - 1] : 0);
+  tot = *total;
+  __syncthreads();   // warp_sums / total are rewritten by the next call
+  return ex;
+}
+
+// Entry (t, slot) of list (b, g) now at list position pos: pos_of follows.
+__device__ __forceinline__ void order_put(const RevIdxArgs &a, const int4 &s, int g, int x,
+                                          int pos) {
+  a.list[pos] = x;
+  const int rl = s.x + ((x >> 5) - s.y) - a.r0;   // the row's index in the chunk
+  a.pos_of[((long long)g * a.Rc + rl) * a.top_k + (x & 31)] = pos;
+}
+
+__global__ void __launch_bounds__(kOrderThreads) revidx_order_kernel(const RevIdxArgs a) {
+  extern __shared__ int sm[];   // kOrderDirect entries, or bitmap + prefix words
+  __shared__ int warp_sums[32], total;
+  const int n_lists = a.q.B * a.G * a.nb;
+  const int tid = threadIdx.x;
+  for (int bgj = blockIdx.x; bgj < n_lists; bgj += gridDim.x) {
+    const int lo = a.list_off[bgj], n = a.list_off[bgj + 1] - lo;
+    if (n <= 1) continue;   // the same for every thread of the CTA
+    const int b = bgj / (a.G * a.nb), g = (bgj / a.nb) % a.G, j = bgj % a.nb;
+    const int4 s = qgeo_seq(a.q, b);
+    if (n <= kOrderDirect) {
+      for (int i = tid; i < n; i += kOrderThreads) sm[i] = a.list[lo + i];
+      __syncthreads();
+      for (int i = tid; i < n; i += kOrderThreads) {
+        const int x = sm[i];
+        int rank = 0;
+        for (int m = 0; m < n; ++m) rank += sm[m] < x;
+        order_put(a, s, g, x, lo + rank);
+      }
+      __syncthreads();
+      continue;
+    }
+    // the sequence's rows in this chunk: positions [t_first, t_first + rows)
+    const int r_first = max(a.r0, s.x);
+    const int rows = min(a.r0 + a.Rc, s.x + s.z) - r_first;
+    const int t_first = s.y + (r_first - s.x);
+    const int nw = (rows + 31) >> 5;   // <= order_words (host bound)
+    uint32_t *bits = reinterpret_cast<uint32_t *>(sm);
+    int *pre = sm + a.order_words;
+    for (int w = tid; w < nw; w += kOrderThreads) bits[w] = 0u;
+    __syncthreads();
+    for (int i = tid; i < n; i += kOrderThreads) {
+      const int u = (a.list[lo + i] >> 5) - t_first;
+      atomicOr(&bits[u >> 5], 1u << (u & 31));
+    }
+    __syncthreads();
+    int carry = 0;
+    for (int base = 0; base < nw; base += kOrderThreads) {
+      const int w = base + tid;
+      const int c = w < nw ? __popc(bits[w]) : 0;
+      int tile_total;
+      const int ex = cta_exclusive_scan(c, warp_sums, &total, tile_total);
+      if (w < nw) pre[w] = carry + ex;
+      carry += tile_total;
+    }
+    __syncthreads();
+    for (int w = tid; w < nw; w += kOrderThreads) {
+      uint32_t m = bits[w];
+      int pos = lo + pre[w];
+      while (m) {
+        const int bit = __ffs(m) - 1;
+        m &= m - 1;
+        const int t = t_first + w * 32 + bit;
+        const long long srow =
+            ((long long)s.w + (long long)g * a.q.sel_gs + (t - s.y)) * a.top_k;
+        int slot = 0;
+        for (int k = 0; k < a.top_k; ++k)
+          if (a.sel[srow + k] == j) slot = k;
+        order_put(a, s, g, t * 32 + slot, pos++);
+      }
+    }
+    __syncthreads();
+  }
+}
+
 }  // namespace
+
+size_t revidx_order_smem(int order_words) {
+  const size_t direct = sizeof(int) * kOrderDirect;
+  const size_t bitmap = sizeof(int) * 2 * size_t(order_words);
+  return direct > bitmap ? direct : bitmap;
+}
 
 cudaError_t launch_revidx(const RevIdxArgs &a, cudaStream_t st) {
   const int n_cnt = a.q.B * a.G * a.nb;
@@ -159,6 +279,14 @@ cudaError_t launch_revidx(const RevIdxArgs &a, cudaStream_t st) {
   if (n > 0) revidx_count_kernel<<<grid, 256, 0, st>>>(a);
   revidx_scan_kernel<<<1, 1024, 0, st>>>(a);
   if (n > 0) revidx_fill_kernel<<<grid, 256, 0, st>>>(a);
+  if (n > 0 && a.order_words > 0) {
+    const size_t smem = revidx_order_smem(a.order_words);
+    e = cudaFuncSetAttribute(revidx_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    const int og = n_cnt < 148 * 8 ? n_cnt : 148 * 8;
+    revidx_order_kernel<<<og, kOrderThreads, smem, st>>>(a);
+  }
   return cudaGetLastError();
 }
 

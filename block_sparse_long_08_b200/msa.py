@@ -212,10 +212,12 @@ def msa_sparse_attn_prefill(q, k, v, sel, *, scale: float = 0.0, want_lse: bool 
 
 
 def msa_sparse_attn_backward(q, k, v, out, lse, dout, sel, *, scale: float = 0.0, dq=None,
-                             dk=None, dv=None, ws=None, stream=None, chunk: int = 0):
+                             dk=None, dv=None, ws=None, stream=None, chunk: int = 0,
+                             block: int = 128):
     """Main-branch gradients for a fixed selection: q [B,L,H,d], k/v
     [B,L,G,d], the forward's out [B,L,H,d] and lse [B,L,H] fp32, dout
-    [B,L,H,d], sel [B,G,L,top_k] -> (dq, dk, dv) bf16, shaped like q, k, v."""
+    [B,L,H,d], sel [B,G,L,top_k] (block ids of `block` tokens) -> (dq, dk,
+    dv) bf16, shaped like q, k, v."""
     for n, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
         _req(t, n, torch.bfloat16)
     _req(lse, "lse", torch.float32)
@@ -223,7 +225,7 @@ def msa_sparse_attn_backward(q, k, v, out, lse, dout, sel, *, scale: float = 0.0
     B, L, H, d = q.shape
     G = k.shape[2]
     top_k = sel.shape[3]
-    p = make_params(B, L, H, G, d, 128, 128, top_k, scale, chunk)
+    p = make_params(B, L, H, G, d, 128, block, top_k, scale, chunk)
     dev = q.device
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk

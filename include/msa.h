@@ -51,10 +51,10 @@
  *     out, an out-of-range decode length) are recorded in a status word at
  *     the start of `ws`; msa_read_status() synchronises the stream and
  *     returns/clears it.
- *   - Supported: d == 128, d_idx in {64, 128}, block == 128,
+ *   - Supported: d == 128, d_idx in {64, 128}, block in {64, 128},
  *     1 <= top_k <= 32, H % G == 0 with H/G in {1,2,4,8,16}, B*L <= 2^26.
- *     Any L: the last block of a sequence may be partial (nb = ceil(L/128)
- *     blocks); only the backward needs L % 128 == 0.  The decode entry
+ *     Any L: the last block of a sequence may be partial (nb =
+ *     ceil(L/block) blocks), in every operation.  The decode entry
  *     points also need G <= 8 (the cache scan scores all groups of a key in
  *     one 8-column tensor-core product).
  *     Other shapes give MSA_ERR_UNSUPPORTED.  B == 0 or L == 0 is a no-op.
@@ -79,7 +79,7 @@ typedef struct msa_params {
   int32_t G;       /* GQA groups = KV heads = index queries per token */
   int32_t d;       /* head dim of q/k/v (128) */
   int32_t d_idx;   /* index dim of q_idx/k_idx (64 or 128) */
-  int32_t block;   /* KV block length (128) */
+  int32_t block;   /* KV block length: 128 (the pages' size) or 64 */
   int32_t top_k;   /* blocks kept per (query, group), local block included */
   float scale;     /* softmax scale of the main branch; 0 -> 1/sqrt(d) */
   int32_t chunk;   /* query rows per chunk of the prefill attention and the
@@ -125,7 +125,7 @@ int msa_index_select(const msa_params *p, const msa_bf16 *q_idx, const msa_bf16 
 /* Main Branch, prefill (explainer §2.2; researchpapers.dev "机制").
  *   q [B,L,H,d], k [B,L,G,d], v [B,L,G,d] bf16                      (in)
  *   sel [B,G,L,top_k] int32: any selection in the layout above: valid
- *     ids first (any order, each < L/block, each block at most once, the
+ *     ids first (any order, each < nb, each block at most once, the
  *     query's own block included for a causal result), -1 padding.   (in)
  *   out [B,L,H,d] bf16                                              (out)
  *   lse [B,L,H] fp32 natural-log softmax normaliser, or NULL         (out)
@@ -319,11 +319,14 @@ int msa_forward_host(const msa_params *p, const msa_bf16 *q_h, const msa_bf16 *k
  * For each (t, h) with probabilities P over its attended tokens s:
  * dZ_s = P_s (do . v_s - do . o), dq = scale sum_s dZ_s k_s, and every
  * attended token gets dk_s += scale dZ_s q, dv_s += P_s do; tokens no query
- * attends to get zero.  dq is bit-identical from run to run; dk and dv sum
- * a key block's queries in the reverse index's list order, which follows
- * atomics, so runs agree up to fp32 summation order.
- * Needs L % 128 == 0.  Queries are processed in the prefill's chunks of
- * packed rows (msa_prefill_chunk_len; p->chunk overrides it), each with its
+ * attends to get zero.  dq, dk and dv are bit-identical from run to run:
+ * dq sums a row's slots in slot order, and dk and dv sum a key block's
+ * queries in query order (the reverse index's lists are sorted).
+ * Any L and either block length: the block that holds a sequence's last
+ * key is partial, and a 64-token block fills half of the kernel's 128-key
+ * tile (the other half is masked out).  Queries are processed in the
+ * prefill's chunks of packed rows (msa_prefill_chunk_len; p->chunk
+ * overrides it), at most 2^19 rows each, each with its
  * own reverse index and one bf16 dq partial row per (query, head, slot) of
  * the chunk (at most about 16 GiB).
  * With more than one chunk, dk and dv are summed across chunks in fp32

@@ -232,17 +232,17 @@ def test_backward_workspace_follows_chunking():
     assert M.msa_prefill_chunk_len(M.make_params(1, L, H, G, top_k=K, chunk=L // 2)) == L // 2
 
 
-def test_any_length_except_backward():
+def test_any_length_and_either_block_in_every_operation():
     """L need not be a multiple of the block length: the last block of a
-    sequence is partial.  Only the backward keeps L % 128 == 0."""
+    sequence is partial.  Every operation takes 64- and 128-token blocks."""
     lib = M.lib()
     for L in (1, 127, 1000, 2049):
-        p = M.make_params(2, L, 16, 4, 128, 128, 128, 5)
-        for op in (M.MSA_OP_INDEX_SELECT, M.MSA_OP_PREFILL_ATTN, M.MSA_OP_DECODE, M.MSA_OP_FORWARD,
-                   M.MSA_OP_FORWARD_VARLEN):
-            assert lib.msa_workspace_bytes(ctypes.byref(p), op) > 0, (L, op, M.msa_last_error())
-        assert lib.msa_workspace_bytes(ctypes.byref(p), M.MSA_OP_BACKWARD) == 0
-        assert "multiple of 128" in M.msa_last_error()
+        for blk in (64, 128):
+            p = M.make_params(2, L, 16, 4, 128, 128, blk, 5)
+            for op in (M.MSA_OP_INDEX_SELECT, M.MSA_OP_PREFILL_ATTN, M.MSA_OP_DECODE,
+                       M.MSA_OP_FORWARD, M.MSA_OP_FORWARD_VARLEN, M.MSA_OP_BACKWARD):
+                assert lib.msa_workspace_bytes(ctypes.byref(p), op) > 0, (L, blk, op,
+                                                                         M.msa_last_error())
     # the ragged-batch workspace holds the uniform forward's plus its tables
     p = M.make_params(4, 4096, 16, 4, 128, 128, 128, 8)
     assert (M.msa_workspace_bytes(p, M.MSA_OP_FORWARD_VARLEN)

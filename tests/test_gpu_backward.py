@@ -43,13 +43,15 @@ def _inputs(shape, seed):
     return x
 
 
-def _forward_backward(x, top_k, sel=None):
+def _forward_backward(x, top_k, sel=None, block=128, chunk=0):
     if sel is None:
         out, sel, lse = M.msa_forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], top_k,
-                                      want_sel=True, want_lse=True)
+                                      want_sel=True, want_lse=True, block=block)
     else:
-        out, lse = M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, want_lse=True)
-    dq, dk, dv = M.msa_sparse_attn_backward(x["q"], x["k"], x["v"], out, lse, x["dout"], sel)
+        out, lse = M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, want_lse=True,
+                                             block=block)
+    dq, dk, dv = M.msa_sparse_attn_backward(x["q"], x["k"], x["v"], out, lse, x["dout"], sel,
+                                            block=block, chunk=chunk)
     torch.cuda.synchronize()
     return sel, dq, dk, dv
 
@@ -88,21 +90,26 @@ def test_backward_blocks_nobody_selects_get_zero():
     _grad_close("dv", P.f64(dv), ref["dv"])
 
 
-def test_backward_run_to_run():
+@pytest.mark.parametrize("L,top_k,chunk", [(2048, 5, 0), (2048, 5, 640), (2304, 18, 0)])
+def test_backward_run_to_run(L, top_k, chunk):
     """dq rows are each computed from their own (query, slot) rows and summed
-    in slot order: bit-identical across runs.  dk and dv sum a key block's
-    items in the order of the reverse index's lists, which follows the
-    count's atomics, so two runs agree up to fp32 summation order."""
-    shape = I.PrefillShape(B=1, L=2048, H=16, G=4, d=128, d_idx=128, top_k=5)
+    in slot order; dk and dv sum a key block's items in the order of the
+    reverse index's lists, which are sorted by query position.  So all
+    three are bit-identical across runs, one chunk or several.  With
+    top_k = 18 over 18 blocks every query selects every earlier block, so
+    the lists of blocks 0 and 1 (2304 and 2176 entries) take the bitmap
+    route of the ordering step and the others the direct one."""
+    shape = I.PrefillShape(B=1, L=L, H=16, G=4, d=128, d_idx=128, top_k=top_k)
     x = _inputs(shape, 26)
-    sel, dq1, dk1, dv1 = _forward_backward(x, 5)
-    out, lse = M.msa_sparse_attn_prefill(x["q"], x["k"], x["v"], sel, want_lse=True)
-    dq2, dk2, dv2 = M.msa_sparse_attn_backward(x["q"], x["k"], x["v"], out, lse, x["dout"], sel)
-    torch.cuda.synchronize()
-    assert torch.equal(dq1, dq2)
-    for a, b in ((dk1, dk2), (dv1, dv2)):
-        a64, b64 = P.f64(a), P.f64(b)
-        assert np.linalg.norm(a64 - b64) <= 2e-3 * np.linalg.norm(a64)
+    sel, dq1, dk1, dv1 = _forward_backward(x, top_k, chunk=chunk)
+    for _ in range(2):
+        _, dq2, dk2, dv2 = _forward_backward(x, top_k, sel=sel, chunk=chunk)
+        assert torch.equal(dq1, dq2)
+        assert torch.equal(dk1, dk2)
+        assert torch.equal(dv1, dv2)
+    ref = O.prefill_backward(x["q"], x["k"], x["v"], sel.cpu().numpy(), x["dout"], block=128)
+    for name, g in (("dq", dq1), ("dk", dk1), ("dv", dv1)):
+        _grad_close(name, P.f64(g), ref[name])
 
 
 def test_backward_32k_sampled():
@@ -181,3 +188,35 @@ def test_backward_query_chunks():
     ref0 = O.prefill_backward(x["q"], x["k"], x["v"], sel0.cpu().numpy(), x["dout"], block=128)
     _grad_close("dk block 0 (8 chunks)", P.f64(dk0[:, :128]), ref0["dk"][:, :128])
     _grad_close("dv block 0 (8 chunks)", P.f64(dv0[:, :128]), ref0["dv"][:, :128])
+
+
+@pytest.mark.parametrize("B,L,H,G,top_k,blk,seed", [
+    (2, 1000, 8, 2, 4, 128, 40),    # partial last block (104 keys), two sequences
+    (1, 2049, 16, 4, 5, 128, 41),   # a last block of one key
+    (1, 1024, 8, 2, 6, 64, 42),     # 64-token blocks: half of the key tile
+    (2, 777, 4, 4, 8, 64, 43),      # 64-token blocks, partial last block, R = 1
+    (1, 640, 32, 2, 32, 64, 44),    # R = 16, top_k = 32 >= nb: dense causal
+])
+def test_backward_any_length_and_block64(B, L, H, G, top_k, blk, seed):
+    shape = I.PrefillShape(B=B, L=L, H=H, G=G, d=128, d_idx=128, top_k=top_k, block=blk)
+    x = _inputs(shape, seed)
+    sel, dq, dk, dv = _forward_backward(x, top_k, block=blk)
+    ref = O.prefill_backward(x["q"], x["k"], x["v"], sel.cpu().numpy(), x["dout"], block=blk)
+    _grad_close("dq", P.f64(dq), ref["dq"])
+    _grad_close("dk", P.f64(dk), ref["dk"])
+    _grad_close("dv", P.f64(dv), ref["dv"])
+
+
+@pytest.mark.parametrize("blk", [64, 128])
+def test_backward_chunks_any_length(blk):
+    """Query chunks of 384 packed rows over two sequences of 1000 (chunks
+    that straddle the sequence boundary): dq equals the one-chunk run bit
+    for bit, dk and dv match the oracle."""
+    shape = I.PrefillShape(B=2, L=1000, H=8, G=2, d=128, d_idx=128, top_k=5, block=blk)
+    x = _inputs(shape, 45)
+    sel, dq1, _, _ = _forward_backward(x, 5, block=blk)
+    _, dq, dk, dv = _forward_backward(x, 5, sel=sel, block=blk, chunk=384)
+    assert torch.equal(dq, dq1)
+    ref = O.prefill_backward(x["q"], x["k"], x["v"], sel.cpu().numpy(), x["dout"], block=blk)
+    for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _grad_close(f"{name} (chunks of 384)", P.f64(g), ref[name])

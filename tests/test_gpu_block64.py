@@ -240,9 +240,3 @@ def test_decode_integer_ties_and_fp8_caches():
         ref = O.decode(x["q"], x["q_idx"], kk, vv, kid, lens, 10, block=BLK, sel_override=s)
         mx, mean = P.out_errors(out_.float().cpu().numpy(), ref["out"])
         assert mx <= P.OUT_MAX_ABS and mean <= P.OUT_MEAN_ABS, (mx, mean)
-
-
-def test_backward_rejects_64_token_blocks():
-    import ctypes
-    p = M.make_params(1, 1024, 8, 2, 128, 128, 64, 4)
-    assert M.lib().msa_workspace_bytes(ctypes.byref(p), M.MSA_OP_BACKWARD) == 0
