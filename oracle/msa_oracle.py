@@ -31,6 +31,12 @@ Sources (cited by page title / address and section):
   gradient into the main attention is cut.  The main branch's backward pass
   is therefore the gradient of its exact attention over the selected tokens
   with the selection held fixed (prefill_backward).
+* [P2] §3.1 (comparison with DeepSeek NSA): NSA runs three parallel
+  branches -- compression, selection and a sliding window -- mixed by a
+  learned gate, where MSA keeps the selection branch alone.  The NSA-style
+  variant here (nsa_branches, nsa_forward) adds the other two branches to
+  MSA's selection.  The page names them without formulas; the readings
+  taken are listed below.
 
 Readings taken where the pages are silent (each is also listed in the
 design notes):
@@ -41,7 +47,14 @@ design notes):
 * ties between equal block scores go to the lower block id;
 * with no more than top_k visible blocks, every visible block is selected;
 * the local block is attended only up to the query itself (s <= t);
-* selections are stored sorted ascending and padded with -1.
+* selections are stored sorted ascending and padded with -1;
+* NSA-style variant: the sliding window of a query t is its `window` most
+  recent tokens, s in [t-window+1, t]; the compression branch summarises
+  block c by the mean of its keys and of its values (no learned weights
+  exist here), and a query attends the summaries of the blocks whose every
+  token is at or before it; a branch with no visible token contributes 0;
+  the gate is given per (query, head, branch) by the caller, and the output
+  is the gate-weighted sum of the three branch outputs.
 
 Every function here is pinned by a CPU test (tests/test_oracle_pins.py)
 against a closed form, a library routine, brute force or an invariant.
@@ -71,6 +84,12 @@ __all__ = [
     "block_scores_all",
     "attend_rows_grad",
     "prefill_backward",
+    "window_tokens",
+    "compress_kv",
+    "compressed_tokens",
+    "attend_rows_or_zero",
+    "nsa_branches",
+    "nsa_forward",
 ]
 
 
@@ -360,3 +379,98 @@ def prefill_backward(q, k, v, sel, dout, block: int = 128, scale: Optional[float
                 np.add.at(dk[b, :, g], tok, gk)
                 np.add.at(dv[b, :, g], tok, gv)
     return {"dq": dq, "dk": dk, "dv": dv}
+
+
+# ---------------------------------------------------------------------------
+# NSA-style variant: compression and sliding-window branches  ([P2] §3.1)
+# ---------------------------------------------------------------------------
+
+def window_tokens(t: int, window: int) -> np.ndarray:
+    """Tokens the sliding-window branch attends for a query at position t:
+    its `window` most recent positions, s in [t-window+1, t] (clipped at 0)."""
+    return np.arange(max(0, t - window + 1), t + 1, dtype=np.int64)
+
+
+def compress_kv(k, v, block: int):
+    """Keys and values of the compression branch: compressed token c stands
+    for block c and is the mean of the block's keys (values).  k, v
+    [B,L,G,d] -> (k_cmp, v_cmp) [B,nb,G,d] fp64, nb = ceil(L/block); a
+    partial last block averages the tokens it has."""
+    k, v = as_f64(k), as_f64(v)
+    B, L, G, d = k.shape
+    nb = (L + block - 1) // block
+    k_cmp = np.zeros((B, nb, G, d))
+    v_cmp = np.zeros((B, nb, G, d))
+    for c in range(nb):
+        lo, hi = c * block, min((c + 1) * block, L)
+        k_cmp[:, c] = k[:, lo:hi].sum(axis=1) / (hi - lo)
+        v_cmp[:, c] = v[:, lo:hi].sum(axis=1) / (hi - lo)
+    return k_cmp, v_cmp
+
+
+def compressed_tokens(t: int, block: int) -> np.ndarray:
+    """Compressed tokens a query at position t may attend: those of the blocks
+    whose every token is at or before t, i.e. c <= (t + 1) // block - 1."""
+    return np.arange((t + 1) // block, dtype=np.int64)
+
+
+def attend_rows_or_zero(q_rows: np.ndarray, k_tok: np.ndarray, v_tok: np.ndarray, scale: float):
+    """attend_rows, except that an empty token set gives a zero output and an
+    lse of -inf (a branch with nothing to attend contributes nothing)."""
+    if k_tok.shape[0] == 0:
+        r = q_rows.shape[0]
+        return np.zeros((r, v_tok.shape[-1])), np.full(r, -np.inf)
+    o, lse, _ = attend_rows(q_rows, k_tok, v_tok, scale)
+    return o, lse
+
+
+def nsa_branches(q, k, v, sel, window: int, block: int = 128, scale: Optional[float] = None,
+                 rows: Optional[Sequence[tuple]] = None):
+    """The three branch outputs of the NSA-style variant, each an exact
+    softmax attention of the query head over its own token set:
+      cmp  compressed tokens compressed_tokens(t) of (k_cmp, v_cmp),
+      slc  MSA's selection: the tokens s <= t of the blocks in sel[b, g, t],
+      win  window_tokens(t, window) of (k, v).
+    rows: optional (b, t) pairs to evaluate (all when None).  Returns dict of
+    out_cmp, out_slc, out_win [B,L,H,d] and lse_cmp, lse_slc, lse_win
+    [B,L,H] (NaN for rows not evaluated)."""
+    q, k, v = as_f64(q), as_f64(k), as_f64(v)
+    sel = np.asarray(sel)
+    B, L, H, d = q.shape
+    G = k.shape[2]
+    r = H // G
+    sc = _scale_of(d, scale)
+    k_cmp, v_cmp = compress_kv(k, v, block)
+    if rows is None:
+        rows = [(b, t) for b in range(B) for t in range(L)]
+    res = {}
+    for name in ("cmp", "slc", "win"):
+        res["out_" + name] = np.full((B, L, H, d), np.nan)
+        res["lse_" + name] = np.full((B, L, H), np.nan)
+    for (b, t) in rows:
+        for g in range(G):
+            heads = list(range(g * r, (g + 1) * r))
+            qr = q[b, t, heads]
+            c = compressed_tokens(t, block)
+            s_tok = selected_tokens([int(x) for x in sel[b, g, t] if x >= 0], t, block)
+            w_tok = window_tokens(t, window)
+            for name, kk, vv in (("cmp", k_cmp[b, c, g], v_cmp[b, c, g]),
+                                 ("slc", k[b, s_tok, g], v[b, s_tok, g]),
+                                 ("win", k[b, w_tok, g], v[b, w_tok, g])):
+                o, l_ = attend_rows_or_zero(qr, kk, vv, sc)
+                res["out_" + name][b, t, heads] = o
+                res["lse_" + name][b, t, heads] = l_
+    return res
+
+
+def nsa_forward(q, k, v, sel, gates, window: int, block: int = 128,
+                scale: Optional[float] = None, rows: Optional[Sequence[tuple]] = None):
+    """NSA-style output: o[t,h] = g_cmp o_cmp + g_slc o_slc + g_win o_win with
+    gates [B,L,H,3] in the order (cmp, slc, win) given by the caller (the
+    learned gate of [P2] §3.1 needs trained weights, which do not exist
+    here).  Returns (out [B,L,H,d], branches dict of nsa_branches)."""
+    br = nsa_branches(q, k, v, sel, window, block, scale, rows)
+    g = np.asarray(gates, dtype=np.float64)
+    out = (g[..., 0:1] * br["out_cmp"] + g[..., 1:2] * br["out_slc"]
+           + g[..., 2:3] * br["out_win"])
+    return out, br

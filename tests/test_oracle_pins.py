@@ -352,6 +352,88 @@ def check_backward_sums():
             assert not g["dk"][0, j * blk:(j + 1) * blk].any()
 
 
+def _nsa_problem(seed, L=96, blk=16, top_k=3):
+    p = _small_problem(seed, L=L)
+    sel = O.prefill(p["q"], p["k"], p["v"], p["q_idx"], p["k_idx"], top_k=top_k, block=blk)["sel"]
+    return p, sel, blk
+
+
+def _band_mask(L, lo_off, device=None):
+    """[L, L] boolean: key s visible to query t iff t - lo_off <= s <= t."""
+    ones = torch.ones(L, L, dtype=torch.bool)
+    return torch.tril(ones) & torch.triu(ones, diagonal=-lo_off)
+
+
+def check_nsa_window():
+    """Sliding-window branch against torch SDPA (fp64) with a band mask built
+    from tril/triu; window = 1 gives v[t] exactly; window >= L is dense
+    causal attention."""
+    p, sel, blk = _nsa_problem(121)
+    L = p["q"].shape[1]
+    for w in (1, 5, 16, 37):
+        br = O.nsa_branches(p["q"], p["k"], p["v"], sel, window=w, block=blk)
+        want = _gqa_sdpa(p["q"], p["k"], p["v"], mask=_band_mask(L, w - 1))
+        np.testing.assert_allclose(br["out_win"], want, rtol=1e-11, atol=1e-12)
+        if w == 1:
+            r = p["q"].shape[2] // p["k"].shape[2]
+            np.testing.assert_array_equal(br["out_win"], np.repeat(p["v"], r, axis=2))
+    br = O.nsa_branches(p["q"], p["k"], p["v"], sel, window=L + 7, block=blk)
+    np.testing.assert_allclose(br["out_win"], _gqa_sdpa(p["q"], p["k"], p["v"], is_causal=True),
+                               rtol=1e-11, atol=1e-12)
+
+
+def check_nsa_compression():
+    """Compression branch: block means against torch's avg_pool1d (a partial
+    last block averaged over its own tokens), the branch output against SDPA
+    over those pooled tokens with compressed token c visible to t iff block
+    c ends at or before t, zero output where no block is complete; block = 1
+    is dense causal attention."""
+    for L, blk in ((96, 16), (90, 16), (40, 1)):
+        p, sel, _ = _nsa_problem(122, L=L, blk=max(blk, 2))
+        B, _, G, d = p["k"].shape
+        pool = lambda x: F.avg_pool1d(torch.from_numpy(x).permute(0, 2, 3, 1).reshape(B * G * d, 1, L),
+                                      blk, blk, ceil_mode=True).reshape(B, G, d, -1).permute(0, 3, 1, 2)
+        kc, vc = O.compress_kv(p["k"], p["v"], blk)
+        np.testing.assert_allclose(kc, pool(p["k"]).numpy(), rtol=1e-13, atol=1e-14)
+        np.testing.assert_allclose(vc, pool(p["v"]).numpy(), rtol=1e-13, atol=1e-14)
+        br = O.nsa_branches(p["q"], p["k"], p["v"], sel, window=4, block=blk)
+        nb = kc.shape[1]
+        t_ = torch.arange(L)[:, None]
+        c_ = torch.arange(nb)[None, :]
+        mask = (c_ + 1) * blk - 1 <= t_                      # [L, nb]
+        has = mask.any(dim=1).numpy()
+        want = _gqa_sdpa(p["q"][:, has], kc, vc, mask=mask[torch.from_numpy(has)])
+        np.testing.assert_allclose(br["out_cmp"][:, has], want, rtol=1e-11, atol=1e-12)
+        assert not br["out_cmp"][:, ~has].any()
+        assert np.all(br["lse_cmp"][:, ~has] == -np.inf)
+        if blk == 1:
+            np.testing.assert_allclose(br["out_cmp"], _gqa_sdpa(p["q"], p["k"], p["v"], is_causal=True),
+                                       rtol=1e-11, atol=1e-12)
+
+
+def check_nsa_gate():
+    """One-hot gates give each branch alone (the selection branch is MSA's
+    prefill output on the same selection); the output is linear in the
+    gates."""
+    p, sel, blk = _nsa_problem(123)
+    B, L, H, _ = p["q"].shape
+    rng = np.random.default_rng(5)
+    out_slc = O.prefill(p["q"], p["k"], p["v"], p["q_idx"], p["k_idx"], top_k=3, block=blk,
+                        sel_override=sel)["out"]
+    outs = []
+    for i in range(3):
+        gates = np.zeros((B, L, H, 3))
+        gates[..., i] = 1.0
+        o, br = O.nsa_forward(p["q"], p["k"], p["v"], sel, gates, window=9, block=blk)
+        np.testing.assert_array_equal(o, br["out_" + ("cmp", "slc", "win")[i]])
+        outs.append(o)
+    np.testing.assert_allclose(outs[1], out_slc, rtol=0, atol=1e-13)
+    gates = rng.uniform(0, 1, (B, L, H, 3))
+    o, _ = O.nsa_forward(p["q"], p["k"], p["v"], sel, gates, window=9, block=blk)
+    want = sum(gates[..., i:i + 1] * outs[i] for i in range(3))
+    np.testing.assert_allclose(o, want, rtol=1e-13, atol=1e-14)
+
+
 CHECKS = {
     "golden": check_golden,
     "e4m3": check_e4m3_against_library_and_closed_forms,
@@ -369,6 +451,9 @@ CHECKS = {
     "backward_finite_differences": check_backward_finite_differences,
     "backward_dense_limit": check_backward_dense_limit,
     "backward_sums": check_backward_sums,
+    "nsa_window": check_nsa_window,
+    "nsa_compression": check_nsa_compression,
+    "nsa_gate": check_nsa_gate,
 }
 
 
@@ -456,6 +541,33 @@ def _grad_dq_through_v(q_rows, k_tok, v_tok, do_rows, scale):
 
 _orig_grad = O.attend_rows_grad
 
+
+def _window_one_more(t, window):
+    return np.arange(max(0, t - window), t + 1, dtype=np.int64)
+
+
+def _compressed_partial_visible(t, block):
+    return np.arange(t // block + 1, dtype=np.int64)
+
+
+def _compressed_before_local(t, block):
+    return np.arange(t // block, dtype=np.int64)
+
+
+def _compress_sum(k, v, block):
+    kc, vc = _orig_compress(k, v, block)
+    return kc * block, vc * block
+
+
+_orig_compress = O.compress_kv
+
+
+def _nsa_gates_swapped(q, k, v, sel, gates, window, block=128, scale=None, rows=None):
+    return _orig_nsa_forward(q, k, v, sel, np.asarray(gates)[..., ::-1], window, block, scale, rows)
+
+
+_orig_nsa_forward = O.nsa_forward
+
 MUTANTS = {
     "no_forced_local": ("select_blocks_row", _select_no_local),
     "ties_to_higher_id": ("select_blocks_row", _select_high_tie),
@@ -469,6 +581,11 @@ MUTANTS = {
     "bwd_delta_dropped": ("attend_rows_grad", _grad_no_delta),
     "bwd_dk_unscaled": ("attend_rows_grad", _grad_dk_unscaled),
     "bwd_dq_through_v": ("attend_rows_grad", _grad_dq_through_v),
+    "nsa_window_one_too_many": ("window_tokens", _window_one_more),
+    "nsa_partial_block_compressed": ("compressed_tokens", _compressed_partial_visible),
+    "nsa_completed_block_left_out": ("compressed_tokens", _compressed_before_local),
+    "nsa_compress_sum": ("compress_kv", _compress_sum),
+    "nsa_gates_swapped": ("nsa_forward", _nsa_gates_swapped),
 }
 
 
