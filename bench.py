@@ -288,6 +288,41 @@ class OracleLeg:
             times.append(time.perf_counter() - t0)
         return times
 
+    def nsa_positions(self, positions, window):
+        """Oracle seconds of each (b, t) position of the NSA-style variant: the
+        selection branch as in prefill_positions, the window branch and the
+        compression branch (every group and head).  The compressed keys and
+        values are made once, before the clock starts, and timed apart
+        (returned second)."""
+        import oracle.msa_oracle as O
+        f64 = O.as_f64
+        s = self.shape
+        r = s.H // s.G
+        sc = 1.0 / math.sqrt(s.d)
+        host = self._prefill_host()
+        t0 = time.perf_counter()
+        cmp_kv = [O.compress_kv(_f64(k)[None], _f64(v)[None], s.block) for (k, v, _) in host]
+        t_cmp = time.perf_counter() - t0
+        pos = list(positions)
+        q_rows = [self.x["q"][b, t].to("cpu") for (b, t) in pos]
+        qi_rows = [self.x["q_idx"][b, t].to("cpu") for (b, t) in pos]
+        times = []
+        for n, (b, t) in enumerate(pos):
+            k, v, k_idx64 = host[b]
+            kc, vc = cmp_kv[b]
+            t0 = time.perf_counter()
+            c = O.compressed_tokens(t, s.block)
+            w_tok = O.window_tokens(t, window)
+            for g in range(s.G):
+                qr = f64(q_rows[n][g * r:(g + 1) * r])
+                bs = O.block_scores_row(f64(qi_rows[n][g]), k_idx64, t, s.block)
+                tok = O.selected_tokens(O.select_blocks_row(bs, t, s.block, s.top_k), t, s.block)
+                O.attend_rows(qr, _f64(k[tok, g]), _f64(v[tok, g]), sc)
+                O.attend_rows(qr, _f64(k[w_tok, g]), _f64(v[w_tok, g]), sc)
+                O.attend_rows_or_zero(qr, kc[0, c, g], vc[0, c, g], sc)
+            times.append(time.perf_counter() - t0)
+        return times, t_cmp
+
     def prefill_full(self):
         """(seconds, (query, group) rows) of the oracle over every position."""
         s = self.shape
@@ -359,7 +394,7 @@ def main():
                          "whose index keys (134 MB) exceed the 126 MB L2)")
     ap.add_argument("--op", default="step",
                     choices=["step", "index", "scores", "attn", "decode", "decode8", "cached",
-                             "bwd"],
+                             "bwd", "nsa_window", "nsa_compressed"],
                     help="time one operation of the step alone (profiling runs; 'cached' runs "
                          "the whole prefill as 8 msa_forward_cached chunks against the caches); "
                          "prints its own short JSON line")
@@ -623,8 +658,18 @@ def run_single_op(args, M, x, dx, dshape, K, sel, out, dout, ws_idx, ws_att, ws_
         ws_b = M.new_workspace(M.make_params(Bq, Lq, Hq, sh_b.G, dq_, sh_b.d_idx, 128, K),
                                M.MSA_OP_BACKWARD, x["q"].device)
 
+    if args.op in ("nsa_window", "nsa_compressed"):   # NSA-style branch kernels (window 512)
+        Bq, Lq, Hq, dq_ = x["q"].shape
+        p_n = M.make_params(Bq, Lq, Hq, x["k"].shape[2], dq_, x["q_idx"].shape[3], 128, K)
+        ws_nsa = M.new_workspace(p_n, M.MSA_OP_NSA_BRANCH, x["q"].device)
+        kc, vc = M.msa_nsa_compress_kv(x["k"], x["v"])
+
     def op():
-        if args.op == "cached":   # the prefill as the serving form: 8 chunks against the caches
+        if args.op == "nsa_window":
+            M.msa_nsa_window_attn(x["q"], x["k"], x["v"], 512, out=out, ws=ws_nsa)
+        elif args.op == "nsa_compressed":
+            M.msa_nsa_compressed_attn(x["q"], kc, vc, out=out, ws=ws_nsa)
+        elif args.op == "cached":   # the prefill as the serving form: 8 chunks against the caches
             for c, (q, q_idx) in enumerate(qc):
                 M.msa_forward_cached(q, q_idx, x["k"], x["v"], x["k_idx"], c * n_c, K, out=outc,
                                      ws=ws_c)
@@ -654,7 +699,8 @@ def run_single_op(args, M, x, dx, dshape, K, sel, out, dout, ws_idx, ws_att, ws_
         op()
     b.record(stream)
     torch.cuda.synchronize()
-    extra = ((ws_c,) if ws_c is not None else ()) + ((ws_b,) if args.op == "bwd" else ())
+    extra = ((ws_c,) if ws_c is not None else ()) + ((ws_b,) if args.op == "bwd" else ()) \
+        + ((ws_nsa,) if args.op in ("nsa_window", "nsa_compressed") else ())
     for w in (ws_idx, ws_att, ws_dec) + extra:
         if M.msa_read_status(w) != 0:
             raise SystemExit("device status error")
@@ -905,6 +951,122 @@ def bench_prefill_config(M, I, dev, args, peaks, name, shape, seed, needles=0,
     return res
 
 
+def nsa_branch_flops(B, L, H, d, window, block):
+    """Algorithmic FLOPs of the window and compression branches: per query and
+    head 4*d per attended key (q.k and p*v), over min(window, t+1) tokens and
+    (t+1)//block compressed tokens."""
+    t = np.arange(L, dtype=np.float64)
+    f_win = B * H * 4 * d * float(np.minimum(window, t + 1).sum())
+    f_cmp = B * H * 4 * d * float(((t + 1) // block).sum())
+    return f_win, f_cmp
+
+
+def bench_nsa_32k(M, I, dev, args, peaks, window=512, iters=10):
+    """The NSA-style variant at the 32K prefill: msa_nsa_forward (MSA's index
+    and selection branches, block compression, the compression and window
+    branches, the gate) timed whole and branch by branch, with an L2 flush
+    between iterations; tensor rooflines of the two query-outer branch
+    kernels; the oracle on stratified positions beside it."""
+    shape = I.PREFILL_32K
+    seed = I.SEEDS["32k"]
+    x = I.prefill_inputs(shape, seed, device=dev)
+    B, L, H, G, d, di, K, blk = (shape.B, shape.L, shape.H, shape.G, shape.d, shape.d_idx,
+                                 shape.top_k, shape.block)
+    p = M.make_params(B, L, H, G, d, di, blk, K)
+    gen = torch.Generator(device="cpu").manual_seed(seed)
+    gates = torch.rand((B, L, H, 3), generator=gen).to(dev)
+    ws = M.new_workspace(p, M.MSA_OP_NSA_FORWARD, dev)
+    ws_b = M.new_workspace(p, M.MSA_OP_NSA_BRANCH, dev)
+    out = torch.empty_like(x["q"])
+    o_b = torch.empty_like(x["q"])
+    nb = (L + blk - 1) // blk
+    kc = torch.empty((B, nb, G, d), dtype=torch.bfloat16, device=dev)
+    vc = torch.empty_like(kc)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def run_all():
+        M.msa_nsa_forward(x["q"], x["k"], x["v"], x["q_idx"], x["k_idx"], gates, K, window,
+                          block=blk, out=out, ws=ws)
+
+    def run_win():
+        M.msa_nsa_window_attn(x["q"], x["k"], x["v"], window, out=o_b, ws=ws_b)
+
+    def run_cmp():
+        M.msa_nsa_compressed_attn(x["q"], kc, vc, block=blk, out=o_b, ws=ws_b)
+
+    def run_compress():
+        M.msa_nsa_compress_kv(x["k"], x["v"], block=blk, k_cmp=kc, v_cmp=vc)
+
+    legs = {"forward": run_all, "window": run_win, "compress_kv": run_compress,
+            "compressed": run_cmp}
+    for _ in range(max(3, args.warmup)):
+        for f in legs.values():
+            f()
+    torch.cuda.synchronize()
+    if M.msa_read_status(ws) != 0 or M.msa_read_status(ws_b) != 0:
+        raise SystemExit("nsa_32k: device status error")
+    times = {k: [] for k in legs}
+    for _ in range(iters):
+        for k, f in legs.items():
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            f()
+            b.record(stream)
+            torch.cuda.synchronize()
+            times[k].append(a.elapsed_time(b))
+    ms = {k: statistics.median(v) for k, v in times.items()}
+    f_win, f_cmp = nsa_branch_flops(B, L, H, d, window, blk)
+    burst = peaks["bf16_tflops"]
+
+    def tensor_roofline(f, t_ms):
+        return {"bound": "tensor", "achieved": f / (t_ms / 1e3) / 1e12, "peak": burst,
+                "unit": "TFLOP/s", "frac": f / (t_ms / 1e3) / 1e12 / burst, "flops": f,
+                "peak_kind": f"bf16 burst ({peaks['source']}): kernel timed alone"}
+
+    nchunks = math.ceil(B * L / M.msa_prefill_chunk_len(p))
+    res = {"workload": f"B={B} L={L} H={H} G={G} d={d} d_idx={di} block={blk} top_k={K}, "
+                       f"window {window}, gates U[0,1)",
+           "seed": seed, "iters": iters, "l2": "256 MB buffer written before every timed call",
+           "forward_ms": ms["forward"], "tokens_per_s": B * L / (ms["forward"] / 1e3),
+           "window_ms": ms["window"], "compress_kv_ms": ms["compress_kv"],
+           "compressed_ms": ms["compressed"],
+           "window_roofline": tensor_roofline(f_win, ms["window"]),
+           "compressed_roofline": tensor_roofline(f_cmp, ms["compressed"]),
+           "compress_kv_roofline": {"bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                                    "bytes": 2 * B * L * G * d * 2 + 2 * B * nb * G * d * 2,
+                                    "achieved": (2 * B * L * G * d * 2 + 2 * B * nb * G * d * 2)
+                                    / (ms["compress_kv"] / 1e3) / 1e9},
+           "gpu_launches": (1 + 5 * nchunks + 4) * iters}
+    res["compress_kv_roofline"]["frac"] = res["compress_kv_roofline"]["achieved"] / peaks["hbm_gbs"]
+    del ws, ws_b, out, o_b, kc, vc, flush
+    torch.cuda.empty_cache()
+    if not args.no_cpu_baseline:
+        leg = OracleLeg(x, None, shape, None)
+        rng = np.random.default_rng(seed)
+        n_strata = 64
+        pos, width = [], []
+        for i in range(n_strata):
+            lo, hi = i * L // n_strata, (i + 1) * L // n_strata
+            pos.append((0, int(rng.integers(lo, hi))))
+            width.append(hi - lo)
+        tms, t_cmp = leg.nsa_positions(pos, window)
+        secs = t_cmp + sum(w * tm for w, tm in zip(width, tms))
+        res["oracle"] = {"seconds": secs, "tokens_per_s": B * L / secs, "cores": oracle_threads(),
+                         "kind": "oracle", "extrapolated": True,
+                         "sample": f"{len(pos) * G} (query, group) rows: one uniform position in "
+                                   f"each of {n_strata} equal strata of [0,L), all groups and "
+                                   f"heads, the three branches; {sum(tms):.1f} s, extrapolated "
+                                   f"by stratum width, plus the block compression "
+                                   f"({t_cmp:.2f} s)"}
+        res["gpu_over_oracle"] = secs / (ms["forward"] / 1e3)
+    del x, gates
+    torch.cuda.empty_cache()
+    return res
+
+
 def bench_ragged_batch(M, I, dev, args, peaks):
     """A serving batch of prompt chunks continuing cached prefixes: 16
     sequences with caches of 131,072 tokens, each continuing at a seeded
@@ -993,6 +1155,7 @@ def bench_configs(M, I, dev, args, peaks, line):
     cfgs["32k_block64"] = bench_prefill_config(M, I, dev, args, peaks, "32k_block64",
                                                I.PREFILL_32K_BLOCK64, I.SEEDS["32k"], iters=10)
     cfgs["ragged_batch"] = bench_ragged_batch(M, I, dev, args, peaks)
+    cfgs["nsa_32k"] = bench_nsa_32k(M, I, dev, args, peaks)
     if "decode_128k" in line:
         d = line["decode_128k"]
         cfgs["decode_128k"] = {"us_per_step": d["us_per_step"], "roofline": d["roofline"],

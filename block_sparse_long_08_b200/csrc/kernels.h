@@ -157,6 +157,25 @@ struct BwdArgs {
   int *unit_ctr;               // work counter (zeroed by the launcher)
   int *status;
 };
+// NSA-style branches (nsa_kernels.cu): query-outer exact attention over a
+// contiguous visible key range per query row.
+struct DenseAttnArgs {
+  int B, L, H, G;              // queries q [B,L,H,d] (the tensor map's tensor)
+  int n_qt;                    // query tiles per sequence: ceil(L / (128 / (H/G)))
+  int mode;                    // 0: window over the tokens, 1: compressed tokens
+  int window, blk;             // mode 0: s in [t-window+1, t]; mode 1: c <= (t+1)/blk - 1
+  float scale, scale_log2;
+  uint16_t *out;               // [B,L,H,d]
+  float *lse;                  // [B,L,H] or null
+  int *status;
+};
+cudaError_t launch_dense_attn(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                              const DenseAttnArgs &a, int num_sms, cudaStream_t st);
+cudaError_t launch_nsa_compress(const uint16_t *k, const uint16_t *v, uint16_t *k_cmp,
+                                uint16_t *v_cmp, int B, int L, int G, int blk, cudaStream_t st);
+cudaError_t launch_nsa_gate(const float *gates, const uint16_t *o_cmp, const uint16_t *o_slc,
+                            const uint16_t *o_win, uint16_t *out, long long rows, cudaStream_t st);
+
 cudaError_t launch_bwd_delta(const BwdArgs &a, cudaStream_t st);   // D for all rows
 cudaError_t launch_backward(const CUtensorMap &tk, const CUtensorMap &tv, const BwdArgs &a,
                             int num_sms, cudaStream_t st);      // one chunk: kernel + dq sums

@@ -548,6 +548,88 @@ int run_decode(const msa_params *p, const msa_bf16 *q, const msa_bf16 *q_idx,
   return MSA_OK;
 }
 
+// ---- NSA-style branches ------------------------------------------------------
+// Workspace of msa_nsa_forward: msa_forward's, then the compressed keys and
+// values and the compression and window branches' outputs.
+struct NsaWs {
+  size_t fwd_end, k_cmp, v_cmp, o_cmp, o_win, end;
+};
+NsaWs nsa_ws(const msa_params *p) {
+  NsaWs w;
+  w.fwd_end = attn_ws(p, msa::kWsHeader + forward_sel_bytes(p)).end;
+  const size_t cmp = align_up(2 * size_t(p->B) * nblocks(p) * p->G * p->d);
+  const size_t o = align_up(2 * size_t(p->B) * p->L * p->H * p->d);
+  size_t x = align_up(w.fwd_end);
+  w.k_cmp = x; x += cmp;
+  w.v_cmp = x; x += cmp;
+  w.o_cmp = x; x += o;
+  w.o_win = x; x += o;
+  w.end = x;
+  return w;
+}
+
+// 4-D map over q [B,L,H,d] as (d, H, L, B): a box is 128/R consecutive
+// queries x the R heads of one group (a 128-row tile), half of d.
+int make_q_tmap(CUtensorMap *m, const void *q, const msa_params *p) {
+  const int r = p->H / p->G;
+  const uint64_t dims[4] = {uint64_t(p->d), uint64_t(p->H), uint64_t(p->L), uint64_t(p->B)};
+  const uint64_t str[3] = {uint64_t(p->d) * 2, uint64_t(p->d) * 2 * p->H,
+                           uint64_t(p->d) * 2 * p->H * p->L};
+  const uint32_t box[4] = {64, uint32_t(r), uint32_t(128 / r), 1};
+  return make_tmap(m, q, 4, dims, str, box);
+}
+
+// 4-D map over key rows [B, rows, G, d] as (d, G, rows, B): a box is 128
+// rows of one KV head, half of d; rows past `rows` load as zeros.
+int make_rows_tmap(CUtensorMap *m, const void *base, const msa_params *p, int rows) {
+  const uint64_t dims[4] = {uint64_t(p->d), uint64_t(p->G), uint64_t(rows), uint64_t(p->B)};
+  const uint64_t str[3] = {uint64_t(p->d) * 2, uint64_t(p->d) * 2 * p->G,
+                           uint64_t(p->d) * 2 * p->G * rows};
+  const uint32_t box[4] = {64, 1, 128, 1};
+  return make_tmap(m, base, 4, dims, str, box);
+}
+
+// One branch: mode 0 = window over the tokens k, v [B,L,G,d]; mode 1 =
+// compressed tokens k, v [B,nb,G,d].
+int run_dense(const msa_params *p, int mode, int window, const msa_bf16 *q, const void *k,
+              const void *v, int rows, msa_bf16 *out, float *lse, void *ws, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  int rc = make_q_tmap(&tq, q, p);
+  if (rc) return rc;
+  rc = make_rows_tmap(&tk, k, p, rows);
+  if (rc) return rc;
+  rc = make_rows_tmap(&tv, v, p, rows);
+  if (rc) return rc;
+  msa::DenseAttnArgs a;
+  a.B = p->B; a.L = p->L; a.H = p->H; a.G = p->G;
+  const int qpi = 128 / (p->H / p->G);
+  a.n_qt = (p->L + qpi - 1) / qpi;
+  a.mode = mode; a.window = window; a.blk = p->block;
+  a.scale = eff_scale(p);
+  a.scale_log2 = a.scale * 1.4426950408889634f;
+  a.out = reinterpret_cast<uint16_t *>(out);
+  a.lse = lse;
+  a.status = status_ptr(ws);
+  cudaError_t e = msa::launch_dense_attn(tq, tk, tv, a, num_sms(), st);
+  if (e != cudaSuccess) return cuda_fail(e, "NSA branch attention launch");
+  return MSA_OK;
+}
+
+int nsa_compress(const msa_params *p, const msa_bf16 *k, const msa_bf16 *v, msa_bf16 *k_cmp,
+                 msa_bf16 *v_cmp, cudaStream_t st) {
+  cudaError_t e = msa::launch_nsa_compress(k, v, k_cmp, v_cmp, p->B, p->L, p->G, p->block, st);
+  if (e != cudaSuccess) return cuda_fail(e, "NSA compression launch");
+  return MSA_OK;
+}
+
+int nsa_gate(const msa_params *p, const float *gates, const msa_bf16 *o_cmp, const msa_bf16 *o_slc,
+             const msa_bf16 *o_win, msa_bf16 *out, cudaStream_t st) {
+  cudaError_t e = msa::launch_nsa_gate(gates, o_cmp, o_slc, o_win, out,
+                                       (long long)p->B * p->L * p->H, st);
+  if (e != cudaSuccess) return cuda_fail(e, "NSA gate launch");
+  return MSA_OK;
+}
+
 }  // namespace
 
 namespace msa {
@@ -595,6 +677,8 @@ size_t msa_workspace_bytes(const msa_params *p, int op) {
     case MSA_OP_FORWARD: return attn_ws(p, msa::kWsHeader + forward_sel_bytes(p)).end;
     case MSA_OP_BACKWARD: return bwd_ws(p).end;
     case MSA_OP_FORWARD_VARLEN: return attn_ws(p, varlen_ws(p).attn_base).end;
+    case MSA_OP_NSA_BRANCH: return msa::kWsHeader;
+    case MSA_OP_NSA_FORWARD: return nsa_ws(p).end;
     default: fail(MSA_ERR_INVALID_ARG, "unknown op %d", op); return 0;
   }
 }
@@ -1009,6 +1093,101 @@ int msa_quantize_e4m3_rows(const msa_bf16 *x, long long rows, int cols, uint8_t 
                                                  reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return MSA_OK;
+}
+
+int msa_nsa_compress_kv(const msa_params *p, const msa_bf16 *k, const msa_bf16 *v,
+                        msa_bf16 *k_cmp, msa_bf16 *v_cmp, msa_stream stream) {
+  g_err[0] = 0;
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (p->B == 0 || p->L == 0) return MSA_OK;
+  if (!k || !v || !k_cmp || !v_cmp) return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(k) || !aligned16(v) || !aligned16(k_cmp) || !aligned16(v_cmp))
+    return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  return nsa_compress(p, k, v, k_cmp, v_cmp, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int msa_nsa_window_attn(const msa_params *p, int32_t window, const msa_bf16 *q,
+                        const msa_bf16 *k, const msa_bf16 *v, msa_bf16 *out, float *lse,
+                        void *ws, size_t ws_bytes, msa_stream stream) {
+  g_err[0] = 0;
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (window < 1) return fail(MSA_ERR_INVALID_ARG, "window=%d must be >= 1", window);
+  if (p->B == 0 || p->L == 0) return MSA_OK;
+  if (!q || !k || !v || !out) return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (lse && !aligned16(lse)))
+    return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  rc = check_ws(ws, ws_bytes, msa::kWsHeader);
+  if (rc) return rc;
+  return run_dense(p, 0, window, q, k, v, p->L, out, lse, ws,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+int msa_nsa_compressed_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k_cmp,
+                            const msa_bf16 *v_cmp, msa_bf16 *out, float *lse, void *ws,
+                            size_t ws_bytes, msa_stream stream) {
+  g_err[0] = 0;
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (p->B == 0 || p->L == 0) return MSA_OK;
+  if (!q || !k_cmp || !v_cmp || !out) return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(q) || !aligned16(k_cmp) || !aligned16(v_cmp) || !aligned16(out) ||
+      (lse && !aligned16(lse)))
+    return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  rc = check_ws(ws, ws_bytes, msa::kWsHeader);
+  if (rc) return rc;
+  return run_dense(p, 1, 0, q, k_cmp, v_cmp, nblocks(p), out, lse, ws,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+int msa_nsa_gate(const msa_params *p, const float *gates, const msa_bf16 *o_cmp,
+                 const msa_bf16 *o_slc, const msa_bf16 *o_win, msa_bf16 *out,
+                 msa_stream stream) {
+  g_err[0] = 0;
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (p->B == 0 || p->L == 0) return MSA_OK;
+  if (!gates || !o_cmp || !o_slc || !o_win || !out)
+    return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(gates) || !aligned16(o_cmp) || !aligned16(o_slc) || !aligned16(o_win) ||
+      !aligned16(out))
+    return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  return nsa_gate(p, gates, o_cmp, o_slc, o_win, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int msa_nsa_forward(const msa_params *p, int32_t window, const msa_bf16 *q, const msa_bf16 *k,
+                    const msa_bf16 *v, const msa_bf16 *q_idx, const msa_bf16 *k_idx,
+                    const float *gates, msa_bf16 *out, int32_t *sel, void *ws, size_t ws_bytes,
+                    msa_stream stream) {
+  g_err[0] = 0;
+  int rc = check_params(p, false);
+  if (rc) return rc;
+  if (window < 1) return fail(MSA_ERR_INVALID_ARG, "window=%d must be >= 1", window);
+  if (p->B == 0 || p->L == 0) return MSA_OK;
+  if (!q || !k || !v || !q_idx || !k_idx || !gates || !out)
+    return fail(MSA_ERR_INVALID_ARG, "NULL tensor pointer");
+  if (!aligned16(gates)) return fail(MSA_ERR_INVALID_ARG, "tensor pointers must be 16-byte aligned");
+  const NsaWs w = nsa_ws(p);
+  rc = check_ws(ws, ws_bytes, w.end);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // selection branch (MSA) into out; its own checks cover q..k_idx, out, sel
+  rc = msa_forward(p, q, k, v, q_idx, k_idx, out, sel, nullptr, ws, w.fwd_end, stream);
+  if (rc) return rc;
+  uint8_t *wsb = reinterpret_cast<uint8_t *>(ws);
+  msa_bf16 *k_cmp = reinterpret_cast<msa_bf16 *>(wsb + w.k_cmp);
+  msa_bf16 *v_cmp = reinterpret_cast<msa_bf16 *>(wsb + w.v_cmp);
+  msa_bf16 *o_cmp = reinterpret_cast<msa_bf16 *>(wsb + w.o_cmp);
+  msa_bf16 *o_win = reinterpret_cast<msa_bf16 *>(wsb + w.o_win);
+  rc = nsa_compress(p, k, v, k_cmp, v_cmp, st);
+  if (rc) return rc;
+  rc = run_dense(p, 1, 0, q, k_cmp, v_cmp, nblocks(p), o_cmp, nullptr, ws, st);
+  if (rc) return rc;
+  rc = run_dense(p, 0, window, q, k, v, p->L, o_win, nullptr, ws, st);
+  if (rc) return rc;
+  return nsa_gate(p, gates, o_cmp, out, o_win, out, st);
 }
 
 }  // extern "C"

@@ -34,6 +34,8 @@ MSA_OP_DECODE = 2
 MSA_OP_FORWARD = 3
 MSA_OP_BACKWARD = 4
 MSA_OP_FORWARD_VARLEN = 5
+MSA_OP_NSA_BRANCH = 6
+MSA_OP_NSA_FORWARD = 7
 
 
 class MSAError(RuntimeError):
@@ -88,6 +90,12 @@ def lib() -> ctypes.CDLL:
         L.msa_sparse_attn_decode_noalloc.restype = ctypes.c_int
         L.msa_sparse_attn_backward.argtypes = [pp, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                                _SZ, _P]
+        L.msa_nsa_compress_kv.argtypes = [pp, _P, _P, _P, _P, _P]
+        L.msa_nsa_window_attn.argtypes = [pp, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.msa_nsa_compressed_attn.argtypes = [pp, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.msa_nsa_gate.argtypes = [pp, _P, _P, _P, _P, _P, _P]
+        L.msa_nsa_forward.argtypes = [pp, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ,
+                                      _P]
         L.msa_workspace_bytes.argtypes = [pp, ctypes.c_int]
         L.msa_workspace_bytes.restype = _SZ
         L.msa_read_status.argtypes = [_P, _P]
@@ -99,7 +107,8 @@ def lib() -> ctypes.CDLL:
                   "msa_forward", "msa_forward_host", "msa_forward_cached", "msa_read_status",
                   "msa_sparse_attn_decode_fp8idx", "msa_quantize_e4m3_rows",
                   "msa_sparse_attn_decode_fp8", "msa_forward_cached_varlen",
-                  "msa_sparse_attn_backward"):
+                  "msa_sparse_attn_backward", "msa_nsa_compress_kv", "msa_nsa_window_attn",
+                  "msa_nsa_compressed_attn", "msa_nsa_gate", "msa_nsa_forward"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -261,6 +270,94 @@ def msa_forward(q, k, v, q_idx, k_idx, top_k: int, *, scale: float = 0.0, want_s
     if want_lse:
         res.append(lse)
     return res[0] if len(res) == 1 else tuple(res)
+
+
+# ---- NSA-style variant: compression and sliding-window branches beside the
+# selection, mixed by caller-given gates (see include/msa.h)
+
+def _nsa_params(q, k, block, scale, top_k=16, d_idx=128):
+    B, L, H, d = q.shape
+    return make_params(B, L, H, k.shape[2], d, d_idx, block, top_k, scale)
+
+
+def msa_nsa_compress_kv(k, v, *, block: int = 128, k_cmp=None, v_cmp=None, stream=None):
+    """Block means of k and v [B,L,G,d] -> (k_cmp, v_cmp) [B,ceil(L/block),G,d]."""
+    _req(k, "k", torch.bfloat16)
+    _req(v, "v", torch.bfloat16)
+    B, L, G, d = k.shape
+    p = make_params(B, L, G, G, d, 128, block, 1)
+    nb = (L + block - 1) // block
+    k_cmp = torch.empty((B, nb, G, d), dtype=torch.bfloat16, device=k.device) if k_cmp is None else k_cmp
+    v_cmp = torch.empty((B, nb, G, d), dtype=torch.bfloat16, device=k.device) if v_cmp is None else v_cmp
+    _check(lib().msa_nsa_compress_kv(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(k_cmp), _ptr(v_cmp),
+                                     _stream(stream)))
+    return k_cmp, v_cmp
+
+
+def msa_nsa_window_attn(q, k, v, window: int, *, scale: float = 0.0, want_lse: bool = False,
+                        out=None, ws=None, stream=None):
+    """Sliding-window branch: each query over its `window` most recent tokens."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _req(t, n, torch.bfloat16)
+    p = _nsa_params(q, k, 128, scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if want_lse else None
+    ws = _ensure_ws(ws, p, MSA_OP_NSA_BRANCH, q.device)
+    _check(lib().msa_nsa_window_attn(ctypes.byref(p), int(window), _ptr(q), _ptr(k), _ptr(v),
+                                     _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
+    return (out, lse) if want_lse else out
+
+
+def msa_nsa_compressed_attn(q, k_cmp, v_cmp, *, block: int = 128, scale: float = 0.0,
+                            want_lse: bool = False, out=None, ws=None, stream=None):
+    """Compression branch: each query over the compressed tokens of the blocks
+    whose every token lies at or before it."""
+    for n, t in (("q", q), ("k_cmp", k_cmp), ("v_cmp", v_cmp)):
+        _req(t, n, torch.bfloat16)
+    p = _nsa_params(q, k_cmp, block, scale)
+    if k_cmp.shape[1] != (q.shape[1] + block - 1) // block:
+        raise ValueError("k_cmp must hold ceil(L / block) compressed tokens")
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if want_lse else None
+    ws = _ensure_ws(ws, p, MSA_OP_NSA_BRANCH, q.device)
+    _check(lib().msa_nsa_compressed_attn(ctypes.byref(p), _ptr(q), _ptr(k_cmp), _ptr(v_cmp),
+                                         _ptr(out), _ptr(lse), _ptr(ws), ws.numel(),
+                                         _stream(stream)))
+    return (out, lse) if want_lse else out
+
+
+def msa_nsa_gate(gates, o_cmp, o_slc, o_win, *, out=None, stream=None):
+    """out = g_cmp o_cmp + g_slc o_slc + g_win o_win, gates [B,L,H,3] fp32."""
+    _req(gates, "gates", torch.float32)
+    for n, t in (("o_cmp", o_cmp), ("o_slc", o_slc), ("o_win", o_win)):
+        _req(t, n, torch.bfloat16)
+    B, L, H, d = o_cmp.shape
+    p = make_params(B, L, H, H, d, 128, 128, 1)   # the gate is per head: any grouping
+    out = torch.empty_like(o_cmp) if out is None else out
+    _check(lib().msa_nsa_gate(ctypes.byref(p), _ptr(gates), _ptr(o_cmp), _ptr(o_slc), _ptr(o_win),
+                              _ptr(out), _stream(stream)))
+    return out
+
+
+def msa_nsa_forward(q, k, v, q_idx, k_idx, gates, top_k: int, window: int, *, block: int = 128,
+                    scale: float = 0.0, want_sel: bool = False, out=None, sel=None, ws=None,
+                    stream=None):
+    """NSA-style prefill: MSA's selection branch, the compression and window
+    branches, and the gate, in one call."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("q_idx", q_idx), ("k_idx", k_idx)):
+        _req(t, n, torch.bfloat16)
+    _req(gates, "gates", torch.float32)
+    B, L, H, d = q.shape
+    G = k.shape[2]
+    p = make_params(B, L, H, G, d, q_idx.shape[3], block, top_k, scale)
+    out = torch.empty_like(q) if out is None else out
+    if sel is None and want_sel:
+        sel = torch.empty((B, G, L, top_k), dtype=torch.int32, device=q.device)
+    ws = _ensure_ws(ws, p, MSA_OP_NSA_FORWARD, q.device)
+    _check(lib().msa_nsa_forward(ctypes.byref(p), int(window), _ptr(q), _ptr(k), _ptr(v),
+                                 _ptr(q_idx), _ptr(k_idx), _ptr(gates), _ptr(out), _ptr(sel),
+                                 _ptr(ws), ws.numel(), _stream(stream)))
+    return (out, sel) if want_sel else out
 
 
 def msa_forward_cached(q, q_idx, k_cache, v_cache, k_idx_cache, t0: int, top_k: int, *,

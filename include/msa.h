@@ -105,7 +105,9 @@ enum {
   MSA_OP_DECODE = 2,
   MSA_OP_FORWARD = 3,
   MSA_OP_BACKWARD = 4,
-  MSA_OP_FORWARD_VARLEN = 5
+  MSA_OP_FORWARD_VARLEN = 5,
+  MSA_OP_NSA_BRANCH = 6,     /* msa_nsa_window_attn, msa_nsa_compressed_attn */
+  MSA_OP_NSA_FORWARD = 7     /* msa_nsa_forward */
 };
 
 /* Index Branch (explainer §2.1; researchpapers.dev "机制").
@@ -337,6 +339,65 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
                              const msa_bf16 *dout, const int32_t *sel, msa_bf16 *dq,
                              msa_bf16 *dk, msa_bf16 *dv, void *ws, size_t ws_bytes,
                              msa_stream stream);
+
+/* ---- NSA-style variant --------------------------------------------------
+ * "MiniMax M3 sparse attention" explainer (mlqm.cn/news/533796), §3.1:
+ * DeepSeek NSA runs three parallel branches -- compression, selection and a
+ * sliding window -- mixed by a learned gate; MSA keeps the selection alone.
+ * These entry points add the other two branches beside MSA's selection.
+ * The page gives them no formulas; the readings implemented:
+ *   window       query t attends its `window` most recent tokens, s in
+ *                [t-window+1, t] (exact softmax attention, scale as p);
+ *   compression  compressed token c is the mean of block c's keys (values),
+ *                block = p->block; query t attends the compressed tokens of
+ *                the blocks whose every token lies at or before t, i.e.
+ *                c <= (t+1)/block - 1; a query with none gets a zero output
+ *                (lse -inf);
+ *   gate         three gates per (query, head) from the caller (the learned
+ *                gate needs trained weights); out = g_cmp o_cmp + g_slc o_slc
+ *                + g_win o_win, accumulated in fp32.
+ * Layouts as above; k_cmp, v_cmp [B,nb,G,d] bf16 with nb = ceil(L/block);
+ * gates [B,L,H,3] fp32 in the order (cmp, slc, win).  Same shape support
+ * as the prefill.  Every branch kernel is query-outer: a 128-row tile of
+ * 128/(H/G) consecutive queries x H/G heads sweeps the key tiles its rows
+ * see twice (row maxima, then P V accumulated in TMEM). */
+
+/* Compressed keys and values: k_cmp[b,c,g] = mean of k[b,s,g] over the
+ * tokens s of block c (a partial last block averages the tokens it has),
+ * fp32 sums rounded to bf16; the same for v.  No workspace. */
+int msa_nsa_compress_kv(const msa_params *p, const msa_bf16 *k, const msa_bf16 *v,
+                        msa_bf16 *k_cmp, msa_bf16 *v_cmp, msa_stream stream);
+
+/* Sliding-window branch: out [B,L,H,d] bf16 and (nullable) lse [B,L,H]
+ * fp32 of each query over its window >= 1 most recent tokens.
+ * ws >= msa_workspace_bytes(p, MSA_OP_NSA_BRANCH) (the status word). */
+int msa_nsa_window_attn(const msa_params *p, int32_t window, const msa_bf16 *q,
+                        const msa_bf16 *k, const msa_bf16 *v, msa_bf16 *out, float *lse,
+                        void *ws, size_t ws_bytes, msa_stream stream);
+
+/* Compression branch: out, lse of each query over the compressed tokens
+ * of its completed blocks (msa_nsa_compress_kv's output).
+ * ws >= msa_workspace_bytes(p, MSA_OP_NSA_BRANCH). */
+int msa_nsa_compressed_attn(const msa_params *p, const msa_bf16 *q, const msa_bf16 *k_cmp,
+                            const msa_bf16 *v_cmp, msa_bf16 *out, float *lse, void *ws,
+                            size_t ws_bytes, msa_stream stream);
+
+/* out = g_cmp o_cmp + g_slc o_slc + g_win o_win per (b, t, h); out may be
+ * one of the three inputs.  No workspace. */
+int msa_nsa_gate(const msa_params *p, const float *gates, const msa_bf16 *o_cmp,
+                 const msa_bf16 *o_slc, const msa_bf16 *o_win, msa_bf16 *out,
+                 msa_stream stream);
+
+/* The whole NSA-style prefill: MSA's index branch and selection branch
+ * (as msa_forward), the compression and window branches, and the gate.
+ * sel [B,G,L,top_k] is nullable.
+ * ws >= msa_workspace_bytes(p, MSA_OP_NSA_FORWARD): msa_forward's, plus
+ * k_cmp, v_cmp and two branch outputs (the selection branch's output is
+ * written to out and gated in place). */
+int msa_nsa_forward(const msa_params *p, int32_t window, const msa_bf16 *q, const msa_bf16 *k,
+                    const msa_bf16 *v, const msa_bf16 *q_idx, const msa_bf16 *k_idx,
+                    const float *gates, msa_bf16 *out, int32_t *sel, void *ws, size_t ws_bytes,
+                    msa_stream stream);
 
 /* Workspace bytes op (MSA_OP_*) needs for these params; 0 when p is invalid
  * (see msa_last_error). */

@@ -171,6 +171,40 @@ def test_backward_rejects_bad_arguments():
     assert lib.msa_sparse_attn_backward(ctypes.byref(p0), *([None] * 10), None, 0, None) == M.MSA_OK
 
 
+def test_nsa_entry_points_reject_bad_arguments():
+    """Argument checks of the NSA-style entry points run before any CUDA
+    call: window >= 1, no NULL tensors, 16-byte alignment, workspace size."""
+    p = M.make_params(1, 1000, 8, 2, 128, 128, 128, 4)
+    lib = M.lib()
+    ok = ctypes.c_void_p(4096)
+    odd = ctypes.c_void_p(4096 + 8)
+    hdr = M.msa_workspace_bytes(p, M.MSA_OP_NSA_BRANCH)
+    assert hdr == 256
+    assert lib.msa_nsa_window_attn(ctypes.byref(p), 0, ok, ok, ok, ok, None, ok, hdr,
+                                   None) == M.MSA_ERR_INVALID_ARG
+    assert lib.msa_nsa_window_attn(ctypes.byref(p), 64, ok, None, ok, ok, None, ok, hdr,
+                                   None) == M.MSA_ERR_INVALID_ARG
+    assert lib.msa_nsa_window_attn(ctypes.byref(p), 64, ok, ok, ok, ok, odd, ok, hdr,
+                                   None) == M.MSA_ERR_INVALID_ARG
+    assert lib.msa_nsa_window_attn(ctypes.byref(p), 64, ok, ok, ok, ok, None, ok, hdr - 1,
+                                   None) == M.MSA_ERR_WORKSPACE
+    assert lib.msa_nsa_compressed_attn(ctypes.byref(p), ok, ok, odd, ok, None, ok, hdr,
+                                       None) == M.MSA_ERR_INVALID_ARG
+    assert lib.msa_nsa_compress_kv(ctypes.byref(p), ok, ok, None, ok, None) == M.MSA_ERR_INVALID_ARG
+    assert lib.msa_nsa_gate(ctypes.byref(p), odd, ok, ok, ok, ok, None) == M.MSA_ERR_INVALID_ARG
+    need = M.msa_workspace_bytes(p, M.MSA_OP_NSA_FORWARD)
+    # msa_forward's workspace, then k_cmp, v_cmp (8 blocks) and two outputs
+    assert need >= (M.msa_workspace_bytes(p, M.MSA_OP_FORWARD) + 2 * 8 * 2 * 128 * 2
+                    + 2 * 1000 * 8 * 128 * 2)
+    args = [ok] * 7
+    assert lib.msa_nsa_forward(ctypes.byref(p), 0, *args, None, ok, need,
+                               None) == M.MSA_ERR_INVALID_ARG
+    assert lib.msa_nsa_forward(ctypes.byref(p), 512, *args, None, ok, need - 1,
+                               None) == M.MSA_ERR_WORKSPACE
+    p0 = M.make_params(0, 1000, 8, 2, 128, 128, 128, 4)
+    assert lib.msa_nsa_window_attn(ctypes.byref(p0), 5, *([None] * 5), None, 0, None) == M.MSA_OK
+
+
 def test_plain_c_program_uses_the_library(tmp_path):
     """The boundary is a C ABI: a C99 program, compiled with warnings as
     errors against include/msa.h alone, links libmsa.so and calls its
