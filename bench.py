@@ -477,7 +477,8 @@ def run_ours(args, shape, dshape, seed, cfg, ws_n, rank, local):
     peaks = load_peaks()
 
     # ---- inputs (device-resident for the kernel-timed leg)
-    need_pre = args.op in ("step", "index", "scores", "attn", "cached", "bwd")
+    need_pre = args.op in ("step", "index", "scores", "attn", "cached", "bwd", "nsa_window",
+                           "nsa_compressed")
     need_dec = args.op in ("step", "decode", "decode8")
     if not need_pre:   # a decode-only profiling run keeps the footprint small
         import dataclasses

@@ -547,8 +547,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int e = 0; e < 4; ++e) {
             const int c = h * 64 + gb * 8 + e * 2;
             const float2 x = fma2(make_float2(v[c], v[c + 1]), sc2, nmb2);
-            // half of the exponentials on the ex2 unit, half on the FMA pipe
-            const float2 pp = make_float2(fast_exp2(x.x), exp2_fma(x.y));
+            const float2 pp = make_float2(fast_exp2(x.x), fast_exp2(x.y));
             l2 = add2(l2, pp);
             w4[e] = pack_bf16x2(pp.x, pp.y);
           }

@@ -137,25 +137,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for the half of a softmax's exponentials that do not
-// go to the ex2 unit.  x = i + f with i the nearest integer (added to
-// 1.5 * 2^23, so the rounding needs no conversion instruction) and f in
-// [-1/2, 1/2]; 2^f is a degree-4 polynomial whose coefficients were fitted
-// by least squares, relative error weighted, on 2000 Chebyshev nodes of
-// [-1/2, 1/2] (relative error below 3e-6 in fp32); 2^i goes into the
-// exponent field.  Arguments below -125 (masked scores, -inf) give 0.
-__device__ __forceinline__ float exp2_fma(float x) {
-  const float t = x + 12582912.0f;
-  const int i = __float_as_int(t) - 0x4B400000;
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(0.009560511f, f, 0.05591704f);
-  p = fmaf(p, f, 0.24024981f);
-  p = fmaf(p, f, 0.69312197f);
-  p = fmaf(p, f, 0.99999917f);
-  const float r = __int_as_float(__float_as_int(p) + int(unsigned(i) << 23));
-  return x < -125.0f ? 0.0f : r;
-}
-
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, uint32_t bar, int x,
                                             int y) {

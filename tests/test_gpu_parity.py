@@ -103,6 +103,34 @@ def test_integer_inputs_select_bit_exact():
     assert ties > 100   # the case really exercises ties
 
 
+@pytest.mark.parametrize("blk,top_k", [(128, 16), (64, 32)])
+def test_sweep_directions_keep_ties_bit_exact(blk, top_k):
+    """512 index work items over 148 CTAs: rounds 1 and 3 sweep their key
+    chunks backward (ids arrive in decreasing order) and rounds 0 and 2
+    forward.  Small-integer inputs make scores exact and ties common, so the
+    fused route must equal the stored-score route, and sampled rows of
+    every round the oracle's selection, bit for bit."""
+    shape = I.PrefillShape(B=2, L=8192, H=32, G=8, d=128, d_idx=128, top_k=top_k, block=blk)
+    x = I.prefill_inputs(shape, 14)
+    q_idx = I.small_integer_like(x["q_idx"], 15, -1, 1)
+    k_idx = I.small_integer_like(x["k_idx"], 16, -1, 1)
+    sel_f = M.msa_index_select(q_idx.to(DEV), k_idx.to(DEV), top_k, block=blk)
+    sel_u, _ = M.msa_index_select(q_idx.to(DEV), k_idx.to(DEV), top_k, block_scores=True, block=blk)
+    torch.cuda.synchronize()
+    assert torch.equal(sel_f, sel_u)
+    sel = sel_f.cpu().numpy()
+    qi, ki = O.as_f64(q_idx), O.as_f64(k_idx)
+    # query tiles 63..0 are items 8*(63-i) .. 8*(63-i)+7: a tile every 3
+    # covers rounds 0-3 (148 items each)
+    for i in range(2, 64, 3):
+        for t in (i * 128, i * 128 + 77, i * 128 + 127):
+            for b in range(2):
+                for g in (0, 5):
+                    bs = O.block_scores_row(qi[b, t, g], ki[b], t, blk)
+                    want = O.select_blocks_row(bs, t, blk, top_k)
+                    assert list(sel[b, g, t]) == want + [-1] * (top_k - len(want)), (b, g, t)
+
+
 def test_zero_index_keys_all_ties():
     shape = I.PrefillShape(B=1, L=1024, H=8, G=2, d=128, d_idx=128, top_k=5)
     x = _prefill(shape, 4)
