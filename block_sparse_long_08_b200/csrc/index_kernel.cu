@@ -31,12 +31,7 @@
 //             memory.
 // The TMEM accumulator is freed as soon as its columns sit in registers, so
 // the next UMMA into that slot waits one TMEM round trip, not the max-pool
-// and list work.
-// The persistent CTAs take their items in rounds (item r*grid + c, snake
-// order), and the rounds sweep their key chunks in alternating directions:
-// forward in even rounds, backward in odd ones.  The CTAs of a round run
-// roughly in step, so a round starts on the k_idx rows the previous round
-// left in L2 instead of re-reading them from HBM once k_idx outgrows L2.  The first warpgroup gives registers to the epilogue
+// and list work.  The first warpgroup gives registers to the epilogue
 // warpgroups (setmaxnreg: 3 x 128 x 168 = 128 x 56 + 256 x 224).
 // One k_idx stage feeds GP groups, which halves L2->SM traffic for GP = 2.
 #include <cuda.h>
@@ -152,19 +147,15 @@ __device__ __forceinline__ void list_insert(float (&ls)[KCAP], int (&lj)[KCAP], 
 }
 
 template <int KCAP>
-__device__ __forceinline__ void list_insert_tail(float (&ls)[KCAP], int (&lj)[KCAP], float s,
-                                                 float c, int j) {
-  // Insert (s, j) when j is above every kept id or below every kept id (the
-  // blocks of one epilogue set arrive in increasing id order in a forward
-  // sweep, decreasing in a backward one).  With c = s (ids above) a kept
-  // entry ranks ahead of the new one exactly when its score is >= s; with
-  // c = the next float above s (ids below) exactly when its score is > s,
-  // i.e. >= c.  The insertion point is the number of such entries and every
-  // slot is updated independently -- no carried compare chain.  Walking k
-  // downwards reads ls[k-1] before it is replaced.
+__device__ __forceinline__ void list_insert_tail(float (&ls)[KCAP], int (&lj)[KCAP], float s, int j) {
+  // Insert (s, j) when j is above every kept id (the blocks of one epilogue
+  // set arrive in increasing id order): a kept entry ranks ahead of the new
+  // one exactly when its score is >= s, so the insertion point is the number
+  // of such entries and every slot is updated independently -- no carried
+  // compare chain.  Walking k downwards reads ls[k-1] before it is replaced.
   bool ge[KCAP];
 #pragma unroll
-  for (int k = 0; k < KCAP; ++k) ge[k] = ls[k] >= c;
+  for (int k = 0; k < KCAP; ++k) ge[k] = ls[k] >= s;
 #pragma unroll
   for (int k = KCAP - 1; k >= 1; --k) {
     ls[k] = ge[k] ? ls[k] : (ge[k - 1] ? s : ls[k - 1]);
@@ -226,20 +217,15 @@ __device__ __forceinline__ float max4x32(const float (&a)[32], const float (&b)[
 }
 
 // One block score of a row: stored (SCORES mode) or offered to the row's
-// running list (FUSED mode; within a set ids arrive in increasing order in a
-// forward sweep, rev = false, and in decreasing order in a backward one).
-// The new entry beats the worst kept one when its score is higher, or equal
-// with the lower id (backward: the new id is the lower one).
+// running list (FUSED mode; ids arrive in increasing order within a set).
 template <int KCAP>
 __device__ __forceinline__ void put_score(const IndexArgs &a, const int4 &sq, int g, int t,
-                                          float (&ls)[KCAP], int (&lj)[KCAP], float sc, int jb,
-                                          bool rev) {
+                                          float (&ls)[KCAP], int (&lj)[KCAP], float sc, int jb) {
   if (a.write_scores) {
     const long long orow = index_out_row(a, sq, g, t);
     if (orow >= 0) a.scores[orow * a.nb + jb] = sc;
-  } else {
-    const float c = rev ? nextafterf(sc, INFINITY) : sc;
-    if (c > ls[KCAP - 1]) list_insert_tail<KCAP>(ls, lj, sc, c, jb);
+  } else if (sc > ls[KCAP - 1]) {
+    list_insert_tail<KCAP>(ls, lj, sc, jb);
   }
 }
 
@@ -321,8 +307,7 @@ __global__ void __launch_bounds__(384, 1)
           if (!mbar_wait(b_kempty + 8 * kst, kph ^ 1, abort_flag, a.status)) { ok = false; break; }
           mbar_arrive_expect_tx(b_kfull + 8 * kst, C::STAGE_BYTES);
           const uint32_t dst = s_k + kst * C::STAGE_BYTES;
-          const int sc = (r & 1) ? (w.stages - 1 - s) : s;   // odd rounds sweep backward
-          const int row0 = w.b * a.L + (2 * sc) * 128;   // 128-key chunks 2sc, 2sc+1
+          const int row0 = w.b * a.L + (2 * s) * 128;   // 128-key chunks 2s, 2s+1
           for (int c = 0; c < C::NCH; ++c) {
             tma_load_2d(dst + c * 32768, &tm_k, b_kfull + 8 * kst, c * 64, row0);
             tma_load_2d(dst + c * 32768 + 16384, &tm_k, b_kfull + 8 * kst, c * 64, row0 + 128);
@@ -399,7 +384,6 @@ __global__ void __launch_bounds__(384, 1)
       const int u = index_item(r, a.n_items);
       if (u < 0) break;
       const IndexWork w = index_work<BLK>(a, u, GP);
-      const bool rev = (r & 1) != 0;   // this round sweeps its chunks backward
       const int t = w.i * 128 + row;   // query tiles hold 128 queries whatever the block
       const int bt = t / BLK;          // this row's local block
       const int4 sq = qgeo_seq(a.q, w.b);
@@ -422,7 +406,7 @@ __global__ void __launch_bounds__(384, 1)
             break;
           }
           tc_fence_after();
-          const int j = 2 * (rev ? (w.stages - 1 - s) : s) + eset;   // 128-key chunk
+          const int j = 2 * s + eset;   // 128-key chunk
           // warp-uniform: a warp's rows are all below or all above 64
           const bool use = (BLK == 128) ? (j < w.i) : (j < w.i || (j == w.i && row >= 64));
           float v0[32], v1[32], v2[32], v3[32];
@@ -441,19 +425,14 @@ __global__ void __launch_bounds__(384, 1)
           ++jc;
           if (use) {
             if (BLK == 128) {
-              put_score<KCAP>(a, sq, w.gp * GP + gi, t, ls[gi], lj[gi], max4x32(v0, v1, v2, v3), j,
-                              rev);
+              put_score<KCAP>(a, sq, w.gp * GP + gi, t, ls[gi], lj[gi], max4x32(v0, v1, v2, v3), j);
             } else {
-              // blocks 2j (columns 0..63) and 2j+1 (64..127), offered in the
-              // sweep's id order; block 2i+1 is a local block, never scored
-              const float s0 = max2x32(v0, v1);
-              if (rev && j < w.i)
+              // blocks 2j (columns 0..63) and 2j+1 (64..127); block 2i+1 is
+              // a local block, never scored
+              put_score<KCAP>(a, sq, w.gp * GP + gi, t, ls[gi], lj[gi], max2x32(v0, v1), 2 * j);
+              if (j < w.i)
                 put_score<KCAP>(a, sq, w.gp * GP + gi, t, ls[gi], lj[gi], max2x32(v2, v3),
-                                2 * j + 1, rev);
-              put_score<KCAP>(a, sq, w.gp * GP + gi, t, ls[gi], lj[gi], s0, 2 * j, rev);
-              if (!rev && j < w.i)
-                put_score<KCAP>(a, sq, w.gp * GP + gi, t, ls[gi], lj[gi], max2x32(v2, v3),
-                                2 * j + 1, rev);
+                                2 * j + 1);
             }
           }
         }

@@ -27,13 +27,19 @@
 //                rescaling.
 //   nsa_gate_kernel        the gate-weighted sum of the three branch outputs.
 //
-// Roles of nsa_dense_attn_kernel (one persistent CTA per SM, 6 warps):
+// Roles of nsa_dense_attn_kernel (one persistent CTA per SM, 12 warps):
 //   warp 0     TMA producer: the item's Q tile, then its K tiles (pass 1),
 //              then K and V tiles interleaved (pass 2) into a ring.
 //   warp 1     TMEM owner and MMA issuer: S into two 128-column slots, O
 //              into a third.  In pass 2 it issues S of tile i+1 before O of
 //              tile i, so the softmax of the next tile overlaps P V.
-//   warps 2-5  softmax warpgroup, one row (TMEM lane) per thread.
+//   warps 4-11 two softmax warpgroups, one row (TMEM lane) per thread each;
+//              warpgroup h takes key columns 64h..64h+63 of every S tile
+//              (and P's 16 KB half h, and d columns 64h.. of O).  The row
+//              maximum and the row sum are associative, so each warpgroup
+//              keeps its own over all tiles and the two are exchanged once
+//              per pass through shared memory.
+//   warps 2-3  idle.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -47,9 +53,9 @@ namespace msa {
 
 namespace {
 
-constexpr int kDenseThreads = 192;
+constexpr int kDenseThreads = 384;
 constexpr int kDTile = 32768;                    // 128 rows x 256 B
-constexpr int kDNkv = 4;                         // K/V ring depth
+constexpr int kDNkv = 3;                         // K/V ring depth
 // shared memory (from a 1024-byte aligned base)
 constexpr int kDSQ = 0;                          // Q tile
 constexpr int kDSP = kDTile;                     // two P tiles
@@ -61,7 +67,8 @@ constexpr int kBQFull = 0, kBQEmpty = 1, kBKvFull = 2, kBKvEmpty = 2 + kDNkv,
               kBPEmpty = kBPFull + 2, kBOFull = kBPEmpty + 2, kBOEmpty = kBOFull + 1,
               kBDrain = kBOEmpty + 1, kDNumBars = kBDrain + 1;
 constexpr int kDCtlMisc = kDNumBars * 8;         // tmem holder, abort flag
-constexpr int kDenseSmem = kDCtl + kDCtlMisc + 16 + 1024;
+constexpr int kDCtlX = kDCtlMisc + 16;            // [2][128] row maxima, [2][128] row sums
+constexpr int kDenseSmem = kDCtl + kDCtlX + 4 * 128 * 4 + 1024;
 static_assert(kDenseSmem <= 232448, "shared memory budget");
 // TMEM columns: S slots 0 and 128, O at 256 (512 allocated)
 constexpr uint32_t kTmO = 256;
@@ -134,12 +141,12 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
     }
     for (int u = 0; u < 2; ++u) {
       mbar_init(bar(kBSFull + u), 1);
-      mbar_init(bar(kBSEmpty + u), 128);
-      mbar_init(bar(kBPFull + u), 128);
+      mbar_init(bar(kBSEmpty + u), 256);
+      mbar_init(bar(kBPFull + u), 256);
       mbar_init(bar(kBPEmpty + u), 1);
     }
     mbar_init(bar(kBOFull), 1);
-    mbar_init(bar(kBOEmpty), 128);
+    mbar_init(bar(kBOEmpty), 256);
     mbar_init(bar(kBDrain), 1);
     *abort_flag = 0;
     mbar_init_fence();
@@ -285,28 +292,30 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
         mbar_wait_drain(bar(kBDrain), 0);
       }
     }
-  } else {
+  } else if (warp >= 4) {
     // ---------------------------------------------------------- softmax
     const int q4 = warp & 3;               // TMEM lane quadrant of this warp
+    const int hc = (warp - 4) >> 2;        // key-column / d half of this warpgroup
     const int row = q4 * 32 + lane;        // tile row = TMEM lane
     const uint32_t tm_lane = tmem_base + (uint32_t(q4 * 32) << 16);
     const int qi = row / R, hh = row % R;
+    float *x_max = reinterpret_cast<float *>(ctl + kDCtlX);   // [2][128]
+    float *x_sum = x_max + 2 * 128;                             // [2][128]
     constexpr int bar_id = 1;
     uint32_t scnt = 0, pcnt = 0;
     int item_n = 0;
     bool ok = true;
-    // S row of the next slot into v (all four loads issued, then one wait)
-    auto load_s = [&](float (&v)[128]) -> bool {
+    // this warpgroup's 64 columns of the next S slot (both loads issued,
+    // then one wait)
+    auto load_s = [&](float (&v)[64]) -> bool {
       const int sl = int(scnt & 1);
       bool w_ok = mbar_wait(bar(kBSFull + sl), (scnt >> 1) & 1, abort_flag, a.status);
-      if (!bar_and_n(bar_id, 128, w_ok)) return false;
+      if (!bar_and_n(bar_id, 256, w_ok)) return false;
       tc_fence_after();
-      float t0[32], t1[32], t2[32], t3[32];
-      const uint32_t ta = tm_lane + sl * 128;
+      float t0[32], t1[32];
+      const uint32_t ta = tm_lane + sl * 128 + hc * 64;
       tmem_ld32(ta, t0);
       tmem_ld32(ta + 32, t1);
-      tmem_ld32(ta + 64, t2);
-      tmem_ld32(ta + 96, t3);
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(kBSEmpty + sl));
@@ -315,8 +324,6 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
       for (int x = 0; x < 32; ++x) {
         v[x] = t0[x];
         v[32 + x] = t1[x];
-        v[64 + x] = t2[x];
-        v[96 + x] = t3[x];
       }
       return true;
     };
@@ -331,81 +338,79 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
       const size_t orow = (size_t(w.b) * a.L + t) * a.H + w.g * R + hh;
       if (w.n_kt == 0) {   // no row of the item sees a key: zero output
         if (valid) {
-          uint4 *dst = reinterpret_cast<uint4 *>(a.out + orow * kHeadDim);
+          uint4 *dst = reinterpret_cast<uint4 *>(a.out + orow * kHeadDim + hc * 64);
 #pragma unroll
-          for (int c = 0; c < 16; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
-          if (a.lse) a.lse[orow] = -INFINITY;
+          for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+          if (a.lse && hc == 0) a.lse[orow] = -INFINITY;
         }
         continue;
       }
       // ---- pass 1: row maximum over the visible columns
       float m = -INFINITY;
       for (int kt = 0; kt < w.n_kt; ++kt) {
-        float v[128];
+        float v[64];
         ok = load_s(v);
         if (!ok) break;
-        const int c0 = lo - (w.kt_lo + kt) * 128, c1 = hi - (w.kt_lo + kt) * 128;
+        const int c0 = lo - (w.kt_lo + kt) * 128 - hc * 64, c1 = hi - (w.kt_lo + kt) * 128 - hc * 64;
 #pragma unroll
-        for (int x = 0; x < 128; ++x) m = (x >= c0 && x <= c1) ? fmaxf(m, v[x]) : m;
+        for (int x = 0; x < 64; ++x) m = (x >= c0 && x <= c1) ? fmaxf(m, v[x]) : m;
       }
       if (!ok) break;
+      x_max[hc * 128 + row] = m;
+      bar_sync_n(bar_id, 256);
+      m = fmaxf(m, x_max[(hc ^ 1) * 128 + row]);
       // ---- pass 2: P = exp2((S - m) * scale log2 e) as bf16, row sums
       const float mb = (m == -INFINITY) ? 0.f : m * a.scale_log2;
       float l = 0.f;
       for (int kt = 0; kt < w.n_kt; ++kt) {
-        float v[128];
+        float v[64];
         ok = load_s(v);
         if (!ok) break;
         const int pb = int(pcnt & 1);
         bool w_ok = mbar_wait(bar(kBPEmpty + pb), ((pcnt >> 1) & 1) ^ 1, abort_flag, a.status);
-        if (!bar_and_n(bar_id, 128, w_ok)) {
+        if (!bar_and_n(bar_id, 256, w_ok)) {
           ok = false;
           break;
         }
-        const int c0 = lo - (w.kt_lo + kt) * 128, c1 = hi - (w.kt_lo + kt) * 128;
-        uint8_t *stile = smem + kDSP + pb * kDTile;
+        const int c0 = lo - (w.kt_lo + kt) * 128 - hc * 64, c1 = hi - (w.kt_lo + kt) * 128 - hc * 64;
+        uint8_t *stile = smem + kDSP + pb * kDTile + hc * 16384;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int gb = 0; gb < 8; ++gb) {
+          uint32_t w4[4];
 #pragma unroll
-          for (int gb = 0; gb < 8; ++gb) {
-            uint32_t w4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = h * 64 + gb * 8 + e * 2;
-              const float p0 =
-                  (c >= c0 && c <= c1) ? fast_exp2(fmaf(v[c], a.scale_log2, -mb)) : 0.f;
-              const float p1 =
-                  (c + 1 >= c0 && c + 1 <= c1) ? fast_exp2(fmaf(v[c + 1], a.scale_log2, -mb)) : 0.f;
-              l += p0 + p1;
-              w4[e] = pack_bf16x2(p0, p1);
-            }
-            *reinterpret_cast<uint4 *>(stile + h * 16384 + sw128_offset(row, gb)) =
-                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          for (int e = 0; e < 4; ++e) {
+            const int c = gb * 8 + e * 2;
+            const float p0 =
+                (c >= c0 && c <= c1) ? fast_exp2(fmaf(v[c], a.scale_log2, -mb)) : 0.f;
+            const float p1 =
+                (c + 1 >= c0 && c + 1 <= c1) ? fast_exp2(fmaf(v[c + 1], a.scale_log2, -mb)) : 0.f;
+            l += p0 + p1;
+            w4[e] = pack_bf16x2(p0, p1);
           }
+          *reinterpret_cast<uint4 *>(stile + sw128_offset(row, gb)) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
         fence_proxy_async_smem();
         mbar_arrive(bar(kBPFull + pb));
         ++pcnt;
       }
       if (!ok) break;
+      x_sum[hc * 128 + row] = l;
       // ---- O / l
       bool w_ok = mbar_wait(bar(kBOFull), item_n & 1, abort_flag, a.status);
-      if (!bar_and_n(bar_id, 128, w_ok)) break;
+      if (!bar_and_n(bar_id, 256, w_ok)) break;   // also publishes the partial sums
+      l += x_sum[(hc ^ 1) * 128 + row];
       tc_fence_after();
-      float o[128];
+      float o[64];
       {
-        float t0[32], t1[32], t2[32], t3[32];
-        tmem_ld32(tm_lane + kTmO, t0);
-        tmem_ld32(tm_lane + kTmO + 32, t1);
-        tmem_ld32(tm_lane + kTmO + 64, t2);
-        tmem_ld32(tm_lane + kTmO + 96, t3);
+        float t0[32], t1[32];
+        tmem_ld32(tm_lane + kTmO + hc * 64, t0);
+        tmem_ld32(tm_lane + kTmO + hc * 64 + 32, t1);
         tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
           o[x] = t0[x];
           o[32 + x] = t1[x];
-          o[64 + x] = t2[x];
-          o[96 + x] = t3[x];
         }
       }
       tc_fence_before();
@@ -413,14 +418,14 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
       ++item_n;
       if (valid) {
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint4 *dst = reinterpret_cast<uint4 *>(a.out + orow * kHeadDim);
+        uint4 *dst = reinterpret_cast<uint4 *>(a.out + orow * kHeadDim + hc * 64);
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
+        for (int c = 0; c < 8; ++c)
           dst[c] = make_uint4(pack_bf16x2(o[8 * c] * inv, o[8 * c + 1] * inv),
                               pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
                               pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
                               pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
-        if (a.lse) a.lse[orow] = l > 0.f ? m * a.scale + __logf(l) : -INFINITY;
+        if (a.lse && hc == 0) a.lse[orow] = l > 0.f ? m * a.scale + __logf(l) : -INFINITY;
       }
     }
   }

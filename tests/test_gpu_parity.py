@@ -104,12 +104,11 @@ def test_integer_inputs_select_bit_exact():
 
 
 @pytest.mark.parametrize("blk,top_k", [(128, 16), (64, 32)])
-def test_sweep_directions_keep_ties_bit_exact(blk, top_k):
-    """512 index work items over 148 CTAs: rounds 1 and 3 sweep their key
-    chunks backward (ids arrive in decreasing order) and rounds 0 and 2
-    forward.  Small-integer inputs make scores exact and ties common, so the
-    fused route must equal the stored-score route, and sampled rows of
-    every round the oracle's selection, bit for bit."""
+def test_many_work_items_keep_ties_bit_exact(blk, top_k):
+    """512 index work items over 148 CTAs, so every CTA takes items in
+    several rounds.  Small-integer inputs make scores exact and ties common,
+    so the fused route must equal the stored-score route, and sampled rows
+    of every round the oracle's selection, bit for bit."""
     shape = I.PrefillShape(B=2, L=8192, H=32, G=8, d=128, d_idx=128, top_k=top_k, block=blk)
     x = I.prefill_inputs(shape, 14)
     q_idx = I.small_integer_like(x["q_idx"], 15, -1, 1)
