@@ -19,26 +19,27 @@
 //                the completed blocks over the summaries.  One work item is
 //                (b, g, 128/R consecutive queries x R heads), a 128-row tile
 //                that one 4-D TMA box brings in.  The key tiles (128 keys)
-//                that any row of the item sees are swept twice.  Pass 1
-//                computes S = Q K^T and each row's masked maximum.  Pass 2
-//                recomputes S, writes P = exp2(S - max) as bf16 and
-//                accumulates O += P V in TMEM across the tiles: with the
-//                final maximum known up front, nothing accumulated needs
-//                rescaling.
+//                that any row of the item sees are swept once: S = Q K^T in
+//                TMEM, P = exp2(S - mr) as bf16 against a per-row reference
+//                maximum mr, O += P V accumulated in TMEM across the tiles.
+//                mr moves only when a tile raises the row's maximum by more
+//                than 2^8 in P; the row's O columns and sum are then scaled
+//                down in place (TMEM load, scale, TMEM store), which happens
+//                a few times per row at most.
 //   nsa_gate_kernel        the gate-weighted sum of the three branch outputs.
 //
 // Roles of nsa_dense_attn_kernel (one persistent CTA per SM, 12 warps):
-//   warp 0     TMA producer: the item's Q tile, then its K tiles (pass 1),
-//              then K and V tiles interleaved (pass 2) into a ring.
+//   warp 0     TMA producer: the item's Q tile, then K and V of each key
+//              tile in turn, into a ring.
 //   warp 1     TMEM owner and MMA issuer: S into two 128-column slots, O
-//              into a third.  In pass 2 it issues S of tile i+1 before O of
-//              tile i, so the softmax of the next tile overlaps P V.
+//              into a third.  It issues S of tile i+1 before O of tile i,
+//              so the softmax of the next tile overlaps P V.
 //   warps 4-11 two softmax warpgroups, one row (TMEM lane) per thread each;
 //              warpgroup h takes key columns 64h..64h+63 of every S tile
-//              (and P's 16 KB half h, and d columns 64h.. of O).  The row
-//              maximum and the row sum are associative, so each warpgroup
-//              keeps its own over all tiles and the two are exchanged once
-//              per pass through shared memory.
+//              (and P's 16 KB half h, and d columns 64h.. of O).  The two
+//              exchange each tile's row maxima through shared memory, so
+//              both halves of a row use one reference, and their row sums
+//              once at the end.
 //   warps 2-3  idle.
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -184,16 +185,9 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
         tma_load_4d(s_base + kDSQ, &tm_q, bar(kBQFull), 0, w.g * R, w.t0, w.b);
         tma_load_4d(s_base + kDSQ + 16384, &tm_q, bar(kBQFull), 64, w.g * R, w.t0, w.b);
         ++qn;
-        // pass 1: K tiles; pass 2: K and V of each tile in turn
-        for (int step = 0; step < 3 * w.n_kt; ++step) {
-          int kt, is_v;
-          if (step < w.n_kt) {
-            kt = step;
-            is_v = 0;
-          } else {
-            kt = (step - w.n_kt) >> 1;
-            is_v = (step - w.n_kt) & 1;
-          }
+        // K and V of each tile in turn
+        for (int step = 0; step < 2 * w.n_kt; ++step) {
+          const int kt = step >> 1, is_v = step & 1;
           const int x = int(kseq % kDNkv);
           ok = mbar_wait(bar(kBKvEmpty + x), ((kseq / kDNkv) & 1) ^ 1, abort_flag, a.status);
           if (!ok) break;
@@ -250,9 +244,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
         ok = mbar_wait(bar(kBQFull), item_n & 1, abort_flag, a.status);
         if (!ok) break;
         tc_fence_after();
-        for (int kt = 0; kt < w.n_kt && ok; ++kt) ok = issue_s(kseq + kt);   // pass 1
-        if (!ok) break;
-        const uint32_t p2 = kseq + w.n_kt;   // pass 2: K_kt at p2 + 2kt, V_kt at p2 + 2kt + 1
+        const uint32_t p2 = kseq;   // K_kt at p2 + 2kt, V_kt at p2 + 2kt + 1
         ok = issue_s(p2);
         for (int kt = 0; kt < w.n_kt && ok; ++kt) {
           if (kt + 1 < w.n_kt) {
@@ -345,34 +337,60 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
         }
         continue;
       }
-      // ---- pass 1: row maximum over the visible columns
-      float m = -INFINITY;
-      for (int kt = 0; kt < w.n_kt; ++kt) {
-        float v[64];
-        ok = load_s(v);
-        if (!ok) break;
-        const int c0 = lo - (w.kt_lo + kt) * 128 - hc * 64, c1 = hi - (w.kt_lo + kt) * 128 - hc * 64;
-#pragma unroll
-        for (int x = 0; x < 64; ++x) m = (x >= c0 && x <= c1) ? fmaxf(m, v[x]) : m;
-      }
-      if (!ok) break;
-      x_max[hc * 128 + row] = m;
-      bar_sync_n(bar_id, 256);
-      m = fmaxf(m, x_max[(hc ^ 1) * 128 + row]);
-      // ---- pass 2: P = exp2((S - m) * scale log2 e) as bf16, row sums
-      const float mb = (m == -INFINITY) ? 0.f : m * a.scale_log2;
+      // ---- one sweep.  P is taken against a reference maximum mr that
+      // moves only when a tile raises the row's maximum past mr by more
+      // than 2^8 in P; then the row's O columns (in TMEM, after the last P V
+      // has landed) and its sum are scaled down to the new reference.  So
+      // P <= 2^8, and O is rescaled a few times per row at most.
+      float mr = -INFINITY;   // reference maximum, raw score units
       float l = 0.f;
       for (int kt = 0; kt < w.n_kt; ++kt) {
         float v[64];
         ok = load_s(v);
         if (!ok) break;
+        const int c0 = lo - (w.kt_lo + kt) * 128 - hc * 64, c1 = hi - (w.kt_lo + kt) * 128 - hc * 64;
+        float tmx = -INFINITY;
+#pragma unroll
+        for (int x = 0; x < 64; ++x) tmx = (x >= c0 && x <= c1) ? fmaxf(tmx, v[x]) : tmx;
+        x_max[hc * 128 + row] = tmx;   // both halves of the row share the reference
+        bar_sync_n(bar_id, 256);
+        tmx = fmaxf(tmx, x_max[(hc ^ 1) * 128 + row]);
+        const bool resc =
+            tmx > -INFINITY && (mr == -INFINITY || (tmx - mr) * a.scale_log2 > 8.f);
+        const float alpha =
+            resc ? (mr == -INFINITY ? 0.f : fast_exp2((mr - tmx) * a.scale_log2)) : 1.f;
+        l *= alpha;
+        if (kt > 0 && __any_sync(0xffffffffu, resc && mr > -INFINITY)) {
+          // O holds the earlier tiles of this warp's rows: wait for the last
+          // P V, then scale this warpgroup's 64 columns in place
+          const uint32_t u = pcnt - 1;
+          bool r_ok = mbar_wait(bar(kBPEmpty + (u & 1)), (u >> 1) & 1, abort_flag, a.status);
+          if (__all_sync(0xffffffffu, r_ok)) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c32 = 0; c32 < 2; ++c32) {   // 32 columns at a time: few live registers
+              float t0[32];
+              const uint32_t to = tm_lane + kTmO + hc * 64 + c32 * 32;
+              tmem_ld32(to, t0);
+              tmem_wait_ld();
+#pragma unroll
+              for (int x = 0; x < 32; ++x) t0[x] *= alpha;
+              tmem_st32(to, t0);
+              tmem_wait_st();
+            }
+            tc_fence_before();
+          } else {
+            ok = false;
+          }
+        }
+        if (resc) mr = tmx;
+        const float mb = (mr == -INFINITY) ? 0.f : mr * a.scale_log2;
         const int pb = int(pcnt & 1);
-        bool w_ok = mbar_wait(bar(kBPEmpty + pb), ((pcnt >> 1) & 1) ^ 1, abort_flag, a.status);
+        bool w_ok = ok && mbar_wait(bar(kBPEmpty + pb), ((pcnt >> 1) & 1) ^ 1, abort_flag, a.status);
         if (!bar_and_n(bar_id, 256, w_ok)) {
           ok = false;
           break;
         }
-        const int c0 = lo - (w.kt_lo + kt) * 128 - hc * 64, c1 = hi - (w.kt_lo + kt) * 128 - hc * 64;
         uint8_t *stile = smem + kDSP + pb * kDTile + hc * 16384;
 #pragma unroll
         for (int gb = 0; gb < 8; ++gb) {
@@ -425,7 +443,7 @@ __global__ void __launch_bounds__(kDenseThreads, 1)
                               pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
                               pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
                               pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
-        if (a.lse && hc == 0) a.lse[orow] = l > 0.f ? m * a.scale + __logf(l) : -INFINITY;
+        if (a.lse && hc == 0) a.lse[orow] = l > 0.f ? mr * a.scale + __logf(l) : -INFINITY;
       }
     }
   }

@@ -149,3 +149,53 @@ def test_gate_in_place():
     torch.cuda.synchronize()
     e = (out.double().cpu() - want).abs()
     assert (e <= 2.0 ** -8 * want.abs() + 1e-6).all(), e.max()
+
+
+def _growing_keys(x, period):
+    """Keys scaled by 2^(s/period) along the sequence, so that a row's
+    maximum keeps rising from key tile to key tile by far more than the 2^8
+    the kernel allows before it rescales its accumulator."""
+    L = x["k"].shape[1]
+    f = torch.pow(2.0, torch.arange(L, dtype=torch.float32, device=x["k"].device) / period)
+    k = (x["k"].float() * f[None, :, None, None]).to(torch.bfloat16)
+    return dict(x, k=k.contiguous())
+
+
+def test_window_branch_rescales_as_the_maximum_grows():
+    """Keys growing 2x every 128 positions: every key tile raises the row
+    maximum, so O and l are rescaled in place tile after tile (window 1024
+    over L = 1024 and 600: dense causal attention)."""
+    for L in (1024, 600):
+        _, x = _inputs(1, L, 8, 2, 73)
+        x = _growing_keys(x, 128.0)
+        out, lse = M.msa_nsa_window_attn(x["q"], x["k"], x["v"], 1024, want_lse=True)
+        torch.cuda.synchronize()
+        sel = np.full((1, 2, L, 1), -1, dtype=np.int32)
+        ref = O.nsa_branches(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), sel, window=1024)
+        _close(out, ref["out_win"], "out_win (growing keys)")
+        g = lse.cpu().numpy().astype(np.float64)
+        rel = np.abs(g - ref["lse_win"]) / np.maximum(1.0, np.abs(ref["lse_win"]))
+        assert rel.max() <= 1e-3, rel.max()
+
+
+def test_compressed_branch_rescales_as_the_maximum_grows():
+    """Compressed keys growing along the sequence (2x every 3000 tokens):
+    the second compressed-token tile raises a late row's maximum by about
+    140 raw score units over the first's, past the kernel's 2^8 threshold
+    (63 units at scale 1/sqrt(128)), while the scores (about 250) stay
+    small enough for the bf16 rounding of the compressed keys to move a
+    logit by only ~0.04."""
+    _, x = _inputs(1, 20000, 8, 8, 74)
+    x = _growing_keys(x, 3000.0)
+    kc, vc = M.msa_nsa_compress_kv(x["k"], x["v"])
+    out, lse = M.msa_nsa_compressed_attn(x["q"], kc, vc, want_lse=True)
+    torch.cuda.synchronize()
+    rows = [(0, t) for t in (127, 5000, 16383, 16384, 16511, 16512, 19999)]
+    sel = np.full((1, 8, 20000, 1), -1, dtype=np.int32)
+    ref = O.nsa_branches(x["q"].cpu(), x["k"].cpu(), x["v"].cpu(), sel, window=1, rows=rows)
+    ti = [t for _, t in rows]
+    _close(out[0, ti], ref["out_cmp"][0, ti], "out_cmp (growing keys)")
+    g = lse[0, ti].cpu().numpy().astype(np.float64)
+    r = ref["lse_cmp"][0, ti]
+    rel = np.abs(g - r) / np.maximum(1.0, np.abs(r))
+    assert rel.max() <= 3e-3, rel.max()
