@@ -360,7 +360,8 @@ int msa_sparse_attn_backward(const msa_params *p, const msa_bf16 *q, const msa_b
  * gates [B,L,H,3] fp32 in the order (cmp, slc, win).  Same shape support
  * as the prefill.  Every branch kernel is query-outer: a 128-row tile of
  * 128/(H/G) consecutive queries x H/G heads sweeps the key tiles its rows
- * see twice (row maxima, then P V accumulated in TMEM). */
+ * see once, accumulating P V in TMEM (rescaled in place when a row's
+ * maximum grows). */
 
 /* Compressed keys and values: k_cmp[b,c,g] = mean of k[b,s,g] over the
  * tokens s of block c (a partial last block averages the tokens it has),
