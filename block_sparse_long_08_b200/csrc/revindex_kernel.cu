@@ -20,16 +20,19 @@
 //   4. order   (when order_words > 0) each list sorted by query position,
 //              so that the order -- and whatever is summed in it -- is the
 //              same from run to run; pos_of follows.  A row selects a block
-//              at most once, so the positions in a list are distinct and an
-//              entry's rank is the number of smaller positions: counted
-//              directly in shared memory for lists of up to kOrderDirect
-//              entries, read from a bitmap over the sequence's rows in the
-//              chunk (and per-word prefix counts) for longer ones, the slot
-//              then found in the row's selection.
+//              at most once, so the positions in a list are distinct.  Up
+//              to kOrderCount entries: an entry's rank is the number of
+//              smaller positions, counted in shared memory; up to
+//              kOrderSort: a bitonic sort in shared memory; longer lists:
+//              ranks read from a bitmap over the sequence's rows in the
+//              chunk (and per-word prefix counts), the slot then found in
+//              the row's selection.
 // Every work item then holds <= qpi queries, so items cost the same and a
 // persistent grid balances itself whatever the causal skew between early
 // and late key blocks.
 #include <cuda_runtime.h>
+
+#include <climits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -157,7 +160,8 @@ __global__ void __launch_bounds__(256) revidx_fill_kernel(const RevIdxArgs a) {
   }
 }
 
-constexpr int kOrderDirect = 2048;
+constexpr int kOrderCount = 256;
+constexpr int kOrderSort = 4096;
 constexpr int kOrderThreads = 256;
 
 // Exclusive prefix of x over the CTA's 256 threads; tot gets the sum (all
@@ -198,7 +202,7 @@ __device__ __forceinline__ void order_put(const RevIdxArgs &a, const int4 &s, in
 }
 
 __global__ void __launch_bounds__(kOrderThreads) revidx_order_kernel(const RevIdxArgs a) {
-  extern __shared__ int sm[];   // kOrderDirect entries, or bitmap + prefix words
+  extern __shared__ int sm[];   // up to kOrderSort entries, or bitmap + prefix words
   __shared__ int warp_sums[32], total;
   const int n_lists = a.q.B * a.G * a.nb;
   const int tid = threadIdx.x;
@@ -207,7 +211,7 @@ __global__ void __launch_bounds__(kOrderThreads) revidx_order_kernel(const RevId
     if (n <= 1) continue;   // the same for every thread of the CTA
     const int b = bgj / (a.G * a.nb), g = (bgj / a.nb) % a.G, j = bgj % a.nb;
     const int4 s = qgeo_seq(a.q, b);
-    if (n <= kOrderDirect) {
+    if (n <= kOrderCount) {
       for (int i = tid; i < n; i += kOrderThreads) sm[i] = a.list[lo + i];
       __syncthreads();
       for (int i = tid; i < n; i += kOrderThreads) {
@@ -216,6 +220,30 @@ __global__ void __launch_bounds__(kOrderThreads) revidx_order_kernel(const RevId
         for (int m = 0; m < n; ++m) rank += sm[m] < x;
         order_put(a, s, g, x, lo + rank);
       }
+      __syncthreads();
+      continue;
+    }
+    if (n <= kOrderSort) {
+      int np = kOrderCount;
+      while (np < n) np <<= 1;
+      for (int i = tid; i < np; i += kOrderThreads) sm[i] = i < n ? a.list[lo + i] : INT_MAX;
+      __syncthreads();
+      for (int k = 2; k <= np; k <<= 1) {   // ascending bitonic network over np entries
+        for (int jj = k >> 1; jj > 0; jj >>= 1) {
+          for (int i = tid; i < np; i += kOrderThreads) {
+            const int l = i ^ jj;
+            if (l > i) {
+              const int x = sm[i], y = sm[l];
+              if ((x > y) == ((i & k) == 0)) {
+                sm[i] = y;
+                sm[l] = x;
+              }
+            }
+          }
+          __syncthreads();
+        }
+      }
+      for (int i = tid; i < n; i += kOrderThreads) order_put(a, s, g, sm[i], lo + i);
       __syncthreads();
       continue;
     }
@@ -265,7 +293,7 @@ __global__ void __launch_bounds__(kOrderThreads) revidx_order_kernel(const RevId
 }  // namespace
 
 size_t revidx_order_smem(int order_words) {
-  const size_t direct = sizeof(int) * kOrderDirect;
+  const size_t direct = sizeof(int) * kOrderSort;
   const size_t bitmap = sizeof(int) * 2 * size_t(order_words);
   return direct > bitmap ? direct : bitmap;
 }

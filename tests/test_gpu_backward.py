@@ -220,3 +220,24 @@ def test_backward_chunks_any_length(blk):
     ref = O.prefill_backward(x["q"], x["k"], x["v"], sel.cpu().numpy(), x["dout"], block=blk)
     for name, g in (("dq", dq), ("dk", dk), ("dv", dv)):
         _grad_close(f"{name} (chunks of 384)", P.f64(g), ref[name])
+
+
+def test_backward_ordering_routes_bit_reproducible():
+    """A selection of block 0 plus the local block for every row: block 0's
+    list holds all 8192 rows (the ordering step's bitmap route, over 4096
+    entries), the local blocks' lists 128 each (direct rank count).  dq, dk
+    and dv must be bit-identical over runs and match the oracle."""
+    L, top_k = 8192, 2
+    shape = I.PrefillShape(B=1, L=L, H=8, G=2, d=128, d_idx=128, top_k=top_k)
+    x = _inputs(shape, 46)
+    t = torch.arange(L, dtype=torch.int32)
+    sel = torch.full((1, 2, L, top_k), -1, dtype=torch.int32)
+    sel[..., 0] = 0
+    sel[..., 1] = torch.where(t // 128 > 0, t // 128, torch.full_like(t, -1))
+    sel = sel.to(DEV)
+    _, dq1, dk1, dv1 = _forward_backward(x, top_k, sel=sel)
+    _, dq2, dk2, dv2 = _forward_backward(x, top_k, sel=sel)
+    assert torch.equal(dq1, dq2) and torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+    ref = O.prefill_backward(x["q"], x["k"], x["v"], sel.cpu().numpy(), x["dout"], block=128)
+    for name, g in (("dq", dq1), ("dk", dk1), ("dv", dv1)):
+        _grad_close(f"{name} (block 0 for every row)", P.f64(g), ref[name])
