@@ -11,8 +11,9 @@
 // or 64 keys (the explainer's §4.2 reasons with 64-token blocks).  Per item:
 //   S = Q K_j^T   (UMMA M=128, N=BLK, K=128, fp32 in TMEM)
 //   softmax       row r: mask s <= t (only on the diagonal block), row max,
-//                 exp2, row sum, P as bf16 into shared memory
-//   O = P V_j     (UMMA, V consumed MN-major straight from its TMA tile)
+//                 exp2, row sum, P as bf16 pairs back into S's TMEM columns
+//   O = P V_j     (UMMA with A = P read from TMEM, V consumed MN-major
+//                 straight from its TMA tile)
 //   partial       O / l (bf16) and lse = ln(sum exp(scale q.k)) per row; a
 //                 second kernel merges a query row's <= top_k partials.
 //
@@ -25,18 +26,21 @@
 //              block (items are ordered by (b, g, j)).
 //   warp 1     TMEM owner and MMA issuer: issues S_i and O_i in whatever
 //              order their inputs become ready (non-blocking barrier probes).
-//   warps 2-7  three gather groups of 64 threads; group k owns shared stage
-//              k and the items i = k (mod 3): it publishes the item's query
-//              list, gathers the q rows (R heads of a query are 256*R
-//              contiguous bytes) with cp.async into the stage's 128B-swizzled
-//              tile, and prefetches its next item's descriptor meanwhile.
+//   warps 2-7  the gather team (192 threads) takes every item in turn: it
+//              publishes the item's query list and gathers the q rows (R
+//              heads of a query are 256*R contiguous bytes) with cp.async
+//              into a free stage's 128B-swizzled tile.
 //   warps 8-15 two softmax warpgroups, even and odd items, each with its own
-//              128-column TMEM slot (S, then O).  After the softmax a group
-//              loads O, stages the bf16 partial rows in the item's stage and
-//              writes them with one bulk copy.
-// A stage holds Q, then P, then the staged partial of one item; with NQ
-// stages the q gather of item i+NQ starts as soon as item i's partial has
-// left.  Seven 32 KB tiles are split between stages and K/V tiles (AttnCfg).
+//              TMEM slot: 128 columns for S (then P over its first BLK/2
+//              columns) and 128 for O; 512 columns in all.  After the softmax
+//              a group loads O, stages the bf16 partial rows in the item's
+//              stage and writes them with one bulk copy per warp.
+// A stage holds Q, then the staged partial of one item; with NQ stages the
+// q gather of item i+NQ starts as soon as item i's partial has left.  Seven
+// 32 KB tiles are split between stages and K/V tiles (AttnCfg).  P goes
+// through TMEM rather than shared memory: it saves the softmax 2048 16-byte
+// shared stores per item and the UMMA a 32 KB shared-memory read, and the
+// SM's shared-memory instruction path is what sets the item period.
 //
 // Partial layout.  The partials of a chunk are indexed by reverse-index list
 // position: the entry at position pos (query t, slot k of group g) owns rows
@@ -60,7 +64,7 @@ namespace {
 constexpr int kAttnThreads = 512;
 constexpr int kTile = 32768;                         // 128 rows x 256 B
 
-// Shared-memory plan per head ratio R.  Seven 32 KB tiles: NQ Q/P/partial
+// Shared-memory plan per head ratio R.  Seven 32 KB tiles: NQ Q/partial
 // stages and NKV K/V tiles.  Four stages (with three K/V tiles, enough when
 // items of one key block come in runs) for R >= 2; for R = 1 the 128-entry
 // item lists leave room for three stages only, with four K/V tiles.
@@ -209,7 +213,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init_fence();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), 256);
+    tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -347,16 +351,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const bool v_ok = !(e & 8u) || mbar_test_wait(bar(C::BAR_KVFULL + xv), (e >> 2) & 1u);
             if (v_ok && mbar_test_wait(bar(C::BAR_PFULL + (no & 1)), (no >> 1) & 1)) {
               tc_fence_after();
-              const uint32_t sp = s_base + C::SMEM_Q + (no % C::NQ) * kTile;
+              // P (bf16 pairs over S's first BLK/2 columns) is A, from TMEM
+              const uint32_t p_tmem = tmem_base + (no & 1) * 128;
               const uint32_t sv = s_base + C::SMEM_KV + xv * kTile;
-              const uint32_t d_tmem = tmem_base + (no & 1) * 128;
+              const uint32_t d_tmem = tmem_base + 256 + (no & 1) * 128;
 #pragma unroll
-              for (int kk = 0; kk < BLK / 16; ++kk) {   // P's keys: 64 per 16 KB half
-                const int c = kk >> 2;
-                const uint32_t off = (kk & 3) * 32;
-                umma_f16_ss(d_tmem, sdesc_sw128(sp + c * 16384 + off, 16, 1024),
-                            sdesc_sw128(sv + kk * 2048, kHalf, 1024), idesc_o, kk > 0);
-              }
+              for (int kk = 0; kk < BLK / 16; ++kk)   // 16 keys (8 columns of P) each
+                umma_f16_ts(d_tmem, p_tmem + kk * 8, sdesc_sw128(sv + kk * 2048, kHalf, 1024),
+                            idesc_o, kk > 0);
               umma_commit(bar(C::BAR_OFULL + (no & 1)));
               // free run m's V tile once item no is known to be its last
               if (no + 1 < ns) {
@@ -538,24 +540,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const float2 nmb2 = make_float2(-mb, -mb);
       float2 l2 = make_float2(0.f, 0.f);
       uint8_t *stage = smem + C::SMEM_Q + s * kTile;
+      // P as bf16 pairs into S's own TMEM columns (S is all in registers):
+      // 64 keys per 32 columns
 #pragma unroll
       for (int h = 0; h < BLK / 64; ++h) {
+        uint32_t pw[32];
 #pragma unroll
-        for (int gb = 0; gb < 8; ++gb) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = h * 64 + gb * 8 + e * 2;
-            const float2 x = fma2(make_float2(v[c], v[c + 1]), sc2, nmb2);
-            const float2 pp = make_float2(fast_exp2(x.x), fast_exp2(x.y));
-            l2 = add2(l2, pp);
-            w4[e] = pack_bf16x2(pp.x, pp.y);
-          }
-          *reinterpret_cast<uint4 *>(stage + h * 16384 + sw128_offset(row, gb)) =
-              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        for (int e = 0; e < 32; ++e) {
+          const int c = h * 64 + 2 * e;
+          const float2 x = fma2(make_float2(v[c], v[c + 1]), sc2, nmb2);
+          const float2 pp = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+          l2 = add2(l2, pp);
+          pw[e] = pack_bf16x2(pp.x, pp.y);
         }
+        tmem_st32u(tm + h * 32, pw);
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::BAR_PFULL + u));
 
@@ -565,10 +565,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       float ov[kHeadDim];   // the item's O row (all of d, whatever the block length)
       {
         float t0[32], t1[32], t2[32], t3[32];
-        tmem_ld32(tm, t0);
-        tmem_ld32(tm + 32, t1);
-        tmem_ld32(tm + 64, t2);
-        tmem_ld32(tm + 96, t3);
+        tmem_ld32(tm + 256, t0);
+        tmem_ld32(tm + 288, t1);
+        tmem_ld32(tm + 320, t2);
+        tmem_ld32(tm + 352, t3);
         tmem_wait_ld();
 #pragma unroll
         for (int x = 0; x < 32; ++x) {
@@ -619,7 +619,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 256);
+    tmem_dealloc(tmem_base, 512);
   }
 }
 
