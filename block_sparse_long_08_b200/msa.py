@@ -6,6 +6,10 @@ The functions carry the C names (msa_index_select, msa_sparse_attn_prefill,
 msa_sparse_attn_decode, msa_forward, msa_workspace_bytes, msa_read_status,
 msa_last_error).  Tensors must be CUDA, contiguous, bf16 (int32 for
 selections and lengths).  Outputs are allocated here unless passed in.
+Every tensor handed to the library, passed in or allocated, is checked
+against the number of elements the call reads or writes (derived from the
+same parameters the call receives), so a short buffer raises ValueError
+here instead of being read or written past its end on the device.
 """
 from __future__ import annotations
 
@@ -165,6 +169,15 @@ def _req(t: torch.Tensor, name: str, dtype) -> torch.Tensor:
     return t
 
 
+def _size(t: torch.Tensor, name: str, dtype, numel: int) -> torch.Tensor:
+    """_req plus the element count the call reads or writes: a short buffer
+    is an error here rather than an access past its end on the device."""
+    _req(t, name, dtype)
+    if t.numel() < numel:
+        raise ValueError(f"{name} has {t.numel()} elements, the call needs {numel}")
+    return t
+
+
 def _stream(stream) -> ctypes.c_void_p:
     s = torch.cuda.current_stream() if stream is None else stream
     return ctypes.c_void_p(s.cuda_stream)
@@ -174,6 +187,7 @@ def _ensure_ws(ws, p, op, device):
     need = msa_workspace_bytes(p, op)
     if ws is None:
         return torch.zeros(need, dtype=torch.uint8, device=device)
+    _req(ws, "ws", torch.uint8)
     if ws.numel() < need:
         raise MSAError(MSA_ERR_WORKSPACE, f"workspace has {ws.numel()} bytes, need {need}")
     return ws
@@ -187,10 +201,12 @@ def msa_index_select(q_idx: torch.Tensor, k_idx: torch.Tensor, top_k: int, *,
     _req(q_idx, "q_idx", torch.bfloat16)
     _req(k_idx, "k_idx", torch.bfloat16)
     B, L, G, di = q_idx.shape
+    _size(k_idx, "k_idx", torch.bfloat16, B * L * di)
     p = make_params(B, L, G, G, 128, di, block, top_k)
     dev = q_idx.device
     if sel is None:
         sel = torch.empty((B, G, L, top_k), dtype=torch.int32, device=dev)
+    _size(sel, "sel", torch.int32, B * G * L * top_k)
     scores = torch.empty((B, G, L, (L + block - 1) // block), dtype=torch.float32,
                          device=dev) if block_scores else None
     ws = _ensure_ws(ws, p, MSA_OP_INDEX_SELECT, dev)
@@ -209,10 +225,14 @@ def msa_sparse_attn_prefill(q, k, v, sel, *, scale: float = 0.0, want_lse: bool 
     B, L, H, d = q.shape
     G = k.shape[2]
     top_k = sel.shape[3]
+    for n, t in (("k", k), ("v", v)):
+        _size(t, n, torch.bfloat16, B * L * G * d)
+    _size(sel, "sel", torch.int32, B * G * L * top_k)
     p = make_params(B, L, H, G, d, 128, block, top_k, scale, chunk)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
+    _size(out, "out", torch.bfloat16, B * L * H * d)
     lse = torch.empty((B, L, H), dtype=torch.float32, device=dev) if want_lse else None
     ws = _ensure_ws(ws, p, MSA_OP_PREFILL_ATTN, dev)
     _check(lib().msa_sparse_attn_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(sel),
@@ -239,6 +259,12 @@ def msa_sparse_attn_backward(q, k, v, out, lse, dout, sel, *, scale: float = 0.0
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    for n, t in (("k", k), ("v", v), ("dk", dk), ("dv", dv)):
+        _size(t, n, torch.bfloat16, B * L * G * d)
+    for n, t in (("out", out), ("dout", dout), ("dq", dq)):
+        _size(t, n, torch.bfloat16, B * L * H * d)
+    _size(lse, "lse", torch.float32, B * L * H)
+    _size(sel, "sel", torch.int32, B * G * L * top_k)
     ws = _ensure_ws(ws, p, MSA_OP_BACKWARD, dev)
     _check(lib().msa_sparse_attn_backward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                           _ptr(lse), _ptr(dout), _ptr(sel), _ptr(dq), _ptr(dk),
@@ -254,12 +280,16 @@ def msa_forward(q, k, v, q_idx, k_idx, top_k: int, *, scale: float = 0.0, want_s
     B, L, H, d = q.shape
     G = k.shape[2]
     di = q_idx.shape[3]
+    _check_prefill_inputs(B, L, G, d, di, k, v, q_idx, k_idx)
     p = make_params(B, L, H, G, d, di, block, top_k, scale, chunk)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
+    _size(out, "out", torch.bfloat16, B * L * H * d)
     if sel is None and want_sel:
         sel = torch.empty((B, G, L, top_k), dtype=torch.int32, device=dev)
+    if sel is not None:
+        _size(sel, "sel", torch.int32, B * G * L * top_k)
     lse = torch.empty((B, L, H), dtype=torch.float32, device=dev) if want_lse else None
     ws = _ensure_ws(ws, p, MSA_OP_FORWARD, dev)
     _check(lib().msa_forward(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(q_idx), _ptr(k_idx),
@@ -270,6 +300,13 @@ def msa_forward(q, k, v, q_idx, k_idx, top_k: int, *, scale: float = 0.0, want_s
     if want_lse:
         res.append(lse)
     return res[0] if len(res) == 1 else tuple(res)
+
+
+def _check_prefill_inputs(B, L, G, d, di, k, v, q_idx, k_idx):
+    for n, t in (("k", k), ("v", v)):
+        _size(t, n, torch.bfloat16, B * L * G * d)
+    _size(q_idx, "q_idx", torch.bfloat16, B * L * G * di)
+    _size(k_idx, "k_idx", torch.bfloat16, B * L * di)
 
 
 # ---- NSA-style variant: compression and sliding-window branches beside the
@@ -289,6 +326,9 @@ def msa_nsa_compress_kv(k, v, *, block: int = 128, k_cmp=None, v_cmp=None, strea
     nb = (L + block - 1) // block
     k_cmp = torch.empty((B, nb, G, d), dtype=torch.bfloat16, device=k.device) if k_cmp is None else k_cmp
     v_cmp = torch.empty((B, nb, G, d), dtype=torch.bfloat16, device=k.device) if v_cmp is None else v_cmp
+    _size(v, "v", torch.bfloat16, B * L * G * d)
+    for n, t in (("k_cmp", k_cmp), ("v_cmp", v_cmp)):
+        _size(t, n, torch.bfloat16, B * nb * G * d)
     _check(lib().msa_nsa_compress_kv(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(k_cmp), _ptr(v_cmp),
                                      _stream(stream)))
     return k_cmp, v_cmp
@@ -300,7 +340,11 @@ def msa_nsa_window_attn(q, k, v, window: int, *, scale: float = 0.0, want_lse: b
     for n, t in (("q", q), ("k", k), ("v", v)):
         _req(t, n, torch.bfloat16)
     p = _nsa_params(q, k, 128, scale)
+    B, L, H, d = q.shape
+    for n, t in (("k", k), ("v", v)):
+        _size(t, n, torch.bfloat16, B * L * k.shape[2] * d)
     out = torch.empty_like(q) if out is None else out
+    _size(out, "out", torch.bfloat16, B * L * H * d)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if want_lse else None
     ws = _ensure_ws(ws, p, MSA_OP_NSA_BRANCH, q.device)
     _check(lib().msa_nsa_window_attn(ctypes.byref(p), int(window), _ptr(q), _ptr(k), _ptr(v),
@@ -317,7 +361,11 @@ def msa_nsa_compressed_attn(q, k_cmp, v_cmp, *, block: int = 128, scale: float =
     p = _nsa_params(q, k_cmp, block, scale)
     if k_cmp.shape[1] != (q.shape[1] + block - 1) // block:
         raise ValueError("k_cmp must hold ceil(L / block) compressed tokens")
+    B, L, H, d = q.shape
+    for n, t in (("k_cmp", k_cmp), ("v_cmp", v_cmp)):
+        _size(t, n, torch.bfloat16, B * k_cmp.shape[1] * k_cmp.shape[2] * d)
     out = torch.empty_like(q) if out is None else out
+    _size(out, "out", torch.bfloat16, B * L * H * d)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if want_lse else None
     ws = _ensure_ws(ws, p, MSA_OP_NSA_BRANCH, q.device)
     _check(lib().msa_nsa_compressed_attn(ctypes.byref(p), _ptr(q), _ptr(k_cmp), _ptr(v_cmp),
@@ -334,6 +382,9 @@ def msa_nsa_gate(gates, o_cmp, o_slc, o_win, *, out=None, stream=None):
     B, L, H, d = o_cmp.shape
     p = make_params(B, L, H, H, d, 128, 128, 1)   # the gate is per head: any grouping
     out = torch.empty_like(o_cmp) if out is None else out
+    _size(gates, "gates", torch.float32, B * L * H * 3)
+    for n, t in (("o_slc", o_slc), ("o_win", o_win), ("out", out)):
+        _size(t, n, torch.bfloat16, B * L * H * d)
     _check(lib().msa_nsa_gate(ctypes.byref(p), _ptr(gates), _ptr(o_cmp), _ptr(o_slc), _ptr(o_win),
                               _ptr(out), _stream(stream)))
     return out
@@ -349,15 +400,26 @@ def msa_nsa_forward(q, k, v, q_idx, k_idx, gates, top_k: int, window: int, *, bl
     _req(gates, "gates", torch.float32)
     B, L, H, d = q.shape
     G = k.shape[2]
+    _check_prefill_inputs(B, L, G, d, q_idx.shape[3], k, v, q_idx, k_idx)
+    _size(gates, "gates", torch.float32, B * L * H * 3)
     p = make_params(B, L, H, G, d, q_idx.shape[3], block, top_k, scale)
     out = torch.empty_like(q) if out is None else out
+    _size(out, "out", torch.bfloat16, B * L * H * d)
     if sel is None and want_sel:
         sel = torch.empty((B, G, L, top_k), dtype=torch.int32, device=q.device)
+    if sel is not None:
+        _size(sel, "sel", torch.int32, B * G * L * top_k)
     ws = _ensure_ws(ws, p, MSA_OP_NSA_FORWARD, q.device)
     _check(lib().msa_nsa_forward(ctypes.byref(p), int(window), _ptr(q), _ptr(k), _ptr(v),
                                  _ptr(q_idx), _ptr(k_idx), _ptr(gates), _ptr(out), _ptr(sel),
                                  _ptr(ws), ws.numel(), _stream(stream)))
     return (out, sel) if want_sel else out
+
+
+def _check_cache_inputs(B, Lmax, G, d, di, k_cache, v_cache, k_idx_cache):
+    for n, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        _size(t, n, torch.bfloat16, B * Lmax * G * d)
+    _size(k_idx_cache, "k_idx_cache", torch.bfloat16, B * Lmax * di)
 
 
 def msa_forward_cached(q, q_idx, k_cache, v_cache, k_idx_cache, t0: int, top_k: int, *,
@@ -374,12 +436,17 @@ def msa_forward_cached(q, q_idx, k_cache, v_cache, k_idx_cache, t0: int, top_k: 
     B, n, H, d = q.shape
     Lmax, G = k_cache.shape[1], k_cache.shape[2]
     di = q_idx.shape[3]
+    _check_cache_inputs(B, Lmax, G, d, di, k_cache, v_cache, k_idx_cache)
+    _size(q_idx, "q_idx", torch.bfloat16, B * n * G * di)
     p = make_params(B, Lmax, H, G, d, di, block, top_k, scale, chunk)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
+    _size(out, "out", torch.bfloat16, B * n * H * d)
     if sel is None and want_sel:
         sel = torch.empty((B, G, n, top_k), dtype=torch.int32, device=dev)
+    if sel is not None:
+        _size(sel, "sel", torch.int32, B * G * n * top_k)
     lse = torch.empty((B, n, H), dtype=torch.float32, device=dev) if want_lse else None
     ws = _ensure_ws(ws, p, MSA_OP_FORWARD, dev)
     _check(lib().msa_forward_cached(ctypes.byref(p), int(t0), int(n), _ptr(q), _ptr(q_idx),
@@ -405,14 +472,21 @@ def msa_forward_cached_varlen(q, q_idx, k_cache, v_cache, k_idx_cache, t0, n, to
         _req(t, n_, torch.bfloat16)
     B, Lmax, G = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
     H, d = q.shape[1], q.shape[2]
+    if len(t0) != B or len(n) != B:
+        raise ValueError(f"t0 and n need one entry per cached sequence ({B})")
     t0a = (ctypes.c_int32 * B)(*[int(v) for v in t0])
     na = (ctypes.c_int32 * B)(*[int(v) for v in n])
-    if sum(int(v) for v in n) != q.shape[0]:
+    N = q.shape[0]
+    if sum(int(v) for v in n) != N:
         raise ValueError("q rows must equal sum(n)")
-    p = make_params(B, Lmax, H, G, d, q_idx.shape[2], block, top_k, scale, chunk)
+    di = q_idx.shape[2]
+    _check_cache_inputs(B, Lmax, G, d, di, k_cache, v_cache, k_idx_cache)
+    _size(q_idx, "q_idx", torch.bfloat16, N * G * di)
+    p = make_params(B, Lmax, H, G, d, di, block, top_k, scale, chunk)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
+    _size(out, "out", torch.bfloat16, N * H * d)
     lse = torch.empty((q.shape[0], H), dtype=torch.float32, device=dev) if want_lse else None
     ws = _ensure_ws(ws, p, MSA_OP_FORWARD_VARLEN, dev)
     _check(lib().msa_forward_cached_varlen(ctypes.byref(p), t0a, na, _ptr(q), _ptr(q_idx),
@@ -448,6 +522,13 @@ def msa_forward_host(q, k, v, q_idx, k_idx, top_k: int, *, out, lse=None, stagin
     B, L, H, d = q.shape
     G = k.shape[2]
     di = q_idx.shape[3]
+    need = {"q": B * L * H * d, "k": B * L * G * d, "v": B * L * G * d, "q_idx": B * L * G * di,
+            "k_idx": B * L * di, "out": B * L * H * d}
+    for n, t in (("k", k), ("v", v), ("q_idx", q_idx), ("k_idx", k_idx), ("out", out)):
+        if t.numel() < need[n]:
+            raise ValueError(f"{n} has {t.numel()} elements, the call needs {need[n]}")
+    if lse is not None and lse.numel() < B * L * H:
+        raise ValueError(f"lse has {lse.numel()} elements, the call needs {B * L * H}")
     p = make_params(B, L, H, G, d, di, block, top_k, scale, chunk)
     dev = torch.device("cuda") if device is None else torch.device(device)
     if staging is None:
@@ -457,7 +538,9 @@ def msa_forward_host(q, k, v, q_idx, k_idx, top_k: int, *, out, lse=None, stagin
         if lse is not None:
             staging["lse"] = torch.empty(lse.shape, dtype=torch.float32, device=dev)
     for n in ("q", "k", "v", "q_idx", "k_idx", "out"):
-        _req(staging[n], "staging " + n, torch.bfloat16)
+        _size(staging[n], "staging " + n, torch.bfloat16, need[n])
+    if lse is not None:
+        _size(staging["lse"], "staging lse", torch.float32, B * L * H)
     st = msa_staging(*(staging[n].data_ptr() for n in ("q", "k", "v", "q_idx", "k_idx", "out")),
                      staging["lse"].data_ptr() if lse is not None else None)
     ws = _ensure_ws(ws, p, MSA_OP_FORWARD, dev)
@@ -467,6 +550,12 @@ def msa_forward_host(q, k, v, q_idx, k_idx, top_k: int, *, out, lse=None, stagin
                                   _ptr(k_idx), _ptr(out), _ptr(lse), ctypes.byref(st), _ptr(ws),
                                   ws.numel(), _stream(stream), _stream(copy_stream)))
     return (out, lse) if lse is not None else out
+
+
+def _check_decode_outputs(B, H, G, d, top_k, out, sel):
+    _size(out, "out", torch.bfloat16, B * H * d)
+    if sel is not None:
+        _size(sel, "sel", torch.int32, B * G * top_k)
 
 
 def msa_sparse_attn_decode(q, q_idx, k_cache, v_cache, k_idx_cache, seq_lens, top_k: int, *,
@@ -481,12 +570,16 @@ def msa_sparse_attn_decode(q, q_idx, k_cache, v_cache, k_idx_cache, seq_lens, to
     B, H, d = q.shape
     Lmax, G = k_cache.shape[1], k_cache.shape[2]
     di = q_idx.shape[2]
+    _check_cache_inputs(B, Lmax, G, d, di, k_cache, v_cache, k_idx_cache)
+    _size(q_idx, "q_idx", torch.bfloat16, B * G * di)
+    _size(seq_lens, "seq_lens", torch.int32, B)
     p = make_params(B, Lmax, H, G, d, di, block, top_k, scale)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
     if sel is None and want_sel:
         sel = torch.empty((B, G, top_k), dtype=torch.int32, device=dev)
+    _check_decode_outputs(B, H, G, d, top_k, out, sel)
     ws = _ensure_ws(ws, p, MSA_OP_DECODE, dev)
     _check(lib().msa_sparse_attn_decode(ctypes.byref(p), _ptr(q), _ptr(q_idx), _ptr(k_cache),
                                         _ptr(v_cache), _ptr(k_idx_cache), _ptr(seq_lens), _ptr(out),
@@ -508,12 +601,20 @@ def msa_sparse_attn_decode_fp8idx(q, q_idx, k_cache, v_cache, k_idx8, k_idx_scal
     _req(seq_lens, "seq_lens", torch.int32)
     B, H, d = q.shape
     Lmax, G = k_cache.shape[1], k_cache.shape[2]
-    p = make_params(B, Lmax, H, G, d, k_idx8.shape[2], block, top_k, scale)
+    di = k_idx8.shape[2]
+    for n_, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        _size(t, n_, torch.bfloat16, B * Lmax * G * d)
+    _size(k_idx8, "k_idx8", torch.uint8, B * Lmax * di)
+    _size(k_idx_scale, "k_idx_scale", torch.float32, B * Lmax)
+    _size(q_idx, "q_idx", torch.bfloat16, B * G * di)
+    _size(seq_lens, "seq_lens", torch.int32, B)
+    p = make_params(B, Lmax, H, G, d, di, block, top_k, scale)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
     if sel is None and want_sel:
         sel = torch.empty((B, G, top_k), dtype=torch.int32, device=dev)
+    _check_decode_outputs(B, H, G, d, top_k, out, sel)
     ws = _ensure_ws(ws, p, MSA_OP_DECODE, dev)
     _check(lib().msa_sparse_attn_decode_fp8idx(ctypes.byref(p), _ptr(q), _ptr(q_idx), _ptr(k_cache),
                                                _ptr(v_cache), _ptr(k_idx8), _ptr(k_idx_scale),
@@ -536,12 +637,22 @@ def msa_sparse_attn_decode_fp8(q, q_idx, k8, k_scale, v8, v_scale, k_idx8, k_idx
     _req(seq_lens, "seq_lens", torch.int32)
     B, H, d = q.shape
     Lmax, G = k8.shape[1], k8.shape[2]
-    p = make_params(B, Lmax, H, G, d, k_idx8.shape[2], block, top_k, scale)
+    di = k_idx8.shape[2]
+    for n_, t in (("k8", k8), ("v8", v8)):
+        _size(t, n_, torch.uint8, B * Lmax * G * d)
+    for n_, t in (("k_scale", k_scale), ("v_scale", v_scale)):
+        _size(t, n_, torch.float32, B * Lmax * G)
+    _size(k_idx8, "k_idx8", torch.uint8, B * Lmax * di)
+    _size(k_idx_scale, "k_idx_scale", torch.float32, B * Lmax)
+    _size(q_idx, "q_idx", torch.bfloat16, B * G * di)
+    _size(seq_lens, "seq_lens", torch.int32, B)
+    p = make_params(B, Lmax, H, G, d, di, block, top_k, scale)
     dev = q.device
     if out is None:
         out = torch.empty_like(q)
     if sel is None and want_sel:
         sel = torch.empty((B, G, top_k), dtype=torch.int32, device=dev)
+    _check_decode_outputs(B, H, G, d, top_k, out, sel)
     ws = _ensure_ws(ws, p, MSA_OP_DECODE, dev)
     _check(lib().msa_sparse_attn_decode_fp8(ctypes.byref(p), _ptr(q), _ptr(q_idx), _ptr(k8),
                                             _ptr(k_scale), _ptr(v8), _ptr(v_scale), _ptr(k_idx8),
@@ -559,6 +670,8 @@ def msa_quantize_e4m3_rows(x, *, codes=None, scale=None, stream=None):
         codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     if scale is None:
         scale = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _size(codes, "codes", torch.uint8, rows * cols)
+    _size(scale, "scale", torch.float32, rows)
     _check(lib().msa_quantize_e4m3_rows(_ptr(x), rows, cols, _ptr(codes), _ptr(scale),
                                         _stream(stream)))
     return codes, scale
@@ -577,11 +690,16 @@ def msa_sparse_attn_decode_noalloc(q, q_idx, k_cache, v_cache, k_idx_cache, seq_
     _req(seq_lens, "seq_lens", torch.int32)
     B, H, d = q.shape
     Lmax, G = k_cache.shape[1], k_cache.shape[2]
-    p = make_params(B, Lmax, H, G, d, q_idx.shape[2], block, top_k, scale)
+    di = q_idx.shape[2]
+    _check_cache_inputs(B, Lmax, G, d, di, k_cache, v_cache, k_idx_cache)
+    _size(q_idx, "q_idx", torch.bfloat16, B * G * di)
+    _size(seq_lens, "seq_lens", torch.int32, B)
+    p = make_params(B, Lmax, H, G, d, di, block, top_k, scale)
     if out is None:
         out = torch.empty_like(q)
     if sel is None and want_sel:
         sel = torch.empty((B, G, top_k), dtype=torch.int32, device=q.device)
+    _check_decode_outputs(B, H, G, d, top_k, out, sel)
     _check(lib().msa_sparse_attn_decode_noalloc(ctypes.byref(p), _ptr(q), _ptr(q_idx), _ptr(k_cache),
                                                 _ptr(v_cache), _ptr(k_idx_cache), _ptr(seq_lens),
                                                 _ptr(out), _ptr(sel), _stream(stream)))
