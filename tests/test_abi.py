@@ -281,3 +281,63 @@ def test_any_length_and_either_block_in_every_operation():
     p = M.make_params(4, 4096, 16, 4, 128, 128, 128, 8)
     assert (M.msa_workspace_bytes(p, M.MSA_OP_FORWARD_VARLEN)
             >= M.msa_workspace_bytes(p, M.MSA_OP_FORWARD) + 4 * (2 * 128 + 16 + 32 * 8))
+
+
+def test_decode_entry_points_reject_bad_arguments():
+    """The bf16 and both FP8 decodes check pointers, alignment (scales
+    4-byte) and the workspace before any launch."""
+    p = M.make_params(2, 4096, 8, 2, 128, 64, 128, 4)
+    lib = M.lib()
+    ok, odd, odd4 = ctypes.c_void_p(4096), ctypes.c_void_p(4104), ctypes.c_void_p(4098)
+    need = M.msa_workspace_bytes(p, M.MSA_OP_DECODE)
+    dec = lambda q, out, ws, nbytes: lib.msa_sparse_attn_decode(ctypes.byref(p), q, ok, ok, ok, ok,
+                                                               ok, out, None, ws, nbytes, None)
+    assert dec(None, ok, ok, need) == M.MSA_ERR_INVALID_ARG
+    assert dec(ok, odd, ok, need) == M.MSA_ERR_INVALID_ARG
+    assert dec(ok, ok, ok, need - 1) == M.MSA_ERR_WORKSPACE
+    assert dec(ok, ok, None, need) == M.MSA_ERR_WORKSPACE
+    p0 = M.make_params(2, 0, 8, 2, 128, 64, 128, 4)   # a decode needs a cache
+    assert lib.msa_sparse_attn_decode(ctypes.byref(p0), ok, ok, ok, ok, ok, ok, ok, None, ok, need,
+                                      None) == M.MSA_ERR_INVALID_ARG
+
+    def fp8idx(k_idx8, scale):
+        return lib.msa_sparse_attn_decode_fp8idx(ctypes.byref(p), ok, ok, ok, ok, k_idx8, scale, ok,
+                                                 ok, None, ok, need, None)
+    assert fp8idx(None, ok) == M.MSA_ERR_INVALID_ARG
+    assert fp8idx(ok, None) == M.MSA_ERR_INVALID_ARG
+    assert fp8idx(odd, ok) == M.MSA_ERR_INVALID_ARG
+    assert fp8idx(ok, odd4) == M.MSA_ERR_INVALID_ARG     # scales need 4-byte alignment
+
+    def fp8(k8, ks, v8, vs, nbytes=need):
+        return lib.msa_sparse_attn_decode_fp8(ctypes.byref(p), ok, ok, k8, ks, v8, vs, ok, ok, ok,
+                                              ok, None, ok, nbytes, None)
+    assert fp8(None, ok, ok, ok) == M.MSA_ERR_INVALID_ARG
+    assert fp8(ok, ok, None, ok) == M.MSA_ERR_INVALID_ARG
+    assert fp8(ok, None, ok, ok) == M.MSA_ERR_INVALID_ARG
+    assert fp8(odd, ok, ok, ok) == M.MSA_ERR_INVALID_ARG
+    assert fp8(ok, ok, ok, odd4) == M.MSA_ERR_INVALID_ARG
+    assert fp8(ok, ok, ok, ok, need - 16) == M.MSA_ERR_WORKSPACE
+    # the no-allocation decode reports bad parameters like the regular one
+    bad = M.make_params(2, 4096, 8, 2, 128, 64, 128, 0)
+    assert lib.msa_sparse_attn_decode_noalloc(ctypes.byref(bad), ok, ok, ok, ok, ok, ok, ok, None,
+                                              None) == M.MSA_ERR_INVALID_ARG
+
+
+def test_prefill_attention_and_quantizer_reject_bad_arguments():
+    p = M.make_params(1, 2048, 8, 2, 128, 64, 128, 4)
+    lib = M.lib()
+    ok, odd = ctypes.c_void_p(4096), ctypes.c_void_p(4104)
+    need = M.msa_workspace_bytes(p, M.MSA_OP_PREFILL_ATTN)
+    att = lambda sel, lse, nbytes: lib.msa_sparse_attn_prefill(ctypes.byref(p), ok, ok, ok, sel, ok,
+                                                               lse, ok, nbytes, None)
+    assert att(None, None, need) == M.MSA_ERR_INVALID_ARG
+    assert att(ok, odd, need) == M.MSA_ERR_INVALID_ARG
+    assert att(ok, None, need - 1) == M.MSA_ERR_WORKSPACE
+    q8 = lambda x, rows, cols, codes, scale: lib.msa_quantize_e4m3_rows(x, rows, cols, codes, scale,
+                                                                        None)
+    assert q8(ok, 4, 0, ok, ok) == M.MSA_ERR_INVALID_ARG
+    assert q8(ok, 4, 24, ok, ok) == M.MSA_ERR_INVALID_ARG    # columns come in 16-byte granules
+    assert q8(ok, -1, 16, ok, ok) == M.MSA_ERR_INVALID_ARG
+    assert q8(None, 0, 16, None, None) == M.MSA_OK           # no rows: nothing to do
+    assert q8(ok, 4, 16, None, ok) == M.MSA_ERR_INVALID_ARG
+    assert q8(ok, 4, 16, ok, odd) == M.MSA_ERR_INVALID_ARG
